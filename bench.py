@@ -1,0 +1,443 @@
+#!/usr/bin/env python
+"""Benchmark of ReHyAt's chunked hybrid attention forward on B200.
+
+Workload (one step = one full forward through the C ABI): the 5 s, 480x832
+Wan2.1-1.3B-shaped layer -- latent 21x30x52 (N = 32760 tokens), batch 2,
+12 heads, D = 128, D' = 128, T_c = 3, T_o = 1, bidirectional, bf16 q/k/v
+drawn by rehyat_inputs (seed 2), fp32 output.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints ONE JSON line (rank 0).  Device time is measured with CUDA events on
+the stream the kernels run on, with a 256 MB L2 flush before every timed step
+(outside the events), max over ranks.  ``--impl reference`` times the fp64
+CPU oracle on a bounded sample instead (rank 0 only).
+
+Multi-GPU: every rank runs the same workload on its own GPU (replicas; the
+path has no exchange step), so ``value`` = all ranks' tokens / max time.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime as _dt
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+WORKLOAD = "wan_480x832_bidir"
+METRIC = "hybrid-attn fwd tokens/s & TFLOP/s (% BF16 tensor peak), 1 B200, 21x30x52 latent"
+L2_FLUSH_BYTES = 256 << 20
+KERNELS_PER_STEP = 3  # per-slice state, chunk scan, attention
+
+
+# --------------------------------------------------------------- workload
+def workload_desc(p):
+    return (f"{WORKLOAD}: B={p.batch}, heads={p.heads}, latent {p.T}x{p.Hs}x{p.Ws} "
+            f"(N={p.N}), D={p.D}, D'={p.Dp}, T_c={p.Tc}, T_o={p.To}, "
+            f"{'causal' if p.causal else 'bidirectional'}, bf16 q/k/v, fp32 y")
+
+
+def algorithmic_work(B, h, T, HW, D, Dp, Tc, To, causal):
+    """Method FLOPs / bytes (not the dense-attention work they avoid).
+
+    softmax: 4*D per (query, window key) pair (q.k and p.v);
+    phi_q, phi_k: 2*D*Dp per token each;  state: 2*Dp*D (+Dp) per token;
+    readout: 2*Dp*D (+2*Dp) per token.  All per (batch, head)."""
+    N = T * HW
+    pairs = 0
+    for t in range(-(-T // Tc)):
+        first, end = t * Tc, min(T, (t + 1) * Tc)
+        w = max(first - To, 0)
+        pairs += (end - first) * HW * (end - w) * HW
+    bh = B * h
+    f_soft = 4.0 * D * pairs * bh
+    f_phi = 2.0 * N * D * Dp * bh
+    f_state = (2.0 * N * Dp * D + N * Dp) * bh
+    f_read = (2.0 * N * Dp * D + 2.0 * N * Dp) * bh
+    return dict(
+        attn_flops=f_soft + f_phi + f_read,       # attention kernel (K3)
+        state_flops=f_phi + f_state,              # per-slice state kernel (K1)
+        total_flops=f_soft + 2 * f_phi + f_state + f_read,
+        exps=float(pairs * bh),
+        # K1 minimal HBM traffic: read k, v (bf16); write per-slice states (fp32)
+        state_bytes=float(bh * (2 * N * D * 2 + T * (Dp * D + Dp) * 4)),
+        # whole op minimal traffic: q, k, v in, y out (fp32), states out
+        io_bytes=float(bh * (3 * N * D * 2 + N * D * 4 + T * (Dp * D + Dp) * 4)),
+        full_softmax_flops=4.0 * D * N * N * bh,
+    )
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=float(d["hbm_gbs"]), bf16_tflops=float(d["bf16_tflops"]),
+                    bf16_tflops_sustained=float(d.get("bf16_tflops_sustained", 0.0)),
+                    source="measured")
+    except (OSError, KeyError, ValueError):
+        return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0,
+                    source="fallback")
+
+
+def kernel_source_sha(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(kernel_key, sha):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        e = d[kernel_key]
+        if e.get("source_sha") == sha:
+            return float(e["dram_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        pass
+    return None
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.proc = None
+        self.lines = []
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self, t0, t1):
+        rows = []
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                ts = _dt.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(parts[1]), float(parts[2]), parts[4:]))
+            except ValueError:
+                continue
+        inside = [r for r in rows if t0 - 0.05 <= r[0] <= t1 + 0.05] or rows[-3:]
+        if not inside:
+            return None
+        sm = sorted(r[1] for r in inside)
+        names = ["active_mask", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        reasons = set()
+        for r in inside:
+            for name, val in zip(names[1:], r[3][1:]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": inside[0][2],
+                "reasons": sorted(reasons), "samples": len(inside)}
+
+
+# ------------------------------------------------------------- CPU oracle
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def plan_oracle_sample(p, budget_s):
+    """Size a bounded sample of the workload for the fp64 oracle (factored
+    form, as it stands): time one chunk of one (batch, head) pair once, then
+    take as many chunks (or whole pairs) as fit in ``budget_s`` seconds."""
+    from oracle import rehyat_oracle as orc
+    nch = -(-p.T // p.Tc)
+    t0 = time.perf_counter()
+    orc.run_problem(p, heads_subset=[0], chunks_subset=[nch // 2])
+    one_chunk = time.perf_counter() - t0
+    if one_chunk * nch > budget_s:
+        return dict(heads=1, chunks=max(1, min(nch, int(budget_s / max(one_chunk, 1e-6)))))
+    BH = p.batch * p.heads
+    return dict(heads=max(1, min(BH, int(budget_s / (one_chunk * nch)))), chunks=nch)
+
+
+def run_oracle_sample(p, plan, start_head=0):
+    from oracle import rehyat_oracle as orc
+    nch = -(-p.T // p.Tc)
+    BH = p.batch * p.heads
+    heads = [(start_head + i) % BH for i in range(plan["heads"])]
+    chunks = list(range(plan["chunks"]))
+    t0 = time.perf_counter()
+    orc.run_problem(p, heads_subset=heads, chunks_subset=None if len(chunks) == nch else chunks)
+    dt = time.perf_counter() - t0
+    rows = sum((min(p.T, (c + 1) * p.Tc) - c * p.Tc) * p.HW for c in chunks)
+    # tokens of the metric count all heads of a token: rows * pairs / heads
+    token_equiv = rows * len(heads) / p.heads
+    return dict(seconds=dt, token_equiv=token_equiv,
+                sample=f"{len(heads)} of {BH} (batch, head) pairs x chunks "
+                       f"{chunks[0]}..{chunks[-1]} of {nch} ({rows} query rows per pair)")
+
+
+# --------------------------------------------------------------- main arms
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    from rehyat_inputs import config_problem
+    p = config_problem(WORKLOAD)
+    per_step = max(0.5, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    plan = plan_oracle_sample(p, per_step)
+    for i in range(args.warmup):
+        run_oracle_sample(p, plan, start_head=i)
+    total_s, total_tok, samples = 0.0, 0.0, []
+    for i in range(args.steps):
+        r = run_oracle_sample(p, plan, start_head=args.warmup + i)
+        total_s += r["seconds"]
+        total_tok += r["token_equiv"]
+        samples.append(r["sample"])
+    value = total_tok / total_s
+    cores = blas_threads()
+    w = algorithmic_work(p.batch, p.heads, p.T, p.HW, p.D, p.Dp, p.Tc, p.To, p.causal)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total_s / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_desc(p), "global_batch": p.batch, "seq_len": p.N,
+                   "parallelism": "none (host cores)"},
+        "tflops": w["total_flops"] / (p.batch * p.N) * value / 1e12,
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"per step: {samples[0]}"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_gpu(args, world, rank, local):
+    import numpy as np
+    import torch
+
+    import linear_attention_video_chunked_b200 as rh
+    from rehyat_inputs import config_problem
+
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=_dt.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    rh.lib()
+
+    p = config_problem(WORKLOAD)
+    B, H, N, D = p.q.shape
+    T, HW, Dp = p.T, p.HW, p.Dp
+    bf = torch.bfloat16
+    tt = lambda a, d: torch.from_numpy(np.ascontiguousarray(a)).to(dev, dtype=d)
+    q, k, v = tt(p.q, bf), tt(p.k, bf), tt(p.v, bf)
+    Wq, bq, Wk, bk = (tt(a, torch.float32) for a in (p.Wq, p.bq, p.Wk, p.bk))
+    y = torch.empty(B, H, N, D, device=dev, dtype=torch.float32)
+    params = rh.make_params(batch=B, heads=H, T=T, Hs=p.Hs, Ws=p.Ws, D=D, Dp=Dp, Tc=p.Tc,
+                            To=p.To, causal=p.causal, in_dtype=rh.BF16, out_dtype=rh.F32)
+    ws_bytes = rh.rehyat_workspace_bytes(params)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    phi = rh.RehyatPhi(Wq.data_ptr(), bq.data_ptr(), Wk.data_ptr(), bk.data_ptr())
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    sh = stream.cuda_stream
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
+        st = rh.rehyat_fwd_state(params, k.data_ptr(), v.data_ptr(), phi, ws.data_ptr(),
+                                 ws_bytes, sh)
+        if st:
+            raise rh.RehyatError(st, "rehyat_fwd_state")
+        if evs:
+            evs[1].record(stream)
+        st = rh.rehyat_fwd_attn(params, q.data_ptr(), k.data_ptr(), v.data_ptr(), phi,
+                                y.data_ptr(), ws.data_ptr(), ws_bytes, None, sh)
+        if st:
+            raise rh.RehyatError(st, "rehyat_fwd_attn")
+        if evs:
+            evs[2].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    time.sleep(0.3)
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_host0 = time.time()
+    for i in range(args.steps):
+        flush.zero_()
+        step(events[i])
+    torch.cuda.synchronize()
+    t_host1 = time.time()
+    if dist:
+        dist.barrier()
+    clocks.stop()
+    step_ms = [e[0].elapsed_time(e[2]) for e in events]
+    state_ms = [e[0].elapsed_time(e[1]) for e in events]
+    attn_ms = [e[1].elapsed_time(e[2]) for e in events]
+    total_ms = sum(step_ms)
+    if dist:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    tokens_per_step = B * N
+    value = world * tokens_per_step * args.steps / (total_ms / 1e3)
+
+    # End to end through the public API, host buffers in and out.
+    qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
+    yh = torch.empty(B, H, N, D, dtype=torch.float32).pin_memory()
+    qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    e2e_steps = max(1, min(args.steps, 10))
+
+    def e2e_step():
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        rh.hybrid_attn(qd, kd, vd, Wq, bq, Wk, bk, T=T, Hs=p.Hs, Ws=p.Ws, Tc=p.Tc, To=p.To,
+                       causal=p.causal, out=y, workspace=ws)
+        yh.copy_(y, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if dist:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+        dist.barrier()
+    e2e_value = world * tokens_per_step * e2e_steps / (e2e_ms / 1e3)
+    h2d = sum(x.numel() * x.element_size() for x in (qh, kh, vh))
+    d2h = yh.numel() * yh.element_size()
+
+    if rank != 0:
+        if dist:
+            dist.destroy_process_group()
+        return 0
+
+    w = algorithmic_work(B, H, T, HW, D, Dp, p.Tc, p.To, p.causal)
+    peaks = load_peaks()
+    attn_avg_s = sum(attn_ms) / len(attn_ms) / 1e3
+    state_avg_s = sum(state_ms) / len(state_ms) / 1e3
+    achieved_tf = w["attn_flops"] / attn_avg_s / 1e12
+    sha = kernel_source_sha(["linear_attention_video_chunked_b200/csrc/tc_attn.cu",
+                             "linear_attention_video_chunked_b200/csrc/simt.cu"])
+    roofline = {"kernel": "attention (window softmax + phi_q readout + joint norm)",
+                "bound": "tensor", "achieved": achieved_tf, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved_tf / peaks["bf16_tflops"],
+                "traffic": load_traffic("attn", sha),
+                "peak_source": f"{peaks['source']} bf16 burst (MEASURED_PEAKS.json)"
+                if peaks["source"] == "measured" else "fallback 1.59 PFLOP/s",
+                "work_per_launch": f"{w['attn_flops']:.4e} FLOP "
+                                   f"(4*D per query-key pair in the window + phi_q + readout)"}
+    state_gbs = w["state_bytes"] / state_avg_s / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": workload_desc(p), "global_batch": B * world, "seq_len": N,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "256 MB write before every timed step (outside the events)"},
+        "tflops": w["total_flops"] / (ms_per_step / 1e3) / 1e12 * world,
+        "pct_bf16_peak": w["total_flops"] / (ms_per_step / 1e3) / 1e12 / peaks["bf16_tflops"],
+        "stages_ms": {"state (per-slice + scan)": sum(state_ms) / len(state_ms),
+                      "attention": sum(attn_ms) / len(attn_ms)},
+        "state_stage_hbm": {"achieved": state_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                            "frac": state_gbs / peaks["hbm_gbs"],
+                            "bytes_per_launch": w["state_bytes"]},
+        "roofline": roofline,
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "api": "linear_attention_video_chunked_b200.hybrid_attn"},
+        "clocks": clocks.summary(t_host0, t_host1),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        r = run_oracle_sample(p, plan_oracle_sample(p, args.cpu_budget))
+        cv = r["token_equiv"] / r["seconds"]
+        line["cpu_baseline"] = {"value": cv, "unit": "tokens/s", "cores": blas_threads(),
+                                "kind": "oracle", "sample": r["sample"],
+                                "seconds": r["seconds"]}
+    print(json.dumps(line), flush=True)
+    if dist:
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["own", "reference"], default="own")
+    ap.add_argument("--cpu-budget", type=float, default=15.0,
+                    help="seconds of fp64 oracle work for the CPU baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+    return run_gpu(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,183 @@
+/*
+ * rehyat.h -- C ABI of librehyat.so: ReHyAt temporally chunked hybrid
+ * attention (forward), for NVIDIA B200 (sm_100a).
+ *
+ * Method: "ReHyAt: Recurrent Hybrid Attention for Video Diffusion
+ * Transformers" (papernotes.org note of the CVPR 2026 paper), Method, Key
+ * designs 1-4.  Notation:
+ *   B batch, heads h, T latent slices of Hs x Ws tokens (HW = Hs*Ws),
+ *   N = T*HW tokens in time-major order (slice, row, column), D head width,
+ *   Dp = D' the total feature width of phi, T_c slices per chunk, T_o overlap
+ *   slices.  Chunk t holds slices [t*T_c, min(T,(t+1)*T_c)); its softmax keys
+ *   start w_t = max(t*T_c - T_o, 0) slices in (Key design 2).
+ *
+ *   For a query i of chunk t, with softmax set S_t = keys of slices
+ *   [w_t, end_t) and linear set L_t (bidirectional: every other token;
+ *   causal: tokens of slices < w_t; Key designs 1 and 4):
+ *     c_i   = max_{j in S_t} (q_i . k_j) * scale           (stabiliser)
+ *     a^S_i = sum_{j in S_t} exp((q_i . k_j) * scale - c_i) v_j,
+ *     n^S_i = sum_{j in S_t} exp((q_i . k_j) * scale - c_i)
+ *     a^L_i = phi_q(q_i) . (sum_{j in L_t} phi_k(k_j) v_j^T),
+ *     n^L_i = phi_q(q_i) . (sum_{j in L_t} phi_k(k_j))
+ *     y_i   = (a^S_i + a^L_i) / (n^S_i + n^L_i)               (joint norm)
+ *   phi(x) = [(x W_1 + b_1)^2, (x W_2 + b_2)^2] (Key design 3, degree-2 form).
+ *
+ * Conventions shared by every entry point:
+ *   - Ownership: the caller allocates and owns every buffer (inputs, outputs,
+ *     phi parameters, workspace, streaming state).  The library never
+ *     allocates, frees or synchronises; all work is enqueued on `stream`
+ *     (a cudaStream_t passed as void*; NULL = the legacy default stream).
+ *   - All pointers are device pointers unless stated, 16-byte aligned.
+ *   - Errors: arguments are checked before any launch; a bad argument
+ *     returns a status and enqueues nothing.  A launch failure returns
+ *     REHYAT_ERR_CUDA.  Faults during execution surface at the caller's next
+ *     synchronisation.  The library never aborts or exits.
+ *   - Determinism: no atomics in any reduction; repeated calls on the same
+ *     inputs give bit-identical results.
+ */
+#ifndef REHYAT_H
+#define REHYAT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define REHYAT_API __attribute__((visibility("default")))
+#else
+#define REHYAT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  REHYAT_OK = 0,
+  REHYAT_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, bad enum */
+  REHYAT_ERR_UNSUPPORTED = 2,  /* D or Dp outside the supported set */
+  REHYAT_ERR_MISALIGNED = 3,   /* a pointer not 16-byte aligned */
+  REHYAT_ERR_WORKSPACE = 4,    /* workspace or state smaller than required */
+  REHYAT_ERR_CUDA = 5          /* a CUDA launch or query failed */
+} rehyat_status;
+
+typedef enum { REHYAT_F32 = 0, REHYAT_BF16 = 1 } rehyat_dtype;
+
+/* Flags for rehyat_params.flags. */
+#define REHYAT_FLAG_FORCE_SIMT 1 /* use the fp32 CUDA-core kernels even where a
+                                    tensor-core kernel exists (testing aid) */
+
+typedef struct {
+  int batch, heads;   /* B >= 1, h >= 1 */
+  int T, Hs, Ws;      /* latent slices and slice height/width, all >= 1 */
+  int D;              /* head width: 32, 64 or 128 */
+  int Dp;             /* total phi width D': 32, 64, 128 or 256 */
+  int Tc, To;         /* chunk slices (>= 1) and overlap slices (>= 0) */
+  int causal;         /* 0 bidirectional, 1 causal (Key design 4) */
+  int in_dtype;       /* rehyat_dtype of q, k, v (and of the streaming ring) */
+  int out_dtype;      /* rehyat_dtype of y */
+  float scale;        /* softmax logit scale; 0 means 1/sqrt(D) */
+  int flags;          /* REHYAT_FLAG_* */
+} rehyat_params;
+
+/* phi parameters, fp32 device arrays, per head:
+ *   W: [heads][2][D][Dp/2]  (part 0 = W_1, part 1 = W_2), row-major
+ *   b: [heads][2][Dp/2]
+ * In bf16 mode (in_dtype == REHYAT_BF16) the W matrices are rounded to bf16
+ * for the tensor-core products; b is added in fp32. */
+typedef struct {
+  const float *Wq, *bq, *Wk, *bk;
+} rehyat_phi;
+
+/* Optional branch partials, fp32 device arrays ([B][h][N][D] for aS, aL;
+ * [B][h][N] for nS, c, nL).  Any member may be NULL.  c is the stabiliser in
+ * natural-log units; aS, nS are relative to it. */
+typedef struct {
+  float *aS, *nS, *c, *aL, *nL;
+} rehyat_debug;
+
+/* ---------------------------------------------------------------------- */
+/* Full-sequence forward (bidirectional or non-recursive causal form).     */
+
+/* Bytes of workspace rehyat_hybrid_attn_fwd needs for these params (0 if the
+ * params are invalid).  Holds the per-slice states sum phi_k(k) v^T and
+ * sum phi_k(k) and the per-chunk linear-set states. */
+REHYAT_API size_t rehyat_workspace_bytes(const rehyat_params* p);
+
+/* y = ReHyAt hybrid attention of (q, k, v), all [B][h][N][D] contiguous.
+ *   q, k, v : in_dtype;  y : out_dtype;  phi : see rehyat_phi (struct in
+ *   host memory, arrays on the device);  workspace: >= ws_bytes bytes of
+ *   device memory that the call may overwrite;  dbg: NULL or partials.
+ * Source: Key designs 1-4 of the ReHyAt note (equations for y, a^S, a^L,
+ * the overlap set and the causal set). */
+REHYAT_API rehyat_status rehyat_hybrid_attn_fwd(const rehyat_params* p, const void* q,
+                                     const void* k, const void* v,
+                                     const rehyat_phi* phi, void* y,
+                                     void* workspace, size_t ws_bytes,
+                                     const rehyat_debug* dbg, void* stream);
+
+/* The same forward in two stages on one stream (rehyat_hybrid_attn_fwd is
+ * exactly rehyat_fwd_state followed by rehyat_fwd_attn on one workspace):
+ *   rehyat_fwd_state: per-slice sums phi_k(k) v^T, phi_k(k) and the
+ *     per-chunk linear-set state (bidirectional: all slices outside the
+ *     chunk's softmax window; causal: the slices before it), into workspace;
+ *   rehyat_fwd_attn: window softmax, phi_q readout of the workspace state
+ *     and joint normalisation, into y.
+ * Lets a caller time or overlap the stages, or reuse one state for several
+ * query sets over the same keys. */
+REHYAT_API rehyat_status rehyat_fwd_state(const rehyat_params* p, const void* k,
+                                          const void* v, const rehyat_phi* phi,
+                                          void* workspace, size_t ws_bytes,
+                                          void* stream);
+REHYAT_API rehyat_status rehyat_fwd_attn(const rehyat_params* p, const void* q,
+                                         const void* k, const void* v,
+                                         const rehyat_phi* phi, void* y,
+                                         const void* workspace, size_t ws_bytes,
+                                         const rehyat_debug* dbg, void* stream);
+
+/* Plain softmax attention over all N keys (no chunking, no linear branch):
+ * the dense comparator the ReHyAt note measures against (Experiments,
+ * efficiency).  Uses batch, heads, T, Hs, Ws, D, in/out dtype and scale of
+ * p; ignores Tc, To, causal and phi. */
+REHYAT_API rehyat_status rehyat_softmax_attn_fwd(const rehyat_params* p, const void* q,
+                                      const void* k, const void* v, void* y,
+                                      void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* Streaming: the causal chunk-wise RNN (Key design 4).                     */
+
+/* Bytes of the opaque streaming state: the running s [B][h][Dp][D] and
+ * z [B][h][Dp] (fp32), a ring holding the keys and values of the last T_o
+ * slices (in_dtype), and a device-side count of slices consumed.  Constant
+ * for any number of steps. */
+REHYAT_API size_t rehyat_state_bytes(const rehyat_params* p);
+
+/* Reset a state to the start of a video: s = 0, z = 0, empty ring. */
+REHYAT_API rehyat_status rehyat_state_init(const rehyat_params* p, void* state,
+                                void* stream);
+
+/* Workspace bytes rehyat_chunk_step needs. */
+REHYAT_API size_t rehyat_step_workspace_bytes(const rehyat_params* p);
+
+/* One step of the chunk-wise RNN: consumes the next `nslices` latent slices
+ * (1 <= nslices <= Tc; the last chunk of a video may be shorter) given as
+ * q, k, v [B][h][nslices*HW][D] (in_dtype) and writes their outputs y
+ * (same shape, out_dtype).  Softmax keys are the ring (up to T_o earlier
+ * slices) plus the chunk; the linear branch reads the state.  Afterwards the
+ * slices that leave the softmax window are added into (s, z) and the ring
+ * keeps the newest T_o slices.  p->causal must be 1. */
+REHYAT_API rehyat_status rehyat_chunk_step(const rehyat_params* p, const void* q,
+                                const void* k, const void* v, int nslices,
+                                const rehyat_phi* phi, void* state, void* y,
+                                void* workspace, size_t ws_bytes,
+                                const rehyat_debug* dbg, void* stream);
+
+/* ---------------------------------------------------------------------- */
+REHYAT_API const char* rehyat_status_string(rehyat_status s);
+
+/* Library ABI version (major*10000 + minor*100 + patch). */
+REHYAT_API int rehyat_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* REHYAT_H */

@@ -1,0 +1,317 @@
+"""Python binding of librehyat.so: ReHyAt chunked hybrid attention on B200.
+
+Two layers:
+
+* ``lib()`` and the ``rehyat_*`` functions are the C ABI of include/rehyat.h,
+  called through ctypes with plain integers for device pointers and streams
+  (argument marshalling only).
+* ``hybrid_attn``, ``softmax_attn`` and ``StreamingState`` take torch CUDA
+  tensors, allocate outputs/workspace with torch and call the C ABI on
+  torch's current stream.  torch provides device memory and streams; every
+  step of the computation runs in the library's CUDA kernels.
+
+There is no CPU fallback: if librehyat.so is missing, ``lib()`` raises.
+Build it with ``python -m linear_attention_video_chunked_b200.build``.
+
+Method: "ReHyAt: Recurrent Hybrid Attention for Video Diffusion
+Transformers" (papernotes.org note), Method, Key designs 1-4.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+__all__ = [
+    "RehyatParams", "RehyatPhi", "RehyatDebug", "RehyatError", "lib", "lib_path",
+    "EXPORTED_SYMBOLS", "F32", "BF16", "FLAG_FORCE_SIMT",
+    "rehyat_workspace_bytes", "rehyat_hybrid_attn_fwd", "rehyat_fwd_state", "rehyat_fwd_attn",
+    "rehyat_softmax_attn_fwd", "rehyat_state_bytes", "rehyat_state_init", "rehyat_step_workspace_bytes",
+    "rehyat_chunk_step", "rehyat_status_string", "rehyat_version",
+    "make_params", "hybrid_attn", "softmax_attn", "StreamingState",
+]
+
+F32, BF16 = 0, 1
+FLAG_FORCE_SIMT = 1
+
+STATUS = {0: "REHYAT_OK", 1: "REHYAT_ERR_INVALID_ARG", 2: "REHYAT_ERR_UNSUPPORTED",
+          3: "REHYAT_ERR_MISALIGNED", 4: "REHYAT_ERR_WORKSPACE", 5: "REHYAT_ERR_CUDA"}
+
+EXPORTED_SYMBOLS = (
+    "rehyat_workspace_bytes", "rehyat_hybrid_attn_fwd", "rehyat_fwd_state",
+    "rehyat_fwd_attn", "rehyat_softmax_attn_fwd", "rehyat_state_bytes", "rehyat_state_init",
+    "rehyat_step_workspace_bytes", "rehyat_chunk_step", "rehyat_status_string",
+    "rehyat_version",
+)
+
+
+class RehyatParams(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int), ("heads", ctypes.c_int), ("T", ctypes.c_int),
+                ("Hs", ctypes.c_int), ("Ws", ctypes.c_int), ("D", ctypes.c_int),
+                ("Dp", ctypes.c_int), ("Tc", ctypes.c_int), ("To", ctypes.c_int),
+                ("causal", ctypes.c_int), ("in_dtype", ctypes.c_int),
+                ("out_dtype", ctypes.c_int), ("scale", ctypes.c_float),
+                ("flags", ctypes.c_int)]
+
+
+class RehyatPhi(ctypes.Structure):
+    _fields_ = [("Wq", ctypes.c_void_p), ("bq", ctypes.c_void_p),
+                ("Wk", ctypes.c_void_p), ("bk", ctypes.c_void_p)]
+
+
+class RehyatDebug(ctypes.Structure):
+    _fields_ = [("aS", ctypes.c_void_p), ("nS", ctypes.c_void_p), ("c", ctypes.c_void_p),
+                ("aL", ctypes.c_void_p), ("nL", ctypes.c_void_p)]
+
+
+class RehyatError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+        self.status = status
+
+
+_LIB = None
+
+
+def lib_path() -> str:
+    return os.path.join(os.path.dirname(os.path.abspath(__file__)), "librehyat.so")
+
+
+def lib() -> ctypes.CDLL:
+    """Load librehyat.so (raises if it has not been built)."""
+    global _LIB
+    if _LIB is None:
+        path = lib_path()
+        if not os.path.exists(path):
+            raise ImportError(f"{path} is missing; build it with "
+                              "`python -m linear_attention_video_chunked_b200.build`")
+        L = ctypes.CDLL(path)
+        P = ctypes.POINTER
+        vp, sz, i = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+        L.rehyat_workspace_bytes.argtypes = [P(RehyatParams)]
+        L.rehyat_workspace_bytes.restype = sz
+        L.rehyat_hybrid_attn_fwd.argtypes = [P(RehyatParams), vp, vp, vp, P(RehyatPhi), vp, vp,
+                                             sz, P(RehyatDebug), vp]
+        L.rehyat_hybrid_attn_fwd.restype = i
+        L.rehyat_fwd_state.argtypes = [P(RehyatParams), vp, vp, P(RehyatPhi), vp, sz, vp]
+        L.rehyat_fwd_state.restype = i
+        L.rehyat_fwd_attn.argtypes = [P(RehyatParams), vp, vp, vp, P(RehyatPhi), vp, vp, sz,
+                                      P(RehyatDebug), vp]
+        L.rehyat_fwd_attn.restype = i
+        L.rehyat_softmax_attn_fwd.argtypes = [P(RehyatParams), vp, vp, vp, vp, vp]
+        L.rehyat_softmax_attn_fwd.restype = i
+        L.rehyat_state_bytes.argtypes = [P(RehyatParams)]
+        L.rehyat_state_bytes.restype = sz
+        L.rehyat_state_init.argtypes = [P(RehyatParams), vp, vp]
+        L.rehyat_state_init.restype = i
+        L.rehyat_step_workspace_bytes.argtypes = [P(RehyatParams)]
+        L.rehyat_step_workspace_bytes.restype = sz
+        L.rehyat_chunk_step.argtypes = [P(RehyatParams), vp, vp, vp, i, P(RehyatPhi), vp, vp, vp,
+                                        sz, P(RehyatDebug), vp]
+        L.rehyat_chunk_step.restype = i
+        L.rehyat_status_string.argtypes = [i]
+        L.rehyat_status_string.restype = ctypes.c_char_p
+        L.rehyat_version.argtypes = []
+        L.rehyat_version.restype = i
+        _LIB = L
+    return _LIB
+
+
+# ---------------------------------------------------------------- raw C ABI
+def rehyat_workspace_bytes(p: RehyatParams) -> int:
+    return lib().rehyat_workspace_bytes(ctypes.byref(p))
+
+
+def rehyat_hybrid_attn_fwd(p, q, k, v, phi, y, workspace, ws_bytes, dbg, stream) -> int:
+    return lib().rehyat_hybrid_attn_fwd(ctypes.byref(p), q, k, v, ctypes.byref(phi), y,
+                                        workspace, ws_bytes,
+                                        None if dbg is None else ctypes.byref(dbg), stream)
+
+
+def rehyat_fwd_state(p, k, v, phi, workspace, ws_bytes, stream) -> int:
+    return lib().rehyat_fwd_state(ctypes.byref(p), k, v, ctypes.byref(phi), workspace, ws_bytes,
+                                  stream)
+
+
+def rehyat_fwd_attn(p, q, k, v, phi, y, workspace, ws_bytes, dbg, stream) -> int:
+    return lib().rehyat_fwd_attn(ctypes.byref(p), q, k, v, ctypes.byref(phi), y, workspace,
+                                 ws_bytes, None if dbg is None else ctypes.byref(dbg), stream)
+
+
+def rehyat_softmax_attn_fwd(p, q, k, v, y, stream) -> int:
+    return lib().rehyat_softmax_attn_fwd(ctypes.byref(p), q, k, v, y, stream)
+
+
+def rehyat_state_bytes(p: RehyatParams) -> int:
+    return lib().rehyat_state_bytes(ctypes.byref(p))
+
+
+def rehyat_state_init(p, state, stream) -> int:
+    return lib().rehyat_state_init(ctypes.byref(p), state, stream)
+
+
+def rehyat_step_workspace_bytes(p: RehyatParams) -> int:
+    return lib().rehyat_step_workspace_bytes(ctypes.byref(p))
+
+
+def rehyat_chunk_step(p, q, k, v, nslices, phi, state, y, workspace, ws_bytes, dbg,
+                      stream) -> int:
+    return lib().rehyat_chunk_step(ctypes.byref(p), q, k, v, nslices, ctypes.byref(phi), state,
+                                   y, workspace, ws_bytes,
+                                   None if dbg is None else ctypes.byref(dbg), stream)
+
+
+def rehyat_status_string(status: int) -> str:
+    return lib().rehyat_status_string(status).decode()
+
+
+def rehyat_version() -> int:
+    return lib().rehyat_version()
+
+
+# ------------------------------------------------------------- torch layer
+def make_params(*, batch, heads, T, Hs, Ws, D, Dp, Tc, To, causal, in_dtype=BF16,
+                out_dtype=F32, scale=0.0, flags=0) -> RehyatParams:
+    return RehyatParams(batch, heads, T, Hs, Ws, D, Dp, Tc, To, int(causal), in_dtype,
+                        out_dtype, float(scale), flags)
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t == torch.bfloat16:
+        return BF16
+    if t == torch.float32:
+        return F32
+    raise TypeError(f"unsupported dtype {t}")
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise RehyatError(status, where)
+
+
+def _stream_handle(stream=None) -> int:
+    torch = _torch()
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _phi_struct(Wq, bq, Wk, bk) -> RehyatPhi:
+    for t in (Wq, bq, Wk, bk):
+        if t.dtype != _torch().float32 or not t.is_cuda or not t.is_contiguous():
+            raise TypeError("phi parameters must be contiguous fp32 CUDA tensors")
+    return RehyatPhi(Wq.data_ptr(), bq.data_ptr(), Wk.data_ptr(), bk.data_ptr())
+
+
+def _debug_tensors(shape4, device):
+    torch = _torch()
+    B, H, N, D = shape4
+    d = dict(aS=torch.empty(B, H, N, D, device=device), nS=torch.empty(B, H, N, device=device),
+             c=torch.empty(B, H, N, device=device), aL=torch.empty(B, H, N, D, device=device),
+             nL=torch.empty(B, H, N, device=device))
+    st = RehyatDebug(*(d[k].data_ptr() for k in ("aS", "nS", "c", "aL", "nL")))
+    return d, st
+
+
+def hybrid_attn(q, k, v, Wq, bq, Wk, bk, *, T, Hs, Ws, Tc, To, causal, out_dtype=None,
+                scale=0.0, debug=False, force_simt=False, workspace=None, out=None,
+                stream=None):
+    """ReHyAt hybrid attention of torch CUDA tensors q, k, v [B, h, N, D].
+
+    Returns y (and a dict of branch partials when ``debug``)."""
+    torch = _torch()
+    B, H, N, D = q.shape
+    if N != T * Hs * Ws:
+        raise ValueError("q.shape[2] must equal T*Hs*Ws")
+    Dp = 2 * Wq.shape[-1]
+    out_dtype = torch.float32 if out_dtype is None else out_dtype
+    p = make_params(batch=B, heads=H, T=T, Hs=Hs, Ws=Ws, D=D, Dp=Dp, Tc=Tc, To=To,
+                    causal=causal, in_dtype=_dtype_code(q.dtype),
+                    out_dtype=_dtype_code(out_dtype), scale=scale,
+                    flags=FLAG_FORCE_SIMT if force_simt else 0)
+    y = torch.empty(B, H, N, D, dtype=out_dtype, device=q.device) if out is None else out
+    nbytes = rehyat_workspace_bytes(p)
+    if nbytes == 0:
+        raise RehyatError(1, "rehyat_workspace_bytes")
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    dbg_t, dbg_s = _debug_tensors((B, H, N, D), q.device) if debug else (None, None)
+    st = rehyat_hybrid_attn_fwd(p, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                _phi_struct(Wq, bq, Wk, bk), y.data_ptr(),
+                                workspace.data_ptr(), workspace.numel(), dbg_s,
+                                _stream_handle(stream))
+    _check(st, "rehyat_hybrid_attn_fwd")
+    return (y, dbg_t) if debug else y
+
+
+def softmax_attn(q, k, v, *, out_dtype=None, scale=0.0, force_simt=False, out=None,
+                 stream=None):
+    """Plain softmax attention over all keys (the dense comparator)."""
+    torch = _torch()
+    B, H, N, D = q.shape
+    out_dtype = torch.float32 if out_dtype is None else out_dtype
+    p = make_params(batch=B, heads=H, T=1, Hs=1, Ws=N, D=D, Dp=32, Tc=1, To=0, causal=0,
+                    in_dtype=_dtype_code(q.dtype), out_dtype=_dtype_code(out_dtype),
+                    scale=scale, flags=FLAG_FORCE_SIMT if force_simt else 0)
+    y = torch.empty(B, H, N, D, dtype=out_dtype, device=q.device) if out is None else out
+    st = rehyat_softmax_attn_fwd(p, q.data_ptr(), k.data_ptr(), v.data_ptr(), y.data_ptr(),
+                                 _stream_handle(stream))
+    _check(st, "rehyat_softmax_attn_fwd")
+    return y
+
+
+class StreamingState:
+    """Caller-owned state of the causal chunk-wise RNN (Key design 4).
+
+    ``step(q, k, v)`` consumes the next chunk ([B, h, n*HW, D], n <= Tc
+    slices) and returns its outputs; memory stays constant over any number of
+    steps.  ``snapshot()``/``restore()`` copy the opaque state bytes."""
+
+    def __init__(self, *, batch, heads, Hs, Ws, D, Dp, Tc, To, Wq, bq, Wk, bk,
+                 in_dtype, out_dtype=None, scale=0.0, force_simt=False, device="cuda"):
+        torch = _torch()
+        self.out_dtype = torch.float32 if out_dtype is None else out_dtype
+        self.HW = Hs * Ws
+        self.Tc = Tc
+        self.p = make_params(batch=batch, heads=heads, T=Tc, Hs=Hs, Ws=Ws, D=D, Dp=Dp, Tc=Tc,
+                             To=To, causal=1, in_dtype=_dtype_code(in_dtype),
+                             out_dtype=_dtype_code(self.out_dtype), scale=scale,
+                             flags=FLAG_FORCE_SIMT if force_simt else 0)
+        self.phi_tensors = (Wq, bq, Wk, bk)
+        self.phi = _phi_struct(Wq, bq, Wk, bk)
+        nstate = rehyat_state_bytes(self.p)
+        nws = rehyat_step_workspace_bytes(self.p)
+        if nstate == 0 or nws == 0:
+            raise RehyatError(1, "rehyat_state_bytes")
+        self.state = torch.empty(nstate, dtype=torch.uint8, device=device)
+        self.workspace = torch.empty(nws, dtype=torch.uint8, device=device)
+        self.reset()
+
+    def reset(self, stream=None):
+        _check(rehyat_state_init(self.p, self.state.data_ptr(), _stream_handle(stream)),
+               "rehyat_state_init")
+
+    def step(self, q, k, v, *, debug=False, out=None, stream=None):
+        torch = _torch()
+        B, H, rows, D = q.shape
+        n = rows // self.HW
+        if n * self.HW != rows:
+            raise ValueError("a chunk must hold whole slices")
+        y = torch.empty(B, H, rows, D, dtype=self.out_dtype, device=q.device) if out is None else out
+        dbg_t, dbg_s = _debug_tensors((B, H, rows, D), q.device) if debug else (None, None)
+        st = rehyat_chunk_step(self.p, q.data_ptr(), k.data_ptr(), v.data_ptr(), n, self.phi,
+                               self.state.data_ptr(), y.data_ptr(), self.workspace.data_ptr(),
+                               self.workspace.numel(), dbg_s, _stream_handle(stream))
+        _check(st, "rehyat_chunk_step")
+        return (y, dbg_t) if debug else y
+
+    def snapshot(self):
+        return self.state.clone()
+
+    def restore(self, saved):
+        self.state.copy_(saved)

@@ -1,0 +1,380 @@
+// C ABI of librehyat.so: argument checks, workspace/state layout, dispatch.
+// The method and every entry point are documented in include/rehyat.h.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "internal.h"
+
+namespace rehyat {
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int elem_bytes(int dtype) { return dtype == REHYAT_BF16 ? 2 : 4; }
+
+rehyat_status check_params(const rehyat_params* p) {
+  if (!p) return REHYAT_ERR_INVALID_ARG;
+  if (p->batch < 1 || p->heads < 1 || p->T < 1 || p->Hs < 1 || p->Ws < 1 || p->Tc < 1 ||
+      p->To < 0)
+    return REHYAT_ERR_INVALID_ARG;
+  if (p->causal != 0 && p->causal != 1) return REHYAT_ERR_INVALID_ARG;
+  if ((p->in_dtype != REHYAT_F32 && p->in_dtype != REHYAT_BF16) ||
+      (p->out_dtype != REHYAT_F32 && p->out_dtype != REHYAT_BF16))
+    return REHYAT_ERR_INVALID_ARG;
+  if (!(p->scale >= 0.f) || isinf(p->scale)) return REHYAT_ERR_INVALID_ARG;
+  if (p->D != 32 && p->D != 64 && p->D != 128) return REHYAT_ERR_UNSUPPORTED;
+  if (p->Dp != 32 && p->Dp != 64 && p->Dp != 128 && p->Dp != 256) return REHYAT_ERR_UNSUPPORTED;
+  // Index arithmetic: rows per (b, h) and grid sizes must fit in 32 bits.
+  const long long HW = static_cast<long long>(p->Hs) * p->Ws;
+  const long long N = HW * p->T;
+  if (N * p->D >= (1LL << 31) || static_cast<long long>(p->batch) * p->heads >= 65535)
+    return REHYAT_ERR_UNSUPPORTED;
+  return REHYAT_OK;
+}
+
+int nchunks_of(const rehyat_params* p) { return (p->T + p->Tc - 1) / p->Tc; }
+
+struct FwdWorkspace {
+  size_t P_off, z_off, SL_off, zL_off, wimg_off, total;
+};
+
+// phi_q weight image (bf16, all heads) used by the tensor-core kernel.
+size_t wimg_bytes(const rehyat_params* p) {
+  return static_cast<size_t>(p->heads) * p->Dp * p->D * 2;
+}
+
+FwdWorkspace fwd_layout(const rehyat_params* p) {
+  const size_t BH = static_cast<size_t>(p->batch) * p->heads;
+  const size_t PD = static_cast<size_t>(p->Dp) * p->D;
+  FwdWorkspace w;
+  w.P_off = 0;
+  w.z_off = align_up(w.P_off + BH * p->T * PD * sizeof(float));
+  w.SL_off = align_up(w.z_off + BH * p->T * p->Dp * sizeof(float));
+  w.zL_off = align_up(w.SL_off + BH * nchunks_of(p) * PD * sizeof(float));
+  w.wimg_off = align_up(w.zL_off + BH * nchunks_of(p) * p->Dp * sizeof(float));
+  w.total = align_up(w.wimg_off + wimg_bytes(p));
+  return w;
+}
+
+// Whether the tensor-core attention kernel (and its weight image) is used.
+bool tc_path(const rehyat_params* p) {
+  return !(p->flags & REHYAT_FLAG_FORCE_SIMT) &&
+         tc_attn_eligible(p->in_dtype == REHYAT_BF16, p->D, p->Dp);
+}
+
+struct StateLayout {
+  size_t s_off, z_off, rk_off, rv_off, total;
+};
+
+StateLayout state_layout(const rehyat_params* p) {
+  const size_t BH = static_cast<size_t>(p->batch) * p->heads;
+  const size_t HW = static_cast<size_t>(p->Hs) * p->Ws;
+  StateLayout s;
+  s.s_off = kAlign;  // header: the slice counter (int64)
+  s.z_off = align_up(s.s_off + BH * p->Dp * p->D * sizeof(float));
+  s.rk_off = align_up(s.z_off + BH * p->Dp * sizeof(float));
+  const size_t ring = BH * p->To * HW * p->D * elem_bytes(p->in_dtype);
+  s.rv_off = align_up(s.rk_off + ring);
+  s.total = align_up(s.rv_off + ring);
+  return s;
+}
+
+struct StepWorkspace {
+  size_t P_off, z_off, wimg_off, total;
+  int nslots;
+};
+
+StepWorkspace step_layout(const rehyat_params* p) {
+  const size_t BH = static_cast<size_t>(p->batch) * p->heads;
+  StepWorkspace w;
+  w.nslots = p->To + p->Tc;  // at most this many slices leave per step
+  w.P_off = 0;
+  w.z_off = align_up(BH * w.nslots * static_cast<size_t>(p->Dp) * p->D * sizeof(float));
+  w.wimg_off = align_up(w.z_off + BH * w.nslots * p->Dp * sizeof(float));
+  w.total = align_up(w.wimg_off + wimg_bytes(p));
+  return w;
+}
+
+float logit_scale(const rehyat_params* p) {
+  return p->scale > 0.f ? p->scale : 1.0f / sqrtf(static_cast<float>(p->D));
+}
+
+AttnParams base_attn(const rehyat_params* p, const void* q, const void* k, const void* v,
+                     const rehyat_phi* phi, void* y, const rehyat_debug* dbg) {
+  AttnParams a = {};
+  a.q = q; a.k = k; a.v = v;
+  a.Wq = phi ? phi->Wq : nullptr;
+  a.bq = phi ? phi->bq : nullptr;
+  a.y = y;
+  if (dbg) {
+    a.dbg_aS = dbg->aS; a.dbg_nS = dbg->nS; a.dbg_c = dbg->c;
+    a.dbg_aL = dbg->aL; a.dbg_nL = dbg->nL;
+  }
+  a.BH = p->batch * p->heads;
+  a.heads = p->heads;
+  a.T = p->T;
+  a.HW = p->Hs * p->Ws;
+  a.D = p->D;
+  a.Dp = p->Dp;
+  a.Tc = p->Tc;
+  a.To = p->To;
+  a.in_bf16 = p->in_dtype == REHYAT_BF16;
+  a.out_bf16 = p->out_dtype == REHYAT_BF16;
+  a.w_bf16 = a.in_bf16;
+  a.scale_log2 = logit_scale(p) * 1.4426950408889634f;
+  return a;
+}
+
+rehyat_status check_phi(const rehyat_phi* phi) {
+  if (!phi || !phi->Wq || !phi->bq || !phi->Wk || !phi->bk) return REHYAT_ERR_INVALID_ARG;
+  if (!aligned16(phi->Wq) || !aligned16(phi->Wk) || (reinterpret_cast<uintptr_t>(phi->bq) & 3) ||
+      (reinterpret_cast<uintptr_t>(phi->bk) & 3))
+    return REHYAT_ERR_MISALIGNED;
+  return REHYAT_OK;
+}
+
+rehyat_status check_dbg(const rehyat_debug* dbg) {
+  if (!dbg) return REHYAT_OK;
+  const void* ptrs[5] = {dbg->aS, dbg->nS, dbg->c, dbg->aL, dbg->nL};
+  for (const void* q : ptrs)
+    if (q && (reinterpret_cast<uintptr_t>(q) & 3)) return REHYAT_ERR_MISALIGNED;
+  return REHYAT_OK;
+}
+
+rehyat_status to_status(cudaError_t e) { return e == cudaSuccess ? REHYAT_OK : REHYAT_ERR_CUDA; }
+
+bool use_tc(const rehyat_params* p, const AttnParams& a) {
+  if (p->flags & REHYAT_FLAG_FORCE_SIMT) return false;
+  return tc_attn_supported(a);
+}
+
+cudaError_t run_attn(const rehyat_params* p, const AttnParams& a, cudaStream_t s) {
+  if (use_tc(p, a)) return launch_attn_tc(a, s);
+  return launch_attn_simt(a, s);
+}
+
+}  // namespace
+}  // namespace rehyat
+
+using namespace rehyat;
+
+extern "C" {
+
+int rehyat_version(void) { return 100; }
+
+const char* rehyat_status_string(rehyat_status s) {
+  switch (s) {
+    case REHYAT_OK: return "ok";
+    case REHYAT_ERR_INVALID_ARG: return "invalid argument";
+    case REHYAT_ERR_UNSUPPORTED: return "unsupported shape";
+    case REHYAT_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case REHYAT_ERR_WORKSPACE: return "workspace or state too small";
+    case REHYAT_ERR_CUDA: return "CUDA launch error";
+  }
+  return "unknown status";
+}
+
+size_t rehyat_workspace_bytes(const rehyat_params* p) {
+  if (check_params(p) != REHYAT_OK) return 0;
+  return fwd_layout(p).total;
+}
+
+rehyat_status rehyat_fwd_state(const rehyat_params* p, const void* k, const void* v,
+                               const rehyat_phi* phi, void* workspace, size_t ws_bytes,
+                               void* stream) {
+  rehyat_status st = check_params(p);
+  if (st != REHYAT_OK) return st;
+  if (!k || !v || !workspace) return REHYAT_ERR_INVALID_ARG;
+  if ((st = check_phi(phi)) != REHYAT_OK) return st;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(workspace)) return REHYAT_ERR_MISALIGNED;
+  const FwdWorkspace w = fwd_layout(p);
+  if (ws_bytes < w.total) return REHYAT_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  float* P = reinterpret_cast<float*>(ws + w.P_off);
+  float* z = reinterpret_cast<float*>(ws + w.z_off);
+  float* SL = reinterpret_cast<float*>(ws + w.SL_off);
+  float* zL = reinterpret_cast<float*>(ws + w.zL_off);
+  const int BH = p->batch * p->heads;
+  const int HW = p->Hs * p->Ws;
+
+  PartialParams pp = {};
+  pp.k = k; pp.v = v;
+  pp.rows_per_bh = static_cast<long long>(p->T) * HW;
+  pp.Wk = phi->Wk; pp.bk = phi->bk;
+  pp.P = P; pp.z = z;
+  pp.BH = BH; pp.heads = p->heads; pp.HW = HW; pp.D = p->D; pp.Dp = p->Dp; pp.To = p->To;
+  pp.nslots = p->T;
+  pp.in_bf16 = p->in_dtype == REHYAT_BF16;
+  pp.w_bf16 = pp.in_bf16;
+  cudaError_t e = launch_partials_simt(pp, s);
+  if (e != cudaSuccess) return to_status(e);
+  e = launch_scan(P, z, SL, zL, BH, p->T, p->Tc, p->To, nchunks_of(p), p->Dp, p->D, p->causal,
+                  s);
+  if (e != cudaSuccess) return to_status(e);
+  if (tc_path(p)) e = launch_wq_image(phi->Wq, ws + w.wimg_off, p->heads, p->D, p->Dp, s);
+  return to_status(e);
+}
+
+rehyat_status rehyat_fwd_attn(const rehyat_params* p, const void* q, const void* k,
+                              const void* v, const rehyat_phi* phi, void* y,
+                              const void* workspace, size_t ws_bytes, const rehyat_debug* dbg,
+                              void* stream) {
+  rehyat_status st = check_params(p);
+  if (st != REHYAT_OK) return st;
+  if (!q || !k || !v || !y || !workspace) return REHYAT_ERR_INVALID_ARG;
+  if ((st = check_phi(phi)) != REHYAT_OK) return st;
+  if ((st = check_dbg(dbg)) != REHYAT_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(y) || !aligned16(workspace))
+    return REHYAT_ERR_MISALIGNED;
+  const FwdWorkspace w = fwd_layout(p);
+  if (ws_bytes < w.total) return REHYAT_ERR_WORKSPACE;
+  const char* ws = static_cast<const char*>(workspace);
+  AttnParams a = base_attn(p, q, k, v, phi, y, dbg);
+  a.rows_per_bh = static_cast<long long>(p->T) * p->Hs * p->Ws;
+  a.SL = reinterpret_cast<const float*>(ws + w.SL_off);
+  a.zL = reinterpret_cast<const float*>(ws + w.zL_off);
+  a.nchunks = nchunks_of(p);
+  if (tc_path(p)) a.wq_img = ws + w.wimg_off;
+  return to_status(run_attn(p, a, static_cast<cudaStream_t>(stream)));
+}
+
+rehyat_status rehyat_hybrid_attn_fwd(const rehyat_params* p, const void* q, const void* k,
+                                     const void* v, const rehyat_phi* phi, void* y,
+                                     void* workspace, size_t ws_bytes,
+                                     const rehyat_debug* dbg, void* stream) {
+  // Check everything both stages need before enqueueing either.
+  rehyat_status st = check_params(p);
+  if (st != REHYAT_OK) return st;
+  if (!q || !k || !v || !y || !workspace) return REHYAT_ERR_INVALID_ARG;
+  if ((st = check_phi(phi)) != REHYAT_OK) return st;
+  if ((st = check_dbg(dbg)) != REHYAT_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(y) || !aligned16(workspace))
+    return REHYAT_ERR_MISALIGNED;
+  if (ws_bytes < fwd_layout(p).total) return REHYAT_ERR_WORKSPACE;
+  st = rehyat_fwd_state(p, k, v, phi, workspace, ws_bytes, stream);
+  if (st != REHYAT_OK) return st;
+  return rehyat_fwd_attn(p, q, k, v, phi, y, workspace, ws_bytes, dbg, stream);
+}
+
+rehyat_status rehyat_softmax_attn_fwd(const rehyat_params* p, const void* q, const void* k,
+                                      const void* v, void* y, void* stream) {
+  rehyat_status st = check_params(p);
+  if (st != REHYAT_OK) return st;
+  if (!q || !k || !v || !y) return REHYAT_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(y))
+    return REHYAT_ERR_MISALIGNED;
+  // One chunk spanning all T slices, no overlap, no linear branch.
+  rehyat_params full = *p;
+  full.Tc = p->T;
+  full.To = 0;
+  AttnParams a = base_attn(&full, q, k, v, nullptr, y, nullptr);
+  a.rows_per_bh = static_cast<long long>(p->T) * p->Hs * p->Ws;
+  a.nchunks = 1;
+  a.full_softmax = 1;
+  return to_status(run_attn(&full, a, static_cast<cudaStream_t>(stream)));
+}
+
+size_t rehyat_state_bytes(const rehyat_params* p) {
+  if (check_params(p) != REHYAT_OK) return 0;
+  return state_layout(p).total;
+}
+
+size_t rehyat_step_workspace_bytes(const rehyat_params* p) {
+  if (check_params(p) != REHYAT_OK) return 0;
+  return step_layout(p).total;
+}
+
+rehyat_status rehyat_state_init(const rehyat_params* p, void* state, void* stream) {
+  rehyat_status st = check_params(p);
+  if (st != REHYAT_OK) return st;
+  if (!state) return REHYAT_ERR_INVALID_ARG;
+  if (!aligned16(state)) return REHYAT_ERR_MISALIGNED;
+  const StateLayout L = state_layout(p);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // Header (counter = 0) and s, z = 0.  The ring needs no clearing: only
+  // slots written since the last reset are ever read.
+  return to_status(cudaMemsetAsync(state, 0, L.rk_off, s));
+}
+
+rehyat_status rehyat_chunk_step(const rehyat_params* p, const void* q, const void* k,
+                                const void* v, int nslices, const rehyat_phi* phi, void* state,
+                                void* y, void* workspace, size_t ws_bytes,
+                                const rehyat_debug* dbg, void* stream) {
+  rehyat_status st = check_params(p);
+  if (st != REHYAT_OK) return st;
+  if (p->causal != 1) return REHYAT_ERR_INVALID_ARG;
+  if (nslices < 1 || nslices > p->Tc) return REHYAT_ERR_INVALID_ARG;
+  if (!q || !k || !v || !y || !state || !workspace) return REHYAT_ERR_INVALID_ARG;
+  if ((st = check_phi(phi)) != REHYAT_OK) return st;
+  if ((st = check_dbg(dbg)) != REHYAT_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(y) || !aligned16(state) ||
+      !aligned16(workspace))
+    return REHYAT_ERR_MISALIGNED;
+  const StepWorkspace w = step_layout(p);
+  if (ws_bytes < w.total) return REHYAT_ERR_WORKSPACE;
+  const StateLayout L = state_layout(p);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* stb = static_cast<char*>(state);
+  long long* seen = reinterpret_cast<long long*>(stb);
+  float* s_state = reinterpret_cast<float*>(stb + L.s_off);
+  float* z_state = reinterpret_cast<float*>(stb + L.z_off);
+  void* rk = stb + L.rk_off;
+  void* rv = stb + L.rv_off;
+  char* ws = static_cast<char*>(workspace);
+  float* P = reinterpret_cast<float*>(ws + w.P_off);
+  float* zp = reinterpret_cast<float*>(ws + w.z_off);
+  const int BH = p->batch * p->heads;
+  const int HW = p->Hs * p->Ws;
+  const long long nrows = static_cast<long long>(nslices) * HW;
+
+  // 1. Softmax over ring + chunk, linear branch from (s, z), joint norm.
+  AttnParams a = base_attn(p, q, k, v, phi, y, dbg);
+  a.rows_per_bh = nrows;
+  a.rk = rk; a.rv = rv;
+  a.ring_rows_per_bh = static_cast<long long>(p->To) * HW;
+  a.seen = seen;
+  a.SL = s_state; a.zL = z_state;
+  a.nchunks = 1;
+  a.nq_slices = nslices;
+  cudaError_t e = cudaSuccess;
+  if (tc_path(p)) {
+    e = launch_wq_image(phi->Wq, ws + w.wimg_off, p->heads, p->D, p->Dp, s);
+    if (e != cudaSuccess) return to_status(e);
+    a.wq_img = ws + w.wimg_off;
+  }
+  e = run_attn(p, a, s);
+  if (e != cudaSuccess) return to_status(e);
+
+  // 2. Fold the slices that leave the softmax window into (s, z).
+  PartialParams pp = {};
+  pp.k = k; pp.v = v;
+  pp.rows_per_bh = nrows;
+  pp.rk = rk; pp.rv = rv;
+  pp.ring_rows_per_bh = a.ring_rows_per_bh;
+  pp.seen = seen;
+  pp.Wk = phi->Wk; pp.bk = phi->bk;
+  pp.P = P; pp.z = zp;
+  pp.BH = BH; pp.heads = p->heads; pp.HW = HW; pp.D = p->D; pp.Dp = p->Dp; pp.To = p->To;
+  pp.nslots = w.nslots;
+  pp.nq_slices = nslices;
+  pp.in_bf16 = p->in_dtype == REHYAT_BF16;
+  pp.w_bf16 = pp.in_bf16;
+  e = launch_partials_simt(pp, s);
+  if (e != cudaSuccess) return to_status(e);
+  e = launch_state_add(P, zp, s_state, z_state, seen, BH, p->Dp, p->D, p->To, nslices,
+                       w.nslots, s);
+  if (e != cudaSuccess) return to_status(e);
+  // 3. Keep the newest T_o slices in the ring; 4. advance the counter.
+  e = launch_ring_update(k, v, rk, rv, seen, BH, HW, p->D, p->To, nslices,
+                         elem_bytes(p->in_dtype), s);
+  if (e != cudaSuccess) return to_status(e);
+  return to_status(launch_advance(seen, nslices, s));
+}
+
+}  // extern "C"

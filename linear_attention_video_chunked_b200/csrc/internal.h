@@ -1,0 +1,93 @@
+// Internal declarations shared by the translation units of librehyat.so.
+// Not part of the C ABI (see include/rehyat.h for that).
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "rehyat.h"
+
+namespace rehyat {
+
+// Softmax window + linear readout + joint normalisation for the query rows of
+// one or more chunks ("Key designs 1, 2 and 4" of the ReHyAt note).
+//
+// Two modes:
+//  * full  (seen == nullptr): chunk t = blockIdx.y covers query rows
+//    [t*Tc*HW, min(T,(t+1)*Tc)*HW) of q; keys are rows [w_t*HW, end_t*HW) of
+//    k, v with w_t = max(t*Tc - To, 0).
+//  * step  (seen != nullptr): one chunk of nq_slices slices; keys are ring
+//    rows [0, min(To, *seen)*HW) followed by all rows of k, v.
+// The linear state of chunk t is SL + (bh*nchunks + t)*Dp*D (image layout,
+// layout.cuh sl_index), zL + (bh*nchunks + t)*Dp.  full_softmax skips the
+// linear branch.
+struct AttnParams {
+  const void *q, *k, *v;
+  long long rows_per_bh;     // rows of q/k/v (and y) per (b, h)
+  const void *rk, *rv;       // ring keys/values [BH][To*HW][D] (step mode)
+  long long ring_rows_per_bh;
+  const long long* seen;     // device slice counter (step mode) or nullptr
+  const float *SL, *zL;      // linear-set state per chunk
+  const float *Wq, *bq;      // phi_q parameters, fp32 [h][2][D][Dp/2], [h][2][Dp/2]
+  const void* wq_img;        // bf16 phi_q weight image per head (tensor-core path) or nullptr
+  void* y;
+  float *dbg_aS, *dbg_nS, *dbg_c, *dbg_aL, *dbg_nL;
+  int BH, heads, T, HW, D, Dp, Tc, To, nchunks, nq_slices;
+  int in_bf16, out_bf16, w_bf16, full_softmax;
+  float scale_log2;          // logit scale * log2(e)
+};
+
+// Per-slice linear state: P_i = sum_{rows of slice i} phi_k(k) v^T ([Dp][D])
+// and z_i = sum phi_k(k) ([Dp]).
+//  * full mode (seen == nullptr): slice i = rows [i*HW, (i+1)*HW) of k, v,
+//    for i in [0, nslots).
+//  * step mode: slot i holds the i-th slice leaving the softmax window; its
+//    global index is g = seen - r + i with r = min(To, seen); it lives in the
+//    ring (slot g % To) if g < seen, else in the chunk (slice g - seen).
+//    Slots past the number of leaving slices are skipped.
+struct PartialParams {
+  const void *k, *v;
+  long long rows_per_bh;
+  const void *rk, *rv;
+  long long ring_rows_per_bh;
+  const long long* seen;
+  const float *Wk, *bk;
+  float *P, *z;              // [BH][nslots][Dp][D], [BH][nslots][Dp]
+  int BH, heads, HW, D, Dp, To, nslots, nq_slices;
+  int in_bf16, w_bf16;
+};
+
+// ---- SIMT (fp32 CUDA-core) kernels: every supported shape, both dtypes.
+cudaError_t launch_attn_simt(const AttnParams& p, cudaStream_t s);
+cudaError_t launch_partials_simt(const PartialParams& p, cudaStream_t s);
+
+// bf16 image of the phi_q weights (layout.cuh, wimg_index) for the
+// tensor-core readout: out [heads][Dp*D].
+cudaError_t launch_wq_image(const float* Wq, void* out, int heads, int D, int Dp,
+                            cudaStream_t s);
+bool tc_attn_eligible(int in_bf16, int D, int Dp);
+
+// Linear-set state per chunk from the per-slice states (full mode).
+// causal: S^L_t = sum_{i < w_t} P_i.  bidirectional: S^L_t = sum_{i < w_t} P_i
+// + sum_{i >= end_t} P_i (prefix plus suffix, no subtraction).  P is plain
+// [Dp][D]; S^L is written in the image layout (layout.cuh, sl_index).
+cudaError_t launch_scan(const float* P, const float* z, float* SL, float* zL,
+                        int BH, int T, int Tc, int To, int nchunks, int Dp,
+                        int D, int causal, cudaStream_t s);
+
+// Streaming helpers (step mode; all read the device slice counter).
+cudaError_t launch_state_add(const float* P, const float* zp, float* s_state,
+                             float* z_state, const long long* seen, int BH,
+                             int Dp, int D, int To, int nq_slices, int nslots,
+                             cudaStream_t s);
+cudaError_t launch_ring_update(const void* k, const void* v, void* rk, void* rv,
+                               const long long* seen, int BH, int HW, int D,
+                               int To, int nq_slices, int elem_bytes,
+                               cudaStream_t s);
+cudaError_t launch_advance(long long* seen, int nq_slices, cudaStream_t s);
+
+// ---- tcgen05 / TMA kernels (bf16, D = 128).  Return cudaErrorNotSupported
+// when the shape is outside what they handle.
+bool tc_attn_supported(const AttnParams& p);
+cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s);
+
+}  // namespace rehyat

@@ -1,0 +1,46 @@
+// Memory layouts shared by the kernels of librehyat.so.
+//
+// Tensor-core operands live in shared memory in the 128-byte-swizzled,
+// K-major form that TMA writes and tcgen05.mma reads: a "box" is a run of
+// 128-byte rows; within each 1024-byte atom (eight rows) the 16-byte chunk c
+// of row r sits at chunk position c ^ (r & 7).  Operands that are not loaded
+// by a tensor map are stored in global memory already in this form (an
+// "image"), so a single bulk copy puts them in place.
+#pragma once
+#include <stdint.h>
+
+namespace rehyat {
+
+// Width of one feature piece of the linear readout (the tensor-core tail
+// processes the D' features in pieces of at most 128).
+__host__ __device__ __forceinline__ int piece_width(int Dp) { return Dp < 128 ? Dp : 128; }
+
+// S^L (and the streaming s): logical [Dp][D] fp32, stored per feature piece
+// as a K-major tf32 operand [D rows][piece features]: boxes of 32 features,
+// each box D rows x 128 bytes.
+__host__ __device__ __forceinline__ long long sl_index(int f, int d, int D, int Dp) {
+  const int pw = piece_width(Dp);
+  const int piece = f / pw;
+  const int fl = f - piece * pw;
+  const int box = fl >> 5;
+  const int chunk = (fl >> 2) & 7;
+  const int w = fl & 3;
+  return static_cast<long long>(piece) * D * pw + static_cast<long long>(box) * D * 32 +
+         d * 32 + ((chunk ^ (d & 7)) << 2) + w;
+}
+
+// phi_q weights of one head: logical W[d][f] (f over both parts), stored per
+// feature piece as a K-major bf16 operand [piece features][D]: boxes of 64
+// D-elements, each box pw rows x 128 bytes.
+__host__ __device__ __forceinline__ long long wimg_index(int f, int d, int D, int Dp) {
+  const int pw = piece_width(Dp);
+  const int piece = f / pw;
+  const int n = f - piece * pw;
+  const int box = d >> 6;
+  const int chunk = (d >> 3) & 7;
+  const int w = d & 7;
+  return static_cast<long long>(piece) * pw * D + static_cast<long long>(box) * pw * 64 +
+         n * 64 + ((chunk ^ (n & 7)) << 3) + w;
+}
+
+}  // namespace rehyat

@@ -1,0 +1,511 @@
+// fp32 CUDA-core kernels for ReHyAt's chunked hybrid attention.
+//
+// They cover every supported shape (D in {32, 64, 128}, Dp in {32..256}) and
+// both input dtypes, compute in fp32 throughout, and are the exact-fp32 path
+// (the tensor-core kernels round P and phi to narrower types).
+//
+// Source of the arithmetic: "ReHyAt: Recurrent Hybrid Attention for Video
+// Diffusion Transformers" (papernotes.org note), Method, Key designs 1-4:
+// window softmax with stabiliser c_t, linear branch phi_q(q) (sum phi_k v^T),
+// joint normalisation, overlap set, causal set and chunk-wise state.
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "internal.h"
+#include "layout.cuh"
+
+namespace rehyat {
+namespace {
+
+constexpr float kLn2 = 0.69314718055994530942f;
+
+__device__ __forceinline__ float load_in(const void* base, long long i, int bf16) {
+  if (bf16) {
+    unsigned short b = reinterpret_cast<const unsigned short*>(base)[i];
+    return __uint_as_float(static_cast<unsigned>(b) << 16);
+  }
+  return reinterpret_cast<const float*>(base)[i];
+}
+
+// Round an fp32 value to the nearest bf16 value (ties to even), kept as fp32.
+__device__ __forceinline__ float round_bf16(float x) {
+  return __bfloat162float(__float2bfloat16_rn(x));
+}
+
+__device__ __forceinline__ float load_w(const float* W, long long i, int w_bf16) {
+  float w = __ldg(W + i);
+  return w_bf16 ? round_bf16(w) : w;
+}
+
+__device__ __forceinline__ void store_out(void* base, long long i, float x, int bf16) {
+  if (bf16)
+    reinterpret_cast<__nv_bfloat16*>(base)[i] = __float2bfloat16_rn(x);
+  else
+    reinterpret_cast<float*>(base)[i] = x;
+}
+
+// phi feature f of part W[h][f / half][:, f % half]: column index helpers.
+__device__ __forceinline__ long long w_index(int h, int D, int Dp, int d, int f) {
+  const int half = Dp >> 1;
+  const int part = f >= half;
+  const int col = f - part * half;
+  return ((static_cast<long long>(h) * 2 + part) * D + d) * half + col;
+}
+__device__ __forceinline__ long long b_index(int h, int Dp, int f) {
+  const int half = Dp >> 1;
+  const int part = f >= half;
+  return (static_cast<long long>(h) * 2 + part) * half + (f - part * half);
+}
+
+// ---------------------------------------------------------------------------
+// Window softmax + linear readout + joint normalisation.
+// Block: 128 threads = 32 query rows x 4 lanes; key tiles of 32.
+// ---------------------------------------------------------------------------
+constexpr int kBQ = 32;
+constexpr int kBK = 32;
+
+template <int D>
+__global__ void __launch_bounds__(128) attn_simt_kernel(AttnParams P) {
+  extern __shared__ float smem[];
+  float* Qs = smem;                        // [kBQ][D]
+  float* Ks = Qs + kBQ * D;                // [kBK][D + 1]
+  float* Vs = Ks + kBK * (D + 1);          // [kBK][D]
+  float* Ps = Vs + kBK * D;                // [kBQ][kBK + 1]
+  float* Fq = Qs + kBQ * D;                // [kBQ][Dp], reuses Ks.. after the loop
+
+  const int tid = threadIdx.x;
+  const int r = tid >> 2;
+  const int lane4 = tid & 3;
+  const int t = blockIdx.y;
+  const int bh = blockIdx.z;
+  const int h = bh % P.heads;
+
+  // Query rows and key ranges of this chunk.
+  long long q_first, q_end;
+  const void *ka, *va, *kb = nullptr, *vb = nullptr;
+  long long ka_off, na, kb_off = 0, nb = 0;
+  if (P.seen == nullptr) {
+    const int first = t * P.Tc;
+    const int end = min(P.T, first + P.Tc);
+    const int w = max(first - P.To, 0);
+    q_first = static_cast<long long>(first) * P.HW;
+    q_end = static_cast<long long>(end) * P.HW;
+    ka = P.k; va = P.v;
+    ka_off = bh * P.rows_per_bh + static_cast<long long>(w) * P.HW;
+    na = static_cast<long long>(end - w) * P.HW;
+  } else {
+    const long long seen = *P.seen;
+    const long long r_slices = seen < P.To ? seen : P.To;
+    q_first = 0;
+    q_end = static_cast<long long>(P.nq_slices) * P.HW;
+    ka = P.rk; va = P.rv;
+    ka_off = bh * P.ring_rows_per_bh;
+    na = r_slices * P.HW;
+    kb = P.k; vb = P.v;
+    kb_off = bh * P.rows_per_bh;
+    nb = q_end;
+  }
+  const long long row0 = q_first + static_cast<long long>(blockIdx.x) * kBQ;
+  if (row0 >= q_end) return;
+  const int nrows = static_cast<int>(min(static_cast<long long>(kBQ), q_end - row0));
+  const long long qrow_base = bh * P.rows_per_bh + row0;
+
+  for (int i = tid; i < kBQ * D; i += 128) {
+    const int rr = i / D, d = i % D;
+    Qs[i] = rr < nrows ? load_in(P.q, (qrow_base + rr) * D + d, P.in_bf16) : 0.f;
+  }
+
+  float o[D / 4];
+#pragma unroll
+  for (int c = 0; c < D / 4; ++c) o[c] = 0.f;
+  float m = -INFINITY, l = 0.f;
+
+  for (int range = 0; range < 2; ++range) {
+    const void* kp = range == 0 ? ka : kb;
+    const void* vp = range == 0 ? va : vb;
+    const long long off = range == 0 ? ka_off : kb_off;
+    const long long n = range == 0 ? na : nb;
+    for (long long kt = 0; kt < n; kt += kBK) {
+      __syncthreads();
+      for (int i = tid; i < kBK * D; i += 128) {
+        const int j = i / D, d = i % D;
+        const bool ok = kt + j < n;
+        const long long gi = (off + kt + j) * D + d;
+        Ks[j * (D + 1) + d] = ok ? load_in(kp, gi, P.in_bf16) : 0.f;
+        Vs[j * D + d] = ok ? load_in(vp, gi, P.in_bf16) : 0.f;
+      }
+      __syncthreads();
+      float s[kBK / 4];
+      float mt = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < kBK / 4; ++i) {
+        const int j = lane4 + 4 * i;
+        float acc = 0.f;
+#pragma unroll 8
+        for (int d = 0; d < D; ++d) acc = fmaf(Qs[r * D + d], Ks[j * (D + 1) + d], acc);
+        s[i] = (kt + j < n) ? acc * P.scale_log2 : -INFINITY;
+        mt = fmaxf(mt, s[i]);
+      }
+      mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
+      mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
+      const float m_new = fmaxf(m, mt);
+      const float alpha = exp2f(m - m_new);
+      float lsum = 0.f;
+#pragma unroll
+      for (int i = 0; i < kBK / 4; ++i) {
+        const float pv = exp2f(s[i] - m_new);
+        Ps[r * (kBK + 1) + lane4 + 4 * i] = pv;
+        lsum += pv;
+      }
+      l = l * alpha + lsum;
+      m = m_new;
+      __syncwarp();
+#pragma unroll
+      for (int c = 0; c < D / 4; ++c) {
+        const int col = lane4 + 4 * c;
+        float acc = o[c] * alpha;
+#pragma unroll 8
+        for (int j = 0; j < kBK; ++j) acc = fmaf(Ps[r * (kBK + 1) + j], Vs[j * D + col], acc);
+        o[c] = acc;
+      }
+    }
+  }
+  l += __shfl_xor_sync(0xffffffffu, l, 1);
+  l += __shfl_xor_sync(0xffffffffu, l, 2);
+
+  // Linear branch: phi_q(q) . S^L and phi_q(q) . z^L.
+  float aL[D / 4];
+  float nL = 0.f;
+#pragma unroll
+  for (int c = 0; c < D / 4; ++c) aL[c] = 0.f;
+  if (!P.full_softmax) {
+    __syncthreads();
+    const int Dp = P.Dp;
+    const float* SL = P.SL + (static_cast<long long>(bh) * P.nchunks + t) * Dp * D;
+    const float* zL = P.zL + (static_cast<long long>(bh) * P.nchunks + t) * Dp;
+    for (int f = lane4; f < Dp; f += 4) {
+      float psi = __ldg(P.bq + b_index(h, Dp, f));
+      for (int d = 0; d < D; ++d)
+        psi = fmaf(Qs[r * D + d], load_w(P.Wq, w_index(h, D, Dp, d, f), P.w_bf16), psi);
+      const float ph = psi * psi;
+      Fq[r * Dp + f] = ph;
+      nL = fmaf(ph, __ldg(zL + f), nL);
+    }
+    nL += __shfl_xor_sync(0xffffffffu, nL, 1);
+    nL += __shfl_xor_sync(0xffffffffu, nL, 2);
+    __syncwarp();
+    for (int f = 0; f < Dp; ++f) {
+      const float ph = Fq[r * Dp + f];
+#pragma unroll
+      for (int c = 0; c < D / 4; ++c)
+        aL[c] = fmaf(ph, __ldg(SL + sl_index(f, lane4 + 4 * c, D, Dp)), aL[c]);
+    }
+  }
+
+  if (r < nrows) {
+    const long long row = qrow_base + r;
+    const float den = l + nL;
+#pragma unroll
+    for (int c = 0; c < D / 4; ++c) {
+      const int col = lane4 + 4 * c;
+      store_out(P.y, row * D + col, __fdiv_rn(o[c] + aL[c], den), P.out_bf16);
+      if (P.dbg_aS) P.dbg_aS[row * D + col] = o[c];
+      if (P.dbg_aL) P.dbg_aL[row * D + col] = aL[c];
+    }
+    if (lane4 == 0) {
+      if (P.dbg_nS) P.dbg_nS[row] = l;
+      if (P.dbg_nL) P.dbg_nL[row] = nL;
+      if (P.dbg_c) P.dbg_c[row] = m * kLn2;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Per-slice state P_i = sum phi_k(k) v^T, z_i = sum phi_k(k).
+// Block: 256 threads = 64 features x 4 lanes; grid (nslots, BH, Dp/64).
+// ---------------------------------------------------------------------------
+constexpr int kTok = 16;
+constexpr int kFeat = 64;
+
+template <int D>
+__global__ void __launch_bounds__(256) partials_simt_kernel(PartialParams P) {
+  __shared__ float Kt[kTok][D + 1];
+  __shared__ float Vt[kTok][D];
+  __shared__ float Ft[kTok][kFeat + 1];
+  const int tid = threadIdx.x;
+  const int fl = tid >> 2;
+  const int lane4 = tid & 3;
+  const int slot = blockIdx.x;
+  const int bh = blockIdx.y;
+  const int f0 = blockIdx.z * kFeat;
+  const int h = bh % P.heads;
+  const int Dp = P.Dp;
+
+  const void *kp, *vp;
+  long long base;  // first row of the slice
+  if (P.seen == nullptr) {
+    kp = P.k; vp = P.v;
+    base = bh * P.rows_per_bh + static_cast<long long>(slot) * P.HW;
+  } else {
+    const long long seen = *P.seen;
+    const long long r = seen < P.To ? seen : P.To;
+    const long long after = seen + P.nq_slices;
+    const long long r2 = after < P.To ? after : P.To;
+    const long long leave = r + P.nq_slices - r2;
+    if (slot >= leave) return;
+    const long long g = seen - r + slot;
+    if (g < seen) {
+      kp = P.rk; vp = P.rv;
+      base = bh * P.ring_rows_per_bh + (g % P.To) * P.HW;
+    } else {
+      kp = P.k; vp = P.v;
+      base = bh * P.rows_per_bh + (g - seen) * P.HW;
+    }
+  }
+
+  float acc[D / 4];
+#pragma unroll
+  for (int c = 0; c < D / 4; ++c) acc[c] = 0.f;
+  float zacc = 0.f;
+
+  for (int j0 = 0; j0 < P.HW; j0 += kTok) {
+    __syncthreads();
+    for (int i = tid; i < kTok * D; i += 256) {
+      const int j = i / D, d = i % D;
+      const bool ok = j0 + j < P.HW;
+      const long long gi = (base + j0 + j) * D + d;
+      Kt[j][d] = ok ? load_in(kp, gi, P.in_bf16) : 0.f;
+      Vt[j][d] = ok ? load_in(vp, gi, P.in_bf16) : 0.f;
+    }
+    __syncthreads();
+    // phi_k for kTok tokens x kFeat features (4 values per thread).
+    for (int i = tid; i < kTok * kFeat; i += 256) {
+      const int j = i / kFeat, fq = i % kFeat;
+      const int f = f0 + fq;
+      float ph = 0.f;
+      if (f < Dp && j0 + j < P.HW) {
+        float psi = __ldg(P.bk + b_index(h, Dp, f));
+        for (int d = 0; d < D; ++d)
+          psi = fmaf(Kt[j][d], load_w(P.Wk, w_index(h, D, Dp, d, f), P.w_bf16), psi);
+        ph = psi * psi;
+      }
+      Ft[j][fq] = ph;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int j = 0; j < kTok; ++j) {
+      const float ph = Ft[j][fl];
+      zacc += ph;
+#pragma unroll
+      for (int c = 0; c < D / 4; ++c) acc[c] = fmaf(ph, Vt[j][lane4 + 4 * c], acc[c]);
+    }
+  }
+  const int f = f0 + fl;
+  if (f < Dp) {
+    float* Pout = P.P + (static_cast<long long>(bh) * P.nslots + slot) * Dp * D + static_cast<long long>(f) * D;
+#pragma unroll
+    for (int c = 0; c < D / 4; ++c) Pout[lane4 + 4 * c] = acc[c];
+    if (lane4 == 0) P.z[(static_cast<long long>(bh) * P.nslots + slot) * Dp + f] = zacc;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Chunk scan: one thread per state element, sequential over slices.
+// ---------------------------------------------------------------------------
+__global__ void scan_kernel(const float* __restrict__ P, const float* __restrict__ z,
+                            float* __restrict__ SL, float* __restrict__ zL, int T, int Tc,
+                            int To, int nchunks, int Dp, int D, int causal) {
+  const long long PD = static_cast<long long>(Dp) * D;
+  const long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int bh = blockIdx.y;
+  const float* src;
+  float* dst;
+  long long stride;
+  if (e < PD) {
+    src = P + bh * T * PD + e;
+    dst = SL + bh * nchunks * PD + sl_index(static_cast<int>(e / D), static_cast<int>(e % D), D, Dp);
+    stride = PD;
+  } else if (e < PD + Dp) {
+    src = z + static_cast<long long>(bh) * T * Dp + (e - PD);
+    dst = zL + static_cast<long long>(bh) * nchunks * Dp + (e - PD);
+    stride = Dp;
+  } else {
+    return;
+  }
+  float pre = 0.f;
+  int s = 0;
+  for (int t = 0; t < nchunks; ++t) {
+    const int w = max(t * Tc - To, 0);
+    for (; s < w; ++s) pre += src[s * stride];
+    dst[t * stride] = pre;
+  }
+  if (!causal) {
+    float suf = 0.f;
+    s = T;
+    for (int t = nchunks - 1; t >= 0; --t) {
+      const int end = min(T, (t + 1) * Tc);
+      while (s > end) {
+        --s;
+        suf += src[s * stride];
+      }
+      dst[t * stride] += suf;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Streaming helpers.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ long long leaving_slices(long long seen, int To, int n) {
+  const long long r = seen < To ? seen : To;
+  const long long after = seen + n;
+  const long long r2 = after < To ? after : To;
+  return r + n - r2;
+}
+
+__global__ void state_add_kernel(const float* __restrict__ P, const float* __restrict__ zp,
+                                 float* __restrict__ s_state, float* __restrict__ z_state,
+                                 const long long* __restrict__ seen, int Dp, int D, int To,
+                                 int nq, int nslots) {
+  const long long PD = static_cast<long long>(Dp) * D;
+  const long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int bh = blockIdx.y;
+  const long long leave = leaving_slices(*seen, To, nq);
+  if (e < PD) {
+    const long long se = bh * PD + sl_index(static_cast<int>(e / D), static_cast<int>(e % D), D, Dp);
+    float acc = s_state[se];
+    for (long long i = 0; i < leave; ++i) acc += P[(bh * nslots + i) * PD + e];
+    s_state[se] = acc;
+  } else if (e < PD + Dp) {
+    const long long f = e - PD;
+    float acc = z_state[static_cast<long long>(bh) * Dp + f];
+    for (long long i = 0; i < leave; ++i) acc += zp[(bh * nslots + i) * Dp + f];
+    z_state[static_cast<long long>(bh) * Dp + f] = acc;
+  }
+}
+
+// Copy chunk slices that stay in the window into their ring slots.
+// grid (nq_slices, BH); 16-byte vectors.
+__global__ void ring_update_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
+                                   uint4* __restrict__ rk, uint4* __restrict__ rv,
+                                   const long long* __restrict__ seen, long long slice_vecs,
+                                   int To, int nq) {
+  const long long sn = *seen;
+  const long long after = sn + nq;
+  const long long keep = after < To ? after : To;
+  const long long g = sn + blockIdx.x;          // global slice of this chunk slice
+  if (g < after - keep) return;                 // leaves the window right away
+  const int bh = blockIdx.y;
+  const uint4* ks = k + (static_cast<long long>(bh) * nq + blockIdx.x) * slice_vecs;
+  const uint4* vs = v + (static_cast<long long>(bh) * nq + blockIdx.x) * slice_vecs;
+  uint4* kd = rk + (static_cast<long long>(bh) * To + (g % To)) * slice_vecs;
+  uint4* vd = rv + (static_cast<long long>(bh) * To + (g % To)) * slice_vecs;
+  for (long long i = threadIdx.x; i < slice_vecs; i += blockDim.x) {
+    kd[i] = ks[i];
+    vd[i] = vs[i];
+  }
+}
+
+__global__ void advance_kernel(long long* seen, int nq) { *seen += nq; }
+
+// bf16 copy of the phi_q weights in the tensor-core image layout.
+__global__ void wq_image_kernel(const float* __restrict__ Wq, __nv_bfloat16* __restrict__ out,
+                                int heads, int D, int Dp) {
+  const long long per_head = static_cast<long long>(Dp) * D;
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= per_head * heads) return;
+  const int h = static_cast<int>(i / per_head);
+  const int rem = static_cast<int>(i % per_head);
+  const int d = rem / Dp, f = rem % Dp;
+  out[h * per_head + wimg_index(f, d, D, Dp)] = __float2bfloat16_rn(Wq[w_index(h, D, Dp, d, f)]);
+}
+
+template <int D>
+cudaError_t launch_attn_simt_d(const AttnParams& p, cudaStream_t s) {
+  const int fl_loop = kBQ * D + kBK * (D + 1) + kBK * D + kBQ * (kBK + 1);
+  const int fl_tail = kBQ * D + kBQ * p.Dp;
+  const size_t bytes = sizeof(float) * static_cast<size_t>(fl_loop > fl_tail ? fl_loop : fl_tail);
+  cudaError_t e = cudaFuncSetAttribute(attn_simt_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(bytes));
+  if (e != cudaSuccess) return e;
+  int qrows_max;  // rows of the largest chunk
+  if (p.seen) qrows_max = p.nq_slices * p.HW;
+  else qrows_max = (p.Tc < p.T ? p.Tc : p.T) * p.HW;
+  dim3 grid((qrows_max + kBQ - 1) / kBQ, p.nchunks, p.BH);
+  attn_simt_kernel<D><<<grid, 128, bytes, s>>>(p);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_partials_simt_d(const PartialParams& p, cudaStream_t s) {
+  dim3 grid(p.nslots, p.BH, (p.Dp + kFeat - 1) / kFeat);
+  partials_simt_kernel<D><<<grid, 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn_simt(const AttnParams& p, cudaStream_t s) {
+  switch (p.D) {
+    case 32: return launch_attn_simt_d<32>(p, s);
+    case 64: return launch_attn_simt_d<64>(p, s);
+    case 128: return launch_attn_simt_d<128>(p, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_partials_simt(const PartialParams& p, cudaStream_t s) {
+  switch (p.D) {
+    case 32: return launch_partials_simt_d<32>(p, s);
+    case 64: return launch_partials_simt_d<64>(p, s);
+    case 128: return launch_partials_simt_d<128>(p, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_scan(const float* P, const float* z, float* SL, float* zL, int BH, int T,
+                        int Tc, int To, int nchunks, int Dp, int D, int causal,
+                        cudaStream_t s) {
+  const long long n = static_cast<long long>(Dp) * D + Dp;
+  dim3 grid(static_cast<unsigned>((n + 255) / 256), BH);
+  scan_kernel<<<grid, 256, 0, s>>>(P, z, SL, zL, T, Tc, To, nchunks, Dp, D, causal);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_state_add(const float* P, const float* zp, float* s_state, float* z_state,
+                             const long long* seen, int BH, int Dp, int D, int To,
+                             int nq_slices, int nslots, cudaStream_t s) {
+  const long long n = static_cast<long long>(Dp) * D + Dp;
+  dim3 grid(static_cast<unsigned>((n + 255) / 256), BH);
+  state_add_kernel<<<grid, 256, 0, s>>>(P, zp, s_state, z_state, seen, Dp, D, To, nq_slices,
+                                        nslots);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ring_update(const void* k, const void* v, void* rk, void* rv,
+                               const long long* seen, int BH, int HW, int D, int To,
+                               int nq_slices, int elem_bytes, cudaStream_t s) {
+  if (To == 0) return cudaSuccess;
+  const long long slice_vecs = static_cast<long long>(HW) * D * elem_bytes / 16;
+  dim3 grid(nq_slices, BH);
+  ring_update_kernel<<<grid, 256, 0, s>>>(
+      static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint4*>(rk),
+      static_cast<uint4*>(rv), seen, slice_vecs, To, nq_slices);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_advance(long long* seen, int nq_slices, cudaStream_t s) {
+  advance_kernel<<<1, 1, 0, s>>>(seen, nq_slices);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_wq_image(const float* Wq, void* out, int heads, int D, int Dp,
+                            cudaStream_t s) {
+  const long long n = static_cast<long long>(heads) * D * Dp;
+  wq_image_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(
+      Wq, static_cast<__nv_bfloat16*>(out), heads, D, Dp);
+  return cudaGetLastError();
+}
+
+}  // namespace rehyat

@@ -127,11 +127,13 @@ def _pairwise_head(q, k, v, Wq, bq, Wk, bk, HW, Tc, To, causal, scale):
 # --------------------------------------------------------------------------
 # Form (ii): per chunk, window softmax + linear state over the linear set.
 # --------------------------------------------------------------------------
-def _factored_head(q, k, v, Wq, bq, Wk, bk, T, HW, Tc, To, causal, scale):
+def _factored_head(q, k, v, Wq, bq, Wk, bk, T, HW, Tc, To, causal, scale, chunks=None):
     N, D = q.shape
     y = np.zeros((N, D))
     parts = _empty_partials(N, D)
-    for first, end, start in chunk_table(T, Tc, To):
+    for t, (first, end, start) in enumerate(chunk_table(T, Tc, To)):
+        if chunks is not None and t not in chunks:
+            continue
         rows = slice(first * HW, end * HW)
         Qc = q[rows]
         Kw, Vw = k[start * HW:end * HW], v[start * HW:end * HW]
@@ -252,11 +254,12 @@ def hybrid_pairwise(q, k, v, Wq, bq, Wk, bk, *, T, HW, Tc, To, causal, scale=Non
 
 
 def hybrid_factored(q, k, v, Wq, bq, Wk, bk, *, T, HW, Tc, To, causal, scale=None,
-                    heads_subset=None):
-    """Form (ii).  ``heads_subset`` restricts work to some flattened (b, h)
-    indices (used to time a bounded sample).  Returns (y, partials)."""
+                    heads_subset=None, chunks_subset=None):
+    """Form (ii).  ``heads_subset`` (flattened (b, h) indices) and
+    ``chunks_subset`` (chunk indices) restrict the work to a sample; rows
+    outside it are left zero.  Returns (y, partials)."""
     sc = _scale_of(q.shape[-1], scale)
-    fn = lambda *a: _factored_head(*a, T, HW, Tc, To, causal, sc)
+    fn = lambda *a: _factored_head(*a, T, HW, Tc, To, causal, sc, chunks_subset)
     return _over_heads(fn, q, k, v, Wq, bq, Wk, bk, heads_subset)
 
 
@@ -277,14 +280,15 @@ def full_softmax(q, k, v, scale=None):
     return np.einsum("bhnm,bhmd->bhnd", E, v) / E.sum(axis=-1)[..., None]
 
 
-def run_problem(p, form="factored", heads_subset=None):
+def run_problem(p, form="factored", heads_subset=None, chunks_subset=None):
     """Run one ``rehyat_inputs.Problem`` through the chosen form."""
     kw = dict(T=p.T, HW=p.HW, Tc=p.Tc, To=p.To)
     args = (p.q, p.k, p.v, p.Wq, p.bq, p.Wk, p.bk)
     if form == "pairwise":
         return hybrid_pairwise(*args, causal=p.causal, **kw)
     if form == "factored":
-        return hybrid_factored(*args, causal=p.causal, heads_subset=heads_subset, **kw)
+        return hybrid_factored(*args, causal=p.causal, heads_subset=heads_subset,
+                               chunks_subset=chunks_subset, **kw)
     if form == "rnn":
         if not p.causal:
             raise ValueError("the RNN form is causal")

@@ -1,0 +1,122 @@
+"""Host-side checks of the C ABI (no GPU needed).
+
+The library loads, exports every function include/rehyat.h declares, sizes
+its workspace/state correctly, and rejects bad arguments with a status before
+launching anything.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import linear_attention_video_chunked_b200 as rh
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                      "rehyat.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"REHYAT_API\s+[\w\s\*]*?\b(rehyat_\w+)\s*\(", text)))
+
+
+def _params(**kw):
+    base = dict(batch=2, heads=3, T=7, Hs=5, Ws=6, D=128, Dp=128, Tc=3, To=1, causal=0,
+                in_dtype=rh.BF16, out_dtype=rh.F32)
+    base.update(kw)
+    return rh.make_params(**base)
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    L = rh.lib()
+    declared = _declared_functions()
+    assert len(declared) >= 9
+    for name in declared:
+        assert hasattr(L, name), name
+        assert ctypes.cast(getattr(L, name), ctypes.c_void_p).value
+    assert set(declared) == set(rh.EXPORTED_SYMBOLS)
+    assert rh.rehyat_version() >= 100
+
+
+def test_status_strings():
+    for code in range(6):
+        assert rh.rehyat_status_string(code)
+    assert rh.rehyat_status_string(0) == "ok"
+
+
+def test_workspace_bytes_layout():
+    p = _params()
+    BH, T, Dp, D, nch = 6, 7, 128, 128, 3
+    need = BH * T * Dp * D * 4 + BH * T * Dp * 4 + BH * nch * Dp * D * 4 + BH * nch * Dp * 4
+    got = rh.rehyat_workspace_bytes(p)
+    assert need <= got <= need + 4 * 256
+    assert got % 256 == 0
+
+
+def test_state_bytes_constant_and_ring_sized_by_overlap():
+    p1 = _params(causal=1, To=1)
+    p2 = _params(causal=1, To=2)
+    b1, b2 = rh.rehyat_state_bytes(p1), rh.rehyat_state_bytes(p2)
+    ring_slice = 6 * 30 * 128 * 2 * 2  # BH * HW * D * bf16 * (k and v)
+    assert abs((b2 - b1) - ring_slice) <= 512
+    # independent of the number of slices in the video
+    assert rh.rehyat_state_bytes(_params(causal=1, T=100)) == b1
+
+
+@pytest.mark.parametrize("bad", [
+    dict(batch=0), dict(heads=-1), dict(T=0), dict(Hs=0), dict(Tc=0), dict(To=-1),
+    dict(causal=2), dict(in_dtype=7), dict(out_dtype=-1), dict(scale=-1.0),
+    dict(scale=float("nan")),
+])
+def test_invalid_params_rejected(bad):
+    p = _params(**bad)
+    assert rh.rehyat_workspace_bytes(p) == 0
+    st = rh.rehyat_hybrid_attn_fwd(p, 16, 16, 16, rh.RehyatPhi(16, 16, 16, 16), 16, 16, 1 << 40,
+                                   None, None)
+    assert st == 1
+
+
+@pytest.mark.parametrize("bad", [dict(D=96), dict(D=256), dict(Dp=48), dict(Dp=512)])
+def test_unsupported_shapes_rejected(bad):
+    p = _params(**bad)
+    assert rh.rehyat_workspace_bytes(p) == 0
+    st = rh.rehyat_hybrid_attn_fwd(p, 16, 16, 16, rh.RehyatPhi(16, 16, 16, 16), 16, 16, 1 << 40,
+                                   None, None)
+    assert st == 2
+
+
+def test_pointer_checks_before_launch():
+    p = _params()
+    phi = rh.RehyatPhi(4096, 4096, 4096, 4096)
+    ws = rh.rehyat_workspace_bytes(p)
+    f = rh.rehyat_hybrid_attn_fwd
+    assert f(p, 0, 4096, 4096, phi, 4096, 4096, ws, None, None) == 1       # null q
+    assert f(p, 4096, 4096, 4096, rh.RehyatPhi(0, 4096, 4096, 4096), 4096, 4096, ws, None,
+             None) == 1                                                    # null phi
+    assert f(p, 4104, 4096, 4096, phi, 4096, 4096, ws, None, None) == 3    # misaligned q
+    assert f(p, 4096, 4096, 4096, phi, 4096, 4096, ws - 1, None, None) == 4  # short ws
+    dbg = rh.RehyatDebug(4098, 0, 0, 0, 0)
+    assert f(p, 4096, 4096, 4096, phi, 4096, 4096, ws, dbg, None) == 3    # misaligned dbg
+
+
+def test_chunk_step_argument_checks():
+    p = _params(causal=1)
+    phi = rh.RehyatPhi(4096, 4096, 4096, 4096)
+    ws = rh.rehyat_step_workspace_bytes(p)
+    step = rh.rehyat_chunk_step
+    assert step(_params(causal=0), 4096, 4096, 4096, 1, phi, 4096, 4096, 4096, ws, None,
+                None) == 1                                                 # not causal
+    assert step(p, 4096, 4096, 4096, 0, phi, 4096, 4096, 4096, ws, None, None) == 1
+    assert step(p, 4096, 4096, 4096, 4, phi, 4096, 4096, 4096, ws, None, None) == 1  # > Tc
+    assert step(p, 4096, 4096, 4096, 2, phi, 0, 4096, 4096, ws, None, None) == 1     # state
+    assert step(p, 4096, 4096, 4096, 2, phi, 4100, 4096, 4096, ws, None, None) == 3
+    assert step(p, 4096, 4096, 4096, 2, phi, 4096, 4096, 4096, ws - 256, None, None) == 4
+    assert rh.rehyat_state_init(p, 0, None) == 1
+    assert rh.rehyat_state_init(p, 4104, None) == 3
+
+
+def test_softmax_entry_checks():
+    p = _params()
+    assert rh.rehyat_softmax_attn_fwd(p, 0, 16, 16, 16, None) == 1
+    assert rh.rehyat_softmax_attn_fwd(p, 24, 16, 16, 16, None) == 3

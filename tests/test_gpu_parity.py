@@ -1,0 +1,250 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on
+the same seeded inputs.
+
+Bars (y): fp32 inputs max abs <= 1e-5; bf16 inputs max abs <= 2e-2 and mean
+abs <= 2e-3.  Branch partials are compared too, because at these feature-map
+scales the linear branch carries most of the weight and would hide softmax
+errors in y.
+"""
+import numpy as np
+import pytest
+import torch
+
+import linear_attention_video_chunked_b200 as rh
+from oracle import rehyat_oracle as orc
+from rehyat_inputs import config_problem, make_problem
+from tests.gpu_util import (assert_close_partials, assert_close_y, device_tensors, err_stats,
+                            run_fwd)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    rh.lib()
+
+
+# ------------------------------------------------------------ tiny fp32 case
+@pytest.mark.parametrize("causal", [False, True])
+def test_tiny_fp32_both_forms(causal):
+    p = config_problem("tiny_f32", causal=causal)
+    ref_y, ref_p = orc.run_problem(p)
+    y, parts = run_fwd(p, debug=True)
+    assert_close_y(y, ref_y, "f32")
+    assert_close_partials(parts, ref_p, "f32")
+
+
+# ----------------------------------------- small ragged shapes, both dtypes
+SMALL = [
+    # B, h, T, Hs, Ws, D, Dp, Tc, To
+    (1, 2, 5, 7, 9, 128, 128, 2, 1),     # HW=63: one ragged tile per slice
+    (1, 2, 7, 10, 13, 128, 128, 3, 2),   # HW=130: tile straddles slices; T % Tc != 0
+    (2, 1, 4, 16, 16, 128, 64, 1, 2),    # To > Tc, spatial-only chunks
+    (1, 3, 6, 8, 12, 64, 256, 2, 0),     # no overlap, wide phi
+    (1, 2, 3, 5, 5, 32, 32, 4, 1),       # one chunk covers everything
+    (1, 1, 9, 11, 12, 128, 128, 3, 1),   # HW=132, several chunks
+]
+
+
+@pytest.mark.parametrize("shape", SMALL, ids=lambda s: "x".join(map(str, s)))
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("force_simt", [False, True], ids=["default", "simt"])
+def test_small_shapes(shape, causal, dtype, force_simt):
+    B, h, T, Hs, Ws, D, Dp, Tc, To = shape
+    p = make_problem(batch=B, heads=h, T=T, Hs=Hs, Ws=Ws, D=D, Dp=Dp, Tc=Tc, To=To,
+                     causal=causal, dtype=dtype, dist="scaled", seed=100 + sum(shape))
+    ref_y, ref_p = orc.run_problem(p)
+    y, parts = run_fwd(p, debug=True, force_simt=force_simt)
+    assert_close_y(y, ref_y, dtype)
+    assert_close_partials(parts, ref_p, dtype)
+
+
+def test_sharp_softmax_lowrank_inputs():
+    """Low-rank-plus-noise q, k (logit std ~4) with a weak feature map, so the
+    softmax branch dominates y."""
+    p = make_problem(batch=1, heads=2, T=6, Hs=12, Ws=20, D=128, Dp=128, Tc=2, To=1,
+                     causal=False, dtype="bf16", dist="lowrank", seed=77, phi_std=0.005)
+    ref_y, ref_p = orc.run_problem(p)
+    y, parts = run_fwd(p, debug=True)
+    assert_close_y(y, ref_y, "bf16")
+    assert_close_partials(parts, ref_p, "bf16")
+    assert np.median(ref_p["nS"] / np.maximum(ref_p["nL"], 1e-30)) > 1.0
+
+
+# ------------------------------------------------------- full-size workloads
+def test_wan_320x480_causal_full():
+    """Latent 21x20x30, 12 heads, D=128, T_c=3, T_o=1, causal, every output."""
+    p = config_problem("wan_320x480_causal")
+    ref_y, ref_p = orc.run_problem(p)
+    y, parts = run_fwd(p, debug=True)
+    assert_close_y(y, ref_y, "bf16")
+    assert_close_partials(parts, ref_p, "bf16")
+
+
+def test_wan_480x832_bidir_sampled_heads():
+    """Latent 21x30x52, batch 2, 12 heads, bidirectional: every output of
+    three sampled (batch, head) pairs against the oracle."""
+    p = config_problem("wan_480x832_bidir")
+    subset = [0, 13, 23]
+    ref_y, ref_p = orc.run_problem(p, heads_subset=subset)
+    y, parts = run_fwd(p, debug=True)
+    B, H = p.batch, p.heads
+    for idx in subset:
+        b, hh = divmod(idx, H)
+        assert_close_y(y[b, hh], ref_y[b, hh], "bf16", f"y[{b},{hh}]")
+        assert_close_partials({k: v[b, hh] for k, v in parts.items()},
+                              {k: v[b, hh] for k, v in ref_p.items()}, "bf16")
+    assert np.all(np.isfinite(y))
+
+
+@pytest.mark.parametrize("name,std,subset", [("wan_320x480_causal", 0.003, None),
+                                             ("wan_480x832_bidir", 0.0045, [1, 5, 18])])
+def test_balanced_branches_full_size(name, std, subset):
+    """Feature-map scale chosen so the median n^L/n^S is near 1 on some heads
+    (and far below on others): both branches are visible in y."""
+    p = config_problem(name, phi_std=std)
+    ref_y, ref_p = orc.run_problem(p, heads_subset=subset)
+    y, parts = run_fwd(p, debug=True)
+    for idx in (subset if subset is not None else range(p.batch * p.heads)):
+        b, hh = divmod(idx, p.heads)
+        assert_close_y(y[b, hh], ref_y[b, hh], "bf16", f"y[{b},{hh}]")
+        assert_close_partials({k: v[b, hh] for k, v in parts.items()},
+                              {k: v[b, hh] for k, v in ref_p.items()}, "bf16")
+
+
+@pytest.mark.parametrize("Tc,To,Dp,causal", [(1, 0, 128, False), (2, 2, 64, True),
+                                             (5, 1, 256, False), (7, 2, 128, True)])
+def test_sweep_points_sampled(Tc, To, Dp, causal):
+    """Points of the T_c / T_o / D' sweep on the 21x30x52 latent with
+    low-rank-plus-noise q, k; one sampled head each."""
+    p = make_problem(batch=1, heads=12, T=21, Hs=30, Ws=52, D=128, Dp=Dp, Tc=Tc, To=To,
+                     causal=causal, dtype="bf16", dist="lowrank", seed=4 + Tc * 10 + To)
+    subset = [5]
+    ref_y, _ = orc.run_problem(p, heads_subset=subset)
+    y = run_fwd(p)
+    assert_close_y(y[0, 5], ref_y[0, 5], "bf16")
+
+
+# ------------------------------------------------------------- comparator
+def test_full_softmax_comparator():
+    p = make_problem(batch=1, heads=2, T=3, Hs=10, Ws=30, D=128, Dp=32, Tc=1, To=0,
+                     causal=False, dtype="bf16", seed=9)
+    dev = device_tensors(p)
+    y = rh.softmax_attn(dev["q"], dev["k"], dev["v"])
+    torch.cuda.synchronize()
+    ref = orc.full_softmax(p.q, p.k, p.v)
+    assert_close_y(y.double().cpu().numpy(), ref, "bf16")
+
+
+# ------------------------------------------------------------- streaming
+def _stream_outputs(p, force_simt=False, dev=None):
+    dev = device_tensors(p) if dev is None else dev
+    st = rh.StreamingState(batch=p.batch, heads=p.heads, Hs=p.Hs, Ws=p.Ws, D=p.D, Dp=p.Dp,
+                           Tc=p.Tc, To=p.To, Wq=dev["Wq"], bq=dev["bq"], Wk=dev["Wk"],
+                           bk=dev["bk"], in_dtype=dev["q"].dtype, force_simt=force_simt)
+    outs = []
+    HW = p.HW
+    for first in range(0, p.T, p.Tc):
+        rows = slice(first * HW, min(p.T, first + p.Tc) * HW)
+        qc, kc, vc = (dev[x][:, :, rows].contiguous() for x in ("q", "k", "v"))
+        outs.append(st.step(qc, kc, vc))
+    torch.cuda.synchronize()
+    return torch.cat(outs, dim=2), st
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("Tc,To", [(3, 1), (2, 3), (1, 0), (4, 2)])
+def test_streaming_matches_rnn_oracle_and_full_causal(dtype, Tc, To):
+    p = make_problem(batch=1, heads=2, T=10, Hs=6, Ws=11, D=128, Dp=128, Tc=Tc, To=To,
+                     causal=True, dtype=dtype, seed=31 + Tc + 7 * To)
+    y_stream, _ = _stream_outputs(p)
+    ref_y, _ = orc.run_problem(p, form="rnn")
+    assert_close_y(y_stream.double().cpu().numpy(), ref_y, dtype)
+    y_full = run_fwd(p)
+    mx, _ = err_stats(y_stream.double().cpu().numpy(), y_full)
+    assert mx <= (2e-2 if dtype == "bf16" else 1e-5)
+
+
+def test_stream_81_slices_constant_memory():
+    """81 slices of 30x52, 27 steps: outputs of sampled heads match the oracle
+    and free device memory does not move across steps."""
+    p = config_problem("stream_81x30x52")
+    dev = device_tensors(p)
+    st = rh.StreamingState(batch=p.batch, heads=p.heads, Hs=p.Hs, Ws=p.Ws, D=p.D, Dp=p.Dp,
+                           Tc=p.Tc, To=p.To, Wq=dev["Wq"], bq=dev["bq"], Wk=dev["Wk"],
+                           bk=dev["bk"], in_dtype=dev["q"].dtype)
+    HW, rows_per = p.HW, p.Tc * p.HW
+    chunks = [tuple(dev[x][:, :, s * rows_per:(s + 1) * rows_per].contiguous()
+                    for x in ("q", "k", "v")) for s in range(27)]
+    out = torch.empty(1, p.heads, rows_per, p.D, device="cuda")
+    ys = []
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    frees = []
+    for s in range(27):
+        st.step(*chunks[s], out=out)
+        ys.append(out[0, 3].double().cpu().numpy())
+        frees.append(torch.cuda.mem_get_info()[0])
+    assert all(f == free0 for f in frees)
+    subset = [3]
+    ref_y, _ = orc.run_problem(p, heads_subset=subset)
+    assert_close_y(np.concatenate(ys), ref_y[0, 3], "bf16")
+
+
+def test_streaming_checkpoint_resume_bit_exact():
+    p = make_problem(batch=1, heads=2, T=9, Hs=6, Ws=11, D=128, Dp=128, Tc=2, To=1,
+                     causal=True, dtype="bf16", seed=41)
+    dev = device_tensors(p)
+    mk = lambda: rh.StreamingState(batch=1, heads=2, Hs=6, Ws=11, D=128, Dp=128, Tc=2, To=1,
+                                   Wq=dev["Wq"], bq=dev["bq"], Wk=dev["Wk"], bk=dev["bk"],
+                                   in_dtype=torch.bfloat16)
+    HW = p.HW
+    chunk = lambda i: tuple(dev[x][:, :, i * 2 * HW:min(9, i * 2 + 2) * HW].contiguous()
+                            for x in ("q", "k", "v"))
+    a = mk()
+    ya = [a.step(*chunk(i)).clone() for i in range(5)]
+    b = mk()
+    for i in range(2):
+        b.step(*chunk(i))
+    saved = b.snapshot().cpu()
+    b.reset()
+    b.step(*chunk(0))  # disturb
+    b.restore(saved.cuda())
+    yb = [b.step(*chunk(i)).clone() for i in range(2, 5)]
+    torch.cuda.synchronize()
+    for i in range(3):
+        assert torch.equal(ya[2 + i], yb[i])
+
+
+# ------------------------------------------------------------- properties
+def test_repeatable_bitwise():
+    p = config_problem("wan_320x480_causal")
+    dev = device_tensors(p)
+    y1 = run_fwd(p, dev=dev)
+    y2 = run_fwd(p, dev=dev)
+    assert np.array_equal(y1, y2)
+
+
+def test_nan_input_propagates_without_fault():
+    p = make_problem(batch=1, heads=1, T=4, Hs=4, Ws=8, D=64, Dp=64, Tc=2, To=1,
+                     causal=True, dtype="bf16", seed=3)
+    dev = device_tensors(p)
+    dev["v"][0, 0, 5, 0] = float("nan")
+    y = run_fwd(p, dev=dev)
+    # slice 0 (rows 0..31) reaches every query, through the softmax window
+    # (chunk 0) or the linear state (chunk 1); only value column 0 is NaN.
+    assert np.isnan(y[0, 0, :, 0]).all()
+    assert np.isfinite(y[0, 0, :, 1:]).all()
+
+
+def test_bf16_output():
+    p = make_problem(batch=1, heads=2, T=5, Hs=7, Ws=9, D=128, Dp=128, Tc=2, To=1,
+                     causal=False, dtype="bf16", seed=8)
+    ref_y, _ = orc.run_problem(p)
+    y = run_fwd(p, out_dtype=torch.bfloat16)
+    mx, mean = err_stats(y, ref_y)
+    # bf16 output adds up to half an ulp of |y| on top of the fp32 result
+    assert mean <= 2e-3 and mx <= 2e-2 + np.abs(ref_y).max() * 2.0 ** -8
