@@ -172,6 +172,19 @@ REHYAT_API rehyat_status rehyat_chunk_step(const rehyat_params* p, const void* q
                                 const rehyat_debug* dbg, void* stream);
 
 /* ---------------------------------------------------------------------- */
+/* Diagnostic: every wait inside the tensor-core kernels is bounded (~2 s);
+ * a wait that runs out sets a bit in a device-side error word and the
+ * kernel returns early instead of hanging.  This reads that word for the
+ * current device into *flags (0 = no timeout since the last reset) and
+ * clears it when reset != 0.  Unlike the other entry points it synchronises
+ * the device (a blocking copy). */
+REHYAT_API rehyat_status rehyat_device_error_flags(unsigned* flags, int reset);
+
+/* Which attention kernel these params select: 1 = the tensor-core kernel
+ * (bf16 inputs, D = 128, Dp in {64, 128, 256}, no REHYAT_FLAG_FORCE_SIMT),
+ * 0 = the fp32 CUDA-core kernel, -1 = invalid params.  Host-only. */
+REHYAT_API int rehyat_attn_path(const rehyat_params* p);
+
 REHYAT_API const char* rehyat_status_string(rehyat_status s);
 
 /* Library ABI version (major*10000 + minor*100 + patch). */

@@ -27,8 +27,8 @@ __all__ = [
     "EXPORTED_SYMBOLS", "F32", "BF16", "FLAG_FORCE_SIMT",
     "rehyat_workspace_bytes", "rehyat_hybrid_attn_fwd", "rehyat_fwd_state", "rehyat_fwd_attn",
     "rehyat_softmax_attn_fwd", "rehyat_state_bytes", "rehyat_state_init", "rehyat_step_workspace_bytes",
-    "rehyat_chunk_step", "rehyat_status_string", "rehyat_version",
-    "make_params", "hybrid_attn", "softmax_attn", "StreamingState",
+    "rehyat_chunk_step", "rehyat_device_error_flags", "rehyat_attn_path",
+    "rehyat_status_string", "rehyat_version", "make_params", "hybrid_attn", "softmax_attn", "StreamingState",
 ]
 
 F32, BF16 = 0, 1
@@ -40,8 +40,8 @@ STATUS = {0: "REHYAT_OK", 1: "REHYAT_ERR_INVALID_ARG", 2: "REHYAT_ERR_UNSUPPORTE
 EXPORTED_SYMBOLS = (
     "rehyat_workspace_bytes", "rehyat_hybrid_attn_fwd", "rehyat_fwd_state",
     "rehyat_fwd_attn", "rehyat_softmax_attn_fwd", "rehyat_state_bytes", "rehyat_state_init",
-    "rehyat_step_workspace_bytes", "rehyat_chunk_step", "rehyat_status_string",
-    "rehyat_version",
+    "rehyat_step_workspace_bytes", "rehyat_chunk_step", "rehyat_device_error_flags",
+    "rehyat_attn_path", "rehyat_status_string", "rehyat_version",
 )
 
 
@@ -109,6 +109,10 @@ def lib() -> ctypes.CDLL:
         L.rehyat_chunk_step.argtypes = [P(RehyatParams), vp, vp, vp, i, P(RehyatPhi), vp, vp, vp,
                                         sz, P(RehyatDebug), vp]
         L.rehyat_chunk_step.restype = i
+        L.rehyat_device_error_flags.argtypes = [P(ctypes.c_uint), i]
+        L.rehyat_device_error_flags.restype = i
+        L.rehyat_attn_path.argtypes = [P(RehyatParams)]
+        L.rehyat_attn_path.restype = i
         L.rehyat_status_string.argtypes = [i]
         L.rehyat_status_string.restype = ctypes.c_char_p
         L.rehyat_version.argtypes = []
@@ -159,6 +163,19 @@ def rehyat_chunk_step(p, q, k, v, nslices, phi, state, y, workspace, ws_bytes, d
     return lib().rehyat_chunk_step(ctypes.byref(p), q, k, v, nslices, ctypes.byref(phi), state,
                                    y, workspace, ws_bytes,
                                    None if dbg is None else ctypes.byref(dbg), stream)
+
+
+def rehyat_device_error_flags(reset: bool = False) -> int:
+    """Timeout bits of the tensor-core kernels' bounded waits (synchronises)."""
+    out = ctypes.c_uint(0)
+    _check(lib().rehyat_device_error_flags(ctypes.byref(out), int(reset)),
+           "rehyat_device_error_flags")
+    return out.value
+
+
+def rehyat_attn_path(p: RehyatParams) -> int:
+    """1 = tensor-core attention kernel, 0 = CUDA-core kernel, -1 = invalid."""
+    return lib().rehyat_attn_path(ctypes.byref(p))
 
 
 def rehyat_status_string(status: int) -> str:

@@ -40,10 +40,10 @@ rehyat_status check_params(const rehyat_params* p) {
 int nchunks_of(const rehyat_params* p) { return (p->T + p->Tc - 1) / p->Tc; }
 
 struct FwdWorkspace {
-  size_t P_off, z_off, SL_off, zL_off, wimg_off, total;
+  size_t P_off, z_off, SL_off, zL_off, wimg_off, wkimg_off, total;
 };
 
-// phi_q weight image (bf16, all heads) used by the tensor-core kernel.
+// phi_q or phi_k weight image (bf16, all heads) for the tensor-core kernels.
 size_t wimg_bytes(const rehyat_params* p) {
   return static_cast<size_t>(p->heads) * p->Dp * p->D * 2;
 }
@@ -57,7 +57,8 @@ FwdWorkspace fwd_layout(const rehyat_params* p) {
   w.SL_off = align_up(w.z_off + BH * p->T * p->Dp * sizeof(float));
   w.zL_off = align_up(w.SL_off + BH * nchunks_of(p) * PD * sizeof(float));
   w.wimg_off = align_up(w.zL_off + BH * nchunks_of(p) * p->Dp * sizeof(float));
-  w.total = align_up(w.wimg_off + wimg_bytes(p));
+  w.wkimg_off = align_up(w.wimg_off + wimg_bytes(p));
+  w.total = align_up(w.wkimg_off + wimg_bytes(p));
   return w;
 }
 
@@ -65,6 +66,19 @@ FwdWorkspace fwd_layout(const rehyat_params* p) {
 bool tc_path(const rehyat_params* p) {
   return !(p->flags & REHYAT_FLAG_FORCE_SIMT) &&
          tc_attn_eligible(p->in_dtype == REHYAT_BF16, p->D, p->Dp);
+}
+
+// Whether the tensor-core per-slice state kernel is used.
+bool tc_state_path(const rehyat_params* p) {
+  return !(p->flags & REHYAT_FLAG_FORCE_SIMT) &&
+         tc_state_eligible(p->in_dtype == REHYAT_BF16, p->D, p->Dp);
+}
+
+// Per-slice states on the path these params select.
+cudaError_t run_partials(const rehyat_params* p, const PartialParams& pp, const void* wk_img,
+                         cudaStream_t s) {
+  if (tc_state_path(p)) return launch_state_tc(pp, wk_img, s);
+  return launch_partials_simt(pp, s);
 }
 
 struct StateLayout {
@@ -85,7 +99,7 @@ StateLayout state_layout(const rehyat_params* p) {
 }
 
 struct StepWorkspace {
-  size_t P_off, z_off, wimg_off, total;
+  size_t P_off, z_off, wimg_off, wkimg_off, total;
   int nslots;
 };
 
@@ -96,7 +110,8 @@ StepWorkspace step_layout(const rehyat_params* p) {
   w.P_off = 0;
   w.z_off = align_up(BH * w.nslots * static_cast<size_t>(p->Dp) * p->D * sizeof(float));
   w.wimg_off = align_up(w.z_off + BH * w.nslots * p->Dp * sizeof(float));
-  w.total = align_up(w.wimg_off + wimg_bytes(p));
+  w.wkimg_off = align_up(w.wimg_off + wimg_bytes(p));
+  w.total = align_up(w.wkimg_off + wimg_bytes(p));
   return w;
 }
 
@@ -167,6 +182,11 @@ extern "C" {
 
 int rehyat_version(void) { return 100; }
 
+int rehyat_attn_path(const rehyat_params* p) {
+  if (check_params(p) != REHYAT_OK) return -1;
+  return tc_path(p) ? 1 : 0;
+}
+
 const char* rehyat_status_string(rehyat_status s) {
   switch (s) {
     case REHYAT_OK: return "ok";
@@ -212,13 +232,15 @@ rehyat_status rehyat_fwd_state(const rehyat_params* p, const void* k, const void
   pp.nslots = p->T;
   pp.in_bf16 = p->in_dtype == REHYAT_BF16;
   pp.w_bf16 = pp.in_bf16;
-  cudaError_t e = launch_partials_simt(pp, s);
+  cudaError_t e = cudaSuccess;
+  if (tc_path(p) || tc_state_path(p))
+    e = launch_w_images(phi->Wq, ws + w.wimg_off, phi->Wk, ws + w.wkimg_off, p->heads, p->D,
+                        p->Dp, s);
   if (e != cudaSuccess) return to_status(e);
-  e = launch_scan(P, z, SL, zL, BH, p->T, p->Tc, p->To, nchunks_of(p), p->Dp, p->D, p->causal,
-                  s);
+  e = run_partials(p, pp, ws + w.wkimg_off, s);
   if (e != cudaSuccess) return to_status(e);
-  if (tc_path(p)) e = launch_wq_image(phi->Wq, ws + w.wimg_off, p->heads, p->D, p->Dp, s);
-  return to_status(e);
+  return to_status(launch_scan(P, z, SL, zL, BH, p->T, p->Tc, p->To, nchunks_of(p), p->Dp,
+                               p->D, p->causal, s));
 }
 
 rehyat_status rehyat_fwd_attn(const rehyat_params* p, const void* q, const void* k,
@@ -343,11 +365,12 @@ rehyat_status rehyat_chunk_step(const rehyat_params* p, const void* q, const voi
   a.nchunks = 1;
   a.nq_slices = nslices;
   cudaError_t e = cudaSuccess;
-  if (tc_path(p)) {
-    e = launch_wq_image(phi->Wq, ws + w.wimg_off, p->heads, p->D, p->Dp, s);
+  if (tc_path(p) || tc_state_path(p)) {
+    e = launch_w_images(phi->Wq, ws + w.wimg_off, phi->Wk, ws + w.wkimg_off, p->heads, p->D,
+                        p->Dp, s);
     if (e != cudaSuccess) return to_status(e);
-    a.wq_img = ws + w.wimg_off;
   }
+  if (tc_path(p)) a.wq_img = ws + w.wimg_off;
   e = run_attn(p, a, s);
   if (e != cudaSuccess) return to_status(e);
 
@@ -365,7 +388,7 @@ rehyat_status rehyat_chunk_step(const rehyat_params* p, const void* q, const voi
   pp.nq_slices = nslices;
   pp.in_bf16 = p->in_dtype == REHYAT_BF16;
   pp.w_bf16 = pp.in_bf16;
-  e = launch_partials_simt(pp, s);
+  e = run_partials(p, pp, ws + w.wkimg_off, s);
   if (e != cudaSuccess) return to_status(e);
   e = launch_state_add(P, zp, s_state, z_state, seen, BH, p->Dp, p->D, p->To, nslices,
                        w.nslots, s);

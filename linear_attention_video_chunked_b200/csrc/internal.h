@@ -60,11 +60,16 @@ struct PartialParams {
 cudaError_t launch_attn_simt(const AttnParams& p, cudaStream_t s);
 cudaError_t launch_partials_simt(const PartialParams& p, cudaStream_t s);
 
-// bf16 image of the phi_q weights (layout.cuh, wimg_index) for the
-// tensor-core readout: out [heads][Dp*D].
-cudaError_t launch_wq_image(const float* Wq, void* out, int heads, int D, int Dp,
-                            cudaStream_t s);
+// bf16 images of the phi weights (layout.cuh, wimg_index) for the
+// tensor-core kernels: out [heads][Dp*D] each.  Wk/out_k may be null.
+cudaError_t launch_w_images(const float* Wq, void* out_q, const float* Wk, void* out_k,
+                            int heads, int D, int Dp, cudaStream_t s);
 bool tc_attn_eligible(int in_bf16, int D, int Dp);
+
+// Tensor-core per-slice state (bf16, D = 128, Dp in {64, 128}); wk_img is
+// the bf16 image of W_k.
+bool tc_state_eligible(int in_bf16, int D, int Dp);
+cudaError_t launch_state_tc(const PartialParams& p, const void* wk_img, cudaStream_t s);
 
 // Linear-set state per chunk from the per-slice states (full mode).
 // causal: S^L_t = sum_{i < w_t} P_i.  bidirectional: S^L_t = sum_{i < w_t} P_i

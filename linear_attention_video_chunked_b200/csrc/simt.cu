@@ -408,16 +408,20 @@ __global__ void ring_update_kernel(const uint4* __restrict__ k, const uint4* __r
 
 __global__ void advance_kernel(long long* seen, int nq) { *seen += nq; }
 
-// bf16 copy of the phi_q weights in the tensor-core image layout.
-__global__ void wq_image_kernel(const float* __restrict__ Wq, __nv_bfloat16* __restrict__ out,
-                                int heads, int D, int Dp) {
+// bf16 copy of phi weights in the tensor-core image layout; blockIdx.y
+// selects the matrix (0: W_q, 1: W_k).
+__global__ void w_image_kernel(const float* __restrict__ Wq, __nv_bfloat16* __restrict__ out_q,
+                               const float* __restrict__ Wk, __nv_bfloat16* __restrict__ out_k,
+                               int heads, int D, int Dp) {
+  const float* Wsrc = blockIdx.y == 0 ? Wq : Wk;
+  __nv_bfloat16* out = blockIdx.y == 0 ? out_q : out_k;
   const long long per_head = static_cast<long long>(Dp) * D;
   const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= per_head * heads) return;
   const int h = static_cast<int>(i / per_head);
   const int rem = static_cast<int>(i % per_head);
   const int d = rem / Dp, f = rem % Dp;
-  out[h * per_head + wimg_index(f, d, D, Dp)] = __float2bfloat16_rn(Wq[w_index(h, D, Dp, d, f)]);
+  out[h * per_head + wimg_index(f, d, D, Dp)] = __float2bfloat16_rn(Wsrc[w_index(h, D, Dp, d, f)]);
 }
 
 template <int D>
@@ -500,11 +504,12 @@ cudaError_t launch_advance(long long* seen, int nq_slices, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_wq_image(const float* Wq, void* out, int heads, int D, int Dp,
-                            cudaStream_t s) {
+cudaError_t launch_w_images(const float* Wq, void* out_q, const float* Wk, void* out_k,
+                            int heads, int D, int Dp, cudaStream_t s) {
   const long long n = static_cast<long long>(heads) * D * Dp;
-  wq_image_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(
-      Wq, static_cast<__nv_bfloat16*>(out), heads, D, Dp);
+  dim3 grid(static_cast<unsigned>((n + 255) / 256), Wk != nullptr ? 2 : 1);
+  w_image_kernel<<<grid, 256, 0, s>>>(Wq, static_cast<__nv_bfloat16*>(out_q), Wk,
+                                      static_cast<__nv_bfloat16*>(out_k), heads, D, Dp);
   return cudaGetLastError();
 }
 

@@ -32,10 +32,9 @@
 
 #include "internal.h"
 #include "layout.cuh"
+#include "tc_common.cuh"
 
 namespace rehyat {
-
-__device__ unsigned int rehyat_tc_error = 0;
 
 namespace {
 
@@ -63,182 +62,21 @@ constexpr uint32_t kSmemBytes = kBarOff + 256 + 1024;  // + alignment slack
 enum {
   B_Q_FULL = 0, B_K_FULL = 1, B_V_FULL = 3, B_KV_EMPTY = 5, B_S_FULL = 7, B_S_FREE = 9,
   B_P_FULL = 11, B_PV_DONE = 12, B_TAIL_FULL = 13, B_PHI_DONE = 14, B_PHI_READY = 15,
-  B_READ_DONE = 16, B_COUNT = 17
+  B_READ_DONE = 16, B_LAST_PV = 17, B_COUNT = 18
 };
+// A parity wait is only meaningful for a waiter at most one phase behind the
+// barrier; B_LAST_PV completes exactly once (after the last P.V), so a role
+// that never followed B_PV_DONE can wait on it safely.
 constexpr uint32_t kTmemSlot = kBarOff + 8 * B_COUNT;       // u32: TMEM base address
 constexpr uint32_t kAbortSlot = kTmemSlot + 4;              // u32: abort flag
 
 constexpr uint32_t kColS0 = 0, kColO = 256, kColAL = 384;
 
-constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at the boost clock
+}  // namespace
 
-// ------------------------------------------------------------ PTX helpers
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
+using namespace tc;
 
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Bounded wait on the phase with the given parity.  On timeout: record the
-// barrier in the global error word, raise the CTA abort flag, return false.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag,
-                                       uint32_t code) {
-  if (mbar_try(bar, parity)) return true;
-  const long long t0 = clock64();
-  for (uint32_t i = 0;; ++i) {
-    if (mbar_try(bar, parity)) return true;
-    if ((i & 255u) == 255u) {
-      if (*abort_flag) return false;
-      if (clock64() - t0 > kWaitCycles) {
-        atomicOr(&rehyat_tc_error, 1u << (code & 31));
-        *abort_flag = 1;
-        return false;
-      }
-    }
-  }
-}
-
-__device__ __forceinline__ void fence_barrier_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-__device__ __forceinline__ void fence_proxy_async() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                            int x, int y, int z) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
-      : "memory");
-}
-
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
-                                          uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-          "r"(dst),
-      "l"(src), "r"(bytes), "r"(bar)
-      : "memory");
-}
-
-// UMMA shared-memory descriptor: 128-byte swizzle, version 1 (sm_100).
-__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
-  return static_cast<uint64_t>((addr & 0x3FFFFu) >> 4) |
-         (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
-         (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
-}
-
-// Instruction descriptor: fp32 accumulate, A K-major, A/B format fmt
-// (1 = bf16, 2 = tf32), B K-major or MN-major.
-__host__ __device__ constexpr uint32_t idesc(int M, int N, uint32_t fmt, bool b_mn_major) {
-  return (1u << 4) | (fmt << 7) | (fmt << 10) | ((b_mn_major ? 1u : 0u) << 16) |
-         (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
-}
-
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t id,
-                                         uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(id), "r"(accumulate));
-}
-
-__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t id,
-                                         uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(id), "r"(accumulate));
-}
-
-__device__ __forceinline__ void mma_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   bar)
-               : "memory");
-}
-
-#define REHYAT_TMEM_LD32(taddr, r)                                                              \
-  asm volatile(                                                                                \
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "  \
-      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "  \
-      "%28, %29, %30, %31}, [%32];"                                                            \
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),    \
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),             \
-        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),          \
-        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),          \
-        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),          \
-        "=r"(r[31])                                                                            \
-      : "r"(taddr))
-
-#define REHYAT_TMEM_ST32(taddr, r)                                                              \
-  asm volatile(                                                                                \
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, " \
-      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "  \
-      "%28, %29, %30, %31, %32};" ::"r"(taddr),                                                \
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),  \
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),        \
-      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),      \
-      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),      \
-      "r"(r[29]), "r"(r[30]), "r"(r[31]))
-
-__device__ __forceinline__ void tmem_wait_ld() {
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_wait_st() {
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  uint32_t r;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
-                                             uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
-               "r"(d)
-               : "memory");
-}
+namespace {
 
 // --------------------------------------------------------------- kernel
 struct TcMaps {
@@ -322,7 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     const uint32_t counts[B_COUNT] = {1, 1, 1, 1, 1, 1, 1, 1, 1, kSoftmaxThreads,
                                       kSoftmaxThreads, kSoftmaxThreads, 1, 1, 1,
-                                      kSoftmaxThreads, 1};
+                                      kSoftmaxThreads, 1, 1};
     for (int i = 0; i < B_COUNT; ++i) mbar_init(bar(i), counts[i]);
     *abort_flag = 0;
     fence_barrier_init();
@@ -364,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t slbytes = static_cast<uint32_t>(pw) * kD * 4;
       for (int pc = 0; pc < npieces && ok; ++pc) {
         if (pc == 0)
-          ok = mbar_wait(bar(B_PV_DONE), (nt - 1) & 1, abort_flag, 2);
+          ok = mbar_wait(bar(B_LAST_PV), 0, abort_flag, 2);
         else
           ok = mbar_wait(bar(B_READ_DONE), (pc - 1) & 1, abort_flag, 3);
         if (!ok) break;
@@ -418,6 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mma_commit(bar(B_PV_DONE));
         mma_commit(bar(B_KV_EMPTY + s));
+        if (j == nt - 1) mma_commit(bar(B_LAST_PV));
       }
       // Linear readout, one feature piece at a time.
       const uint32_t id_phi = idesc(kBM, pw, 1, false);
@@ -452,9 +291,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     float m_used = -INFINITY, m_max = -INFINITY, l = 0.f;
     bool ok = true;
+    // Warp-uniform outcome, so an abort never splits a warp before the
+    // warp-collective TMEM accesses.
+    auto wait_all = [&](uint32_t b, uint32_t parity, uint32_t code) {
+      return __all_sync(0xffffffffu, mbar_wait(b, parity, abort_flag, code));
+    };
     for (int j = 0; j < nt && ok; ++j) {
       const int s = j & 1;
-      ok = mbar_wait(bar(B_S_FULL + s), (j >> 1) & 1, abort_flag, 11);
+      ok = wait_all(bar(B_S_FULL + s), (j >> 1) & 1, 11);
       if (!ok) break;
       tc_fence_after();
       uint32_t xr[128];
@@ -494,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       l = l * alpha + lsum;
       if (j > 0) {
-        ok = mbar_wait(bar(B_PV_DONE), (j - 1) & 1, abort_flag, 12);
+        ok = wait_all(bar(B_PV_DONE), (j - 1) & 1, 12);
         if (!ok) break;
         tc_fence_after();
         if (__any_sync(0xffffffffu, rescale)) {
@@ -522,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (nvalid < kBN) {
         // Zero the V rows past the last valid key so 0 * garbage stays 0.
-        ok = mbar_wait(bar(B_V_FULL + s), (j >> 1) & 1, abort_flag, 13);
+        ok = wait_all(bar(B_V_FULL + s), (j >> 1) & 1, 13);
         if (!ok) break;
         if (r >= nvalid) {
           const uint32_t vrow = base + kStageOff + s * kStageBytes + 32768 + r * 128;
@@ -542,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float nL = 0.f;
     const float* zL = linear ? P.zL + (static_cast<long long>(bh) * P.nchunks + t) * Dp : nullptr;
     for (int pc = 0; pc < npieces && ok; ++pc) {
-      ok = mbar_wait(bar(B_PHI_DONE), pc & 1, abort_flag, 14);
+      ok = wait_all(bar(B_PHI_DONE), pc & 1, 14);
       if (!ok) break;
       tc_fence_after();
       for (int c = 0; c < pw / 32; ++c) {
@@ -573,9 +417,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok) {
       if (npieces > 0)
-        ok = mbar_wait(bar(B_READ_DONE), (npieces - 1) & 1, abort_flag, 15);
+        ok = wait_all(bar(B_READ_DONE), (npieces - 1) & 1, 15);
       else
-        ok = mbar_wait(bar(B_PV_DONE), (nt - 1) & 1, abort_flag, 15);
+        ok = wait_all(bar(B_PV_DONE), (nt - 1) & 1, 15);
     }
     if (ok) {
       tc_fence_after();
@@ -631,6 +475,276 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ===========================================================================
+// Per-slice linear state on tensor cores ("Key designs 1 and 4": the linear
+// branch's sum of phi_k(k) v^T and of phi_k(k)):
+//   P_s = phi_k(K_s)^T V_s  ([Dp][D] fp32),  z_s = sum_j phi_k(k_j)  ([Dp]).
+// One CTA per (slice, b*h), or per leaving slice in step mode.  Per 128-token
+// tile: psi = K W_k (tcgen05, bf16) -> phi = (psi + b)^2 in registers (thread
+// = token, TMEM lane) -> bf16 phi^T tile in shared memory (MN-major A) ->
+// P += phi^T V and z += phi^T 1 (tcgen05, fp32 accumulators in TMEM).
+// Roles as in the attention kernel: warps 0-3 convert + epilogue, warp 4 TMA,
+// warp 5 MMA.  Dp in {64, 128}; features past Dp are zero rows of phi^T.
+// ===========================================================================
+namespace st {
+constexpr int kThreads = 192;
+constexpr uint32_t kStageOff = 0;        // 2 stages x (K 32 KB + V 32 KB)
+constexpr uint32_t kStageBytes = 65536;
+constexpr uint32_t kWOff = 131072;       // W_k image, Dp x 128 bf16 (<= 32 KB)
+constexpr uint32_t kPhiOff = 163840;     // phi^T tile, 2 boxes x 16 KB
+constexpr uint32_t kOnesOff = 196608;    // all-ones B operand for z, 2 boxes x 2 KB
+constexpr uint32_t kBiasOff = 200704;    // b_k, Dp fp32
+constexpr uint32_t kBarOff = 201728;
+enum { K_FULL = 0, V_FULL = 2, KV_EMPTY = 4, PSI_FULL = 6, PSI_FREE = 8, PHI_FULL = 10,
+       ACC_DONE = 11, W_FULL = 12, NBAR = 13 };
+constexpr uint32_t kTmemSlot = kBarOff + 8 * NBAR;
+constexpr uint32_t kAbortSlot = kTmemSlot + 4;
+constexpr uint32_t kSmemBytes = kBarOff + 128 + 1024;
+constexpr uint32_t kColPsi = 0, kColP = 256, kColZ = 384;
+}  // namespace st
+
+struct StMaps {
+  CUtensorMap k, v, rk, rv;
+};
+
+__global__ void __launch_bounds__(st::kThreads, 1)
+    tc_state_kernel(const __grid_constant__ StMaps maps, const PartialParams P,
+                    const __nv_bfloat16* __restrict__ wk_img) {
+  // Local names shadow the attention kernel's constants of the same names.
+  constexpr int kThreads = st::kThreads;
+  constexpr uint32_t kStageOff = st::kStageOff, kStageBytes = st::kStageBytes;
+  constexpr uint32_t kWOff = st::kWOff, kPhiOff = st::kPhiOff, kOnesOff = st::kOnesOff;
+  constexpr uint32_t kBiasOff = st::kBiasOff, kBarOff = st::kBarOff;
+  constexpr uint32_t kTmemSlot = st::kTmemSlot, kAbortSlot = st::kAbortSlot;
+  constexpr uint32_t kColPsi = st::kColPsi, kColP = st::kColP, kColZ = st::kColZ;
+  constexpr int K_FULL = st::K_FULL, V_FULL = st::V_FULL, KV_EMPTY = st::KV_EMPTY;
+  constexpr int PSI_FULL = st::PSI_FULL, PSI_FREE = st::PSI_FREE, PHI_FULL = st::PHI_FULL;
+  constexpr int ACC_DONE = st::ACC_DONE, W_FULL = st::W_FULL, NBAR = st::NBAR;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* sbase = smem_raw + (base - raw);
+  auto bar = [&](int i) { return base + kBarOff + 8u * i; };
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(sbase + kAbortSlot);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int slot = blockIdx.x;
+  const int bh = blockIdx.y;
+  const int h = bh % P.heads;
+  const int Dp = P.Dp;
+  const int HW = P.HW;
+
+  // Which rows hold this slice (same rules as the CUDA-core kernel).
+  const CUtensorMap *mk, *mv;
+  int row0;
+  if (P.seen == nullptr) {
+    mk = &maps.k; mv = &maps.v;
+    row0 = slot * HW;
+  } else {
+    const long long seen = *P.seen;
+    const long long r = seen < P.To ? seen : P.To;
+    const long long after = seen + P.nq_slices;
+    const long long r2 = after < P.To ? after : P.To;
+    if (slot >= r + P.nq_slices - r2) return;
+    const long long g = seen - r + slot;
+    if (g < seen) {
+      mk = &maps.rk; mv = &maps.rv;
+      row0 = static_cast<int>(g % P.To) * HW;
+    } else {
+      mk = &maps.k; mv = &maps.v;
+      row0 = static_cast<int>(g - seen) * HW;
+    }
+  }
+  const int nt = (HW + 127) / 128;
+
+  if (tid == 0) {
+    const uint32_t counts[NBAR] = {1, 1, 1, 1, 1, 1, 1, 1, 128, 128, 128, 1, 1};
+    for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), counts[i]);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  // All-ones B operand (any swizzle of ones is ones) and the bias vector.
+  for (int i = tid; i < 1024; i += kThreads)
+    reinterpret_cast<uint32_t*>(sbase + kOnesOff)[i] = 0x3F803F80u;
+  for (int f = tid; f < Dp; f += kThreads) {
+    const int half = Dp >> 1, part = f >= half;
+    reinterpret_cast<float*>(sbase + kBiasOff)[f] = P.bk[(h * 2 + part) * half + (f - part * half)];
+  }
+  fence_proxy_async();
+  if (warp == 5) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     base + kTmemSlot),
+                 "r"(512));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sbase + kTmemSlot);
+
+  if (warp == 4) {
+    if (lane == 0) {
+      bool ok = true;
+      const uint32_t wbytes = static_cast<uint32_t>(Dp) * 128 * 2;
+      mbar_expect_tx(bar(W_FULL), wbytes);
+      bulk_load(base + kWOff, wk_img + static_cast<long long>(h) * Dp * 128, wbytes, bar(W_FULL));
+      for (int j = 0; j < nt && ok; ++j) {
+        const int s = j & 1;
+        if (j >= 2) ok = mbar_wait(bar(KV_EMPTY + s), ((j - 2) >> 1) & 1, abort_flag, 16);
+        if (!ok) break;
+        const uint32_t kdst = base + kStageOff + s * kStageBytes;
+        const int row = row0 + j * 128;
+        mbar_expect_tx(bar(K_FULL + s), 32768);
+        tma_load_3d(kdst, mk, bar(K_FULL + s), 0, row, bh);
+        tma_load_3d(kdst + 16384, mk, bar(K_FULL + s), 64, row, bh);
+        mbar_expect_tx(bar(V_FULL + s), 32768);
+        tma_load_3d(kdst + 32768, mv, bar(V_FULL + s), 0, row, bh);
+        tma_load_3d(kdst + 49152, mv, bar(V_FULL + s), 64, row, bh);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    if (lane == 0) {
+      const uint32_t id_psi = idesc_ab(128, Dp, 1, false, false);
+      const uint32_t id_st = idesc_ab(128, 128, 1, true, true);
+      const uint32_t id_z = idesc_ab(128, 16, 1, true, false);
+      bool ok = mbar_wait(bar(W_FULL), 0, abort_flag, 17);
+      auto issue_psi = [&](int i) -> bool {
+        const int s = i & 1;
+        if (!mbar_wait(bar(K_FULL + s), (i >> 1) & 1, abort_flag, 18)) return false;
+        if (i >= 2 && !mbar_wait(bar(PSI_FREE + s), ((i - 2) >> 1) & 1, abort_flag, 19))
+          return false;
+        tc_fence_after();
+        const uint32_t kaddr = base + kStageOff + s * kStageBytes;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
+          const uint32_t woff = (kk >> 2) * (Dp * 128) + (kk & 3) * 32;
+          mma_bf16(tmem + kColPsi + s * 128, sdesc(kaddr + koff, 16, 1024),
+                   sdesc(base + kWOff + woff, 16, 1024), id_psi, kk > 0);
+        }
+        mma_commit(bar(PSI_FULL + s));
+        return true;
+      };
+      if (ok) ok = issue_psi(0);
+      for (int j = 0; j < nt && ok; ++j) {
+        if (j + 1 < nt) ok = issue_psi(j + 1);
+        if (!ok) break;
+        const int s = j & 1;
+        ok = mbar_wait(bar(PHI_FULL), j & 1, abort_flag, 20) &&
+             mbar_wait(bar(V_FULL + s), (j >> 1) & 1, abort_flag, 21);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t vaddr = base + kStageOff + s * kStageBytes + 32768;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t a = sdesc(base + kPhiOff + kk * 2048, 16384, 1024);
+          const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+          mma_bf16(tmem + kColP, a, sdesc(vaddr + kk * 2048, 16384, 1024), id_st, acc);
+          mma_bf16(tmem + kColZ, a,
+                   sdesc(base + kOnesOff + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024), id_z, acc);
+        }
+        mma_commit(bar(ACC_DONE));
+        mma_commit(bar(KV_EMPTY + s));
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---- convert: thread r = token row r of the tile (TMEM lane r) ----
+    const int r = tid;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const float* bias = reinterpret_cast<const float*>(sbase + kBiasOff);
+    auto wait_all = [&](uint32_t b, uint32_t parity, uint32_t code) {
+      return __all_sync(0xffffffffu, mbar_wait(b, parity, abort_flag, code));
+    };
+    bool ok = true;
+    for (int j = 0; j < nt && ok; ++j) {
+      const int s = j & 1;
+      ok = wait_all(bar(PSI_FULL + s), (j >> 1) & 1, 22);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t ps[128];
+      REHYAT_TMEM_LD32(lane_base + kColPsi + s * 128, ps);
+      REHYAT_TMEM_LD32(lane_base + kColPsi + s * 128 + 32, (ps + 32));
+      if (Dp > 64) {
+        REHYAT_TMEM_LD32(lane_base + kColPsi + s * 128 + 64, (ps + 64));
+        REHYAT_TMEM_LD32(lane_base + kColPsi + s * 128 + 96, (ps + 96));
+      }
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar(PSI_FREE + s));
+      const int nvalid = min(128, HW - j * 128);
+      const bool valid = r < nvalid;
+      uint32_t pk[64];
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        float v0 = 0.f, v1 = 0.f;
+        if (valid && 2 * i < Dp) {
+          const float a0 = __uint_as_float(ps[2 * i]) + bias[2 * i];
+          const float a1 = __uint_as_float(ps[2 * i + 1]) + bias[2 * i + 1];
+          v0 = a0 * a0;
+          v1 = a1 * a1;
+        }
+        pk[i] = pack_bf16(v0, v1);
+      }
+      if (j > 0) {
+        ok = wait_all(bar(ACC_DONE), (j - 1) & 1, 23);
+        if (!ok) break;
+      }
+      // Token row r of the MN-major phi^T tile: features 64g..64g+63 in box g.
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const uint32_t box = c >> 3, ch = c & 7;
+        st_shared_v4(base + kPhiOff + box * 16384 + r * 128 + ((ch ^ (r & 7)) << 4), pk[4 * c],
+                     pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      }
+      if (nvalid < 128) {
+        ok = wait_all(bar(V_FULL + s), (j >> 1) & 1, 24);
+        if (!ok) break;
+        if (!valid) {
+          const uint32_t vrow = base + kStageOff + s * kStageBytes + 32768 + r * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            st_shared_v4(vrow + c * 16, 0, 0, 0, 0);
+            st_shared_v4(vrow + 16384 + c * 16, 0, 0, 0, 0);
+          }
+        }
+      }
+      fence_proxy_async();
+      tc_fence_before();
+      mbar_arrive(bar(PHI_FULL));
+    }
+    if (ok) ok = wait_all(bar(ACC_DONE), (nt - 1) & 1, 25);
+    if (ok) {
+      tc_fence_after();
+      // Thread r = feature r (accumulator lane r).
+      const long long obase = (static_cast<long long>(bh) * P.nslots + slot);
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[32];
+        REHYAT_TMEM_LD32(lane_base + kColP + c * 32, v);
+        tmem_wait_ld();
+        if (r < Dp) {
+          float4* dst = reinterpret_cast<float4*>(P.P + (obase * Dp + r) * 128 + c * 32);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                 __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+        }
+      }
+      uint32_t zv[32];
+      REHYAT_TMEM_LD32(lane_base + kColZ, zv);
+      tmem_wait_ld();
+      if (r < Dp) P.z[obase * Dp + r] = __uint_as_float(zv[0]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+  }
+}
+
 // ------------------------------------------------------------ host side
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -661,6 +775,32 @@ bool make_map(CUtensorMap* m, const void* ptr, long long rows, int planes) {
 }
 
 }  // namespace
+
+bool tc_state_eligible(int in_bf16, int D, int Dp) {
+  return in_bf16 && D == kD && (Dp == 64 || Dp == 128) && encode_fn() != nullptr;
+}
+
+cudaError_t launch_state_tc(const PartialParams& p, const void* wk_img, cudaStream_t s) {
+  StMaps maps;
+  memset(&maps, 0, sizeof(maps));
+  if (!make_map(&maps.k, p.k, p.rows_per_bh, p.BH) || !make_map(&maps.v, p.v, p.rows_per_bh, p.BH))
+    return cudaErrorInvalidValue;
+  if (p.seen && p.ring_rows_per_bh > 0) {
+    if (!make_map(&maps.rk, p.rk, p.ring_rows_per_bh, p.BH) ||
+        !make_map(&maps.rv, p.rv, p.ring_rows_per_bh, p.BH))
+      return cudaErrorInvalidValue;
+  } else {
+    maps.rk = maps.k;
+    maps.rv = maps.v;
+  }
+  cudaError_t e = cudaFuncSetAttribute(tc_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(st::kSmemBytes));
+  if (e != cudaSuccess) return e;
+  dim3 grid(p.nslots, p.BH);
+  tc_state_kernel<<<grid, st::kThreads, st::kSmemBytes, s>>>(
+      maps, p, static_cast<const __nv_bfloat16*>(wk_img));
+  return cudaGetLastError();
+}
 
 bool tc_attn_eligible(int in_bf16, int D, int Dp) {
   return in_bf16 && D == kD && (Dp == 64 || Dp == 128 || Dp == 256);
@@ -701,3 +841,15 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s) {
 }
 
 }  // namespace rehyat
+
+extern "C" rehyat_status rehyat_device_error_flags(unsigned* flags, int reset) {
+  if (!flags) return REHYAT_ERR_INVALID_ARG;
+  if (cudaMemcpyFromSymbol(flags, rehyat::rehyat_tc_error, sizeof(unsigned)) != cudaSuccess)
+    return REHYAT_ERR_CUDA;
+  if (reset) {
+    const unsigned zero = 0;
+    if (cudaMemcpyToSymbol(rehyat::rehyat_tc_error, &zero, sizeof(unsigned)) != cudaSuccess)
+      return REHYAT_ERR_CUDA;
+  }
+  return REHYAT_OK;
+}

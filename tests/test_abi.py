@@ -39,6 +39,17 @@ def test_library_loads_and_exports_every_declared_symbol():
     assert rh.rehyat_version() >= 100
 
 
+def test_attention_path_selection():
+    assert rh.rehyat_attn_path(_params()) == 1                       # bf16, D=128, Dp=128
+    assert rh.rehyat_attn_path(_params(Dp=64)) == 1
+    assert rh.rehyat_attn_path(_params(Dp=256)) == 1
+    assert rh.rehyat_attn_path(_params(Dp=32)) == 0                  # CUDA-core kernel
+    assert rh.rehyat_attn_path(_params(D=64)) == 0
+    assert rh.rehyat_attn_path(_params(in_dtype=rh.F32)) == 0
+    assert rh.rehyat_attn_path(_params(flags=rh.FLAG_FORCE_SIMT)) == 0
+    assert rh.rehyat_attn_path(_params(T=0)) == -1
+
+
 def test_status_strings():
     for code in range(6):
         assert rh.rehyat_status_string(code)
@@ -49,8 +60,9 @@ def test_workspace_bytes_layout():
     p = _params()
     BH, T, Dp, D, nch = 6, 7, 128, 128, 3
     need = BH * T * Dp * D * 4 + BH * T * Dp * 4 + BH * nch * Dp * D * 4 + BH * nch * Dp * 4
+    need += 3 * Dp * D * 2  # bf16 phi_q weight image, per head
     got = rh.rehyat_workspace_bytes(p)
-    assert need <= got <= need + 4 * 256
+    assert need <= got <= need + 5 * 256
     assert got % 256 == 0
 
 

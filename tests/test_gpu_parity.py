@@ -24,6 +24,10 @@ def _cuda():
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA GPU")
     rh.lib()
+    rh.rehyat_device_error_flags(reset=True)
+    yield
+    # No bounded wait inside the tensor-core kernels ran out during the module.
+    assert rh.rehyat_device_error_flags() == 0
 
 
 # ------------------------------------------------------------ tiny fp32 case
