@@ -377,8 +377,8 @@ def run_gpu(args, world, rank, local):
     attn_avg_s = sum(attn_ms) / len(attn_ms) / 1e3
     state_avg_s = sum(state_ms) / len(state_ms) / 1e3
     achieved_tf = w["attn_flops"] / attn_avg_s / 1e12
-    sha = kernel_source_sha(["linear_attention_video_chunked_b200/csrc/tc_attn.cu",
-                             "linear_attention_video_chunked_b200/csrc/simt.cu"])
+    sha = kernel_source_sha(["linear_attention_video_chunked_b200/csrc/tc_kernels.cu",
+                             "linear_attention_video_chunked_b200/csrc/tc_common.cuh"])
     roofline = {"kernel": "attention (window softmax + phi_q readout + joint norm)",
                 "bound": "tensor", "achieved": achieved_tf, "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": achieved_tf / peaks["bf16_tflops"],

@@ -46,23 +46,27 @@ constexpr int kSoftmaxThreads = 128;
 constexpr int kProducerWarp = 4;
 constexpr int kMmaWarp = 5;
 
-// Shared memory map (offsets from a 1024-aligned base).
-constexpr uint32_t kQOff = 0;                        // Q: 2 boxes x 16 KB
-constexpr uint32_t kStageOff = 32768;                // 2 stages x (K 32 KB + V 32 KB)
-constexpr uint32_t kStageBytes = 65536;
-constexpr uint32_t kPOff = kStageOff + 2 * kStageBytes;  // P: 2 boxes x 16 KB
-constexpr uint32_t kBarOff = kPOff + 32768;
-// Tail reuse of the stage/P region.
-constexpr uint32_t kWOff = kStageOff;                // phi_q weight piece (<= 32 KB)
-constexpr uint32_t kSLOff = kStageOff + 32768;       // S^L piece (<= 64 KB)
-constexpr uint32_t kPhiOff = kStageOff + 98304;      // phi_q(q) piece fp32 (<= 64 KB)
+// Shared memory map (offsets from a 1024-aligned base).  K and V have
+// separate rings: a K tile is released as soon as q.k^T has read it, a V tile
+// only after P.V, so the next K loads start two S-products ahead.
+constexpr int kKStages = 3, kVStages = 2;
+constexpr uint32_t kTileBytes = 32768;               // one 128 x 128 bf16 tile (2 boxes)
+constexpr uint32_t kQOff = 0;                        // Q tile
+constexpr uint32_t kKOff = 32768;                    // K ring, 3 tiles
+constexpr uint32_t kVOff = kKOff + kKStages * kTileBytes;   // V ring, 2 tiles
+constexpr uint32_t kPOff = kVOff + kVStages * kTileBytes;   // P tile
+constexpr uint32_t kBarOff = kPOff + kTileBytes;
+// Tail reuse of the K/V rings once the last P.V is done.
+constexpr uint32_t kWOff = kKOff;                    // phi_q weight piece (<= 32 KB)
+constexpr uint32_t kSLOff = kKOff + 32768;           // S^L piece (<= 64 KB)
+constexpr uint32_t kPhiOff = kVOff;                  // phi_q(q) piece fp32 (<= 64 KB)
 constexpr uint32_t kSmemBytes = kBarOff + 256 + 1024;  // + alignment slack
 
 // Barrier slots (8 bytes each).
 enum {
-  B_Q_FULL = 0, B_K_FULL = 1, B_V_FULL = 3, B_KV_EMPTY = 5, B_S_FULL = 7, B_S_FREE = 9,
-  B_P_FULL = 11, B_PV_DONE = 12, B_TAIL_FULL = 13, B_PHI_DONE = 14, B_PHI_READY = 15,
-  B_READ_DONE = 16, B_LAST_PV = 17, B_COUNT = 18
+  B_Q_FULL = 0, B_K_FULL = 1, B_K_EMPTY = 4, B_V_FULL = 7, B_V_EMPTY = 9, B_S_FULL = 11,
+  B_S_FREE = 13, B_P_FULL = 15, B_PV_DONE = 16, B_TAIL_FULL = 17, B_PHI_DONE = 18,
+  B_PHI_READY = 19, B_READ_DONE = 20, B_LAST_PV = 21, B_COUNT = 22
 };
 // A parity wait is only meaningful for a waiter at most one phase behind the
 // barrier; B_LAST_PV completes exactly once (after the last P.V), so a role
@@ -158,10 +162,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---- setup ----
   if (tid == 0) {
-    const uint32_t counts[B_COUNT] = {1, 1, 1, 1, 1, 1, 1, 1, 1, kSoftmaxThreads,
-                                      kSoftmaxThreads, kSoftmaxThreads, 1, 1, 1,
-                                      kSoftmaxThreads, 1, 1};
-    for (int i = 0; i < B_COUNT; ++i) mbar_init(bar(i), counts[i]);
+    for (int i = 0; i < B_COUNT; ++i) {
+      const bool by_softmax = (i == B_S_FREE || i == B_S_FREE + 1 || i == B_P_FULL ||
+                               i == B_PHI_READY);
+      mbar_init(bar(i), by_softmax ? kSoftmaxThreads : 1);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -184,18 +189,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load_3d(base + kQOff, &maps.q, bar(B_Q_FULL), 0, row0, bh);
       tma_load_3d(base + kQOff + 16384, &maps.q, bar(B_Q_FULL), 64, row0, bh);
       for (int j = 0; j < nt && ok; ++j) {
-        const int s = j & 1;
-        if (j >= 2) ok = mbar_wait(bar(B_KV_EMPTY + s), ((j - 2) >> 1) & 1, abort_flag, 1);
-        if (!ok) break;
         const TileSrc src = tile_src(j);
-        const uint32_t kdst = base + kStageOff + s * kStageBytes;
-        const uint32_t vdst = kdst + 32768;
-        mbar_expect_tx(bar(B_K_FULL + s), 32768);
-        tma_load_3d(kdst, src.map_k, bar(B_K_FULL + s), 0, src.row, bh);
-        tma_load_3d(kdst + 16384, src.map_k, bar(B_K_FULL + s), 64, src.row, bh);
-        mbar_expect_tx(bar(B_V_FULL + s), 32768);
-        tma_load_3d(vdst, src.map_v, bar(B_V_FULL + s), 0, src.row, bh);
-        tma_load_3d(vdst + 16384, src.map_v, bar(B_V_FULL + s), 64, src.row, bh);
+        const int ks = j % kKStages;
+        if (j >= kKStages)
+          ok = mbar_wait(bar(B_K_EMPTY + ks), ((j - kKStages) / kKStages) & 1, abort_flag, 1);
+        if (!ok) break;
+        const uint32_t kdst = base + kKOff + ks * kTileBytes;
+        mbar_expect_tx(bar(B_K_FULL + ks), kTileBytes);
+        tma_load_3d(kdst, src.map_k, bar(B_K_FULL + ks), 0, src.row, bh);
+        tma_load_3d(kdst + 16384, src.map_k, bar(B_K_FULL + ks), 64, src.row, bh);
+        const int vs = j & 1;
+        if (j >= kVStages) ok = mbar_wait(bar(B_V_EMPTY + vs), ((j - 2) >> 1) & 1, abort_flag, 26);
+        if (!ok) break;
+        const uint32_t vdst = base + kVOff + vs * kTileBytes;
+        mbar_expect_tx(bar(B_V_FULL + vs), kTileBytes);
+        tma_load_3d(vdst, src.map_v, bar(B_V_FULL + vs), 0, src.row, bh);
+        tma_load_3d(vdst + 16384, src.map_v, bar(B_V_FULL + vs), 64, src.row, bh);
       }
       // Readout operands, one feature piece at a time, into the freed stages.
       const uint32_t wbytes = static_cast<uint32_t>(pw) * kD * 2;
@@ -223,11 +232,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = mbar_wait(bar(B_Q_FULL), 0, abort_flag, 4);
       auto issue_s = [&](int i) -> bool {
         const int s = i & 1;
-        if (!mbar_wait(bar(B_K_FULL + s), (i >> 1) & 1, abort_flag, 5)) return false;
+        const int ks = i % kKStages;
+        if (!mbar_wait(bar(B_K_FULL + ks), (i / kKStages) & 1, abort_flag, 5)) return false;
         if (i >= 2 && !mbar_wait(bar(B_S_FREE + s), ((i - 2) >> 1) & 1, abort_flag, 6))
           return false;
         tc_fence_after();
-        const uint32_t kaddr = base + kStageOff + s * kStageBytes;
+        const uint32_t kaddr = base + kKOff + ks * kTileBytes;
         const uint32_t d = tmem + kColS0 + s * 128;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
@@ -236,6 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                    kk > 0);
         }
         mma_commit(bar(B_S_FULL + s));
+        mma_commit(bar(B_K_EMPTY + ks));
         return true;
       };
       if (ok) ok = issue_s(0);
@@ -247,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
              mbar_wait(bar(B_V_FULL + s), (j >> 1) & 1, abort_flag, 8);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t vaddr = base + kStageOff + s * kStageBytes + 32768;
+        const uint32_t vaddr = base + kVOff + s * kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t a = sdesc(base + kPOff + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
@@ -255,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_bf16(tmem + kColO, a, b, id_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(bar(B_PV_DONE));
-        mma_commit(bar(B_KV_EMPTY + s));
+        mma_commit(bar(B_V_EMPTY + s));
         if (j == nt - 1) mma_commit(bar(B_LAST_PV));
       }
       // Linear readout, one feature piece at a time.
@@ -310,33 +321,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         REHYAT_TMEM_LD32(sa + 96, (xr + 96));
         tmem_wait_ld();
       }
-      float x[128];
       tc_fence_before();
       mbar_arrive(bar(B_S_FREE + s));
       const int nvalid = tile_src(j).nvalid;
-      float mt = -INFINITY;
+      if (nvalid < kBN) {  // ragged tile (warp-uniform): mask keys past the end
 #pragma unroll
-      for (int i = 0; i < 128; ++i) {
-        x[i] = (i < nvalid) ? __uint_as_float(xr[i]) * P.scale_log2 : -INFINITY;
-        mt = fmaxf(mt, x[i]);
+        for (int i = 0; i < 128; ++i)
+          if (i >= nvalid) xr[i] = __float_as_uint(-INFINITY);
       }
-      m_max = fmaxf(m_max, mt);
+      // Row max of the raw logits as a tree (the scale is positive).
+      float mx[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) mx[i] = __uint_as_float(xr[i]);
+#pragma unroll
+      for (int i = 16; i < 128; ++i) mx[i & 15] = fmaxf(mx[i & 15], __uint_as_float(xr[i]));
+#pragma unroll
+      for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+        for (int i = 0; i < w; ++i) mx[i] = fmaxf(mx[i], mx[i + w]);
+      m_max = fmaxf(m_max, mx[0] * P.scale_log2);
       float alpha = 1.f;
       const bool rescale = m_max > m_used + 8.f;
       if (rescale) {
         alpha = ex2(m_used - m_max);  // 0 on the first tile
         m_used = m_max;
       }
+      // p = 2^(s * scale * log2(e) - m_used), one FFMA + one MUFU each; the
+      // row sum uses 8 independent accumulators.
+      const float neg_m = -m_used;
       uint32_t pk[64];
-      float lsum = 0.f;
+      float ls[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) ls[i] = 0.f;
 #pragma unroll
       for (int i = 0; i < 64; ++i) {
-        const float p0 = ex2(x[2 * i] - m_used);
-        const float p1 = ex2(x[2 * i + 1] - m_used);
+        const float p0 = ex2(fmaf(__uint_as_float(xr[2 * i]), P.scale_log2, neg_m));
+        const float p1 = ex2(fmaf(__uint_as_float(xr[2 * i + 1]), P.scale_log2, neg_m));
         pk[i] = pack_bf16(p0, p1);
-        lsum += __uint_as_float(pk[i] << 16) + __uint_as_float(pk[i] & 0xFFFF0000u);
+        ls[i & 7] += p0 + p1;
       }
-      l = l * alpha + lsum;
+      l = l * alpha + (((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7])));
       if (j > 0) {
         ok = wait_all(bar(B_PV_DONE), (j - 1) & 1, 12);
         if (!ok) break;
@@ -369,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = wait_all(bar(B_V_FULL + s), (j >> 1) & 1, 13);
         if (!ok) break;
         if (r >= nvalid) {
-          const uint32_t vrow = base + kStageOff + s * kStageBytes + 32768 + r * 128;
+          const uint32_t vrow = base + kVOff + s * kTileBytes + r * 128;
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             st_shared_v4(vrow + c * 16, 0, 0, 0, 0);
