@@ -57,7 +57,9 @@ typedef enum {
   REHYAT_ERR_UNSUPPORTED = 2,  /* D or Dp outside the supported set */
   REHYAT_ERR_MISALIGNED = 3,   /* a pointer not 16-byte aligned */
   REHYAT_ERR_WORKSPACE = 4,    /* workspace or state smaller than required */
-  REHYAT_ERR_CUDA = 5          /* a CUDA launch or query failed */
+  REHYAT_ERR_CUDA = 5,         /* a CUDA launch or query failed */
+  REHYAT_ERR_SCRATCH_LIMIT = 6 /* problem needs more workspace than the fixed
+                                  scratch of rehyat_hybrid_attn_fwd_noalloc */
 } rehyat_status;
 
 typedef enum { REHYAT_F32 = 0, REHYAT_BF16 = 1 } rehyat_dtype;
@@ -133,6 +135,32 @@ REHYAT_API rehyat_status rehyat_fwd_attn(const rehyat_params* p, const void* q,
                                          const rehyat_phi* phi, void* y,
                                          const void* workspace, size_t ws_bytes,
                                          const rehyat_debug* dbg, void* stream);
+
+/* The full forward without a caller-supplied workspace, for callers that
+ * cannot allocate device memory (code running under another runtime's
+ * allocator or memory pool, plug-in hosts that forbid allocation after
+ * start-up, tools that only pass along buffers they were given).  The
+ * paper has no counterpart: this is a packaging variant of
+ * rehyat_hybrid_attn_fwd, with identical arguments minus the workspace and
+ * identical results.
+ *   - Scratch: a 32 MiB __device__ array inside the library.  Every GPU that
+ *     loads the library holds it until the process exits.  Problems whose
+ *     rehyat_workspace_bytes exceeds 32 MiB return REHYAT_ERR_SCRATCH_LIMIT
+ *     and enqueue nothing (e.g. one 21x20x30 layer with 12 heads fits, the
+ *     batch-2 21x30x52 layer does not).
+ *   - Allocates nothing: no cudaMalloc/cudaFree and no allocating library
+ *     call.  The first call on each device looks up the array's device
+ *     address (cudaGetSymbolAddress, with that device current); make that
+ *     first call before any stream capture.
+ *   - The array is shared by every call on a device and keeps the last
+ *     call's contents (each call overwrites all of it that it reads, so no
+ *     clearing is needed).  Calls that overlap on the GPU (other streams,
+ *     other host threads) race on it: serialise them. */
+REHYAT_API rehyat_status rehyat_hybrid_attn_fwd_noalloc(const rehyat_params* p, const void* q,
+                                                        const void* k, const void* v,
+                                                        const rehyat_phi* phi, void* y,
+                                                        const rehyat_debug* dbg,
+                                                        void* stream);
 
 /* Plain softmax attention over all N keys (no chunking, no linear branch):
  * the dense comparator the ReHyAt note measures against (Experiments,

@@ -28,20 +28,22 @@ __all__ = [
     "rehyat_workspace_bytes", "rehyat_hybrid_attn_fwd", "rehyat_fwd_state", "rehyat_fwd_attn",
     "rehyat_softmax_attn_fwd", "rehyat_state_bytes", "rehyat_state_init", "rehyat_step_workspace_bytes",
     "rehyat_chunk_step", "rehyat_device_error_flags", "rehyat_attn_path",
-    "rehyat_status_string", "rehyat_version", "make_params", "hybrid_attn", "softmax_attn", "StreamingState",
+    "rehyat_status_string", "rehyat_version", "rehyat_hybrid_attn_fwd_noalloc", "make_params", "hybrid_attn", "softmax_attn", "StreamingState",
 ]
 
 F32, BF16 = 0, 1
 FLAG_FORCE_SIMT = 1
 
 STATUS = {0: "REHYAT_OK", 1: "REHYAT_ERR_INVALID_ARG", 2: "REHYAT_ERR_UNSUPPORTED",
-          3: "REHYAT_ERR_MISALIGNED", 4: "REHYAT_ERR_WORKSPACE", 5: "REHYAT_ERR_CUDA"}
+          3: "REHYAT_ERR_MISALIGNED", 4: "REHYAT_ERR_WORKSPACE", 5: "REHYAT_ERR_CUDA",
+          6: "REHYAT_ERR_SCRATCH_LIMIT"}
 
 EXPORTED_SYMBOLS = (
     "rehyat_workspace_bytes", "rehyat_hybrid_attn_fwd", "rehyat_fwd_state",
     "rehyat_fwd_attn", "rehyat_softmax_attn_fwd", "rehyat_state_bytes", "rehyat_state_init",
     "rehyat_step_workspace_bytes", "rehyat_chunk_step", "rehyat_device_error_flags",
     "rehyat_attn_path", "rehyat_status_string", "rehyat_version",
+    "rehyat_hybrid_attn_fwd_noalloc",
 )
 
 
@@ -98,6 +100,9 @@ def lib() -> ctypes.CDLL:
         L.rehyat_fwd_attn.argtypes = [P(RehyatParams), vp, vp, vp, P(RehyatPhi), vp, vp, sz,
                                       P(RehyatDebug), vp]
         L.rehyat_fwd_attn.restype = i
+        L.rehyat_hybrid_attn_fwd_noalloc.argtypes = [P(RehyatParams), vp, vp, vp, P(RehyatPhi),
+                                                     vp, P(RehyatDebug), vp]
+        L.rehyat_hybrid_attn_fwd_noalloc.restype = i
         L.rehyat_softmax_attn_fwd.argtypes = [P(RehyatParams), vp, vp, vp, vp, vp]
         L.rehyat_softmax_attn_fwd.restype = i
         L.rehyat_state_bytes.argtypes = [P(RehyatParams)]
@@ -140,6 +145,14 @@ def rehyat_fwd_state(p, k, v, phi, workspace, ws_bytes, stream) -> int:
 def rehyat_fwd_attn(p, q, k, v, phi, y, workspace, ws_bytes, dbg, stream) -> int:
     return lib().rehyat_fwd_attn(ctypes.byref(p), q, k, v, ctypes.byref(phi), y, workspace,
                                  ws_bytes, None if dbg is None else ctypes.byref(dbg), stream)
+
+
+def rehyat_hybrid_attn_fwd_noalloc(p, q, k, v, phi, y, dbg, stream) -> int:
+    """The full forward on the library's built-in 32 MiB device scratch, for
+    callers that cannot allocate a workspace (see include/rehyat.h)."""
+    return lib().rehyat_hybrid_attn_fwd_noalloc(ctypes.byref(p), q, k, v, ctypes.byref(phi), y,
+                                                None if dbg is None else ctypes.byref(dbg),
+                                                stream)
 
 
 def rehyat_softmax_attn_fwd(p, q, k, v, y, stream) -> int:

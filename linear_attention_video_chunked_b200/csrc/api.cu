@@ -195,6 +195,7 @@ const char* rehyat_status_string(rehyat_status s) {
     case REHYAT_ERR_MISALIGNED: return "pointer not 16-byte aligned";
     case REHYAT_ERR_WORKSPACE: return "workspace or state too small";
     case REHYAT_ERR_CUDA: return "CUDA launch error";
+    case REHYAT_ERR_SCRATCH_LIMIT: return "problem needs more than the built-in 32 MiB scratch";
   }
   return "unknown status";
 }

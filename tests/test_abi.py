@@ -51,8 +51,8 @@ def test_attention_path_selection():
 
 
 def test_status_strings():
-    for code in range(6):
-        assert rh.rehyat_status_string(code)
+    for code in range(7):
+        assert rh.rehyat_status_string(code) != "unknown status"
     assert rh.rehyat_status_string(0) == "ok"
 
 
@@ -60,9 +60,9 @@ def test_workspace_bytes_layout():
     p = _params()
     BH, T, Dp, D, nch = 6, 7, 128, 128, 3
     need = BH * T * Dp * D * 4 + BH * T * Dp * 4 + BH * nch * Dp * D * 4 + BH * nch * Dp * 4
-    need += 3 * Dp * D * 2  # bf16 phi_q weight image, per head
+    need += 2 * 3 * Dp * D * 2  # bf16 phi_q and phi_k weight images, per head
     got = rh.rehyat_workspace_bytes(p)
-    assert need <= got <= need + 5 * 256
+    assert need <= got <= need + 6 * 256
     assert got % 256 == 0
 
 
