@@ -209,6 +209,96 @@ def run_oracle_sample(p, plan, start_head=0):
                        f"{chunks[0]}..{chunks[-1]} of {nch} ({rows} query rows per pair)")
 
 
+# ------------------------------------------------------ extra measurements
+def measure_full_softmax(rh, q, k, v, y, flush, stream, calls=3):
+    """Plain softmax over all N keys on the same tensors (the dense
+    comparator the ReHyAt note measures against), device time per call."""
+    import torch
+    B, H, N, D = q.shape
+    p = rh.make_params(batch=B, heads=H, T=1, Hs=1, Ws=N, D=D, Dp=32, Tc=1, To=0, causal=0,
+                       in_dtype=rh.BF16, out_dtype=rh.F32)
+    sh = stream.cuda_stream
+    call = lambda: rh.rehyat_softmax_attn_fwd(p, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                              y.data_ptr(), sh)
+    if call():
+        raise RuntimeError("rehyat_softmax_attn_fwd failed")
+    times = []
+    for _ in range(calls):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        call()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    return {"ms": sum(times) / len(times), "calls": calls,
+            "what": "rehyat_softmax_attn_fwd on the same q, k, v (all N keys per query)"}
+
+
+def measure_streaming(rh, dev, flush, stream):
+    """Chunk-wise RNN over 81 slices of 30x52 (27 steps of T_c = 3, T_o = 1,
+    12 heads, D = D' = 128): per-step device time, steady-state tokens/s,
+    free device memory before and after the 27 steps."""
+    import torch
+    g = torch.Generator(device=dev).manual_seed(3)
+    H, HW, D, Dp, Tc, To, T = 12, 30 * 52, 128, 128, 3, 1, 81
+    rows = Tc * HW
+
+    def draw(shape, scale=1.0):
+        return torch.randn(shape, generator=g, device=dev, dtype=torch.float32) * scale
+
+    s = 0.5 + 1.5 * torch.rand((3, H, 1, 1), generator=g, device=dev)
+    q = (draw((1, H, T * HW, D)) * s[0]).to(torch.bfloat16)
+    k = (draw((1, H, T * HW, D)) * s[1]).to(torch.bfloat16)
+    v = (draw((1, H, T * HW, D)) * s[2]).to(torch.bfloat16)
+    Wq, Wk = draw((H, 2, D, Dp // 2), 0.1), draw((H, 2, D, Dp // 2), 0.1)
+    bq, bk = draw((H, 2, Dp // 2), 0.1), draw((H, 2, Dp // 2), 0.1)
+    chunks = [tuple(x[:, :, i * rows:(i + 1) * rows].contiguous() for x in (q, k, v))
+              for i in range(T // Tc)]
+    del q, k, v
+    st = rh.StreamingState(batch=1, heads=H, Hs=30, Ws=52, D=D, Dp=Dp, Tc=Tc, To=To, Wq=Wq,
+                           bq=bq, Wk=Wk, bk=bk, in_dtype=torch.bfloat16, device=dev)
+    out = torch.empty(1, H, rows, D, device=dev)
+    for c in chunks[:3]:  # warm-up
+        st.step(*c, out=out)
+    st.reset()
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info(dev)[0]
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in chunks]
+    for (e0, e1), c in zip(evs, chunks):
+        e0.record(stream)
+        st.step(*c, out=out)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    free1 = torch.cuda.mem_get_info(dev)[0]
+    ms = [e0.elapsed_time(e1) for e0, e1 in evs]
+    steady = sorted(ms[2:])[len(ms[2:]) // 2]
+    return {"workload": "81 slices of 30x52, 12 heads, D=D'=128, T_c=3, T_o=1, bf16, "
+                        "27 rehyat_chunk_step calls (inputs from a seeded torch generator)",
+            "steps": len(ms), "ms_per_step_median_steady": steady,
+            "ms_first_steps": ms[:3], "tokens_per_s_steady": rows / (steady / 1e3),
+            "free_bytes_before": free0, "free_bytes_after": free1,
+            "device_memory_constant": free0 == free1}
+
+
+# ------------------------------------------------------------ multi-rank
+def max_over_ranks(ms, dist=None, device=None):
+    """Device time of the slowest rank (every rank calls this, in order)."""
+    if dist is None:
+        return float(ms)
+    import torch
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, tokens_per_step, steps, max_ms):
+    """Whole-job tokens/s: every rank runs the same workload (replicas), so
+    the job processed world * tokens_per_step * steps tokens in max_ms."""
+    return world * tokens_per_step * steps / (max_ms / 1e3)
+
+
 # --------------------------------------------------------------- main arms
 def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -324,14 +414,10 @@ def run_gpu(args, world, rank, local):
     step_ms = [e[0].elapsed_time(e[2]) for e in events]
     state_ms = [e[0].elapsed_time(e[1]) for e in events]
     attn_ms = [e[1].elapsed_time(e[2]) for e in events]
-    total_ms = sum(step_ms)
-    if dist:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dist, dev)
     ms_per_step = total_ms / args.steps
     tokens_per_step = B * N
-    value = world * tokens_per_step * args.steps / (total_ms / 1e3)
+    value = job_throughput(world, tokens_per_step, args.steps, total_ms)
 
     # End to end through the public API, host buffers in and out.
     qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
@@ -357,15 +443,20 @@ def run_gpu(args, world, rank, local):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
     if dist:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
         dist.barrier()
-    e2e_value = world * tokens_per_step * e2e_steps / (e2e_ms / 1e3)
+    e2e_value = job_throughput(world, tokens_per_step, e2e_steps, e2e_ms)
     h2d = sum(x.numel() * x.element_size() for x in (qh, kh, vh))
     d2h = yh.numel() * yh.element_size()
+    del qh, kh, vh, yh, qd, kd, vd
+
+    extra = {}
+    if not args.no_extras:
+        extra["full_softmax"] = measure_full_softmax(rh, q, k, v, y, flush, stream)
+        del q, k, v, y, ws
+        torch.cuda.empty_cache()
+        extra["streaming"] = measure_streaming(rh, dev, flush, stream)
 
     if rank != 0:
         if dist:
@@ -410,6 +501,12 @@ def run_gpu(args, world, rank, local):
                 "api": "linear_attention_video_chunked_b200.hybrid_attn"},
         "clocks": clocks.summary(t_host0, t_host1),
     }
+    line.update(extra)
+    if "full_softmax" in extra:
+        fs = extra["full_softmax"]
+        fs["tflops"] = w["full_softmax_flops"] / (fs["ms"] / 1e3) / 1e12
+        fs["frac_bf16_peak"] = fs["tflops"] / peaks["bf16_tflops"]
+        fs["hybrid_speedup"] = fs["ms"] / ms_per_step
     if world == 1 and not args.no_cpu_baseline:
         r = run_oracle_sample(p, plan_oracle_sample(p, args.cpu_budget))
         cv = r["token_equiv"] / r["seconds"]
@@ -431,6 +528,8 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of fp64 oracle work for the CPU baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the full-softmax comparator and the streaming measurement")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     world, rank, local = dist_setup()
