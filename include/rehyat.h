@@ -67,6 +67,9 @@ typedef enum { REHYAT_F32 = 0, REHYAT_BF16 = 1 } rehyat_dtype;
 /* Flags for rehyat_params.flags. */
 #define REHYAT_FLAG_FORCE_SIMT 1 /* use the fp32 CUDA-core kernels even where a
                                     tensor-core kernel exists (testing aid) */
+#define REHYAT_FLAG_ONE_TILE 2   /* tensor-core attention: use the one-query-tile
+                                    kernel (the default for Dp = 256) instead of
+                                    the two-tile kernel (testing aid) */
 
 typedef struct {
   int batch, heads;   /* B >= 1, h >= 1 */

@@ -33,6 +33,7 @@ __all__ = [
 
 F32, BF16 = 0, 1
 FLAG_FORCE_SIMT = 1
+FLAG_ONE_TILE = 2
 
 STATUS = {0: "REHYAT_OK", 1: "REHYAT_ERR_INVALID_ARG", 2: "REHYAT_ERR_UNSUPPORTED",
           3: "REHYAT_ERR_MISALIGNED", 4: "REHYAT_ERR_WORKSPACE", 5: "REHYAT_ERR_CUDA",
@@ -249,8 +250,8 @@ def _debug_tensors(shape4, device):
 
 
 def hybrid_attn(q, k, v, Wq, bq, Wk, bk, *, T, Hs, Ws, Tc, To, causal, out_dtype=None,
-                scale=0.0, debug=False, force_simt=False, workspace=None, out=None,
-                stream=None):
+                scale=0.0, debug=False, force_simt=False, one_tile=False, workspace=None,
+                out=None, stream=None):
     """ReHyAt hybrid attention of torch CUDA tensors q, k, v [B, h, N, D].
 
     Returns y (and a dict of branch partials when ``debug``)."""
@@ -263,7 +264,8 @@ def hybrid_attn(q, k, v, Wq, bq, Wk, bk, *, T, Hs, Ws, Tc, To, causal, out_dtype
     p = make_params(batch=B, heads=H, T=T, Hs=Hs, Ws=Ws, D=D, Dp=Dp, Tc=Tc, To=To,
                     causal=causal, in_dtype=_dtype_code(q.dtype),
                     out_dtype=_dtype_code(out_dtype), scale=scale,
-                    flags=FLAG_FORCE_SIMT if force_simt else 0)
+                    flags=(FLAG_FORCE_SIMT if force_simt else 0) |
+                    (FLAG_ONE_TILE if one_tile else 0))
     y = torch.empty(B, H, N, D, dtype=out_dtype, device=q.device) if out is None else out
     nbytes = rehyat_workspace_bytes(p)
     if nbytes == 0:

@@ -141,6 +141,7 @@ AttnParams base_attn(const rehyat_params* p, const void* q, const void* k, const
   a.in_bf16 = p->in_dtype == REHYAT_BF16;
   a.out_bf16 = p->out_dtype == REHYAT_BF16;
   a.w_bf16 = a.in_bf16;
+  a.one_tile = (p->flags & REHYAT_FLAG_ONE_TILE) != 0;
   a.scale_log2 = logit_scale(p) * 1.4426950408889634f;
   return a;
 }

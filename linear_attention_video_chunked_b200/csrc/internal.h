@@ -33,6 +33,7 @@ struct AttnParams {
   float *dbg_aS, *dbg_nS, *dbg_c, *dbg_aL, *dbg_nL;
   int BH, heads, T, HW, D, Dp, Tc, To, nchunks, nq_slices;
   int in_bf16, out_bf16, w_bf16, full_softmax;
+  int one_tile;              // tensor-core path: force the one-query-tile kernel
   float scale_log2;          // logit scale * log2(e)
 };
 

@@ -500,6 +500,462 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ===========================================================================
+// Attention kernel with two query tiles per CTA (used when D' <= 128).
+//
+// Same computation as tc_attn_kernel, arranged so the tensor core alternates
+// between two 128-row query tiles A and B of one chunk: while softmax
+// warpgroup A turns S_A(j) into P_A(j), the MMA warp runs q.k^T of tile B and
+// P.V of tile A, and the other way round.  P stays in TMEM (bf16, two per
+// 32-bit column, over the first 64 columns of its S buffer) and feeds P.V as
+// the A operand straight from TMEM, so shared memory only holds Q_A, Q_B and
+// the K (3 stages) and V (2 stages) rings.  The linear readout multiplies
+// phi_q(q) by 1/f (f = exp2(m_used - m_max) <= 1) and accumulates into O, so
+// y = f*O / (f*n^S + n^L).
+//
+// Roles (320 threads): warps 0-3 softmax + epilogue of tile A, warps 4-7 of
+// tile B, warp 8 TMA, warp 9 MMA and TMEM owner.
+// TMEM: S_A [0,128) O_A [128,256) S_B [256,384) O_B [384,512).
+// ===========================================================================
+namespace a2 {
+constexpr int kThreads = 320;
+constexpr uint32_t kQOff = 0;                      // Q_A, Q_B
+constexpr uint32_t kKOff = 65536;                  // K ring, 3 x 32 KB
+constexpr uint32_t kVOff = kKOff + 3 * 32768;      // V ring, 2 x 32 KB
+constexpr uint32_t kBarOff = kVOff + 2 * 32768;
+constexpr uint32_t kWOff = kKOff;                  // tail: phi_q weights (<= 32 KB)
+constexpr uint32_t kSLOff = kKOff + 32768;         // tail: S^L (<= 64 KB)
+constexpr uint32_t kPhiOff0 = kVOff;               // tail: phi_q(Q_A)/f (<= 64 KB)
+constexpr uint32_t kPhiOff1 = kQOff;               // tail: phi_q(Q_B)/f, over Q (<= 64 KB)
+enum { Q_FULL = 0, K_FULL = 1, K_EMPTY = 4, V_FULL = 7, V_EMPTY = 9, S_FULL = 11, P_FULL = 13,
+       PV_DONE = 15, LAST_PV = 17, TAIL_FULL = 18, PHI_DONE = 19, PHI_READY = 20, READ_DONE = 22,
+       NBAR = 23 };
+constexpr uint32_t kTmemSlot = kBarOff + 8 * NBAR;
+constexpr uint32_t kAbortSlot = kTmemSlot + 4;
+constexpr uint32_t kSmemBytes = kBarOff + 256 + 1024;
+}  // namespace a2
+
+__global__ void __launch_bounds__(a2::kThreads, 1)
+    tc_attn2_kernel(const __grid_constant__ TcMaps maps, const AttnParams P,
+                    const __nv_bfloat16* __restrict__ wq_img) {
+  using a2::kQOff;
+  using a2::kKOff;
+  using a2::kVOff;
+  using a2::kBarOff;
+  using a2::kWOff;
+  using a2::kSLOff;
+  using a2::kPhiOff0;
+  using a2::kPhiOff1;
+  using a2::kTmemSlot;
+  using a2::kAbortSlot;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* sbase = smem_raw + (base - raw);
+  auto bar = [&](int i) { return base + kBarOff + 8u * i; };
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(sbase + kAbortSlot);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int t = blockIdx.y;
+  const int bh = blockIdx.z;
+  const int h = bh % P.heads;
+
+  int q_first, q_end, na, nb, a_row0;
+  const bool step_mode = P.seen != nullptr;
+  if (!step_mode) {
+    const int first = t * P.Tc;
+    const int end = min(P.T, first + P.Tc);
+    const int w = max(first - P.To, 0);
+    q_first = first * P.HW;
+    q_end = end * P.HW;
+    a_row0 = w * P.HW;
+    na = (end - w) * P.HW;
+    nb = 0;
+  } else {
+    const long long seen = *P.seen;
+    const int r_slices = static_cast<int>(seen < P.To ? seen : P.To);
+    q_first = 0;
+    q_end = P.nq_slices * P.HW;
+    a_row0 = 0;
+    na = r_slices * P.HW;
+    nb = q_end;
+  }
+  const int row0 = q_first + blockIdx.x * 2 * kBM;
+  if (row0 >= q_end) return;
+  const int nrows_t[2] = {min(kBM, q_end - row0), max(0, min(kBM, q_end - row0 - kBM))};
+  const bool has_b = nrows_t[1] > 0;
+  const int nta = (na + kBN - 1) / kBN;
+  const int nt = nta + (nb + kBN - 1) / kBN;
+  const bool linear = !P.full_softmax;
+  const int Dp = P.Dp;  // <= 128 here: one feature piece
+
+  auto tile_src = [&](int j) {
+    TileSrc s;
+    if (j < nta) {
+      s.map_k = step_mode ? &maps.rk : &maps.k;
+      s.map_v = step_mode ? &maps.rv : &maps.v;
+      s.row = a_row0 + j * kBN;
+      s.nvalid = min(kBN, na - j * kBN);
+    } else {
+      const int jb = j - nta;
+      s.map_k = &maps.k;
+      s.map_v = &maps.v;
+      s.row = jb * kBN;
+      s.nvalid = min(kBN, nb - jb * kBN);
+    }
+    return s;
+  };
+
+  if (tid == 0) {
+    for (int i = 0; i < a2::NBAR; ++i) {
+      const bool by_warpgroup = i == a2::P_FULL || i == a2::P_FULL + 1 || i == a2::PHI_READY ||
+                                i == a2::PHI_READY + 1;
+      mbar_init(bar(i), by_warpgroup ? kSoftmaxThreads : 1);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 9) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     base + kTmemSlot),
+                 "r"(512));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sbase + kTmemSlot);
+
+  if (warp == 8) {
+    // ================================================= TMA producer
+    if (lane == 0) {
+      bool ok = true;
+      mbar_expect_tx(bar(a2::Q_FULL), 4 * 16384);
+      tma_load_3d(base + kQOff, &maps.q, bar(a2::Q_FULL), 0, row0, bh);
+      tma_load_3d(base + kQOff + 16384, &maps.q, bar(a2::Q_FULL), 64, row0, bh);
+      tma_load_3d(base + kQOff + 32768, &maps.q, bar(a2::Q_FULL), 0, row0 + kBM, bh);
+      tma_load_3d(base + kQOff + 49152, &maps.q, bar(a2::Q_FULL), 64, row0 + kBM, bh);
+      for (int j = 0; j < nt && ok; ++j) {
+        const TileSrc src = tile_src(j);
+        const int ks = j % 3;
+        if (j >= 3) ok = mbar_wait(bar(a2::K_EMPTY + ks), ((j - 3) / 3) & 1, abort_flag, 1);
+        if (!ok) break;
+        const uint32_t kdst = base + kKOff + ks * 32768;
+        mbar_expect_tx(bar(a2::K_FULL + ks), 32768);
+        tma_load_3d(kdst, src.map_k, bar(a2::K_FULL + ks), 0, src.row, bh);
+        tma_load_3d(kdst + 16384, src.map_k, bar(a2::K_FULL + ks), 64, src.row, bh);
+        const int vs = j & 1;
+        if (j >= 2) ok = mbar_wait(bar(a2::V_EMPTY + vs), ((j - 2) >> 1) & 1, abort_flag, 26);
+        if (!ok) break;
+        const uint32_t vdst = base + kVOff + vs * 32768;
+        mbar_expect_tx(bar(a2::V_FULL + vs), 32768);
+        tma_load_3d(vdst, src.map_v, bar(a2::V_FULL + vs), 0, src.row, bh);
+        tma_load_3d(vdst + 16384, src.map_v, bar(a2::V_FULL + vs), 64, src.row, bh);
+      }
+      if (linear && ok) {
+        const uint32_t wbytes = static_cast<uint32_t>(Dp) * kD * 2;
+        const uint32_t slbytes = static_cast<uint32_t>(Dp) * kD * 4;
+        ok = mbar_wait(bar(a2::LAST_PV), 0, abort_flag, 2);
+        if (ok) {
+          mbar_expect_tx(bar(a2::TAIL_FULL), wbytes + slbytes);
+          bulk_load(base + kWOff, wq_img + static_cast<long long>(h) * Dp * kD, wbytes,
+                    bar(a2::TAIL_FULL));
+          bulk_load(base + kSLOff, P.SL + (static_cast<long long>(bh) * P.nchunks + t) * Dp * kD,
+                    slbytes, bar(a2::TAIL_FULL));
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ================================================= MMA issuer
+    if (lane == 0) {
+      const uint32_t id_qk = idesc(kBM, kBN, 1, false);
+      const uint32_t id_pv = idesc(kBM, kD, 1, true);
+      const int ntiles = has_b ? 2 : 1;
+      bool ok = mbar_wait(bar(a2::Q_FULL), 0, abort_flag, 4);
+      auto issue_s = [&](int tile, int j) {
+        const uint32_t kaddr = base + kKOff + (j % 3) * 32768;
+        const uint32_t qaddr = base + kQOff + tile * 32768;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_bf16(tmem + tile * 256, sdesc(qaddr + off, 16, 1024), sdesc(kaddr + off, 16, 1024),
+                   id_qk, kk > 0);
+        }
+        mma_commit(bar(a2::S_FULL + tile));
+      };
+      auto issue_pv = [&](int tile, int j) {
+        const uint32_t vaddr = base + kVOff + (j & 1) * 32768;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ts(tmem + tile * 256 + 128, tmem + tile * 256 + kk * 8,
+                      sdesc(vaddr + kk * 2048, 16384, 1024), id_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(bar(a2::PV_DONE + tile));
+      };
+      if (ok) ok = mbar_wait(bar(a2::K_FULL), 0, abort_flag, 5);
+      if (ok) {
+        tc_fence_after();
+        for (int tile = 0; tile < ntiles; ++tile) issue_s(tile, 0);
+        mma_commit(bar(a2::K_EMPTY));
+      }
+      for (int j = 0; j < nt && ok; ++j) {
+        const int vs = j & 1;
+        const bool more = j + 1 < nt;
+        ok = mbar_wait(bar(a2::V_FULL + vs), (j >> 1) & 1, abort_flag, 8);
+        if (ok && more)
+          ok = mbar_wait(bar(a2::K_FULL + (j + 1) % 3), ((j + 1) / 3) & 1, abort_flag, 5);
+        for (int tile = 0; tile < ntiles && ok; ++tile) {
+          ok = mbar_wait(bar(a2::P_FULL + tile), j & 1, abort_flag, 7);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(tile, j);                  // reads P(j) from this tile's S columns
+          if (more) issue_s(tile, j + 1);     // then overwrites them (in-order pipe)
+        }
+        if (!ok) break;
+        mma_commit(bar(a2::V_EMPTY + vs));
+        if (more) mma_commit(bar(a2::K_EMPTY + (j + 1) % 3));
+        if (j == nt - 1) mma_commit(bar(a2::LAST_PV));
+      }
+      if (linear && ok) {
+        ok = mbar_wait(bar(a2::TAIL_FULL), 0, abort_flag, 9);
+        if (ok) {
+          tc_fence_after();
+          const uint32_t id_phi = idesc(kBM, Dp, 1, false);
+          for (int tile = 0; tile < ntiles; ++tile)
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t qoff = tile * 32768 + (kk >> 2) * 16384 + (kk & 3) * 32;
+              const uint32_t woff = (kk >> 2) * (Dp * 128) + (kk & 3) * 32;
+              mma_bf16(tmem + tile * 256, sdesc(base + kQOff + qoff, 16, 1024),
+                       sdesc(base + kWOff + woff, 16, 1024), id_phi, kk > 0);
+            }
+          mma_commit(bar(a2::PHI_DONE));
+          const uint32_t id_rd = idesc(kBM, kD, 2, false);
+          for (int tile = 0; tile < ntiles && ok; ++tile) {
+            ok = mbar_wait(bar(a2::PHI_READY + tile), 0, abort_flag, 10);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t phi = base + (tile ? kPhiOff1 : kPhiOff0);
+            for (int kk = 0; kk < Dp / 8; ++kk) {
+              const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+              mma_tf32(tmem + tile * 256 + 128, sdesc(phi + off, 16, 1024),
+                       sdesc(base + kSLOff + off, 16, 1024), id_rd, 1u);
+            }
+          }
+          if (ok) mma_commit(bar(a2::READ_DONE));
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp < 8 && (warp < 4 || has_b)) {
+    // ================================================= softmax / epilogue
+    const int tile = warp >> 2;
+    const int r = tid & 127;                 // row within the tile == TMEM lane
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t s_col = tile * 256, o_col = s_col + 128;
+    const int nrows = nrows_t[tile];
+    float m_used = -INFINITY, m_max = -INFINITY, l = 0.f;
+    bool ok = true;
+    auto wait_all = [&](uint32_t b, uint32_t parity, uint32_t code) {
+      return __all_sync(0xffffffffu, mbar_wait(b, parity, abort_flag, code));
+    };
+    for (int j = 0; j < nt && ok; ++j) {
+      // S_FULL(j) also covers this tile's P.V of step j-1 (issued earlier).
+      ok = wait_all(bar(a2::S_FULL + tile), j & 1, 11);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t xr[128];
+      REHYAT_TMEM_LD32(lane_base + s_col + 0, (xr + 0));
+      REHYAT_TMEM_LD32(lane_base + s_col + 32, (xr + 32));
+      REHYAT_TMEM_LD32(lane_base + s_col + 64, (xr + 64));
+      REHYAT_TMEM_LD32(lane_base + s_col + 96, (xr + 96));
+      tmem_wait_ld();
+      const int nvalid = tile_src(j).nvalid;
+      if (nvalid < kBN) {
+#pragma unroll
+        for (int i = 0; i < 128; ++i)
+          if (i >= nvalid) xr[i] = __float_as_uint(-INFINITY);
+      }
+      float mx[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) mx[i] = __uint_as_float(xr[i]);
+#pragma unroll
+      for (int i = 16; i < 128; ++i) mx[i & 15] = fmaxf(mx[i & 15], __uint_as_float(xr[i]));
+#pragma unroll
+      for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+        for (int i = 0; i < w; ++i) mx[i] = fmaxf(mx[i], mx[i + w]);
+      m_max = fmaxf(m_max, mx[0] * P.scale_log2);
+      float alpha = 1.f;
+      const bool rescale = m_max > m_used + 8.f;
+      if (rescale) {
+        alpha = ex2(m_used - m_max);
+        m_used = m_max;
+      }
+      const float neg_m = -m_used;
+      float ls[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) ls[i] = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = ex2(fmaf(__uint_as_float(xr[32 * c + 2 * i]), P.scale_log2, neg_m));
+          const float p1 = ex2(fmaf(__uint_as_float(xr[32 * c + 2 * i + 1]), P.scale_log2, neg_m));
+          pk[i] = pack_bf16(p0, p1);
+          ls[i & 7] += p0 + p1;
+        }
+        REHYAT_TMEM_ST16(lane_base + s_col + c * 16, pk);
+      }
+      // After the P stores (S is dead by now): bring the earlier a^S to the
+      // new reference point; this tile's P.V of step j-1 is complete (covered
+      // by S_FULL(j)).  Warp-collective; rows that did not move use alpha = 1.
+      if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+        uint32_t o[32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          REHYAT_TMEM_LD32(lane_base + o_col + c * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          REHYAT_TMEM_ST32(lane_base + o_col + c * 32, o);
+        }
+      }
+      tmem_wait_st();
+      l = l * alpha + (((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7])));
+      if (tile == 0 && nvalid < kBN) {
+        // Zero the V rows past the last valid key (shared by both tiles;
+        // tile B's P.V is issued after tile A's P_FULL).
+        ok = wait_all(bar(a2::V_FULL + (j & 1)), (j >> 1) & 1, 13);
+        if (!ok) break;
+        if (r >= nvalid) {
+          const uint32_t vrow = base + kVOff + (j & 1) * 32768 + r * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            st_shared_v4(vrow + c * 16, 0, 0, 0, 0);
+            st_shared_v4(vrow + 16384 + c * 16, 0, 0, 0, 0);
+          }
+        }
+        fence_proxy_async();
+      }
+      tc_fence_before();
+      mbar_arrive(bar(a2::P_FULL + tile));
+    }
+    const float fscale = ex2(m_used - m_max);
+    const long long grow = static_cast<long long>(bh) * P.rows_per_bh + row0 + tile * kBM + r;
+    const bool dbg_split = P.dbg_aS != nullptr || P.dbg_aL != nullptr;
+    float nL = 0.f;
+    if (ok && linear) {
+      if (dbg_split) {
+        // a^S before the readout adds into O (debug export only).
+        ok = wait_all(bar(a2::LAST_PV), 0, 14);
+        if (ok) {
+          tc_fence_after();
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            REHYAT_TMEM_LD32(lane_base + o_col + c * 32, o);
+            tmem_wait_ld();
+            if (r < nrows && P.dbg_aS)
+              for (int i = 0; i < 32; ++i)
+                P.dbg_aS[grow * kD + c * 32 + i] = __uint_as_float(o[i]) * fscale;
+            if (r < nrows && P.dbg_aL)  // a^S for now; replaced by a^L below
+              for (int i = 0; i < 32; ++i)
+                P.dbg_aL[grow * kD + c * 32 + i] = __uint_as_float(o[i]) * fscale;
+          }
+        }
+      }
+      if (ok) ok = wait_all(bar(a2::PHI_DONE), 0, 14);
+      if (ok) {
+        tc_fence_after();
+        const float inv_f = 1.0f / fscale;
+        const float* zL = P.zL + (static_cast<long long>(bh) * P.nchunks + t) * Dp;
+        const uint32_t phi = base + (tile ? kPhiOff1 : kPhiOff0);
+        for (int c = 0; c < Dp / 32; ++c) {
+          uint32_t v[32];
+          REHYAT_TMEM_LD32(lane_base + s_col + c * 32, v);
+          tmem_wait_ld();
+          float ph[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int f = c * 32 + i;
+            const int part = f >= (Dp >> 1);
+            const float b = __ldg(P.bq + (h * 2 + part) * (Dp >> 1) + (f - part * (Dp >> 1)));
+            const float psi = __uint_as_float(v[i]) + b;
+            ph[i] = psi * psi;
+            nL = fmaf(ph[i], __ldg(zL + f), nL);
+            ph[i] *= inv_f;
+          }
+          const uint32_t rowaddr = phi + c * 16384 + r * 128;
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch)
+            st_shared_v4(rowaddr + ((ch ^ (r & 7)) << 4), __float_as_uint(ph[4 * ch]),
+                         __float_as_uint(ph[4 * ch + 1]), __float_as_uint(ph[4 * ch + 2]),
+                         __float_as_uint(ph[4 * ch + 3]));
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        mbar_arrive(bar(a2::PHI_READY + tile));
+        ok = wait_all(bar(a2::READ_DONE), 0, 15);
+      }
+    } else if (ok) {
+      ok = wait_all(bar(a2::LAST_PV), 0, 15);
+    }
+    if (ok) {
+      tc_fence_after();
+      const float nS = l * fscale;
+      const float den = nS + nL;
+      for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        REHYAT_TMEM_LD32(lane_base + o_col + c * 32, o);
+        tmem_wait_ld();
+        if (r < nrows) {
+          float yv[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float num = __uint_as_float(o[i]) * fscale;  // a^S + a^L
+            yv[i] = __fdiv_rn(num, den);
+            if (P.dbg_aL) {
+              float* d = P.dbg_aL + grow * kD + c * 32 + i;
+              *d = linear ? num - *d : 0.f;
+            }
+            if (P.dbg_aS && !linear) P.dbg_aS[grow * kD + c * 32 + i] = num;
+          }
+          if (P.out_bf16) {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(P.y) + grow * kD +
+                                                  c * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_uint4(pack_bf16(yv[8 * i], yv[8 * i + 1]),
+                                  pack_bf16(yv[8 * i + 2], yv[8 * i + 3]),
+                                  pack_bf16(yv[8 * i + 4], yv[8 * i + 5]),
+                                  pack_bf16(yv[8 * i + 6], yv[8 * i + 7]));
+          } else {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(P.y) + grow * kD + c * 32);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(yv[4 * i], yv[4 * i + 1], yv[4 * i + 2], yv[4 * i + 3]);
+          }
+        }
+      }
+      if (r < nrows) {
+        if (P.dbg_nS) P.dbg_nS[grow] = nS;
+        if (P.dbg_nL) P.dbg_nL[grow] = nL;
+        if (P.dbg_c) P.dbg_c[grow] = m_max * 0.69314718055994530942f;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+  }
+}
+
+// ===========================================================================
 // Per-slice linear state on tensor cores ("Key designs 1 and 4": the linear
 // branch's sum of phi_k(k) v^T and of phi_k(k)):
 //   P_s = phi_k(K_s)^T V_s  ([Dp][D] fp32),  z_s = sum_j phi_k(k_j)  ([Dp]).
@@ -854,13 +1310,24 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s) {
       maps.rv = maps.v;
     }
   }
-  cudaError_t e = cudaFuncSetAttribute(tc_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(kSmemBytes));
-  if (e != cudaSuccess) return e;
   const int qrows_max = p.seen ? p.nq_slices * p.HW : (p.Tc < p.T ? p.Tc : p.T) * p.HW;
-  dim3 grid((qrows_max + kBM - 1) / kBM, p.nchunks, p.BH);
-  tc_attn_kernel<<<grid, kThreads, kSmemBytes, s>>>(
-      maps, p, static_cast<const __nv_bfloat16*>(p.wq_img));
+  const bool two_tiles = !p.one_tile && (p.full_softmax || p.Dp <= 128);
+  cudaError_t e;
+  if (two_tiles) {
+    e = cudaFuncSetAttribute(tc_attn2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(a2::kSmemBytes));
+    if (e != cudaSuccess) return e;
+    dim3 grid((qrows_max + 2 * kBM - 1) / (2 * kBM), p.nchunks, p.BH);
+    tc_attn2_kernel<<<grid, a2::kThreads, a2::kSmemBytes, s>>>(
+        maps, p, static_cast<const __nv_bfloat16*>(p.wq_img));
+  } else {
+    e = cudaFuncSetAttribute(tc_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmemBytes));
+    if (e != cudaSuccess) return e;
+    dim3 grid((qrows_max + kBM - 1) / kBM, p.nchunks, p.BH);
+    tc_attn_kernel<<<grid, kThreads, kSmemBytes, s>>>(
+        maps, p, static_cast<const __nv_bfloat16*>(p.wq_img));
+  }
   return cudaGetLastError();
 }
 

@@ -23,11 +23,12 @@ def device_tensors(p, device="cuda"):
                 bq=t(p.bq, torch.float32), Wk=t(p.Wk, torch.float32), bk=t(p.bk, torch.float32))
 
 
-def run_fwd(p, *, debug=False, force_simt=False, dev=None, out_dtype=None):
+def run_fwd(p, *, debug=False, force_simt=False, one_tile=False, dev=None, out_dtype=None):
     dev = device_tensors(p) if dev is None else dev
     res = rh.hybrid_attn(dev["q"], dev["k"], dev["v"], dev["Wq"], dev["bq"], dev["Wk"], dev["bk"],
                          T=p.T, Hs=p.Hs, Ws=p.Ws, Tc=p.Tc, To=p.To, causal=p.causal,
-                         debug=debug, force_simt=force_simt, out_dtype=out_dtype)
+                         debug=debug, force_simt=force_simt, one_tile=one_tile,
+                         out_dtype=out_dtype)
     torch.cuda.synchronize()
     if debug:
         y, parts = res

@@ -55,13 +55,17 @@ SMALL = [
 @pytest.mark.parametrize("shape", SMALL, ids=lambda s: "x".join(map(str, s)))
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
-@pytest.mark.parametrize("force_simt", [False, True], ids=["default", "simt"])
-def test_small_shapes(shape, causal, dtype, force_simt):
+@pytest.mark.parametrize("path", ["default", "simt", "one_tile"])
+def test_small_shapes(shape, causal, dtype, path):
+    """default = two-query-tile tensor-core kernel (bf16, D=128, D'<=128),
+    one_tile = the one-tile tensor-core kernel, simt = fp32 CUDA cores."""
     B, h, T, Hs, Ws, D, Dp, Tc, To = shape
+    if path == "one_tile" and dtype == "f32":
+        pytest.skip("tensor-core kernels take bf16 inputs")
     p = make_problem(batch=B, heads=h, T=T, Hs=Hs, Ws=Ws, D=D, Dp=Dp, Tc=Tc, To=To,
                      causal=causal, dtype=dtype, dist="scaled", seed=100 + sum(shape))
     ref_y, ref_p = orc.run_problem(p)
-    y, parts = run_fwd(p, debug=True, force_simt=force_simt)
+    y, parts = run_fwd(p, debug=True, force_simt=path == "simt", one_tile=path == "one_tile")
     assert_close_y(y, ref_y, dtype)
     assert_close_partials(parts, ref_p, dtype)
 
