@@ -274,12 +274,118 @@ def measure_streaming(rh, dev, flush, stream):
     free1 = torch.cuda.mem_get_info(dev)[0]
     ms = [e0.elapsed_time(e1) for e0, e1 in evs]
     steady = sorted(ms[2:])[len(ms[2:]) // 2]
+    y_eager = out.clone()
+
+    # The same 27 steps as one captured step replayed per chunk (the chunk is
+    # copied into fixed input buffers first; the copy is inside the timing).
+    st.reset()
+    qb, kb, vb = (torch.empty_like(x) for x in chunks[0])
+    outg = torch.empty_like(out)
+    graph = st.capture_step(qb, kb, vb, outg)
+    gevs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in chunks]
+    for (e0, e1), c in zip(gevs, chunks):
+        e0.record(stream)
+        qb.copy_(c[0])
+        kb.copy_(c[1])
+        vb.copy_(c[2])
+        graph.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    gms = [e0.elapsed_time(e1) for e0, e1 in gevs]
+    gsteady = sorted(gms[2:])[len(gms[2:]) // 2]
+    same = bool(torch.equal(outg, y_eager))
+    del graph
     return {"workload": "81 slices of 30x52, 12 heads, D=D'=128, T_c=3, T_o=1, bf16, "
                         "27 rehyat_chunk_step calls (inputs from a seeded torch generator)",
             "steps": len(ms), "ms_per_step_median_steady": steady,
             "ms_first_steps": ms[:3], "tokens_per_s_steady": rows / (steady / 1e3),
+            "graph_ms_per_step_median_steady": gsteady,
+            "graph_tokens_per_s_steady": rows / (gsteady / 1e3),
+            "graph_last_chunk_bitwise_equal_to_eager": same,
             "free_bytes_before": free0, "free_bytes_after": free1,
             "device_memory_constant": free0 == free1}
+
+
+def run_sweep(args):
+    """T_c in {1,2,3,5,7} x T_o in {0,1,2} x D' in {64,128,256} x {bidirectional,
+    causal} on the 21x30x52 latent (batch 2, 12 heads, D = 128, bf16), q and k
+    low-rank (rank 8) plus N(0, 0.3^2) noise, v ~ N(0,1), from a seeded torch
+    generator.  One JSON line per point: step time, tokens/s and the
+    attention kernel's fraction of the measured bf16 peak."""
+    import torch
+    import linear_attention_video_chunked_b200 as rh
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    g = torch.Generator(device=dev).manual_seed(4)
+    B, H, T, Hs, Ws, D = 2, 12, 21, 30, 52, 128
+    HW, N = Hs * Ws, T * Hs * Ws
+    G = torch.randn(H, 8, D, generator=g, device=dev) / math.sqrt(8.0)
+
+    def lowrank():
+        u = torch.randn(B, H, N, 8, generator=g, device=dev)
+        x = torch.einsum("bhnr,hrd->bhnd", u, G)
+        return (x + 0.3 * torch.randn(B, H, N, D, generator=g, device=dev)).to(torch.bfloat16)
+
+    q, k = lowrank(), lowrank()
+    v = torch.randn(B, H, N, D, generator=g, device=dev).to(torch.bfloat16)
+    y = torch.empty(B, H, N, D, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    peaks = load_peaks()
+    stream = torch.cuda.current_stream()
+    for Dp in (64, 128, 256):
+        Wq, Wk = (0.1 * torch.randn(H, 2, D, Dp // 2, generator=g, device=dev) for _ in range(2))
+        bq, bk = (0.1 * torch.randn(H, 2, Dp // 2, generator=g, device=dev) for _ in range(2))
+        phi = rh.RehyatPhi(Wq.data_ptr(), bq.data_ptr(), Wk.data_ptr(), bk.data_ptr())
+        for causal in (0, 1):
+            for Tc in (1, 2, 3, 5, 7):
+                for To in (0, 1, 2):
+                    p = rh.make_params(batch=B, heads=H, T=T, Hs=Hs, Ws=Ws, D=D, Dp=Dp, Tc=Tc,
+                                       To=To, causal=causal, in_dtype=rh.BF16, out_dtype=rh.F32)
+                    nbytes = rh.rehyat_workspace_bytes(p)
+                    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+
+                    def call(evs=None):
+                        if evs:
+                            evs[0].record(stream)
+                        rh.rehyat_fwd_state(p, k.data_ptr(), v.data_ptr(), phi, ws.data_ptr(),
+                                            nbytes, stream.cuda_stream)
+                        if evs:
+                            evs[1].record(stream)
+                        st = rh.rehyat_fwd_attn(p, q.data_ptr(), k.data_ptr(), v.data_ptr(), phi,
+                                                y.data_ptr(), ws.data_ptr(), nbytes, None,
+                                                stream.cuda_stream)
+                        if st:
+                            raise rh.RehyatError(st, "rehyat_fwd_attn")
+                        if evs:
+                            evs[2].record(stream)
+
+                    for _ in range(3):
+                        call()
+                    times = []
+                    for _ in range(max(3, args.steps // 6)):
+                        flush.zero_()
+                        evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+                        call(evs)
+                        torch.cuda.synchronize()
+                        times.append((evs[0].elapsed_time(evs[2]), evs[1].elapsed_time(evs[2])))
+                    step_ms = sum(t[0] for t in times) / len(times)
+                    attn_ms = sum(t[1] for t in times) / len(times)
+                    w = algorithmic_work(B, H, T, HW, D, Dp, Tc, To, causal)
+                    attn_tf = w["attn_flops"] / (attn_ms / 1e3) / 1e12
+                    print(json.dumps({
+                        "sweep": "21x30x52", "Tc": Tc, "To": To, "Dp": Dp,
+                        "form": "causal" if causal else "bidirectional",
+                        "attn_kernel": "tensor-core two-tile" if rh.rehyat_attn_path(p) == 1 and Dp <= 128
+                        else ("tensor-core one-tile" if rh.rehyat_attn_path(p) == 1 else "CUDA-core"),
+                        "ms_per_step": step_ms, "tokens_per_s": B * N / (step_ms / 1e3),
+                        "attn_ms": attn_ms, "attn_tflops": attn_tf,
+                        "attn_frac_bf16_peak": attn_tf / peaks["bf16_tflops"],
+                        "total_tflop": w["total_flops"] / 1e12,
+                        "full_softmax_over_hybrid_flops": w["full_softmax_flops"] / w["total_flops"],
+                    }), flush=True)
+                    del ws
+    return 0
 
 
 # ------------------------------------------------------------ multi-rank
@@ -528,11 +634,15 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of fp64 oracle work for the CPU baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="T_c/T_o/D'/form sweep on the 21x30x52 latent, one JSON line per point")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the full-softmax comparator and the streaming measurement")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     world, rank, local = dist_setup()
+    if args.sweep:
+        return run_sweep(args) if rank == 0 else 0
     if args.impl == "reference":
         return run_reference(args, world, rank)
     return run_gpu(args, world, rank, local)

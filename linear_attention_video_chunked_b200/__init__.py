@@ -77,6 +77,10 @@ _LIB = None
 
 
 def lib_path() -> str:
+    """librehyat.so next to this file, or the file named by REHYAT_LIBRARY."""
+    override = os.environ.get("REHYAT_LIBRARY")
+    if override:
+        return override
     return os.path.join(os.path.dirname(os.path.abspath(__file__)), "librehyat.so")
 
 
@@ -347,3 +351,25 @@ class StreamingState:
 
     def restore(self, saved):
         self.state.copy_(saved)
+
+    def capture_step(self, q, k, v, out):
+        """Record one step on fixed buffers q, k, v, out as a CUDA graph.
+
+        The slice counter lives in the state on the device, so the same graph
+        advances the recurrence each time it is replayed: copy the next chunk
+        into q, k, v, then ``graph.replay()``; the outputs land in ``out``.
+        The state is left as it was before the call."""
+        torch = _torch()
+        saved = self.snapshot()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):  # warm-up launch outside the capture
+            self.step(q, k, v, out=out)
+        torch.cuda.current_stream().wait_stream(side)
+        self.restore(saved)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            self.step(q, k, v, out=out)
+        torch.cuda.synchronize()
+        self.restore(saved)
+        return graph

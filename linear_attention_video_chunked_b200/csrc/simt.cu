@@ -332,23 +332,40 @@ __global__ void scan_kernel(const float* __restrict__ P, const float* __restrict
   } else {
     return;
   }
+  // Slices are read in batches of 8 independent loads (the walk over slices
+  // is otherwise one dependent load at a time), then folded in order; chunk
+  // t receives the prefix when it reaches its window start w_t and, in the
+  // bidirectional form, the suffix from its end end_t on.
+  constexpr int kBatch = 8;
+  float v[kBatch];
   float pre = 0.f;
-  int s = 0;
-  for (int t = 0; t < nchunks; ++t) {
-    const int w = max(t * Tc - To, 0);
-    for (; s < w; ++s) pre += src[s * stride];
-    dst[t * stride] = pre;
+  int tp = 0;
+  while (tp < nchunks && max(tp * Tc - To, 0) == 0) dst[static_cast<long long>(tp++) * stride] = 0.f;
+  for (int s0 = 0; s0 < T && tp < nchunks; s0 += kBatch) {
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i)
+      v[i] = s0 + i < T ? src[static_cast<long long>(s0 + i) * stride] : 0.f;
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      pre += v[i];  // = sum over slices < s0 + i + 1
+      while (tp < nchunks && max(tp * Tc - To, 0) == s0 + i + 1)
+        dst[static_cast<long long>(tp++) * stride] = pre;
+    }
   }
   if (!causal) {
     float suf = 0.f;
-    s = T;
-    for (int t = nchunks - 1; t >= 0; --t) {
-      const int end = min(T, (t + 1) * Tc);
-      while (s > end) {
-        --s;
-        suf += src[s * stride];
+    int ts = nchunks - 1;
+    while (ts >= 0 && min(T, (ts + 1) * Tc) >= T) --ts;  // nothing after the last chunk
+    for (int s1 = T; s1 > 0 && ts >= 0; s1 -= kBatch) {
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i)
+        v[i] = s1 - 1 - i >= 0 ? src[static_cast<long long>(s1 - 1 - i) * stride] : 0.f;
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) {
+        suf += v[i];  // = sum over slices >= s1 - 1 - i
+        while (ts >= 0 && min(T, (ts + 1) * Tc) == s1 - 1 - i)
+          dst[static_cast<long long>(ts--) * stride] += suf;
       }
-      dst[t * stride] += suf;
     }
   }
 }
@@ -386,6 +403,8 @@ __global__ void state_add_kernel(const float* __restrict__ P, const float* __res
 
 // Copy chunk slices that stay in the window into their ring slots.
 // grid (nq_slices, BH); 16-byte vectors.
+constexpr int kRingBlocksPerSlice = 16;
+
 __global__ void ring_update_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
                                    uint4* __restrict__ rk, uint4* __restrict__ rv,
                                    const long long* __restrict__ seen, long long slice_vecs,
@@ -393,14 +412,17 @@ __global__ void ring_update_kernel(const uint4* __restrict__ k, const uint4* __r
   const long long sn = *seen;
   const long long after = sn + nq;
   const long long keep = after < To ? after : To;
-  const long long g = sn + blockIdx.x;          // global slice of this chunk slice
-  if (g < after - keep) return;                 // leaves the window right away
+  const int slice = blockIdx.x / kRingBlocksPerSlice;  // chunk slice of this block
+  const int part = blockIdx.x % kRingBlocksPerSlice;
+  const long long g = sn + slice;                      // its global slice index
+  if (g < after - keep) return;                        // leaves the window right away
   const int bh = blockIdx.y;
-  const uint4* ks = k + (static_cast<long long>(bh) * nq + blockIdx.x) * slice_vecs;
-  const uint4* vs = v + (static_cast<long long>(bh) * nq + blockIdx.x) * slice_vecs;
+  const uint4* ks = k + (static_cast<long long>(bh) * nq + slice) * slice_vecs;
+  const uint4* vs = v + (static_cast<long long>(bh) * nq + slice) * slice_vecs;
   uint4* kd = rk + (static_cast<long long>(bh) * To + (g % To)) * slice_vecs;
   uint4* vd = rv + (static_cast<long long>(bh) * To + (g % To)) * slice_vecs;
-  for (long long i = threadIdx.x; i < slice_vecs; i += blockDim.x) {
+  for (long long i = static_cast<long long>(part) * blockDim.x + threadIdx.x; i < slice_vecs;
+       i += static_cast<long long>(blockDim.x) * kRingBlocksPerSlice) {
     kd[i] = ks[i];
     vd[i] = vs[i];
   }
@@ -492,7 +514,7 @@ cudaError_t launch_ring_update(const void* k, const void* v, void* rk, void* rv,
                                int nq_slices, int elem_bytes, cudaStream_t s) {
   if (To == 0) return cudaSuccess;
   const long long slice_vecs = static_cast<long long>(HW) * D * elem_bytes / 16;
-  dim3 grid(nq_slices, BH);
+  dim3 grid(nq_slices * kRingBlocksPerSlice, BH);
   ring_update_kernel<<<grid, 256, 0, s>>>(
       static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint4*>(rk),
       static_cast<uint4*>(rv), seen, slice_vecs, To, nq_slices);

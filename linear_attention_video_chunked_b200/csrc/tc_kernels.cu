@@ -518,6 +518,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ===========================================================================
 namespace a2 {
 constexpr int kThreads = 320;
+// One fp32 pair in kPolyEvery takes the FMA-pipe exp2 (0 = all on MUFU).
+// Measured on the 21x30x52 workload (attention ms): all on MUFU 2.85,
+// one in 8 pairs 2.97, one in 4 3.01, one in 2 3.05 -- the softmax is
+// issue/latency bound here, not MUFU bound, so MUFU only by default.
+#ifndef REHYAT_POLY_EVERY
+#define REHYAT_POLY_EVERY 0
+#endif
+constexpr int kPolyEvery = REHYAT_POLY_EVERY;
 constexpr uint32_t kQOff = 0;                      // Q_A, Q_B
 constexpr uint32_t kKOff = 65536;                  // K ring, 3 x 32 KB
 constexpr uint32_t kVOff = kKOff + 3 * 32768;      // V ring, 2 x 32 KB
@@ -547,6 +555,7 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
   using a2::kPhiOff1;
   using a2::kTmemSlot;
   using a2::kAbortSlot;
+  using a2::kPolyEvery;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -765,23 +774,26 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
       ok = wait_all(bar(a2::S_FULL + tile), j & 1, 11);
       if (!ok) break;
       tc_fence_after();
-      uint32_t xr[128];
-      REHYAT_TMEM_LD32(lane_base + s_col + 0, (xr + 0));
-      REHYAT_TMEM_LD32(lane_base + s_col + 32, (xr + 32));
-      REHYAT_TMEM_LD32(lane_base + s_col + 64, (xr + 64));
-      REHYAT_TMEM_LD32(lane_base + s_col + 96, (xr + 96));
-      tmem_wait_ld();
       const int nvalid = tile_src(j).nvalid;
-      if (nvalid < kBN) {
-#pragma unroll
-        for (int i = 0; i < 128; ++i)
-          if (i >= nvalid) xr[i] = __float_as_uint(-INFINITY);
-      }
+      // Pass 1: row max over S, streamed from TMEM 64 columns at a time (S
+      // never sits whole in registers, which would spill).
       float mx[16];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) mx[i] = __uint_as_float(xr[i]);
+      for (int i = 0; i < 16; ++i) mx[i] = -INFINITY;
 #pragma unroll
-      for (int i = 16; i < 128; ++i) mx[i & 15] = fmaxf(mx[i & 15], __uint_as_float(xr[i]));
+      for (int h2 = 0; h2 < 2; ++h2) {
+        uint32_t xr[64];
+        REHYAT_TMEM_LD32(lane_base + s_col + 64 * h2, xr);
+        REHYAT_TMEM_LD32(lane_base + s_col + 64 * h2 + 32, (xr + 32));
+        tmem_wait_ld();
+        if (nvalid < kBN) {  // ragged tile (warp-uniform): keys past the end
+#pragma unroll
+          for (int i = 0; i < 64; ++i)
+            if (64 * h2 + i >= nvalid) xr[i] = __float_as_uint(-INFINITY);
+        }
+#pragma unroll
+        for (int i = 0; i < 64; ++i) mx[i & 15] = fmaxf(mx[i & 15], __uint_as_float(xr[i]));
+      }
 #pragma unroll
       for (int w = 8; w >= 1; w >>= 1)
 #pragma unroll
@@ -793,22 +805,49 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
         alpha = ex2(m_used - m_max);
         m_used = m_max;
       }
-      const float neg_m = -m_used;
-      float ls[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) ls[i] = 0.f;
+      // p = 2^(s * scale * log2(e) - m_used) on packed fp32 pairs; one pair
+      // in kPolyEvery goes through the FMA-pipe exp2 (exp2_poly2) instead of
+      // MUFU, which at D = 128 is as busy as the tensor core.
+      const uint64_t scale2 = f2_pack(P.scale_log2, P.scale_log2);
+      const uint64_t negm2 = f2_pack(-m_used, -m_used);
+      uint64_t ls2[4] = {0, 0, 0, 0};
+      // Pass 2: re-read S 32 columns at a time and write P (bf16 pairs) over
+      // the S columns already consumed: P piece c lands in [16c, 16c + 16).
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
+        uint32_t xr[32];
+        REHYAT_TMEM_LD32(lane_base + s_col + 32 * c, xr);
+        tmem_wait_ld();
+        if (nvalid < kBN) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (32 * c + i >= nvalid) xr[i] = __float_as_uint(-INFINITY);
+        }
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float p0 = ex2(fmaf(__uint_as_float(xr[32 * c + 2 * i]), P.scale_log2, neg_m));
-          const float p1 = ex2(fmaf(__uint_as_float(xr[32 * c + 2 * i + 1]), P.scale_log2, neg_m));
+          const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(xr[2 * i]),
+                                             __uint_as_float(xr[2 * i + 1])),
+                                     scale2, negm2);
+          uint64_t p2;
+          if (kPolyEvery > 0 && (i % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
+            p2 = exp2_poly2(x2);
+          } else {
+            float a0, a1;
+            f2_unpack(x2, a0, a1);
+            p2 = f2_pack(ex2(a0), ex2(a1));
+          }
+          float p0, p1;
+          f2_unpack(p2, p0, p1);
           pk[i] = pack_bf16(p0, p1);
-          ls[i & 7] += p0 + p1;
+          ls2[i & 3] = f2_add(ls2[i & 3], p2);
         }
         REHYAT_TMEM_ST16(lane_base + s_col + c * 16, pk);
       }
+      float ls[8];
+      f2_unpack(f2_add(ls2[0], ls2[1]), ls[0], ls[1]);
+      f2_unpack(f2_add(ls2[2], ls2[3]), ls[2], ls[3]);
+      ls[4] = ls[5] = ls[6] = ls[7] = 0.f;
       // After the P stores (S is dead by now): bring the earlier a^S to the
       // new reference point; this tile's P.V of step j-1 is complete (covered
       // by S_FULL(j)).  Warp-collective; rows that did not move use alpha = 1.
@@ -932,10 +971,17 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
                                   pack_bf16(yv[8 * i + 4], yv[8 * i + 5]),
                                   pack_bf16(yv[8 * i + 6], yv[8 * i + 7]));
           } else {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(P.y) + grow * kD + c * 32);
+            // fp32 rows go through shared memory (the K ring is free now:
+            // tile A at kKOff, tile B 64 KB above), 16-byte chunk cc of row
+            // r at position cc ^ (r & 7) so neither side has bank conflicts.
+            const uint32_t srow = base + kKOff + tile * 65536 + r * 512;
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              dst[i] = make_float4(yv[4 * i], yv[4 * i + 1], yv[4 * i + 2], yv[4 * i + 3]);
+            for (int i = 0; i < 8; ++i) {
+              const uint32_t cc = c * 8 + i;
+              st_shared_v4(srow + ((cc ^ (r & 7)) << 4), __float_as_uint(yv[4 * i]),
+                           __float_as_uint(yv[4 * i + 1]), __float_as_uint(yv[4 * i + 2]),
+                           __float_as_uint(yv[4 * i + 3]));
+            }
           }
         }
       }
@@ -943,6 +989,22 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
         if (P.dbg_nS) P.dbg_nS[grow] = nS;
         if (P.dbg_nL) P.dbg_nL[grow] = nL;
         if (P.dbg_c) P.dbg_c[grow] = m_max * 0.69314718055994530942f;
+      }
+    }
+    // Every thread of this warpgroup gets here (aborted or not), so the
+    // named barrier cannot hang.  Then each warp writes whole 512-byte rows
+    // of the staged fp32 output: lane l stores chunk l (coalesced).
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + tile), "r"(kSoftmaxThreads) : "memory");
+    if (ok && !P.out_bf16) {
+      const long long grow0 = static_cast<long long>(bh) * P.rows_per_bh + row0 + tile * kBM;
+      for (int rr = warp & 3; rr < nrows; rr += 4) {
+        const uint32_t src = base + kKOff + tile * 65536 + rr * 512 + ((lane ^ (rr & 7)) << 4);
+        uint32_t a0, a1, a2, a3;
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(a0), "=r"(a1), "=r"(a2), "=r"(a3)
+                     : "r"(src));
+        reinterpret_cast<uint4*>(static_cast<float*>(P.y) + (grow0 + rr) * kD)[lane] =
+            make_uint4(a0, a1, a2, a3);
       }
     }
   }
@@ -1225,6 +1287,302 @@ __global__ void __launch_bounds__(st::kThreads, 1)
   }
 }
 
+// ===========================================================================
+// Persistent per-slice state kernel (full mode): the same sums as
+// tc_state_kernel, with each CTA streaming a contiguous run of (b*h, slice)
+// items through one K/V pipeline that does not drain between slices.
+//   warps 0-3  convert: psi (TMEM) -> phi = (psi + b)^2 -> bf16 phi^T tile;
+//   warps 4-7  epilogue: drain the finished slice's P and z from TMEM;
+//   warp 8     TMA (K, V tiles; the W_k image when the head changes);
+//   warp 9     MMA (psi = K W_k, P += phi^T V, z += phi^T 1) and TMEM owner.
+// TMEM: psi [0,128), P accumulators [128,256) [256,384) (alternating per
+// slice), z accumulators [384,400) [400,416).  D' in {64, 128}.
+// ===========================================================================
+namespace sp {
+constexpr int kThreads = 320;
+constexpr uint32_t kKOff = 0;          // K ring, 2 x 32 KB
+constexpr uint32_t kVOff = 65536;      // V ring, 2 x 32 KB
+constexpr uint32_t kWOff = 131072;     // W_k image of the current head (<= 32 KB)
+constexpr uint32_t kPhiOff = 163840;   // phi^T tile, 2 boxes x 16 KB
+constexpr uint32_t kOnesOff = 196608;  // all-ones B operand for z (4 KB)
+constexpr uint32_t kBiasOff = 200704;  // b_k of the current head (<= 512 B)
+constexpr uint32_t kBarOff = 201216;
+enum { K_FULL = 0, V_FULL = 2, K_EMPTY = 4, V_EMPTY = 6, PSI_FULL = 8, PSI_FREE = 9,
+       PHI_FULL = 10, PHI_EMPTY = 11, ACC_DONE = 12, P_FREE = 14, W_FULL = 16, W_FREE = 17,
+       NBAR = 18 };
+constexpr uint32_t kTmemSlot = kBarOff + 8 * NBAR;
+constexpr uint32_t kAbortSlot = kTmemSlot + 4;
+constexpr uint32_t kSmemBytes = kBarOff + 256 + 1024;
+constexpr uint32_t kColPsi = 0, kColP = 128, kColZ = 384;
+}  // namespace sp
+
+__global__ void __launch_bounds__(sp::kThreads, 1)
+    tc_state_persistent_kernel(const __grid_constant__ StMaps maps, const PartialParams P,
+                               const __nv_bfloat16* __restrict__ wk_img, int items_per_cta) {
+  // Local names shadow the attention kernel's constants of the same names.
+  constexpr int kThreads = sp::kThreads;
+  constexpr uint32_t kKOff = sp::kKOff, kVOff = sp::kVOff, kWOff = sp::kWOff;
+  constexpr uint32_t kPhiOff = sp::kPhiOff, kOnesOff = sp::kOnesOff, kBiasOff = sp::kBiasOff;
+  constexpr uint32_t kColPsi = sp::kColPsi, kColP = sp::kColP, kColZ = sp::kColZ;
+  using sp::K_FULL;
+  using sp::V_FULL;
+  using sp::K_EMPTY;
+  using sp::V_EMPTY;
+  using sp::PSI_FULL;
+  using sp::PSI_FREE;
+  using sp::PHI_FULL;
+  using sp::PHI_EMPTY;
+  using sp::ACC_DONE;
+  using sp::P_FREE;
+  using sp::W_FULL;
+  using sp::W_FREE;
+  using sp::NBAR;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* sbase = smem_raw + (base - raw);
+  auto bar = [&](int i) { return base + sp::kBarOff + 8u * i; };
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(sbase + sp::kAbortSlot);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int Dp = P.Dp, HW = P.HW, T = P.nslots;
+  const int total = P.BH * T;
+  const int it0 = blockIdx.x * items_per_cta;
+  const int it1 = min(total, it0 + items_per_cta);
+  if (it0 >= it1) return;
+  const int nitems = it1 - it0;
+  const int nt = (HW + 127) / 128;
+  const int TT = nitems * nt;  // tiles of this CTA
+  auto head_of = [&](int il) { return ((it0 + il) / T) % P.heads; };
+
+  if (tid == 0) {
+    for (int i = 0; i < NBAR; ++i) {
+      const bool by_group = i == PSI_FREE || i == PHI_FULL || i == P_FREE || i == P_FREE + 1;
+      mbar_init(bar(i), by_group ? 128 : 1);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  for (int i = tid; i < 1024; i += kThreads)
+    reinterpret_cast<uint32_t*>(sbase + kOnesOff)[i] = 0x3F803F80u;
+  fence_proxy_async();
+  if (warp == 9) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     base + sp::kTmemSlot),
+                 "r"(512));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sbase + sp::kTmemSlot);
+  const uint32_t wbytes = static_cast<uint32_t>(Dp) * 128 * 2;
+
+  if (warp == 8) {
+    // ================================================= TMA producer
+    if (lane == 0) {
+      bool ok = true;
+      int wloads = 0;
+      for (int il = 0; il < nitems && ok; ++il) {
+        const int item = it0 + il, bh = item / T, slice = item % T, h = bh % P.heads;
+        if (il == 0 || h != head_of(il - 1)) {
+          if (il > 0) ok = mbar_wait(bar(W_FREE), (wloads - 1) & 1, abort_flag, 27);
+          if (!ok) break;
+          mbar_expect_tx(bar(W_FULL), wbytes);
+          bulk_load(base + kWOff, wk_img + static_cast<long long>(h) * Dp * 128, wbytes,
+                    bar(W_FULL));
+          ++wloads;
+        }
+        for (int j = 0; j < nt && ok; ++j) {
+          const int gt = il * nt + j, s = gt & 1;
+          const int row = slice * HW + j * 128;
+          if (gt >= 2) ok = mbar_wait(bar(K_EMPTY + s), ((gt - 2) >> 1) & 1, abort_flag, 28);
+          if (!ok) break;
+          mbar_expect_tx(bar(K_FULL + s), 32768);
+          tma_load_3d(base + kKOff + s * 32768, &maps.k, bar(K_FULL + s), 0, row, bh);
+          tma_load_3d(base + kKOff + s * 32768 + 16384, &maps.k, bar(K_FULL + s), 64, row, bh);
+          if (gt >= 2) ok = mbar_wait(bar(V_EMPTY + s), ((gt - 2) >> 1) & 1, abort_flag, 29);
+          if (!ok) break;
+          mbar_expect_tx(bar(V_FULL + s), 32768);
+          tma_load_3d(base + kVOff + s * 32768, &maps.v, bar(V_FULL + s), 0, row, bh);
+          tma_load_3d(base + kVOff + s * 32768 + 16384, &maps.v, bar(V_FULL + s), 64, row, bh);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ================================================= MMA issuer
+    if (lane == 0) {
+      const uint32_t id_psi = idesc_ab(128, Dp, 1, false, false);
+      const uint32_t id_st = idesc_ab(128, 128, 1, true, true);
+      const uint32_t id_z = idesc_ab(128, 16, 1, true, false);
+      bool ok = true;
+      int wwaits = 0;
+      // psi for global tile gt (item il, tile j): waits for its K tile, for
+      // the converter to have read psi(gt - 1), and for the head's W_k.
+      auto issue_psi = [&](int gt) -> bool {
+        const int il = gt / nt, s = gt & 1;
+        if (gt % nt == 0 && (il == 0 || head_of(il) != head_of(il - 1))) {
+          if (il > 0) mma_commit(bar(W_FREE));  // tracks every earlier MMA
+          if (!mbar_wait(bar(W_FULL), wwaits & 1, abort_flag, 30)) return false;
+          ++wwaits;
+        }
+        if (!mbar_wait(bar(K_FULL + s), (gt >> 1) & 1, abort_flag, 31)) return false;
+        if (gt >= 1 && !mbar_wait(bar(PSI_FREE), (gt - 1) & 1, abort_flag, 32)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
+          const uint32_t woff = (kk >> 2) * (Dp * 128) + (kk & 3) * 32;
+          mma_bf16(tmem + kColPsi, sdesc(base + kKOff + s * 32768 + koff, 16, 1024),
+                   sdesc(base + kWOff + woff, 16, 1024), id_psi, kk > 0);
+        }
+        mma_commit(bar(PSI_FULL));
+        mma_commit(bar(K_EMPTY + s));
+        return true;
+      };
+      ok = issue_psi(0);
+      for (int gt = 0; gt < TT && ok; ++gt) {
+        const int il = gt / nt, j = gt % nt, s = gt & 1, pb = il & 1;
+        if (gt + 1 < TT) ok = issue_psi(gt + 1);
+        if (!ok) break;
+        if (j == 0 && il >= 2) ok = mbar_wait(bar(P_FREE + pb), ((il - 2) >> 1) & 1, abort_flag, 33);
+        if (ok) ok = mbar_wait(bar(PHI_FULL), gt & 1, abort_flag, 34) &&
+                     mbar_wait(bar(V_FULL + s), (gt >> 1) & 1, abort_flag, 35);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t a = sdesc(base + kPhiOff + kk * 2048, 16384, 1024);
+          const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+          mma_bf16(tmem + kColP + pb * 128, a,
+                   sdesc(base + kVOff + s * 32768 + kk * 2048, 16384, 1024), id_st, acc);
+          mma_bf16(tmem + kColZ + pb * 16, a,
+                   sdesc(base + kOnesOff + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024), id_z,
+                   acc);
+        }
+        mma_commit(bar(PHI_EMPTY));
+        mma_commit(bar(V_EMPTY + s));
+        if (j == nt - 1) mma_commit(bar(ACC_DONE + pb));
+      }
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // ================================================= convert (thread = token)
+    const int r = tid;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    float* bias = reinterpret_cast<float*>(sbase + kBiasOff);
+    auto wait_all = [&](uint32_t b, uint32_t parity, uint32_t code) {
+      return __all_sync(0xffffffffu, mbar_wait(b, parity, abort_flag, code));
+    };
+    bool ok = true;
+    for (int gt = 0; gt < TT; ++gt) {
+      const int il = gt / nt, j = gt % nt, s = gt & 1;
+      if (j == 0 && (il == 0 || head_of(il) != head_of(il - 1))) {
+        // New head: load its b_k (the 4 convert warps sync on barrier 1).
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        const int h = head_of(il), half = Dp >> 1;
+        if (r < Dp) {
+          const int part = r >= half;
+          bias[r] = P.bk[(h * 2 + part) * half + (r - part * half)];
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+      }
+      if (ok) ok = wait_all(bar(PSI_FULL), gt & 1, 36);
+      if (ok && gt >= 1) ok = wait_all(bar(PHI_EMPTY), (gt - 1) & 1, 37);
+      const int nvalid = min(128, HW - j * 128);
+      const bool valid = r < nvalid;
+      if (ok) {
+        tc_fence_after();
+        // psi streamed from TMEM 32 features at a time straight into the
+        // phi^T tile (token row r; features 64g..64g+63 in box g).
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint32_t pk[16];
+          if (q4 * 32 < Dp) {  // warp-uniform
+            uint32_t ps[32];
+            REHYAT_TMEM_LD32(lane_base + kColPsi + q4 * 32, ps);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              float v0 = 0.f, v1 = 0.f;
+              if (valid) {
+                const float a0 = __uint_as_float(ps[2 * i]) + bias[q4 * 32 + 2 * i];
+                const float a1 = __uint_as_float(ps[2 * i + 1]) + bias[q4 * 32 + 2 * i + 1];
+                v0 = a0 * a0;
+                v1 = a1 * a1;
+              }
+              pk[i] = pack_bf16(v0, v1);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pk[i] = 0u;
+          }
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) {
+            const int c = q4 * 4 + c4;  // 16-byte chunk of the 256-byte row
+            const uint32_t box = c >> 3, ch = c & 7;
+            st_shared_v4(base + kPhiOff + box * 16384 + r * 128 + ((ch ^ (r & 7)) << 4),
+                         pk[4 * c4], pk[4 * c4 + 1], pk[4 * c4 + 2], pk[4 * c4 + 3]);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(bar(PSI_FREE));
+        if (nvalid < 128) {
+          ok = wait_all(bar(V_FULL + s), (gt >> 1) & 1, 38);
+          if (ok && !valid) {
+            const uint32_t vrow = base + kVOff + s * 32768 + r * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              st_shared_v4(vrow + c * 16, 0, 0, 0, 0);
+              st_shared_v4(vrow + 16384 + c * 16, 0, 0, 0, 0);
+            }
+          }
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        mbar_arrive(bar(PHI_FULL));
+      }
+    }
+  } else if (warp < 8) {
+    // ================================================= epilogue (thread = feature)
+    const int r = tid - 128;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    bool ok = true;
+    for (int il = 0; il < nitems && ok; ++il) {
+      const int pb = il & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(ACC_DONE + pb), (il >> 1) & 1, abort_flag, 39));
+      if (!ok) break;
+      tc_fence_after();
+      const long long obase = static_cast<long long>(it0 + il);  // (bh*T + slice)
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[32];
+        REHYAT_TMEM_LD32(lane_base + kColP + pb * 128 + c * 32, v);
+        tmem_wait_ld();
+        if (r < Dp) {
+          float4* dst = reinterpret_cast<float4*>(P.P + (obase * Dp + r) * 128 + c * 32);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                 __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+        }
+      }
+      uint32_t zv[32];
+      REHYAT_TMEM_LD32(lane_base + kColZ + pb * 16, zv);
+      tmem_wait_ld();
+      if (r < Dp) P.z[obase * Dp + r] = __uint_as_float(zv[0]);
+      tc_fence_before();
+      mbar_arrive(bar(P_FREE + pb));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+  }
+}
+
 // ------------------------------------------------------------ host side
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -1273,8 +1631,25 @@ cudaError_t launch_state_tc(const PartialParams& p, const void* wk_img, cudaStre
     maps.rk = maps.k;
     maps.rv = maps.v;
   }
-  cudaError_t e = cudaFuncSetAttribute(tc_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(st::kSmemBytes));
+  cudaError_t e;
+  if (p.seen == nullptr) {
+    // Full forward: persistent CTAs, each with the same number of slices.
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int total = p.BH * p.nslots;
+    const int per_cta = (total + sms - 1) / sms;
+    const int ctas = (total + per_cta - 1) / per_cta;
+    e = cudaFuncSetAttribute(tc_state_persistent_kernel,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(sp::kSmemBytes));
+    if (e != cudaSuccess) return e;
+    tc_state_persistent_kernel<<<ctas, sp::kThreads, sp::kSmemBytes, s>>>(
+        maps, p, static_cast<const __nv_bfloat16*>(wk_img), per_cta);
+    return cudaGetLastError();
+  }
+  e = cudaFuncSetAttribute(tc_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(st::kSmemBytes));
   if (e != cudaSuccess) return e;
   dim3 grid(p.nslots, p.BH);
   tc_state_kernel<<<grid, st::kThreads, st::kSmemBytes, s>>>(

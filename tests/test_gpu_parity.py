@@ -202,6 +202,31 @@ def test_stream_81_slices_constant_memory():
     assert_close_y(np.concatenate(ys), ref_y[0, 3], "bf16")
 
 
+def test_streaming_cuda_graph_replay_matches_eager():
+    """One captured step replayed per chunk equals the eager steps bit for
+    bit (the slice counter is read on the device)."""
+    p = make_problem(batch=1, heads=2, T=10, Hs=6, Ws=11, D=128, Dp=128, Tc=2, To=1,
+                     causal=True, dtype="bf16", seed=43)
+    y_eager, st = _stream_outputs(p)
+    dev = device_tensors(p)
+    st.reset()
+    HW, rows = p.HW, p.Tc * p.HW
+    qb, kb, vb = (torch.empty(1, 2, rows, 128, device="cuda", dtype=torch.bfloat16)
+                  for _ in range(3))
+    out = torch.empty(1, 2, rows, 128, device="cuda")
+    graph = st.capture_step(qb, kb, vb, out)
+    outs = []
+    for i in range(p.T // p.Tc):
+        sl = slice(i * rows, (i + 1) * rows)
+        qb.copy_(dev["q"][:, :, sl])
+        kb.copy_(dev["k"][:, :, sl])
+        vb.copy_(dev["v"][:, :, sl])
+        graph.replay()
+        outs.append(out.clone())
+    torch.cuda.synchronize()
+    assert torch.equal(torch.cat(outs, dim=2), y_eager)
+
+
 def test_streaming_checkpoint_resume_bit_exact():
     p = make_problem(batch=1, heads=2, T=9, Hs=6, Ws=11, D=128, Dp=128, Tc=2, To=1,
                      causal=True, dtype="bf16", seed=41)
