@@ -69,15 +69,17 @@ bool tc_path(const rehyat_params* p) {
 }
 
 // Whether the tensor-core per-slice state kernel is used.
-bool tc_state_path(const rehyat_params* p) {
+// `step` selects the chunk-step fold (a window of slices per call) rather
+// than the full forward's per-slice sums.
+bool tc_state_path(const rehyat_params* p, bool step) {
   return !(p->flags & REHYAT_FLAG_FORCE_SIMT) &&
-         tc_state_eligible(p->in_dtype == REHYAT_BF16, p->D, p->Dp);
+         tc_state_eligible(p->in_dtype == REHYAT_BF16, p->D, p->Dp, step);
 }
 
 // Per-slice states on the path these params select.
 cudaError_t run_partials(const rehyat_params* p, const PartialParams& pp, const void* wk_img,
                          cudaStream_t s) {
-  if (tc_state_path(p)) return launch_state_tc(pp, wk_img, s);
+  if (tc_state_path(p, pp.seen != nullptr)) return launch_state_tc(pp, wk_img, s);
   return launch_partials_simt(pp, s);
 }
 
@@ -235,7 +237,7 @@ rehyat_status rehyat_fwd_state(const rehyat_params* p, const void* k, const void
   pp.in_bf16 = p->in_dtype == REHYAT_BF16;
   pp.w_bf16 = pp.in_bf16;
   cudaError_t e = cudaSuccess;
-  if (tc_path(p) || tc_state_path(p))
+  if (tc_path(p) || tc_state_path(p, false))
     e = launch_w_images(phi->Wq, ws + w.wimg_off, phi->Wk, ws + w.wkimg_off, p->heads, p->D,
                         p->Dp, s);
   if (e != cudaSuccess) return to_status(e);
@@ -367,7 +369,7 @@ rehyat_status rehyat_chunk_step(const rehyat_params* p, const void* q, const voi
   a.nchunks = 1;
   a.nq_slices = nslices;
   cudaError_t e = cudaSuccess;
-  if (tc_path(p) || tc_state_path(p)) {
+  if (tc_path(p) || tc_state_path(p, true)) {
     e = launch_w_images(phi->Wq, ws + w.wimg_off, phi->Wk, ws + w.wkimg_off, p->heads, p->D,
                         p->Dp, s);
     if (e != cudaSuccess) return to_status(e);

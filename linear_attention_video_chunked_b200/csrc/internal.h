@@ -69,7 +69,7 @@ bool tc_attn_eligible(int in_bf16, int D, int Dp);
 
 // Tensor-core per-slice state (bf16, D = 128, Dp in {64, 128}); wk_img is
 // the bf16 image of W_k.
-bool tc_state_eligible(int in_bf16, int D, int Dp);
+bool tc_state_eligible(int in_bf16, int D, int Dp, bool step);
 cudaError_t launch_state_tc(const PartialParams& p, const void* wk_img, cudaStream_t s);
 
 // Linear-set state per chunk from the per-slice states (full mode).

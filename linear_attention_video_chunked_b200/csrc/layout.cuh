@@ -29,6 +29,20 @@ __host__ __device__ __forceinline__ long long sl_index(int f, int d, int D, int 
          d * 32 + ((chunk ^ (d & 7)) << 2) + w;
 }
 
+// Inverse of sl_index: the (feature, column) stored at image offset o.
+__host__ __device__ __forceinline__ void sl_coords(long long o, int D, int Dp, int* f, int* d) {
+  const int pw = piece_width(Dp);
+  const long long piece = o / (static_cast<long long>(D) * pw);
+  const int r1 = static_cast<int>(o - piece * D * pw);
+  const int box = r1 / (D * 32);
+  const int r2 = r1 - box * D * 32;
+  const int dd = r2 >> 5;
+  const int r3 = r2 & 31;
+  const int chunk = (r3 >> 2) ^ (dd & 7);
+  *d = dd;
+  *f = static_cast<int>(piece) * pw + box * 32 + chunk * 4 + (r3 & 3);
+}
+
 // phi_q weights of one head: logical W[d][f] (f over both parts), stored per
 // feature piece as a K-major bf16 operand [piece features][D]: boxes of 64
 // D-elements, each box pw rows x 128 bytes.

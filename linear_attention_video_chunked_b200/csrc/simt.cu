@@ -322,8 +322,12 @@ __global__ void scan_kernel(const float* __restrict__ P, const float* __restrict
   float* dst;
   long long stride;
   if (e < PD) {
-    src = P + bh * T * PD + e;
-    dst = SL + bh * nchunks * PD + sl_index(static_cast<int>(e / D), static_cast<int>(e % D), D, Dp);
+    // e walks the S^L image (coalesced stores); gather the matching element
+    // of the plain per-slice states (a block's reads cover whole sectors).
+    int f, d;
+    sl_coords(e, D, Dp, &f, &d);
+    src = P + bh * T * PD + static_cast<long long>(f) * D + d;
+    dst = SL + bh * nchunks * PD + e;
     stride = PD;
   } else if (e < PD + Dp) {
     src = z + static_cast<long long>(bh) * T * Dp + (e - PD);
@@ -389,9 +393,13 @@ __global__ void state_add_kernel(const float* __restrict__ P, const float* __res
   const int bh = blockIdx.y;
   const long long leave = leaving_slices(*seen, To, nq);
   if (e < PD) {
-    const long long se = bh * PD + sl_index(static_cast<int>(e / D), static_cast<int>(e % D), D, Dp);
+    // e walks the image layout of s (coalesced); gather from the plain slots.
+    int f, d;
+    sl_coords(e, D, Dp, &f, &d);
+    const long long se = bh * PD + e;
+    const long long pe = static_cast<long long>(f) * D + d;
     float acc = s_state[se];
-    for (long long i = 0; i < leave; ++i) acc += P[(bh * nslots + i) * PD + e];
+    for (long long i = 0; i < leave; ++i) acc += P[(bh * nslots + i) * PD + pe];
     s_state[se] = acc;
   } else if (e < PD + Dp) {
     const long long f = e - PD;

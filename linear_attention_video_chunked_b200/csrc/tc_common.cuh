@@ -103,6 +103,13 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t 
          (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
+// UMMA descriptor without swizzle whose strides are zero: every 8-row x
+// 16-byte core matrix of the operand is the same 128 bytes at addr (used for
+// an all-ones operand without storing a full tile).
+__device__ __forceinline__ uint64_t sdesc_repeat(uint32_t addr) {
+  return static_cast<uint64_t>((addr & 0x3FFFFu) >> 4) | (1ull << 46);
+}
+
 // Instruction descriptor: fp32 accumulate, A K-major, A/B format fmt
 // (1 = bf16, 2 = tf32), B K-major or MN-major.
 __host__ __device__ constexpr uint32_t idesc(int M, int N, uint32_t fmt, bool b_mn_major) {

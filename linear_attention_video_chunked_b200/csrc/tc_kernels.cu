@@ -1296,20 +1296,24 @@ __global__ void __launch_bounds__(st::kThreads, 1)
 //   warp 8     TMA (K, V tiles; the W_k image when the head changes);
 //   warp 9     MMA (psi = K W_k, P += phi^T V, z += phi^T 1) and TMEM owner.
 // TMEM: psi [0,128), P accumulators [128,256) [256,384) (alternating per
-// slice), z accumulators [384,400) [400,416).  D' in {64, 128}.
+// slice), z accumulators [384,400) [400,416).  D' in {64, 128, 256}: with
+// D' = 256 an item is one 128-feature half of a slice (items run over
+// (b*h, half, slice), so W_k changes only at half or head boundaries).
 // ===========================================================================
 namespace sp {
 constexpr int kThreads = 320;
-constexpr uint32_t kKOff = 0;          // K ring, 2 x 32 KB
-constexpr uint32_t kVOff = 65536;      // V ring, 2 x 32 KB
-constexpr uint32_t kWOff = 131072;     // W_k image of the current head (<= 32 KB)
-constexpr uint32_t kPhiOff = 163840;   // phi^T tile, 2 boxes x 16 KB
-constexpr uint32_t kOnesOff = 196608;  // all-ones B operand for z (4 KB)
-constexpr uint32_t kBiasOff = 200704;  // b_k of the current head (<= 512 B)
-constexpr uint32_t kBarOff = 201216;
-enum { K_FULL = 0, V_FULL = 2, K_EMPTY = 4, V_EMPTY = 6, PSI_FULL = 8, PSI_FREE = 9,
-       PHI_FULL = 10, PHI_EMPTY = 11, ACC_DONE = 12, P_FREE = 14, W_FULL = 16, W_FREE = 17,
-       NBAR = 18 };
+// K has 3 stages (released once psi = K W_k has read it), V has 2 (released
+// after phi^T V): the next K tiles load two products ahead.
+constexpr uint32_t kKOff = 0;          // K ring, 3 x 32 KB
+constexpr uint32_t kVOff = 98304;      // V ring, 2 x 32 KB
+constexpr uint32_t kWOff = 163840;     // W_k image of the current head (<= 32 KB)
+constexpr uint32_t kPhiOff = 196608;   // phi^T tile, 2 boxes x 16 KB
+constexpr uint32_t kOnesOff = 229376;  // 128 B of bf16 ones (one repeated core matrix)
+constexpr uint32_t kBiasOff = 229632;  // b_k of the current head (<= 512 B)
+constexpr uint32_t kBarOff = 230144;
+enum { K_FULL = 0, K_EMPTY = 3, V_FULL = 6, V_EMPTY = 8, PSI_FULL = 10, PSI_FREE = 11,
+       PHI_FULL = 12, PHI_EMPTY = 13, ACC_DONE = 14, P_FREE = 16, W_FULL = 18, W_FREE = 19,
+       NBAR = 20 };
 constexpr uint32_t kTmemSlot = kBarOff + 8 * NBAR;
 constexpr uint32_t kAbortSlot = kTmemSlot + 4;
 constexpr uint32_t kSmemBytes = kBarOff + 256 + 1024;
@@ -1345,14 +1349,25 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(sbase + sp::kAbortSlot);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int Dp = P.Dp, HW = P.HW, T = P.nslots;
-  const int total = P.BH * T;
+  const int pw = Dp < 128 ? Dp : 128;  // features per item
+  const int halves = Dp / pw;
+  const int total = P.BH * halves * T;
   const int it0 = blockIdx.x * items_per_cta;
   const int it1 = min(total, it0 + items_per_cta);
   if (it0 >= it1) return;
   const int nitems = it1 - it0;
   const int nt = (HW + 127) / 128;
   const int TT = nitems * nt;  // tiles of this CTA
-  auto head_of = [&](int il) { return ((it0 + il) / T) % P.heads; };
+  // Item i = (bh, half, slice) in that order; the W_k piece (and b_k) an
+  // item needs is keyed by (head, half).
+  auto wkey_of = [&](int il) {
+    const int i = it0 + il, bh = i / (halves * T), hf = (i / T) % halves;
+    return (bh % P.heads) * halves + hf;
+  };
+  auto slice_row_of = [&](int il) {  // output row (bh * T + slice) of item il
+    const int i = it0 + il;
+    return static_cast<long long>(i / (halves * T)) * T + i % T;
+  };
 
   if (tid == 0) {
     for (int i = 0; i < NBAR; ++i) {
@@ -1362,8 +1377,7 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
     *abort_flag = 0;
     fence_barrier_init();
   }
-  for (int i = tid; i < 1024; i += kThreads)
-    reinterpret_cast<uint32_t*>(sbase + kOnesOff)[i] = 0x3F803F80u;
+  if (tid < 32) reinterpret_cast<uint32_t*>(sbase + kOnesOff)[tid] = 0x3F803F80u;  // 128 B
   fence_proxy_async();
   if (warp == 9) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -1375,7 +1389,7 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sbase + sp::kTmemSlot);
-  const uint32_t wbytes = static_cast<uint32_t>(Dp) * 128 * 2;
+  const uint32_t wbytes = static_cast<uint32_t>(pw) * 128 * 2;
 
   if (warp == 8) {
     // ================================================= TMA producer
@@ -1383,23 +1397,25 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
       bool ok = true;
       int wloads = 0;
       for (int il = 0; il < nitems && ok; ++il) {
-        const int item = it0 + il, bh = item / T, slice = item % T, h = bh % P.heads;
-        if (il == 0 || h != head_of(il - 1)) {
+        const int item = it0 + il, bh = item / (halves * T), slice = item % T;
+        const int wkey = wkey_of(il);
+        if (il == 0 || wkey != wkey_of(il - 1)) {
           if (il > 0) ok = mbar_wait(bar(W_FREE), (wloads - 1) & 1, abort_flag, 27);
           if (!ok) break;
+          // The image of head h holds its D' features as pieces of pw rows.
           mbar_expect_tx(bar(W_FULL), wbytes);
-          bulk_load(base + kWOff, wk_img + static_cast<long long>(h) * Dp * 128, wbytes,
+          bulk_load(base + kWOff, wk_img + static_cast<long long>(wkey) * pw * 128, wbytes,
                     bar(W_FULL));
           ++wloads;
         }
         for (int j = 0; j < nt && ok; ++j) {
-          const int gt = il * nt + j, s = gt & 1;
+          const int gt = il * nt + j, s = gt & 1, ks = gt % 3;
           const int row = slice * HW + j * 128;
-          if (gt >= 2) ok = mbar_wait(bar(K_EMPTY + s), ((gt - 2) >> 1) & 1, abort_flag, 28);
+          if (gt >= 3) ok = mbar_wait(bar(K_EMPTY + ks), ((gt - 3) / 3) & 1, abort_flag, 28);
           if (!ok) break;
-          mbar_expect_tx(bar(K_FULL + s), 32768);
-          tma_load_3d(base + kKOff + s * 32768, &maps.k, bar(K_FULL + s), 0, row, bh);
-          tma_load_3d(base + kKOff + s * 32768 + 16384, &maps.k, bar(K_FULL + s), 64, row, bh);
+          mbar_expect_tx(bar(K_FULL + ks), 32768);
+          tma_load_3d(base + kKOff + ks * 32768, &maps.k, bar(K_FULL + ks), 0, row, bh);
+          tma_load_3d(base + kKOff + ks * 32768 + 16384, &maps.k, bar(K_FULL + ks), 64, row, bh);
           if (gt >= 2) ok = mbar_wait(bar(V_EMPTY + s), ((gt - 2) >> 1) & 1, abort_flag, 29);
           if (!ok) break;
           mbar_expect_tx(bar(V_FULL + s), 32768);
@@ -1412,7 +1428,7 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
   } else if (warp == 9) {
     // ================================================= MMA issuer
     if (lane == 0) {
-      const uint32_t id_psi = idesc_ab(128, Dp, 1, false, false);
+      const uint32_t id_psi = idesc_ab(128, pw, 1, false, false);
       const uint32_t id_st = idesc_ab(128, 128, 1, true, true);
       const uint32_t id_z = idesc_ab(128, 16, 1, true, false);
       bool ok = true;
@@ -1421,23 +1437,25 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
       // the converter to have read psi(gt - 1), and for the head's W_k.
       auto issue_psi = [&](int gt) -> bool {
         const int il = gt / nt, s = gt & 1;
-        if (gt % nt == 0 && (il == 0 || head_of(il) != head_of(il - 1))) {
+        if (gt % nt == 0 && (il == 0 || wkey_of(il) != wkey_of(il - 1))) {
           if (il > 0) mma_commit(bar(W_FREE));  // tracks every earlier MMA
           if (!mbar_wait(bar(W_FULL), wwaits & 1, abort_flag, 30)) return false;
           ++wwaits;
         }
-        if (!mbar_wait(bar(K_FULL + s), (gt >> 1) & 1, abort_flag, 31)) return false;
+        (void)s;
+        const int ks = gt % 3;
+        if (!mbar_wait(bar(K_FULL + ks), (gt / 3) & 1, abort_flag, 31)) return false;
         if (gt >= 1 && !mbar_wait(bar(PSI_FREE), (gt - 1) & 1, abort_flag, 32)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-          const uint32_t woff = (kk >> 2) * (Dp * 128) + (kk & 3) * 32;
-          mma_bf16(tmem + kColPsi, sdesc(base + kKOff + s * 32768 + koff, 16, 1024),
+          const uint32_t woff = (kk >> 2) * (pw * 128) + (kk & 3) * 32;
+          mma_bf16(tmem + kColPsi, sdesc(base + kKOff + ks * 32768 + koff, 16, 1024),
                    sdesc(base + kWOff + woff, 16, 1024), id_psi, kk > 0);
         }
         mma_commit(bar(PSI_FULL));
-        mma_commit(bar(K_EMPTY + s));
+        mma_commit(bar(K_EMPTY + ks));
         return true;
       };
       ok = issue_psi(0);
@@ -1456,9 +1474,7 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
           const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
           mma_bf16(tmem + kColP + pb * 128, a,
                    sdesc(base + kVOff + s * 32768 + kk * 2048, 16384, 1024), id_st, acc);
-          mma_bf16(tmem + kColZ + pb * 16, a,
-                   sdesc(base + kOnesOff + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024), id_z,
-                   acc);
+          mma_bf16(tmem + kColZ + pb * 16, a, sdesc_repeat(base + kOnesOff), id_z, acc);
         }
         mma_commit(bar(PHI_EMPTY));
         mma_commit(bar(V_EMPTY + s));
@@ -1477,14 +1493,11 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
     bool ok = true;
     for (int gt = 0; gt < TT; ++gt) {
       const int il = gt / nt, j = gt % nt, s = gt & 1;
-      if (j == 0 && (il == 0 || head_of(il) != head_of(il - 1))) {
-        // New head: load its b_k (the 4 convert warps sync on barrier 1).
+      if (j == 0 && (il == 0 || wkey_of(il) != wkey_of(il - 1))) {
+        // New (head, half): load its b_k features (b_k of head h is h's D'
+        // consecutive features; the 4 convert warps sync on barrier 1).
         asm volatile("bar.sync 1, 128;" ::: "memory");
-        const int h = head_of(il), half = Dp >> 1;
-        if (r < Dp) {
-          const int part = r >= half;
-          bias[r] = P.bk[(h * 2 + part) * half + (r - part * half)];
-        }
+        if (r < pw) bias[r] = P.bk[wkey_of(il) * pw + r];
         asm volatile("bar.sync 1, 128;" ::: "memory");
       }
       if (ok) ok = wait_all(bar(PSI_FULL), gt & 1, 36);
@@ -1498,7 +1511,7 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
           uint32_t pk[16];
-          if (q4 * 32 < Dp) {  // warp-uniform
+          if (q4 * 32 < pw) {  // warp-uniform
             uint32_t ps[32];
             REHYAT_TMEM_LD32(lane_base + kColPsi + q4 * 32, ps);
             tmem_wait_ld();
@@ -1553,13 +1566,14 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(bar(ACC_DONE + pb), (il >> 1) & 1, abort_flag, 39));
       if (!ok) break;
       tc_fence_after();
-      const long long obase = static_cast<long long>(it0 + il);  // (bh*T + slice)
+      // Feature row f = half * pw + r of slice (bh*T + slice).
+      const long long frow = slice_row_of(il) * Dp + ((it0 + il) / T) % halves * pw + r;
       for (int c = 0; c < 4; ++c) {
         uint32_t v[32];
         REHYAT_TMEM_LD32(lane_base + kColP + pb * 128 + c * 32, v);
         tmem_wait_ld();
-        if (r < Dp) {
-          float4* dst = reinterpret_cast<float4*>(P.P + (obase * Dp + r) * 128 + c * 32);
+        if (r < pw) {
+          float4* dst = reinterpret_cast<float4*>(P.P + frow * 128 + c * 32);
 #pragma unroll
           for (int i = 0; i < 8; ++i)
             dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
@@ -1569,7 +1583,7 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
       uint32_t zv[32];
       REHYAT_TMEM_LD32(lane_base + kColZ + pb * 16, zv);
       tmem_wait_ld();
-      if (r < Dp) P.z[obase * Dp + r] = __uint_as_float(zv[0]);
+      if (r < pw) P.z[frow] = __uint_as_float(zv[0]);
       tc_fence_before();
       mbar_arrive(bar(P_FREE + pb));
     }
@@ -1614,8 +1628,11 @@ bool make_map(CUtensorMap* m, const void* ptr, long long rows, int planes) {
 
 }  // namespace
 
-bool tc_state_eligible(int in_bf16, int D, int Dp) {
-  return in_bf16 && D == kD && (Dp == 64 || Dp == 128) && encode_fn() != nullptr;
+bool tc_state_eligible(int in_bf16, int D, int Dp, bool step) {
+  // The step-mode kernel holds all D' features of a slice in one CTA (at most
+  // 128); the persistent full-mode kernel splits D' = 256 into halves.
+  const bool dp_ok = Dp == 64 || Dp == 128 || (!step && Dp == 256);
+  return in_bf16 && D == kD && dp_ok && encode_fn() != nullptr;
 }
 
 cudaError_t launch_state_tc(const PartialParams& p, const void* wk_img, cudaStream_t s) {
@@ -1637,7 +1654,7 @@ cudaError_t launch_state_tc(const PartialParams& p, const void* wk_img, cudaStre
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess)
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int total = p.BH * p.nslots;
+    const int total = p.BH * p.nslots * (p.Dp > 128 ? p.Dp / 128 : 1);
     const int per_cta = (total + sms - 1) / sms;
     const int ctas = (total + per_cta - 1) / per_cta;
     e = cudaFuncSetAttribute(tc_state_persistent_kernel,

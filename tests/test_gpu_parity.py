@@ -49,6 +49,7 @@ SMALL = [
     (1, 3, 6, 8, 12, 64, 256, 2, 0),     # no overlap, wide phi
     (1, 2, 3, 5, 5, 32, 32, 4, 1),       # one chunk covers everything
     (1, 1, 9, 11, 12, 128, 128, 3, 1),   # HW=132, several chunks
+    (1, 2, 5, 9, 15, 128, 256, 2, 1),    # D'=256 on the tensor-core state path
 ]
 
 
@@ -121,6 +122,18 @@ def test_balanced_branches_full_size(name, std, subset):
         assert_close_y(y[b, hh], ref_y[b, hh], "bf16", f"y[{b},{hh}]")
         assert_close_partials({k: v[b, hh] for k, v in parts.items()},
                               {k: v[b, hh] for k, v in ref_p.items()}, "bf16")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_wide_phi_several_items_per_cta(causal):
+    """D'=256 with more (b*h, half, slice) items than SMs, so persistent
+    state CTAs cross half and head boundaries and reload W_k mid-run."""
+    p = make_problem(batch=1, heads=4, T=20, Hs=8, Ws=17, D=128, Dp=256, Tc=3, To=1,
+                     causal=causal, dtype="bf16", dist="scaled", seed=77)
+    ref_y, ref_p = orc.run_problem(p)
+    y, parts = run_fwd(p, debug=True)
+    assert_close_y(y, ref_y, "bf16")
+    assert_close_partials(parts, ref_p, "bf16")
 
 
 @pytest.mark.parametrize("Tc,To,Dp,causal", [(1, 0, 128, False), (2, 2, 64, True),

@@ -1,0 +1,56 @@
+"""Host-side check of the shared-memory image layouts (csrc/layout.cuh):
+sl_index is a bijection on [0, D*D') and sl_coords inverts it, and the
+weight image index is a bijection too, for every supported (D, D')."""
+import os
+import shutil
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+CSRC = os.path.join(ROOT, "linear_attention_video_chunked_b200", "csrc")
+
+PROGRAM = r"""
+#include <cstdio>
+#include <vector>
+#include "layout.cuh"
+using namespace rehyat;
+int main() {
+  int bad = 0;
+  const int Ds[] = {32, 64, 128}, Dps[] = {32, 64, 128, 256};
+  for (int D : Ds) for (int Dp : Dps) {
+    std::vector<int> seen(D * Dp, 0), seen_w(D * Dp, 0);
+    for (int f = 0; f < Dp; ++f) for (int d = 0; d < D; ++d) {
+      const long long o = sl_index(f, d, D, Dp);
+      if (o < 0 || o >= (long long)D * Dp) { ++bad; continue; }
+      seen[o]++;
+      int f2, d2;
+      sl_coords(o, D, Dp, &f2, &d2);
+      if (f2 != f || d2 != d) ++bad;
+      if (D >= 64) {
+        const long long w = wimg_index(f, d, D, Dp);
+        if (w < 0 || w >= (long long)D * Dp) ++bad; else seen_w[w]++;
+      }
+    }
+    for (int i = 0; i < D * Dp; ++i) {
+      if (seen[i] != 1) ++bad;
+      if (D >= 64 && seen_w[i] != 1) ++bad;
+    }
+  }
+  std::printf("%d\n", bad);
+  return bad != 0;
+}
+"""
+
+
+def test_image_layouts_are_bijections(tmp_path):
+    nvcc = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
+    if not os.path.exists(nvcc):
+        pytest.skip("nvcc not available")
+    src = tmp_path / "t.cu"
+    src.write_text(PROGRAM)
+    exe = tmp_path / "t"
+    subprocess.run([nvcc, "-std=c++17", "-I" + CSRC, str(src), "-o", str(exe)], check=True,
+                   capture_output=True, timeout=300)
+    res = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert res.returncode == 0 and res.stdout.strip() == "0", res.stdout
