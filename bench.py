@@ -35,7 +35,7 @@ if ROOT not in sys.path:
 WORKLOAD = "wan_480x832_bidir"
 METRIC = "hybrid-attn fwd tokens/s & TFLOP/s (% BF16 tensor peak), 1 B200, 21x30x52 latent"
 L2_FLUSH_BYTES = 256 << 20
-KERNELS_PER_STEP = 5  # weight images (x2: state and attention calls), per-slice state, chunk scan, attention
+KERNELS_PER_STEP = 4  # weight images, per-slice state, chunk scan, attention
 
 
 # --------------------------------------------------------------- workload

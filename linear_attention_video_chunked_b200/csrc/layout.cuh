@@ -29,6 +29,20 @@ __host__ __device__ __forceinline__ long long sl_index(int f, int d, int D, int 
          d * 32 + ((chunk ^ (d & 7)) << 2) + w;
 }
 
+// sl_index split into a part that depends on the feature only and the
+// offset of column d within the feature's run (for writers that walk d with
+// f fixed); piece widths are multiples of 32 whenever D' has several pieces.
+__host__ __device__ __forceinline__ long long sl_feature_base(int f, int D, int Dp) {
+  const int pw = piece_width(Dp);
+  const int piece = f / pw;
+  const int fl = f - piece * pw;
+  return static_cast<long long>(piece) * D * pw + static_cast<long long>(fl >> 5) * D * 32 +
+         (fl & 3);
+}
+__host__ __device__ __forceinline__ int sl_column_offset(int f, int d) {
+  return d * 32 + ((((f >> 2) & 7) ^ (d & 7)) << 2);
+}
+
 // Inverse of sl_index: the (feature, column) stored at image offset o.
 __host__ __device__ __forceinline__ void sl_coords(long long o, int D, int Dp, int* f, int* d) {
   const int pw = piece_width(Dp);

@@ -302,9 +302,11 @@ __global__ void __launch_bounds__(256) partials_simt_kernel(PartialParams P) {
   }
   const int f = f0 + fl;
   if (f < Dp) {
-    float* Pout = P.P + (static_cast<long long>(bh) * P.nslots + slot) * Dp * D + static_cast<long long>(f) * D;
+    // Per-slice states are stored in the S^L image layout.
+    float* Pout = P.P + (static_cast<long long>(bh) * P.nslots + slot) * Dp * D +
+                  sl_feature_base(f, D, Dp);
 #pragma unroll
-    for (int c = 0; c < D / 4; ++c) Pout[lane4 + 4 * c] = acc[c];
+    for (int c = 0; c < D / 4; ++c) Pout[sl_column_offset(f, lane4 + 4 * c)] = acc[c];
     if (lane4 == 0) P.z[(static_cast<long long>(bh) * P.nslots + slot) * Dp + f] = zacc;
   }
 }
@@ -322,11 +324,8 @@ __global__ void scan_kernel(const float* __restrict__ P, const float* __restrict
   float* dst;
   long long stride;
   if (e < PD) {
-    // e walks the S^L image (coalesced stores); gather the matching element
-    // of the plain per-slice states (a block's reads cover whole sectors).
-    int f, d;
-    sl_coords(e, D, Dp, &f, &d);
-    src = P + bh * T * PD + static_cast<long long>(f) * D + d;
+    // Per-slice states and S^L share the image layout: element e of each.
+    src = P + bh * T * PD + e;
     dst = SL + bh * nchunks * PD + e;
     stride = PD;
   } else if (e < PD + Dp) {
@@ -393,13 +392,10 @@ __global__ void state_add_kernel(const float* __restrict__ P, const float* __res
   const int bh = blockIdx.y;
   const long long leave = leaving_slices(*seen, To, nq);
   if (e < PD) {
-    // e walks the image layout of s (coalesced); gather from the plain slots.
-    int f, d;
-    sl_coords(e, D, Dp, &f, &d);
+    // s and the per-slot states share the image layout: element e of each.
     const long long se = bh * PD + e;
-    const long long pe = static_cast<long long>(f) * D + d;
     float acc = s_state[se];
-    for (long long i = 0; i < leave; ++i) acc += P[(bh * nslots + i) * PD + pe];
+    for (long long i = 0; i < leave; ++i) acc += P[(bh * nslots + i) * PD + e];
     s_state[se] = acc;
   } else if (e < PD + Dp) {
     const long long f = e - PD;

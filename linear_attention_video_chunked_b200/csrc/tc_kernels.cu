@@ -1258,18 +1258,17 @@ __global__ void __launch_bounds__(st::kThreads, 1)
     if (ok) ok = wait_all(bar(ACC_DONE), (nt - 1) & 1, 25);
     if (ok) {
       tc_fence_after();
-      // Thread r = feature r (accumulator lane r).
+      // Thread r = feature r (accumulator lane r); the state is stored in the
+      // S^L image layout (a warp writes one 128-byte row per column).
       const long long obase = (static_cast<long long>(bh) * P.nslots + slot);
+      float* prow = P.P + obase * Dp * 128 + sl_feature_base(r, 128, Dp);
       for (int c = 0; c < 4; ++c) {
         uint32_t v[32];
         REHYAT_TMEM_LD32(lane_base + kColP + c * 32, v);
         tmem_wait_ld();
         if (r < Dp) {
-          float4* dst = reinterpret_cast<float4*>(P.P + (obase * Dp + r) * 128 + c * 32);
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                 __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+          for (int i = 0; i < 32; ++i) prow[sl_column_offset(r, c * 32 + i)] = __uint_as_float(v[i]);
         }
       }
       uint32_t zv[32];
@@ -1289,53 +1288,51 @@ __global__ void __launch_bounds__(st::kThreads, 1)
 
 // ===========================================================================
 // Persistent per-slice state kernel (full mode): the same sums as
-// tc_state_kernel, with each CTA streaming a contiguous run of (b*h, slice)
-// items through one K/V pipeline that does not drain between slices.
-//   warps 0-3  convert: psi (TMEM) -> phi = (psi + b)^2 -> bf16 phi^T tile;
-//   warps 4-7  epilogue: drain the finished slice's P and z from TMEM;
-//   warp 8     TMA (K, V tiles; the W_k image when the head changes);
-//   warp 9     MMA (psi = K W_k, P += phi^T V, z += phi^T 1) and TMEM owner.
-// TMEM: psi [0,128), P accumulators [128,256) [256,384) (alternating per
-// slice), z accumulators [384,400) [400,416).  D' in {64, 128, 256}: with
-// D' = 256 an item is one 128-feature half of a slice (items run over
-// (b*h, half, slice), so W_k changes only at half or head boundaries).
+// tc_state_kernel, with each CTA streaming a contiguous run of items through
+// one K/V pipeline that does not drain between slices.  The feature map is
+// computed transposed, psi^T = W_k^T K^T (TMEM lane = feature, column =
+// token), so each converter thread owns one feature: it squares psi + b in
+// place, rounds to bf16 and leaves phi^T in TMEM as the A operand of
+// P += phi^T V (the TMEM-A form), and it sums z = sum_t phi itself.
+//   warps 0-3  convert (thread = feature), z;
+//   warps 4-7  epilogue: drain the finished slice's P from TMEM;
+//   warp 8     TMA (K, V tiles; the W_k piece when (head, half) changes);
+//   warp 9     MMA (psi^T, P += phi^T V) and TMEM owner.
+// TMEM: psi/phi buffers [0,128) [128,256) (alternating per token tile), P
+// accumulators [256,384) [384,512) (alternating per item).
+// D' in {64, 128, 256}: with D' = 256 an item is one 128-feature half of a
+// slice (items run over (b*h, half, slice), so W_k changes only at half or
+// head boundaries); with D' = 64 the upper 64 W_k rows stay zero.
 // ===========================================================================
 namespace sp {
 constexpr int kThreads = 320;
-// K has 3 stages (released once psi = K W_k has read it), V has 2 (released
-// after phi^T V): the next K tiles load two products ahead.
+constexpr int kStages = 3;             // K and V ring depth
 constexpr uint32_t kKOff = 0;          // K ring, 3 x 32 KB
-constexpr uint32_t kVOff = 98304;      // V ring, 2 x 32 KB
-constexpr uint32_t kWOff = 163840;     // W_k image of the current head (<= 32 KB)
-constexpr uint32_t kPhiOff = 196608;   // phi^T tile, 2 boxes x 16 KB
-constexpr uint32_t kOnesOff = 229376;  // 128 B of bf16 ones (one repeated core matrix)
-constexpr uint32_t kBiasOff = 229632;  // b_k of the current head (<= 512 B)
-constexpr uint32_t kBarOff = 230144;
-enum { K_FULL = 0, K_EMPTY = 3, V_FULL = 6, V_EMPTY = 8, PSI_FULL = 10, PSI_FREE = 11,
-       PHI_FULL = 12, PHI_EMPTY = 13, ACC_DONE = 14, P_FREE = 16, W_FULL = 18, W_FREE = 19,
-       NBAR = 20 };
+constexpr uint32_t kVOff = 98304;      // V ring, 3 x 32 KB
+constexpr uint32_t kWOff = 196608;     // W_k piece, 2 boxes x 128 rows x 128 B
+constexpr uint32_t kBarOff = 229376;
+enum { K_FULL = 0, K_EMPTY = 3, V_FULL = 6, V_EMPTY = 9, PSI_FULL = 12, PHI_FULL = 14,
+       BUF_FREE = 16, ACC_DONE = 18, P_FREE = 20, W_FULL = 22, W_FREE = 23, NBAR = 24 };
 constexpr uint32_t kTmemSlot = kBarOff + 8 * NBAR;
 constexpr uint32_t kAbortSlot = kTmemSlot + 4;
 constexpr uint32_t kSmemBytes = kBarOff + 256 + 1024;
-constexpr uint32_t kColPsi = 0, kColP = 128, kColZ = 384;
+constexpr uint32_t kColBuf = 0, kColP = 256;
 }  // namespace sp
 
 __global__ void __launch_bounds__(sp::kThreads, 1)
     tc_state_persistent_kernel(const __grid_constant__ StMaps maps, const PartialParams P,
                                const __nv_bfloat16* __restrict__ wk_img, int items_per_cta) {
   // Local names shadow the attention kernel's constants of the same names.
-  constexpr int kThreads = sp::kThreads;
+  constexpr int kS = sp::kStages;
   constexpr uint32_t kKOff = sp::kKOff, kVOff = sp::kVOff, kWOff = sp::kWOff;
-  constexpr uint32_t kPhiOff = sp::kPhiOff, kOnesOff = sp::kOnesOff, kBiasOff = sp::kBiasOff;
-  constexpr uint32_t kColPsi = sp::kColPsi, kColP = sp::kColP, kColZ = sp::kColZ;
+  constexpr uint32_t kColBuf = sp::kColBuf, kColP = sp::kColP;
   using sp::K_FULL;
-  using sp::V_FULL;
   using sp::K_EMPTY;
+  using sp::V_FULL;
   using sp::V_EMPTY;
   using sp::PSI_FULL;
-  using sp::PSI_FREE;
   using sp::PHI_FULL;
-  using sp::PHI_EMPTY;
+  using sp::BUF_FREE;
   using sp::ACC_DONE;
   using sp::P_FREE;
   using sp::W_FULL;
@@ -1357,27 +1354,36 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
   if (it0 >= it1) return;
   const int nitems = it1 - it0;
   const int nt = (HW + 127) / 128;
-  const int TT = nitems * nt;  // tiles of this CTA
+  const int TT = nitems * nt;  // token tiles of this CTA
   // Item i = (bh, half, slice) in that order; the W_k piece (and b_k) an
   // item needs is keyed by (head, half).
   auto wkey_of = [&](int il) {
     const int i = it0 + il, bh = i / (halves * T), hf = (i / T) % halves;
     return (bh % P.heads) * halves + hf;
   };
-  auto slice_row_of = [&](int il) {  // output row (bh * T + slice) of item il
+  auto new_w = [&](int il) { return il == 0 || wkey_of(il) != wkey_of(il - 1); };
+  // First output row (feature half * pw of slice bh * T + slice) of item il.
+  auto out_row = [&](int il) {
     const int i = it0 + il;
-    return static_cast<long long>(i / (halves * T)) * T + i % T;
+    return (static_cast<long long>(i / (halves * T)) * T + i % T) * Dp + (i / T) % halves * pw;
   };
 
   if (tid == 0) {
     for (int i = 0; i < NBAR; ++i) {
-      const bool by_group = i == PSI_FREE || i == PHI_FULL || i == P_FREE || i == P_FREE + 1;
+      const bool by_group = i == PHI_FULL || i == PHI_FULL + 1 || i == P_FREE || i == P_FREE + 1;
       mbar_init(bar(i), by_group ? 128 : 1);
     }
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (tid < 32) reinterpret_cast<uint32_t*>(sbase + kOnesOff)[tid] = 0x3F803F80u;  // 128 B
+  if (pw < 128) {
+    // Rows pw..127 of both W_k boxes stay zero (the bulk loads fill rows
+    // 0..pw-1), so psi^T is 0 on the unused lanes.
+    const int per_box = (128 - pw) * 8;  // 16-byte chunks
+    for (int c = tid; c < 2 * per_box; c += sp::kThreads)
+      st_shared_v4(base + kWOff + (c / per_box) * 16384 + pw * 128 + (c % per_box) * 16, 0, 0,
+                   0, 0);
+  }
   fence_proxy_async();
   if (warp == 9) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -1389,38 +1395,39 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sbase + sp::kTmemSlot);
-  const uint32_t wbytes = static_cast<uint32_t>(pw) * 128 * 2;
 
   if (warp == 8) {
     // ================================================= TMA producer
     if (lane == 0) {
       bool ok = true;
       int wloads = 0;
+      const uint32_t box_bytes = static_cast<uint32_t>(pw) * 128;  // one 64-column box
       for (int il = 0; il < nitems && ok; ++il) {
         const int item = it0 + il, bh = item / (halves * T), slice = item % T;
-        const int wkey = wkey_of(il);
-        if (il == 0 || wkey != wkey_of(il - 1)) {
+        if (new_w(il)) {
           if (il > 0) ok = mbar_wait(bar(W_FREE), (wloads - 1) & 1, abort_flag, 27);
           if (!ok) break;
-          // The image of head h holds its D' features as pieces of pw rows.
-          mbar_expect_tx(bar(W_FULL), wbytes);
-          bulk_load(base + kWOff, wk_img + static_cast<long long>(wkey) * pw * 128, wbytes,
-                    bar(W_FULL));
+          // Head h's image holds its D' features as pieces of pw rows, each
+          // piece two boxes of pw rows x 64 columns.
+          const __nv_bfloat16* src = wk_img + static_cast<long long>(wkey_of(il)) * pw * 128;
+          mbar_expect_tx(bar(W_FULL), 2 * box_bytes);
+          bulk_load(base + kWOff, src, box_bytes, bar(W_FULL));
+          bulk_load(base + kWOff + 16384, src + pw * 64, box_bytes, bar(W_FULL));
           ++wloads;
         }
         for (int j = 0; j < nt && ok; ++j) {
-          const int gt = il * nt + j, s = gt & 1, ks = gt % 3;
+          const int gt = il * nt + j, st = gt % kS, ph = ((gt - kS) / kS) & 1;
           const int row = slice * HW + j * 128;
-          if (gt >= 3) ok = mbar_wait(bar(K_EMPTY + ks), ((gt - 3) / 3) & 1, abort_flag, 28);
+          if (gt >= kS) ok = mbar_wait(bar(K_EMPTY + st), ph, abort_flag, 28);
           if (!ok) break;
-          mbar_expect_tx(bar(K_FULL + ks), 32768);
-          tma_load_3d(base + kKOff + ks * 32768, &maps.k, bar(K_FULL + ks), 0, row, bh);
-          tma_load_3d(base + kKOff + ks * 32768 + 16384, &maps.k, bar(K_FULL + ks), 64, row, bh);
-          if (gt >= 2) ok = mbar_wait(bar(V_EMPTY + s), ((gt - 2) >> 1) & 1, abort_flag, 29);
+          mbar_expect_tx(bar(K_FULL + st), 32768);
+          tma_load_3d(base + kKOff + st * 32768, &maps.k, bar(K_FULL + st), 0, row, bh);
+          tma_load_3d(base + kKOff + st * 32768 + 16384, &maps.k, bar(K_FULL + st), 64, row, bh);
+          if (gt >= kS) ok = mbar_wait(bar(V_EMPTY + st), ph, abort_flag, 29);
           if (!ok) break;
-          mbar_expect_tx(bar(V_FULL + s), 32768);
-          tma_load_3d(base + kVOff + s * 32768, &maps.v, bar(V_FULL + s), 0, row, bh);
-          tma_load_3d(base + kVOff + s * 32768 + 16384, &maps.v, bar(V_FULL + s), 64, row, bh);
+          mbar_expect_tx(bar(V_FULL + st), 32768);
+          tma_load_3d(base + kVOff + st * 32768, &maps.v, bar(V_FULL + st), 0, row, bh);
+          tma_load_3d(base + kVOff + st * 32768 + 16384, &maps.v, bar(V_FULL + st), 64, row, bh);
         }
       }
     }
@@ -1428,137 +1435,126 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
   } else if (warp == 9) {
     // ================================================= MMA issuer
     if (lane == 0) {
-      const uint32_t id_psi = idesc_ab(128, pw, 1, false, false);
-      const uint32_t id_st = idesc_ab(128, 128, 1, true, true);
-      const uint32_t id_z = idesc_ab(128, 16, 1, true, false);
+      const uint32_t id_psi = idesc(128, 128, 1, false);  // W_k piece and K tile, K-major
+      const uint32_t id_pv = idesc(128, 128, 1, true);    // phi^T from TMEM, V MN-major
       bool ok = true;
       int wwaits = 0;
-      // psi for global tile gt (item il, tile j): waits for its K tile, for
-      // the converter to have read psi(gt - 1), and for the head's W_k.
+      // psi^T for token tile gt into buffer gt & 1: waits for its K tile,
+      // for phi^T V of tile gt - 2 to have read that buffer, and for W_k.
       auto issue_psi = [&](int gt) -> bool {
-        const int il = gt / nt, s = gt & 1;
-        if (gt % nt == 0 && (il == 0 || wkey_of(il) != wkey_of(il - 1))) {
+        const int il = gt / nt, b = gt & 1, st = gt % kS;
+        if (gt % nt == 0 && new_w(il)) {
           if (il > 0) mma_commit(bar(W_FREE));  // tracks every earlier MMA
           if (!mbar_wait(bar(W_FULL), wwaits & 1, abort_flag, 30)) return false;
           ++wwaits;
         }
-        (void)s;
-        const int ks = gt % 3;
-        if (!mbar_wait(bar(K_FULL + ks), (gt / 3) & 1, abort_flag, 31)) return false;
-        if (gt >= 1 && !mbar_wait(bar(PSI_FREE), (gt - 1) & 1, abort_flag, 32)) return false;
+        if (!mbar_wait(bar(K_FULL + st), (gt / kS) & 1, abort_flag, 31)) return false;
+        if (gt >= 2 && !mbar_wait(bar(BUF_FREE + b), ((gt - 2) >> 1) & 1, abort_flag, 32))
+          return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-          const uint32_t woff = (kk >> 2) * (pw * 128) + (kk & 3) * 32;
-          mma_bf16(tmem + kColPsi, sdesc(base + kKOff + ks * 32768 + koff, 16, 1024),
-                   sdesc(base + kWOff + woff, 16, 1024), id_psi, kk > 0);
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_bf16(tmem + kColBuf + b * 128, sdesc(base + kWOff + off, 16, 1024),
+                   sdesc(base + kKOff + st * 32768 + off, 16, 1024), id_psi, kk > 0);
         }
-        mma_commit(bar(PSI_FULL));
-        mma_commit(bar(K_EMPTY + ks));
+        mma_commit(bar(PSI_FULL + b));
+        mma_commit(bar(K_EMPTY + st));
         return true;
       };
       ok = issue_psi(0);
       for (int gt = 0; gt < TT && ok; ++gt) {
-        const int il = gt / nt, j = gt % nt, s = gt & 1, pb = il & 1;
+        const int il = gt / nt, j = gt % nt, b = gt & 1, st = gt % kS, pb = il & 1;
         if (gt + 1 < TT) ok = issue_psi(gt + 1);
         if (!ok) break;
-        if (j == 0 && il >= 2) ok = mbar_wait(bar(P_FREE + pb), ((il - 2) >> 1) & 1, abort_flag, 33);
-        if (ok) ok = mbar_wait(bar(PHI_FULL), gt & 1, abort_flag, 34) &&
-                     mbar_wait(bar(V_FULL + s), (gt >> 1) & 1, abort_flag, 35);
+        if (j == 0 && il >= 2)
+          ok = mbar_wait(bar(P_FREE + pb), ((il - 2) >> 1) & 1, abort_flag, 33);
+        if (ok) ok = mbar_wait(bar(PHI_FULL + b), (gt >> 1) & 1, abort_flag, 34) &&
+                     mbar_wait(bar(V_FULL + st), (gt / kS) & 1, abort_flag, 35);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t a = sdesc(base + kPhiOff + kk * 2048, 16384, 1024);
-          const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
-          mma_bf16(tmem + kColP + pb * 128, a,
-                   sdesc(base + kVOff + s * 32768 + kk * 2048, 16384, 1024), id_st, acc);
-          mma_bf16(tmem + kColZ + pb * 16, a, sdesc_repeat(base + kOnesOff), id_z, acc);
-        }
-        mma_commit(bar(PHI_EMPTY));
-        mma_commit(bar(V_EMPTY + s));
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ts(tmem + kColP + pb * 128, tmem + kColBuf + b * 128 + kk * 8,
+                      sdesc(base + kVOff + st * 32768 + kk * 2048, 16384, 1024), id_pv,
+                      (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(bar(BUF_FREE + b));
+        mma_commit(bar(V_EMPTY + st));
         if (j == nt - 1) mma_commit(bar(ACC_DONE + pb));
       }
     }
     __syncwarp();
   } else if (warp < 4) {
-    // ================================================= convert (thread = token)
-    const int r = tid;
+    // ================================================= convert (thread = feature)
+    const int f = tid;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    float* bias = reinterpret_cast<float*>(sbase + kBiasOff);
     auto wait_all = [&](uint32_t b, uint32_t parity, uint32_t code) {
       return __all_sync(0xffffffffu, mbar_wait(b, parity, abort_flag, code));
     };
     bool ok = true;
-    for (int gt = 0; gt < TT; ++gt) {
-      const int il = gt / nt, j = gt % nt, s = gt & 1;
-      if (j == 0 && (il == 0 || wkey_of(il) != wkey_of(il - 1))) {
-        // New (head, half): load its b_k features (b_k of head h is h's D'
-        // consecutive features; the 4 convert warps sync on barrier 1).
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (r < pw) bias[r] = P.bk[wkey_of(il) * pw + r];
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-      }
-      if (ok) ok = wait_all(bar(PSI_FULL), gt & 1, 36);
-      if (ok && gt >= 1) ok = wait_all(bar(PHI_EMPTY), (gt - 1) & 1, 37);
+    float bias = 0.f;
+    uint64_t zacc = f2_pack(0.f, 0.f);  // z over even / odd tokens
+    for (int gt = 0; gt < TT && ok; ++gt) {
+      const int il = gt / nt, j = gt % nt, b = gt & 1, st = gt % kS;
+      // b_k of head h is h's D' consecutive features.
+      if (j == 0 && new_w(il)) bias = f < pw ? P.bk[wkey_of(il) * pw + f] : 0.f;
+      ok = wait_all(bar(PSI_FULL + b), (gt >> 1) & 1, 36);
+      if (!ok) break;
+      tc_fence_after();
       const int nvalid = min(128, HW - j * 128);
-      const bool valid = r < nvalid;
-      if (ok) {
-        tc_fence_after();
-        // psi streamed from TMEM 32 features at a time straight into the
-        // phi^T tile (token row r; features 64g..64g+63 in box g).
+      const uint32_t cols = lane_base + kColBuf + b * 128;
+      const uint64_t b2 = f2_pack(bias, bias);
+      // 32 tokens at a time: phi of tokens 32c.. is written as 16 packed
+      // columns at 16c, behind the columns already read.
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          uint32_t pk[16];
-          if (q4 * 32 < pw) {  // warp-uniform
-            uint32_t ps[32];
-            REHYAT_TMEM_LD32(lane_base + kColPsi + q4 * 32, ps);
-            tmem_wait_ld();
+      for (int c = 0; c < 4; ++c) {
+        uint32_t ps[32], pk[16];
+        REHYAT_TMEM_LD32(cols + c * 32, ps);
+        tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              float v0 = 0.f, v1 = 0.f;
-              if (valid) {
-                const float a0 = __uint_as_float(ps[2 * i]) + bias[q4 * 32 + 2 * i];
-                const float a1 = __uint_as_float(ps[2 * i + 1]) + bias[q4 * 32 + 2 * i + 1];
-                v0 = a0 * a0;
-                v1 = a1 * a1;
-              }
-              pk[i] = pack_bf16(v0, v1);
-            }
-          } else {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) pk[i] = 0u;
+        for (int i = 0; i < 16; ++i) {
+          uint64_t a = f2_add(f2_pack(__uint_as_float(ps[2 * i]), __uint_as_float(ps[2 * i + 1])),
+                              b2);
+          a = f2_fma(a, a, 0ull);
+          float v0, v1;
+          f2_unpack(a, v0, v1);
+          if (nvalid < 128) {  // tokens past the slice contribute nothing
+            const int t = c * 32 + 2 * i;
+            v0 = t < nvalid ? v0 : 0.f;
+            v1 = t + 1 < nvalid ? v1 : 0.f;
           }
-#pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) {
-            const int c = q4 * 4 + c4;  // 16-byte chunk of the 256-byte row
-            const uint32_t box = c >> 3, ch = c & 7;
-            st_shared_v4(base + kPhiOff + box * 16384 + r * 128 + ((ch ^ (r & 7)) << 4),
-                         pk[4 * c4], pk[4 * c4 + 1], pk[4 * c4 + 2], pk[4 * c4 + 3]);
-          }
+          pk[i] = pack_bf16(v0, v1);
+          // z sums the same bf16-rounded values that enter phi^T V.
+          zacc = f2_add(zacc, f2_pack(__uint_as_float(pk[i] << 16),
+                                      __uint_as_float(pk[i] & 0xFFFF0000u)));
         }
-        tc_fence_before();
-        mbar_arrive(bar(PSI_FREE));
-        if (nvalid < 128) {
-          ok = wait_all(bar(V_FULL + s), (gt >> 1) & 1, 38);
-          if (ok && !valid) {
-            const uint32_t vrow = base + kVOff + s * 32768 + r * 128;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              st_shared_v4(vrow + c * 16, 0, 0, 0, 0);
-              st_shared_v4(vrow + 16384 + c * 16, 0, 0, 0, 0);
-            }
-          }
+        REHYAT_TMEM_ST16(cols + c * 16, pk);
+      }
+      tmem_wait_st();
+      if (nvalid < 128) {
+        // V rows past the slice are zeroed so that 0 * V stays 0 for any V.
+        ok = wait_all(bar(V_FULL + st), (gt / kS) & 1, 37);
+        if (!ok) break;
+        const int nchunks = (128 - nvalid) * 16;
+        for (int i = f; i < nchunks; i += 128) {
+          const int row = nvalid + (i >> 4), ch = i & 15;
+          st_shared_v4(base + kVOff + st * 32768 + (ch >> 3) * 16384 + row * 128 + (ch & 7) * 16,
+                       0, 0, 0, 0);
         }
         fence_proxy_async();
-        tc_fence_before();
-        mbar_arrive(bar(PHI_FULL));
+      }
+      tc_fence_before();
+      mbar_arrive(bar(PHI_FULL + b));
+      if (j == nt - 1) {
+        float z0, z1;
+        f2_unpack(zacc, z0, z1);
+        if (f < pw) P.z[out_row(il) + f] = z0 + z1;
+        zacc = f2_pack(0.f, 0.f);
       }
     }
   } else if (warp < 8) {
     // ================================================= epilogue (thread = feature)
-    const int r = tid - 128;
+    const int f = tid - 128;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     bool ok = true;
     for (int il = 0; il < nitems && ok; ++il) {
@@ -1566,24 +1562,20 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(bar(ACC_DONE + pb), (il >> 1) & 1, abort_flag, 39));
       if (!ok) break;
       tc_fence_after();
-      // Feature row f = half * pw + r of slice (bh*T + slice).
-      const long long frow = slice_row_of(il) * Dp + ((it0 + il) / T) % halves * pw + r;
+      // Feature fg of the slice; the state is stored in the S^L image layout
+      // (a warp writes one 128-byte row per column).
+      const long long orow = out_row(il);  // slice * D' + half * pw
+      const int fg = static_cast<int>(orow % Dp) + f;
+      float* prow = P.P + (orow - orow % Dp) * 128 + sl_feature_base(fg, 128, Dp);
       for (int c = 0; c < 4; ++c) {
         uint32_t v[32];
         REHYAT_TMEM_LD32(lane_base + kColP + pb * 128 + c * 32, v);
         tmem_wait_ld();
-        if (r < pw) {
-          float4* dst = reinterpret_cast<float4*>(P.P + frow * 128 + c * 32);
+        if (f < pw) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                 __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+          for (int i = 0; i < 32; ++i) prow[sl_column_offset(fg, c * 32 + i)] = __uint_as_float(v[i]);
         }
       }
-      uint32_t zv[32];
-      REHYAT_TMEM_LD32(lane_base + kColZ + pb * 16, zv);
-      tmem_wait_ld();
-      if (r < pw) P.z[frow] = __uint_as_float(zv[0]);
       tc_fence_before();
       mbar_arrive(bar(P_FREE + pb));
     }

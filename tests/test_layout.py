@@ -1,6 +1,7 @@
 """Host-side check of the shared-memory image layouts (csrc/layout.cuh):
-sl_index is a bijection on [0, D*D') and sl_coords inverts it, and the
-weight image index is a bijection too, for every supported (D, D')."""
+sl_index is a bijection on [0, D*D'), sl_coords inverts it, the split form
+(feature base + column offset) agrees with it, and the weight image index is
+a bijection too, for every supported (D, D')."""
 import os
 import shutil
 import subprocess
@@ -27,6 +28,7 @@ int main() {
       int f2, d2;
       sl_coords(o, D, Dp, &f2, &d2);
       if (f2 != f || d2 != d) ++bad;
+      if (sl_feature_base(f, D, Dp) + sl_column_offset(f, d) != o) ++bad;
       if (D >= 64) {
         const long long w = wimg_index(f, d, D, Dp);
         if (w < 0 || w >= (long long)D * Dp) ++bad; else seen_w[w]++;
