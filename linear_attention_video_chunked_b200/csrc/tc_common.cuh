@@ -48,9 +48,11 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
 
 // Bounded wait on the phase with the given parity.  On timeout: record the
 // barrier in the global error word, raise the CTA abort flag, return false.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag,
-                                       uint32_t code) {
-  if (mbar_try(bar, parity)) return true;
+// The slow path is a real call; mbar_wait below tries inline first, so a
+// phase that has already completed costs no call (a call from a warp-
+// specialised thread spills its live registers around it).
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity,
+                                            volatile uint32_t* abort_flag, uint32_t code) {
   const long long t0 = clock64();
   for (uint32_t i = 0;; ++i) {
     if (mbar_try(bar, parity)) return true;
@@ -63,6 +65,14 @@ __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile u
       }
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
+                                          volatile uint32_t* abort_flag, uint32_t code) {
+#pragma unroll 1
+  for (int i = 0; i < 4; ++i)  // try_wait itself suspends the thread for a while
+    if (mbar_try(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, abort_flag, code);
 }
 
 __device__ __forceinline__ void fence_barrier_init() {
@@ -246,6 +256,27 @@ __device__ __forceinline__ void tmem_wait_ld() {
 }
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// tcgen05.wait::ld that also names the 32 destination registers of the load
+// it completes, so the compiler cannot move their uses above the wait (used
+// when a second load is in flight while the first one's values are used).
+#define REHYAT_TMEM_WAIT_LD32(r)                                                                \
+  asm volatile("tcgen05.wait::ld.sync.aligned;"                                                \
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),       \
+                 "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),     \
+                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), \
+                 "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), \
+                 "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), \
+                 "+r"(r[30]), "+r"(r[31])                                                      \
+               :                                                                               \
+               : "memory")
+
+// max(a, b, c) in one instruction (three-input form of max.f32).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 __device__ __forceinline__ float ex2(float x) {

@@ -526,6 +526,10 @@ constexpr int kThreads = 320;
 #define REHYAT_POLY_EVERY 0
 #endif
 constexpr int kPolyEvery = REHYAT_POLY_EVERY;
+#ifndef REHYAT_TRUNC_P
+#define REHYAT_TRUNC_P 0
+#endif
+constexpr bool kTruncP = REHYAT_TRUNC_P != 0;
 constexpr uint32_t kQOff = 0;                      // Q_A, Q_B
 constexpr uint32_t kKOff = 65536;                  // K ring, 3 x 32 KB
 constexpr uint32_t kVOff = kKOff + 3 * 32768;      // V ring, 2 x 32 KB
@@ -556,6 +560,7 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
   using a2::kTmemSlot;
   using a2::kAbortSlot;
   using a2::kPolyEvery;
+  using a2::kTruncP;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -775,30 +780,49 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const int nvalid = tile_src(j).nvalid;
-      // Pass 1: row max over S, streamed from TMEM 64 columns at a time (S
-      // never sits whole in registers, which would spill).
-      float mx[16];
+      const bool ragged = nvalid < kBN;  // warp-uniform: keys past the end
+      // S is streamed from TMEM 32 columns at a time through two register
+      // buffers: the next load is in flight while the current chunk is used
+      // (S never sits whole in registers, which would spill).
+      uint32_t xa[32], xb[32];
+      auto mask = [&](uint32_t* x, int c) {
+        if (ragged) {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) mx[i] = -INFINITY;
-#pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        uint32_t xr[64];
-        REHYAT_TMEM_LD32(lane_base + s_col + 64 * h2, xr);
-        REHYAT_TMEM_LD32(lane_base + s_col + 64 * h2 + 32, (xr + 32));
-        tmem_wait_ld();
-        if (nvalid < kBN) {  // ragged tile (warp-uniform): keys past the end
-#pragma unroll
-          for (int i = 0; i < 64; ++i)
-            if (64 * h2 + i >= nvalid) xr[i] = __float_as_uint(-INFINITY);
+          for (int i = 0; i < 32; ++i)
+            if (32 * c + i >= nvalid) x[i] = __float_as_uint(-INFINITY);
         }
+      };
+      float mx[8];
 #pragma unroll
-        for (int i = 0; i < 64; ++i) mx[i & 15] = fmaxf(mx[i & 15], __uint_as_float(xr[i]));
-      }
+      for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
+      auto max_chunk = [&](const uint32_t* x) {
 #pragma unroll
-      for (int w = 8; w >= 1; w >>= 1)
-#pragma unroll
-        for (int i = 0; i < w; ++i) mx[i] = fmaxf(mx[i], mx[i + w]);
-      m_max = fmaxf(m_max, mx[0] * P.scale_log2);
+        for (int i = 0; i < 8; ++i)
+          mx[i] = fmax3(mx[i], fmax3(__uint_as_float(x[i]), __uint_as_float(x[i + 8]),
+                                     __uint_as_float(x[i + 16])),
+                        __uint_as_float(x[i + 24]));
+      };
+      // Pass 1: row max.
+      REHYAT_TMEM_LD32(lane_base + s_col, xa);
+      REHYAT_TMEM_WAIT_LD32(xa);
+      REHYAT_TMEM_LD32(lane_base + s_col + 32, xb);
+      mask(xa, 0);
+      max_chunk(xa);
+      REHYAT_TMEM_WAIT_LD32(xb);
+      REHYAT_TMEM_LD32(lane_base + s_col + 64, xa);
+      mask(xb, 1);
+      max_chunk(xb);
+      REHYAT_TMEM_WAIT_LD32(xa);
+      REHYAT_TMEM_LD32(lane_base + s_col + 96, xb);
+      mask(xa, 2);
+      max_chunk(xa);
+      REHYAT_TMEM_WAIT_LD32(xb);
+      REHYAT_TMEM_LD32(lane_base + s_col, xa);  // pass 2, chunk 0
+      mask(xb, 3);
+      max_chunk(xb);
+      m_max = fmaxf(m_max, fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
+                                 fmaxf(mx[6], mx[7])) *
+                               P.scale_log2);
       float alpha = 1.f;
       const bool rescale = m_max > m_used + 8.f;
       if (rescale) {
@@ -811,23 +835,15 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
       const uint64_t scale2 = f2_pack(P.scale_log2, P.scale_log2);
       const uint64_t negm2 = f2_pack(-m_used, -m_used);
       uint64_t ls2[4] = {0, 0, 0, 0};
-      // Pass 2: re-read S 32 columns at a time and write P (bf16 pairs) over
-      // the S columns already consumed: P piece c lands in [16c, 16c + 16).
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t xr[32];
-        REHYAT_TMEM_LD32(lane_base + s_col + 32 * c, xr);
-        tmem_wait_ld();
-        if (nvalid < kBN) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (32 * c + i >= nvalid) xr[i] = __float_as_uint(-INFINITY);
-        }
+      // Pass 2: P (bf16 pairs) of chunk c is written over S columns already
+      // consumed, [16c, 16c + 16), while chunk c + 1 is being loaded.
+      auto exp_chunk = [&](uint32_t* x, int c) {
+        mask(x, c);
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(xr[2 * i]),
-                                             __uint_as_float(xr[2 * i + 1])),
+          const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(x[2 * i]),
+                                             __uint_as_float(x[2 * i + 1])),
                                      scale2, negm2);
           uint64_t p2;
           if (kPolyEvery > 0 && (i % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
@@ -839,11 +855,32 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
           }
           float p0, p1;
           f2_unpack(p2, p0, p1);
-          pk[i] = pack_bf16(p0, p1);
-          ls2[i & 3] = f2_add(ls2[i & 3], p2);
+          if (kTruncP) {
+            // bf16 by truncation (one byte permute on the ALU pipe instead of
+            // a conversion on the pipe that also runs ex2); the row sum takes
+            // the same truncated values, so P.V and l stay consistent.
+            const uint32_t u0 = __float_as_uint(p0), u1 = __float_as_uint(p1);
+            pk[i] = __byte_perm(u0, u1, 0x7632);
+            ls2[i & 3] = f2_add(ls2[i & 3], f2_pack(__uint_as_float(u0 & 0xFFFF0000u),
+                                                    __uint_as_float(u1 & 0xFFFF0000u)));
+          } else {
+            pk[i] = pack_bf16(p0, p1);
+            ls2[i & 3] = f2_add(ls2[i & 3], p2);
+          }
         }
         REHYAT_TMEM_ST16(lane_base + s_col + c * 16, pk);
-      }
+      };
+      REHYAT_TMEM_WAIT_LD32(xa);
+      REHYAT_TMEM_LD32(lane_base + s_col + 32, xb);
+      exp_chunk(xa, 0);
+      REHYAT_TMEM_WAIT_LD32(xb);
+      REHYAT_TMEM_LD32(lane_base + s_col + 64, xa);
+      exp_chunk(xb, 1);
+      REHYAT_TMEM_WAIT_LD32(xa);
+      REHYAT_TMEM_LD32(lane_base + s_col + 96, xb);
+      exp_chunk(xa, 2);
+      REHYAT_TMEM_WAIT_LD32(xb);
+      exp_chunk(xb, 3);
       float ls[8];
       f2_unpack(f2_add(ls2[0], ls2[1]), ls[0], ls[1]);
       f2_unpack(f2_add(ls2[2], ls2[3]), ls[2], ls[3]);
