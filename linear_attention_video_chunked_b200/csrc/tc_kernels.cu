@@ -1354,6 +1354,35 @@ constexpr uint32_t kTmemSlot = kBarOff + 8 * NBAR;
 constexpr uint32_t kAbortSlot = kTmemSlot + 4;
 constexpr uint32_t kSmemBytes = kBarOff + 256 + 1024;
 constexpr uint32_t kColBuf = 0, kColP = 256;
+
+// Walk over a CTA's run of items i = q * T + slice, q = bh * halves + half,
+// with a division only when one (bh, half) run of slices ends.
+struct ItemWalk {
+  int T, halves, heads, pw;
+  int slice = 0, q = 0;
+  int wkey = 0;       // (head, half) key of the W_k piece the item needs
+  bool wnew = true;   // first item, or wkey differs from the previous item's
+  __device__ int bh() const { return halves == 2 ? q >> 1 : q; }
+  __device__ int half() const { return q - bh() * halves; }
+  __device__ int key() const { return (bh() % heads) * halves + half(); }
+  __device__ long long slice_index() const { return static_cast<long long>(bh()) * T + slice; }
+  __device__ void start(int item) {
+    slice = item % T;
+    q = item / T;
+    wkey = key();
+    wnew = true;
+  }
+  __device__ void next() {
+    wnew = false;
+    if (++slice == T) {
+      slice = 0;
+      ++q;
+      const int k = key();
+      wnew = k != wkey;
+      wkey = k;
+    }
+  }
+};
 }  // namespace sp
 
 __global__ void __launch_bounds__(sp::kThreads, 1)
@@ -1392,18 +1421,6 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
   const int nitems = it1 - it0;
   const int nt = (HW + 127) / 128;
   const int TT = nitems * nt;  // token tiles of this CTA
-  // Item i = (bh, half, slice) in that order; the W_k piece (and b_k) an
-  // item needs is keyed by (head, half).
-  auto wkey_of = [&](int il) {
-    const int i = it0 + il, bh = i / (halves * T), hf = (i / T) % halves;
-    return (bh % P.heads) * halves + hf;
-  };
-  auto new_w = [&](int il) { return il == 0 || wkey_of(il) != wkey_of(il - 1); };
-  // First output row (feature half * pw of slice bh * T + slice) of item il.
-  auto out_row = [&](int il) {
-    const int i = it0 + il;
-    return (static_cast<long long>(i / (halves * T)) * T + i % T) * Dp + (i / T) % halves * pw;
-  };
 
   if (tid == 0) {
     for (int i = 0; i < NBAR; ++i) {
@@ -1439,32 +1456,38 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
       bool ok = true;
       int wloads = 0;
       const uint32_t box_bytes = static_cast<uint32_t>(pw) * 128;  // one 64-column box
-      for (int il = 0; il < nitems && ok; ++il) {
-        const int item = it0 + il, bh = item / (halves * T), slice = item % T;
-        if (new_w(il)) {
+      sp::ItemWalk w{T, halves, P.heads, pw};
+      w.start(it0);
+      int gt = 0, st = 0, uses = 0;  // tile index, its ring stage, earlier uses of the stage
+      for (int il = 0; il < nitems && ok; ++il, w.next()) {
+        if (w.wnew) {
           if (il > 0) ok = mbar_wait(bar(W_FREE), (wloads - 1) & 1, abort_flag, 27);
           if (!ok) break;
           // Head h's image holds its D' features as pieces of pw rows, each
           // piece two boxes of pw rows x 64 columns.
-          const __nv_bfloat16* src = wk_img + static_cast<long long>(wkey_of(il)) * pw * 128;
+          const __nv_bfloat16* src = wk_img + static_cast<long long>(w.wkey) * pw * 128;
           mbar_expect_tx(bar(W_FULL), 2 * box_bytes);
           bulk_load(base + kWOff, src, box_bytes, bar(W_FULL));
           bulk_load(base + kWOff + 16384, src + pw * 64, box_bytes, bar(W_FULL));
           ++wloads;
         }
-        for (int j = 0; j < nt && ok; ++j) {
-          const int gt = il * nt + j, st = gt % kS, ph = ((gt - kS) / kS) & 1;
-          const int row = slice * HW + j * 128;
-          if (gt >= kS) ok = mbar_wait(bar(K_EMPTY + st), ph, abort_flag, 28);
+        const int bh = w.bh(), row0 = w.slice * HW;
+        for (int j = 0; j < nt && ok; ++j, ++gt) {
+          const int row = row0 + j * 128;
+          if (gt >= kS) ok = mbar_wait(bar(K_EMPTY + st), (uses - 1) & 1, abort_flag, 28);
           if (!ok) break;
           mbar_expect_tx(bar(K_FULL + st), 32768);
           tma_load_3d(base + kKOff + st * 32768, &maps.k, bar(K_FULL + st), 0, row, bh);
           tma_load_3d(base + kKOff + st * 32768 + 16384, &maps.k, bar(K_FULL + st), 64, row, bh);
-          if (gt >= kS) ok = mbar_wait(bar(V_EMPTY + st), ph, abort_flag, 29);
+          if (gt >= kS) ok = mbar_wait(bar(V_EMPTY + st), (uses - 1) & 1, abort_flag, 29);
           if (!ok) break;
           mbar_expect_tx(bar(V_FULL + st), 32768);
           tma_load_3d(base + kVOff + st * 32768, &maps.v, bar(V_FULL + st), 0, row, bh);
           tma_load_3d(base + kVOff + st * 32768 + 16384, &maps.v, bar(V_FULL + st), 64, row, bh);
+          if (++st == kS) {
+            st = 0;
+            ++uses;
+          }
         }
       }
     }
@@ -1476,48 +1499,72 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
       const uint32_t id_pv = idesc(128, 128, 1, true);    // phi^T from TMEM, V MN-major
       bool ok = true;
       int wwaits = 0;
-      // psi^T for token tile gt into buffer gt & 1: waits for its K tile,
-      // for phi^T V of tile gt - 2 to have read that buffer, and for W_k.
-      auto issue_psi = [&](int gt) -> bool {
-        const int il = gt / nt, b = gt & 1, st = gt % kS;
-        if (gt % nt == 0 && new_w(il)) {
-          if (il > 0) mma_commit(bar(W_FREE));  // tracks every earlier MMA
+      // The next psi^T to issue: its tile index, item walk, tile in item,
+      // K stage and earlier uses of that stage.
+      sp::ItemWalk wp{T, halves, P.heads, pw};
+      wp.start(it0);
+      int pgt = 0, pj = 0, pst = 0, puses = 0;
+      // psi^T for token tile pgt into buffer pgt & 1: waits for its K tile,
+      // for phi^T V of tile pgt - 2 to have read that buffer, and for W_k.
+      auto issue_psi = [&]() -> bool {
+        const int b = pgt & 1;
+        if (pj == 0 && wp.wnew) {
+          if (pgt > 0) mma_commit(bar(W_FREE));  // tracks every earlier MMA
           if (!mbar_wait(bar(W_FULL), wwaits & 1, abort_flag, 30)) return false;
           ++wwaits;
         }
-        if (!mbar_wait(bar(K_FULL + st), (gt / kS) & 1, abort_flag, 31)) return false;
-        if (gt >= 2 && !mbar_wait(bar(BUF_FREE + b), ((gt - 2) >> 1) & 1, abort_flag, 32))
+        if (!mbar_wait(bar(K_FULL + pst), puses & 1, abort_flag, 31)) return false;
+        if (pgt >= 2 && !mbar_wait(bar(BUF_FREE + b), ((pgt - 2) >> 1) & 1, abort_flag, 32))
           return false;
         tc_fence_after();
+        const uint64_t wdesc = sdesc(base + kWOff, 16, 1024);
+        const uint64_t kdesc = sdesc(base + kKOff + pst * 32768, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_bf16(tmem + kColBuf + b * 128, sdesc(base + kWOff + off, 16, 1024),
-                   sdesc(base + kKOff + st * 32768 + off, 16, 1024), id_psi, kk > 0);
+          // Descriptor start addresses are in 16-byte units (no carry: < 2^14).
+          const uint64_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+          mma_bf16(tmem + kColBuf + b * 128, wdesc + off, kdesc + off, id_psi, kk > 0);
         }
         mma_commit(bar(PSI_FULL + b));
-        mma_commit(bar(K_EMPTY + st));
+        mma_commit(bar(K_EMPTY + pst));
+        ++pgt;
+        if (++pst == kS) {
+          pst = 0;
+          ++puses;
+        }
+        if (++pj == nt) {
+          pj = 0;
+          wp.next();
+        }
         return true;
       };
-      ok = issue_psi(0);
-      for (int gt = 0; gt < TT && ok; ++gt) {
-        const int il = gt / nt, j = gt % nt, b = gt & 1, st = gt % kS, pb = il & 1;
-        if (gt + 1 < TT) ok = issue_psi(gt + 1);
-        if (!ok) break;
-        if (j == 0 && il >= 2)
-          ok = mbar_wait(bar(P_FREE + pb), ((il - 2) >> 1) & 1, abort_flag, 33);
-        if (ok) ok = mbar_wait(bar(PHI_FULL + b), (gt >> 1) & 1, abort_flag, 34) &&
-                     mbar_wait(bar(V_FULL + st), (gt / kS) & 1, abort_flag, 35);
-        if (!ok) break;
-        tc_fence_after();
+      ok = issue_psi();
+      int gt = 0, vst = 0, vuses = 0;
+      for (int il = 0; il < nitems && ok; ++il) {
+        const int pb = il & 1;
+        for (int j = 0; j < nt && ok; ++j, ++gt) {
+          const int b = gt & 1;
+          if (gt + 1 < TT) ok = issue_psi();
+          if (!ok) break;
+          if (j == 0 && il >= 2)
+            ok = mbar_wait(bar(P_FREE + pb), ((il - 2) >> 1) & 1, abort_flag, 33);
+          if (ok) ok = mbar_wait(bar(PHI_FULL + b), (gt >> 1) & 1, abort_flag, 34) &&
+                       mbar_wait(bar(V_FULL + vst), vuses & 1, abort_flag, 35);
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t vdesc = sdesc(base + kVOff + vst * 32768, 16384, 1024);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts(tmem + kColP + pb * 128, tmem + kColBuf + b * 128 + kk * 8,
-                      sdesc(base + kVOff + st * 32768 + kk * 2048, 16384, 1024), id_pv,
-                      (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(bar(BUF_FREE + b));
-        mma_commit(bar(V_EMPTY + st));
-        if (j == nt - 1) mma_commit(bar(ACC_DONE + pb));
+          for (int kk = 0; kk < 8; ++kk)
+            mma_bf16_ts(tmem + kColP + pb * 128, tmem + kColBuf + b * 128 + kk * 8,
+                        vdesc + ((kk * 2048) >> 4), id_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(bar(BUF_FREE + b));
+          mma_commit(bar(V_EMPTY + vst));
+          if (j == nt - 1) mma_commit(bar(ACC_DONE + pb));
+          if (++vst == kS) {
+            vst = 0;
+            ++vuses;
+          }
+        }
       }
     }
     __syncwarp();
@@ -1531,61 +1578,70 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
     bool ok = true;
     float bias = 0.f;
     uint64_t zacc = f2_pack(0.f, 0.f);  // z over even / odd tokens
-    for (int gt = 0; gt < TT && ok; ++gt) {
-      const int il = gt / nt, j = gt % nt, b = gt & 1, st = gt % kS;
+    sp::ItemWalk w{T, halves, P.heads, pw};
+    w.start(it0);
+    int gt = 0, vst = 0, vuses = 0;
+    for (int il = 0; il < nitems && ok; ++il, w.next()) {
       // b_k of head h is h's D' consecutive features.
-      if (j == 0 && new_w(il)) bias = f < pw ? P.bk[wkey_of(il) * pw + f] : 0.f;
-      ok = wait_all(bar(PSI_FULL + b), (gt >> 1) & 1, 36);
-      if (!ok) break;
-      tc_fence_after();
-      const int nvalid = min(128, HW - j * 128);
-      const uint32_t cols = lane_base + kColBuf + b * 128;
+      if (w.wnew) bias = f < pw ? P.bk[w.wkey * pw + f] : 0.f;
       const uint64_t b2 = f2_pack(bias, bias);
-      // 32 tokens at a time: phi of tokens 32c.. is written as 16 packed
-      // columns at 16c, behind the columns already read.
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t ps[32], pk[16];
-        REHYAT_TMEM_LD32(cols + c * 32, ps);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          uint64_t a = f2_add(f2_pack(__uint_as_float(ps[2 * i]), __uint_as_float(ps[2 * i + 1])),
-                              b2);
-          a = f2_fma(a, a, 0ull);
-          float v0, v1;
-          f2_unpack(a, v0, v1);
-          if (nvalid < 128) {  // tokens past the slice contribute nothing
-            const int t = c * 32 + 2 * i;
-            v0 = t < nvalid ? v0 : 0.f;
-            v1 = t + 1 < nvalid ? v1 : 0.f;
-          }
-          pk[i] = pack_bf16(v0, v1);
-          // z sums the same bf16-rounded values that enter phi^T V.
-          zacc = f2_add(zacc, f2_pack(__uint_as_float(pk[i] << 16),
-                                      __uint_as_float(pk[i] & 0xFFFF0000u)));
-        }
-        REHYAT_TMEM_ST16(cols + c * 16, pk);
-      }
-      tmem_wait_st();
-      if (nvalid < 128) {
-        // V rows past the slice are zeroed so that 0 * V stays 0 for any V.
-        ok = wait_all(bar(V_FULL + st), (gt / kS) & 1, 37);
+      for (int j = 0; j < nt && ok; ++j, ++gt) {
+        const int b = gt & 1;
+        ok = wait_all(bar(PSI_FULL + b), (gt >> 1) & 1, 36);
         if (!ok) break;
-        const int nchunks = (128 - nvalid) * 16;
-        for (int i = f; i < nchunks; i += 128) {
-          const int row = nvalid + (i >> 4), ch = i & 15;
-          st_shared_v4(base + kVOff + st * 32768 + (ch >> 3) * 16384 + row * 128 + (ch & 7) * 16,
-                       0, 0, 0, 0);
+        tc_fence_after();
+        const int nvalid = min(128, HW - j * 128);
+        const uint32_t cols = lane_base + kColBuf + b * 128;
+        // 32 tokens at a time: phi of tokens 32c.. is written as 16 packed
+        // columns at 16c, behind the columns already read.
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t ps[32], pk[16];
+          REHYAT_TMEM_LD32(cols + c * 32, ps);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            uint64_t a = f2_add(
+                f2_pack(__uint_as_float(ps[2 * i]), __uint_as_float(ps[2 * i + 1])), b2);
+            a = f2_fma(a, a, 0ull);
+            float v0, v1;
+            f2_unpack(a, v0, v1);
+            if (nvalid < 128) {  // tokens past the slice contribute nothing
+              const int t = c * 32 + 2 * i;
+              v0 = t < nvalid ? v0 : 0.f;
+              v1 = t + 1 < nvalid ? v1 : 0.f;
+            }
+            pk[i] = pack_bf16(v0, v1);
+            // z sums the same bf16-rounded values that enter phi^T V.
+            zacc = f2_add(zacc, f2_pack(__uint_as_float(pk[i] << 16),
+                                        __uint_as_float(pk[i] & 0xFFFF0000u)));
+          }
+          REHYAT_TMEM_ST16(cols + c * 16, pk);
         }
-        fence_proxy_async();
+        tmem_wait_st();
+        if (nvalid < 128) {
+          // V rows past the slice are zeroed so that 0 * V stays 0 for any V.
+          ok = wait_all(bar(V_FULL + vst), vuses & 1, 37);
+          if (!ok) break;
+          const int nchunks = (128 - nvalid) * 16;
+          for (int i = f; i < nchunks; i += 128) {
+            const int row = nvalid + (i >> 4), ch = i & 15;
+            st_shared_v4(base + kVOff + vst * 32768 + (ch >> 3) * 16384 + row * 128 + (ch & 7) * 16,
+                         0, 0, 0, 0);
+          }
+          fence_proxy_async();
+        }
+        tc_fence_before();
+        mbar_arrive(bar(PHI_FULL + b));
+        if (++vst == kS) {
+          vst = 0;
+          ++vuses;
+        }
       }
-      tc_fence_before();
-      mbar_arrive(bar(PHI_FULL + b));
-      if (j == nt - 1) {
+      if (ok) {
         float z0, z1;
         f2_unpack(zacc, z0, z1);
-        if (f < pw) P.z[out_row(il) + f] = z0 + z1;
+        if (f < pw) P.z[w.slice_index() * Dp + w.half() * pw + f] = z0 + z1;
         zacc = f2_pack(0.f, 0.f);
       }
     }
@@ -1594,16 +1650,17 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
     const int f = tid - 128;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     bool ok = true;
-    for (int il = 0; il < nitems && ok; ++il) {
+    sp::ItemWalk w{T, halves, P.heads, pw};
+    w.start(it0);
+    for (int il = 0; il < nitems && ok; ++il, w.next()) {
       const int pb = il & 1;
       ok = __all_sync(0xffffffffu, mbar_wait(bar(ACC_DONE + pb), (il >> 1) & 1, abort_flag, 39));
       if (!ok) break;
       tc_fence_after();
       // Feature fg of the slice; the state is stored in the S^L image layout
       // (a warp writes one 128-byte row per column).
-      const long long orow = out_row(il);  // slice * D' + half * pw
-      const int fg = static_cast<int>(orow % Dp) + f;
-      float* prow = P.P + (orow - orow % Dp) * 128 + sl_feature_base(fg, 128, Dp);
+      const int fg = w.half() * pw + f;
+      float* prow = P.P + w.slice_index() * Dp * 128 + sl_feature_base(fg, 128, Dp);
       for (int c = 0; c < 4; ++c) {
         uint32_t v[32];
         REHYAT_TMEM_LD32(lane_base + kColP + pb * 128 + c * 32, v);
