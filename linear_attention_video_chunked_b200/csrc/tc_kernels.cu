@@ -540,10 +540,12 @@ constexpr uint32_t kPhiOff0 = kVOff;               // tail: phi_q(Q_A)/f (<= 64 
 constexpr uint32_t kPhiOff1 = kQOff;               // tail: phi_q(Q_B)/f, over Q (<= 64 KB)
 enum { Q_FULL = 0, K_FULL = 1, K_EMPTY = 4, V_FULL = 7, V_EMPTY = 9, S_FULL = 11, P_FULL = 13,
        PV_DONE = 15, LAST_PV = 17, TAIL_FULL = 18, PHI_DONE = 19, PHI_READY = 20, READ_DONE = 22,
-       NBAR = 23 };
+       VEC_READY = 23, NBAR = 24 };
 constexpr uint32_t kTmemSlot = kBarOff + 8 * NBAR;
 constexpr uint32_t kAbortSlot = kTmemSlot + 4;
-constexpr uint32_t kSmemBytes = kBarOff + 256 + 1024;
+// b_q of the head and z^L of the chunk (D' floats each), shared by both tiles.
+constexpr uint32_t kVecOff = kBarOff + 256;
+constexpr uint32_t kSmemBytes = kVecOff + 1024 + 1024;
 }  // namespace a2
 
 __global__ void __launch_bounds__(a2::kThreads, 1)
@@ -624,7 +626,7 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
   if (tid == 0) {
     for (int i = 0; i < a2::NBAR; ++i) {
       const bool by_warpgroup = i == a2::P_FULL || i == a2::P_FULL + 1 || i == a2::PHI_READY ||
-                                i == a2::PHI_READY + 1;
+                                i == a2::PHI_READY + 1 || i == a2::VEC_READY;
       mbar_init(bar(i), by_warpgroup ? kSoftmaxThreads : 1);
     }
     *abort_flag = 0;
@@ -670,7 +672,11 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
       if (linear && ok) {
         const uint32_t wbytes = static_cast<uint32_t>(Dp) * kD * 2;
         const uint32_t slbytes = static_cast<uint32_t>(Dp) * kD * 4;
-        ok = mbar_wait(bar(a2::LAST_PV), 0, abort_flag, 2);
+        // The tail operands go into the K ring as soon as the last three K
+        // tiles have been consumed (their q.k^T MMAs completed), while the
+        // last softmax steps and P.V still run.
+        for (int tt = max(0, nt - 3); tt < nt && ok; ++tt)
+          ok = mbar_wait(bar(a2::K_EMPTY + tt % 3), (tt / 3) & 1, abort_flag, 2);
         if (ok) {
           mbar_expect_tx(bar(a2::TAIL_FULL), wbytes + slbytes);
           bulk_load(base + kWOff, wq_img + static_cast<long long>(h) * Dp * kD, wbytes,
@@ -774,6 +780,16 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
     auto wait_all = [&](uint32_t b, uint32_t parity, uint32_t code) {
       return __all_sync(0xffffffffu, mbar_wait(b, parity, abort_flag, code));
     };
+    float* vec = reinterpret_cast<float*>(sbase + a2::kVecOff);  // [b_q (D') | z^L (D')]
+    if (linear && tile == 0) {
+      // Tile A's warpgroup stages b_q and z^L for the tail while it waits
+      // for the first scores (b_q of head h is h's D' consecutive values).
+      if (r < Dp) {
+        vec[r] = __ldg(P.bq + h * Dp + r);
+        vec[Dp + r] = __ldg(P.zL + (static_cast<long long>(bh) * P.nchunks + t) * Dp + r);
+      }
+      mbar_arrive(bar(a2::VEC_READY));
+    }
     for (int j = 0; j < nt && ok; ++j) {
       // S_FULL(j) also covers this tile's P.V of step j-1 (issued earlier).
       ok = wait_all(bar(a2::S_FULL + tile), j & 1, 11);
@@ -942,11 +958,10 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
           }
         }
       }
-      if (ok) ok = wait_all(bar(a2::PHI_DONE), 0, 14);
+      if (ok) ok = wait_all(bar(a2::VEC_READY), 0, 14) && wait_all(bar(a2::PHI_DONE), 0, 14);
       if (ok) {
         tc_fence_after();
         const float inv_f = 1.0f / fscale;
-        const float* zL = P.zL + (static_cast<long long>(bh) * P.nchunks + t) * Dp;
         const uint32_t phi = base + (tile ? kPhiOff1 : kPhiOff0);
         for (int c = 0; c < Dp / 32; ++c) {
           uint32_t v[32];
@@ -956,11 +971,9 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const int f = c * 32 + i;
-            const int part = f >= (Dp >> 1);
-            const float b = __ldg(P.bq + (h * 2 + part) * (Dp >> 1) + (f - part * (Dp >> 1)));
-            const float psi = __uint_as_float(v[i]) + b;
+            const float psi = __uint_as_float(v[i]) + vec[f];
             ph[i] = psi * psi;
-            nL = fmaf(ph[i], __ldg(zL + f), nL);
+            nL = fmaf(ph[i], vec[Dp + f], nL);
             ph[i] *= inv_f;
           }
           const uint32_t rowaddr = phi + c * 16384 + r * 128;
@@ -982,6 +995,9 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
       tc_fence_after();
       const float nS = l * fscale;
       const float den = nS + nL;
+      // y = f * O / den: one IEEE division per row, then a product per value.
+      const float ysc = __fdiv_rn(fscale, den);
+      const bool dbg_num = P.dbg_aL != nullptr || (P.dbg_aS != nullptr && !linear);
       for (int c = 0; c < 4; ++c) {
         uint32_t o[32];
         REHYAT_TMEM_LD32(lane_base + o_col + c * 32, o);
@@ -989,14 +1005,16 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
         if (r < nrows) {
           float yv[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float num = __uint_as_float(o[i]) * fscale;  // a^S + a^L
-            yv[i] = __fdiv_rn(num, den);
-            if (P.dbg_aL) {
-              float* d = P.dbg_aL + grow * kD + c * 32 + i;
-              *d = linear ? num - *d : 0.f;
+          for (int i = 0; i < 32; ++i) yv[i] = __uint_as_float(o[i]) * ysc;
+          if (dbg_num) {
+            for (int i = 0; i < 32; ++i) {
+              const float num = __uint_as_float(o[i]) * fscale;  // a^S + a^L
+              if (P.dbg_aL) {
+                float* d = P.dbg_aL + grow * kD + c * 32 + i;
+                *d = linear ? num - *d : 0.f;
+              }
+              if (P.dbg_aS && !linear) P.dbg_aS[grow * kD + c * 32 + i] = num;
             }
-            if (P.dbg_aS && !linear) P.dbg_aS[grow * kD + c * 32 + i] = num;
           }
           if (P.out_bf16) {
             uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(P.y) + grow * kD +
