@@ -178,8 +178,9 @@ REHYAT_API rehyat_status rehyat_softmax_attn_fwd(const rehyat_params* p, const v
 
 /* Bytes of the opaque streaming state: the running s [B][h][Dp][D] and
  * z [B][h][Dp] (fp32), a ring holding the keys and values of the last T_o
- * slices (in_dtype), and a device-side count of slices consumed.  Constant
- * for any number of steps. */
+ * slices (in_dtype), and a device-side count of slices consumed (with a
+ * completion count that is zero between steps).  Constant for any number of
+ * steps; a copy taken between steps restores the stream exactly. */
 REHYAT_API size_t rehyat_state_bytes(const rehyat_params* p);
 
 /* Reset a state to the start of a video: s = 0, z = 0, empty ring. */

@@ -69,17 +69,15 @@ bool tc_path(const rehyat_params* p) {
 }
 
 // Whether the tensor-core per-slice state kernel is used.
-// `step` selects the chunk-step fold (a window of slices per call) rather
-// than the full forward's per-slice sums.
-bool tc_state_path(const rehyat_params* p, bool step) {
+bool tc_state_path(const rehyat_params* p) {
   return !(p->flags & REHYAT_FLAG_FORCE_SIMT) &&
-         tc_state_eligible(p->in_dtype == REHYAT_BF16, p->D, p->Dp, step);
+         tc_state_eligible(p->in_dtype == REHYAT_BF16, p->D, p->Dp);
 }
 
 // Per-slice states on the path these params select.
 cudaError_t run_partials(const rehyat_params* p, const PartialParams& pp, const void* wk_img,
                          cudaStream_t s) {
-  if (tc_state_path(p, pp.seen != nullptr)) return launch_state_tc(pp, wk_img, s);
+  if (tc_state_path(p)) return launch_state_tc(pp, wk_img, s);
   return launch_partials_simt(pp, s);
 }
 
@@ -87,11 +85,16 @@ struct StateLayout {
   size_t s_off, z_off, rk_off, rv_off, total;
 };
 
+// Streaming state header (kAlign bytes, zeroed by rehyat_state_init): the
+// int64 count of slices consumed at offset 0, and at kStepDoneOffset the
+// uint32 completion count the step-finish kernel uses (0 between steps).
+constexpr size_t kStepDoneOffset = 64;
+
 StateLayout state_layout(const rehyat_params* p) {
   const size_t BH = static_cast<size_t>(p->batch) * p->heads;
   const size_t HW = static_cast<size_t>(p->Hs) * p->Ws;
   StateLayout s;
-  s.s_off = kAlign;  // header: the slice counter (int64)
+  s.s_off = kAlign;  // header: slice counter, step completion count
   s.z_off = align_up(s.s_off + BH * p->Dp * p->D * sizeof(float));
   s.rk_off = align_up(s.z_off + BH * p->Dp * sizeof(float));
   const size_t ring = BH * p->To * HW * p->D * elem_bytes(p->in_dtype);
@@ -237,7 +240,7 @@ rehyat_status rehyat_fwd_state(const rehyat_params* p, const void* k, const void
   pp.in_bf16 = p->in_dtype == REHYAT_BF16;
   pp.w_bf16 = pp.in_bf16;
   cudaError_t e = cudaSuccess;
-  if (tc_path(p) || tc_state_path(p, false))
+  if (tc_path(p) || tc_state_path(p))
     e = launch_w_images(phi->Wq, ws + w.wimg_off, phi->Wk, ws + w.wkimg_off, p->heads, p->D,
                         p->Dp, s);
   if (e != cudaSuccess) return to_status(e);
@@ -369,7 +372,7 @@ rehyat_status rehyat_chunk_step(const rehyat_params* p, const void* q, const voi
   a.nchunks = 1;
   a.nq_slices = nslices;
   cudaError_t e = cudaSuccess;
-  if (tc_path(p) || tc_state_path(p, true)) {
+  if (tc_path(p) || tc_state_path(p)) {
     e = launch_w_images(phi->Wq, ws + w.wimg_off, phi->Wk, ws + w.wkimg_off, p->heads, p->D,
                         p->Dp, s);
     if (e != cudaSuccess) return to_status(e);
@@ -394,14 +397,12 @@ rehyat_status rehyat_chunk_step(const rehyat_params* p, const void* q, const voi
   pp.w_bf16 = pp.in_bf16;
   e = run_partials(p, pp, ws + w.wkimg_off, s);
   if (e != cudaSuccess) return to_status(e);
-  e = launch_state_add(P, zp, s_state, z_state, seen, BH, p->Dp, p->D, p->To, nslices,
-                       w.nslots, s);
-  if (e != cudaSuccess) return to_status(e);
-  // 3. Keep the newest T_o slices in the ring; 4. advance the counter.
-  e = launch_ring_update(k, v, rk, rv, seen, BH, HW, p->D, p->To, nslices,
-                         elem_bytes(p->in_dtype), s);
-  if (e != cudaSuccess) return to_status(e);
-  return to_status(launch_advance(seen, nslices, s));
+  // 3. Add them into (s, z), keep the newest T_o slices in the ring and
+  // advance the counter, in one launch.
+  unsigned* done = reinterpret_cast<unsigned*>(stb + kStepDoneOffset);
+  return to_status(launch_step_finish(P, zp, s_state, z_state, seen, done, BH, p->Dp, p->D,
+                                      p->To, nslices, w.nslots, k, v, rk, rv, HW,
+                                      elem_bytes(p->in_dtype), s));
 }
 
 }  // extern "C"

@@ -69,7 +69,7 @@ bool tc_attn_eligible(int in_bf16, int D, int Dp);
 
 // Tensor-core per-slice state (bf16, D = 128, Dp in {64, 128}); wk_img is
 // the bf16 image of W_k.
-bool tc_state_eligible(int in_bf16, int D, int Dp, bool step);
+bool tc_state_eligible(int in_bf16, int D, int Dp);
 cudaError_t launch_state_tc(const PartialParams& p, const void* wk_img, cudaStream_t s);
 
 // Linear-set state per chunk from the per-slice states (full mode).
@@ -81,15 +81,13 @@ cudaError_t launch_scan(const float* P, const float* z, float* SL, float* zL,
                         int D, int causal, cudaStream_t s);
 
 // Streaming helpers (step mode; all read the device slice counter).
-cudaError_t launch_state_add(const float* P, const float* zp, float* s_state,
-                             float* z_state, const long long* seen, int BH,
-                             int Dp, int D, int To, int nq_slices, int nslots,
-                             cudaStream_t s);
-cudaError_t launch_ring_update(const void* k, const void* v, void* rk, void* rv,
-                               const long long* seen, int BH, int HW, int D,
-                               int To, int nq_slices, int elem_bytes,
-                               cudaStream_t s);
-cudaError_t launch_advance(long long* seen, int nq_slices, cudaStream_t s);
+// End of a streaming step: fold the leaving slices' states into (s, z), copy
+// the staying chunk slices into the ring, advance the slice counter (done:
+// a zeroed completion count in the state header, reset by the kernel).
+cudaError_t launch_step_finish(const float* P, const float* zp, float* s_state, float* z_state,
+                               long long* seen, unsigned* done, int BH, int Dp, int D, int To,
+                               int nq_slices, int nslots, const void* k, const void* v, void* rk,
+                               void* rv, int HW, int elem_bytes, cudaStream_t s);
 
 // ---- tcgen05 / TMA kernels (bf16, D = 128).  Return cudaErrorNotSupported
 // when the shape is outside what they handle.

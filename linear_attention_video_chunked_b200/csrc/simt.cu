@@ -383,56 +383,70 @@ __device__ __forceinline__ long long leaving_slices(long long seen, int To, int 
   return r + n - r2;
 }
 
-__global__ void state_add_kernel(const float* __restrict__ P, const float* __restrict__ zp,
-                                 float* __restrict__ s_state, float* __restrict__ z_state,
-                                 const long long* __restrict__ seen, int Dp, int D, int To,
-                                 int nq, int nslots) {
-  const long long PD = static_cast<long long>(Dp) * D;
-  const long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int bh = blockIdx.y;
-  const long long leave = leaving_slices(*seen, To, nq);
-  if (e < PD) {
-    // s and the per-slot states share the image layout: element e of each.
-    const long long se = bh * PD + e;
-    float acc = s_state[se];
-    for (long long i = 0; i < leave; ++i) acc += P[(bh * nslots + i) * PD + e];
-    s_state[se] = acc;
-  } else if (e < PD + Dp) {
-    const long long f = e - PD;
-    float acc = z_state[static_cast<long long>(bh) * Dp + f];
-    for (long long i = 0; i < leave; ++i) acc += zp[(bh * nslots + i) * Dp + f];
-    z_state[static_cast<long long>(bh) * Dp + f] = acc;
-  }
-}
-
-// Copy chunk slices that stay in the window into their ring slots.
-// grid (nq_slices, BH); 16-byte vectors.
+// End of a streaming step, one launch (grid (nadd + nring, BH)):
+//  * blocks [0, nadd): (s, z) += the states of the slices that left the
+//    window this step (per-slot states from the fold, same image layout);
+//  * blocks [nadd, nadd + nring): the chunk slices that stay in the window
+//    are copied into their ring slots (slice g in slot g mod T_o), 16-byte
+//    vectors, kRingBlocksPerSlice blocks per chunk slice;
+//  * the slice counter advances by nq, written by the last block to finish
+//    (a completion count in the state header), after every block has read
+//    the old value.
 constexpr int kRingBlocksPerSlice = 16;
 
-__global__ void ring_update_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
-                                   uint4* __restrict__ rk, uint4* __restrict__ rv,
-                                   const long long* __restrict__ seen, long long slice_vecs,
-                                   int To, int nq) {
+__global__ void step_finish_kernel(const float* __restrict__ P, const float* __restrict__ zp,
+                                   float* __restrict__ s_state, float* __restrict__ z_state,
+                                   long long* seen, unsigned* done, int Dp, int D, int To,
+                                   int nq, int nslots, int nadd, const uint4* __restrict__ k,
+                                   const uint4* __restrict__ v, uint4* __restrict__ rk,
+                                   uint4* __restrict__ rv, long long slice_vecs) {
   const long long sn = *seen;
-  const long long after = sn + nq;
-  const long long keep = after < To ? after : To;
-  const int slice = blockIdx.x / kRingBlocksPerSlice;  // chunk slice of this block
-  const int part = blockIdx.x % kRingBlocksPerSlice;
-  const long long g = sn + slice;                      // its global slice index
-  if (g < after - keep) return;                        // leaves the window right away
   const int bh = blockIdx.y;
-  const uint4* ks = k + (static_cast<long long>(bh) * nq + slice) * slice_vecs;
-  const uint4* vs = v + (static_cast<long long>(bh) * nq + slice) * slice_vecs;
-  uint4* kd = rk + (static_cast<long long>(bh) * To + (g % To)) * slice_vecs;
-  uint4* vd = rv + (static_cast<long long>(bh) * To + (g % To)) * slice_vecs;
-  for (long long i = static_cast<long long>(part) * blockDim.x + threadIdx.x; i < slice_vecs;
-       i += static_cast<long long>(blockDim.x) * kRingBlocksPerSlice) {
-    kd[i] = ks[i];
-    vd[i] = vs[i];
+  if (static_cast<int>(blockIdx.x) < nadd) {
+    const long long PD = static_cast<long long>(Dp) * D;
+    const long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const long long leave = leaving_slices(sn, To, nq);
+    if (e < PD) {
+      const long long se = bh * PD + e;
+      float acc = s_state[se];
+      for (long long i = 0; i < leave; ++i) acc += P[(bh * nslots + i) * PD + e];
+      s_state[se] = acc;
+    } else if (e < PD + Dp) {
+      const long long f = e - PD;
+      float acc = z_state[static_cast<long long>(bh) * Dp + f];
+      for (long long i = 0; i < leave; ++i) acc += zp[(bh * nslots + i) * Dp + f];
+      z_state[static_cast<long long>(bh) * Dp + f] = acc;
+    }
+  } else {
+    const int rb = blockIdx.x - nadd;
+    const long long after = sn + nq;
+    const long long keep = after < To ? after : To;
+    const int slice = rb / kRingBlocksPerSlice;  // chunk slice of this block
+    const int part = rb % kRingBlocksPerSlice;
+    const long long g = sn + slice;              // its global slice index
+    if (g >= after - keep) {                     // it stays in the window
+      const uint4* ks = k + (static_cast<long long>(bh) * nq + slice) * slice_vecs;
+      const uint4* vs = v + (static_cast<long long>(bh) * nq + slice) * slice_vecs;
+      uint4* kd = rk + (static_cast<long long>(bh) * To + (g % To)) * slice_vecs;
+      uint4* vd = rv + (static_cast<long long>(bh) * To + (g % To)) * slice_vecs;
+      for (long long i = static_cast<long long>(part) * blockDim.x + threadIdx.x; i < slice_vecs;
+           i += static_cast<long long>(blockDim.x) * kRingBlocksPerSlice) {
+        kd[i] = ks[i];
+        vd[i] = vs[i];
+      }
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const unsigned nblocks = gridDim.x * gridDim.y;
+    if (atomicAdd(done, 1u) == nblocks - 1) {
+      *seen = sn + nq;
+      *done = 0;
+      __threadfence();
+    }
   }
 }
-
-__global__ void advance_kernel(long long* seen, int nq) { *seen += nq; }
 
 // bf16 copy of phi weights in the tensor-core image layout; blockIdx.y
 // selects the matrix (0: W_q, 1: W_k).
@@ -503,30 +517,19 @@ cudaError_t launch_scan(const float* P, const float* z, float* SL, float* zL, in
   return cudaGetLastError();
 }
 
-cudaError_t launch_state_add(const float* P, const float* zp, float* s_state, float* z_state,
-                             const long long* seen, int BH, int Dp, int D, int To,
-                             int nq_slices, int nslots, cudaStream_t s) {
+cudaError_t launch_step_finish(const float* P, const float* zp, float* s_state, float* z_state,
+                               long long* seen, unsigned* done, int BH, int Dp, int D, int To,
+                               int nq_slices, int nslots, const void* k, const void* v, void* rk,
+                               void* rv, int HW, int elem_bytes, cudaStream_t s) {
   const long long n = static_cast<long long>(Dp) * D + Dp;
-  dim3 grid(static_cast<unsigned>((n + 255) / 256), BH);
-  state_add_kernel<<<grid, 256, 0, s>>>(P, zp, s_state, z_state, seen, Dp, D, To, nq_slices,
-                                        nslots);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_ring_update(const void* k, const void* v, void* rk, void* rv,
-                               const long long* seen, int BH, int HW, int D, int To,
-                               int nq_slices, int elem_bytes, cudaStream_t s) {
-  if (To == 0) return cudaSuccess;
+  const int nadd = static_cast<int>((n + 255) / 256);
+  const int nring = To > 0 ? nq_slices * kRingBlocksPerSlice : 0;
   const long long slice_vecs = static_cast<long long>(HW) * D * elem_bytes / 16;
-  dim3 grid(nq_slices * kRingBlocksPerSlice, BH);
-  ring_update_kernel<<<grid, 256, 0, s>>>(
+  dim3 grid(nadd + nring, BH);
+  step_finish_kernel<<<grid, 256, 0, s>>>(
+      P, zp, s_state, z_state, seen, done, Dp, D, To, nq_slices, nslots, nadd,
       static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint4*>(rk),
-      static_cast<uint4*>(rv), seen, slice_vecs, To, nq_slices);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_advance(long long* seen, int nq_slices, cudaStream_t s) {
-  advance_kernel<<<1, 1, 0, s>>>(seen, nq_slices);
+      static_cast<uint4*>(rv), slice_vecs);
   return cudaGetLastError();
 }
 

@@ -103,6 +103,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sbase = smem_raw + (base - raw);
   auto bar = [&](int i) { return base + kBarOff + 8u * i; };
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(sbase + kAbortSlot);
+  // A streaming step's fold (launched next, programmatic dependent) may start
+  // once every CTA of this grid has started: it touches nothing this reads.
+  asm volatile("griddepcontrol.launch_dependents;");
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -569,6 +572,9 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
   uint8_t* sbase = smem_raw + (base - raw);
   auto bar = [&](int i) { return base + kBarOff + 8u * i; };
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(sbase + kAbortSlot);
+  // A streaming step's fold (launched next, programmatic dependent) may start
+  // once every CTA of this grid has started: it touches nothing this reads.
+  asm volatile("griddepcontrol.launch_dependents;");
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -1073,278 +1079,13 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
 }
 
 // ===========================================================================
-// Per-slice linear state on tensor cores ("Key designs 1 and 4": the linear
-// branch's sum of phi_k(k) v^T and of phi_k(k)):
-//   P_s = phi_k(K_s)^T V_s  ([Dp][D] fp32),  z_s = sum_j phi_k(k_j)  ([Dp]).
-// One CTA per (slice, b*h), or per leaving slice in step mode.  Per 128-token
-// tile: psi = K W_k (tcgen05, bf16) -> phi = (psi + b)^2 in registers (thread
-// = token, TMEM lane) -> bf16 phi^T tile in shared memory (MN-major A) ->
-// P += phi^T V and z += phi^T 1 (tcgen05, fp32 accumulators in TMEM).
-// Roles as in the attention kernel: warps 0-3 convert + epilogue, warp 4 TMA,
-// warp 5 MMA.  Dp in {64, 128}; features past Dp are zero rows of phi^T.
-// ===========================================================================
-namespace st {
-constexpr int kThreads = 192;
-constexpr uint32_t kStageOff = 0;        // 2 stages x (K 32 KB + V 32 KB)
-constexpr uint32_t kStageBytes = 65536;
-constexpr uint32_t kWOff = 131072;       // W_k image, Dp x 128 bf16 (<= 32 KB)
-constexpr uint32_t kPhiOff = 163840;     // phi^T tile, 2 boxes x 16 KB
-constexpr uint32_t kOnesOff = 196608;    // all-ones B operand for z, 2 boxes x 2 KB
-constexpr uint32_t kBiasOff = 200704;    // b_k, Dp fp32
-constexpr uint32_t kBarOff = 201728;
-enum { K_FULL = 0, V_FULL = 2, KV_EMPTY = 4, PSI_FULL = 6, PSI_FREE = 8, PHI_FULL = 10,
-       ACC_DONE = 11, W_FULL = 12, NBAR = 13 };
-constexpr uint32_t kTmemSlot = kBarOff + 8 * NBAR;
-constexpr uint32_t kAbortSlot = kTmemSlot + 4;
-constexpr uint32_t kSmemBytes = kBarOff + 128 + 1024;
-constexpr uint32_t kColPsi = 0, kColP = 256, kColZ = 384;
-}  // namespace st
-
-struct StMaps {
-  CUtensorMap k, v, rk, rv;
-};
-
-__global__ void __launch_bounds__(st::kThreads, 1)
-    tc_state_kernel(const __grid_constant__ StMaps maps, const PartialParams P,
-                    const __nv_bfloat16* __restrict__ wk_img) {
-  // Local names shadow the attention kernel's constants of the same names.
-  constexpr int kThreads = st::kThreads;
-  constexpr uint32_t kStageOff = st::kStageOff, kStageBytes = st::kStageBytes;
-  constexpr uint32_t kWOff = st::kWOff, kPhiOff = st::kPhiOff, kOnesOff = st::kOnesOff;
-  constexpr uint32_t kBiasOff = st::kBiasOff, kBarOff = st::kBarOff;
-  constexpr uint32_t kTmemSlot = st::kTmemSlot, kAbortSlot = st::kAbortSlot;
-  constexpr uint32_t kColPsi = st::kColPsi, kColP = st::kColP, kColZ = st::kColZ;
-  constexpr int K_FULL = st::K_FULL, V_FULL = st::V_FULL, KV_EMPTY = st::KV_EMPTY;
-  constexpr int PSI_FULL = st::PSI_FULL, PSI_FREE = st::PSI_FREE, PHI_FULL = st::PHI_FULL;
-  constexpr int ACC_DONE = st::ACC_DONE, W_FULL = st::W_FULL, NBAR = st::NBAR;
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw = smem_u32(smem_raw);
-  const uint32_t base = (raw + 1023u) & ~1023u;
-  uint8_t* sbase = smem_raw + (base - raw);
-  auto bar = [&](int i) { return base + kBarOff + 8u * i; };
-  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(sbase + kAbortSlot);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int slot = blockIdx.x;
-  const int bh = blockIdx.y;
-  const int h = bh % P.heads;
-  const int Dp = P.Dp;
-  const int HW = P.HW;
-
-  // Which rows hold this slice (same rules as the CUDA-core kernel).
-  const CUtensorMap *mk, *mv;
-  int row0;
-  if (P.seen == nullptr) {
-    mk = &maps.k; mv = &maps.v;
-    row0 = slot * HW;
-  } else {
-    const long long seen = *P.seen;
-    const long long r = seen < P.To ? seen : P.To;
-    const long long after = seen + P.nq_slices;
-    const long long r2 = after < P.To ? after : P.To;
-    if (slot >= r + P.nq_slices - r2) return;
-    const long long g = seen - r + slot;
-    if (g < seen) {
-      mk = &maps.rk; mv = &maps.rv;
-      row0 = static_cast<int>(g % P.To) * HW;
-    } else {
-      mk = &maps.k; mv = &maps.v;
-      row0 = static_cast<int>(g - seen) * HW;
-    }
-  }
-  const int nt = (HW + 127) / 128;
-
-  if (tid == 0) {
-    const uint32_t counts[NBAR] = {1, 1, 1, 1, 1, 1, 1, 1, 128, 128, 128, 1, 1};
-    for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), counts[i]);
-    *abort_flag = 0;
-    fence_barrier_init();
-  }
-  // All-ones B operand (any swizzle of ones is ones) and the bias vector.
-  for (int i = tid; i < 1024; i += kThreads)
-    reinterpret_cast<uint32_t*>(sbase + kOnesOff)[i] = 0x3F803F80u;
-  for (int f = tid; f < Dp; f += kThreads) {
-    const int half = Dp >> 1, part = f >= half;
-    reinterpret_cast<float*>(sbase + kBiasOff)[f] = P.bk[(h * 2 + part) * half + (f - part * half)];
-  }
-  fence_proxy_async();
-  if (warp == 5) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     base + kTmemSlot),
-                 "r"(512));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sbase + kTmemSlot);
-
-  if (warp == 4) {
-    if (lane == 0) {
-      bool ok = true;
-      const uint32_t wbytes = static_cast<uint32_t>(Dp) * 128 * 2;
-      mbar_expect_tx(bar(W_FULL), wbytes);
-      bulk_load(base + kWOff, wk_img + static_cast<long long>(h) * Dp * 128, wbytes, bar(W_FULL));
-      for (int j = 0; j < nt && ok; ++j) {
-        const int s = j & 1;
-        if (j >= 2) ok = mbar_wait(bar(KV_EMPTY + s), ((j - 2) >> 1) & 1, abort_flag, 16);
-        if (!ok) break;
-        const uint32_t kdst = base + kStageOff + s * kStageBytes;
-        const int row = row0 + j * 128;
-        mbar_expect_tx(bar(K_FULL + s), 32768);
-        tma_load_3d(kdst, mk, bar(K_FULL + s), 0, row, bh);
-        tma_load_3d(kdst + 16384, mk, bar(K_FULL + s), 64, row, bh);
-        mbar_expect_tx(bar(V_FULL + s), 32768);
-        tma_load_3d(kdst + 32768, mv, bar(V_FULL + s), 0, row, bh);
-        tma_load_3d(kdst + 49152, mv, bar(V_FULL + s), 64, row, bh);
-      }
-    }
-    __syncwarp();
-  } else if (warp == 5) {
-    if (lane == 0) {
-      const uint32_t id_psi = idesc_ab(128, Dp, 1, false, false);
-      const uint32_t id_st = idesc_ab(128, 128, 1, true, true);
-      const uint32_t id_z = idesc_ab(128, 16, 1, true, false);
-      bool ok = mbar_wait(bar(W_FULL), 0, abort_flag, 17);
-      auto issue_psi = [&](int i) -> bool {
-        const int s = i & 1;
-        if (!mbar_wait(bar(K_FULL + s), (i >> 1) & 1, abort_flag, 18)) return false;
-        if (i >= 2 && !mbar_wait(bar(PSI_FREE + s), ((i - 2) >> 1) & 1, abort_flag, 19))
-          return false;
-        tc_fence_after();
-        const uint32_t kaddr = base + kStageOff + s * kStageBytes;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-          const uint32_t woff = (kk >> 2) * (Dp * 128) + (kk & 3) * 32;
-          mma_bf16(tmem + kColPsi + s * 128, sdesc(kaddr + koff, 16, 1024),
-                   sdesc(base + kWOff + woff, 16, 1024), id_psi, kk > 0);
-        }
-        mma_commit(bar(PSI_FULL + s));
-        return true;
-      };
-      if (ok) ok = issue_psi(0);
-      for (int j = 0; j < nt && ok; ++j) {
-        if (j + 1 < nt) ok = issue_psi(j + 1);
-        if (!ok) break;
-        const int s = j & 1;
-        ok = mbar_wait(bar(PHI_FULL), j & 1, abort_flag, 20) &&
-             mbar_wait(bar(V_FULL + s), (j >> 1) & 1, abort_flag, 21);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t vaddr = base + kStageOff + s * kStageBytes + 32768;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t a = sdesc(base + kPhiOff + kk * 2048, 16384, 1024);
-          const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
-          mma_bf16(tmem + kColP, a, sdesc(vaddr + kk * 2048, 16384, 1024), id_st, acc);
-          mma_bf16(tmem + kColZ, a,
-                   sdesc(base + kOnesOff + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024), id_z, acc);
-        }
-        mma_commit(bar(ACC_DONE));
-        mma_commit(bar(KV_EMPTY + s));
-      }
-    }
-    __syncwarp();
-  } else {
-    // ---- convert: thread r = token row r of the tile (TMEM lane r) ----
-    const int r = tid;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    const float* bias = reinterpret_cast<const float*>(sbase + kBiasOff);
-    auto wait_all = [&](uint32_t b, uint32_t parity, uint32_t code) {
-      return __all_sync(0xffffffffu, mbar_wait(b, parity, abort_flag, code));
-    };
-    bool ok = true;
-    for (int j = 0; j < nt && ok; ++j) {
-      const int s = j & 1;
-      ok = wait_all(bar(PSI_FULL + s), (j >> 1) & 1, 22);
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t ps[128];
-      REHYAT_TMEM_LD32(lane_base + kColPsi + s * 128, ps);
-      REHYAT_TMEM_LD32(lane_base + kColPsi + s * 128 + 32, (ps + 32));
-      if (Dp > 64) {
-        REHYAT_TMEM_LD32(lane_base + kColPsi + s * 128 + 64, (ps + 64));
-        REHYAT_TMEM_LD32(lane_base + kColPsi + s * 128 + 96, (ps + 96));
-      }
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(bar(PSI_FREE + s));
-      const int nvalid = min(128, HW - j * 128);
-      const bool valid = r < nvalid;
-      uint32_t pk[64];
-#pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        float v0 = 0.f, v1 = 0.f;
-        if (valid && 2 * i < Dp) {
-          const float a0 = __uint_as_float(ps[2 * i]) + bias[2 * i];
-          const float a1 = __uint_as_float(ps[2 * i + 1]) + bias[2 * i + 1];
-          v0 = a0 * a0;
-          v1 = a1 * a1;
-        }
-        pk[i] = pack_bf16(v0, v1);
-      }
-      if (j > 0) {
-        ok = wait_all(bar(ACC_DONE), (j - 1) & 1, 23);
-        if (!ok) break;
-      }
-      // Token row r of the MN-major phi^T tile: features 64g..64g+63 in box g.
-#pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const uint32_t box = c >> 3, ch = c & 7;
-        st_shared_v4(base + kPhiOff + box * 16384 + r * 128 + ((ch ^ (r & 7)) << 4), pk[4 * c],
-                     pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      }
-      if (nvalid < 128) {
-        ok = wait_all(bar(V_FULL + s), (j >> 1) & 1, 24);
-        if (!ok) break;
-        if (!valid) {
-          const uint32_t vrow = base + kStageOff + s * kStageBytes + 32768 + r * 128;
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            st_shared_v4(vrow + c * 16, 0, 0, 0, 0);
-            st_shared_v4(vrow + 16384 + c * 16, 0, 0, 0, 0);
-          }
-        }
-      }
-      fence_proxy_async();
-      tc_fence_before();
-      mbar_arrive(bar(PHI_FULL));
-    }
-    if (ok) ok = wait_all(bar(ACC_DONE), (nt - 1) & 1, 25);
-    if (ok) {
-      tc_fence_after();
-      // Thread r = feature r (accumulator lane r); the state is stored in the
-      // S^L image layout (a warp writes one 128-byte row per column).
-      const long long obase = (static_cast<long long>(bh) * P.nslots + slot);
-      float* prow = P.P + obase * Dp * 128 + sl_feature_base(r, 128, Dp);
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[32];
-        REHYAT_TMEM_LD32(lane_base + kColP + c * 32, v);
-        tmem_wait_ld();
-        if (r < Dp) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) prow[sl_column_offset(r, c * 32 + i)] = __uint_as_float(v[i]);
-        }
-      }
-      uint32_t zv[32];
-      REHYAT_TMEM_LD32(lane_base + kColZ, zv);
-      tmem_wait_ld();
-      if (r < Dp) P.z[obase * Dp + r] = __uint_as_float(zv[0]);
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 5) {
-    tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
-  }
-}
-
-// ===========================================================================
-// Persistent per-slice state kernel (full mode): the same sums as
-// tc_state_kernel, with each CTA streaming a contiguous run of items through
-// one K/V pipeline that does not drain between slices.  The feature map is
+// Per-slice linear state on tensor cores (the linear branch's sums of
+// phi_k(k) v^T and of phi_k(k), "Key designs 1 and 4"):
+//   P_s = phi_k(K_s)^T V_s  ([D'][D] fp32),  z_s = sum_j phi_k(k_j)  ([D']),
+// for every slice (full forward) or for the slices leaving the softmax window
+// in a streaming step.  Persistent CTAs each stream a contiguous run of
+// items through one K/V pipeline that does not drain between slices.  The
+// feature map is
 // computed transposed, psi^T = W_k^T K^T (TMEM lane = feature, column =
 // token), so each converter thread owns one feature: it squares psi + b in
 // place, rounds to bf16 and leaves phi^T in TMEM as the A operand of
@@ -1359,6 +1100,12 @@ __global__ void __launch_bounds__(st::kThreads, 1)
 // slice (items run over (b*h, half, slice), so W_k changes only at half or
 // head boundaries); with D' = 64 the upper 64 W_k rows stay zero.
 // ===========================================================================
+// Tensor maps of the state kernel: k, v of the chunk (or of all slices) and
+// the ring's k, v (streaming; equal to k, v otherwise).
+struct StMaps {
+  CUtensorMap k, v, rk, rv;
+};
+
 namespace sp {
 constexpr int kThreads = 320;
 constexpr int kStages = 3;             // K and V ring depth
@@ -1375,29 +1122,30 @@ constexpr uint32_t kColBuf = 0, kColP = 256;
 
 // Walk over a CTA's run of items i = q * T + slice, q = bh * halves + half,
 // with a division only when one (bh, half) run of slices ends.
+// Items past `active` slices of a run (streaming: slots beyond the number of
+// slices leaving the window this step) are skipped by every role alike.
 struct ItemWalk {
-  int T, halves, heads, pw;
+  int T, halves, heads, pw, active;
   int slice = 0, q = 0;
-  int wkey = 0;       // (head, half) key of the W_k piece the item needs
-  bool wnew = true;   // first item, or wkey differs from the previous item's
+  int wkey = 0;  // (head, half) key of the W_k piece the item needs
   __device__ int bh() const { return halves == 2 ? q >> 1 : q; }
   __device__ int half() const { return q - bh() * halves; }
   __device__ int key() const { return (bh() % heads) * halves + half(); }
-  __device__ long long slice_index() const { return static_cast<long long>(bh()) * T + slice; }
+  __device__ bool on() const { return slice < active; }
+  // Output slot of the item: (bh, slice) with `nslots` slots per (b,h).
+  __device__ long long out_index(int nslots) const {
+    return static_cast<long long>(bh()) * nslots + slice;
+  }
   __device__ void start(int item) {
     slice = item % T;
     q = item / T;
     wkey = key();
-    wnew = true;
   }
   __device__ void next() {
-    wnew = false;
     if (++slice == T) {
       slice = 0;
       ++q;
-      const int k = key();
-      wnew = k != wkey;
-      wkey = k;
+      wkey = key();
     }
   }
 };
@@ -1429,16 +1177,42 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
   auto bar = [&](int i) { return base + sp::kBarOff + 8u * i; };
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(sbase + sp::kAbortSlot);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int Dp = P.Dp, HW = P.HW, T = P.nslots;
+  const int Dp = P.Dp, HW = P.HW;
   const int pw = Dp < 128 ? Dp : 128;  // features per item
   const int halves = Dp / pw;
+  // Full forward: items (bh, half, slice) over all slices.  Streaming fold:
+  // items (bh, half, slot) over the chunk's slots, of which the first
+  // `leave` hold slices leaving the window (slot i = global slice
+  // seen - min(seen, T_o) + i, in the ring if already seen, else in the chunk).
+  const bool step = P.seen != nullptr;
+  const int T = step ? P.nq_slices : P.nslots;
+  const long long seen0 = step ? *P.seen : 0;
+  const long long rseen = seen0 < P.To ? seen0 : P.To;
+  int leave = T;
+  if (step) {
+    const long long after = seen0 + P.nq_slices;
+    leave = static_cast<int>(rseen + P.nq_slices - (after < P.To ? after : P.To));
+  }
   const int total = P.BH * halves * T;
   const int it0 = blockIdx.x * items_per_cta;
   const int it1 = min(total, it0 + items_per_cta);
-  if (it0 >= it1) return;
+  // Launched as a programmatic dependent of the attention kernel of the same
+  // streaming step, this grid overlaps it; waiting here before exit makes
+  // this grid's completion imply the attention kernel's (no-op otherwise).
+  auto dependency_wait = [] { asm volatile("griddepcontrol.wait;" ::: "memory"); };
+  if (it0 >= it1) {
+    dependency_wait();
+    return;
+  }
   const int nitems = it1 - it0;
   const int nt = (HW + 127) / 128;
-  const int TT = nitems * nt;  // token tiles of this CTA
+  int nactive = 0;
+  {
+    sp::ItemWalk w{T, halves, P.heads, pw, leave};
+    w.start(it0);
+    for (int il = 0; il < nitems; ++il, w.next()) nactive += w.on();
+  }
+  const int TT = nactive * nt;  // token tiles of this CTA
 
   if (tid == 0) {
     for (int i = 0; i < NBAR; ++i) {
@@ -1472,14 +1246,16 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
     // ================================================= TMA producer
     if (lane == 0) {
       bool ok = true;
-      int wloads = 0;
+      int wloads = 0, wkey = -1;
       const uint32_t box_bytes = static_cast<uint32_t>(pw) * 128;  // one 64-column box
-      sp::ItemWalk w{T, halves, P.heads, pw};
+      sp::ItemWalk w{T, halves, P.heads, pw, leave};
       w.start(it0);
       int gt = 0, st = 0, uses = 0;  // tile index, its ring stage, earlier uses of the stage
       for (int il = 0; il < nitems && ok; ++il, w.next()) {
-        if (w.wnew) {
-          if (il > 0) ok = mbar_wait(bar(W_FREE), (wloads - 1) & 1, abort_flag, 27);
+        if (!w.on()) continue;
+        if (w.wkey != wkey) {
+          wkey = w.wkey;
+          if (wloads > 0) ok = mbar_wait(bar(W_FREE), (wloads - 1) & 1, abort_flag, 27);
           if (!ok) break;
           // Head h's image holds its D' features as pieces of pw rows, each
           // piece two boxes of pw rows x 64 columns.
@@ -1489,19 +1265,32 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
           bulk_load(base + kWOff + 16384, src + pw * 64, box_bytes, bar(W_FULL));
           ++wloads;
         }
-        const int bh = w.bh(), row0 = w.slice * HW;
+        const int bh = w.bh();
+        const CUtensorMap* mk = &maps.k;
+        const CUtensorMap* mv = &maps.v;
+        int row0 = w.slice * HW;
+        if (step) {
+          const long long g = seen0 - rseen + w.slice;  // global slice of this slot
+          if (g < seen0) {
+            mk = &maps.rk;
+            mv = &maps.rv;
+            row0 = static_cast<int>(g % P.To) * HW;
+          } else {
+            row0 = static_cast<int>(g - seen0) * HW;
+          }
+        }
         for (int j = 0; j < nt && ok; ++j, ++gt) {
           const int row = row0 + j * 128;
           if (gt >= kS) ok = mbar_wait(bar(K_EMPTY + st), (uses - 1) & 1, abort_flag, 28);
           if (!ok) break;
           mbar_expect_tx(bar(K_FULL + st), 32768);
-          tma_load_3d(base + kKOff + st * 32768, &maps.k, bar(K_FULL + st), 0, row, bh);
-          tma_load_3d(base + kKOff + st * 32768 + 16384, &maps.k, bar(K_FULL + st), 64, row, bh);
+          tma_load_3d(base + kKOff + st * 32768, mk, bar(K_FULL + st), 0, row, bh);
+          tma_load_3d(base + kKOff + st * 32768 + 16384, mk, bar(K_FULL + st), 64, row, bh);
           if (gt >= kS) ok = mbar_wait(bar(V_EMPTY + st), (uses - 1) & 1, abort_flag, 29);
           if (!ok) break;
           mbar_expect_tx(bar(V_FULL + st), 32768);
-          tma_load_3d(base + kVOff + st * 32768, &maps.v, bar(V_FULL + st), 0, row, bh);
-          tma_load_3d(base + kVOff + st * 32768 + 16384, &maps.v, bar(V_FULL + st), 64, row, bh);
+          tma_load_3d(base + kVOff + st * 32768, mv, bar(V_FULL + st), 0, row, bh);
+          tma_load_3d(base + kVOff + st * 32768 + 16384, mv, bar(V_FULL + st), 64, row, bh);
           if (++st == kS) {
             st = 0;
             ++uses;
@@ -1516,17 +1305,20 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
       const uint32_t id_psi = idesc(128, 128, 1, false);  // W_k piece and K tile, K-major
       const uint32_t id_pv = idesc(128, 128, 1, true);    // phi^T from TMEM, V MN-major
       bool ok = true;
-      int wwaits = 0;
-      // The next psi^T to issue: its tile index, item walk, tile in item,
-      // K stage and earlier uses of that stage.
-      sp::ItemWalk wp{T, halves, P.heads, pw};
+      int wwaits = 0, wkey = -1;
+      // The next psi^T to issue: its tile index, item walk (on active
+      // items), tile in item, K stage and earlier uses of that stage.
+      sp::ItemWalk wp{T, halves, P.heads, pw, leave};
       wp.start(it0);
+      if (TT > 0)
+        while (!wp.on()) wp.next();
       int pgt = 0, pj = 0, pst = 0, puses = 0;
       // psi^T for token tile pgt into buffer pgt & 1: waits for its K tile,
       // for phi^T V of tile pgt - 2 to have read that buffer, and for W_k.
       auto issue_psi = [&]() -> bool {
         const int b = pgt & 1;
-        if (pj == 0 && wp.wnew) {
+        if (pj == 0 && wp.wkey != wkey) {
+          wkey = wp.wkey;
           if (pgt > 0) mma_commit(bar(W_FREE));  // tracks every earlier MMA
           if (!mbar_wait(bar(W_FULL), wwaits & 1, abort_flag, 30)) return false;
           ++wwaits;
@@ -1550,22 +1342,23 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
           pst = 0;
           ++puses;
         }
-        if (++pj == nt) {
+        if (++pj == nt && pgt < TT) {  // on to the next active item
           pj = 0;
-          wp.next();
+          do wp.next();
+          while (!wp.on());
         }
         return true;
       };
-      ok = issue_psi();
+      if (TT > 0) ok = issue_psi();
       int gt = 0, vst = 0, vuses = 0;
-      for (int il = 0; il < nitems && ok; ++il) {
-        const int pb = il & 1;
+      for (int ia = 0; ia < nactive && ok; ++ia) {  // active items
+        const int pb = ia & 1;
         for (int j = 0; j < nt && ok; ++j, ++gt) {
           const int b = gt & 1;
           if (gt + 1 < TT) ok = issue_psi();
           if (!ok) break;
-          if (j == 0 && il >= 2)
-            ok = mbar_wait(bar(P_FREE + pb), ((il - 2) >> 1) & 1, abort_flag, 33);
+          if (j == 0 && ia >= 2)
+            ok = mbar_wait(bar(P_FREE + pb), ((ia - 2) >> 1) & 1, abort_flag, 33);
           if (ok) ok = mbar_wait(bar(PHI_FULL + b), (gt >> 1) & 1, abort_flag, 34) &&
                        mbar_wait(bar(V_FULL + vst), vuses & 1, abort_flag, 35);
           if (!ok) break;
@@ -1596,12 +1389,16 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
     bool ok = true;
     float bias = 0.f;
     uint64_t zacc = f2_pack(0.f, 0.f);  // z over even / odd tokens
-    sp::ItemWalk w{T, halves, P.heads, pw};
+    sp::ItemWalk w{T, halves, P.heads, pw, leave};
     w.start(it0);
-    int gt = 0, vst = 0, vuses = 0;
+    int gt = 0, vst = 0, vuses = 0, wkey = -1;
     for (int il = 0; il < nitems && ok; ++il, w.next()) {
+      if (!w.on()) continue;
       // b_k of head h is h's D' consecutive features.
-      if (w.wnew) bias = f < pw ? P.bk[w.wkey * pw + f] : 0.f;
+      if (w.wkey != wkey) {
+        wkey = w.wkey;
+        bias = f < pw ? P.bk[wkey * pw + f] : 0.f;
+      }
       const uint64_t b2 = f2_pack(bias, bias);
       for (int j = 0; j < nt && ok; ++j, ++gt) {
         const int b = gt & 1;
@@ -1659,7 +1456,7 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
       if (ok) {
         float z0, z1;
         f2_unpack(zacc, z0, z1);
-        if (f < pw) P.z[w.slice_index() * Dp + w.half() * pw + f] = z0 + z1;
+        if (f < pw) P.z[w.out_index(P.nslots) * Dp + w.half() * pw + f] = z0 + z1;
         zacc = f2_pack(0.f, 0.f);
       }
     }
@@ -1668,17 +1465,20 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
     const int f = tid - 128;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     bool ok = true;
-    sp::ItemWalk w{T, halves, P.heads, pw};
+    sp::ItemWalk w{T, halves, P.heads, pw, leave};
     w.start(it0);
+    int ia = 0;  // active items so far
     for (int il = 0; il < nitems && ok; ++il, w.next()) {
-      const int pb = il & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(ACC_DONE + pb), (il >> 1) & 1, abort_flag, 39));
+      if (!w.on()) continue;
+      const int pb = ia & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(ACC_DONE + pb), (ia >> 1) & 1, abort_flag, 39));
+      ++ia;
       if (!ok) break;
       tc_fence_after();
       // Feature fg of the slice; the state is stored in the S^L image layout
       // (a warp writes one 128-byte row per column).
       const int fg = w.half() * pw + f;
-      float* prow = P.P + w.slice_index() * Dp * 128 + sl_feature_base(fg, 128, Dp);
+      float* prow = P.P + w.out_index(P.nslots) * Dp * 128 + sl_feature_base(fg, 128, Dp);
       for (int c = 0; c < 4; ++c) {
         uint32_t v[32];
         REHYAT_TMEM_LD32(lane_base + kColP + pb * 128 + c * 32, v);
@@ -1699,6 +1499,7 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
   }
+  dependency_wait();
 }
 
 // ------------------------------------------------------------ host side
@@ -1732,11 +1533,8 @@ bool make_map(CUtensorMap* m, const void* ptr, long long rows, int planes) {
 
 }  // namespace
 
-bool tc_state_eligible(int in_bf16, int D, int Dp, bool step) {
-  // The step-mode kernel holds all D' features of a slice in one CTA (at most
-  // 128); the persistent full-mode kernel splits D' = 256 into halves.
-  const bool dp_ok = Dp == 64 || Dp == 128 || (!step && Dp == 256);
-  return in_bf16 && D == kD && dp_ok && encode_fn() != nullptr;
+bool tc_state_eligible(int in_bf16, int D, int Dp) {
+  return in_bf16 && D == kD && (Dp == 64 || Dp == 128 || Dp == 256) && encode_fn() != nullptr;
 }
 
 cudaError_t launch_state_tc(const PartialParams& p, const void* wk_img, cudaStream_t s) {
@@ -1752,30 +1550,38 @@ cudaError_t launch_state_tc(const PartialParams& p, const void* wk_img, cudaStre
     maps.rk = maps.k;
     maps.rv = maps.v;
   }
-  cudaError_t e;
+  // Persistent CTAs, each with the same number of items.
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int per_bh = (p.seen ? p.nq_slices : p.nslots) * (p.Dp > 128 ? p.Dp / 128 : 1);
+  const int total = p.BH * per_bh;
+  const int per_cta = (total + sms - 1) / sms;
+  const int ctas = (total + per_cta - 1) / per_cta;
+  cudaError_t e = cudaFuncSetAttribute(tc_state_persistent_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(sp::kSmemBytes));
+  if (e != cudaSuccess) return e;
+  const __nv_bfloat16* wk = static_cast<const __nv_bfloat16*>(wk_img);
   if (p.seen == nullptr) {
-    // Full forward: persistent CTAs, each with the same number of slices.
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int total = p.BH * p.nslots * (p.Dp > 128 ? p.Dp / 128 : 1);
-    const int per_cta = (total + sms - 1) / sms;
-    const int ctas = (total + per_cta - 1) / per_cta;
-    e = cudaFuncSetAttribute(tc_state_persistent_kernel,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(sp::kSmemBytes));
-    if (e != cudaSuccess) return e;
-    tc_state_persistent_kernel<<<ctas, sp::kThreads, sp::kSmemBytes, s>>>(
-        maps, p, static_cast<const __nv_bfloat16*>(wk_img), per_cta);
+    tc_state_persistent_kernel<<<ctas, sp::kThreads, sp::kSmemBytes, s>>>(maps, p, wk, per_cta);
     return cudaGetLastError();
   }
-  e = cudaFuncSetAttribute(tc_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(st::kSmemBytes));
-  if (e != cudaSuccess) return e;
-  dim3 grid(p.nslots, p.BH);
-  tc_state_kernel<<<grid, st::kThreads, st::kSmemBytes, s>>>(
-      maps, p, static_cast<const __nv_bfloat16*>(wk_img));
-  return cudaGetLastError();
+  // Streaming fold: it reads only k, v, the ring and W_k and writes only the
+  // per-slot states, so it may start while the attention kernel launched
+  // just before it is still running (programmatic dependent launch); the
+  // kernel waits for that grid before it exits.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ctas);
+  cfg.blockDim = dim3(sp::kThreads);
+  cfg.dynamicSmemBytes = sp::kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, tc_state_persistent_kernel, maps, p, wk, per_cta);
 }
 
 bool tc_attn_eligible(int in_bf16, int D, int Dp) {
