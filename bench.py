@@ -277,7 +277,8 @@ def measure_streaming(rh, dev, flush, stream):
     y_eager = out.clone()
 
     # The same 27 steps as one captured step replayed per chunk (the chunk is
-    # copied into fixed input buffers first; the copy is inside the timing).
+    # copied into fixed input buffers first; the copies, 43 MB per step, are
+    # inside the timing).
     st.reset()
     qb, kb, vb = (torch.empty_like(x) for x in chunks[0])
     outg = torch.empty_like(out)
@@ -296,6 +297,20 @@ def measure_streaming(rh, dev, flush, stream):
     gsteady = sorted(gms[2:])[len(gms[2:]) // 2]
     same = bool(torch.equal(outg, y_eager))
     del graph
+
+    # All 27 steps captured as one graph over the chunks in place (no input
+    # copies), replayed once: the whole stream with a single graph launch.
+    st.reset()
+    outs = torch.empty_like(out)
+    seq = st.capture_steps(chunks, outs)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    seq.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    seq_ms = e0.elapsed_time(e1)
+    seq_same = bool(torch.equal(outs, y_eager))
+    del seq
     return {"workload": "81 slices of 30x52, 12 heads, D=D'=128, T_c=3, T_o=1, bf16, "
                         "27 rehyat_chunk_step calls (inputs from a seeded torch generator)",
             "steps": len(ms), "ms_per_step_median_steady": steady,
@@ -303,6 +318,9 @@ def measure_streaming(rh, dev, flush, stream):
             "graph_ms_per_step_median_steady": gsteady,
             "graph_tokens_per_s_steady": rows / (gsteady / 1e3),
             "graph_last_chunk_bitwise_equal_to_eager": same,
+            "sequence_graph_ms_per_step": seq_ms / len(chunks),
+            "sequence_graph_tokens_per_s": rows * len(chunks) / (seq_ms / 1e3),
+            "sequence_graph_last_chunk_bitwise_equal_to_eager": seq_same,
             "free_bytes_before": free0, "free_bytes_after": free1,
             "device_memory_constant": free0 == free1}
 

@@ -352,6 +352,28 @@ class StreamingState:
     def restore(self, saved):
         self.state.copy_(saved)
 
+    def capture_steps(self, chunks, out):
+        """Record consecutive steps, one per (q, k, v) chunk of ``chunks``, as
+        one CUDA graph: each step reads its own chunk tensors and writes
+        ``out``.  Replaying it runs the whole sequence from the state's
+        current slice count with one launch of the graph.  The state is left
+        as it was before the call."""
+        torch = _torch()
+        saved = self.snapshot()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):  # warm-up launch outside the capture
+            self.step(*chunks[0], out=out)
+        torch.cuda.current_stream().wait_stream(side)
+        self.restore(saved)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for c in chunks:
+                self.step(*c, out=out)
+        torch.cuda.synchronize()
+        self.restore(saved)
+        return graph
+
     def capture_step(self, q, k, v, out):
         """Record one step on fixed buffers q, k, v, out as a CUDA graph.
 

@@ -189,6 +189,17 @@ def test_streaming_matches_rnn_oracle_and_full_causal(dtype, Tc, To):
     assert mx <= (2e-2 if dtype == "bf16" else 1e-5)
 
 
+@pytest.mark.parametrize("Dp,Tc,To", [(256, 3, 1), (64, 2, 2)])
+def test_streaming_wide_and_narrow_phi(Dp, Tc, To):
+    """The streaming fold on the tensor-core state kernel with D' = 256
+    (two 128-feature halves per leaving slice) and D' = 64."""
+    p = make_problem(batch=1, heads=3, T=11, Hs=9, Ws=15, D=128, Dp=Dp, Tc=Tc, To=To,
+                     causal=True, dtype="bf16", seed=57 + Dp + Tc)
+    y_stream, _ = _stream_outputs(p)
+    ref_y, _ = orc.run_problem(p, form="rnn")
+    assert_close_y(y_stream.double().cpu().numpy(), ref_y, "bf16")
+
+
 def test_stream_81_slices_constant_memory():
     """81 slices of 30x52, 27 steps: outputs of sampled heads match the oracle
     and free device memory does not move across steps."""
@@ -238,6 +249,27 @@ def test_streaming_cuda_graph_replay_matches_eager():
         outs.append(out.clone())
     torch.cuda.synchronize()
     assert torch.equal(torch.cat(outs, dim=2), y_eager)
+
+
+def test_streaming_sequence_graph_matches_eager():
+    """All steps of a stream captured as one CUDA graph (each step on its own
+    chunk tensors) and replayed once give the eager outputs bit for bit, and
+    a second replay after a reset gives them again."""
+    p = make_problem(batch=1, heads=2, T=10, Hs=6, Ws=11, D=128, Dp=128, Tc=2, To=1,
+                     causal=True, dtype="bf16", seed=43)
+    y_eager, st = _stream_outputs(p)
+    dev = device_tensors(p)
+    rows = p.Tc * p.HW
+    chunks = [tuple(dev[n][:, :, i * rows:(i + 1) * rows].contiguous() for n in "qkv")
+              for i in range(p.T // p.Tc)]
+    st.reset()
+    out = torch.empty(1, 2, rows, 128, device="cuda")
+    graph = st.capture_steps(chunks, out)
+    for _ in range(2):
+        st.reset()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, y_eager[:, :, -rows:])
 
 
 def test_streaming_checkpoint_resume_bit_exact():
