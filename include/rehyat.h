@@ -204,6 +204,39 @@ REHYAT_API rehyat_status rehyat_chunk_step(const rehyat_params* p, const void* q
                                 const rehyat_debug* dbg, void* stream);
 
 /* ---------------------------------------------------------------------- */
+/* Backward for the feature maps (Key design 5: the first training stage,
+ * block-wise attention distillation, updates only phi_q and phi_k).       */
+
+/* Gradients of the phi parameters, fp32 device arrays laid out like
+ * rehyat_phi: dWq, dWk [heads][2][D][Dp/2], dbq, dbk [heads][2][Dp/2]. */
+typedef struct {
+  float *dWq, *dbq, *dWk, *dbk;
+} rehyat_phi_grad;
+
+/* Workspace bytes rehyat_phi_bwd needs (0 if p is invalid). */
+REHYAT_API size_t rehyat_phi_bwd_workspace_bytes(const rehyat_params* p);
+
+/* dL/dW_q, dL/db_q, dL/dW_k, dL/db_k of a scalar loss L, given the forward's
+ * inputs q, k, v (in_dtype, [B][h][N][D]), its output y (fp32), the upstream
+ * gradient dy = dL/dy (fp32, same shape) and den [B][h][N] (fp32), the
+ * forward's joint denominator n^S + n^L per query (the nS + nL of
+ * rehyat_debug).  The full forward's form is used (p->causal selects it).
+ * With g = dy:  dL/dphi_q(q_i) = (S_L g_i - z_L (g_i.y_i)) / den_i;  a key j
+ * in the linear set of chunk t receives G_t v_j + h_t with
+ * G_t = sum_i phi_q(q_i) g_i^T / den_i, h_t = -sum_i phi_q(q_i)(g_i.y_i)/den_i;
+ * through phi = [(xW_1+b_1)^2, (xW_2+b_2)^2], du = 2u * dphi, dW = sum x^T du,
+ * db = sum du, summed over the batch (parameters are per head).  The
+ * gradients are overwritten, not accumulated; fp32 arithmetic; the
+ * reductions run in a fixed order, so repeated calls agree bit for bit.
+ * Pointers: q, k, v, y, dy, workspace 16-byte aligned; den and the gradient
+ * arrays 4-byte aligned.  Errors as for rehyat_hybrid_attn_fwd. */
+REHYAT_API rehyat_status rehyat_phi_bwd(const rehyat_params* p, const void* q, const void* k,
+                                        const void* v, const float* y, const float* dy,
+                                        const float* den, const rehyat_phi* phi,
+                                        const rehyat_phi_grad* grad, void* workspace,
+                                        size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------- */
 /* Diagnostic: every wait inside the tensor-core kernels is bounded (~2 s);
  * a wait that runs out sets a bit in a device-side error word and the
  * kernel returns early instead of hanging.  This reads that word for the

@@ -28,7 +28,9 @@ __all__ = [
     "rehyat_workspace_bytes", "rehyat_hybrid_attn_fwd", "rehyat_fwd_state", "rehyat_fwd_attn",
     "rehyat_softmax_attn_fwd", "rehyat_state_bytes", "rehyat_state_init", "rehyat_step_workspace_bytes",
     "rehyat_chunk_step", "rehyat_device_error_flags", "rehyat_attn_path",
-    "rehyat_status_string", "rehyat_version", "rehyat_hybrid_attn_fwd_noalloc", "make_params", "hybrid_attn", "softmax_attn", "StreamingState",
+    "rehyat_status_string", "rehyat_version", "rehyat_hybrid_attn_fwd_noalloc",
+    "RehyatPhiGrad", "rehyat_phi_bwd_workspace_bytes", "rehyat_phi_bwd",
+    "make_params", "hybrid_attn", "softmax_attn", "phi_grad", "StreamingState",
 ]
 
 F32, BF16 = 0, 1
@@ -44,7 +46,7 @@ EXPORTED_SYMBOLS = (
     "rehyat_fwd_attn", "rehyat_softmax_attn_fwd", "rehyat_state_bytes", "rehyat_state_init",
     "rehyat_step_workspace_bytes", "rehyat_chunk_step", "rehyat_device_error_flags",
     "rehyat_attn_path", "rehyat_status_string", "rehyat_version",
-    "rehyat_hybrid_attn_fwd_noalloc",
+    "rehyat_hybrid_attn_fwd_noalloc", "rehyat_phi_bwd_workspace_bytes", "rehyat_phi_bwd",
 )
 
 
@@ -65,6 +67,11 @@ class RehyatPhi(ctypes.Structure):
 class RehyatDebug(ctypes.Structure):
     _fields_ = [("aS", ctypes.c_void_p), ("nS", ctypes.c_void_p), ("c", ctypes.c_void_p),
                 ("aL", ctypes.c_void_p), ("nL", ctypes.c_void_p)]
+
+
+class RehyatPhiGrad(ctypes.Structure):
+    _fields_ = [("dWq", ctypes.c_void_p), ("dbq", ctypes.c_void_p),
+                ("dWk", ctypes.c_void_p), ("dbk", ctypes.c_void_p)]
 
 
 class RehyatError(RuntimeError):
@@ -127,6 +134,11 @@ def lib() -> ctypes.CDLL:
         L.rehyat_status_string.restype = ctypes.c_char_p
         L.rehyat_version.argtypes = []
         L.rehyat_version.restype = i
+        L.rehyat_phi_bwd_workspace_bytes.argtypes = [P(RehyatParams)]
+        L.rehyat_phi_bwd_workspace_bytes.restype = sz
+        L.rehyat_phi_bwd.argtypes = [P(RehyatParams), vp, vp, vp, vp, vp, vp, P(RehyatPhi),
+                                     P(RehyatPhiGrad), vp, sz, vp]
+        L.rehyat_phi_bwd.restype = i
         _LIB = L
     return _LIB
 
@@ -158,6 +170,15 @@ def rehyat_hybrid_attn_fwd_noalloc(p, q, k, v, phi, y, dbg, stream) -> int:
     return lib().rehyat_hybrid_attn_fwd_noalloc(ctypes.byref(p), q, k, v, ctypes.byref(phi), y,
                                                 None if dbg is None else ctypes.byref(dbg),
                                                 stream)
+
+
+def rehyat_phi_bwd_workspace_bytes(p: RehyatParams) -> int:
+    return lib().rehyat_phi_bwd_workspace_bytes(ctypes.byref(p))
+
+
+def rehyat_phi_bwd(p, q, k, v, y, dy, den, phi, grad, workspace, ws_bytes, stream) -> int:
+    return lib().rehyat_phi_bwd(ctypes.byref(p), q, k, v, y, dy, den, ctypes.byref(phi),
+                                ctypes.byref(grad), workspace, ws_bytes, stream)
 
 
 def rehyat_softmax_attn_fwd(p, q, k, v, y, stream) -> int:
@@ -283,6 +304,36 @@ def hybrid_attn(q, k, v, Wq, bq, Wk, bk, *, T, Hs, Ws, Tc, To, causal, out_dtype
                                 _stream_handle(stream))
     _check(st, "rehyat_hybrid_attn_fwd")
     return (y, dbg_t) if debug else y
+
+
+def phi_grad(q, k, v, y, dy, den, Wq, bq, Wk, bk, *, T, Hs, Ws, Tc, To, causal, scale=0.0,
+             force_simt=False, workspace=None, stream=None):
+    """Gradients of L with respect to the phi parameters, given the forward's
+    q, k, v, its fp32 output y, dy = dL/dy (fp32) and den = n^S + n^L per
+    query (``parts["nS"] + parts["nL"]`` of ``hybrid_attn(..., debug=True)``).
+    Returns dict(dWq, dbq, dWk, dbk) shaped like the parameters."""
+    torch = _torch()
+    B, H, N, D = q.shape
+    Dp = 2 * Wq.shape[-1]
+    for t in (y, dy, den):
+        if t.dtype != torch.float32 or not t.is_contiguous():
+            raise TypeError("y, dy and den must be contiguous fp32 tensors")
+    p = make_params(batch=B, heads=H, T=T, Hs=Hs, Ws=Ws, D=D, Dp=Dp, Tc=Tc, To=To,
+                    causal=causal, in_dtype=_dtype_code(q.dtype), out_dtype=F32, scale=scale,
+                    flags=FLAG_FORCE_SIMT if force_simt else 0)
+    nbytes = rehyat_phi_bwd_workspace_bytes(p)
+    if nbytes == 0:
+        raise RehyatError(1, "rehyat_phi_bwd_workspace_bytes")
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    g = {name: torch.empty_like(t) for name, t in
+         (("dWq", Wq), ("dbq", bq), ("dWk", Wk), ("dbk", bk))}
+    grad = RehyatPhiGrad(*(g[n].data_ptr() for n in ("dWq", "dbq", "dWk", "dbk")))
+    st = rehyat_phi_bwd(p, q.data_ptr(), k.data_ptr(), v.data_ptr(), y.data_ptr(), dy.data_ptr(),
+                        den.data_ptr(), _phi_struct(Wq, bq, Wk, bk), grad, workspace.data_ptr(),
+                        workspace.numel(), _stream_handle(stream))
+    _check(st, "rehyat_phi_bwd")
+    return g
 
 
 def softmax_attn(q, k, v, *, out_dtype=None, scale=0.0, force_simt=False, out=None,

@@ -179,6 +179,39 @@ cudaError_t run_attn(const rehyat_params* p, const AttnParams& a, cudaStream_t s
   return launch_attn_simt(a, s);
 }
 
+// Per-slice states and the linear-set state per chunk into the workspace
+// laid out by fwd_layout (weight images, per-slice state kernel, chunk scan);
+// arguments already checked.
+rehyat_status state_pass(const rehyat_params* p, const void* k, const void* v,
+                         const rehyat_phi* phi, char* ws, cudaStream_t s) {
+  const FwdWorkspace w = fwd_layout(p);
+  float* P = reinterpret_cast<float*>(ws + w.P_off);
+  float* z = reinterpret_cast<float*>(ws + w.z_off);
+  float* SL = reinterpret_cast<float*>(ws + w.SL_off);
+  float* zL = reinterpret_cast<float*>(ws + w.zL_off);
+  const int BH = p->batch * p->heads;
+  const int HW = p->Hs * p->Ws;
+
+  PartialParams pp = {};
+  pp.k = k; pp.v = v;
+  pp.rows_per_bh = static_cast<long long>(p->T) * HW;
+  pp.Wk = phi->Wk; pp.bk = phi->bk;
+  pp.P = P; pp.z = z;
+  pp.BH = BH; pp.heads = p->heads; pp.HW = HW; pp.D = p->D; pp.Dp = p->Dp; pp.To = p->To;
+  pp.nslots = p->T;
+  pp.in_bf16 = p->in_dtype == REHYAT_BF16;
+  pp.w_bf16 = pp.in_bf16;
+  cudaError_t e = cudaSuccess;
+  if (tc_path(p) || tc_state_path(p))
+    e = launch_w_images(phi->Wq, ws + w.wimg_off, phi->Wk, ws + w.wkimg_off, p->heads, p->D,
+                        p->Dp, s);
+  if (e != cudaSuccess) return to_status(e);
+  e = run_partials(p, pp, ws + w.wkimg_off, s);
+  if (e != cudaSuccess) return to_status(e);
+  return to_status(launch_scan(P, z, SL, zL, BH, p->T, p->Tc, p->To, nchunks_of(p), p->Dp,
+                               p->D, p->causal, s));
+}
+
 }  // namespace
 }  // namespace rehyat
 
@@ -219,35 +252,9 @@ rehyat_status rehyat_fwd_state(const rehyat_params* p, const void* k, const void
   if (!k || !v || !workspace) return REHYAT_ERR_INVALID_ARG;
   if ((st = check_phi(phi)) != REHYAT_OK) return st;
   if (!aligned16(k) || !aligned16(v) || !aligned16(workspace)) return REHYAT_ERR_MISALIGNED;
-  const FwdWorkspace w = fwd_layout(p);
-  if (ws_bytes < w.total) return REHYAT_ERR_WORKSPACE;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  char* ws = static_cast<char*>(workspace);
-  float* P = reinterpret_cast<float*>(ws + w.P_off);
-  float* z = reinterpret_cast<float*>(ws + w.z_off);
-  float* SL = reinterpret_cast<float*>(ws + w.SL_off);
-  float* zL = reinterpret_cast<float*>(ws + w.zL_off);
-  const int BH = p->batch * p->heads;
-  const int HW = p->Hs * p->Ws;
-
-  PartialParams pp = {};
-  pp.k = k; pp.v = v;
-  pp.rows_per_bh = static_cast<long long>(p->T) * HW;
-  pp.Wk = phi->Wk; pp.bk = phi->bk;
-  pp.P = P; pp.z = z;
-  pp.BH = BH; pp.heads = p->heads; pp.HW = HW; pp.D = p->D; pp.Dp = p->Dp; pp.To = p->To;
-  pp.nslots = p->T;
-  pp.in_bf16 = p->in_dtype == REHYAT_BF16;
-  pp.w_bf16 = pp.in_bf16;
-  cudaError_t e = cudaSuccess;
-  if (tc_path(p) || tc_state_path(p))
-    e = launch_w_images(phi->Wq, ws + w.wimg_off, phi->Wk, ws + w.wkimg_off, p->heads, p->D,
-                        p->Dp, s);
-  if (e != cudaSuccess) return to_status(e);
-  e = run_partials(p, pp, ws + w.wkimg_off, s);
-  if (e != cudaSuccess) return to_status(e);
-  return to_status(launch_scan(P, z, SL, zL, BH, p->T, p->Tc, p->To, nchunks_of(p), p->Dp,
-                               p->D, p->causal, s));
+  if (ws_bytes < fwd_layout(p).total) return REHYAT_ERR_WORKSPACE;
+  return state_pass(p, k, v, phi, static_cast<char*>(workspace),
+                    static_cast<cudaStream_t>(stream));
 }
 
 rehyat_status rehyat_fwd_attn(const rehyat_params* p, const void* q, const void* k,
@@ -403,6 +410,48 @@ rehyat_status rehyat_chunk_step(const rehyat_params* p, const void* q, const voi
   return to_status(launch_step_finish(P, zp, s_state, z_state, seen, done, BH, p->Dp, p->D,
                                       p->To, nslices, w.nslots, k, v, rk, rv, HW,
                                       elem_bytes(p->in_dtype), s));
+}
+
+size_t rehyat_phi_bwd_workspace_bytes(const rehyat_params* p) {
+  if (check_params(p) != REHYAT_OK) return 0;
+  int QS, KS;
+  phi_bwd_split(p->T, p->Tc, p->Hs * p->Ws, &QS, &KS);
+  const size_t parts = phi_bwd_partial_floats(p->batch * p->heads, p->T, nchunks_of(p), p->D,
+                                              p->Dp, QS, KS);
+  return fwd_layout(p).total + align_up(parts * sizeof(float));
+}
+
+rehyat_status rehyat_phi_bwd(const rehyat_params* p, const void* q, const void* k, const void* v,
+                             const float* y, const float* dy, const float* den,
+                             const rehyat_phi* phi, const rehyat_phi_grad* grad,
+                             void* workspace, size_t ws_bytes, void* stream) {
+  rehyat_status st = check_params(p);
+  if (st != REHYAT_OK) return st;
+  if (!q || !k || !v || !y || !dy || !den || !grad || !workspace) return REHYAT_ERR_INVALID_ARG;
+  if (!grad->dWq || !grad->dbq || !grad->dWk || !grad->dbk) return REHYAT_ERR_INVALID_ARG;
+  if ((st = check_phi(phi)) != REHYAT_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(y) || !aligned16(dy) ||
+      !aligned16(workspace) || (reinterpret_cast<uintptr_t>(den) & 3) ||
+      (reinterpret_cast<uintptr_t>(grad->dWq) & 3) || (reinterpret_cast<uintptr_t>(grad->dbq) & 3) ||
+      (reinterpret_cast<uintptr_t>(grad->dWk) & 3) || (reinterpret_cast<uintptr_t>(grad->dbk) & 3))
+    return REHYAT_ERR_MISALIGNED;
+  if (ws_bytes < rehyat_phi_bwd_workspace_bytes(p)) return REHYAT_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  // The linear-set state of every chunk, as the forward computes it.
+  if ((st = state_pass(p, k, v, phi, ws, s)) != REHYAT_OK) return st;
+  const FwdWorkspace w = fwd_layout(p);
+  PhiBwdArgs a;
+  a.q = q; a.k = k; a.v = v; a.y = y; a.dy = dy; a.den = den;
+  a.Wq = phi->Wq; a.bq = phi->bq; a.Wk = phi->Wk; a.bk = phi->bk;
+  a.SL = reinterpret_cast<const float*>(ws + w.SL_off);
+  a.zL = reinterpret_cast<const float*>(ws + w.zL_off);
+  a.partials = reinterpret_cast<float*>(ws + w.total);
+  a.dWq = grad->dWq; a.dbq = grad->dbq; a.dWk = grad->dWk; a.dbk = grad->dbk;
+  a.batch = p->batch; a.heads = p->heads; a.T = p->T; a.HW = p->Hs * p->Ws; a.D = p->D;
+  a.Dp = p->Dp; a.Tc = p->Tc; a.To = p->To; a.causal = p->causal; a.nchunks = nchunks_of(p);
+  a.in_bf16 = p->in_dtype == REHYAT_BF16;
+  return to_status(launch_phi_bwd(a, s));
 }
 
 }  // extern "C"

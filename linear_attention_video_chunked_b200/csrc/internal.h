@@ -57,6 +57,23 @@ struct PartialParams {
   int in_bf16, w_bf16;
 };
 
+// Gradient of the feature-map parameters (phi_bwd.cu).  q, k, v in the
+// forward's input dtype; y, dy, den fp32; SL, zL the linear-set state per
+// chunk as the forward's state pass leaves it; partials: a scratch array of
+// phi_bwd_partial_floats(...) floats.  Outputs overwrite dWq, dbq, dWk, dbk.
+struct PhiBwdArgs {
+  const void *q, *k, *v;
+  const float *y, *dy, *den;
+  const float *Wq, *bq, *Wk, *bk;
+  const float *SL, *zL;
+  float *partials;
+  float *dWq, *dbq, *dWk, *dbk;
+  int batch, heads, T, HW, D, Dp, Tc, To, causal, nchunks, in_bf16;
+};
+void phi_bwd_split(int T, int Tc, int HW, int* QS, int* KS);
+size_t phi_bwd_partial_floats(int BH, int T, int nchunks, int D, int Dp, int QS, int KS);
+cudaError_t launch_phi_bwd(const PhiBwdArgs& a, cudaStream_t s);
+
 // ---- SIMT (fp32 CUDA-core) kernels: every supported shape, both dtypes.
 cudaError_t launch_attn_simt(const AttnParams& p, cudaStream_t s);
 cudaError_t launch_partials_simt(const PartialParams& p, cudaStream_t s);

@@ -1,0 +1,121 @@
+"""GPU parity of the feature-map backward (rehyat_phi_bwd, through the C ABI)
+against the fp64 gradient oracle on the same seeded inputs.
+
+Bar (per gradient tensor, error relative to its largest magnitude):
+* fp32 CUDA-core forward and state pass (force_simt): <= 1e-4 -- only fp32
+  rounding separates the two;
+* default tensor-core forward and state pass, bf16 inputs: <= 3e-2 -- the
+  forward rounds P and phi_k to bf16 (relative 2^-9 per element), which
+  reaches y, the denominators and S_L that the gradient is built from.
+"""
+import numpy as np
+import pytest
+import torch
+
+import linear_attention_video_chunked_b200 as rh
+from oracle.rehyat_phi_grad import phi_grads
+from rehyat_inputs import config_problem, make_problem
+from tests.gpu_util import device_tensors
+
+pytestmark = pytest.mark.gpu
+
+NAMES = ("dWq", "dbq", "dWk", "dbk")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    rh.lib()
+    yield
+
+
+def _gpu_grads(p, dy, force_simt, dev=None):
+    dev = device_tensors(p) if dev is None else dev
+    kw = dict(T=p.T, Hs=p.Hs, Ws=p.Ws, Tc=p.Tc, To=p.To, causal=p.causal)
+    y, parts = rh.hybrid_attn(dev["q"], dev["k"], dev["v"], dev["Wq"], dev["bq"], dev["Wk"],
+                              dev["bk"], debug=True, force_simt=force_simt, **kw)
+    den = (parts["nS"] + parts["nL"]).contiguous()
+    dyt = torch.tensor(dy, dtype=torch.float32, device="cuda")
+    g = rh.phi_grad(dev["q"], dev["k"], dev["v"], y, dyt, den, dev["Wq"], dev["bq"], dev["Wk"],
+                    dev["bk"], force_simt=force_simt, **kw)
+    torch.cuda.synchronize()
+    return {n: g[n].double().cpu().numpy() for n in NAMES}
+
+
+def _ref(p, dy, heads=None):
+    if heads is None:
+        return phi_grads(p.q, p.k, p.v, p.Wq, p.bq, p.Wk, p.bk, dy, T=p.T, HW=p.HW, Tc=p.Tc,
+                         To=p.To, causal=p.causal)
+    # Per-head parameters: the gradient of head h only needs head h's data.
+    sel = lambda a: np.asarray(a)[:, heads]
+    r = phi_grads(sel(p.q), sel(p.k), sel(p.v), np.asarray(p.Wq)[heads],
+                  np.asarray(p.bq)[heads], np.asarray(p.Wk)[heads], np.asarray(p.bk)[heads],
+                  np.asarray(dy)[:, heads], T=p.T, HW=p.HW, Tc=p.Tc, To=p.To, causal=p.causal)
+    return r
+
+
+def _check(got, ref, tol, heads=None):
+    for n in NAMES:
+        g = got[n] if heads is None else got[n][heads]
+        scale = np.abs(ref[n]).max()
+        err = np.abs(g - ref[n]).max()
+        assert err <= tol * max(scale, 1e-30), f"{n}: max err {err:.3e} vs max |ref| {scale:.3e}"
+
+
+SHAPES = [
+    # B, h, T, Hs, Ws, D, Dp, Tc, To, causal
+    (2, 2, 5, 7, 9, 128, 128, 2, 1, False),   # ragged tiles, batch sum
+    (1, 2, 7, 10, 13, 128, 128, 3, 2, True),
+    (1, 3, 6, 8, 12, 64, 256, 2, 0, False),   # two feature pieces
+    (1, 2, 9, 11, 12, 32, 64, 3, 4, True),    # T_o > T_c
+]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_phi_grad_simt_forward_tight(shape, dtype):
+    B, h, T, Hs, Ws, D, Dp, Tc, To, causal = shape
+    p = make_problem(batch=B, heads=h, T=T, Hs=Hs, Ws=Ws, D=D, Dp=Dp, Tc=Tc, To=To,
+                     causal=causal, dtype=dtype, seed=200 + sum(shape[:9]), phi_std=0.1)
+    dy = np.random.default_rng(7).standard_normal(np.shape(p.q))
+    _check(_gpu_grads(p, dy, force_simt=True), _ref(p, dy), 1e-4)
+
+
+@pytest.mark.parametrize("shape", SHAPES[:3], ids=lambda s: "x".join(map(str, s)))
+def test_phi_grad_tensor_core_path(shape):
+    B, h, T, Hs, Ws, D, Dp, Tc, To, causal = shape
+    p = make_problem(batch=B, heads=h, T=T, Hs=Hs, Ws=Ws, D=D, Dp=Dp, Tc=Tc, To=To,
+                     causal=causal, dtype="bf16", seed=300 + sum(shape[:9]), phi_std=0.1)
+    dy = np.random.default_rng(8).standard_normal(np.shape(p.q))
+    _check(_gpu_grads(p, dy, force_simt=False), _ref(p, dy), 3e-2)
+
+
+def test_phi_grad_no_linear_set_is_zero():
+    p = make_problem(batch=1, heads=2, T=4, Hs=5, Ws=6, D=64, Dp=64, Tc=4, To=1, causal=False,
+                     dtype="f32", seed=9)
+    dy = np.random.default_rng(9).standard_normal(np.shape(p.q))
+    got = _gpu_grads(p, dy, force_simt=True)
+    for n in NAMES:
+        assert np.all(got[n] == 0.0), n
+
+
+def test_phi_grad_repeatable_bitwise():
+    p = make_problem(batch=1, heads=2, T=6, Hs=8, Ws=9, D=128, Dp=128, Tc=2, To=1, causal=True,
+                     dtype="bf16", seed=10)
+    dy = np.random.default_rng(10).standard_normal(np.shape(p.q))
+    dev = device_tensors(p)
+    a = _gpu_grads(p, dy, force_simt=False, dev=dev)
+    b = _gpu_grads(p, dy, force_simt=False, dev=dev)
+    for n in NAMES:
+        assert np.array_equal(a[n], b[n]), n
+
+
+def test_phi_grad_wan_320x480_causal_sampled_heads():
+    """Latent 21x20x30, 12 heads, D = D' = 128, T_c = 3, T_o = 1, causal: the
+    gradients of three sampled heads against the oracle (fp32 forward)."""
+    p = config_problem("wan_320x480_causal")
+    dy = np.random.default_rng(11).standard_normal(np.shape(p.q)).astype(np.float32)
+    heads = [0, 5, 11]
+    got = _gpu_grads(p, dy, force_simt=True)
+    _check(got, _ref(p, dy, heads), 1e-4, heads)
