@@ -235,6 +235,62 @@ def measure_full_softmax(rh, q, k, v, y, flush, stream, calls=3):
             "what": "rehyat_softmax_attn_fwd on the same q, k, v (all N keys per query)"}
 
 
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # CUDA-core fp32 FMA peak at 1965 MHz
+
+
+def measure_phi_backward(rh, p, q, k, v, Wq, bq, Wk, bk, flush, stream, calls=3):
+    """rehyat_phi_bwd on the bench workload: forward with the denominators
+    exported (nS, nL), an upstream gradient from a seeded torch generator,
+    then device time per backward call (fp32 CUDA-core kernels)."""
+    import torch
+    B, H, N, D = q.shape
+    dev = q.device
+    params = rh.make_params(batch=B, heads=H, T=p.T, Hs=p.Hs, Ws=p.Ws, D=D, Dp=p.Dp, Tc=p.Tc,
+                            To=p.To, causal=p.causal, in_dtype=rh.BF16, out_dtype=rh.F32)
+    sh = stream.cuda_stream
+    phi = rh.RehyatPhi(Wq.data_ptr(), bq.data_ptr(), Wk.data_ptr(), bk.data_ptr())
+    y = torch.empty(B, H, N, D, device=dev)
+    nS = torch.empty(B, H, N, device=dev)
+    nL = torch.empty(B, H, N, device=dev)
+    dbg = rh.RehyatDebug(None, nS.data_ptr(), None, None, nL.data_ptr())
+    ws = torch.empty(max(rh.rehyat_workspace_bytes(params), rh.rehyat_phi_bwd_workspace_bytes(params)),
+                     dtype=torch.uint8, device=dev)
+    if rh.rehyat_hybrid_attn_fwd(params, q.data_ptr(), k.data_ptr(), v.data_ptr(), phi,
+                                 y.data_ptr(), ws.data_ptr(), ws.numel(), dbg, sh):
+        raise RuntimeError("rehyat_hybrid_attn_fwd failed")
+    den = nS + nL
+    g = torch.Generator(device=dev).manual_seed(5)
+    dy = torch.randn(B, H, N, D, generator=g, device=dev)
+    grads = {n: torch.empty_like(t) for n, t in (("dWq", Wq), ("dbq", bq), ("dWk", Wk), ("dbk", bk))}
+    gs = rh.RehyatPhiGrad(*(grads[n].data_ptr() for n in ("dWq", "dbq", "dWk", "dbk")))
+    call = lambda: rh.rehyat_phi_bwd(params, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                     y.data_ptr(), dy.data_ptr(), den.data_ptr(), phi, gs,
+                                     ws.data_ptr(), ws.numel(), sh)
+    if call():
+        raise RuntimeError("rehyat_phi_bwd failed")
+    times = []
+    for _ in range(calls):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        call()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    ms = sum(times) / len(times)
+    # Algorithmic FLOPs of the backward proper (per token and (b,h): u_q, dphi_q,
+    # dW_q, G_t on the q side, u_k, dphi_k, dW_k on the k side, each 2*D*D'),
+    # plus the state pass it repeats (phi_k and phi_k^T v: 4*D*D').
+    flops = B * H * N * D * p.Dp * 2.0 * (7 + 2)
+    del y, nS, nL, ws, dy
+    return {"ms": ms, "calls": calls, "tflops": flops / (ms / 1e3) / 1e12,
+            "roofline": {"bound": "alu", "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
+                         "frac": flops / (ms / 1e3) / 1e12 / FP32_ALU_TFLOPS,
+                         "peak_source": "148 SMs x 128 fp32 FMA lanes x 2 x 1965 MHz"},
+            "what": "rehyat_phi_bwd (dW_q, db_q, dW_k, db_k) on the bench workload, bf16 "
+                    "q/k/v, fp32 y, dy, den; includes its state pass"}
+
+
 def measure_streaming(rh, dev, flush, stream):
     """Chunk-wise RNN over 81 slices of 30x52 (27 steps of T_c = 3, T_o = 1,
     12 heads, D = D' = 128): per-step device time, steady-state tokens/s,
@@ -578,7 +634,11 @@ def run_gpu(args, world, rank, local):
     extra = {}
     if not args.no_extras:
         extra["full_softmax"] = measure_full_softmax(rh, q, k, v, y, flush, stream)
-        del q, k, v, y, ws
+        del y, ws
+        torch.cuda.empty_cache()
+        extra["phi_backward"] = measure_phi_backward(rh, p, q, k, v, Wq, bq, Wk, bk, flush,
+                                                     stream)
+        del q, k, v
         torch.cuda.empty_cache()
         extra["streaming"] = measure_streaming(rh, dev, flush, stream)
 
