@@ -15,6 +15,10 @@ __device__ unsigned int rehyat_tc_error = 0;
 namespace tc {
 
 constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at the boost clock
+#ifndef REHYAT_TEST_FIRST
+#define REHYAT_TEST_FIRST 1
+#endif
+constexpr bool kTestFirst = REHYAT_TEST_FIRST != 0;
 
 // ------------------------------------------------------------ PTX helpers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -67,10 +71,27 @@ __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity,
   }
 }
 
+// Non-blocking check of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
                                           volatile uint32_t* abort_flag, uint32_t code) {
+  // A phase that has already completed is seen by the non-blocking test;
+  // otherwise try_wait suspends the thread until the phase completes (or a
+  // time limit passes).
+  if (kTestFirst && mbar_test(bar, parity)) return true;
 #pragma unroll 1
-  for (int i = 0; i < 4; ++i)  // try_wait itself suspends the thread for a while
+  for (int i = 0; i < 4; ++i)
     if (mbar_try(bar, parity)) return true;
   return mbar_wait_slow(bar, parity, abort_flag, code);
 }

@@ -1094,8 +1094,11 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
 //   warps 4-7  epilogue: drain the finished slice's P from TMEM;
 //   warp 8     TMA (K, V tiles; the W_k piece when (head, half) changes);
 //   warp 9     MMA (psi^T, P += phi^T V) and TMEM owner.
-// TMEM: psi/phi buffers [0,128) [128,256) (alternating per token tile), P
-// accumulators [256,384) [384,512) (alternating per item).
+// TMEM: psi^T buffers [0,128) [128,256) and phi^T buffers [256,320) [320,384)
+// (alternating per token tile; phi^T is bf16 pairs, so psi^T of the tile
+// after next can be written as soon as the converter has read this one),
+// one P accumulator [384,512) (the epilogue drains it while the next item's
+// first tile is converted).
 // D' in {64, 128, 256}: with D' = 256 an item is one 128-feature half of a
 // slice (items run over (b*h, half, slice), so W_k changes only at half or
 // head boundaries); with D' = 64 the upper 64 W_k rows stay zero.
@@ -1113,12 +1116,15 @@ constexpr uint32_t kKOff = 0;          // K ring, 3 x 32 KB
 constexpr uint32_t kVOff = 98304;      // V ring, 3 x 32 KB
 constexpr uint32_t kWOff = 196608;     // W_k piece, 2 boxes x 128 rows x 128 B
 constexpr uint32_t kBarOff = 229376;
-enum { K_FULL = 0, K_EMPTY = 3, V_FULL = 6, V_EMPTY = 9, PSI_FULL = 12, PHI_FULL = 14,
-       BUF_FREE = 16, ACC_DONE = 18, P_FREE = 20, W_FULL = 22, W_FREE = 23, NBAR = 24 };
+enum { K_FULL = 0, K_EMPTY = 3, V_FULL = 6, V_EMPTY = 9, PSI_FULL = 12, PSI_FREE = 14,
+       PHI_FULL = 16, PHI_FREE = 18, ACC_DONE = 20, P_FREE = 21, W_FULL = 22, W_FREE = 23,
+       NBAR = 24 };
 constexpr uint32_t kTmemSlot = kBarOff + 8 * NBAR;
 constexpr uint32_t kAbortSlot = kTmemSlot + 4;
 constexpr uint32_t kSmemBytes = kBarOff + 256 + 1024;
-constexpr uint32_t kColBuf = 0, kColP = 256;
+// TMEM: psi^T fp32 [0,128) [128,256), phi^T bf16 pairs [256,320) [320,384)
+// (each alternating per token tile), P accumulator [384,512).
+constexpr uint32_t kColPsi = 0, kColPhi = 256, kColP = 384;
 
 // Walk over a CTA's run of items i = q * T + slice, q = bh * halves + half,
 // with a division only when one (bh, half) run of slices ends.
@@ -1157,14 +1163,15 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
   // Local names shadow the attention kernel's constants of the same names.
   constexpr int kS = sp::kStages;
   constexpr uint32_t kKOff = sp::kKOff, kVOff = sp::kVOff, kWOff = sp::kWOff;
-  constexpr uint32_t kColBuf = sp::kColBuf, kColP = sp::kColP;
+  constexpr uint32_t kColPsi = sp::kColPsi, kColPhi = sp::kColPhi, kColP = sp::kColP;
   using sp::K_FULL;
   using sp::K_EMPTY;
   using sp::V_FULL;
   using sp::V_EMPTY;
   using sp::PSI_FULL;
+  using sp::PSI_FREE;
   using sp::PHI_FULL;
-  using sp::BUF_FREE;
+  using sp::PHI_FREE;
   using sp::ACC_DONE;
   using sp::P_FREE;
   using sp::W_FULL;
@@ -1216,7 +1223,8 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
 
   if (tid == 0) {
     for (int i = 0; i < NBAR; ++i) {
-      const bool by_group = i == PHI_FULL || i == PHI_FULL + 1 || i == P_FREE || i == P_FREE + 1;
+      const bool by_group = i == PSI_FREE || i == PSI_FREE + 1 || i == PHI_FULL ||
+                            i == PHI_FULL + 1 || i == P_FREE;
       mbar_init(bar(i), by_group ? 128 : 1);
     }
     *abort_flag = 0;
@@ -1324,7 +1332,7 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
           ++wwaits;
         }
         if (!mbar_wait(bar(K_FULL + pst), puses & 1, abort_flag, 31)) return false;
-        if (pgt >= 2 && !mbar_wait(bar(BUF_FREE + b), ((pgt - 2) >> 1) & 1, abort_flag, 32))
+        if (pgt >= 2 && !mbar_wait(bar(PSI_FREE + b), ((pgt - 2) >> 1) & 1, abort_flag, 32))
           return false;
         tc_fence_after();
         const uint64_t wdesc = sdesc(base + kWOff, 16, 1024);
@@ -1333,7 +1341,7 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
         for (int kk = 0; kk < 8; ++kk) {
           // Descriptor start addresses are in 16-byte units (no carry: < 2^14).
           const uint64_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
-          mma_bf16(tmem + kColBuf + b * 128, wdesc + off, kdesc + off, id_psi, kk > 0);
+          mma_bf16(tmem + kColPsi + b * 128, wdesc + off, kdesc + off, id_psi, kk > 0);
         }
         mma_commit(bar(PSI_FULL + b));
         mma_commit(bar(K_EMPTY + pst));
@@ -1352,13 +1360,12 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
       if (TT > 0) ok = issue_psi();
       int gt = 0, vst = 0, vuses = 0;
       for (int ia = 0; ia < nactive && ok; ++ia) {  // active items
-        const int pb = ia & 1;
         for (int j = 0; j < nt && ok; ++j, ++gt) {
           const int b = gt & 1;
           if (gt + 1 < TT) ok = issue_psi();
           if (!ok) break;
-          if (j == 0 && ia >= 2)
-            ok = mbar_wait(bar(P_FREE + pb), ((ia - 2) >> 1) & 1, abort_flag, 33);
+          if (j == 0 && ia >= 1)  // the epilogue has drained the previous item
+            ok = mbar_wait(bar(P_FREE), (ia - 1) & 1, abort_flag, 33);
           if (ok) ok = mbar_wait(bar(PHI_FULL + b), (gt >> 1) & 1, abort_flag, 34) &&
                        mbar_wait(bar(V_FULL + vst), vuses & 1, abort_flag, 35);
           if (!ok) break;
@@ -1366,11 +1373,11 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
           const uint64_t vdesc = sdesc(base + kVOff + vst * 32768, 16384, 1024);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_bf16_ts(tmem + kColP + pb * 128, tmem + kColBuf + b * 128 + kk * 8,
+            mma_bf16_ts(tmem + kColP, tmem + kColPhi + b * 64 + kk * 8,
                         vdesc + ((kk * 2048) >> 4), id_pv, (j > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(bar(BUF_FREE + b));
+          mma_commit(bar(PHI_FREE + b));
           mma_commit(bar(V_EMPTY + vst));
-          if (j == nt - 1) mma_commit(bar(ACC_DONE + pb));
+          if (j == nt - 1) mma_commit(bar(ACC_DONE));
           if (++vst == kS) {
             vst = 0;
             ++vuses;
@@ -1403,12 +1410,15 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
       for (int j = 0; j < nt && ok; ++j, ++gt) {
         const int b = gt & 1;
         ok = wait_all(bar(PSI_FULL + b), (gt >> 1) & 1, 36);
+        // phi^T buffer b is free once phi^T V of tile gt - 2 has read it.
+        if (ok && gt >= 2) ok = wait_all(bar(PHI_FREE + b), ((gt - 2) >> 1) & 1, 38);
         if (!ok) break;
         tc_fence_after();
         const int nvalid = min(128, HW - j * 128);
-        const uint32_t cols = lane_base + kColBuf + b * 128;
-        // 32 tokens at a time: phi of tokens 32c.. is written as 16 packed
-        // columns at 16c, behind the columns already read.
+        const uint32_t cols = lane_base + kColPsi + b * 128;
+        const uint32_t pcols = lane_base + kColPhi + b * 64;
+        // 32 tokens at a time: phi of tokens 32c.. becomes 16 packed columns
+        // at 16c of the phi^T buffer.
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t ps[32], pk[16];
@@ -1431,7 +1441,7 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
             zacc = f2_add(zacc, f2_pack(__uint_as_float(pk[i] << 16),
                                         __uint_as_float(pk[i] & 0xFFFF0000u)));
           }
-          REHYAT_TMEM_ST16(cols + c * 16, pk);
+          REHYAT_TMEM_ST16(pcols + c * 16, pk);
         }
         tmem_wait_st();
         if (nvalid < 128) {
@@ -1447,6 +1457,7 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
           fence_proxy_async();
         }
         tc_fence_before();
+        mbar_arrive(bar(PSI_FREE + b));
         mbar_arrive(bar(PHI_FULL + b));
         if (++vst == kS) {
           vst = 0;
@@ -1470,8 +1481,7 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
     int ia = 0;  // active items so far
     for (int il = 0; il < nitems && ok; ++il, w.next()) {
       if (!w.on()) continue;
-      const int pb = ia & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(ACC_DONE + pb), (ia >> 1) & 1, abort_flag, 39));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(ACC_DONE), ia & 1, abort_flag, 39));
       ++ia;
       if (!ok) break;
       tc_fence_after();
@@ -1481,7 +1491,7 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
       float* prow = P.P + w.out_index(P.nslots) * Dp * 128 + sl_feature_base(fg, 128, Dp);
       for (int c = 0; c < 4; ++c) {
         uint32_t v[32];
-        REHYAT_TMEM_LD32(lane_base + kColP + pb * 128 + c * 32, v);
+        REHYAT_TMEM_LD32(lane_base + kColP + c * 32, v);
         tmem_wait_ld();
         if (f < pw) {
 #pragma unroll
@@ -1489,7 +1499,7 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(bar(P_FREE + pb));
+      mbar_arrive(bar(P_FREE));
     }
   }
 
