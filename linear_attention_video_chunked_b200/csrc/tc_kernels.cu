@@ -1093,7 +1093,9 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
 //   warps 0-3  convert (thread = feature), z;
 //   warps 4-7  epilogue: drain the finished slice's P from TMEM;
 //   warp 8     TMA (K, V tiles; the W_k piece when (head, half) changes);
-//   warp 9     MMA (psi^T, P += phi^T V) and TMEM owner.
+//   warp 9     MMA psi^T = W_k^T K^T, and TMEM owner;
+//   warp 10    MMA P += phi^T V (a second issuer, so the two streams' waits
+//              and issue overheads overlap in front of one tensor pipe).
 // TMEM: psi^T buffers [0,128) [128,256) and phi^T buffers [256,320) [320,384)
 // (alternating per token tile; phi^T is bf16 pairs, so psi^T of the tile
 // after next can be written as soon as the converter has read this one),
@@ -1110,7 +1112,7 @@ struct StMaps {
 };
 
 namespace sp {
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
 constexpr int kStages = 3;             // K and V ring depth
 constexpr uint32_t kKOff = 0;          // K ring, 3 x 32 KB
 constexpr uint32_t kVOff = 98304;      // V ring, 3 x 32 KB
@@ -1308,10 +1310,9 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
     }
     __syncwarp();
   } else if (warp == 9) {
-    // ================================================= MMA issuer
+    // ================================================= psi^T MMA issuer
     if (lane == 0) {
       const uint32_t id_psi = idesc(128, 128, 1, false);  // W_k piece and K tile, K-major
-      const uint32_t id_pv = idesc(128, 128, 1, true);    // phi^T from TMEM, V MN-major
       bool ok = true;
       int wwaits = 0, wkey = -1;
       // The next psi^T to issue: its tile index, item walk (on active
@@ -1357,13 +1358,21 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
         }
         return true;
       };
-      if (TT > 0) ok = issue_psi();
+      for (int g = 0; g < TT && ok; ++g) ok = issue_psi();
+    }
+    __syncwarp();
+  } else if (warp == 10) {
+    // ================================================= phi^T V MMA issuer
+    // (a second issuing thread: its MMAs read phi^T and V and accumulate P,
+    // operands the psi^T issuer never touches; each commit tracks this
+    // thread's own MMAs)
+    if (lane == 0) {
+      const uint32_t id_pv = idesc(128, 128, 1, true);  // phi^T from TMEM, V MN-major
+      bool ok = true;
       int gt = 0, vst = 0, vuses = 0;
       for (int ia = 0; ia < nactive && ok; ++ia) {  // active items
         for (int j = 0; j < nt && ok; ++j, ++gt) {
           const int b = gt & 1;
-          if (gt + 1 < TT) ok = issue_psi();
-          if (!ok) break;
           if (j == 0 && ia >= 1)  // the epilogue has drained the previous item
             ok = mbar_wait(bar(P_FREE), (ia - 1) & 1, abort_flag, 33);
           if (ok) ok = mbar_wait(bar(PHI_FULL + b), (gt >> 1) & 1, abort_flag, 34) &&
