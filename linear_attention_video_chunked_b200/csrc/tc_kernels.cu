@@ -24,6 +24,8 @@
 //
 // Every wait is bounded: a barrier that does not complete within ~2 s of
 // clock sets an error bit in rehyat_tc_error and the kernel unwinds.
+#include <atomic>
+
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -1092,7 +1094,8 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
 // P += phi^T V (the TMEM-A form), and it sums z = sum_t phi itself.
 //   warps 0-3  convert (thread = feature), z;
 //   warps 4-7  epilogue: drain the finished slice's P from TMEM;
-//   warp 8     TMA (K, V tiles; the W_k piece when (head, half) changes);
+//   warp 8     TMA of K tiles (and the W_k piece when (head, half) changes);
+//   warp 11    TMA of V tiles;
 //   warp 9     MMA psi^T = W_k^T K^T, and TMEM owner;
 //   warp 10    MMA P += phi^T V (a second issuer, so the two streams' waits
 //              and issue overheads overlap in front of one tensor pipe).
@@ -1112,7 +1115,7 @@ struct StMaps {
 };
 
 namespace sp {
-constexpr int kThreads = 352;
+constexpr int kThreads = 384;
 constexpr int kStages = 3;             // K and V ring depth
 constexpr uint32_t kKOff = 0;          // K ring, 3 x 32 KB
 constexpr uint32_t kVOff = 98304;      // V ring, 3 x 32 KB
@@ -1252,18 +1255,23 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sbase + sp::kTmemSlot);
 
-  if (warp == 8) {
-    // ================================================= TMA producer
+  if (warp == 8 || warp == 11) {
+    // ================================================= TMA producers
+    // warp 8 loads K tiles (and the W_k piece), warp 11 V tiles, so K runs
+    // ahead on its own ring (psi^T) while V waits for phi^T V to free stages.
     if (lane == 0) {
+      const bool kside = warp == 8;
       bool ok = true;
       int wloads = 0, wkey = -1;
       const uint32_t box_bytes = static_cast<uint32_t>(pw) * 128;  // one 64-column box
+      const uint32_t ring = kside ? kKOff : kVOff;
+      const int full = kside ? K_FULL : V_FULL, empty = kside ? K_EMPTY : V_EMPTY;
       sp::ItemWalk w{T, halves, P.heads, pw, leave};
       w.start(it0);
       int gt = 0, st = 0, uses = 0;  // tile index, its ring stage, earlier uses of the stage
       for (int il = 0; il < nitems && ok; ++il, w.next()) {
         if (!w.on()) continue;
-        if (w.wkey != wkey) {
+        if (kside && w.wkey != wkey) {
           wkey = w.wkey;
           if (wloads > 0) ok = mbar_wait(bar(W_FREE), (wloads - 1) & 1, abort_flag, 27);
           if (!ok) break;
@@ -1276,14 +1284,12 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
           ++wloads;
         }
         const int bh = w.bh();
-        const CUtensorMap* mk = &maps.k;
-        const CUtensorMap* mv = &maps.v;
+        const CUtensorMap* map = kside ? &maps.k : &maps.v;
         int row0 = w.slice * HW;
         if (step) {
           const long long g = seen0 - rseen + w.slice;  // global slice of this slot
           if (g < seen0) {
-            mk = &maps.rk;
-            mv = &maps.rv;
+            map = kside ? &maps.rk : &maps.rv;
             row0 = static_cast<int>(g % P.To) * HW;
           } else {
             row0 = static_cast<int>(g - seen0) * HW;
@@ -1291,16 +1297,11 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
         }
         for (int j = 0; j < nt && ok; ++j, ++gt) {
           const int row = row0 + j * 128;
-          if (gt >= kS) ok = mbar_wait(bar(K_EMPTY + st), (uses - 1) & 1, abort_flag, 28);
+          if (gt >= kS) ok = mbar_wait(bar(empty + st), (uses - 1) & 1, abort_flag, kside ? 28 : 29);
           if (!ok) break;
-          mbar_expect_tx(bar(K_FULL + st), 32768);
-          tma_load_3d(base + kKOff + st * 32768, mk, bar(K_FULL + st), 0, row, bh);
-          tma_load_3d(base + kKOff + st * 32768 + 16384, mk, bar(K_FULL + st), 64, row, bh);
-          if (gt >= kS) ok = mbar_wait(bar(V_EMPTY + st), (uses - 1) & 1, abort_flag, 29);
-          if (!ok) break;
-          mbar_expect_tx(bar(V_FULL + st), 32768);
-          tma_load_3d(base + kVOff + st * 32768, mv, bar(V_FULL + st), 0, row, bh);
-          tma_load_3d(base + kVOff + st * 32768 + 16384, mv, bar(V_FULL + st), 64, row, bh);
+          mbar_expect_tx(bar(full + st), 32768);
+          tma_load_3d(base + ring + st * 32768, map, bar(full + st), 0, row, bh);
+          tma_load_3d(base + ring + st * 32768 + 16384, map, bar(full + st), 64, row, bh);
           if (++st == kS) {
             st = 0;
             ++uses;
@@ -1522,6 +1523,36 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
 }
 
 // ------------------------------------------------------------ host side
+// Per-device one-time launch setup: SM count, and the dynamic shared-memory
+// limit of each tensor-core kernel (the attribute is per context, so it is
+// set once per device and kernel, not on every call).
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sm_count[kMaxDevices];
+std::atomic<unsigned> g_smem_set[kMaxDevices];
+
+int sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  int n = g_sm_count[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    g_sm_count[dev].store(n, std::memory_order_relaxed);
+  }
+  return n;
+}
+
+template <typename Kernel>
+cudaError_t ensure_smem(Kernel* fn, unsigned bit, uint32_t bytes) {
+  int dev = 0;
+  const bool cached = cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxDevices;
+  if (cached && (g_smem_set[dev].load(std::memory_order_acquire) & (1u << bit))) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(bytes));
+  if (e == cudaSuccess && cached) g_smem_set[dev].fetch_or(1u << bit, std::memory_order_release);
+  return e;
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (!fn) {
@@ -1570,16 +1601,12 @@ cudaError_t launch_state_tc(const PartialParams& p, const void* wk_img, cudaStre
     maps.rv = maps.v;
   }
   // Persistent CTAs, each with the same number of items.
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess)
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = sm_count();
   const int per_bh = (p.seen ? p.nq_slices : p.nslots) * (p.Dp > 128 ? p.Dp / 128 : 1);
   const int total = p.BH * per_bh;
   const int per_cta = (total + sms - 1) / sms;
   const int ctas = (total + per_cta - 1) / per_cta;
-  cudaError_t e = cudaFuncSetAttribute(tc_state_persistent_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(sp::kSmemBytes));
+  const cudaError_t e = ensure_smem(tc_state_persistent_kernel, 0, sp::kSmemBytes);
   if (e != cudaSuccess) return e;
   const __nv_bfloat16* wk = static_cast<const __nv_bfloat16*>(wk_img);
   if (p.seen == nullptr) {
@@ -1635,15 +1662,13 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s) {
   const bool two_tiles = !p.one_tile && (p.full_softmax || p.Dp <= 128);
   cudaError_t e;
   if (two_tiles) {
-    e = cudaFuncSetAttribute(tc_attn2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(a2::kSmemBytes));
+    e = ensure_smem(tc_attn2_kernel, 1, a2::kSmemBytes);
     if (e != cudaSuccess) return e;
     dim3 grid((qrows_max + 2 * kBM - 1) / (2 * kBM), p.nchunks, p.BH);
     tc_attn2_kernel<<<grid, a2::kThreads, a2::kSmemBytes, s>>>(
         maps, p, static_cast<const __nv_bfloat16*>(p.wq_img));
   } else {
-    e = cudaFuncSetAttribute(tc_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kSmemBytes));
+    e = ensure_smem(tc_attn_kernel, 2, kSmemBytes);
     if (e != cudaSuccess) return e;
     dim3 grid((qrows_max + kBM - 1) / kBM, p.nchunks, p.BH);
     tc_attn_kernel<<<grid, kThreads, kSmemBytes, s>>>(
