@@ -1,0 +1,86 @@
+"""Pins of the general feature map and of the phi-given forward oracle
+(oracle/rehyat_phi_mlp.py), CPU only.
+
+* GELU against scipy.stats.norm.cdf (x * Phi(x)) and its odd part
+  gelu(x) - gelu(-x) = x;
+* the P-part powers: part i of phi equals the i-th power of part i of the
+  P = 1 map (which is psi itself);
+* the phi-given forward with phi computed by the degree-2 closed form equals
+  the pinned factored forward, and with a general (partly negative) phi it
+  equals a brute-force pairwise evaluation of the masked definition.
+"""
+import numpy as np
+import pytest
+from scipy.stats import norm
+
+from oracle import rehyat_oracle as orc
+from oracle.rehyat_phi_mlp import feature_map_mlp, gelu, hybrid_phi_given
+from rehyat_inputs import make_problem
+
+
+def test_gelu_matches_normal_cdf_and_odd_part():
+    x = np.random.default_rng(0).standard_normal(1000) * 3
+    assert np.allclose(gelu(x), x * norm.cdf(x), rtol=1e-13, atol=1e-15)
+    assert np.allclose(gelu(x) - gelu(-x), x, rtol=1e-13, atol=1e-14)
+    assert gelu(0.0) == 0.0
+
+
+@pytest.mark.parametrize("P", [1, 2, 4])
+def test_parts_are_powers_of_psi(P):
+    rng = np.random.default_rng(1)
+    D, Dh, Dp = 8, 24, 16
+    x = rng.standard_normal((5, D))
+    Wa, ba = rng.standard_normal((D, Dh)) * 0.3, rng.standard_normal(Dh) * 0.1
+    Wb, bb = rng.standard_normal((Dh, Dp)) * 0.3, rng.standard_normal(Dp) * 0.1
+    psi = feature_map_mlp(x, Wa, ba, Wb, bb, 1)
+    phi = feature_map_mlp(x, Wa, ba, Wb, bb, P)
+    w = Dp // P
+    for i in range(P):
+        assert np.allclose(phi[:, i * w:(i + 1) * w], psi[:, i * w:(i + 1) * w] ** (i + 1),
+                           rtol=1e-13)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_phi_given_equals_factored_with_closed_form_phi(causal):
+    p = make_problem(batch=1, heads=2, T=5, Hs=2, Ws=3, D=8, Dp=8, Tc=2, To=1, causal=causal,
+                     dtype="f32", seed=3, phi_std=0.3)
+    fq = np.stack([np.stack([orc.feature_map(p.q[b, h], p.Wq[h], p.bq[h]) for h in range(2)])
+                   for b in range(1)])
+    fk = np.stack([np.stack([orc.feature_map(p.k[b, h], p.Wk[h], p.bk[h]) for h in range(2)])
+                   for b in range(1)])
+    y, parts = hybrid_phi_given(p.q, p.k, p.v, fq, fk, T=p.T, HW=p.HW, Tc=p.Tc, To=p.To,
+                                causal=causal)
+    ref_y, ref_p = orc.run_problem(p)
+    assert np.allclose(y, ref_y, rtol=1e-12, atol=1e-14)
+    for key in ref_p:
+        assert np.allclose(parts[key], ref_p[key], rtol=1e-12, atol=1e-14), key
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_phi_given_equals_pairwise_definition(causal):
+    """General phi with a degree-1 part (negative values allowed)."""
+    rng = np.random.default_rng(4)
+    T, HW, D, Dp, Tc, To = 6, 3, 4, 6, 2, 1
+    N = T * HW
+    q, k, v = (rng.standard_normal((1, 1, N, D)) for _ in range(3))
+    fq = rng.standard_normal((1, 1, N, Dp)) * 0.2
+    fk = rng.standard_normal((1, 1, N, Dp)) * 0.2
+    y, _ = hybrid_phi_given(q, k, v, fq, fk, T=T, HW=HW, Tc=Tc, To=To, causal=causal)
+    scale = 1 / np.sqrt(D)
+    Np = Tc * HW
+    for i in range(N):
+        t = i // Np
+        lo, hi = max(t * Np - To * HW, 0), min((t + 1) * Np, N)
+        num = np.zeros(D)
+        den = 0.0
+        c = max((q[0, 0, i] @ k[0, 0, j]) * scale for j in range(lo, hi))
+        for j in range(N):
+            if lo <= j < hi:
+                w = np.exp((q[0, 0, i] @ k[0, 0, j]) * scale - c)
+            elif (j < lo) or (not causal and j >= hi):
+                w = fq[0, 0, i] @ fk[0, 0, j]
+            else:
+                w = 0.0
+            num += w * v[0, 0, j]
+            den += w
+        assert np.allclose(y[0, 0, i], num / den, rtol=1e-10, atol=1e-12), i
