@@ -204,6 +204,40 @@ REHYAT_API rehyat_status rehyat_chunk_step(const rehyat_params* p, const void* q
                                 const rehyat_debug* dbg, void* stream);
 
 /* ---------------------------------------------------------------------- */
+/* General feature maps (Key design 3: phi_q, phi_k from a light per-head
+ * embedding network whose output psi is cut into P equal parts, part i
+ * raised to the i-th power, phi = [psi_1^1, ..., psi_P^P]).                */
+
+/* The same forward as rehyat_hybrid_attn_fwd with the feature maps given as
+ * arrays: phi_q = phi_q(q), phi_k = phi_k(k), fp32 [B][h][N][Dp], 16-byte
+ * aligned (any map, e.g. rehyat_feature_map_mlp's).  phi values may be
+ * negative (a degree-1 part), so n^L may be negative; y is the joint
+ * normalisation as written, without clamping the denominator.  Workspace as
+ * rehyat_workspace_bytes(p); other arguments and errors as for
+ * rehyat_hybrid_attn_fwd. */
+REHYAT_API rehyat_status rehyat_hybrid_attn_fwd_phi(const rehyat_params* p, const void* q,
+                                                    const void* k, const void* v,
+                                                    const float* phi_q, const float* phi_k,
+                                                    void* y, void* workspace, size_t ws_bytes,
+                                                    const rehyat_debug* dbg, void* stream);
+
+/* Per-head 2-layer MLP feature map, fp32 device arrays:
+ *   Wa [heads][D][Dh], ba [heads][Dh], Wb [heads][Dh][Dp], bb [heads][Dp];
+ *   psi = GELU(x Wa + ba) Wb + bb with GELU(u) = u * Phi(u) (exact form),
+ *   phi = [psi_1^1, ..., psi_P^P] over P = parts equal parts (Dp % parts == 0). */
+typedef struct {
+  const float *Wa, *ba, *Wb, *bb;
+  int Dh, parts;
+} rehyat_phi_mlp;
+
+/* phi [B][h][N][Dp] (fp32) of x [B][h][N][D] (p->in_dtype), N = T*Hs*Ws,
+ * heads and shapes from p (Tc, To, causal unused).  Dh <= 512.  Pointers
+ * 4-byte aligned.  REHYAT_ERR_INVALID_ARG for parts < 1 or Dp % parts != 0. */
+REHYAT_API rehyat_status rehyat_feature_map_mlp(const rehyat_params* p, const void* x,
+                                                const rehyat_phi_mlp* mlp, float* phi,
+                                                void* stream);
+
+/* ---------------------------------------------------------------------- */
 /* Backward for the feature maps (Key design 5: the first training stage,
  * block-wise attention distillation, updates only phi_q and phi_k).       */
 

@@ -30,7 +30,9 @@ __all__ = [
     "rehyat_chunk_step", "rehyat_device_error_flags", "rehyat_attn_path",
     "rehyat_status_string", "rehyat_version", "rehyat_hybrid_attn_fwd_noalloc",
     "RehyatPhiGrad", "rehyat_phi_bwd_workspace_bytes", "rehyat_phi_bwd",
-    "make_params", "hybrid_attn", "softmax_attn", "phi_grad", "StreamingState",
+    "RehyatPhiMlp", "rehyat_hybrid_attn_fwd_phi", "rehyat_feature_map_mlp",
+    "make_params", "hybrid_attn", "hybrid_attn_phi", "feature_map_mlp", "softmax_attn",
+    "phi_grad", "StreamingState",
 ]
 
 F32, BF16 = 0, 1
@@ -47,6 +49,7 @@ EXPORTED_SYMBOLS = (
     "rehyat_step_workspace_bytes", "rehyat_chunk_step", "rehyat_device_error_flags",
     "rehyat_attn_path", "rehyat_status_string", "rehyat_version",
     "rehyat_hybrid_attn_fwd_noalloc", "rehyat_phi_bwd_workspace_bytes", "rehyat_phi_bwd",
+    "rehyat_hybrid_attn_fwd_phi", "rehyat_feature_map_mlp",
 )
 
 
@@ -72,6 +75,11 @@ class RehyatDebug(ctypes.Structure):
 class RehyatPhiGrad(ctypes.Structure):
     _fields_ = [("dWq", ctypes.c_void_p), ("dbq", ctypes.c_void_p),
                 ("dWk", ctypes.c_void_p), ("dbk", ctypes.c_void_p)]
+
+
+class RehyatPhiMlp(ctypes.Structure):
+    _fields_ = [("Wa", ctypes.c_void_p), ("ba", ctypes.c_void_p), ("Wb", ctypes.c_void_p),
+                ("bb", ctypes.c_void_p), ("Dh", ctypes.c_int), ("parts", ctypes.c_int)]
 
 
 class RehyatError(RuntimeError):
@@ -139,6 +147,11 @@ def lib() -> ctypes.CDLL:
         L.rehyat_phi_bwd.argtypes = [P(RehyatParams), vp, vp, vp, vp, vp, vp, P(RehyatPhi),
                                      P(RehyatPhiGrad), vp, sz, vp]
         L.rehyat_phi_bwd.restype = i
+        L.rehyat_hybrid_attn_fwd_phi.argtypes = [P(RehyatParams), vp, vp, vp, vp, vp, vp, vp, sz,
+                                                 vp, vp]
+        L.rehyat_hybrid_attn_fwd_phi.restype = i
+        L.rehyat_feature_map_mlp.argtypes = [P(RehyatParams), vp, P(RehyatPhiMlp), vp, vp]
+        L.rehyat_feature_map_mlp.restype = i
         _LIB = L
     return _LIB
 
@@ -179,6 +192,17 @@ def rehyat_phi_bwd_workspace_bytes(p: RehyatParams) -> int:
 def rehyat_phi_bwd(p, q, k, v, y, dy, den, phi, grad, workspace, ws_bytes, stream) -> int:
     return lib().rehyat_phi_bwd(ctypes.byref(p), q, k, v, y, dy, den, ctypes.byref(phi),
                                 ctypes.byref(grad), workspace, ws_bytes, stream)
+
+
+def rehyat_hybrid_attn_fwd_phi(p, q, k, v, phi_q, phi_k, y, workspace, ws_bytes, dbg,
+                               stream) -> int:
+    return lib().rehyat_hybrid_attn_fwd_phi(ctypes.byref(p), q, k, v, phi_q, phi_k, y, workspace,
+                                            ws_bytes, None if dbg is None else ctypes.byref(dbg),
+                                            stream)
+
+
+def rehyat_feature_map_mlp(p, x, mlp, phi, stream) -> int:
+    return lib().rehyat_feature_map_mlp(ctypes.byref(p), x, ctypes.byref(mlp), phi, stream)
 
 
 def rehyat_softmax_attn_fwd(p, q, k, v, y, stream) -> int:
@@ -303,6 +327,57 @@ def hybrid_attn(q, k, v, Wq, bq, Wk, bk, *, T, Hs, Ws, Tc, To, causal, out_dtype
                                 workspace.data_ptr(), workspace.numel(), dbg_s,
                                 _stream_handle(stream))
     _check(st, "rehyat_hybrid_attn_fwd")
+    return (y, dbg_t) if debug else y
+
+
+def feature_map_mlp(x, Wa, ba, Wb, bb, *, parts, T, Hs, Ws, stream=None):
+    """phi = [psi_1^1, ..., psi_P^P], psi = GELU(x Wa + ba) Wb + bb per head,
+    of a torch CUDA tensor x [B, h, N, D]; Wa [h, D, Dh], ba [h, Dh],
+    Wb [h, Dh, D'], bb [h, D'] fp32.  Returns fp32 [B, h, N, D']."""
+    torch = _torch()
+    B, H, N, D = x.shape
+    Dh, Dp = Wa.shape[-1], Wb.shape[-1]
+    for t in (Wa, ba, Wb, bb):
+        if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous():
+            raise TypeError("MLP parameters must be contiguous fp32 CUDA tensors")
+    p = make_params(batch=B, heads=H, T=T, Hs=Hs, Ws=Ws, D=D, Dp=Dp, Tc=1, To=0, causal=0,
+                    in_dtype=_dtype_code(x.dtype), out_dtype=F32)
+    phi = torch.empty(B, H, N, Dp, dtype=torch.float32, device=x.device)
+    mlp = RehyatPhiMlp(Wa.data_ptr(), ba.data_ptr(), Wb.data_ptr(), bb.data_ptr(), Dh, parts)
+    _check(rehyat_feature_map_mlp(p, x.data_ptr(), mlp, phi.data_ptr(), _stream_handle(stream)),
+           "rehyat_feature_map_mlp")
+    return phi
+
+
+def hybrid_attn_phi(q, k, v, phi_q, phi_k, *, T, Hs, Ws, Tc, To, causal, out_dtype=None,
+                    scale=0.0, debug=False, force_simt=False, workspace=None, out=None,
+                    stream=None):
+    """The hybrid forward with the feature maps given: phi_q = phi_q(q) and
+    phi_k = phi_k(k), fp32 [B, h, N, D'] CUDA tensors.  Returns y (and the
+    branch partials when ``debug``)."""
+    torch = _torch()
+    B, H, N, D = q.shape
+    Dp = phi_q.shape[-1]
+    for t in (phi_q, phi_k):
+        if t.dtype != torch.float32 or not t.is_contiguous() or t.shape[:3] != q.shape[:3]:
+            raise TypeError("phi_q, phi_k must be contiguous fp32 [B, h, N, D'] tensors")
+    out_dtype = torch.float32 if out_dtype is None else out_dtype
+    p = make_params(batch=B, heads=H, T=T, Hs=Hs, Ws=Ws, D=D, Dp=Dp, Tc=Tc, To=To,
+                    causal=causal, in_dtype=_dtype_code(q.dtype),
+                    out_dtype=_dtype_code(out_dtype), scale=scale,
+                    flags=FLAG_FORCE_SIMT if force_simt else 0)
+    y = torch.empty(B, H, N, D, dtype=out_dtype, device=q.device) if out is None else out
+    nbytes = rehyat_workspace_bytes(p)
+    if nbytes == 0:
+        raise RehyatError(1, "rehyat_workspace_bytes")
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    dbg_t, dbg_s = _debug_tensors((B, H, N, D), q.device) if debug else (None, None)
+    st = rehyat_hybrid_attn_fwd_phi(p, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                    phi_q.data_ptr(), phi_k.data_ptr(), y.data_ptr(),
+                                    workspace.data_ptr(), workspace.numel(), dbg_s,
+                                    _stream_handle(stream))
+    _check(st, "rehyat_hybrid_attn_fwd_phi")
     return (y, dbg_t) if debug else y
 
 

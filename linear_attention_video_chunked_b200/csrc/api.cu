@@ -182,8 +182,10 @@ cudaError_t run_attn(const rehyat_params* p, const AttnParams& a, cudaStream_t s
 // Per-slice states and the linear-set state per chunk into the workspace
 // laid out by fwd_layout (weight images, per-slice state kernel, chunk scan);
 // arguments already checked.
+// With phi_k given ([BH][N][Dp] fp32), phi is unused (may be null).
 rehyat_status state_pass(const rehyat_params* p, const void* k, const void* v,
-                         const rehyat_phi* phi, char* ws, cudaStream_t s) {
+                         const rehyat_phi* phi, char* ws, cudaStream_t s,
+                         const float* phi_k = nullptr) {
   const FwdWorkspace w = fwd_layout(p);
   float* P = reinterpret_cast<float*>(ws + w.P_off);
   float* z = reinterpret_cast<float*>(ws + w.z_off);
@@ -195,14 +197,16 @@ rehyat_status state_pass(const rehyat_params* p, const void* k, const void* v,
   PartialParams pp = {};
   pp.k = k; pp.v = v;
   pp.rows_per_bh = static_cast<long long>(p->T) * HW;
-  pp.Wk = phi->Wk; pp.bk = phi->bk;
+  pp.Wk = phi_k ? nullptr : phi->Wk;
+  pp.bk = phi_k ? nullptr : phi->bk;
+  pp.phi_k = phi_k;
   pp.P = P; pp.z = z;
   pp.BH = BH; pp.heads = p->heads; pp.HW = HW; pp.D = p->D; pp.Dp = p->Dp; pp.To = p->To;
   pp.nslots = p->T;
   pp.in_bf16 = p->in_dtype == REHYAT_BF16;
   pp.w_bf16 = pp.in_bf16;
   cudaError_t e = cudaSuccess;
-  if (tc_path(p) || tc_state_path(p))
+  if (!phi_k && (tc_path(p) || tc_state_path(p)))
     e = launch_w_images(phi->Wq, ws + w.wimg_off, phi->Wk, ws + w.wkimg_off, p->heads, p->D,
                         p->Dp, s);
   if (e != cudaSuccess) return to_status(e);
@@ -410,6 +414,50 @@ rehyat_status rehyat_chunk_step(const rehyat_params* p, const void* q, const voi
   return to_status(launch_step_finish(P, zp, s_state, z_state, seen, done, BH, p->Dp, p->D,
                                       p->To, nslices, w.nslots, k, v, rk, rv, HW,
                                       elem_bytes(p->in_dtype), s));
+}
+
+rehyat_status rehyat_hybrid_attn_fwd_phi(const rehyat_params* p, const void* q, const void* k,
+                                         const void* v, const float* phi_q, const float* phi_k,
+                                         void* y, void* workspace, size_t ws_bytes,
+                                         const rehyat_debug* dbg, void* stream) {
+  rehyat_status st = check_params(p);
+  if (st != REHYAT_OK) return st;
+  if (!q || !k || !v || !phi_q || !phi_k || !y || !workspace) return REHYAT_ERR_INVALID_ARG;
+  if ((st = check_dbg(dbg)) != REHYAT_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(y) || !aligned16(phi_q) ||
+      !aligned16(phi_k) || !aligned16(workspace))
+    return REHYAT_ERR_MISALIGNED;
+  const FwdWorkspace w = fwd_layout(p);
+  if (ws_bytes < w.total) return REHYAT_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  if ((st = state_pass(p, k, v, nullptr, ws, s, phi_k)) != REHYAT_OK) return st;
+  AttnParams a = base_attn(p, q, k, v, nullptr, y, dbg);
+  a.phi_q = phi_q;
+  a.rows_per_bh = static_cast<long long>(p->T) * p->Hs * p->Ws;
+  a.SL = reinterpret_cast<const float*>(ws + w.SL_off);
+  a.zL = reinterpret_cast<const float*>(ws + w.zL_off);
+  a.nchunks = nchunks_of(p);
+  return to_status(run_attn(p, a, s));
+}
+
+rehyat_status rehyat_feature_map_mlp(const rehyat_params* p, const void* x,
+                                     const rehyat_phi_mlp* mlp, float* phi, void* stream) {
+  rehyat_status st = check_params(p);
+  if (st != REHYAT_OK) return st;
+  if (!x || !mlp || !phi || !mlp->Wa || !mlp->ba || !mlp->Wb || !mlp->bb)
+    return REHYAT_ERR_INVALID_ARG;
+  if (mlp->parts < 1 || p->Dp % mlp->parts != 0 || mlp->Dh < 1) return REHYAT_ERR_INVALID_ARG;
+  if (mlp->Dh > 512) return REHYAT_ERR_UNSUPPORTED;
+  const void* ptrs[6] = {x, phi, mlp->Wa, mlp->ba, mlp->Wb, mlp->bb};
+  for (const void* q : ptrs)
+    if (reinterpret_cast<uintptr_t>(q) & 3) return REHYAT_ERR_MISALIGNED;
+  PhiMlpArgs a;
+  a.x = x; a.Wa = mlp->Wa; a.ba = mlp->ba; a.Wb = mlp->Wb; a.bb = mlp->bb; a.phi = phi;
+  a.N = static_cast<long long>(p->T) * p->Hs * p->Ws;
+  a.BH = p->batch * p->heads; a.heads = p->heads; a.D = p->D; a.Dh = mlp->Dh; a.Dp = p->Dp;
+  a.parts = mlp->parts; a.in_bf16 = p->in_dtype == REHYAT_BF16;
+  return to_status(launch_phi_mlp(a, static_cast<cudaStream_t>(stream)));
 }
 
 size_t rehyat_phi_bwd_workspace_bytes(const rehyat_params* p) {

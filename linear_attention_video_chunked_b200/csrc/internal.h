@@ -29,6 +29,7 @@ struct AttnParams {
   const float *SL, *zL;      // linear-set state per chunk
   const float *Wq, *bq;      // phi_q parameters, fp32 [h][2][D][Dp/2], [h][2][Dp/2]
   const void* wq_img;        // bf16 phi_q weight image per head (tensor-core path) or nullptr
+  const float* phi_q;        // phi_q(q) given as [BH][rows][Dp] fp32 (then Wq, bq unused) or nullptr
   void* y;
   float *dbg_aS, *dbg_nS, *dbg_c, *dbg_aL, *dbg_nL;
   int BH, heads, T, HW, D, Dp, Tc, To, nchunks, nq_slices;
@@ -52,6 +53,7 @@ struct PartialParams {
   long long ring_rows_per_bh;
   const long long* seen;
   const float *Wk, *bk;
+  const float* phi_k;        // phi_k(k) given as [BH][rows][Dp] fp32 (then Wk, bk unused) or nullptr
   float *P, *z;              // [BH][nslots][Dp][D], [BH][nslots][Dp]
   int BH, heads, HW, D, Dp, To, nslots, nq_slices;
   int in_bf16, w_bf16;
@@ -73,6 +75,18 @@ struct PhiBwdArgs {
 void phi_bwd_split(int T, int Tc, int HW, int* QS, int* KS);
 size_t phi_bwd_partial_floats(int BH, int T, int nchunks, int D, int Dp, int QS, int KS);
 cudaError_t launch_phi_bwd(const PhiBwdArgs& a, cudaStream_t s);
+
+// General feature map (phi_mlp.cu): phi = [psi_1^1 .. psi_P^P],
+// psi = GELU(x W_a + b_a) W_b + b_b per head; x [BH][N][D] (in dtype),
+// phi [BH][N][Dp] fp32.
+struct PhiMlpArgs {
+  const void* x;
+  const float *Wa, *ba, *Wb, *bb;
+  float* phi;
+  long long N;
+  int BH, heads, D, Dh, Dp, parts, in_bf16;
+};
+cudaError_t launch_phi_mlp(const PhiMlpArgs& a, cudaStream_t s);
 
 // ---- SIMT (fp32 CUDA-core) kernels: every supported shape, both dtypes.
 cudaError_t launch_attn_simt(const AttnParams& p, cudaStream_t s);

@@ -184,10 +184,15 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(AttnParams P) {
     const float* SL = P.SL + (static_cast<long long>(bh) * P.nchunks + t) * Dp * D;
     const float* zL = P.zL + (static_cast<long long>(bh) * P.nchunks + t) * Dp;
     for (int f = lane4; f < Dp; f += 4) {
-      float psi = __ldg(P.bq + b_index(h, Dp, f));
-      for (int d = 0; d < D; ++d)
-        psi = fmaf(Qs[r * D + d], load_w(P.Wq, w_index(h, D, Dp, d, f), P.w_bf16), psi);
-      const float ph = psi * psi;
+      float ph;
+      if (P.phi_q) {  // phi_q(q) given
+        ph = r < nrows ? __ldg(P.phi_q + (qrow_base + r) * Dp + f) : 0.f;
+      } else {
+        float psi = __ldg(P.bq + b_index(h, Dp, f));
+        for (int d = 0; d < D; ++d)
+          psi = fmaf(Qs[r * D + d], load_w(P.Wq, w_index(h, D, Dp, d, f), P.w_bf16), psi);
+        ph = psi * psi;
+      }
       Fq[r * Dp + f] = ph;
       nL = fmaf(ph, __ldg(zL + f), nL);
     }
@@ -284,10 +289,14 @@ __global__ void __launch_bounds__(256) partials_simt_kernel(PartialParams P) {
       const int f = f0 + fq;
       float ph = 0.f;
       if (f < Dp && j0 + j < P.HW) {
-        float psi = __ldg(P.bk + b_index(h, Dp, f));
-        for (int d = 0; d < D; ++d)
-          psi = fmaf(Kt[j][d], load_w(P.Wk, w_index(h, D, Dp, d, f), P.w_bf16), psi);
-        ph = psi * psi;
+        if (P.phi_k) {  // phi_k(k) given (full forward: rows as in k)
+          ph = __ldg(P.phi_k + (base + j0 + j) * Dp + f);
+        } else {
+          float psi = __ldg(P.bk + b_index(h, Dp, f));
+          for (int d = 0; d < D; ++d)
+            psi = fmaf(Kt[j][d], load_w(P.Wk, w_index(h, D, Dp, d, f), P.w_bf16), psi);
+          ph = psi * psi;
+        }
       }
       Ft[j][fq] = ph;
     }

@@ -612,6 +612,7 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
   const int nta = (na + kBN - 1) / kBN;
   const int nt = nta + (nb + kBN - 1) / kBN;
   const bool linear = !P.full_softmax;
+  const bool phi_given = P.phi_q != nullptr;  // phi_q(q) read from P.phi_q
   const int Dp = P.Dp;  // <= 128 here: one feature piece
 
   auto tile_src = [&](int j) {
@@ -686,9 +687,11 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
         for (int tt = max(0, nt - 3); tt < nt && ok; ++tt)
           ok = mbar_wait(bar(a2::K_EMPTY + tt % 3), (tt / 3) & 1, abort_flag, 2);
         if (ok) {
-          mbar_expect_tx(bar(a2::TAIL_FULL), wbytes + slbytes);
-          bulk_load(base + kWOff, wq_img + static_cast<long long>(h) * Dp * kD, wbytes,
-                    bar(a2::TAIL_FULL));
+          // With phi_q(q) given there is no W_q image to load.
+          mbar_expect_tx(bar(a2::TAIL_FULL), (phi_given ? 0u : wbytes) + slbytes);
+          if (!phi_given)
+            bulk_load(base + kWOff, wq_img + static_cast<long long>(h) * Dp * kD, wbytes,
+                      bar(a2::TAIL_FULL));
           bulk_load(base + kSLOff, P.SL + (static_cast<long long>(bh) * P.nchunks + t) * Dp * kD,
                     slbytes, bar(a2::TAIL_FULL));
         }
@@ -749,16 +752,18 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
         ok = mbar_wait(bar(a2::TAIL_FULL), 0, abort_flag, 9);
         if (ok) {
           tc_fence_after();
-          const uint32_t id_phi = idesc(kBM, Dp, 1, false);
-          for (int tile = 0; tile < ntiles; ++tile)
+          if (!phi_given) {
+            const uint32_t id_phi = idesc(kBM, Dp, 1, false);
+            for (int tile = 0; tile < ntiles; ++tile)
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint32_t qoff = tile * 32768 + (kk >> 2) * 16384 + (kk & 3) * 32;
-              const uint32_t woff = (kk >> 2) * (Dp * 128) + (kk & 3) * 32;
-              mma_bf16(tmem + tile * 256, sdesc(base + kQOff + qoff, 16, 1024),
-                       sdesc(base + kWOff + woff, 16, 1024), id_phi, kk > 0);
-            }
-          mma_commit(bar(a2::PHI_DONE));
+              for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t qoff = tile * 32768 + (kk >> 2) * 16384 + (kk & 3) * 32;
+                const uint32_t woff = (kk >> 2) * (Dp * 128) + (kk & 3) * 32;
+                mma_bf16(tmem + tile * 256, sdesc(base + kQOff + qoff, 16, 1024),
+                         sdesc(base + kWOff + woff, 16, 1024), id_phi, kk > 0);
+              }
+            mma_commit(bar(a2::PHI_DONE));
+          }
           const uint32_t id_rd = idesc(kBM, kD, 2, false);
           for (int tile = 0; tile < ntiles && ok; ++tile) {
             ok = mbar_wait(bar(a2::PHI_READY + tile), 0, abort_flag, 10);
@@ -793,7 +798,7 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
       // Tile A's warpgroup stages b_q and z^L for the tail while it waits
       // for the first scores (b_q of head h is h's D' consecutive values).
       if (r < Dp) {
-        vec[r] = __ldg(P.bq + h * Dp + r);
+        vec[r] = phi_given ? 0.f : __ldg(P.bq + h * Dp + r);
         vec[Dp + r] = __ldg(P.zL + (static_cast<long long>(bh) * P.nchunks + t) * Dp + r);
       }
       mbar_arrive(bar(a2::VEC_READY));
@@ -966,22 +971,41 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
           }
         }
       }
-      if (ok) ok = wait_all(bar(a2::VEC_READY), 0, 14) && wait_all(bar(a2::PHI_DONE), 0, 14);
+      // phi_q(q) is staged into the V ring (tile A) and over Q (tile B):
+      // with the closed form that waits for the phi MMAs (which read Q);
+      // with phi_q given, for the last P.V (every MMA of the loop is done).
+      if (ok) ok = wait_all(bar(a2::VEC_READY), 0, 14) &&
+                   wait_all(bar(phi_given ? a2::LAST_PV : a2::PHI_DONE), 0, 14);
       if (ok) {
         tc_fence_after();
         const float inv_f = 1.0f / fscale;
         const uint32_t phi = base + (tile ? kPhiOff1 : kPhiOff0);
+        const float* given = phi_given && r < nrows ? P.phi_q + grow * Dp : nullptr;
         for (int c = 0; c < Dp / 32; ++c) {
-          uint32_t v[32];
-          REHYAT_TMEM_LD32(lane_base + s_col + c * 32, v);
-          tmem_wait_ld();
           float ph[32];
+          if (phi_given) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              const float4 g4 = given ? __ldg(reinterpret_cast<const float4*>(given + c * 32 + i))
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+              ph[i] = g4.x;
+              ph[i + 1] = g4.y;
+              ph[i + 2] = g4.z;
+              ph[i + 3] = g4.w;
+            }
+          } else {
+            uint32_t v[32];
+            REHYAT_TMEM_LD32(lane_base + s_col + c * 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float psi = __uint_as_float(v[i]) + vec[c * 32 + i];
+              ph[i] = psi * psi;
+            }
+          }
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            const int f = c * 32 + i;
-            const float psi = __uint_as_float(v[i]) + vec[f];
-            ph[i] = psi * psi;
-            nL = fmaf(ph[i], vec[Dp + f], nL);
+            nL = fmaf(ph[i], vec[Dp + c * 32 + i], nL);
             ph[i] *= inv_f;
           }
           const uint32_t rowaddr = phi + c * 16384 + r * 128;
@@ -1197,6 +1221,7 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
   // `leave` hold slices leaving the window (slot i = global slice
   // seen - min(seen, T_o) + i, in the ring if already seen, else in the chunk).
   const bool step = P.seen != nullptr;
+  const bool phi_given = P.phi_k != nullptr;  // phi_k(k) read from P.phi_k (full forward)
   const int T = step ? P.nq_slices : P.nslots;
   const long long seen0 = step ? *P.seen : 0;
   const long long rseen = seen0 < P.To ? seen0 : P.To;
@@ -1259,7 +1284,7 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
     // ================================================= TMA producers
     // warp 8 loads K tiles (and the W_k piece), warp 11 V tiles, so K runs
     // ahead on its own ring (psi^T) while V waits for phi^T V to free stages.
-    if (lane == 0) {
+    if (lane == 0 && !(warp == 8 && phi_given)) {  // no K or W_k with phi_k given
       const bool kside = warp == 8;
       bool ok = true;
       int wloads = 0, wkey = -1;
@@ -1359,7 +1384,8 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
         }
         return true;
       };
-      for (int g = 0; g < TT && ok; ++g) ok = issue_psi();
+      if (!phi_given)
+        for (int g = 0; g < TT && ok; ++g) ok = issue_psi();
     }
     __syncwarp();
   } else if (warp == 10) {
@@ -1414,12 +1440,18 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
       // b_k of head h is h's D' consecutive features.
       if (w.wkey != wkey) {
         wkey = w.wkey;
-        bias = f < pw ? P.bk[wkey * pw + f] : 0.f;
+        bias = f < pw && !phi_given ? P.bk[wkey * pw + f] : 0.f;
       }
       const uint64_t b2 = f2_pack(bias, bias);
+      // phi_k(k) given: this thread's feature column of the item's rows.
+      const float* given = phi_given && f < pw
+                               ? P.phi_k + (static_cast<long long>(w.bh()) * P.rows_per_bh +
+                                            static_cast<long long>(w.slice) * HW) * Dp +
+                                     w.half() * pw + f
+                               : nullptr;
       for (int j = 0; j < nt && ok; ++j, ++gt) {
         const int b = gt & 1;
-        ok = wait_all(bar(PSI_FULL + b), (gt >> 1) & 1, 36);
+        if (!phi_given) ok = wait_all(bar(PSI_FULL + b), (gt >> 1) & 1, 36);
         // phi^T buffer b is free once phi^T V of tile gt - 2 has read it.
         if (ok && gt >= 2) ok = wait_all(bar(PHI_FREE + b), ((gt - 2) >> 1) & 1, 38);
         if (!ok) break;
@@ -1432,13 +1464,25 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t ps[32], pk[16];
-          REHYAT_TMEM_LD32(cols + c * 32, ps);
-          tmem_wait_ld();
+          if (phi_given) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int t = c * 32 + i;
+              ps[i] = __float_as_uint(given && t < nvalid
+                                          ? __ldg(given + static_cast<long long>(j * 128 + t) * Dp)
+                                          : 0.f);
+            }
+          } else {
+            REHYAT_TMEM_LD32(cols + c * 32, ps);
+            tmem_wait_ld();
+          }
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            uint64_t a = f2_add(
-                f2_pack(__uint_as_float(ps[2 * i]), __uint_as_float(ps[2 * i + 1])), b2);
-            a = f2_fma(a, a, 0ull);
+            uint64_t a = f2_pack(__uint_as_float(ps[2 * i]), __uint_as_float(ps[2 * i + 1]));
+            if (!phi_given) {  // phi = (psi + b)^2
+              a = f2_add(a, b2);
+              a = f2_fma(a, a, 0ull);
+            }
             float v0, v1;
             f2_unpack(a, v0, v1);
             if (nvalid < 128) {  // tokens past the slice contribute nothing
@@ -1467,7 +1511,7 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
           fence_proxy_async();
         }
         tc_fence_before();
-        mbar_arrive(bar(PSI_FREE + b));
+        if (!phi_given) mbar_arrive(bar(PSI_FREE + b));
         mbar_arrive(bar(PHI_FULL + b));
         if (++vst == kS) {
           vst = 0;
@@ -1636,8 +1680,15 @@ bool tc_attn_eligible(int in_bf16, int D, int Dp) {
 
 bool tc_attn_supported(const AttnParams& p) {
   if (!p.in_bf16 || p.D != kD) return false;
-  if (!p.full_softmax && (!tc_attn_eligible(p.in_bf16, p.D, p.Dp) || p.wq_img == nullptr))
-    return false;
+  if (!p.full_softmax) {
+    if (!tc_attn_eligible(p.in_bf16, p.D, p.Dp)) return false;
+    // phi_q given: the two-query-tile kernel (D' <= 128) reads it in its tail.
+    if (p.phi_q != nullptr) {
+      if (p.Dp > 128 || p.one_tile) return false;
+    } else if (p.wq_img == nullptr) {
+      return false;
+    }
+  }
   return encode_fn() != nullptr;
 }
 

@@ -1,0 +1,134 @@
+"""GPU parity of the general feature map (rehyat_feature_map_mlp) and of the
+forward with given feature maps (rehyat_hybrid_attn_fwd_phi), through the C
+ABI, against the fp64 oracle (oracle/rehyat_phi_mlp.py) on the same seeded
+inputs.  Bars as for the forward: fp32 inputs max abs <= 1e-5 on y; bf16
+inputs max abs <= 2e-2, mean abs <= 2e-3; the feature map itself (fp32 CUDA
+cores vs fp64) within 1e-5 relative to its largest value.
+"""
+import numpy as np
+import pytest
+import torch
+
+import linear_attention_video_chunked_b200 as rh
+from oracle import rehyat_oracle as orc
+from oracle.rehyat_phi_mlp import feature_map_mlp, hybrid_phi_given
+from rehyat_inputs import make_problem
+from tests.gpu_util import assert_close_partials, assert_close_y, device_tensors
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    rh.lib()
+    rh.rehyat_device_error_flags(reset=True)
+    yield
+    assert rh.rehyat_device_error_flags() == 0
+
+
+def _mlp_params(H, D, Dh, Dp, seed, scale=1.0):
+    rng = np.random.default_rng(seed)
+    Wa = rng.standard_normal((H, D, Dh)) / np.sqrt(D)
+    ba = rng.standard_normal((H, Dh)) * 0.1
+    Wb = rng.standard_normal((H, Dh, Dp)) / np.sqrt(Dh) * scale
+    bb = rng.standard_normal((H, Dp)) * 0.1 * scale
+    return [a.astype(np.float32) for a in (Wa, ba, Wb, bb)]
+
+
+def _oracle_phi(x, params, parts):
+    B, H = x.shape[:2]
+    Wa, ba, Wb, bb = params
+    return np.stack([np.stack([feature_map_mlp(x[b, h], Wa[h], ba[h], Wb[h], bb[h], parts)
+                               for h in range(H)]) for b in range(B)])
+
+
+def _cuda32(a):
+    return torch.tensor(np.asarray(a, np.float32), device="cuda").contiguous()
+
+
+@pytest.mark.parametrize("parts,dtype", [(1, "f32"), (2, "f32"), (4, "bf16")])
+def test_feature_map_mlp_matches_oracle(parts, dtype):
+    p = make_problem(batch=2, heads=3, T=3, Hs=5, Ws=7, D=64, Dp=128, Tc=1, To=0, causal=False,
+                     dtype=dtype, seed=70 + parts)
+    params = _mlp_params(3, 64, 96, 128, 71 + parts)
+    dev = device_tensors(p)
+    got = rh.feature_map_mlp(dev["q"], *(_cuda32(a) for a in params), parts=parts, T=p.T,
+                             Hs=p.Hs, Ws=p.Ws)
+    torch.cuda.synchronize()
+    ref = _oracle_phi(np.asarray(p.q, np.float64), params, parts)
+    err = np.abs(got.double().cpu().numpy() - ref).max()
+    assert err <= 1e-5 * np.abs(ref).max(), err
+
+
+def _closed_form_phi(p):
+    fq = np.stack([np.stack([orc.feature_map(p.q[b, h], p.Wq[h], p.bq[h])
+                             for h in range(p.heads)]) for b in range(p.batch)])
+    fk = np.stack([np.stack([orc.feature_map(p.k[b, h], p.Wk[h], p.bk[h])
+                             for h in range(p.heads)]) for b in range(p.batch)])
+    return fq.astype(np.float32), fk.astype(np.float32)
+
+
+def _run_phi(p, fq, fk, force_simt):
+    dev = device_tensors(p)
+    y, parts = rh.hybrid_attn_phi(dev["q"], dev["k"], dev["v"], _cuda32(fq), _cuda32(fk), T=p.T,
+                                  Hs=p.Hs, Ws=p.Ws, Tc=p.Tc, To=p.To, causal=p.causal,
+                                  debug=True, force_simt=force_simt)
+    torch.cuda.synchronize()
+    return y.double().cpu().numpy(), {k: v.double().cpu().numpy() for k, v in parts.items()}
+
+
+SHAPES = [
+    # B, h, T, Hs, Ws, D, Dp, Tc, To, causal
+    (1, 2, 5, 7, 9, 128, 128, 2, 1, False),    # ragged tiles
+    (1, 2, 7, 10, 13, 128, 64, 3, 2, True),
+    (1, 2, 5, 9, 15, 128, 256, 2, 1, False),   # D' = 256: state halves, CUDA-core attention
+]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_phi_given_closed_form(shape, dtype):
+    """Closed-form phi passed as arrays: equals the oracle's phi-given forward
+    (itself pinned to the closed-form forward)."""
+    B, h, T, Hs, Ws, D, Dp, Tc, To, causal = shape
+    p = make_problem(batch=B, heads=h, T=T, Hs=Hs, Ws=Ws, D=D, Dp=Dp, Tc=Tc, To=To,
+                     causal=causal, dtype=dtype, dist="scaled", seed=400 + sum(shape[:9]))
+    fq, fk = _closed_form_phi(p)
+    ref_y, ref_p = hybrid_phi_given(p.q, p.k, p.v, fq, fk, T=p.T, HW=p.HW, Tc=p.Tc, To=p.To,
+                                    causal=p.causal)
+    y, parts = _run_phi(p, fq, fk, force_simt=dtype == "f32")
+    assert_close_y(y, ref_y, dtype)
+    assert_close_partials(parts, ref_p, dtype)
+
+
+@pytest.mark.parametrize("dtype,parts_n", [("bf16", 2), ("f32", 2), ("bf16", 4)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_mlp_phi_end_to_end(dtype, parts_n, causal):
+    """General phi (a degree-1 part, so negative values) from the library's
+    MLP kernel through the phi-given forward, against the oracle."""
+    p = make_problem(batch=1, heads=2, T=6, Hs=8, Ws=12, D=128, Dp=128, Tc=2, To=1,
+                     causal=causal, dtype=dtype, dist="scaled", seed=500 + parts_n)
+    params = _mlp_params(2, 128, 384, 128, 501, scale=0.5)
+    dev = device_tensors(p)
+    kw = dict(T=p.T, Hs=p.Hs, Ws=p.Ws)
+    pq = rh.feature_map_mlp(dev["q"], *(_cuda32(a) for a in params), parts=parts_n, **kw)
+    pk = rh.feature_map_mlp(dev["k"], *(_cuda32(a) for a in params), parts=parts_n, **kw)
+    y, parts = rh.hybrid_attn_phi(dev["q"], dev["k"], dev["v"], pq, pk, Tc=p.Tc, To=p.To,
+                                  causal=p.causal, debug=True, force_simt=dtype == "f32", **kw)
+    torch.cuda.synchronize()
+    fq = _oracle_phi(np.asarray(p.q, np.float64), params, parts_n)
+    fk = _oracle_phi(np.asarray(p.k, np.float64), params, parts_n)
+    assert fq.min() < 0 and fk.min() < 0  # the degree-1 part is signed
+    ref_y, ref_p = hybrid_phi_given(p.q, p.k, p.v, fq, fk, T=p.T, HW=p.HW, Tc=p.Tc, To=p.To,
+                                    causal=p.causal)
+    assert_close_y(y.double().cpu().numpy(), ref_y, dtype)
+    # The linear partials are signed here: compare them against their scale.
+    got = {k: v.double().cpu().numpy() for k, v in parts.items()}
+    assert_close_y(got["aS"] / got["nS"][..., None], ref_p["aS"] / ref_p["nS"][..., None], dtype,
+                   "aS/nS")
+    rel = 1e-5 if dtype == "f32" else 2e-2
+    for key in ("nL", "aL"):
+        err = np.abs(got[key] - ref_p[key]).max()
+        assert err <= rel * np.abs(ref_p[key]).max(), (key, err)
