@@ -291,6 +291,60 @@ def measure_phi_backward(rh, p, q, k, v, Wq, bq, Wk, bk, flush, stream, calls=3)
                     "q/k/v, fp32 y, dy, den; includes its state pass"}
 
 
+def measure_general_phi(rh, p, q, k, v, flush, stream, calls=3):
+    """General feature maps on the bench workload: the per-head 2-layer MLP
+    (hidden width 3D, P = 2 parts) for q and for k, then the forward with the
+    maps given (rehyat_hybrid_attn_fwd_phi).  Device time per call of each."""
+    import torch
+    B, H, N, D = q.shape
+    dev = q.device
+    Dp, Dh = p.Dp, 3 * D
+    g = torch.Generator(device=dev).manual_seed(6)
+    Wa = torch.randn(H, D, Dh, generator=g, device=dev) / D ** 0.5
+    ba = 0.1 * torch.randn(H, Dh, generator=g, device=dev)
+    Wb = 0.5 * torch.randn(H, Dh, Dp, generator=g, device=dev) / Dh ** 0.5
+    bb = 0.05 * torch.randn(H, Dp, generator=g, device=dev)
+    params = rh.make_params(batch=B, heads=H, T=p.T, Hs=p.Hs, Ws=p.Ws, D=D, Dp=Dp, Tc=p.Tc,
+                            To=p.To, causal=p.causal, in_dtype=rh.BF16, out_dtype=rh.F32)
+    sh = stream.cuda_stream
+    mlp = rh.RehyatPhiMlp(Wa.data_ptr(), ba.data_ptr(), Wb.data_ptr(), bb.data_ptr(), Dh, 2)
+    pq = torch.empty(B, H, N, Dp, device=dev)
+    pk = torch.empty(B, H, N, Dp, device=dev)
+    y = torch.empty(B, H, N, D, device=dev)
+    ws = torch.empty(rh.rehyat_workspace_bytes(params), dtype=torch.uint8, device=dev)
+    feat = lambda: (rh.rehyat_feature_map_mlp(params, q.data_ptr(), mlp, pq.data_ptr(), sh) or
+                    rh.rehyat_feature_map_mlp(params, k.data_ptr(), mlp, pk.data_ptr(), sh))
+    fwd = lambda: rh.rehyat_hybrid_attn_fwd_phi(params, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                                pq.data_ptr(), pk.data_ptr(), y.data_ptr(),
+                                                ws.data_ptr(), ws.numel(), None, sh)
+    if feat() or fwd():
+        raise RuntimeError("general feature map path failed")
+
+    def timed(fn):
+        times = []
+        for _ in range(calls):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1))
+        return sum(times) / len(times)
+
+    feat_ms, fwd_ms = timed(feat), timed(fwd)
+    feat_flops = 2 * B * H * N * (2.0 * D * Dh + 2.0 * Dh * Dp)  # q and k
+    del pq, pk, y, ws
+    return {"feature_maps_ms": feat_ms,
+            "feature_maps_tflops": feat_flops / (feat_ms / 1e3) / 1e12,
+            "feature_maps_alu_frac": feat_flops / (feat_ms / 1e3) / 1e12 / FP32_ALU_TFLOPS,
+            "forward_phi_given_ms": fwd_ms,
+            "forward_phi_given_tokens_per_s": B * N / (fwd_ms / 1e3),
+            "what": "rehyat_feature_map_mlp for q and k (hidden 3D = 384, P = 2, fp32 CUDA "
+                    "cores), then rehyat_hybrid_attn_fwd_phi (tensor-core path) on the bench "
+                    "workload"}
+
+
 def measure_streaming(rh, dev, flush, stream):
     """Chunk-wise RNN over 81 slices of 30x52 (27 steps of T_c = 3, T_o = 1,
     12 heads, D = D' = 128): per-step device time, steady-state tokens/s,
@@ -638,6 +692,8 @@ def run_gpu(args, world, rank, local):
         torch.cuda.empty_cache()
         extra["phi_backward"] = measure_phi_backward(rh, p, q, k, v, Wq, bq, Wk, bk, flush,
                                                      stream)
+        torch.cuda.empty_cache()
+        extra["general_phi"] = measure_general_phi(rh, p, q, k, v, flush, stream)
         del q, k, v
         torch.cuda.empty_cache()
         extra["streaming"] = measure_streaming(rh, dev, flush, stream)

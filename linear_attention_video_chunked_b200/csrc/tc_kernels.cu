@@ -1186,6 +1186,10 @@ struct ItemWalk {
 };
 }  // namespace sp
 
+// kPhiGiven: phi_k(k) is read from P.phi_k (full forward) instead of being
+// computed from K and W_k (a separate instantiation, so the default path
+// carries no branch for it).
+template <bool kPhiGiven>
 __global__ void __launch_bounds__(sp::kThreads, 1)
     tc_state_persistent_kernel(const __grid_constant__ StMaps maps, const PartialParams P,
                                const __nv_bfloat16* __restrict__ wk_img, int items_per_cta) {
@@ -1221,7 +1225,7 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
   // `leave` hold slices leaving the window (slot i = global slice
   // seen - min(seen, T_o) + i, in the ring if already seen, else in the chunk).
   const bool step = P.seen != nullptr;
-  const bool phi_given = P.phi_k != nullptr;  // phi_k(k) read from P.phi_k (full forward)
+  constexpr bool phi_given = kPhiGiven;
   const int T = step ? P.nq_slices : P.nslots;
   const long long seen0 = step ? *P.seen : 0;
   const long long rseen = seen0 < P.To ? seen0 : P.To;
@@ -1650,11 +1654,19 @@ cudaError_t launch_state_tc(const PartialParams& p, const void* wk_img, cudaStre
   const int total = p.BH * per_bh;
   const int per_cta = (total + sms - 1) / sms;
   const int ctas = (total + per_cta - 1) / per_cta;
-  const cudaError_t e = ensure_smem(tc_state_persistent_kernel, 0, sp::kSmemBytes);
-  if (e != cudaSuccess) return e;
   const __nv_bfloat16* wk = static_cast<const __nv_bfloat16*>(wk_img);
+  if (p.phi_k != nullptr) {  // full forward with phi_k(k) given
+    const cudaError_t e = ensure_smem(tc_state_persistent_kernel<true>, 3, sp::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    tc_state_persistent_kernel<true><<<ctas, sp::kThreads, sp::kSmemBytes, s>>>(maps, p, wk,
+                                                                                per_cta);
+    return cudaGetLastError();
+  }
+  const cudaError_t e = ensure_smem(tc_state_persistent_kernel<false>, 0, sp::kSmemBytes);
+  if (e != cudaSuccess) return e;
   if (p.seen == nullptr) {
-    tc_state_persistent_kernel<<<ctas, sp::kThreads, sp::kSmemBytes, s>>>(maps, p, wk, per_cta);
+    tc_state_persistent_kernel<false><<<ctas, sp::kThreads, sp::kSmemBytes, s>>>(maps, p, wk,
+                                                                                 per_cta);
     return cudaGetLastError();
   }
   // Streaming fold: it reads only k, v, the ring and W_k and writes only the
@@ -1671,7 +1683,7 @@ cudaError_t launch_state_tc(const PartialParams& p, const void* wk_img, cudaStre
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, tc_state_persistent_kernel, maps, p, wk, per_cta);
+  return cudaLaunchKernelEx(&cfg, tc_state_persistent_kernel<false>, maps, p, wk, per_cta);
 }
 
 bool tc_attn_eligible(int in_bf16, int D, int Dp) {
