@@ -9,8 +9,9 @@ drawn by rehyat_inputs (seed 2), fp32 output.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
 Prints ONE JSON line (rank 0).  Device time is measured with CUDA events on
-the stream the kernels run on, with a 256 MB L2 flush before every timed step
-(outside the events), max over ranks.  ``--impl reference`` times the fp64
+the stream the kernels run on, with an L2 flush before every timed step
+(outside the events: a 256 MB write, then a 256 MB read of a second buffer,
+so that no input and no dirty line is left in L2), max over ranks.  ``--impl reference`` times the fp64
 CPU oracle on a bounded sample instead (rank 0 only).
 
 Multi-GPU: every rank runs the same workload on its own GPU (replicas; the
@@ -36,6 +37,24 @@ WORKLOAD = "wan_480x832_bidir"
 METRIC = "hybrid-attn fwd tokens/s & TFLOP/s (% BF16 tensor peak), 1 B200, 21x30x52 latent"
 L2_FLUSH_BYTES = 256 << 20
 KERNELS_PER_STEP = 4  # weight images, per-slice state, chunk scan, attention
+
+
+class L2Flush:
+    """Empties L2 (126 MB on B200) between timed steps: a 256 MB write evicts
+    every input, and a 256 MB read of a second buffer then evicts the write's
+    dirty lines, so the timed kernels neither find their inputs in L2 nor pay
+    for writing back data that is not theirs."""
+
+    def __init__(self, torch, dev):
+        n = L2_FLUSH_BYTES // 4
+        self.wbuf = torch.empty(n, dtype=torch.float32, device=dev)
+        self.rbuf = torch.zeros(n, dtype=torch.float32, device=dev)
+        self.sink = torch.empty((), dtype=torch.float32, device=dev)
+        self.torch = torch
+
+    def __call__(self):
+        self.wbuf.zero_()
+        self.torch.sum(self.rbuf, dim=0, out=self.sink)
 
 
 # --------------------------------------------------------------- workload
@@ -224,7 +243,7 @@ def measure_full_softmax(rh, q, k, v, y, flush, stream, calls=3):
         raise RuntimeError("rehyat_softmax_attn_fwd failed")
     times = []
     for _ in range(calls):
-        flush.zero_()
+        flush()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         call()
@@ -270,7 +289,7 @@ def measure_phi_backward(rh, p, q, k, v, Wq, bq, Wk, bk, flush, stream, calls=3)
         raise RuntimeError("rehyat_phi_bwd failed")
     times = []
     for _ in range(calls):
-        flush.zero_()
+        flush()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         call()
@@ -323,7 +342,7 @@ def measure_general_phi(rh, p, q, k, v, flush, stream, calls=3):
     def timed(fn):
         times = []
         for _ in range(calls):
-            flush.zero_()
+            flush()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             fn()
@@ -458,7 +477,7 @@ def run_sweep(args):
     q, k = lowrank(), lowrank()
     v = torch.randn(B, H, N, D, generator=g, device=dev).to(torch.bfloat16)
     y = torch.empty(B, H, N, D, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush = L2Flush(torch, dev)
     peaks = load_peaks()
     stream = torch.cuda.current_stream()
     for Dp in (64, 128, 256):
@@ -492,7 +511,7 @@ def run_sweep(args):
                         call()
                     times = []
                     for _ in range(max(3, args.steps // 6)):
-                        flush.zero_()
+                        flush()
                         evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
                         call(evs)
                         torch.cuda.synchronize()
@@ -605,7 +624,7 @@ def run_gpu(args, world, rank, local):
     ws_bytes = rh.rehyat_workspace_bytes(params)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     phi = rh.RehyatPhi(Wq.data_ptr(), bq.data_ptr(), Wk.data_ptr(), bk.data_ptr())
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush = L2Flush(torch, dev)
     stream = torch.cuda.current_stream()
     sh = stream.cuda_stream
 
@@ -626,7 +645,7 @@ def run_gpu(args, world, rank, local):
             evs[2].record(stream)
 
     for _ in range(args.warmup):
-        flush.zero_()
+        flush()
         step()
     torch.cuda.synchronize()
 
@@ -638,7 +657,7 @@ def run_gpu(args, world, rank, local):
     torch.cuda.synchronize()
     t_host0 = time.time()
     for i in range(args.steps):
-        flush.zero_()
+        flush()
         step(events[i])
     torch.cuda.synchronize()
     t_host1 = time.time()
@@ -726,7 +745,7 @@ def run_gpu(args, world, rank, local):
         "data": "synthetic",
         "config": {"workload": workload_desc(p), "global_batch": B * world, "seq_len": N,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "256 MB write before every timed step (outside the events)"},
+                   "l2": "flushed before every timed step, outside the events: 256 MB write, then 256 MB read of a second buffer"},
         "tflops": w["total_flops"] / (ms_per_step / 1e3) / 1e12 * world,
         "pct_bf16_peak": w["total_flops"] / (ms_per_step / 1e3) / 1e12 / peaks["bf16_tflops"],
         "stages_ms": {"state (per-slice + scan)": sum(state_ms) / len(state_ms),

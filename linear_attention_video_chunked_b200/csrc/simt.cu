@@ -326,6 +326,9 @@ __global__ void __launch_bounds__(256) partials_simt_kernel(PartialParams P) {
 __global__ void scan_kernel(const float* __restrict__ P, const float* __restrict__ z,
                             float* __restrict__ SL, float* __restrict__ zL, int T, int Tc,
                             int To, int nchunks, int Dp, int D, int causal) {
+  // Launched as a programmatic dependent of the per-slice state kernel: wait
+  // for that grid (and its writes) before reading P, z.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const long long PD = static_cast<long long>(Dp) * D;
   const long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int bh = blockIdx.y;
@@ -462,6 +465,9 @@ __global__ void step_finish_kernel(const float* __restrict__ P, const float* __r
 __global__ void w_image_kernel(const float* __restrict__ Wq, __nv_bfloat16* __restrict__ out_q,
                                const float* __restrict__ Wk, __nv_bfloat16* __restrict__ out_k,
                                int heads, int D, int Dp) {
+  // The per-slice state kernel that follows may start now; it waits for
+  // this grid before its first read of the W_k image.
+  asm volatile("griddepcontrol.launch_dependents;");
   const float* Wsrc = blockIdx.y == 0 ? Wq : Wk;
   __nv_bfloat16* out = blockIdx.y == 0 ? out_q : out_k;
   const long long per_head = static_cast<long long>(Dp) * D;
@@ -521,9 +527,18 @@ cudaError_t launch_scan(const float* P, const float* z, float* SL, float* zL, in
                         int Tc, int To, int nchunks, int Dp, int D, int causal,
                         cudaStream_t s) {
   const long long n = static_cast<long long>(Dp) * D + Dp;
-  dim3 grid(static_cast<unsigned>((n + 255) / 256), BH);
-  scan_kernel<<<grid, 256, 0, s>>>(P, z, SL, zL, T, Tc, To, nchunks, Dp, D, causal);
-  return cudaGetLastError();
+  // Programmatic dependent launch: the grid is scheduled while the state
+  // kernel before it still runs, and waits for it on the device.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>((n + 255) / 256), BH);
+  cfg.blockDim = dim3(256);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, scan_kernel, P, z, SL, zL, T, Tc, To, nchunks, Dp, D, causal);
 }
 
 cudaError_t launch_step_finish(const float* P, const float* zp, float* s_state, float* z_state,

@@ -1241,6 +1241,7 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
   // streaming step, this grid overlaps it; waiting here before exit makes
   // this grid's completion imply the attention kernel's (no-op otherwise).
   auto dependency_wait = [] { asm volatile("griddepcontrol.wait;" ::: "memory"); };
+  asm volatile("griddepcontrol.launch_dependents;");  // the chunk scan waits on the device
   if (it0 >= it1) {
     dependency_wait();
     return;
@@ -1304,6 +1305,9 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
           wkey = w.wkey;
           if (wloads > 0) ok = mbar_wait(bar(W_FREE), (wloads - 1) & 1, abort_flag, 27);
           if (!ok) break;
+          // Full forward: the W_k image comes from the grid launched just
+          // before this one (programmatic dependent launch).
+          if (!step && wloads == 0) dependency_wait();
           // Head h's image holds its D' features as pieces of pw rows, each
           // piece two boxes of pw rows x 64 columns.
           const __nv_bfloat16* src = wk_img + static_cast<long long>(w.wkey) * pw * 128;
@@ -1664,15 +1668,12 @@ cudaError_t launch_state_tc(const PartialParams& p, const void* wk_img, cudaStre
   }
   const cudaError_t e = ensure_smem(tc_state_persistent_kernel<false>, 0, sp::kSmemBytes);
   if (e != cudaSuccess) return e;
-  if (p.seen == nullptr) {
-    tc_state_persistent_kernel<false><<<ctas, sp::kThreads, sp::kSmemBytes, s>>>(maps, p, wk,
-                                                                                 per_cta);
-    return cudaGetLastError();
-  }
-  // Streaming fold: it reads only k, v, the ring and W_k and writes only the
-  // per-slot states, so it may start while the attention kernel launched
-  // just before it is still running (programmatic dependent launch); the
-  // kernel waits for that grid before it exits.
+  // Programmatic dependent launch in both modes.  Full forward: the grid
+  // before this one writes the W_k image; the K/V loads start at once and
+  // the W_k load waits for that grid on the device.  Streaming fold: it reads
+  // only k, v, the ring and W_k and writes only the per-slot states, so it
+  // may run beside the attention kernel launched just before it.  Either way
+  // the kernel waits for the earlier grid before it exits.
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(ctas);
   cfg.blockDim = dim3(sp::kThreads);
