@@ -37,6 +37,7 @@ WORKLOAD = "wan_480x832_bidir"
 METRIC = "hybrid-attn fwd tokens/s & TFLOP/s (% BF16 tensor peak), 1 B200, 21x30x52 latent"
 L2_FLUSH_BYTES = 256 << 20
 KERNELS_PER_STEP = 4  # weight images, per-slice state, chunk scan, attention
+EXTRAS = ("full_softmax", "phi_backward", "general_phi", "streaming")
 
 
 class L2Flush:
@@ -331,8 +332,13 @@ def measure_general_phi(rh, p, q, k, v, flush, stream, calls=3):
     pk = torch.empty(B, H, N, Dp, device=dev)
     y = torch.empty(B, H, N, D, device=dev)
     ws = torch.empty(rh.rehyat_workspace_bytes(params), dtype=torch.uint8, device=dev)
-    feat = lambda: (rh.rehyat_feature_map_mlp(params, q.data_ptr(), mlp, pq.data_ptr(), sh) or
-                    rh.rehyat_feature_map_mlp(params, k.data_ptr(), mlp, pk.data_ptr(), sh))
+    mlp_bytes = rh.rehyat_feature_map_mlp_workspace_bytes(params, mlp, q.data_ptr(), pq.data_ptr())
+    mws = torch.empty(max(mlp_bytes, 16), dtype=torch.uint8, device=dev)
+    tensor_cores = mlp_bytes > 0
+    feat = lambda: (rh.rehyat_feature_map_mlp(params, q.data_ptr(), mlp, pq.data_ptr(),
+                                              mws.data_ptr(), mlp_bytes, sh) or
+                    rh.rehyat_feature_map_mlp(params, k.data_ptr(), mlp, pk.data_ptr(),
+                                              mws.data_ptr(), mlp_bytes, sh))
     fwd = lambda: rh.rehyat_hybrid_attn_fwd_phi(params, q.data_ptr(), k.data_ptr(), v.data_ptr(),
                                                 pq.data_ptr(), pk.data_ptr(), y.data_ptr(),
                                                 ws.data_ptr(), ws.numel(), None, sh)
@@ -353,15 +359,29 @@ def measure_general_phi(rh, p, q, k, v, flush, stream, calls=3):
 
     feat_ms, fwd_ms = timed(feat), timed(fwd)
     feat_flops = 2 * B * H * N * (2.0 * D * Dh + 2.0 * Dh * Dp)  # q and k
-    del pq, pk, y, ws
-    return {"feature_maps_ms": feat_ms,
-            "feature_maps_tflops": feat_flops / (feat_ms / 1e3) / 1e12,
-            "feature_maps_alu_frac": feat_flops / (feat_ms / 1e3) / 1e12 / FP32_ALU_TFLOPS,
-            "forward_phi_given_ms": fwd_ms,
-            "forward_phi_given_tokens_per_s": B * N / (fwd_ms / 1e3),
-            "what": "rehyat_feature_map_mlp for q and k (hidden 3D = 384, P = 2, fp32 CUDA "
-                    "cores), then rehyat_hybrid_attn_fwd_phi (tensor-core path) on the bench "
-                    "workload"}
+    # Algorithmic bytes: x in (bf16) and phi out (fp32) for q and k; the
+    # weights (2.4 MB of images) are negligible.
+    feat_bytes = 2 * B * H * N * (D * 2 + Dp * 4)
+    peaks = load_peaks()
+    tflops = feat_flops / (feat_ms / 1e3) / 1e12
+    gbs = feat_bytes / (feat_ms / 1e3) / 1e9
+    del pq, pk, y, ws, mws
+    out = {"feature_maps_ms": feat_ms,
+           "feature_maps_path": "tensor cores (bf16 operands)" if tensor_cores
+           else "fp32 CUDA cores",
+           "feature_maps_tflops": tflops,
+           "feature_maps_gbs": gbs,
+           "forward_phi_given_ms": fwd_ms,
+           "forward_phi_given_tokens_per_s": B * N / (fwd_ms / 1e3),
+           "what": "rehyat_feature_map_mlp for q and k (hidden 3D = 384, P = 2), then "
+                   "rehyat_hybrid_attn_fwd_phi (tensor-core path) on the bench workload"}
+    if tensor_cores:
+        # Both bounds are near: 3.09e11 FLOP and 1.21 GB per pair of maps.
+        out["feature_maps_frac_bf16_peak"] = tflops / peaks["bf16_tflops"]
+        out["feature_maps_frac_hbm"] = gbs / peaks["hbm_gbs"]
+    else:
+        out["feature_maps_alu_frac"] = tflops / FP32_ALU_TFLOPS
+    return out
 
 
 def measure_streaming(rh, dev, flush, stream):
@@ -705,16 +725,22 @@ def run_gpu(args, world, rank, local):
     del qh, kh, vh, yh, qd, kd, vd
 
     extra = {}
-    if not args.no_extras:
+    want = set(EXTRAS if args.extras is None else args.extras.split(","))
+    if args.no_extras:
+        want = set()
+    if "full_softmax" in want:
         extra["full_softmax"] = measure_full_softmax(rh, q, k, v, y, flush, stream)
-        del y, ws
-        torch.cuda.empty_cache()
+    del y, ws
+    torch.cuda.empty_cache()
+    if "phi_backward" in want:
         extra["phi_backward"] = measure_phi_backward(rh, p, q, k, v, Wq, bq, Wk, bk, flush,
                                                      stream)
         torch.cuda.empty_cache()
+    if "general_phi" in want:
         extra["general_phi"] = measure_general_phi(rh, p, q, k, v, flush, stream)
-        del q, k, v
-        torch.cuda.empty_cache()
+    del q, k, v
+    torch.cuda.empty_cache()
+    if "streaming" in want:
         extra["streaming"] = measure_streaming(rh, dev, flush, stream)
 
     if rank != 0:
@@ -790,7 +816,10 @@ def main(argv=None):
     ap.add_argument("--sweep", action="store_true",
                     help="T_c/T_o/D'/form sweep on the 21x30x52 latent, one JSON line per point")
     ap.add_argument("--no-extras", action="store_true",
-                    help="skip the full-softmax comparator and the streaming measurement")
+                    help="skip the measurements beside the step (comparator, backward, "
+                         "general feature maps, streaming)")
+    ap.add_argument("--extras", default=None,
+                    help="comma-separated subset of " + ",".join(EXTRAS))
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     world, rank, local = dist_setup()

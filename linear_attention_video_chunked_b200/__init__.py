@@ -31,6 +31,7 @@ __all__ = [
     "rehyat_status_string", "rehyat_version", "rehyat_hybrid_attn_fwd_noalloc",
     "RehyatPhiGrad", "rehyat_phi_bwd_workspace_bytes", "rehyat_phi_bwd",
     "RehyatPhiMlp", "rehyat_hybrid_attn_fwd_phi", "rehyat_feature_map_mlp",
+    "rehyat_feature_map_mlp_workspace_bytes",
     "make_params", "hybrid_attn", "hybrid_attn_phi", "feature_map_mlp", "softmax_attn",
     "phi_grad", "StreamingState",
 ]
@@ -50,6 +51,7 @@ EXPORTED_SYMBOLS = (
     "rehyat_attn_path", "rehyat_status_string", "rehyat_version",
     "rehyat_hybrid_attn_fwd_noalloc", "rehyat_phi_bwd_workspace_bytes", "rehyat_phi_bwd",
     "rehyat_hybrid_attn_fwd_phi", "rehyat_feature_map_mlp",
+    "rehyat_feature_map_mlp_workspace_bytes",
 )
 
 
@@ -150,8 +152,12 @@ def lib() -> ctypes.CDLL:
         L.rehyat_hybrid_attn_fwd_phi.argtypes = [P(RehyatParams), vp, vp, vp, vp, vp, vp, vp, sz,
                                                  vp, vp]
         L.rehyat_hybrid_attn_fwd_phi.restype = i
-        L.rehyat_feature_map_mlp.argtypes = [P(RehyatParams), vp, P(RehyatPhiMlp), vp, vp]
+        L.rehyat_feature_map_mlp.argtypes = [P(RehyatParams), vp, P(RehyatPhiMlp), vp, vp,
+                                             ctypes.c_size_t, vp]
         L.rehyat_feature_map_mlp.restype = i
+        L.rehyat_feature_map_mlp_workspace_bytes.argtypes = [P(RehyatParams), P(RehyatPhiMlp),
+                                                             vp, vp]
+        L.rehyat_feature_map_mlp_workspace_bytes.restype = ctypes.c_size_t
         _LIB = L
     return _LIB
 
@@ -201,8 +207,14 @@ def rehyat_hybrid_attn_fwd_phi(p, q, k, v, phi_q, phi_k, y, workspace, ws_bytes,
                                             stream)
 
 
-def rehyat_feature_map_mlp(p, x, mlp, phi, stream) -> int:
-    return lib().rehyat_feature_map_mlp(ctypes.byref(p), x, ctypes.byref(mlp), phi, stream)
+def rehyat_feature_map_mlp_workspace_bytes(p, mlp, x, phi) -> int:
+    return lib().rehyat_feature_map_mlp_workspace_bytes(ctypes.byref(p), ctypes.byref(mlp), x,
+                                                        phi)
+
+
+def rehyat_feature_map_mlp(p, x, mlp, phi, workspace, ws_bytes, stream) -> int:
+    return lib().rehyat_feature_map_mlp(ctypes.byref(p), x, ctypes.byref(mlp), phi, workspace,
+                                        ws_bytes, stream)
 
 
 def rehyat_softmax_attn_fwd(p, q, k, v, y, stream) -> int:
@@ -330,10 +342,12 @@ def hybrid_attn(q, k, v, Wq, bq, Wk, bk, *, T, Hs, Ws, Tc, To, causal, out_dtype
     return (y, dbg_t) if debug else y
 
 
-def feature_map_mlp(x, Wa, ba, Wb, bb, *, parts, T, Hs, Ws, stream=None):
+def feature_map_mlp(x, Wa, ba, Wb, bb, *, parts, T, Hs, Ws, stream=None, force_simt=False,
+                    workspace=None, out=None):
     """phi = [psi_1^1, ..., psi_P^P], psi = GELU(x Wa + ba) Wb + bb per head,
     of a torch CUDA tensor x [B, h, N, D]; Wa [h, D, Dh], ba [h, Dh],
-    Wb [h, Dh, D'], bb [h, D'] fp32.  Returns fp32 [B, h, N, D']."""
+    Wb [h, Dh, D'], bb [h, D'] fp32.  Returns fp32 [B, h, N, D'].  bf16 x with
+    D = 128 runs on the tensor cores (bf16 operands) unless force_simt."""
     torch = _torch()
     B, H, N, D = x.shape
     Dh, Dp = Wa.shape[-1], Wb.shape[-1]
@@ -341,11 +355,17 @@ def feature_map_mlp(x, Wa, ba, Wb, bb, *, parts, T, Hs, Ws, stream=None):
         if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous():
             raise TypeError("MLP parameters must be contiguous fp32 CUDA tensors")
     p = make_params(batch=B, heads=H, T=T, Hs=Hs, Ws=Ws, D=D, Dp=Dp, Tc=1, To=0, causal=0,
-                    in_dtype=_dtype_code(x.dtype), out_dtype=F32)
-    phi = torch.empty(B, H, N, Dp, dtype=torch.float32, device=x.device)
+                    in_dtype=_dtype_code(x.dtype), out_dtype=F32,
+                    flags=FLAG_FORCE_SIMT if force_simt else 0)
+    phi = out if out is not None else torch.empty(B, H, N, Dp, dtype=torch.float32,
+                                                  device=x.device)
     mlp = RehyatPhiMlp(Wa.data_ptr(), ba.data_ptr(), Wb.data_ptr(), bb.data_ptr(), Dh, parts)
-    _check(rehyat_feature_map_mlp(p, x.data_ptr(), mlp, phi.data_ptr(), _stream_handle(stream)),
-           "rehyat_feature_map_mlp")
+    nbytes = rehyat_feature_map_mlp_workspace_bytes(p, mlp, x.data_ptr(), phi.data_ptr())
+    if nbytes and (workspace is None or workspace.numel() < nbytes):
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=x.device)
+    ws_ptr = workspace.data_ptr() if nbytes else None
+    _check(rehyat_feature_map_mlp(p, x.data_ptr(), mlp, phi.data_ptr(), ws_ptr, nbytes,
+                                  _stream_handle(stream)), "rehyat_feature_map_mlp")
     return phi
 
 

@@ -216,6 +216,28 @@ rehyat_status state_pass(const rehyat_params* p, const void* k, const void* v,
                                p->D, p->causal, s));
 }
 
+// Checks and marshals the feature-map call; REHYAT_OK and *a filled, or the error.
+rehyat_status mlp_args(const rehyat_params* p, const void* x, const rehyat_phi_mlp* mlp,
+                       float* phi, PhiMlpArgs* a) {
+  rehyat_status st = check_params(p);
+  if (st != REHYAT_OK) return st;
+  if (!x || !mlp || !phi || !mlp->Wa || !mlp->ba || !mlp->Wb || !mlp->bb)
+    return REHYAT_ERR_INVALID_ARG;
+  if (mlp->parts < 1 || p->Dp % mlp->parts != 0 || mlp->Dh < 1) return REHYAT_ERR_INVALID_ARG;
+  if (mlp->Dh > 512) return REHYAT_ERR_UNSUPPORTED;
+  const void* ptrs[6] = {x, phi, mlp->Wa, mlp->ba, mlp->Wb, mlp->bb};
+  for (const void* q : ptrs)
+    if (reinterpret_cast<uintptr_t>(q) & 3) return REHYAT_ERR_MISALIGNED;
+  a->x = x; a->Wa = mlp->Wa; a->ba = mlp->ba; a->Wb = mlp->Wb; a->bb = mlp->bb; a->phi = phi;
+  a->N = static_cast<long long>(p->T) * p->Hs * p->Ws;
+  a->BH = p->batch * p->heads; a->heads = p->heads; a->D = p->D; a->Dh = mlp->Dh;
+  a->Dp = p->Dp; a->parts = mlp->parts; a->in_bf16 = p->in_dtype == REHYAT_BF16;
+  return REHYAT_OK;
+}
+
+bool mlp_tc(const rehyat_params* p, const PhiMlpArgs& a) {
+  return !(p->flags & REHYAT_FLAG_FORCE_SIMT) && tc_phi_mlp_eligible(a);
+}
 }  // namespace
 }  // namespace rehyat
 
@@ -441,23 +463,25 @@ rehyat_status rehyat_hybrid_attn_fwd_phi(const rehyat_params* p, const void* q, 
   return to_status(run_attn(p, a, s));
 }
 
-rehyat_status rehyat_feature_map_mlp(const rehyat_params* p, const void* x,
-                                     const rehyat_phi_mlp* mlp, float* phi, void* stream) {
-  rehyat_status st = check_params(p);
-  if (st != REHYAT_OK) return st;
-  if (!x || !mlp || !phi || !mlp->Wa || !mlp->ba || !mlp->Wb || !mlp->bb)
-    return REHYAT_ERR_INVALID_ARG;
-  if (mlp->parts < 1 || p->Dp % mlp->parts != 0 || mlp->Dh < 1) return REHYAT_ERR_INVALID_ARG;
-  if (mlp->Dh > 512) return REHYAT_ERR_UNSUPPORTED;
-  const void* ptrs[6] = {x, phi, mlp->Wa, mlp->ba, mlp->Wb, mlp->bb};
-  for (const void* q : ptrs)
-    if (reinterpret_cast<uintptr_t>(q) & 3) return REHYAT_ERR_MISALIGNED;
+size_t rehyat_feature_map_mlp_workspace_bytes(const rehyat_params* p, const rehyat_phi_mlp* mlp,
+                                              const void* x, const float* phi) {
   PhiMlpArgs a;
-  a.x = x; a.Wa = mlp->Wa; a.ba = mlp->ba; a.Wb = mlp->Wb; a.bb = mlp->bb; a.phi = phi;
-  a.N = static_cast<long long>(p->T) * p->Hs * p->Ws;
-  a.BH = p->batch * p->heads; a.heads = p->heads; a.D = p->D; a.Dh = mlp->Dh; a.Dp = p->Dp;
-  a.parts = mlp->parts; a.in_bf16 = p->in_dtype == REHYAT_BF16;
-  return to_status(launch_phi_mlp(a, static_cast<cudaStream_t>(stream)));
+  if (mlp_args(p, x, mlp, const_cast<float*>(phi), &a) != REHYAT_OK || !mlp_tc(p, a)) return 0;
+  return align_up(phi_mlp_image_bytes(a.heads, a.Dh, a.Dp));
+}
+
+rehyat_status rehyat_feature_map_mlp(const rehyat_params* p, const void* x,
+                                     const rehyat_phi_mlp* mlp, float* phi, void* workspace,
+                                     size_t ws_bytes, void* stream) {
+  PhiMlpArgs a;
+  const rehyat_status st = mlp_args(p, x, mlp, phi, &a);
+  if (st != REHYAT_OK) return st;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!mlp_tc(p, a)) return to_status(launch_phi_mlp(a, s));
+  if (!workspace || ws_bytes < phi_mlp_image_bytes(a.heads, a.Dh, a.Dp))
+    return REHYAT_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return REHYAT_ERR_MISALIGNED;
+  return to_status(launch_phi_mlp_tc(a, workspace, s));
 }
 
 size_t rehyat_phi_bwd_workspace_bytes(const rehyat_params* p) {

@@ -87,6 +87,12 @@ struct PhiMlpArgs {
   int BH, heads, D, Dh, Dp, parts, in_bf16;
 };
 cudaError_t launch_phi_mlp(const PhiMlpArgs& a, cudaStream_t s);
+// Tensor-core version (bf16 x, D = 128, D_h a multiple of 128, D' in
+// {64, 128}, x and phi 16-byte aligned, shared memory permitting); images
+// holds phi_mlp_image_bytes of bf16 weight images it writes first.
+bool tc_phi_mlp_eligible(const PhiMlpArgs& a);
+size_t phi_mlp_image_bytes(int heads, int Dh, int Dp);
+cudaError_t launch_phi_mlp_tc(const PhiMlpArgs& a, void* images, cudaStream_t s);
 
 // ---- SIMT (fp32 CUDA-core) kernels: every supported shape, both dtypes.
 cudaError_t launch_attn_simt(const AttnParams& p, cudaStream_t s);

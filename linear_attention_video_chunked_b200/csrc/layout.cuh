@@ -71,4 +71,18 @@ __host__ __device__ __forceinline__ long long wimg_index(int f, int d, int D, in
          n * 64 + ((chunk ^ (n & 7)) << 3) + w;
 }
 
+// A K-major bf16 operand [N rows][K] (K a multiple of 128) stored as pieces
+// of 128 K-elements (two 64-element boxes) by rp = min(N, 128) rows, piece
+// (kp, np) at ((kp * (N / rp) + np) * 2 * rp * 64); within a piece, box b
+// of row r at (b * rp + r) * 64.  Used for the two weight matrices of the
+// general feature map: W_a^T as [D_h][D] and W_b^T as [D'][D_h].
+__host__ __device__ __forceinline__ long long kpiece_img_index(int n, int k, int N) {
+  const int rp = N < 128 ? N : 128;
+  const int np = n / rp, r = n - np * rp;
+  const int kp = k >> 7, kk = k & 127;
+  const int box = kk >> 6, chunk = (kk >> 3) & 7, w = kk & 7;
+  return (static_cast<long long>(kp) * (N / rp) + np) * 2 * rp * 64 +
+         static_cast<long long>(box) * rp * 64 + r * 64 + ((chunk ^ (r & 7)) << 3) + w;
+}
+
 }  // namespace rehyat

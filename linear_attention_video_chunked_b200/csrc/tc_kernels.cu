@@ -1743,6 +1743,9 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s) {
 
 }  // namespace rehyat
 
+// The general feature map's tensor-core kernel shares this unit's helpers.
+#include "tc_phi_mlp.cuh"
+
 extern "C" rehyat_status rehyat_device_error_flags(unsigned* flags, int reset) {
   if (!flags) return REHYAT_ERR_INVALID_ARG;
   if (cudaMemcpyFromSymbol(flags, rehyat::rehyat_tc_error, sizeof(unsigned)) != cudaSuccess)

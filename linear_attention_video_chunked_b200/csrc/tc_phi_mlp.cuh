@@ -1,0 +1,395 @@
+// Tensor-core general feature map of ReHyAt for B200 (sm_100a).
+//
+// Source: "ReHyAt: Recurrent Hybrid Attention for Video Diffusion
+// Transformers" (papernotes.org note), Method, Key design 3: phi maps a head's
+// query or key through a light per-head embedding network whose output psi
+// is cut into P equal parts, part i raised to the power i:
+//   psi = GELU(x W_a + b_a) W_b + b_b,  GELU(u) = u * Phi(u) (exact form),
+//   phi = [psi_1^1, ..., psi_P^P].
+//
+// One persistent CTA per SM walks 128-token tiles of (head, batch, tile)
+// order, so a CTA changes weights at most a few times.  Per tile, the hidden
+// layer is computed in pieces of 128 columns:
+//   H_j   = X W_a[:, j]          tcgen05 (bf16 operands, fp32 in TMEM)
+//   G_j   = GELU(H_j + b_a)      converter warps, rounded to bf16 in place
+//   Psi  += G_j W_b[j, :]         tcgen05 with G_j read from TMEM (A operand)
+// then the epilogue warps add b_b, raise each part to its power and store
+// phi in fp32.  H has two TMEM buffers, so the product of piece j + 1 runs
+// while piece j is converted; Psi has two, so one tile is stored while the
+// next accumulates.
+//
+// Roles (448 threads):
+//   warps 0-7   converters: warp w reads TMEM lanes 32 (w mod 4) .. (the
+//               tile's rows) and hidden columns 64 (w / 4) .. of a piece;
+//   warps 8-11  epilogue: thread = token row, all D' columns;
+//   warp 12     TMA producer (one lane): X tiles, weight images;
+//   warp 13     MMA issuer (one lane) and TMEM owner.
+// TMEM (512 columns): H [0,128) [128,256), Psi [256,384) [384,512).
+// Shared memory: X tile (32 KB), then the bf16 images of W_a^T and W_b^T of
+// the current head (layout.cuh, kpiece_img_index), then the barriers.
+//
+// This file is part of the translation unit of tc_kernels.cu (it shares the
+// wait helpers, the error word and the tensor-map helpers defined there).
+
+namespace rehyat {
+namespace {
+
+namespace mlp {
+constexpr int kThreads = 448;
+constexpr int kEpiWarp0 = 8, kProducerWarp = 12, kMmaWarp = 13;
+constexpr uint32_t kXOff = 0, kWOff = 32768;
+enum { X_FULL = 0, X_EMPTY = 1, W_FULL = 2, W_FREE = 3, H_FULL = 4, PACKED = 6, PSI_FULL = 8,
+       PSI_FREE = 10, NBAR = 12 };
+constexpr uint32_t kColH = 0, kColPsi = 256;
+constexpr uint32_t kMaxSmem = 232448;  // opt-in dynamic shared memory per block
+
+// Bytes of one head's weight images: W_a^T [D_h][128] and W_b^T [D'][D_h].
+__host__ __device__ constexpr uint32_t w_bytes(int Dh, int Dp) {
+  return static_cast<uint32_t>(Dh) * 256u + static_cast<uint32_t>(Dp) * Dh * 2u;
+}
+__host__ __device__ constexpr uint32_t bar_off(int Dh, int Dp) { return kWOff + w_bytes(Dh, Dp); }
+__host__ __device__ constexpr uint32_t smem_bytes(int Dh, int Dp) {
+  return bar_off(Dh, Dp) + 256u + 1024u;  // barriers, TMEM slot, abort flag; alignment slack
+}
+
+struct Args {
+  const __nv_bfloat16* img;  // [heads][w_bytes / 2] weight images
+  const float* ba;           // [heads][Dh]
+  const float* bb;           // [heads][Dp]
+  float* phi;                // [B*heads][N][Dp]
+  long long N;
+  int batch, heads, Dh, Dp, parts, ntile, tiles_per_cta;
+};
+
+// Tile it of the walk: it = (h * batch + b) * ntile + tile.
+struct Tile {
+  int h, b, tile;
+};
+__device__ __forceinline__ Tile tile_of(int it, int batch, int ntile) {
+  Tile t;
+  const int hb = it / ntile;
+  t.tile = it - hb * ntile;
+  t.h = hb / batch;
+  t.b = hb - t.h * batch;
+  return t;
+}
+
+__device__ __forceinline__ float gelu(float u) {
+  return 0.5f * u * (1.f + erff(u * 0.70710678118654752f));
+}
+}  // namespace mlp
+
+__global__ void __launch_bounds__(mlp::kThreads, 1)
+    tc_phi_mlp_kernel(const __grid_constant__ CUtensorMap xmap, const mlp::Args a) {
+  // Local names shadow the attention kernel's constants of the same names.
+  constexpr int kProducerWarp = mlp::kProducerWarp, kMmaWarp = mlp::kMmaWarp;
+  constexpr int kEpiWarp0 = mlp::kEpiWarp0;
+  constexpr uint32_t kXOff = mlp::kXOff, kWOff = mlp::kWOff;
+  constexpr uint32_t kColH = mlp::kColH, kColPsi = mlp::kColPsi;
+  using mlp::X_FULL;
+  using mlp::X_EMPTY;
+  using mlp::W_FULL;
+  using mlp::W_FREE;
+  using mlp::H_FULL;
+  using mlp::PACKED;
+  using mlp::PSI_FULL;
+  using mlp::PSI_FREE;
+  using mlp::NBAR;
+  using mlp::Tile;
+  using mlp::tile_of;
+  using mlp::bar_off;
+  using mlp::w_bytes;
+  using mlp::gelu;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* sbase = smem_raw + (base - raw);
+  const int Dh = a.Dh, Dp = a.Dp;
+  const uint32_t boff = bar_off(Dh, Dp);
+  auto bar = [&](int i) { return base + boff + 8u * i; };
+  const uint32_t tmem_slot = boff + 8u * NBAR;
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(sbase + tmem_slot + 4);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int J = Dh >> 7;  // hidden pieces of 128
+  const int total = a.heads * a.batch * a.ntile;
+  const int it0 = blockIdx.x * a.tiles_per_cta;
+  const int it1 = min(total, it0 + a.tiles_per_cta);
+  if (it0 >= it1) return;
+
+  if (tid == 0) {
+    for (int i = 0; i < NBAR; ++i) {
+      uint32_t count = 1;
+      if (i == PACKED || i == PACKED + 1) count = 8;      // one arrive per converter warp
+      if (i == PSI_FREE || i == PSI_FREE + 1) count = 4;  // one per epilogue warp
+      mbar_init(bar(i), count);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == kMmaWarp) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     base + tmem_slot),
+                 "r"(512));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sbase + tmem_slot);
+
+  if (warp == kProducerWarp) {
+    // ================================================= TMA producer
+    if (lane == 0) {
+      bool ok = true;
+      int wl = 0, head = -1;
+      const uint32_t wb = w_bytes(Dh, Dp);
+      for (int it = it0, tl = 0; it < it1 && ok; ++it, ++tl) {
+        const Tile t = tile_of(it, a.batch, a.ntile);
+        if (t.h != head) {
+          head = t.h;
+          if (wl > 0) ok = mbar_wait(bar(W_FREE), (wl - 1) & 1, abort_flag, 40);
+          if (!ok) break;
+          const uint8_t* src = reinterpret_cast<const uint8_t*>(a.img) +
+                               static_cast<long long>(t.h) * wb;
+          mbar_expect_tx(bar(W_FULL), wb);
+          for (uint32_t o = 0; o < wb; o += 32768u)
+            bulk_load(base + kWOff + o, src + o, wb - o < 32768u ? wb - o : 32768u, bar(W_FULL));
+          ++wl;
+        }
+        if (tl > 0) ok = mbar_wait(bar(X_EMPTY), (tl - 1) & 1, abort_flag, 41);
+        if (!ok) break;
+        const int plane = t.b * a.heads + t.h;
+        mbar_expect_tx(bar(X_FULL), 32768);
+        tma_load_3d(base + kXOff, &xmap, bar(X_FULL), 0, t.tile * 128, plane);
+        tma_load_3d(base + kXOff + 16384, &xmap, bar(X_FULL), 64, t.tile * 128, plane);
+      }
+    }
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    // ================================================= MMA issuer
+    if (lane == 0) {
+      const uint32_t id1 = idesc(128, 128, 1, false);  // X . W_a piece, both K-major
+      const uint32_t id2 = idesc(128, Dp, 1, false);   // G (TMEM) . W_b piece
+      const uint64_t xdesc = sdesc(base + kXOff, 16, 1024);
+      const uint32_t wb_off = kWOff + static_cast<uint32_t>(Dh) * 256u;
+      bool ok = true;
+      int wwaits = 0, head = -1;
+      int pend = -1, pend_tl = 0, pend_j = 0;  // piece whose second product is not issued
+      // Second product of piece g (tile tl, piece j): waits for its GELU
+      // output, and at j = 0 for the epilogue to have drained Psi buffer
+      // tl & 1 (tile tl - 2).
+      auto issue_g2 = [&](int g, int tl, int j) -> bool {
+        const int b = g & 1, pb = tl & 1;
+        if (!mbar_wait(bar(PACKED + b), (g >> 1) & 1, abort_flag, 42)) return false;
+        if (j == 0 && tl >= 2 && !mbar_wait(bar(PSI_FREE + pb), ((tl - 2) >> 1) & 1, abort_flag, 43))
+          return false;
+        tc_fence_after();
+        const uint64_t bdesc = sdesc(base + wb_off + static_cast<uint32_t>(j * Dp) * 256u, 16, 1024);
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+          // k-step s: hidden 16 s .. of the piece; the converter half s / 4
+          // left its 32 packed columns at the start of its 64 input columns.
+          const uint32_t acol = tmem + kColH + b * 128 + (s >> 2) * 64 + (s & 3) * 8;
+          const uint64_t off = static_cast<uint64_t>(((s >> 2) * Dp * 128 + (s & 3) * 32) >> 4);
+          mma_bf16_ts(tmem + kColPsi + pb * 128, acol, bdesc + off, id2,
+                      (j > 0 || s > 0) ? 1u : 0u);
+        }
+        if (j == J - 1) mma_commit(bar(PSI_FULL + pb));
+        return true;
+      };
+      int gp = 0;
+      for (int it = it0, tl = 0; it < it1 && ok; ++it, ++tl) {
+        const Tile t = tile_of(it, a.batch, a.ntile);
+        for (int j = 0; j < J && ok; ++j, ++gp) {
+          if (j == 0) {
+            if (t.h != head) {
+              // Finish every product that reads the old weights, then let
+              // the producer replace them.
+              if (pend >= 0) {
+                ok = issue_g2(pend, pend_tl, pend_j);
+                pend = -1;
+                if (!ok) break;
+                mma_commit(bar(W_FREE));
+              }
+              head = t.h;
+              ok = mbar_wait(bar(W_FULL), wwaits & 1, abort_flag, 44);
+              ++wwaits;
+              if (!ok) break;
+            }
+            ok = mbar_wait(bar(X_FULL), tl & 1, abort_flag, 45);
+            if (!ok) break;
+          }
+          tc_fence_after();
+          // H buffer gp & 1 was last read by the second product of piece
+          // gp - 2, issued before this point (one thread's tcgen05 ops run
+          // in order), after its converters had finished with it.
+          const int b = gp & 1;
+          const uint64_t wdesc = sdesc(base + kWOff + static_cast<uint32_t>(j) * 32768u, 16, 1024);
+#pragma unroll
+          for (int s = 0; s < 8; ++s) {
+            const uint64_t off = static_cast<uint64_t>(((s >> 2) * 16384 + (s & 3) * 32) >> 4);
+            mma_bf16(tmem + kColH + b * 128, xdesc + off, wdesc + off, id1, s > 0 ? 1u : 0u);
+          }
+          mma_commit(bar(H_FULL + b));
+          if (j == J - 1) mma_commit(bar(X_EMPTY));
+          if (pend >= 0) ok = issue_g2(pend, pend_tl, pend_j);
+          pend = gp;
+          pend_tl = tl;
+          pend_j = j;
+        }
+      }
+      if (ok && pend >= 0) issue_g2(pend, pend_tl, pend_j);
+    }
+    __syncwarp();
+  } else if (warp < kEpiWarp0) {
+    // ================================================= converters
+    const int hc = warp >> 2;  // column half of a piece
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    bool ok = true;
+    int gp = 0;
+    for (int it = it0; it < it1 && ok; ++it) {
+      const Tile t = tile_of(it, a.batch, a.ntile);
+      for (int j = 0; j < J; ++j, ++gp) {
+        const int b = gp & 1;
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(H_FULL + b), (gp >> 1) & 1, abort_flag, 46));
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t col = lane_base + kColH + b * 128 + hc * 64;
+        const float* bias = a.ba + static_cast<long long>(t.h) * Dh + j * 128 + hc * 64;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          // Columns 32c..32c+31 become packed columns 16c..16c+15, which
+          // this thread has already read (chunk 0 writes over its own input).
+          uint32_t r[32];
+          REHYAT_TMEM_LD32(col + c * 32, r);
+          REHYAT_TMEM_WAIT_LD32(r);
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float u0 = __uint_as_float(r[2 * i]) + __ldg(bias + c * 32 + 2 * i);
+            const float u1 = __uint_as_float(r[2 * i + 1]) + __ldg(bias + c * 32 + 2 * i + 1);
+            pk[i] = pack_bf16(gelu(u0), gelu(u1));
+          }
+          REHYAT_TMEM_ST16(col + c * 16, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(PACKED + b));
+      }
+    }
+  } else {
+    // ================================================= epilogue (thread = token)
+    const int q = warp - kEpiWarp0;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    const int width = Dp / a.parts;
+    bool ok = true;
+    int tl = 0;
+    for (int it = it0; it < it1 && ok; ++it, ++tl) {
+      const Tile t = tile_of(it, a.batch, a.ntile);
+      const int pb = tl & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(PSI_FULL + pb), (tl >> 1) & 1, abort_flag, 47));
+      if (!ok) break;
+      tc_fence_after();
+      const long long row = static_cast<long long>(t.tile) * 128 + q * 32 + lane;
+      const bool valid = row < a.N;
+      float* out = a.phi + (static_cast<long long>(t.b * a.heads + t.h) * a.N + row) * Dp;
+      const float* bias = a.bb + static_cast<long long>(t.h) * Dp;
+      for (int c0 = 0; c0 < Dp; c0 += 32) {
+        uint32_t r[32];
+        REHYAT_TMEM_LD32(lane_base + kColPsi + pb * 128 + c0, r);
+        REHYAT_TMEM_WAIT_LD32(r);
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int f = c0 + i;
+          const float x = __uint_as_float(r[i]) + __ldg(bias + f);
+          const int power = f / width + 1;  // the same for every lane
+          float y = x;
+          for (int e = 1; e < power; ++e) y *= x;
+          v[i] = y;
+        }
+        if (valid) {
+          float4* o4 = reinterpret_cast<float4*>(out + c0);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            o4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(PSI_FREE + pb));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+  }
+}
+
+// bf16 weight images of every head: W_a^T [D_h][D] then W_b^T [D'][D_h]
+// (kpiece_img_index), one thread per weight, reads coalesced along the
+// fastest index of W_a [D][D_h] and W_b [D_h][D'].
+__global__ void phi_mlp_image_kernel(const float* __restrict__ Wa, const float* __restrict__ Wb,
+                                     __nv_bfloat16* __restrict__ img, int Dh, int Dp) {
+  const int h = blockIdx.y;
+  const long long na = static_cast<long long>(Dh) * 128, nb = static_cast<long long>(Dh) * Dp;
+  const long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  __nv_bfloat16* out = img + static_cast<long long>(h) * (na + nb);
+  if (e < na) {
+    const int d = static_cast<int>(e / Dh), j = static_cast<int>(e % Dh);
+    out[kpiece_img_index(j, d, Dh)] = __float2bfloat16_rn(Wa[h * na + e]);
+  } else if (e < na + nb) {
+    const long long e2 = e - na;
+    const int j = static_cast<int>(e2 / Dp), f = static_cast<int>(e2 % Dp);
+    out[na + kpiece_img_index(f, j, Dp)] = __float2bfloat16_rn(Wb[h * nb + e2]);
+  }
+}
+
+}  // namespace
+
+bool tc_phi_mlp_eligible(const PhiMlpArgs& a) {
+  return a.in_bf16 && a.D == kD && a.Dh >= 128 && a.Dh % 128 == 0 && (a.Dp == 64 || a.Dp == 128) &&
+         mlp::smem_bytes(a.Dh, a.Dp) <= mlp::kMaxSmem &&
+         (reinterpret_cast<uintptr_t>(a.x) & 15) == 0 &&
+         (reinterpret_cast<uintptr_t>(a.phi) & 15) == 0 && encode_fn() != nullptr;
+}
+
+size_t phi_mlp_image_bytes(int heads, int Dh, int Dp) {
+  return static_cast<size_t>(heads) * mlp::w_bytes(Dh, Dp);
+}
+
+cudaError_t launch_phi_mlp_tc(const PhiMlpArgs& a, void* images, cudaStream_t s) {
+  const long long nw = static_cast<long long>(a.Dh) * (128 + a.Dp);
+  phi_mlp_image_kernel<<<dim3(static_cast<unsigned>((nw + 255) / 256), a.heads), 256, 0, s>>>(
+      a.Wa, a.Wb, static_cast<__nv_bfloat16*>(images), a.Dh, a.Dp);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  CUtensorMap xmap;
+  if (!make_map(&xmap, a.x, a.N, a.BH)) return cudaErrorInvalidValue;
+  mlp::Args m;
+  m.img = static_cast<const __nv_bfloat16*>(images);
+  m.ba = a.ba;
+  m.bb = a.bb;
+  m.phi = a.phi;
+  m.N = a.N;
+  m.batch = a.BH / a.heads;
+  m.heads = a.heads;
+  m.Dh = a.Dh;
+  m.Dp = a.Dp;
+  m.parts = a.parts;
+  m.ntile = static_cast<int>((a.N + 127) / 128);
+  const int total = a.BH * m.ntile;
+  const int sms = sm_count();
+  m.tiles_per_cta = (total + sms - 1) / sms;
+  const int ctas = (total + m.tiles_per_cta - 1) / m.tiles_per_cta;
+  e = ensure_smem(tc_phi_mlp_kernel, 4, mlp::kMaxSmem);
+  if (e != cudaSuccess) return e;
+  tc_phi_mlp_kernel<<<ctas, mlp::kThreads, mlp::smem_bytes(a.Dh, a.Dp), s>>>(xmap, m);
+  return cudaGetLastError();
+}
+
+}  // namespace rehyat

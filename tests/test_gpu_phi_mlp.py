@@ -2,8 +2,13 @@
 forward with given feature maps (rehyat_hybrid_attn_fwd_phi), through the C
 ABI, against the fp64 oracle (oracle/rehyat_phi_mlp.py) on the same seeded
 inputs.  Bars as for the forward: fp32 inputs max abs <= 1e-5 on y; bf16
-inputs max abs <= 2e-2, mean abs <= 2e-3; the feature map itself (fp32 CUDA
-cores vs fp64) within 1e-5 relative to its largest value.
+inputs max abs <= 2e-2, mean abs <= 2e-3.  The feature map itself: on CUDA
+cores (fp32) within 1e-5 relative to its largest value; on the tensor cores
+(bf16 operands) within the first-order bound of rounding W_a, GELU(.) and
+W_b to bf16 (unit roundoff u = 2^-8), element by element:
+  |d psi_f| <= u * sum_j |W_b[j,f]| (1.13 sum_d |x_d W_a[d,j]| + 2 |g_j|),
+  |d phi|   <= (|psi| + |d psi|)^i - |psi|^i   for part i,
+with 1.13 >= max |GELU'|, times 1.1 for second-order and fp32 terms.
 """
 import numpy as np
 import pytest
@@ -14,6 +19,7 @@ from oracle import rehyat_oracle as orc
 from oracle.rehyat_phi_mlp import feature_map_mlp, hybrid_phi_given
 from rehyat_inputs import make_problem
 from tests.gpu_util import assert_close_partials, assert_close_y, device_tensors
+from tests.mlp_bound import bf16_bound
 
 pytestmark = pytest.mark.gpu
 
@@ -132,3 +138,100 @@ def test_mlp_phi_end_to_end(dtype, parts_n, causal):
     for key in ("nL", "aL"):
         err = np.abs(got[key] - ref_p[key]).max()
         assert err <= rel * np.abs(ref_p[key]).max(), (key, err)
+
+
+# ------------------------------------------------ tensor-core feature map
+def _tc_map(x_dev, params, parts, T, Hs, Ws):
+    """phi (fp32 CUDA tensor) from the tensor-core path of the C ABI."""
+    B, H, N, D = x_dev.shape
+    Dh, Dp = params[0].shape[-1], params[2].shape[-1]
+    p = rh.make_params(batch=B, heads=H, T=T, Hs=Hs, Ws=Ws, D=D, Dp=Dp, Tc=1, To=0, causal=0,
+                       in_dtype=rh.BF16, out_dtype=rh.F32)
+    dev = [_cuda32(t) for t in params]
+    phi = torch.empty(B, H, N, Dp, dtype=torch.float32, device="cuda")
+    mlp = rh.RehyatPhiMlp(*(t.data_ptr() for t in dev), Dh, parts)
+    nbytes = rh.rehyat_feature_map_mlp_workspace_bytes(p, mlp, x_dev.data_ptr(), phi.data_ptr())
+    assert nbytes > 0, "tensor-core path not selected"
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    st = rh.rehyat_feature_map_mlp(p, x_dev.data_ptr(), mlp, phi.data_ptr(), ws.data_ptr(),
+                                   nbytes, torch.cuda.current_stream().cuda_stream)
+    assert st == 0, rh.rehyat_status_string(st)
+    # Too small a workspace is refused before any launch.
+    assert rh.rehyat_feature_map_mlp(p, x_dev.data_ptr(), mlp, phi.data_ptr(), ws.data_ptr(),
+                                     nbytes - 16, None) == 4  # REHYAT_ERR_WORKSPACE
+    torch.cuda.synchronize()
+    return phi
+
+
+TC_SHAPES = [
+    # B, h, T, Hs, Ws, Dh, Dp, parts: what it covers
+    (1, 2, 1, 5, 19, 128, 128, 2),     # N = 95 < 128: one ragged tile per (b,h)
+    (1, 3, 1, 43, 179, 384, 128, 2),   # 61 tiles per head: a CTA of 2 tiles spans two heads
+    (2, 4, 2, 9, 289, 256, 64, 4),     # 41 tiles per (b,h), 3 per CTA; D' = 64, P = 4
+    (1, 2, 3, 7, 13, 512, 64, 1),      # D_h = 512 (largest that fits with D' = 64), P = 1
+]
+
+
+@pytest.mark.parametrize("shape", TC_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_feature_map_mlp_tensor_cores_withinbf16_bound(shape):
+    B, H, T, Hs, Ws, Dh, Dp, parts = shape
+    p = make_problem(batch=B, heads=H, T=T, Hs=Hs, Ws=Ws, D=128, Dp=Dp, Tc=1, To=0,
+                     causal=False, dtype="bf16", seed=600 + Dh + parts)
+    params = _mlp_params(H, 128, Dh, Dp, 601 + Dh, scale=0.5)
+    got = _tc_map(device_tensors(p)["q"], params, parts, T, Hs, Ws).double().cpu().numpy()
+    Wa, ba, Wb, bb = params
+    x = np.asarray(p.q, np.float64)
+    for b in range(B):
+        for h in range(H):
+            ref = feature_map_mlp(x[b, h], Wa[h], ba[h], Wb[h], bb[h], parts)
+            bound = bf16_bound(x[b, h], Wa[h], ba[h], Wb[h], bb[h], parts)
+            err = np.abs(got[b, h] - ref)
+            worst = np.unravel_index(np.argmax(err - bound), err.shape)
+            assert np.all(err <= bound + 1e-6 * np.abs(ref).max()), (b, h, worst, err[worst],
+                                                                       bound[worst])
+            # The bound is not vacuous: the typical error is far inside it.
+            assert np.median(err) < 0.25 * np.median(bound) + 1e-12
+
+
+def test_feature_map_mlp_tensor_cores_full_size_sampled_rows():
+    """The general-phi bench configuration (B = 2, h = 12, 21 x 30 x 52,
+    D_h = 3D = 384, D' = 128, P = 2) in the launch the bench times, checked
+    on 64 sampled tokens of every (b, h) against the oracle."""
+    B, H, T, Hs, Ws, Dh, Dp, parts = 2, 12, 21, 30, 52, 384, 128, 2
+    N = T * Hs * Ws
+    g = torch.Generator().manual_seed(7)
+    x = (torch.randn(B, H, N, 128, generator=g) * 1.5).to(torch.bfloat16)
+    params = _mlp_params(H, 128, Dh, Dp, 602, scale=0.5)
+    rows = np.random.default_rng(8).choice(N, size=64, replace=False)
+    rows[:2] = [0, N - 1]
+    idx = torch.tensor(rows)
+    got = _tc_map(x.cuda(), params, parts, T, Hs, Ws)[:, :, idx.cuda()].double().cpu().numpy()
+    xs = x[:, :, idx].double().numpy()
+    Wa, ba, Wb, bb = params
+    for b in range(B):
+        for h in range(H):
+            xr = xs[b, h]
+            ref = feature_map_mlp(xr, Wa[h], ba[h], Wb[h], bb[h], parts)
+            bound = bf16_bound(xr, Wa[h], ba[h], Wb[h], bb[h], parts)
+            err = np.abs(got[b, h] - ref)
+            assert np.all(err <= bound + 1e-6 * np.abs(ref).max()), (b, h, err.max())
+
+
+def test_feature_map_mlp_force_simt_and_fp32_take_cuda_cores():
+    """FLAG_FORCE_SIMT (and fp32 x) select the fp32 CUDA-core kernel, which
+    needs no workspace and meets the fp32 bar."""
+    p = make_problem(batch=1, heads=2, T=2, Hs=5, Ws=7, D=128, Dp=128, Tc=1, To=0,
+                     causal=False, dtype="bf16", seed=77)
+    params = _mlp_params(2, 128, 256, 128, 78)
+    dev = device_tensors(p)
+    got = rh.feature_map_mlp(dev["q"], *(_cuda32(a) for a in params), parts=2, T=p.T, Hs=p.Hs,
+                             Ws=p.Ws, force_simt=True)
+    torch.cuda.synchronize()
+    ref = _oracle_phi(np.asarray(p.q, np.float64), params, 2)
+    err = np.abs(got.double().cpu().numpy() - ref).max()
+    assert err <= 1e-5 * np.abs(ref).max(), err
+    pf = rh.make_params(batch=1, heads=2, T=p.T, Hs=p.Hs, Ws=p.Ws, D=128, Dp=128, Tc=1, To=0,
+                        causal=0, in_dtype=rh.F32, out_dtype=rh.F32)
+    mlp = rh.RehyatPhiMlp(*(_cuda32(a).data_ptr() for a in params), 256, 2)
+    assert rh.rehyat_feature_map_mlp_workspace_bytes(pf, mlp, dev["q"].data_ptr(),
+                                                     got.data_ptr()) == 0

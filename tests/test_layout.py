@@ -1,7 +1,8 @@
 """Host-side check of the shared-memory image layouts (csrc/layout.cuh):
 sl_index is a bijection on [0, D*D'), sl_coords inverts it, the split form
 (feature base + column offset) agrees with it, and the weight image index is
-a bijection too, for every supported (D, D')."""
+a bijection too, for every supported (D, D'); so is the K-pieced image of the
+general feature map's weights."""
 import os
 import shutil
 import subprocess
@@ -38,6 +39,21 @@ int main() {
       if (seen[i] != 1) ++bad;
       if (D >= 64 && seen_w[i] != 1) ++bad;
     }
+  }
+  // K-pieced weight images of the general feature map: W_a^T [Dh][128] and
+  // W_b^T [Dp][Dh] are bijections onto [0, N*K).
+  const int Ns[] = {64, 128, 256, 384, 512}, Ks[] = {128, 256, 384, 512};
+  for (int N : Ns) for (int K : Ks) {
+    std::vector<int> seen_k((size_t)N * K, 0);
+    for (int n = 0; n < N; ++n) for (int k = 0; k < K; ++k) {
+      const long long o = kpiece_img_index(n, k, N);
+      if (o < 0 || o >= (long long)N * K) { ++bad; continue; }
+      seen_k[o]++;
+      // 16-byte chunks stay within their 128-byte row; row r of a box at r * 64.
+      const int rp = N < 128 ? N : 128;
+      if ((o % 64) / 8 != (((k & 127) >> 3) & 7 ^ ((n % rp) & 7))) ++bad;
+    }
+    for (long long i = 0; i < (long long)N * K; ++i) if (seen_k[i] != 1) ++bad;
   }
   std::printf("%d\n", bad);
   return bad != 0;

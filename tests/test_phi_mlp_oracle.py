@@ -84,3 +84,37 @@ def test_phi_given_equals_pairwise_definition(causal):
             num += w * v[0, 0, j]
             den += w
         assert np.allclose(y[0, 0, i], num / den, rtol=1e-10, atol=1e-12), i
+
+
+def _bf16(a):
+    import torch
+    return torch.tensor(np.asarray(a, np.float32)).to(torch.bfloat16).double().numpy()
+
+
+@pytest.mark.parametrize("P", [1, 2, 4])
+def test_bf16_bound_covers_emulated_bf16_map(P):
+    """The tolerance used for the tensor-core map (tests/mlp_bound.py) holds
+    for an fp64 emulation that rounds W_a, GELU(.) and W_b to bf16 the way
+    the kernel does, and is tight enough to catch a dropped bias or a wrong
+    power (each exceeds it)."""
+    from tests.mlp_bound import bf16_bound
+    rng = np.random.default_rng(9)
+    D, Dh, Dp = 128, 256, 64
+    x = _bf16(rng.standard_normal((200, D)) * 1.5)
+    Wa = rng.standard_normal((D, Dh)) / np.sqrt(D)
+    ba = rng.standard_normal(Dh) * 0.1
+    Wb = rng.standard_normal((Dh, Dp)) / np.sqrt(Dh) * 0.5
+    bb = rng.standard_normal(Dp) * 0.05
+    ref = feature_map_mlp(x, Wa, ba, Wb, bb, P)
+    g = _bf16(gelu(x @ _bf16(Wa) + ba))
+    psi = g @ _bf16(Wb) + bb
+    w = Dp // P
+    emu = np.concatenate([psi[:, i * w:(i + 1) * w] ** (i + 1) for i in range(P)], axis=1)
+    bound = bf16_bound(x, Wa, ba, Wb, bb, P)
+    assert np.all(np.abs(emu - ref) <= bound)
+    no_bias = np.concatenate([(psi - bb)[:, i * w:(i + 1) * w] ** (i + 1) for i in range(P)],
+                             axis=1)
+    assert np.any(np.abs(no_bias - ref) > bound)
+    if P > 1:
+        wrong_power = psi ** 2
+        assert np.any(np.abs(wrong_power - ref) > bound)
