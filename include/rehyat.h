@@ -233,7 +233,7 @@ typedef struct {
 /* Workspace bytes rehyat_feature_map_mlp needs for these shapes (0 when it
  * runs on CUDA cores, or if p or mlp is invalid).  The tensor-core path
  * (bf16 x, D = 128, Dh a multiple of 128 with Dh * 256 + Dp * Dh * 2 <=
- * 198,656, Dp in {64, 128}, x and phi 16-byte aligned, no
+ * 198,656, Dp in {64, 128}, x, phi, ba and bb 16-byte aligned, no
  * REHYAT_FLAG_FORCE_SIMT) keeps bf16 images of Wa and Wb there. */
 REHYAT_API size_t rehyat_feature_map_mlp_workspace_bytes(const rehyat_params* p,
                                                          const rehyat_phi_mlp* mlp,
@@ -244,8 +244,9 @@ REHYAT_API size_t rehyat_feature_map_mlp_workspace_bytes(const rehyat_params* p,
  * 4-byte aligned; workspace (caller-owned, 16-byte aligned, may be NULL when
  * the size above is 0) of at least rehyat_feature_map_mlp_workspace_bytes
  * bytes.  Tensor-core path: x, W_a, GELU(.) and W_b enter the products as
- * bf16 (fp32 accumulation, b_a, b_b and the powers in fp32); CUDA-core path:
- * fp32 throughout.  REHYAT_ERR_INVALID_ARG for parts < 1 or Dp % parts != 0;
+ * bf16 (fp32 accumulation, b_a, b_b and the powers in fp32; erf inside GELU
+ * from Abramowitz & Stegun 7.1.26, |error| <= 1.5e-7); CUDA-core path: fp32
+ * throughout (erff).  REHYAT_ERR_INVALID_ARG for parts < 1 or Dp % parts != 0;
  * REHYAT_ERR_WORKSPACE if ws_bytes is too small. */
 REHYAT_API rehyat_status rehyat_feature_map_mlp(const rehyat_params* p, const void* x,
                                                 const rehyat_phi_mlp* mlp, float* phi,

@@ -74,8 +74,29 @@ __device__ __forceinline__ Tile tile_of(int it, int batch, int ntile) {
   return t;
 }
 
+// GELU(u) = u Phi(u) with Phi(u) = (1 + erf(u / sqrt 2)) / 2 and erf from
+// Abramowitz & Stegun, Handbook of Mathematical Functions, 7.1.26 (after
+// Hastings): for x >= 0, erf(x) = 1 - q(x) with q = t (a1 + t (a2 + t (a3 +
+// t (a4 + t a5)))) exp(-x^2), t = 1 / (1 + p x), |error| <= 1.5e-7 -- far
+// below the bf16 rounding the result gets next.  Phi(u) = 1 - q/2 for u >= 0
+// and q/2 for u < 0 (no cancellation in the tail).  One reciprocal and one
+// exponential on MUFU, five FMAs.
 __device__ __forceinline__ float gelu(float u) {
-  return 0.5f * u * (1.f + erff(u * 0.70710678118654752f));
+  constexpr float kP = 0.3275911f;
+  constexpr float kA1 = 0.254829592f, kA2 = -0.284496736f, kA3 = 1.421413741f;
+  constexpr float kA4 = -1.453152027f, kA5 = 1.061405429f;
+  constexpr float kInvSqrt2 = 0.70710678118654752f;
+  constexpr float kNegLog2e = -1.4426950408889634f;
+  const float x = fabsf(u) * kInvSqrt2;
+  float t;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(t) : "f"(fmaf(kP, x, 1.f)));
+  float poly = fmaf(kA5, t, kA4);
+  poly = fmaf(poly, t, kA3);
+  poly = fmaf(poly, t, kA2);
+  poly = fmaf(poly, t, kA1);
+  const float q = poly * t * ex2(x * x * kNegLog2e);
+  const float phi = u >= 0.f ? fmaf(-0.5f, q, 1.f) : 0.5f * q;
+  return u * phi;
 }
 }  // namespace mlp
 
@@ -255,23 +276,37 @@ __global__ void __launch_bounds__(mlp::kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         const uint32_t col = lane_base + kColH + b * 128 + hc * 64;
-        const float* bias = a.ba + static_cast<long long>(t.h) * Dh + j * 128 + hc * 64;
+        // b_a of these 64 hidden columns (16-byte aligned; the same address
+        // in every lane, so each load is a broadcast).
+        const float4* bias4 = reinterpret_cast<const float4*>(
+            a.ba + static_cast<long long>(t.h) * Dh + j * 128 + hc * 64);
+        // Both 32-column chunks are loaded up front.  Columns 32c..32c+31
+        // become packed columns 16c..16c+15, which this thread has already
+        // read (chunk 0 writes over its own input).
+        uint32_t r0[32], r1[32];
+        REHYAT_TMEM_LD32(col, r0);
+        REHYAT_TMEM_LD32(col + 32, r1);
+        float4 bq[8];
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          // Columns 32c..32c+31 become packed columns 16c..16c+15, which
-          // this thread has already read (chunk 0 writes over its own input).
-          uint32_t r[32];
-          REHYAT_TMEM_LD32(col + c * 32, r);
-          REHYAT_TMEM_WAIT_LD32(r);
+        for (int i = 0; i < 8; ++i) bq[i] = __ldg(bias4 + i);
+        auto convert = [&](const uint32_t* r, uint32_t dst) {
           uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float u0 = __uint_as_float(r[2 * i]) + __ldg(bias + c * 32 + 2 * i);
-            const float u1 = __uint_as_float(r[2 * i + 1]) + __ldg(bias + c * 32 + 2 * i + 1);
-            pk[i] = pack_bf16(gelu(u0), gelu(u1));
+          for (int i = 0; i < 8; ++i) {
+            const float4 b4 = bq[i];
+            pk[2 * i] = pack_bf16(gelu(__uint_as_float(r[4 * i]) + b4.x),
+                                  gelu(__uint_as_float(r[4 * i + 1]) + b4.y));
+            pk[2 * i + 1] = pack_bf16(gelu(__uint_as_float(r[4 * i + 2]) + b4.z),
+                                      gelu(__uint_as_float(r[4 * i + 3]) + b4.w));
           }
-          REHYAT_TMEM_ST16(col + c * 16, pk);
-        }
+          REHYAT_TMEM_ST16(dst, pk);
+        };
+        REHYAT_TMEM_WAIT_LD32(r0);
+        REHYAT_TMEM_WAIT_LD32(r1);
+        convert(r0, col);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) bq[i] = __ldg(bias4 + 8 + i);
+        convert(r1, col + 16);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -294,16 +329,25 @@ __global__ void __launch_bounds__(mlp::kThreads, 1)
       const long long row = static_cast<long long>(t.tile) * 128 + q * 32 + lane;
       const bool valid = row < a.N;
       float* out = a.phi + (static_cast<long long>(t.b * a.heads + t.h) * a.N + row) * Dp;
-      const float* bias = a.bb + static_cast<long long>(t.h) * Dp;
+      const float4* bias4 = reinterpret_cast<const float4*>(a.bb + static_cast<long long>(t.h) * Dp);
       for (int c0 = 0; c0 < Dp; c0 += 32) {
         uint32_t r[32];
         REHYAT_TMEM_LD32(lane_base + kColPsi + pb * 128 + c0, r);
+        float bv[32];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float4 b4 = __ldg(bias4 + c0 / 4 + i);
+          bv[4 * i] = b4.x;
+          bv[4 * i + 1] = b4.y;
+          bv[4 * i + 2] = b4.z;
+          bv[4 * i + 3] = b4.w;
+        }
         REHYAT_TMEM_WAIT_LD32(r);
         float v[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const int f = c0 + i;
-          const float x = __uint_as_float(r[i]) + __ldg(bias + f);
+          const float x = __uint_as_float(r[i]) + bv[i];
           const int power = f / width + 1;  // the same for every lane
           float y = x;
           for (int e = 1; e < power; ++e) y *= x;
@@ -355,6 +399,8 @@ bool tc_phi_mlp_eligible(const PhiMlpArgs& a) {
   return a.in_bf16 && a.D == kD && a.Dh >= 128 && a.Dh % 128 == 0 && (a.Dp == 64 || a.Dp == 128) &&
          mlp::smem_bytes(a.Dh, a.Dp) <= mlp::kMaxSmem &&
          (reinterpret_cast<uintptr_t>(a.x) & 15) == 0 &&
+         (reinterpret_cast<uintptr_t>(a.ba) & 15) == 0 &&
+         (reinterpret_cast<uintptr_t>(a.bb) & 15) == 0 &&
          (reinterpret_cast<uintptr_t>(a.phi) & 15) == 0 && encode_fn() != nullptr;
 }
 

@@ -235,3 +235,27 @@ def test_feature_map_mlp_force_simt_and_fp32_take_cuda_cores():
     mlp = rh.RehyatPhiMlp(*(_cuda32(a).data_ptr() for a in params), 256, 2)
     assert rh.rehyat_feature_map_mlp_workspace_bytes(pf, mlp, dev["q"].data_ptr(),
                                                      got.data_ptr()) == 0
+
+
+def test_feature_map_mlp_tensor_cores_gelu_identity_weights():
+    """W_a = W_b = I (exact in bf16), one part: psi = bf16(GELU(x + b_a)) + b_b,
+    so the kernel's GELU is seen directly: within one bf16 rounding (2^-8
+    relative) of the exact GELU plus 1e-6 |u| for its erf approximation."""
+    B, H, T, Hs, Ws = 1, 2, 1, 16, 40
+    N = T * Hs * Ws
+    g = torch.Generator().manual_seed(11)
+    x = (torch.randn(B, H, N, 128, generator=g) * 3.0).to(torch.bfloat16)
+    eye = np.stack([np.eye(128)] * H)
+    rng = np.random.default_rng(12)
+    ba = rng.standard_normal((H, 128)) * 0.5
+    bb = rng.standard_normal((H, 128)) * 0.1
+    params = [a.astype(np.float32) for a in (eye, ba, eye, bb)]
+    got = _tc_map(x.cuda(), params, 1, T, Hs, Ws).double().cpu().numpy()
+    u = (x.double().numpy() + params[1].astype(np.float64)[None, :, None, :]).astype(np.float32)
+    u = u.astype(np.float64)
+    from scipy.special import erf
+    gl = 0.5 * u * (1.0 + erf(u / np.sqrt(2.0)))
+    err = np.abs(got - params[3].astype(np.float64)[None, :, None, :] - gl)
+    bar = 2.0 ** -8 * np.abs(gl) + 1e-6 * np.maximum(1.0, np.abs(u))
+    assert np.all(err <= bar), float((err - bar).max())
+    assert (u < -3).any() and (u > 3).any()

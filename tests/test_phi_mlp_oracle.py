@@ -118,3 +118,26 @@ def test_bf16_bound_covers_emulated_bf16_map(P):
     if P > 1:
         wrong_power = psi ** 2
         assert np.any(np.abs(wrong_power - ref) > bound)
+
+
+def test_tensor_core_gelu_constants_meet_published_bound():
+    """The erf approximation in the tensor-core feature map (Abramowitz &
+    Stegun 7.1.26) with the constants as written in its source reproduces
+    erf within the handbook's 1.5e-7, and Phi for negative arguments without
+    cancellation."""
+    import os
+    import re
+    from scipy.special import erf
+    src = open(os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                            "linear_attention_video_chunked_b200", "csrc",
+                            "tc_phi_mlp.cuh")).read()
+    c = {k: float(v) for k, v in re.findall(r"\b(kP|kA[1-5]) = (-?[0-9.]+)f", src)}
+    assert set(c) == {"kP", "kA1", "kA2", "kA3", "kA4", "kA5"}
+    x = np.linspace(0.0, 8.0, 20001)
+    t = 1.0 / (1.0 + c["kP"] * x)
+    q = t * (c["kA1"] + t * (c["kA2"] + t * (c["kA3"] + t * (c["kA4"] + t * c["kA5"])))) * \
+        np.exp(-x * x)
+    assert np.abs((1.0 - q) - erf(x)).max() <= 1.5e-7
+    # Phi(u) for u < 0 is q/2: absolute error stays <= 0.75e-7.
+    u = -x * np.sqrt(2.0)
+    assert np.abs(0.5 * q - 0.5 * (1.0 + erf(u / np.sqrt(2.0)))).max() <= 0.75e-7
