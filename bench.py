@@ -38,6 +38,7 @@ METRIC = "hybrid-attn fwd tokens/s & TFLOP/s (% BF16 tensor peak), 1 B200, 21x30
 L2_FLUSH_BYTES = 256 << 20
 KERNELS_PER_STEP = 4  # weight images, per-slice state, chunk scan, attention
 EXTRAS = ("full_softmax", "phi_backward", "general_phi", "streaming")
+E2E_HEADS_PER_SLAB = 2
 
 
 class L2Flush:
@@ -692,19 +693,22 @@ def run_gpu(args, world, rank, local):
     tokens_per_step = B * N
     value = job_throughput(world, tokens_per_step, args.steps, total_ms)
 
-    # End to end through the public API, host buffers in and out.
+    # End to end through the C ABI with host buffers: rehyat_hybrid_attn_fwd_host
+    # uploads q, k, v from pinned host memory and downloads y, slabs of two
+    # heads in flight on three streams; every copy is inside the timed region.
     qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
     yh = torch.empty(B, H, N, D, dtype=torch.float32).pin_memory()
-    qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    per_slab = E2E_HEADS_PER_SLAB
+    hws_bytes = rh.rehyat_host_workspace_bytes(params, per_slab)
+    hws = torch.empty(hws_bytes, dtype=torch.uint8, device=dev)
     e2e_steps = max(1, min(args.steps, 10))
 
     def e2e_step():
-        qd.copy_(qh, non_blocking=True)
-        kd.copy_(kh, non_blocking=True)
-        vd.copy_(vh, non_blocking=True)
-        rh.hybrid_attn(qd, kd, vd, Wq, bq, Wk, bk, T=T, Hs=p.Hs, Ws=p.Ws, Tc=p.Tc, To=p.To,
-                       causal=p.causal, out=y, workspace=ws)
-        yh.copy_(y, non_blocking=True)
+        st = rh.rehyat_hybrid_attn_fwd_host(params, qh.data_ptr(), kh.data_ptr(), vh.data_ptr(),
+                                            phi, yh.data_ptr(), per_slab, hws.data_ptr(),
+                                            hws_bytes, sh)
+        if st:
+            raise rh.RehyatError(st, "rehyat_hybrid_attn_fwd_host")
 
     e2e_step()
     torch.cuda.synchronize()
@@ -722,7 +726,7 @@ def run_gpu(args, world, rank, local):
     e2e_value = job_throughput(world, tokens_per_step, e2e_steps, e2e_ms)
     h2d = sum(x.numel() * x.element_size() for x in (qh, kh, vh))
     d2h = yh.numel() * yh.element_size()
-    del qh, kh, vh, yh, qd, kd, vd
+    del qh, kh, vh, yh, hws
 
     extra = {}
     want = set(EXTRAS if args.extras is None else args.extras.split(","))
@@ -783,7 +787,8 @@ def run_gpu(args, world, rank, local):
         "gpu_launches": KERNELS_PER_STEP * args.steps,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-                "api": "linear_attention_video_chunked_b200.hybrid_attn"},
+                "api": "rehyat_hybrid_attn_fwd_host (C ABI), pinned host q, k, v, y",
+                "heads_per_slab": E2E_HEADS_PER_SLAB},
         "clocks": clocks.summary(t_host0, t_host1),
     }
     line.update(extra)

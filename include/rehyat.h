@@ -221,6 +221,37 @@ REHYAT_API rehyat_status rehyat_hybrid_attn_fwd_phi(const rehyat_params* p, cons
                                                     void* y, void* workspace, size_t ws_bytes,
                                                     const rehyat_debug* dbg, void* stream);
 
+/* ---------------------------------------------------------------------- */
+/* Host-resident tensors.  The forward is per (batch, head) (Key designs
+ * 1-4: window softmax, linear state and joint normalisation never mix
+ * heads), so it can run in slabs of consecutive heads while the next slab's
+ * inputs are uploaded and the previous slab's output is downloaded.      */
+
+/* Device workspace bytes for rehyat_hybrid_attn_fwd_host with slabs of
+ * heads_per_slab heads (<= 0 or >= heads: one slab per batch element): three
+ * slots of q, k, v, y for one slab plus one slab's forward workspace
+ * (0 if p is invalid). */
+REHYAT_API size_t rehyat_host_workspace_bytes(const rehyat_params* p, int heads_per_slab);
+
+/* rehyat_hybrid_attn_fwd with q, k, v (p->in_dtype) and y (p->out_dtype) in
+ * HOST memory, same [B][h][N][D] layouts; phi and workspace on the device.
+ * Host buffers should be page-locked (cudaHostAlloc / cudaHostRegister):
+ * pageable memory still works but its copies do not overlap.  Slab s
+ * (batch s / G, heads (s mod G) * heads_per_slab ..., G groups of heads)
+ * goes through device slot s mod 3: upload on an internal copy stream, the
+ * forward on `stream`, download on a second internal copy stream, ordered
+ * by events.  The copies start after the work already on `stream`, and
+ * `stream` waits for the last download: synchronising `stream` makes y
+ * valid on the host.  The copy streams are created on first use per device
+ * and kept.  Results equal rehyat_hybrid_attn_fwd's bit for bit.  Errors as
+ * for rehyat_hybrid_attn_fwd; REHYAT_ERR_WORKSPACE if ws_bytes <
+ * rehyat_host_workspace_bytes; workspace 16-byte aligned. */
+REHYAT_API rehyat_status rehyat_hybrid_attn_fwd_host(const rehyat_params* p, const void* q,
+                                                     const void* k, const void* v,
+                                                     const rehyat_phi* phi, void* y,
+                                                     int heads_per_slab, void* workspace,
+                                                     size_t ws_bytes, void* stream);
+
 /* Per-head 2-layer MLP feature map, fp32 device arrays:
  *   Wa [heads][D][Dh], ba [heads][Dh], Wb [heads][Dh][Dp], bb [heads][Dp];
  *   psi = GELU(x Wa + ba) Wb + bb with GELU(u) = u * Phi(u) (exact form),

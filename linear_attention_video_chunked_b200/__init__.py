@@ -31,7 +31,8 @@ __all__ = [
     "rehyat_status_string", "rehyat_version", "rehyat_hybrid_attn_fwd_noalloc",
     "RehyatPhiGrad", "rehyat_phi_bwd_workspace_bytes", "rehyat_phi_bwd",
     "RehyatPhiMlp", "rehyat_hybrid_attn_fwd_phi", "rehyat_feature_map_mlp",
-    "rehyat_feature_map_mlp_workspace_bytes",
+    "rehyat_feature_map_mlp_workspace_bytes", "rehyat_host_workspace_bytes",
+    "rehyat_hybrid_attn_fwd_host", "hybrid_attn_host",
     "make_params", "hybrid_attn", "hybrid_attn_phi", "feature_map_mlp", "softmax_attn",
     "phi_grad", "StreamingState",
 ]
@@ -51,7 +52,8 @@ EXPORTED_SYMBOLS = (
     "rehyat_attn_path", "rehyat_status_string", "rehyat_version",
     "rehyat_hybrid_attn_fwd_noalloc", "rehyat_phi_bwd_workspace_bytes", "rehyat_phi_bwd",
     "rehyat_hybrid_attn_fwd_phi", "rehyat_feature_map_mlp",
-    "rehyat_feature_map_mlp_workspace_bytes",
+    "rehyat_feature_map_mlp_workspace_bytes", "rehyat_host_workspace_bytes",
+    "rehyat_hybrid_attn_fwd_host",
 )
 
 
@@ -158,6 +160,11 @@ def lib() -> ctypes.CDLL:
         L.rehyat_feature_map_mlp_workspace_bytes.argtypes = [P(RehyatParams), P(RehyatPhiMlp),
                                                              vp, vp]
         L.rehyat_feature_map_mlp_workspace_bytes.restype = ctypes.c_size_t
+        L.rehyat_host_workspace_bytes.argtypes = [P(RehyatParams), i]
+        L.rehyat_host_workspace_bytes.restype = ctypes.c_size_t
+        L.rehyat_hybrid_attn_fwd_host.argtypes = [P(RehyatParams), vp, vp, vp, P(RehyatPhi), vp,
+                                                  i, vp, ctypes.c_size_t, vp]
+        L.rehyat_hybrid_attn_fwd_host.restype = i
         _LIB = L
     return _LIB
 
@@ -205,6 +212,16 @@ def rehyat_hybrid_attn_fwd_phi(p, q, k, v, phi_q, phi_k, y, workspace, ws_bytes,
     return lib().rehyat_hybrid_attn_fwd_phi(ctypes.byref(p), q, k, v, phi_q, phi_k, y, workspace,
                                             ws_bytes, None if dbg is None else ctypes.byref(dbg),
                                             stream)
+
+
+def rehyat_host_workspace_bytes(p, heads_per_slab) -> int:
+    return lib().rehyat_host_workspace_bytes(ctypes.byref(p), heads_per_slab)
+
+
+def rehyat_hybrid_attn_fwd_host(p, q, k, v, phi, y, heads_per_slab, workspace, ws_bytes,
+                                stream) -> int:
+    return lib().rehyat_hybrid_attn_fwd_host(ctypes.byref(p), q, k, v, ctypes.byref(phi), y,
+                                             heads_per_slab, workspace, ws_bytes, stream)
 
 
 def rehyat_feature_map_mlp_workspace_bytes(p, mlp, x, phi) -> int:
@@ -340,6 +357,33 @@ def hybrid_attn(q, k, v, Wq, bq, Wk, bk, *, T, Hs, Ws, Tc, To, causal, out_dtype
                                 _stream_handle(stream))
     _check(st, "rehyat_hybrid_attn_fwd")
     return (y, dbg_t) if debug else y
+
+
+def hybrid_attn_host(q, k, v, Wq, bq, Wk, bk, *, T, Hs, Ws, Tc, To, causal, out=None,
+                     heads_per_slab=2, workspace=None, stream=None):
+    """hybrid_attn on CPU tensors q, k, v [B, h, N, D] (pin them for overlap):
+    slabs of heads are uploaded, computed and downloaded concurrently by
+    rehyat_hybrid_attn_fwd_host; the phi parameters are CUDA tensors.
+    Returns y (fp32, CPU; `out` if given), valid after `stream` syncs (this
+    function synchronises it)."""
+    torch = _torch()
+    B, H, N, D = q.shape
+    Dp = 2 * Wq.shape[-1]
+    p = make_params(batch=B, heads=H, T=T, Hs=Hs, Ws=Ws, D=D, Dp=Dp, Tc=Tc, To=To,
+                    causal=causal, in_dtype=_dtype_code(q.dtype), out_dtype=F32)
+    y = torch.empty(B, H, N, D, dtype=torch.float32, pin_memory=True) if out is None else out
+    nbytes = rehyat_host_workspace_bytes(p, heads_per_slab)
+    if nbytes == 0:
+        raise RehyatError(1, "rehyat_host_workspace_bytes")
+    if workspace is None or workspace.numel() < nbytes:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=Wq.device)
+    st = rehyat_hybrid_attn_fwd_host(p, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                     _phi_struct(Wq, bq, Wk, bk), y.data_ptr(), heads_per_slab,
+                                     workspace.data_ptr(), workspace.numel(),
+                                     _stream_handle(stream))
+    _check(st, "rehyat_hybrid_attn_fwd_host")
+    (stream or torch.cuda.current_stream()).synchronize()
+    return y
 
 
 def feature_map_mlp(x, Wa, ba, Wb, bb, *, parts, T, Hs, Ws, stream=None, force_simt=False,

@@ -527,6 +527,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // half over S columns [0,32), of the high half over [64,96).
 // ===========================================================================
 namespace a2 {
+// 18 warps: two of the four sub-partitions hold five warps, and each has
+// 16,384 registers, so a thread gets at most 96 (the launch bound below).
 constexpr int kThreads = 576;
 constexpr int kProducerWarp = 16, kMmaWarp = 17;
 constexpr int kHalfThreads = 128;  // one half of a tile's softmax threads
@@ -563,7 +565,7 @@ constexpr uint32_t kXchgOff = kVecOff + 512;
 constexpr uint32_t kSmemBytes = kXchgOff + 1024 + 1024;
 }  // namespace a2
 
-__global__ void __maxnreg__(112)
+__global__ void __launch_bounds__(a2::kThreads, 1)
     tc_attn2_kernel(const __grid_constant__ TcMaps maps, const AttnParams P,
                     const __nv_bfloat16* __restrict__ wq_img) {
   using a2::kQOff;
