@@ -517,21 +517,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 // phi_q(q) by 1/f (f = exp2(m_used - m_max) <= 1) and accumulates into O, so
 // y = f*O / (f*n^S + n^L).
 //
-// Roles (576 threads): every query row is shared by two warps of the same
-// TMEM lane quadrant, one per half of the 128 key columns.  Warps 0-3 (tile
-// A) and 4-7 (tile B) take key columns 0-63 and run the epilogue; warps 8-11
-// (A) and 12-15 (B) take columns 64-127; the two halves exchange their
-// partial row maxima through shared memory each step.  Warp 16 TMA, warp 17
-// MMA and TMEM owner.
-// TMEM: S_A [0,128) O_A [128,256) S_B [256,384) O_B [384,512); P of the low
-// half over S columns [0,32), of the high half over [64,96).
+// Roles (320 threads): warps 0-3 softmax + epilogue of tile A, warps 4-7 of
+// tile B, warp 8 TMA, warp 9 MMA and TMEM owner.
+// TMEM: S_A [0,128) O_A [128,256) S_B [256,384) O_B [384,512).
 // ===========================================================================
 namespace a2 {
-// 18 warps: two of the four sub-partitions hold five warps, and each has
-// 16,384 registers, so a thread gets at most 96 (the launch bound below).
-constexpr int kThreads = 576;
-constexpr int kProducerWarp = 16, kMmaWarp = 17;
-constexpr int kHalfThreads = 128;  // one half of a tile's softmax threads
+constexpr int kThreads = 320;
 // One fp32 pair in kPolyEvery takes the FMA-pipe exp2 (0 = all on MUFU).
 // Measured on the 21x30x52 workload (attention ms): all on MUFU 2.85,
 // one in 8 pairs 2.97, one in 4 3.01, one in 2 3.05 -- the softmax is
@@ -554,15 +545,12 @@ constexpr uint32_t kPhiOff0 = kVOff;               // tail: phi_q(Q_A)/f (<= 64 
 constexpr uint32_t kPhiOff1 = kQOff;               // tail: phi_q(Q_B)/f, over Q (<= 64 KB)
 enum { Q_FULL = 0, K_FULL = 1, K_EMPTY = 4, V_FULL = 7, V_EMPTY = 9, S_FULL = 11, P_FULL = 13,
        PV_DONE = 15, LAST_PV = 17, TAIL_FULL = 18, PHI_DONE = 19, PHI_READY = 20, READ_DONE = 22,
-       VEC_READY = 23, XA = 24, XB = 26, NBAR = 28 };
+       VEC_READY = 23, NBAR = 24 };
 constexpr uint32_t kTmemSlot = kBarOff + 8 * NBAR;
 constexpr uint32_t kAbortSlot = kTmemSlot + 4;
-// z^L of the chunk (D' floats), shared by both tiles.
+// b_q of the head and z^L of the chunk (D' floats each), shared by both tiles.
 constexpr uint32_t kVecOff = kBarOff + 256;
-// Per tile and row, the slot through which the two halves of a row trade
-// their partial maxima (and, after the loop, the high half's row sum).
-constexpr uint32_t kXchgOff = kVecOff + 512;
-constexpr uint32_t kSmemBytes = kXchgOff + 1024 + 1024;
+constexpr uint32_t kSmemBytes = kVecOff + 1024 + 1024;
 }  // namespace a2
 
 __global__ void __launch_bounds__(a2::kThreads, 1)
@@ -646,15 +634,14 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
 
   if (tid == 0) {
     for (int i = 0; i < a2::NBAR; ++i) {
-      const bool by_half = i == a2::PHI_READY || i == a2::PHI_READY + 1 || i == a2::VEC_READY ||
-                           i == a2::XA || i == a2::XA + 1 || i == a2::XB || i == a2::XB + 1;
-      const bool by_tile = i == a2::P_FULL || i == a2::P_FULL + 1;
-      mbar_init(bar(i), by_tile ? 2 * a2::kHalfThreads : by_half ? a2::kHalfThreads : 1);
+      const bool by_warpgroup = i == a2::P_FULL || i == a2::P_FULL + 1 || i == a2::PHI_READY ||
+                                i == a2::PHI_READY + 1 || i == a2::VEC_READY;
+      mbar_init(bar(i), by_warpgroup ? kSoftmaxThreads : 1);
     }
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == a2::kMmaWarp) {
+  if (warp == 9) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      base + kTmemSlot),
                  "r"(512));
@@ -665,7 +652,7 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sbase + kTmemSlot);
 
-  if (warp == a2::kProducerWarp) {
+  if (warp == 8) {
     // ================================================= TMA producer
     if (lane == 0) {
       bool ok = true;
@@ -711,7 +698,7 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == a2::kMmaWarp) {
+  } else if (warp == 9) {
     // ================================================= MMA issuer
     if (lane == 0) {
       const uint32_t id_qk = idesc(kBM, kBN, 1, false);
@@ -731,11 +718,9 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
       };
       auto issue_pv = [&](int tile, int j) {
         const uint32_t vaddr = base + kVOff + (j & 1) * 32768;
-        // Keys 16 kk..: the low half's P at columns 8 kk, the high half's
-        // (kk >= 4) at 64 + 8 (kk - 4).
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts(tmem + tile * 256 + 128, tmem + tile * 256 + kk * 8 + (kk >= 4 ? 32 : 0),
+          mma_bf16_ts(tmem + tile * 256 + 128, tmem + tile * 256 + kk * 8,
                       sdesc(vaddr + kk * 2048, 16384, 1024), id_pv, (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit(bar(a2::PV_DONE + tile));
       };
@@ -796,26 +781,26 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp < 16 && ((warp & 4) == 0 || has_b)) {
+  } else if (warp < 8 && (warp < 4 || has_b)) {
     // ================================================= softmax / epilogue
-    const int tile = (warp >> 2) & 1;
-    const int half = warp >> 3;               // key columns 64 half .. 64 half + 63
-    const int r = tid & 127;                  // row within the tile == TMEM lane
+    const int tile = warp >> 2;
+    const int r = tid & 127;                 // row within the tile == TMEM lane
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const uint32_t s_col = tile * 256, o_col = s_col + 128;
-    const uint32_t h_col = s_col + half * 64;  // this half's S columns, then its P
     const int nrows = nrows_t[tile];
     float m_used = -INFINITY, m_max = -INFINITY, l = 0.f;
     bool ok = true;
     auto wait_all = [&](uint32_t b, uint32_t parity, uint32_t code) {
       return __all_sync(0xffffffffu, mbar_wait(b, parity, abort_flag, code));
     };
-    float* vec = reinterpret_cast<float*>(sbase + a2::kVecOff);  // z^L (D')
-    volatile float* xchg = reinterpret_cast<volatile float*>(sbase + a2::kXchgOff) + tile * 128 + r;
-    if (linear && tile == 0 && half == 0) {
-      // Tile A's low half stages z^L for the tail while it waits for its
-      // first scores.
-      if (r < Dp) vec[r] = __ldg(P.zL + (static_cast<long long>(bh) * P.nchunks + t) * Dp + r);
+    float* vec = reinterpret_cast<float*>(sbase + a2::kVecOff);  // [b_q (D') | z^L (D')]
+    if (linear && tile == 0) {
+      // Tile A's warpgroup stages b_q and z^L for the tail while it waits
+      // for the first scores (b_q of head h is h's D' consecutive values).
+      if (r < Dp) {
+        vec[r] = phi_given ? 0.f : __ldg(P.bq + h * Dp + r);
+        vec[Dp + r] = __ldg(P.zL + (static_cast<long long>(bh) * P.nchunks + t) * Dp + r);
+      }
       mbar_arrive(bar(a2::VEC_READY));
     }
     for (int j = 0; j < nt && ok; ++j) {
@@ -825,10 +810,11 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
       tc_fence_after();
       const int nvalid = tile_src(j).nvalid;
       const bool ragged = nvalid < kBN;  // warp-uniform: keys past the end
-      // This half's 64 columns of S are streamed from TMEM 32 at a time
-      // through two register buffers (the next load in flight).
+      // S is streamed from TMEM 32 columns at a time through two register
+      // buffers: the next load is in flight while the current chunk is used
+      // (S never sits whole in registers, which would spill).
       uint32_t xa[32], xb[32];
-      auto mask = [&](uint32_t* x, int c) {  // c: key chunk 0..3 of the tile
+      auto mask = [&](uint32_t* x, int c) {
         if (ragged) {
 #pragma unroll
           for (int i = 0; i < 32; ++i)
@@ -845,33 +831,27 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
                                      __uint_as_float(x[i + 16])),
                         __uint_as_float(x[i + 24]));
       };
-      // Pass 1: partial row max over this half.
-      REHYAT_TMEM_LD32(lane_base + h_col, xa);
+      // Pass 1: row max.
+      REHYAT_TMEM_LD32(lane_base + s_col, xa);
       REHYAT_TMEM_WAIT_LD32(xa);
-      REHYAT_TMEM_LD32(lane_base + h_col + 32, xb);
-      mask(xa, 2 * half);
+      REHYAT_TMEM_LD32(lane_base + s_col + 32, xb);
+      mask(xa, 0);
       max_chunk(xa);
       REHYAT_TMEM_WAIT_LD32(xb);
-      REHYAT_TMEM_LD32(lane_base + h_col, xa);  // pass 2, chunk 0
-      mask(xb, 2 * half + 1);
+      REHYAT_TMEM_LD32(lane_base + s_col + 64, xa);
+      mask(xb, 1);
       max_chunk(xb);
-      float pm = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
-                       fmaxf(mx[6], mx[7]));
-      // Row max of both halves: the high half posts its value, the low half
-      // combines and posts the result (one slot per row, bounded waits).
-      if (half == 1) {
-        *xchg = pm;
-        mbar_arrive(bar(a2::XA + tile));
-        ok = wait_all(bar(a2::XB + tile), j & 1, 16);
-        pm = *xchg;
-      } else {
-        ok = wait_all(bar(a2::XA + tile), j & 1, 17);
-        pm = fmaxf(pm, *xchg);
-        *xchg = pm;
-        mbar_arrive(bar(a2::XB + tile));
-      }
-      if (!ok) break;
-      m_max = fmaxf(m_max, pm * P.scale_log2);
+      REHYAT_TMEM_WAIT_LD32(xa);
+      REHYAT_TMEM_LD32(lane_base + s_col + 96, xb);
+      mask(xa, 2);
+      max_chunk(xa);
+      REHYAT_TMEM_WAIT_LD32(xb);
+      REHYAT_TMEM_LD32(lane_base + s_col, xa);  // pass 2, chunk 0
+      mask(xb, 3);
+      max_chunk(xb);
+      m_max = fmaxf(m_max, fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
+                                 fmaxf(mx[6], mx[7])) *
+                               P.scale_log2);
       float alpha = 1.f;
       const bool rescale = m_max > m_used + 8.f;
       if (rescale) {
@@ -880,15 +860,14 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
       }
       // p = 2^(s * scale * log2(e) - m_used) on packed fp32 pairs; one pair
       // in kPolyEvery goes through the FMA-pipe exp2 (exp2_poly2) instead of
-      // MUFU.
+      // MUFU, which at D = 128 is as busy as the tensor core.
       const uint64_t scale2 = f2_pack(P.scale_log2, P.scale_log2);
       const uint64_t negm2 = f2_pack(-m_used, -m_used);
       uint64_t ls2[4] = {0, 0, 0, 0};
-      // Pass 2: P (bf16 pairs) of chunk c is written over this half's S
-      // columns already consumed, [16c, 16c + 16) of them, while chunk c + 1
-      // is being loaded.
+      // Pass 2: P (bf16 pairs) of chunk c is written over S columns already
+      // consumed, [16c, 16c + 16), while chunk c + 1 is being loaded.
       auto exp_chunk = [&](uint32_t* x, int c) {
-        mask(x, 2 * half + c);
+        mask(x, c);
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -906,6 +885,9 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
           float p0, p1;
           f2_unpack(p2, p0, p1);
           if (kTruncP) {
+            // bf16 by truncation (one byte permute on the ALU pipe instead of
+            // a conversion on the pipe that also runs ex2); the row sum takes
+            // the same truncated values, so P.V and l stay consistent.
             const uint32_t u0 = __float_as_uint(p0), u1 = __float_as_uint(p1);
             pk[i] = __byte_perm(u0, u1, 0x7632);
             ls2[i & 3] = f2_add(ls2[i & 3], f2_pack(__uint_as_float(u0 & 0xFFFF0000u),
@@ -915,35 +897,40 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
             ls2[i & 3] = f2_add(ls2[i & 3], p2);
           }
         }
-        REHYAT_TMEM_ST16(lane_base + h_col + c * 16, pk);
+        REHYAT_TMEM_ST16(lane_base + s_col + c * 16, pk);
       };
       REHYAT_TMEM_WAIT_LD32(xa);
-      REHYAT_TMEM_LD32(lane_base + h_col + 32, xb);
+      REHYAT_TMEM_LD32(lane_base + s_col + 32, xb);
       exp_chunk(xa, 0);
       REHYAT_TMEM_WAIT_LD32(xb);
+      REHYAT_TMEM_LD32(lane_base + s_col + 64, xa);
       exp_chunk(xb, 1);
-      float ls[4];
+      REHYAT_TMEM_WAIT_LD32(xa);
+      REHYAT_TMEM_LD32(lane_base + s_col + 96, xb);
+      exp_chunk(xa, 2);
+      REHYAT_TMEM_WAIT_LD32(xb);
+      exp_chunk(xb, 3);
+      float ls[8];
       f2_unpack(f2_add(ls2[0], ls2[1]), ls[0], ls[1]);
       f2_unpack(f2_add(ls2[2], ls2[3]), ls[2], ls[3]);
-      // After the P stores (S is dead by now): bring this half's 64 columns
-      // of the earlier a^S to the new reference point; this tile's P.V of
-      // step j-1 is complete (covered by S_FULL(j)).  Warp-collective; rows
-      // that did not move use alpha = 1.
+      ls[4] = ls[5] = ls[6] = ls[7] = 0.f;
+      // After the P stores (S is dead by now): bring the earlier a^S to the
+      // new reference point; this tile's P.V of step j-1 is complete (covered
+      // by S_FULL(j)).  Warp-collective; rows that did not move use alpha = 1.
       if (j > 0 && __any_sync(0xffffffffu, rescale)) {
         uint32_t o[32];
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const uint32_t oc = lane_base + o_col + half * 64 + c * 32;
-          REHYAT_TMEM_LD32(oc, o);
+        for (int c = 0; c < 4; ++c) {
+          REHYAT_TMEM_LD32(lane_base + o_col + c * 32, o);
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          REHYAT_TMEM_ST32(oc, o);
+          REHYAT_TMEM_ST32(lane_base + o_col + c * 32, o);
         }
       }
       tmem_wait_st();
-      l = l * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
-      if (tile == 0 && half == 0 && nvalid < kBN) {
+      l = l * alpha + (((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7])));
+      if (tile == 0 && nvalid < kBN) {
         // Zero the V rows past the last valid key (shared by both tiles;
         // tile B's P.V is issued after tile A's P_FULL).
         ok = wait_all(bar(a2::V_FULL + (j & 1)), (j >> 1) & 1, 13);
@@ -961,170 +948,157 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
       tc_fence_before();
       mbar_arrive(bar(a2::P_FULL + tile));
     }
-    // The row sum of the high half joins the low half's, through the same
-    // slot (phase nt of XA); the high half's work ends here.
-    if (half == 1) {
-      if (ok) {
-        *xchg = l;
-        mbar_arrive(bar(a2::XA + tile));
-      }
-    } else {
-      if (ok) {
-        ok = wait_all(bar(a2::XA + tile), nt & 1, 18);
-        if (ok) l += *xchg;
-      }
-      const float fscale = ex2(m_used - m_max);
-      const long long grow = static_cast<long long>(bh) * P.rows_per_bh + row0 + tile * kBM + r;
-      const bool dbg_split = P.dbg_aS != nullptr || P.dbg_aL != nullptr;
-      float nL = 0.f;
-      if (ok && linear) {
-        if (dbg_split) {
-          // a^S before the readout adds into O (debug export only).
-          ok = wait_all(bar(a2::LAST_PV), 0, 14);
-          if (ok) {
-            tc_fence_after();
-            for (int c = 0; c < 4; ++c) {
-              uint32_t o[32];
-              REHYAT_TMEM_LD32(lane_base + o_col + c * 32, o);
-              tmem_wait_ld();
-              if (r < nrows && P.dbg_aS)
-                for (int i = 0; i < 32; ++i)
-                  P.dbg_aS[grow * kD + c * 32 + i] = __uint_as_float(o[i]) * fscale;
-              if (r < nrows && P.dbg_aL)  // a^S for now; replaced by a^L below
-                for (int i = 0; i < 32; ++i)
-                  P.dbg_aL[grow * kD + c * 32 + i] = __uint_as_float(o[i]) * fscale;
-            }
-          }
-        }
-        // phi_q(q) is staged into the V ring (tile A) and over Q (tile B):
-        // with the closed form that waits for the phi MMAs (which read Q);
-        // with phi_q given, for the last P.V (every MMA of the loop is done).
-        if (ok) ok = wait_all(bar(a2::VEC_READY), 0, 14) &&
-                     wait_all(bar(phi_given ? a2::LAST_PV : a2::PHI_DONE), 0, 14);
+    const float fscale = ex2(m_used - m_max);
+    const long long grow = static_cast<long long>(bh) * P.rows_per_bh + row0 + tile * kBM + r;
+    const bool dbg_split = P.dbg_aS != nullptr || P.dbg_aL != nullptr;
+    float nL = 0.f;
+    if (ok && linear) {
+      if (dbg_split) {
+        // a^S before the readout adds into O (debug export only).
+        ok = wait_all(bar(a2::LAST_PV), 0, 14);
         if (ok) {
           tc_fence_after();
-          const float inv_f = 1.0f / fscale;
-          const uint32_t phi = base + (tile ? kPhiOff1 : kPhiOff0);
-          const float* given = phi_given && r < nrows ? P.phi_q + grow * Dp : nullptr;
-          for (int c = 0; c < Dp / 32; ++c) {
-            float ph[32];
-            if (phi_given) {
-  #pragma unroll
-              for (int i = 0; i < 32; i += 4) {
-                const float4 g4 = given ? __ldg(reinterpret_cast<const float4*>(given + c * 32 + i))
-                                        : make_float4(0.f, 0.f, 0.f, 0.f);
-                ph[i] = g4.x;
-                ph[i + 1] = g4.y;
-                ph[i + 2] = g4.z;
-                ph[i + 3] = g4.w;
-              }
-            } else {
-              uint32_t v[32];
-              REHYAT_TMEM_LD32(lane_base + s_col + c * 32, v);
-              tmem_wait_ld();
-  #pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const float psi = __uint_as_float(v[i]) + __ldg(P.bq + h * Dp + c * 32 + i);
-                ph[i] = psi * psi;
-              }
-            }
-  #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              nL = fmaf(ph[i], vec[c * 32 + i], nL);
-              ph[i] *= inv_f;
-            }
-            const uint32_t rowaddr = phi + c * 16384 + r * 128;
-  #pragma unroll
-            for (int ch = 0; ch < 8; ++ch)
-              st_shared_v4(rowaddr + ((ch ^ (r & 7)) << 4), __float_as_uint(ph[4 * ch]),
-                           __float_as_uint(ph[4 * ch + 1]), __float_as_uint(ph[4 * ch + 2]),
-                           __float_as_uint(ph[4 * ch + 3]));
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            REHYAT_TMEM_LD32(lane_base + o_col + c * 32, o);
+            tmem_wait_ld();
+            if (r < nrows && P.dbg_aS)
+              for (int i = 0; i < 32; ++i)
+                P.dbg_aS[grow * kD + c * 32 + i] = __uint_as_float(o[i]) * fscale;
+            if (r < nrows && P.dbg_aL)  // a^S for now; replaced by a^L below
+              for (int i = 0; i < 32; ++i)
+                P.dbg_aL[grow * kD + c * 32 + i] = __uint_as_float(o[i]) * fscale;
           }
-          fence_proxy_async();
-          tc_fence_before();
-          mbar_arrive(bar(a2::PHI_READY + tile));
-          ok = wait_all(bar(a2::READ_DONE), 0, 15);
         }
-      } else if (ok) {
-        ok = wait_all(bar(a2::LAST_PV), 0, 15);
       }
+      // phi_q(q) is staged into the V ring (tile A) and over Q (tile B):
+      // with the closed form that waits for the phi MMAs (which read Q);
+      // with phi_q given, for the last P.V (every MMA of the loop is done).
+      if (ok) ok = wait_all(bar(a2::VEC_READY), 0, 14) &&
+                   wait_all(bar(phi_given ? a2::LAST_PV : a2::PHI_DONE), 0, 14);
       if (ok) {
         tc_fence_after();
-        const float nS = l * fscale;
-        const float den = nS + nL;
-        // y = f * O / den: one IEEE division per row, then a product per value.
-        const float ysc = __fdiv_rn(fscale, den);
-        const bool dbg_num = P.dbg_aL != nullptr || (P.dbg_aS != nullptr && !linear);
-        for (int c = 0; c < 4; ++c) {
-          uint32_t o[32];
-          REHYAT_TMEM_LD32(lane_base + o_col + c * 32, o);
-          tmem_wait_ld();
-          if (r < nrows) {
-            float yv[32];
-  #pragma unroll
-            for (int i = 0; i < 32; ++i) yv[i] = __uint_as_float(o[i]) * ysc;
-            if (dbg_num) {
-              for (int i = 0; i < 32; ++i) {
-                const float num = __uint_as_float(o[i]) * fscale;  // a^S + a^L
-                if (P.dbg_aL) {
-                  float* d = P.dbg_aL + grow * kD + c * 32 + i;
-                  *d = linear ? num - *d : 0.f;
-                }
-                if (P.dbg_aS && !linear) P.dbg_aS[grow * kD + c * 32 + i] = num;
-              }
+        const float inv_f = 1.0f / fscale;
+        const uint32_t phi = base + (tile ? kPhiOff1 : kPhiOff0);
+        const float* given = phi_given && r < nrows ? P.phi_q + grow * Dp : nullptr;
+        for (int c = 0; c < Dp / 32; ++c) {
+          float ph[32];
+          if (phi_given) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              const float4 g4 = given ? __ldg(reinterpret_cast<const float4*>(given + c * 32 + i))
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+              ph[i] = g4.x;
+              ph[i + 1] = g4.y;
+              ph[i + 2] = g4.z;
+              ph[i + 3] = g4.w;
             }
-            if (P.out_bf16) {
-              uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(P.y) + grow * kD +
-                                                    c * 32);
-  #pragma unroll
-              for (int i = 0; i < 4; ++i)
-                dst[i] = make_uint4(pack_bf16(yv[8 * i], yv[8 * i + 1]),
-                                    pack_bf16(yv[8 * i + 2], yv[8 * i + 3]),
-                                    pack_bf16(yv[8 * i + 4], yv[8 * i + 5]),
-                                    pack_bf16(yv[8 * i + 6], yv[8 * i + 7]));
-            } else {
-              // fp32 rows go through shared memory (the K ring is free now:
-              // tile A at kKOff, tile B 64 KB above), 16-byte chunk cc of row
-              // r at position cc ^ (r & 7) so neither side has bank conflicts.
-              const uint32_t srow = base + kKOff + tile * 65536 + r * 512;
-  #pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const uint32_t cc = c * 8 + i;
-                st_shared_v4(srow + ((cc ^ (r & 7)) << 4), __float_as_uint(yv[4 * i]),
-                             __float_as_uint(yv[4 * i + 1]), __float_as_uint(yv[4 * i + 2]),
-                             __float_as_uint(yv[4 * i + 3]));
+          } else {
+            uint32_t v[32];
+            REHYAT_TMEM_LD32(lane_base + s_col + c * 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float psi = __uint_as_float(v[i]) + vec[c * 32 + i];
+              ph[i] = psi * psi;
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            nL = fmaf(ph[i], vec[Dp + c * 32 + i], nL);
+            ph[i] *= inv_f;
+          }
+          const uint32_t rowaddr = phi + c * 16384 + r * 128;
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch)
+            st_shared_v4(rowaddr + ((ch ^ (r & 7)) << 4), __float_as_uint(ph[4 * ch]),
+                         __float_as_uint(ph[4 * ch + 1]), __float_as_uint(ph[4 * ch + 2]),
+                         __float_as_uint(ph[4 * ch + 3]));
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        mbar_arrive(bar(a2::PHI_READY + tile));
+        ok = wait_all(bar(a2::READ_DONE), 0, 15);
+      }
+    } else if (ok) {
+      ok = wait_all(bar(a2::LAST_PV), 0, 15);
+    }
+    if (ok) {
+      tc_fence_after();
+      const float nS = l * fscale;
+      const float den = nS + nL;
+      // y = f * O / den: one IEEE division per row, then a product per value.
+      const float ysc = __fdiv_rn(fscale, den);
+      const bool dbg_num = P.dbg_aL != nullptr || (P.dbg_aS != nullptr && !linear);
+      for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        REHYAT_TMEM_LD32(lane_base + o_col + c * 32, o);
+        tmem_wait_ld();
+        if (r < nrows) {
+          float yv[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) yv[i] = __uint_as_float(o[i]) * ysc;
+          if (dbg_num) {
+            for (int i = 0; i < 32; ++i) {
+              const float num = __uint_as_float(o[i]) * fscale;  // a^S + a^L
+              if (P.dbg_aL) {
+                float* d = P.dbg_aL + grow * kD + c * 32 + i;
+                *d = linear ? num - *d : 0.f;
               }
+              if (P.dbg_aS && !linear) P.dbg_aS[grow * kD + c * 32 + i] = num;
+            }
+          }
+          if (P.out_bf16) {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(P.y) + grow * kD +
+                                                  c * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_uint4(pack_bf16(yv[8 * i], yv[8 * i + 1]),
+                                  pack_bf16(yv[8 * i + 2], yv[8 * i + 3]),
+                                  pack_bf16(yv[8 * i + 4], yv[8 * i + 5]),
+                                  pack_bf16(yv[8 * i + 6], yv[8 * i + 7]));
+          } else {
+            // fp32 rows go through shared memory (the K ring is free now:
+            // tile A at kKOff, tile B 64 KB above), 16-byte chunk cc of row
+            // r at position cc ^ (r & 7) so neither side has bank conflicts.
+            const uint32_t srow = base + kKOff + tile * 65536 + r * 512;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const uint32_t cc = c * 8 + i;
+              st_shared_v4(srow + ((cc ^ (r & 7)) << 4), __float_as_uint(yv[4 * i]),
+                           __float_as_uint(yv[4 * i + 1]), __float_as_uint(yv[4 * i + 2]),
+                           __float_as_uint(yv[4 * i + 3]));
             }
           }
         }
-        if (r < nrows) {
-          if (P.dbg_nS) P.dbg_nS[grow] = nS;
-          if (P.dbg_nL) P.dbg_nL[grow] = nL;
-          if (P.dbg_c) P.dbg_c[grow] = m_max * 0.69314718055994530942f;
-        }
       }
-      // Every thread of this warpgroup gets here (aborted or not), so the
-      // named barrier cannot hang.  Then each warp writes whole 512-byte rows
-      // of the staged fp32 output: lane l stores chunk l (coalesced).
-      asm volatile("bar.sync %0, %1;" ::"r"(1 + tile), "r"(kSoftmaxThreads) : "memory");
-      if (ok && !P.out_bf16) {
-        const long long grow0 = static_cast<long long>(bh) * P.rows_per_bh + row0 + tile * kBM;
-        for (int rr = warp & 3; rr < nrows; rr += 4) {
-          const uint32_t src = base + kKOff + tile * 65536 + rr * 512 + ((lane ^ (rr & 7)) << 4);
-          uint32_t a0, a1, a2, a3;
-          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                       : "=r"(a0), "=r"(a1), "=r"(a2), "=r"(a3)
-                       : "r"(src));
-          reinterpret_cast<uint4*>(static_cast<float*>(P.y) + (grow0 + rr) * kD)[lane] =
-              make_uint4(a0, a1, a2, a3);
-        }
+      if (r < nrows) {
+        if (P.dbg_nS) P.dbg_nS[grow] = nS;
+        if (P.dbg_nL) P.dbg_nL[grow] = nL;
+        if (P.dbg_c) P.dbg_c[grow] = m_max * 0.69314718055994530942f;
+      }
+    }
+    // Every thread of this warpgroup gets here (aborted or not), so the
+    // named barrier cannot hang.  Then each warp writes whole 512-byte rows
+    // of the staged fp32 output: lane l stores chunk l (coalesced).
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + tile), "r"(kSoftmaxThreads) : "memory");
+    if (ok && !P.out_bf16) {
+      const long long grow0 = static_cast<long long>(bh) * P.rows_per_bh + row0 + tile * kBM;
+      for (int rr = warp & 3; rr < nrows; rr += 4) {
+        const uint32_t src = base + kKOff + tile * 65536 + rr * 512 + ((lane ^ (rr & 7)) << 4);
+        uint32_t a0, a1, a2, a3;
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(a0), "=r"(a1), "=r"(a2), "=r"(a3)
+                     : "r"(src));
+        reinterpret_cast<uint4*>(static_cast<float*>(P.y) + (grow0 + rr) * kD)[lane] =
+            make_uint4(a0, a1, a2, a3);
       }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == a2::kMmaWarp) {
+  if (warp == 9) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
   }
