@@ -276,7 +276,7 @@ REHYAT_API size_t rehyat_feature_map_mlp_workspace_bytes(const rehyat_params* p,
  * the size above is 0) of at least rehyat_feature_map_mlp_workspace_bytes
  * bytes.  Tensor-core path: x, W_a, GELU(.) and W_b enter the products as
  * bf16 (fp32 accumulation, b_a, b_b and the powers in fp32; erf inside GELU
- * from Abramowitz & Stegun 7.1.26, |error| <= 1.5e-7); CUDA-core path: fp32
+ * from Abramowitz & Stegun 7.1.28, |error| <= 3e-7); CUDA-core path: fp32
  * throughout (erff).  REHYAT_ERR_INVALID_ARG for parts < 1 or Dp % parts != 0;
  * REHYAT_ERR_WORKSPACE if ws_bytes is too small. */
 REHYAT_API rehyat_status rehyat_feature_map_mlp(const rehyat_params* p, const void* x,

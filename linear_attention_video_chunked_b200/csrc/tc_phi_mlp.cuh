@@ -75,28 +75,78 @@ __device__ __forceinline__ Tile tile_of(int it, int batch, int ntile) {
 }
 
 // GELU(u) = u Phi(u) with Phi(u) = (1 + erf(u / sqrt 2)) / 2 and erf from
-// Abramowitz & Stegun, Handbook of Mathematical Functions, 7.1.26 (after
-// Hastings): for x >= 0, erf(x) = 1 - q(x) with q = t (a1 + t (a2 + t (a3 +
-// t (a4 + t a5)))) exp(-x^2), t = 1 / (1 + p x), |error| <= 1.5e-7 -- far
-// below the bf16 rounding the result gets next.  Phi(u) = 1 - q/2 for u >= 0
-// and q/2 for u < 0 (no cancellation in the tail).  One reciprocal and one
-// exponential on MUFU, five FMAs.
+// Abramowitz & Stegun, Handbook of Mathematical Functions, 7.1.28: for
+// x >= 0, erf(x) = 1 - 1 / (1 + a1 x + a2 x^2 + ... + a6 x^6)^16 with
+// |error| <= 3e-7 -- far below the bf16 rounding the result gets next.
+// Phi(u) = 1 - r/2 for u >= 0 and r/2 for u < 0, r = 1 / poly^16 (no
+// cancellation in the tail; poly^16 overflows to +inf far out, where
+// r = 0).  One reciprocal on MUFU, ten FMA-pipe operations.
 __device__ __forceinline__ float gelu(float u) {
-  constexpr float kP = 0.3275911f;
-  constexpr float kA1 = 0.254829592f, kA2 = -0.284496736f, kA3 = 1.421413741f;
-  constexpr float kA4 = -1.453152027f, kA5 = 1.061405429f;
+  constexpr float kA1 = 0.0705230784f, kA2 = 0.0422820123f, kA3 = 0.0092705272f;
+  constexpr float kA4 = 0.0001520143f, kA5 = 0.0002765672f, kA6 = 0.0000430638f;
   constexpr float kInvSqrt2 = 0.70710678118654752f;
-  constexpr float kNegLog2e = -1.4426950408889634f;
   const float x = fabsf(u) * kInvSqrt2;
-  float t;
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(t) : "f"(fmaf(kP, x, 1.f)));
-  float poly = fmaf(kA5, t, kA4);
-  poly = fmaf(poly, t, kA3);
-  poly = fmaf(poly, t, kA2);
-  poly = fmaf(poly, t, kA1);
-  const float q = poly * t * ex2(x * x * kNegLog2e);
-  const float phi = u >= 0.f ? fmaf(-0.5f, q, 1.f) : 0.5f * q;
+  float poly = fmaf(kA6, x, kA5);
+  poly = fmaf(poly, x, kA4);
+  poly = fmaf(poly, x, kA3);
+  poly = fmaf(poly, x, kA2);
+  poly = fmaf(poly, x, kA1);
+  poly = fmaf(poly, x, 1.f);
+  poly *= poly;  // ^2
+  poly *= poly;  // ^4
+  poly *= poly;  // ^8
+  poly *= poly;  // ^16
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(poly));
+  const float phi = u >= 0.f ? fmaf(-0.5f, r, 1.f) : 0.5f * r;
   return u * phi;
+}
+
+// Epilogue of one tile row: psi = Psi + b_b over D' columns read from TMEM,
+// part i (columns i W .. (i + 1) W - 1, W = D' / P) raised to the power i + 1,
+// stored as fp32.  kDp, kP > 0: the part width is a compile-time constant and
+// the power is applied with kP - 1 predicated products; kP = 0: any P, the
+// power advances at part boundaries.
+template <int kDp, int kP>
+__device__ __forceinline__ void store_row(float* out, const float4* bias4, uint32_t taddr,
+                                          bool valid, int Dp, int parts) {
+  const int dp = kDp > 0 ? kDp : Dp;
+  const int width = kP > 0 ? (kDp > 0 ? kDp : Dp) / kP : Dp / parts;
+  int power = 1, next = width;  // kP = 0: power of the current column, next boundary
+#pragma unroll 1
+  for (int c0 = 0; c0 < (kDp > 0 ? kDp : 128); c0 += 32) {
+    if (kDp == 0 && c0 >= dp) break;
+    uint32_t r[32];
+    REHYAT_TMEM_LD32(taddr + c0, r);
+    REHYAT_TMEM_WAIT_LD32(r);
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float4 b4 = __ldg(bias4 + (c0 + i) / 4);  // one load per 4 columns after unrolling
+      const float bi = (i & 3) == 0 ? b4.x : (i & 3) == 1 ? b4.y : (i & 3) == 2 ? b4.z : b4.w;
+      const float x = __uint_as_float(r[i]) + bi;
+      float y = x;
+      if (kP > 0) {
+        const int pw = (c0 + i) / width + 1;  // division by a constant, uniform
+#pragma unroll
+        for (int e = 1; e < kP; ++e)
+          if (e < pw) y *= x;
+      } else {
+        if (c0 + i == next) {  // the same for every lane
+          ++power;
+          next += width;
+        }
+        for (int e = 1; e < power; ++e) y *= x;
+      }
+      v[i] = y;
+    }
+    if (valid) {
+      float4* o4 = reinterpret_cast<float4*>(out + c0);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        o4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    }
+  }
 }
 }  // namespace mlp
 
@@ -121,6 +171,7 @@ __global__ void __launch_bounds__(mlp::kThreads, 1)
   using mlp::bar_off;
   using mlp::w_bytes;
   using mlp::gelu;
+  using mlp::store_row;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -286,14 +337,11 @@ __global__ void __launch_bounds__(mlp::kThreads, 1)
         uint32_t r0[32], r1[32];
         REHYAT_TMEM_LD32(col, r0);
         REHYAT_TMEM_LD32(col + 32, r1);
-        float4 bq[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) bq[i] = __ldg(bias4 + i);
-        auto convert = [&](const uint32_t* r, uint32_t dst) {
+        auto convert = [&](const uint32_t* r, uint32_t dst, const float4* b) {
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            const float4 b4 = bq[i];
+            const float4 b4 = __ldg(b + i);
             pk[2 * i] = pack_bf16(gelu(__uint_as_float(r[4 * i]) + b4.x),
                                   gelu(__uint_as_float(r[4 * i + 1]) + b4.y));
             pk[2 * i + 1] = pack_bf16(gelu(__uint_as_float(r[4 * i + 2]) + b4.z),
@@ -303,10 +351,8 @@ __global__ void __launch_bounds__(mlp::kThreads, 1)
         };
         REHYAT_TMEM_WAIT_LD32(r0);
         REHYAT_TMEM_WAIT_LD32(r1);
-        convert(r0, col);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) bq[i] = __ldg(bias4 + 8 + i);
-        convert(r1, col + 16);
+        convert(r0, col, bias4);
+        convert(r1, col + 16, bias4 + 8);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -317,7 +363,6 @@ __global__ void __launch_bounds__(mlp::kThreads, 1)
     // ================================================= epilogue (thread = token)
     const int q = warp - kEpiWarp0;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
-    const int width = Dp / a.parts;
     bool ok = true;
     int tl = 0;
     for (int it = it0; it < it1 && ok; ++it, ++tl) {
@@ -330,36 +375,14 @@ __global__ void __launch_bounds__(mlp::kThreads, 1)
       const bool valid = row < a.N;
       float* out = a.phi + (static_cast<long long>(t.b * a.heads + t.h) * a.N + row) * Dp;
       const float4* bias4 = reinterpret_cast<const float4*>(a.bb + static_cast<long long>(t.h) * Dp);
-      for (int c0 = 0; c0 < Dp; c0 += 32) {
-        uint32_t r[32];
-        REHYAT_TMEM_LD32(lane_base + kColPsi + pb * 128 + c0, r);
-        float bv[32];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float4 b4 = __ldg(bias4 + c0 / 4 + i);
-          bv[4 * i] = b4.x;
-          bv[4 * i + 1] = b4.y;
-          bv[4 * i + 2] = b4.z;
-          bv[4 * i + 3] = b4.w;
-        }
-        REHYAT_TMEM_WAIT_LD32(r);
-        float v[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int f = c0 + i;
-          const float x = __uint_as_float(r[i]) + bv[i];
-          const int power = f / width + 1;  // the same for every lane
-          float y = x;
-          for (int e = 1; e < power; ++e) y *= x;
-          v[i] = y;
-        }
-        if (valid) {
-          float4* o4 = reinterpret_cast<float4*>(out + c0);
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            o4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-        }
-      }
+      const uint32_t taddr = lane_base + kColPsi + pb * 128;
+      if (Dp == 128 && a.parts == 2) store_row<128, 2>(out, bias4, taddr, valid, Dp, a.parts);
+      else if (Dp == 128 && a.parts == 1) store_row<128, 1>(out, bias4, taddr, valid, Dp, a.parts);
+      else if (Dp == 128 && a.parts == 4) store_row<128, 4>(out, bias4, taddr, valid, Dp, a.parts);
+      else if (Dp == 64 && a.parts == 2) store_row<64, 2>(out, bias4, taddr, valid, Dp, a.parts);
+      else if (Dp == 64 && a.parts == 1) store_row<64, 1>(out, bias4, taddr, valid, Dp, a.parts);
+      else if (Dp == 64 && a.parts == 4) store_row<64, 4>(out, bias4, taddr, valid, Dp, a.parts);
+      else store_row<0, 0>(out, bias4, taddr, valid, Dp, a.parts);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(PSI_FREE + pb));
