@@ -78,28 +78,40 @@ __device__ __forceinline__ Tile tile_of(int it, int batch, int ntile) {
 // Abramowitz & Stegun, Handbook of Mathematical Functions, 7.1.28: for
 // x >= 0, erf(x) = 1 - 1 / (1 + a1 x + a2 x^2 + ... + a6 x^6)^16 with
 // |error| <= 3e-7 -- far below the bf16 rounding the result gets next.
-// Phi(u) = 1 - r/2 for u >= 0 and r/2 for u < 0, r = 1 / poly^16 (no
-// cancellation in the tail; poly^16 overflows to +inf far out, where
-// r = 0).  One reciprocal on MUFU, ten FMA-pipe operations.
-__device__ __forceinline__ float gelu(float u) {
-  constexpr float kA1 = 0.0705230784f, kA2 = 0.0422820123f, kA3 = 0.0092705272f;
-  constexpr float kA4 = 0.0001520143f, kA5 = 0.0002765672f, kA6 = 0.0000430638f;
-  constexpr float kInvSqrt2 = 0.70710678118654752f;
-  const float x = fabsf(u) * kInvSqrt2;
-  float poly = fmaf(kA6, x, kA5);
-  poly = fmaf(poly, x, kA4);
-  poly = fmaf(poly, x, kA3);
-  poly = fmaf(poly, x, kA2);
-  poly = fmaf(poly, x, kA1);
-  poly = fmaf(poly, x, 1.f);
-  poly *= poly;  // ^2
-  poly *= poly;  // ^4
-  poly *= poly;  // ^8
-  poly *= poly;  // ^16
-  float r;
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(poly));
-  const float phi = u >= 0.f ? fmaf(-0.5f, r, 1.f) : 0.5f * r;
-  return u * phi;
+// With r = 1 / poly^16, Phi(u) = 1 - r/2 for u >= 0 and r/2 for u < 0 (no
+// cancellation in the tail; poly^16 overflows to +inf far out, where r = 0).
+constexpr float kErfA1 = 0.0705230784f, kErfA2 = 0.0422820123f, kErfA3 = 0.0092705272f;
+constexpr float kErfA4 = 0.0001520143f, kErfA5 = 0.0002765672f, kErfA6 = 0.0000430638f;
+
+// GELU of two values at once on packed fp32 pairs (sm_100 f32x2 FMA / MUL),
+// rounded to a bf16 pair, written as
+//   GELU(u) = max(u, 0) - |u| r / 2,  r = 1 / poly(|u| / sqrt 2)^16,
+// which is u (1 - r/2) for u >= 0 and u r / 2 for u < 0.  One MUFU
+// reciprocal per value, about ten FMA-pipe instructions per pair.
+__device__ __forceinline__ uint32_t gelu2_bf16(float u0, float u1) {
+  const uint64_t u = f2_pack(u0, u1);
+  const uint64_t au = u & 0x7FFFFFFF7FFFFFFFull;  // |u| of both
+  const uint64_t x = f2_mul(au, f2_pack(0.70710678118654752f, 0.70710678118654752f));
+  auto c2 = [](float c) { return f2_pack(c, c); };
+  uint64_t poly = f2_fma(c2(kErfA6), x, c2(kErfA5));
+  poly = f2_fma(poly, x, c2(kErfA4));
+  poly = f2_fma(poly, x, c2(kErfA3));
+  poly = f2_fma(poly, x, c2(kErfA2));
+  poly = f2_fma(poly, x, c2(kErfA1));
+  poly = f2_fma(poly, x, c2(1.f));
+  poly = f2_mul(poly, poly);  // ^2
+  poly = f2_mul(poly, poly);  // ^4
+  poly = f2_mul(poly, poly);  // ^8
+  poly = f2_mul(poly, poly);  // ^16
+  float p0, p1, r0, r1;
+  f2_unpack(poly, p0, p1);
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r0) : "f"(p0));
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r1) : "f"(p1));
+  const uint64_t t = f2_mul(au, f2_pack(r0, r1));
+  const uint64_t g = f2_fma(t, c2(-0.5f), f2_pack(fmaxf(u0, 0.f), fmaxf(u1, 0.f)));
+  float g0, g1;
+  f2_unpack(g, g0, g1);
+  return pack_bf16(g0, g1);
 }
 
 // Epilogue of one tile row: psi = Psi + b_b over D' columns read from TMEM,
@@ -170,7 +182,7 @@ __global__ void __launch_bounds__(mlp::kThreads, 1)
   using mlp::tile_of;
   using mlp::bar_off;
   using mlp::w_bytes;
-  using mlp::gelu;
+  using mlp::gelu2_bf16;
   using mlp::store_row;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -342,10 +354,10 @@ __global__ void __launch_bounds__(mlp::kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const float4 b4 = __ldg(b + i);
-            pk[2 * i] = pack_bf16(gelu(__uint_as_float(r[4 * i]) + b4.x),
-                                  gelu(__uint_as_float(r[4 * i + 1]) + b4.y));
-            pk[2 * i + 1] = pack_bf16(gelu(__uint_as_float(r[4 * i + 2]) + b4.z),
-                                      gelu(__uint_as_float(r[4 * i + 3]) + b4.w));
+            pk[2 * i] = gelu2_bf16(__uint_as_float(r[4 * i]) + b4.x,
+                                   __uint_as_float(r[4 * i + 1]) + b4.y);
+            pk[2 * i + 1] = gelu2_bf16(__uint_as_float(r[4 * i + 2]) + b4.z,
+                                       __uint_as_float(r[4 * i + 3]) + b4.w);
           }
           REHYAT_TMEM_ST16(dst, pk);
         };
