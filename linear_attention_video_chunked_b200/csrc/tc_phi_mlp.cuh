@@ -83,6 +83,12 @@ __device__ __forceinline__ Tile tile_of(int it, int batch, int ntile) {
 constexpr float kErfA1 = 0.0705230784f, kErfA2 = 0.0422820123f, kErfA3 = 0.0092705272f;
 constexpr float kErfA4 = 0.0001520143f, kErfA5 = 0.0002765672f, kErfA6 = 0.0000430638f;
 
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 // GELU of two values at once on packed fp32 pairs (sm_100 f32x2 FMA / MUL),
 // rounded to a bf16 pair, written as
 //   GELU(u) = max(u, 0) - |u| r / 2,  r = 1 / poly(|u| / sqrt 2)^16,
