@@ -127,8 +127,13 @@ def _pairwise_head(q, k, v, Wq, bq, Wk, bk, HW, Tc, To, causal, scale):
 # --------------------------------------------------------------------------
 # Form (ii): per chunk, window softmax + linear state over the linear set.
 # --------------------------------------------------------------------------
-def _factored_head(q, k, v, Wq, bq, Wk, bk, T, HW, Tc, To, causal, scale, chunks=None):
+def _factored_head(q, k, v, Wq, bq, Wk, bk, T, HW, Tc, To, causal, scale, chunks=None,
+                   q_logit=None, k_logit=None):
+    # q_logit, k_logit: the vectors the softmax logits are formed from when
+    # they differ from q, k (the fp8 softmax variant); phi always sees q, k.
     N, D = q.shape
+    ql = q if q_logit is None else q_logit
+    kl = k if k_logit is None else k_logit
     y = np.zeros((N, D))
     parts = _empty_partials(N, D)
     for t, (first, end, start) in enumerate(chunk_table(T, Tc, To)):
@@ -137,7 +142,7 @@ def _factored_head(q, k, v, Wq, bq, Wk, bk, T, HW, Tc, To, causal, scale, chunks
         rows = slice(first * HW, end * HW)
         Qc = q[rows]
         Kw, Vw = k[start * HW:end * HW], v[start * HW:end * HW]
-        logits = (Qc @ Kw.T) * scale
+        logits = (ql[rows] @ kl[start * HW:end * HW].T) * scale
         c = logits.max(axis=1)
         E = np.exp(logits - c[:, None])
         aS = E @ Vw
