@@ -37,7 +37,7 @@ WORKLOAD = "wan_480x832_bidir"
 METRIC = "hybrid-attn fwd tokens/s & TFLOP/s (% BF16 tensor peak), 1 B200, 21x30x52 latent"
 L2_FLUSH_BYTES = 256 << 20
 KERNELS_PER_STEP = 4  # weight images, per-slice state, chunk scan, attention
-EXTRAS = ("full_softmax", "phi_backward", "general_phi", "streaming")
+EXTRAS = ("full_softmax", "fp8_qk", "phi_backward", "general_phi", "streaming")
 E2E_HEADS_PER_SLAB = 2
 
 
@@ -383,6 +383,62 @@ def measure_general_phi(rh, p, q, k, v, flush, stream, calls=3):
     else:
         out["feature_maps_alu_frac"] = tflops / FP32_ALU_TFLOPS
     return out
+
+
+def measure_fp8_qk(rh, p, q, k, v, phi, flush, stream, calls=5):
+    """The fp8 softmax-branch variant (REHYAT_FLAG_FP8_QK) on the bench
+    layer: the same step (state stage, then the E4M3 copies of q and k and the
+    attention kernel with q.k^T on kind::f8f6f4), device time per stage."""
+    import torch
+    B, H, N, D = q.shape
+    params = rh.make_params(batch=B, heads=H, T=p.T, Hs=p.Hs, Ws=p.Ws, D=D, Dp=p.Dp, Tc=p.Tc,
+                            To=p.To, causal=p.causal, in_dtype=rh.BF16, out_dtype=rh.F32,
+                            flags=rh.FLAG_FP8_QK)
+    nbytes = rh.rehyat_workspace_bytes(params)
+    if nbytes == 0:
+        return {"unavailable": "REHYAT_FLAG_FP8_QK not supported for this layer"}
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    y = torch.empty(B, H, N, D, device=q.device)
+    sh = stream.cuda_stream
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
+        st = rh.rehyat_fwd_state(params, k.data_ptr(), v.data_ptr(), phi, ws.data_ptr(), nbytes,
+                                 sh)
+        if evs:
+            evs[1].record(stream)
+        st = st or rh.rehyat_fwd_attn(params, q.data_ptr(), k.data_ptr(), v.data_ptr(), phi,
+                                      y.data_ptr(), ws.data_ptr(), nbytes, None, sh)
+        if evs:
+            evs[2].record(stream)
+        if st:
+            raise rh.RehyatError(st, "fp8 forward")
+
+    for _ in range(3):
+        flush()
+        step()
+    torch.cuda.synchronize()
+    t_step, t_attn = [], []
+    for _ in range(calls):
+        flush()
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        step(evs)
+        torch.cuda.synchronize()
+        t_step.append(evs[0].elapsed_time(evs[2]))
+        t_attn.append(evs[1].elapsed_time(evs[2]))
+    w = algorithmic_work(B, H, p.T, p.HW, D, p.Dp, p.Tc, p.To, p.causal)
+    peaks = load_peaks()
+    ms, attn_ms = sum(t_step) / calls, sum(t_attn) / calls
+    del ws, y
+    return {"ms_per_step": ms, "attention_stage_ms": attn_ms,
+            "tokens_per_s": B * N / (ms / 1e3),
+            "attention_tflops": w["attn_flops"] / (attn_ms / 1e3) / 1e12,
+            "attention_frac_bf16_peak": w["attn_flops"] / (attn_ms / 1e3) / 1e12
+            / peaks["bf16_tflops"],
+            "what": "REHYAT_FLAG_FP8_QK: q.k^T from E4M3 copies of q, k (kind::f8f6f4), P.V "
+                    "and the linear branch bf16; the attention stage includes the E4M3 "
+                    "conversion kernel"}
 
 
 def measure_streaming(rh, dev, flush, stream):
@@ -736,6 +792,9 @@ def run_gpu(args, world, rank, local):
         extra["full_softmax"] = measure_full_softmax(rh, q, k, v, y, flush, stream)
     del y, ws
     torch.cuda.empty_cache()
+    if "fp8_qk" in want:
+        extra["fp8_qk"] = measure_fp8_qk(rh, p, q, k, v, phi, flush, stream)
+        torch.cuda.empty_cache()
     if "phi_backward" in want:
         extra["phi_backward"] = measure_phi_backward(rh, p, q, k, v, Wq, bq, Wk, bk, flush,
                                                      stream)

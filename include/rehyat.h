@@ -70,6 +70,18 @@ typedef enum { REHYAT_F32 = 0, REHYAT_BF16 = 1 } rehyat_dtype;
 #define REHYAT_FLAG_ONE_TILE 2   /* tensor-core attention: use the one-query-tile
                                     kernel (the default for Dp = 256) instead of
                                     the two-tile kernel (testing aid) */
+#define REHYAT_FLAG_FP8_QK 4     /* fp8 softmax branch: the logits q.k^T are formed
+                                    from q and k rounded to E4M3 (round to nearest
+                                    even, saturating at +-448, unit scale) on the
+                                    tensor cores (kind::f8f6f4); P.V, the feature
+                                    maps and the linear branch keep bf16.  Full
+                                    forward only (rehyat_hybrid_attn_fwd, the
+                                    split stages, the host-buffer forward), bf16
+                                    inputs, D = 128, Dp <= 128; every other entry
+                                    point returns REHYAT_ERR_UNSUPPORTED with it.
+                                    The workspace grows by the two E4M3 copies
+                                    (2 * B * h * N * D bytes), which
+                                    rehyat_fwd_attn writes. */
 
 typedef struct {
   int batch, heads;   /* B >= 1, h >= 1 */
@@ -136,7 +148,7 @@ REHYAT_API rehyat_status rehyat_fwd_state(const rehyat_params* p, const void* k,
 REHYAT_API rehyat_status rehyat_fwd_attn(const rehyat_params* p, const void* q,
                                          const void* k, const void* v,
                                          const rehyat_phi* phi, void* y,
-                                         const void* workspace, size_t ws_bytes,
+                                         void* workspace, size_t ws_bytes,
                                          const rehyat_debug* dbg, void* stream);
 
 /* The full forward without a caller-supplied workspace, for callers that

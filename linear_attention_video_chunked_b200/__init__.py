@@ -24,7 +24,7 @@ from typing import Optional
 
 __all__ = [
     "RehyatParams", "RehyatPhi", "RehyatDebug", "RehyatError", "lib", "lib_path",
-    "EXPORTED_SYMBOLS", "F32", "BF16", "FLAG_FORCE_SIMT",
+    "EXPORTED_SYMBOLS", "F32", "BF16", "FLAG_FORCE_SIMT", "FLAG_FP8_QK",
     "rehyat_workspace_bytes", "rehyat_hybrid_attn_fwd", "rehyat_fwd_state", "rehyat_fwd_attn",
     "rehyat_softmax_attn_fwd", "rehyat_state_bytes", "rehyat_state_init", "rehyat_step_workspace_bytes",
     "rehyat_chunk_step", "rehyat_device_error_flags", "rehyat_attn_path",
@@ -40,6 +40,7 @@ __all__ = [
 F32, BF16 = 0, 1
 FLAG_FORCE_SIMT = 1
 FLAG_ONE_TILE = 2
+FLAG_FP8_QK = 4
 
 STATUS = {0: "REHYAT_OK", 1: "REHYAT_ERR_INVALID_ARG", 2: "REHYAT_ERR_UNSUPPORTED",
           3: "REHYAT_ERR_MISALIGNED", 4: "REHYAT_ERR_WORKSPACE", 5: "REHYAT_ERR_CUDA",
@@ -328,11 +329,13 @@ def _debug_tensors(shape4, device):
 
 
 def hybrid_attn(q, k, v, Wq, bq, Wk, bk, *, T, Hs, Ws, Tc, To, causal, out_dtype=None,
-                scale=0.0, debug=False, force_simt=False, one_tile=False, workspace=None,
-                out=None, stream=None):
+                scale=0.0, debug=False, force_simt=False, one_tile=False, fp8_qk=False,
+                workspace=None, out=None, stream=None):
     """ReHyAt hybrid attention of torch CUDA tensors q, k, v [B, h, N, D].
 
-    Returns y (and a dict of branch partials when ``debug``)."""
+    ``fp8_qk``: the softmax logits from E4M3 copies of q and k
+    (REHYAT_FLAG_FP8_QK).  Returns y (and a dict of branch partials when
+    ``debug``)."""
     torch = _torch()
     B, H, N, D = q.shape
     if N != T * Hs * Ws:
@@ -343,12 +346,12 @@ def hybrid_attn(q, k, v, Wq, bq, Wk, bk, *, T, Hs, Ws, Tc, To, causal, out_dtype
                     causal=causal, in_dtype=_dtype_code(q.dtype),
                     out_dtype=_dtype_code(out_dtype), scale=scale,
                     flags=(FLAG_FORCE_SIMT if force_simt else 0) |
-                    (FLAG_ONE_TILE if one_tile else 0))
+                    (FLAG_ONE_TILE if one_tile else 0) | (FLAG_FP8_QK if fp8_qk else 0))
     y = torch.empty(B, H, N, D, dtype=out_dtype, device=q.device) if out is None else out
     nbytes = rehyat_workspace_bytes(p)
     if nbytes == 0:
         raise RehyatError(1, "rehyat_workspace_bytes")
-    if workspace is None:
+    if workspace is None or workspace.numel() < nbytes:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
     dbg_t, dbg_s = _debug_tensors((B, H, N, D), q.device) if debug else (None, None)
     st = rehyat_hybrid_attn_fwd(p, q.data_ptr(), k.data_ptr(), v.data_ptr(),

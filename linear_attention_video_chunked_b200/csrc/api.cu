@@ -34,13 +34,23 @@ rehyat_status check_params(const rehyat_params* p) {
   const long long N = HW * p->T;
   if (N * p->D >= (1LL << 31) || static_cast<long long>(p->batch) * p->heads >= 65535)
     return REHYAT_ERR_UNSUPPORTED;
+  // The fp8 softmax variant runs on the two-query-tile tensor-core kernel only.
+  if ((p->flags & REHYAT_FLAG_FP8_QK) &&
+      (p->in_dtype != REHYAT_BF16 || p->D != 128 || p->Dp > 128 ||
+       (p->flags & (REHYAT_FLAG_FORCE_SIMT | REHYAT_FLAG_ONE_TILE))))
+    return REHYAT_ERR_UNSUPPORTED;
   return REHYAT_OK;
+}
+
+// Entry points without an fp8 softmax variant.
+rehyat_status no_fp8(const rehyat_params* p) {
+  return (p && (p->flags & REHYAT_FLAG_FP8_QK)) ? REHYAT_ERR_UNSUPPORTED : REHYAT_OK;
 }
 
 int nchunks_of(const rehyat_params* p) { return (p->T + p->Tc - 1) / p->Tc; }
 
 struct FwdWorkspace {
-  size_t P_off, z_off, SL_off, zL_off, wimg_off, wkimg_off, total;
+  size_t P_off, z_off, SL_off, zL_off, wimg_off, wkimg_off, q8_off, k8_off, total;
 };
 
 // phi_q or phi_k weight image (bf16, all heads) for the tensor-core kernels.
@@ -58,7 +68,12 @@ FwdWorkspace fwd_layout(const rehyat_params* p) {
   w.zL_off = align_up(w.SL_off + BH * nchunks_of(p) * PD * sizeof(float));
   w.wimg_off = align_up(w.zL_off + BH * nchunks_of(p) * p->Dp * sizeof(float));
   w.wkimg_off = align_up(w.wimg_off + wimg_bytes(p));
-  w.total = align_up(w.wkimg_off + wimg_bytes(p));
+  w.q8_off = w.k8_off = w.total = align_up(w.wkimg_off + wimg_bytes(p));
+  if (p->flags & REHYAT_FLAG_FP8_QK) {  // E4M3 copies of q and k
+    const size_t n8 = BH * p->T * static_cast<size_t>(p->Hs) * p->Ws * p->D;
+    w.k8_off = align_up(w.q8_off + n8);
+    w.total = align_up(w.k8_off + n8);
+  }
   return w;
 }
 
@@ -175,6 +190,8 @@ bool use_tc(const rehyat_params* p, const AttnParams& a) {
 }
 
 cudaError_t run_attn(const rehyat_params* p, const AttnParams& a, cudaStream_t s) {
+  if (a.q8 != nullptr)  // the fp8 variant exists on the tensor-core kernel only
+    return use_tc(p, a) ? launch_attn_tc(a, s) : cudaErrorNotSupported;
   if (use_tc(p, a)) return launch_attn_tc(a, s);
   return launch_attn_simt(a, s);
 }
@@ -285,7 +302,7 @@ rehyat_status rehyat_fwd_state(const rehyat_params* p, const void* k, const void
 
 rehyat_status rehyat_fwd_attn(const rehyat_params* p, const void* q, const void* k,
                               const void* v, const rehyat_phi* phi, void* y,
-                              const void* workspace, size_t ws_bytes, const rehyat_debug* dbg,
+                              void* workspace, size_t ws_bytes, const rehyat_debug* dbg,
                               void* stream) {
   rehyat_status st = check_params(p);
   if (st != REHYAT_OK) return st;
@@ -296,14 +313,22 @@ rehyat_status rehyat_fwd_attn(const rehyat_params* p, const void* q, const void*
     return REHYAT_ERR_MISALIGNED;
   const FwdWorkspace w = fwd_layout(p);
   if (ws_bytes < w.total) return REHYAT_ERR_WORKSPACE;
-  const char* ws = static_cast<const char*>(workspace);
+  char* ws = static_cast<char*>(workspace);
   AttnParams a = base_attn(p, q, k, v, phi, y, dbg);
   a.rows_per_bh = static_cast<long long>(p->T) * p->Hs * p->Ws;
   a.SL = reinterpret_cast<const float*>(ws + w.SL_off);
   a.zL = reinterpret_cast<const float*>(ws + w.zL_off);
   a.nchunks = nchunks_of(p);
   if (tc_path(p)) a.wq_img = ws + w.wimg_off;
-  return to_status(run_attn(p, a, static_cast<cudaStream_t>(stream)));
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (p->flags & REHYAT_FLAG_FP8_QK) {
+    const cudaError_t e = launch_e4m3(q, k, ws + w.q8_off, ws + w.k8_off,
+                                      static_cast<long long>(a.BH) * a.rows_per_bh * p->D, s);
+    if (e != cudaSuccess) return to_status(e);
+    a.q8 = ws + w.q8_off;
+    a.k8 = ws + w.k8_off;
+  }
+  return to_status(run_attn(p, a, s));
 }
 
 rehyat_status rehyat_hybrid_attn_fwd(const rehyat_params* p, const void* q, const void* k,
@@ -328,6 +353,7 @@ rehyat_status rehyat_softmax_attn_fwd(const rehyat_params* p, const void* q, con
                                       const void* v, void* y, void* stream) {
   rehyat_status st = check_params(p);
   if (st != REHYAT_OK) return st;
+  if ((st = no_fp8(p)) != REHYAT_OK) return st;
   if (!q || !k || !v || !y) return REHYAT_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(y))
     return REHYAT_ERR_MISALIGNED;
@@ -343,18 +369,19 @@ rehyat_status rehyat_softmax_attn_fwd(const rehyat_params* p, const void* q, con
 }
 
 size_t rehyat_state_bytes(const rehyat_params* p) {
-  if (check_params(p) != REHYAT_OK) return 0;
+  if (check_params(p) != REHYAT_OK || no_fp8(p) != REHYAT_OK) return 0;
   return state_layout(p).total;
 }
 
 size_t rehyat_step_workspace_bytes(const rehyat_params* p) {
-  if (check_params(p) != REHYAT_OK) return 0;
+  if (check_params(p) != REHYAT_OK || no_fp8(p) != REHYAT_OK) return 0;
   return step_layout(p).total;
 }
 
 rehyat_status rehyat_state_init(const rehyat_params* p, void* state, void* stream) {
   rehyat_status st = check_params(p);
   if (st != REHYAT_OK) return st;
+  if ((st = no_fp8(p)) != REHYAT_OK) return st;
   if (!state) return REHYAT_ERR_INVALID_ARG;
   if (!aligned16(state)) return REHYAT_ERR_MISALIGNED;
   const StateLayout L = state_layout(p);
@@ -370,6 +397,7 @@ rehyat_status rehyat_chunk_step(const rehyat_params* p, const void* q, const voi
                                 const rehyat_debug* dbg, void* stream) {
   rehyat_status st = check_params(p);
   if (st != REHYAT_OK) return st;
+  if ((st = no_fp8(p)) != REHYAT_OK) return st;
   if (p->causal != 1) return REHYAT_ERR_INVALID_ARG;
   if (nslices < 1 || nslices > p->Tc) return REHYAT_ERR_INVALID_ARG;
   if (!q || !k || !v || !y || !state || !workspace) return REHYAT_ERR_INVALID_ARG;
@@ -444,6 +472,7 @@ rehyat_status rehyat_hybrid_attn_fwd_phi(const rehyat_params* p, const void* q, 
                                          const rehyat_debug* dbg, void* stream) {
   rehyat_status st = check_params(p);
   if (st != REHYAT_OK) return st;
+  if ((st = no_fp8(p)) != REHYAT_OK) return st;
   if (!q || !k || !v || !phi_q || !phi_k || !y || !workspace) return REHYAT_ERR_INVALID_ARG;
   if ((st = check_dbg(dbg)) != REHYAT_OK) return st;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(y) || !aligned16(phi_q) ||
@@ -485,7 +514,7 @@ rehyat_status rehyat_feature_map_mlp(const rehyat_params* p, const void* x,
 }
 
 size_t rehyat_phi_bwd_workspace_bytes(const rehyat_params* p) {
-  if (check_params(p) != REHYAT_OK) return 0;
+  if (check_params(p) != REHYAT_OK || no_fp8(p) != REHYAT_OK) return 0;
   int QS, KS;
   phi_bwd_split(p->T, p->Tc, p->Hs * p->Ws, &QS, &KS);
   const size_t parts = phi_bwd_partial_floats(p->batch * p->heads, p->T, nchunks_of(p), p->D,
@@ -499,6 +528,7 @@ rehyat_status rehyat_phi_bwd(const rehyat_params* p, const void* q, const void* 
                              void* workspace, size_t ws_bytes, void* stream) {
   rehyat_status st = check_params(p);
   if (st != REHYAT_OK) return st;
+  if ((st = no_fp8(p)) != REHYAT_OK) return st;
   if (!q || !k || !v || !y || !dy || !den || !grad || !workspace) return REHYAT_ERR_INVALID_ARG;
   if (!grad->dWq || !grad->dbq || !grad->dWk || !grad->dbk) return REHYAT_ERR_INVALID_ARG;
   if ((st = check_phi(phi)) != REHYAT_OK) return st;

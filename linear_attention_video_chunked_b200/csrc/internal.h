@@ -30,6 +30,7 @@ struct AttnParams {
   const float *Wq, *bq;      // phi_q parameters, fp32 [h][2][D][Dp/2], [h][2][Dp/2]
   const void* wq_img;        // bf16 phi_q weight image per head (tensor-core path) or nullptr
   const float* phi_q;        // phi_q(q) given as [BH][rows][Dp] fp32 (then Wq, bq unused) or nullptr
+  const void *q8, *k8;       // E4M3 copies of q, k for the softmax logits (fp8 variant) or nullptr
   void* y;
   float *dbg_aS, *dbg_nS, *dbg_c, *dbg_aL, *dbg_nL;
   int BH, heads, T, HW, D, Dp, Tc, To, nchunks, nq_slices;
@@ -100,6 +101,11 @@ cudaError_t launch_partials_simt(const PartialParams& p, cudaStream_t s);
 
 // bf16 images of the phi weights (layout.cuh, wimg_index) for the
 // tensor-core kernels: out [heads][Dp*D] each.  Wk/out_k may be null.
+// E4M3 copies of two bf16 arrays of n elements each (round to nearest even,
+// saturating at +-448), n a multiple of 8; pointers 16-byte aligned.
+cudaError_t launch_e4m3(const void* a, const void* b, void* a8, void* b8, long long n,
+                        cudaStream_t s);
+
 cudaError_t launch_w_images(const float* Wq, void* out_q, const float* Wk, void* out_k,
                             int heads, int D, int Dp, cudaStream_t s);
 bool tc_attn_eligible(int in_bf16, int D, int Dp);

@@ -9,6 +9,7 @@
 // window softmax with stabiliser c_t, linear branch phi_q(q) (sum phi_k v^T),
 // joint normalisation, overlap set, causal set and chunk-wise state.
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <math.h>
 
 #include "internal.h"
@@ -460,6 +461,31 @@ __global__ void step_finish_kernel(const float* __restrict__ P, const float* __r
   }
 }
 
+// E4M3 copies of q and k for the fp8 softmax variant: eight bf16 values in,
+// eight E4M3 bytes out per thread and array (round to nearest even,
+// saturating at +-448).
+__device__ __forceinline__ uint2 bf16x8_to_e4m3(uint4 v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t out[2] = {0, 0};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xFFFF0000u);
+    const __nv_fp8x2_storage_t p = __nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE,
+                                                            __NV_E4M3);
+    out[i >> 1] |= static_cast<uint32_t>(p) << (16 * (i & 1));
+  }
+  return make_uint2(out[0], out[1]);
+}
+
+__global__ void e4m3_kernel(const uint4* __restrict__ a, const uint4* __restrict__ b,
+                            uint2* __restrict__ a8, uint2* __restrict__ b8, long long n8) {
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    a8[i] = bf16x8_to_e4m3(__ldg(a + i));
+    b8[i] = bf16x8_to_e4m3(__ldg(b + i));
+  }
+}
+
 // bf16 copy of phi weights in the tensor-core image layout; blockIdx.y
 // selects the matrix (0: W_q, 1: W_k).
 __global__ void w_image_kernel(const float* __restrict__ Wq, __nv_bfloat16* __restrict__ out_q,
@@ -554,6 +580,15 @@ cudaError_t launch_step_finish(const float* P, const float* zp, float* s_state, 
       P, zp, s_state, z_state, seen, done, Dp, D, To, nq_slices, nslots, nadd,
       static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint4*>(rk),
       static_cast<uint4*>(rv), slice_vecs);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_e4m3(const void* a, const void* b, void* a8, void* b8, long long n,
+                        cudaStream_t s) {
+  const long long n8 = n / 8;
+  const int blocks = static_cast<int>(n8 / 256 + 1 < 4096 ? n8 / 256 + 1 : 4096);
+  e4m3_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint4*>(a), static_cast<const uint4*>(b),
+                                     static_cast<uint2*>(a8), static_cast<uint2*>(b8), n8);
   return cudaGetLastError();
 }
 

@@ -142,7 +142,8 @@ __device__ __forceinline__ uint64_t sdesc_repeat(uint32_t addr) {
 }
 
 // Instruction descriptor: fp32 accumulate, A K-major, A/B format fmt
-// (1 = bf16, 2 = tf32), B K-major or MN-major.
+// (kind::f16: 1 = bf16; kind::tf32: 2 = tf32; kind::f8f6f4: 0 = E4M3),
+// B K-major or MN-major.
 __host__ __device__ constexpr uint32_t idesc(int M, int N, uint32_t fmt, bool b_mn_major) {
   return (1u << 4) | (fmt << 7) | (fmt << 10) | ((b_mn_major ? 1u : 0u) << 16) |
          (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
@@ -169,6 +170,16 @@ __device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a, uint64_t b
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(id), "r"(accumulate));
+}
+
+// D (+)= A.B with A and B in E4M3 (8-bit float), fp32 accumulators, K = 32.
+__device__ __forceinline__ void mma_e4m3(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t id,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a), "l"(b), "r"(id), "r"(accumulate));
 }
 

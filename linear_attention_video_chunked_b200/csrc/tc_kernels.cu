@@ -87,6 +87,7 @@ namespace {
 // --------------------------------------------------------------- kernel
 struct TcMaps {
   CUtensorMap q, k, v, rk, rv;
+  CUtensorMap q8, k8;  // E4M3 copies of q, k (fp8 softmax variant)
 };
 
 struct TileSrc {
@@ -543,6 +544,12 @@ constexpr uint32_t kWOff = kKOff;                  // tail: phi_q weights (<= 32
 constexpr uint32_t kSLOff = kKOff + 32768;         // tail: S^L (<= 64 KB)
 constexpr uint32_t kPhiOff0 = kVOff;               // tail: phi_q(Q_A)/f (<= 64 KB)
 constexpr uint32_t kPhiOff1 = kQOff;               // tail: phi_q(Q_B)/f, over Q (<= 64 KB)
+// fp8 softmax variant: E4M3 K tiles are 16 KB (one 128-byte box per row), so
+// the K ring takes 48 KB and the E4M3 Q_A, Q_B sit in the 32 KB after it;
+// the bf16 Q stays for the phi_q tail, whose operands reuse [kKOff, kVOff)
+// once the last q.k^T has run.
+constexpr uint32_t kK8Stage = 16384;
+constexpr uint32_t kQ8Off = kKOff + 3 * kK8Stage;
 enum { Q_FULL = 0, K_FULL = 1, K_EMPTY = 4, V_FULL = 7, V_EMPTY = 9, S_FULL = 11, P_FULL = 13,
        PV_DONE = 15, LAST_PV = 17, TAIL_FULL = 18, PHI_DONE = 19, PHI_READY = 20, READ_DONE = 22,
        VEC_READY = 23, NBAR = 24 };
@@ -553,6 +560,9 @@ constexpr uint32_t kVecOff = kBarOff + 256;
 constexpr uint32_t kSmemBytes = kVecOff + 1024 + 1024;
 }  // namespace a2
 
+// kFp8: q.k^T from the E4M3 copies of q and k (tcgen05 kind::f8f6f4, K = 32
+// per instruction); everything else as in the bf16 kernel.
+template <bool kFp8>
 __global__ void __launch_bounds__(a2::kThreads, 1)
     tc_attn2_kernel(const __grid_constant__ TcMaps maps, const AttnParams P,
                     const __nv_bfloat16* __restrict__ wq_img) {
@@ -656,20 +666,30 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
     // ================================================= TMA producer
     if (lane == 0) {
       bool ok = true;
-      mbar_expect_tx(bar(a2::Q_FULL), 4 * 16384);
+      mbar_expect_tx(bar(a2::Q_FULL), (kFp8 ? 6 : 4) * 16384);
       tma_load_3d(base + kQOff, &maps.q, bar(a2::Q_FULL), 0, row0, bh);
       tma_load_3d(base + kQOff + 16384, &maps.q, bar(a2::Q_FULL), 64, row0, bh);
       tma_load_3d(base + kQOff + 32768, &maps.q, bar(a2::Q_FULL), 0, row0 + kBM, bh);
       tma_load_3d(base + kQOff + 49152, &maps.q, bar(a2::Q_FULL), 64, row0 + kBM, bh);
+      if (kFp8) {
+        tma_load_3d(base + a2::kQ8Off, &maps.q8, bar(a2::Q_FULL), 0, row0, bh);
+        tma_load_3d(base + a2::kQ8Off + 16384, &maps.q8, bar(a2::Q_FULL), 0, row0 + kBM, bh);
+      }
       for (int j = 0; j < nt && ok; ++j) {
         const TileSrc src = tile_src(j);
         const int ks = j % 3;
         if (j >= 3) ok = mbar_wait(bar(a2::K_EMPTY + ks), ((j - 3) / 3) & 1, abort_flag, 1);
         if (!ok) break;
-        const uint32_t kdst = base + kKOff + ks * 32768;
-        mbar_expect_tx(bar(a2::K_FULL + ks), 32768);
-        tma_load_3d(kdst, src.map_k, bar(a2::K_FULL + ks), 0, src.row, bh);
-        tma_load_3d(kdst + 16384, src.map_k, bar(a2::K_FULL + ks), 64, src.row, bh);
+        if (kFp8) {
+          const uint32_t kdst = base + kKOff + ks * a2::kK8Stage;
+          mbar_expect_tx(bar(a2::K_FULL + ks), a2::kK8Stage);
+          tma_load_3d(kdst, &maps.k8, bar(a2::K_FULL + ks), 0, src.row, bh);
+        } else {
+          const uint32_t kdst = base + kKOff + ks * 32768;
+          mbar_expect_tx(bar(a2::K_FULL + ks), 32768);
+          tma_load_3d(kdst, src.map_k, bar(a2::K_FULL + ks), 0, src.row, bh);
+          tma_load_3d(kdst + 16384, src.map_k, bar(a2::K_FULL + ks), 64, src.row, bh);
+        }
         const int vs = j & 1;
         if (j >= 2) ok = mbar_wait(bar(a2::V_EMPTY + vs), ((j - 2) >> 1) & 1, abort_flag, 26);
         if (!ok) break;
@@ -706,13 +726,24 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
       const int ntiles = has_b ? 2 : 1;
       bool ok = mbar_wait(bar(a2::Q_FULL), 0, abort_flag, 4);
       auto issue_s = [&](int tile, int j) {
-        const uint32_t kaddr = base + kKOff + (j % 3) * 32768;
-        const uint32_t qaddr = base + kQOff + tile * 32768;
+        if (kFp8) {
+          // E4M3 rows are 128 bytes: one box, 32 elements (32 bytes) a step.
+          const uint32_t kaddr = base + kKOff + (j % 3) * a2::kK8Stage;
+          const uint32_t qaddr = base + a2::kQ8Off + tile * 16384;
+          const uint32_t id_qk8 = idesc(kBM, kBN, 0, false);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_bf16(tmem + tile * 256, sdesc(qaddr + off, 16, 1024), sdesc(kaddr + off, 16, 1024),
-                   id_qk, kk > 0);
+          for (int kk = 0; kk < 4; ++kk)
+            mma_e4m3(tmem + tile * 256, sdesc(qaddr + kk * 32, 16, 1024),
+                     sdesc(kaddr + kk * 32, 16, 1024), id_qk8, kk > 0);
+        } else {
+          const uint32_t kaddr = base + kKOff + (j % 3) * 32768;
+          const uint32_t qaddr = base + kQOff + tile * 32768;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            mma_bf16(tmem + tile * 256, sdesc(qaddr + off, 16, 1024),
+                     sdesc(kaddr + off, 16, 1024), id_qk, kk > 0);
+          }
         }
         mma_commit(bar(a2::S_FULL + tile));
       };
@@ -1618,6 +1649,22 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+// 3D 8-bit map over [planes][rows][128] with a 128 x 128 x 1 box (one 128-byte
+// row per token), 128B swizzle.
+bool make_map8(CUtensorMap* m, const void* ptr, long long rows, int planes) {
+  auto fn = encode_fn();
+  if (!fn || rows <= 0) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(planes)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(kD),
+                           static_cast<cuuint64_t>(rows) * kD};
+  cuuint32_t box[3] = {128, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 3D bf16 map over [planes][rows][128] with a 64 x 128 x 1 box, 128B swizzle.
 bool make_map(CUtensorMap* m, const void* ptr, long long rows, int planes) {
   auto fn = encode_fn();
@@ -1725,11 +1772,20 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s) {
   const int qrows_max = p.seen ? p.nq_slices * p.HW : (p.Tc < p.T ? p.Tc : p.T) * p.HW;
   const bool two_tiles = !p.one_tile && (p.full_softmax || p.Dp <= 128);
   cudaError_t e;
-  if (two_tiles) {
-    e = ensure_smem(tc_attn2_kernel, 1, a2::kSmemBytes);
+  if (p.q8 != nullptr) {  // fp8 softmax variant (full forward, two-tile kernel only)
+    if (!two_tiles || p.seen || !make_map8(&maps.q8, p.q8, p.rows_per_bh, p.BH) ||
+        !make_map8(&maps.k8, p.k8, p.rows_per_bh, p.BH))
+      return cudaErrorInvalidValue;
+    e = ensure_smem(tc_attn2_kernel<true>, 5, a2::kSmemBytes);
     if (e != cudaSuccess) return e;
     dim3 grid((qrows_max + 2 * kBM - 1) / (2 * kBM), p.nchunks, p.BH);
-    tc_attn2_kernel<<<grid, a2::kThreads, a2::kSmemBytes, s>>>(
+    tc_attn2_kernel<true><<<grid, a2::kThreads, a2::kSmemBytes, s>>>(
+        maps, p, static_cast<const __nv_bfloat16*>(p.wq_img));
+  } else if (two_tiles) {
+    e = ensure_smem(tc_attn2_kernel<false>, 1, a2::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    dim3 grid((qrows_max + 2 * kBM - 1) / (2 * kBM), p.nchunks, p.BH);
+    tc_attn2_kernel<false><<<grid, a2::kThreads, a2::kSmemBytes, s>>>(
         maps, p, static_cast<const __nv_bfloat16*>(p.wq_img));
   } else {
     e = ensure_smem(tc_attn_kernel, 2, kSmemBytes);
