@@ -120,49 +120,70 @@ __device__ __forceinline__ uint32_t gelu2_bf16(float u0, float u1) {
   return pack_bf16(g0, g1);
 }
 
-// Epilogue of one tile row: psi = Psi + b_b over D' columns read from TMEM,
-// part i (columns i W .. (i + 1) W - 1, W = D' / P) raised to the power i + 1,
-// stored as fp32.  kDp, kP > 0: the part width is a compile-time constant and
-// the power is applied with kP - 1 predicated products; kP = 0: any P, the
-// power advances at part boundaries.
+// tcgen05.ld of 16 lanes x 256 bits, four times along the columns (32
+// columns): thread t holds, for repetition r, rows t/4 and t/4 + 8 of the 16
+// lanes at columns 8 r + 2 (t mod 4) and + 1 -- four consecutive threads hold
+// 8 consecutive columns of a row, so their stores fill whole 32-byte sectors.
+#define REHYAT_TMEM_LD16x256_X4(taddr, r)                                                       \
+  asm volatile(                                                                                \
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "  \
+      "%11, %12, %13, %14, %15}, [%16];"                                                       \
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),    \
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),             \
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])                                                  \
+      : "r"(taddr))
+
+// Epilogue of one warp's 32 tile rows (TMEM lane quadrant at tq): psi = Psi +
+// b_b over the D' columns, part i (columns i W .. (i + 1) W - 1, W = D' / P)
+// raised to the power i + 1, stored as fp32 rows of out (row 0 = the warp's
+// first row, `rows` of them valid).  kDp, kP > 0: the part width is a
+// compile-time constant and the power is applied with kP - 1 predicated
+// products; kP = 0: any P (a division per value).
 template <int kDp, int kP>
-__device__ __forceinline__ void store_row(float* out, const float4* bias4, uint32_t taddr,
-                                          bool valid, int Dp, int parts) {
+__device__ __forceinline__ void store_rows(float* out, const float* bias, uint32_t tq, int rows,
+                                           int Dp, int parts) {
   const int dp = kDp > 0 ? kDp : Dp;
-  const int width = kP > 0 ? (kDp > 0 ? kDp : Dp) / kP : Dp / parts;
-  int power = 1, next = width;  // kP = 0: power of the current column, next boundary
+  const int width = kP > 0 ? dp / kP : Dp / parts;
+  const int t = threadIdx.x & 31;
 #pragma unroll 1
-  for (int c0 = 0; c0 < (kDp > 0 ? kDp : 128); c0 += 32) {
-    if (kDp == 0 && c0 >= dp) break;
-    uint32_t r[32];
-    REHYAT_TMEM_LD32(taddr + c0, r);
-    REHYAT_TMEM_WAIT_LD32(r);
-    float v[32];
+  for (int lh = 0; lh < 2; ++lh) {
+    const int ra = 16 * lh + (t >> 2), rb = ra + 8;
+#pragma unroll 1
+    for (int c0 = 0; c0 < dp; c0 += 32) {
+      uint32_t r[16];
+      REHYAT_TMEM_LD16x256_X4(tq + (static_cast<uint32_t>(16 * lh) << 16) + c0, r);
+      asm volatile("tcgen05.wait::ld.sync.aligned;"
+                   : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                     "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                     "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+                   :
+                   : "memory");
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const float4 b4 = __ldg(bias4 + (c0 + i) / 4);  // one load per 4 columns after unrolling
-      const float bi = (i & 3) == 0 ? b4.x : (i & 3) == 1 ? b4.y : (i & 3) == 2 ? b4.z : b4.w;
-      const float x = __uint_as_float(r[i]) + bi;
-      float y = x;
-      if (kP > 0) {
-        const int pw = (c0 + i) / width + 1;  // division by a constant, uniform
+      for (int rep = 0; rep < 4; ++rep) {
+        const int c = c0 + 8 * rep + 2 * (t & 3);
+        const float2 b2 = __ldg(reinterpret_cast<const float2*>(bias + c));
+        float v[4];
 #pragma unroll
-        for (int e = 1; e < kP; ++e)
-          if (e < pw) y *= x;
-      } else {
-        if (c0 + i == next) {  // the same for every lane
-          ++power;
-          next += width;
+        for (int e = 0; e < 4; ++e) {
+          const float x = __uint_as_float(r[4 * rep + e]) + ((e & 1) ? b2.y : b2.x);
+          const int pw = (c + (e & 1)) / width + 1;
+          float y = x;
+          if (kP > 0) {
+#pragma unroll
+            for (int m = 1; m < kP; ++m)
+              if (m < pw) y *= x;
+          } else {
+            for (int m = 1; m < pw; ++m) y *= x;
+          }
+          v[e] = y;
         }
-        for (int e = 1; e < power; ++e) y *= x;
+        if (ra < rows)
+          *reinterpret_cast<float2*>(out + static_cast<long long>(ra) * dp + c) =
+              make_float2(v[0], v[1]);
+        if (rb < rows)
+          *reinterpret_cast<float2*>(out + static_cast<long long>(rb) * dp + c) =
+              make_float2(v[2], v[3]);
       }
-      v[i] = y;
-    }
-    if (valid) {
-      float4* o4 = reinterpret_cast<float4*>(out + c0);
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        o4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
     }
   }
 }
@@ -189,7 +210,7 @@ __global__ void __launch_bounds__(mlp::kThreads, 1)
   using mlp::bar_off;
   using mlp::w_bytes;
   using mlp::gelu2_bf16;
-  using mlp::store_row;
+  using mlp::store_rows;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -389,18 +410,19 @@ __global__ void __launch_bounds__(mlp::kThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(bar(PSI_FULL + pb), (tl >> 1) & 1, abort_flag, 47));
       if (!ok) break;
       tc_fence_after();
-      const long long row = static_cast<long long>(t.tile) * 128 + q * 32 + lane;
-      const bool valid = row < a.N;
-      float* out = a.phi + (static_cast<long long>(t.b * a.heads + t.h) * a.N + row) * Dp;
-      const float4* bias4 = reinterpret_cast<const float4*>(a.bb + static_cast<long long>(t.h) * Dp);
-      const uint32_t taddr = lane_base + kColPsi + pb * 128;
-      if (Dp == 128 && a.parts == 2) store_row<128, 2>(out, bias4, taddr, valid, Dp, a.parts);
-      else if (Dp == 128 && a.parts == 1) store_row<128, 1>(out, bias4, taddr, valid, Dp, a.parts);
-      else if (Dp == 128 && a.parts == 4) store_row<128, 4>(out, bias4, taddr, valid, Dp, a.parts);
-      else if (Dp == 64 && a.parts == 2) store_row<64, 2>(out, bias4, taddr, valid, Dp, a.parts);
-      else if (Dp == 64 && a.parts == 1) store_row<64, 1>(out, bias4, taddr, valid, Dp, a.parts);
-      else if (Dp == 64 && a.parts == 4) store_row<64, 4>(out, bias4, taddr, valid, Dp, a.parts);
-      else store_row<0, 0>(out, bias4, taddr, valid, Dp, a.parts);
+      const long long row0 = static_cast<long long>(t.tile) * 128 + q * 32;
+      const int rows = static_cast<int>(min(32LL, a.N - row0));
+      float* out = a.phi + (static_cast<long long>(t.b * a.heads + t.h) * a.N + row0) * Dp;
+      const float* bias = a.bb + static_cast<long long>(t.h) * Dp;
+      const uint32_t tq = lane_base + kColPsi + pb * 128;
+      const int P = a.parts;
+      if (Dp == 128 && P == 2) store_rows<128, 2>(out, bias, tq, rows, Dp, P);
+      else if (Dp == 128 && P == 1) store_rows<128, 1>(out, bias, tq, rows, Dp, P);
+      else if (Dp == 128 && P == 4) store_rows<128, 4>(out, bias, tq, rows, Dp, P);
+      else if (Dp == 64 && P == 2) store_rows<64, 2>(out, bias, tq, rows, Dp, P);
+      else if (Dp == 64 && P == 1) store_rows<64, 1>(out, bias, tq, rows, Dp, P);
+      else if (Dp == 64 && P == 4) store_rows<64, 4>(out, bias, tq, rows, Dp, P);
+      else store_rows<0, 0>(out, bias, tq, rows, Dp, P);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(PSI_FREE + pb));
