@@ -324,8 +324,6 @@ __global__ void __launch_bounds__(256) partials_simt_kernel(PartialParams P) {
 // ---------------------------------------------------------------------------
 // Chunk scan: one thread per state element, sequential over slices.
 // ---------------------------------------------------------------------------
-constexpr int kScanRegSlices = 32;  // slices the scan keeps in registers
-
 __global__ void scan_kernel(const float* __restrict__ P, const float* __restrict__ z,
                             float* __restrict__ SL, float* __restrict__ zL, int T, int Tc,
                             int To, int nchunks, int Dp, int D, int causal) {
@@ -350,29 +348,10 @@ __global__ void scan_kernel(const float* __restrict__ P, const float* __restrict
   } else {
     return;
   }
-  if (T <= kScanRegSlices) {
-    // All T values in registers, read once; chunk t's linear set (slices
-    // before its window start w_t and, bidirectional, from its end end_t
-    // on) summed in slice order with predicated adds -- no subtraction and
-    // one write per output.
-    float v[kScanRegSlices];
-#pragma unroll
-    for (int i = 0; i < kScanRegSlices; ++i)
-      v[i] = i < T ? src[static_cast<long long>(i) * stride] : 0.f;
-    for (int t = 0; t < nchunks; ++t) {
-      const int w = max(t * Tc - To, 0), end = min(T, (t + 1) * Tc);
-      float acc = 0.f;
-#pragma unroll
-      for (int i = 0; i < kScanRegSlices; ++i)
-        if (i < w || (!causal && i >= end && i < T)) acc += v[i];
-      dst[static_cast<long long>(t) * stride] = acc;
-    }
-    return;
-  }
-  // Longer sequences: slices are read in batches of 8 independent loads (the
-  // walk over slices is otherwise one dependent load at a time), then folded
-  // in order; chunk t receives the prefix when it reaches its window start
-  // w_t and, in the bidirectional form, the suffix from its end end_t on.
+  // Slices are read in batches of 8 independent loads (the walk over slices
+  // is otherwise one dependent load at a time), then folded in order; chunk
+  // t receives the prefix when it reaches its window start w_t and, in the
+  // bidirectional form, the suffix from its end end_t on.
   constexpr int kBatch = 8;
   float v[kBatch];
   float pre = 0.f;
