@@ -553,6 +553,10 @@ rehyat_status rehyat_phi_bwd(const rehyat_params* p, const void* q, const void* 
   a.batch = p->batch; a.heads = p->heads; a.T = p->T; a.HW = p->Hs * p->Ws; a.D = p->D;
   a.Dp = p->Dp; a.Tc = p->Tc; a.To = p->To; a.causal = p->causal; a.nchunks = nchunks_of(p);
   a.in_bf16 = p->in_dtype == REHYAT_BF16;
+  // Tensor-core q and k passes where the weight images exist (bf16, D = D' = 128).
+  a.tc = tc_path(p) && tc_phi_bwd_eligible(a.in_bf16, p->D, p->Dp);
+  a.wq_img = a.tc ? ws + w.wimg_off : nullptr;
+  a.wk_img = a.tc ? ws + w.wkimg_off : nullptr;
   return to_status(launch_phi_bwd(a, s));
 }
 

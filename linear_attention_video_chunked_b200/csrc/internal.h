@@ -69,10 +69,27 @@ struct PhiBwdArgs {
   const float *y, *dy, *den;
   const float *Wq, *bq, *Wk, *bk;
   const float *SL, *zL;
+  const void *wq_img, *wk_img;  // bf16 weight images (tensor-core passes) or nullptr
   float *partials;
   float *dWq, *dbq, *dWk, *dbk;
   int batch, heads, T, HW, D, Dp, Tc, To, causal, nchunks, in_bf16;
+  int tc;                       // run the q and k passes on tcgen05
 };
+// One tensor-core pass of the feature-map backward (tc_phi_bwd.cuh; bf16
+// inputs, D = D' = 128), writing the CUDA-core passes' partial layout.
+struct PhiBwdTcArgs {
+  const void *x, *v;          // q or k (the pass's rows), and v (k pass), bf16 [BH][N][128]
+  const float *dy, *y, *den;  // q pass: dL/dy, y, n^S + n^L
+  const void* w_img;          // bf16 image of W_q or W_k, [heads][Dp * D]
+  const float* b;             // b_q or b_k [heads][Dp]
+  const float* M;             // q: S_L per chunk (image layout); k: Ghat blocks per slice
+  const float* vec;           // q: z_L per chunk (k: hhat, inside the Ghat block)
+  float* part;                // partial blocks of the pass
+  int BH, heads, T, HW, Tc, nchunks, splits, q_side;
+};
+bool tc_phi_bwd_eligible(int in_bf16, int D, int Dp);
+cudaError_t launch_phi_bwd_tc(const PhiBwdTcArgs& a, cudaStream_t s);
+
 void phi_bwd_split(int T, int Tc, int HW, int* QS, int* KS);
 size_t phi_bwd_partial_floats(int BH, int T, int nchunks, int D, int Dp, int QS, int KS);
 cudaError_t launch_phi_bwd(const PhiBwdArgs& a, cudaStream_t s);

@@ -420,6 +420,27 @@ cudaError_t launch_phi_bwd(const PhiBwdArgs& a, cudaStream_t s) {
   bp.qpart = a.partials;
   bp.ghat = bp.qpart + z * a.nchunks * bp.QS * (2 * static_cast<size_t>(a.D) * kPiece + 2 * kPiece);
   bp.kpart = bp.ghat + z * a.T * (static_cast<size_t>(kPiece) * a.D + kPiece);
+  if (a.tc) {
+    // q and k passes on tcgen05; the Ghat and reduction passes as below.
+    PhiBwdTcArgs t = {};
+    t.BH = bp.BH; t.heads = bp.heads; t.T = bp.T; t.HW = bp.HW; t.Tc = bp.Tc;
+    t.nchunks = bp.nchunks;
+    t.x = a.q; t.dy = a.dy; t.y = a.y; t.den = a.den; t.w_img = a.wq_img; t.b = a.bq;
+    t.M = a.SL; t.vec = a.zL; t.part = bp.qpart; t.splits = bp.QS; t.q_side = 1;
+    cudaError_t e = launch_phi_bwd_tc(t, s);
+    if (e != cudaSuccess) return e;
+    const long long ng = static_cast<long long>(kPiece) * a.D + kPiece;
+    phi_bwd_ghat_kernel<<<dim3(static_cast<unsigned>((ng + 255) / 256), bp.T, bp.BH * bp.FP),
+                          256, 0, s>>>(bp);
+    t.x = a.k; t.v = a.v; t.w_img = a.wk_img; t.b = a.bk; t.M = bp.ghat; t.vec = nullptr;
+    t.part = bp.kpart; t.splits = bp.KS; t.q_side = 0;
+    e = launch_phi_bwd_tc(t, s);
+    if (e != cudaSuccess) return e;
+    const long long nr = (static_cast<long long>(a.D) * bp.Dp + bp.Dp) * bp.heads;
+    phi_bwd_reduce_kernel<<<dim3(static_cast<unsigned>((nr + 255) / 256), 2), 256, 0, s>>>(
+        bp, a.dWq, a.dbq, a.dWk, a.dbk, a.batch);
+    return cudaGetLastError();
+  }
   switch (a.D) {
     case 32: return launch_bwd_d<32>(bp, a, s);
     case 64: return launch_bwd_d<64>(bp, a, s);

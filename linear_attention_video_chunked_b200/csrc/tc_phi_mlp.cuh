@@ -502,3 +502,6 @@ cudaError_t launch_phi_mlp_tc(const PhiMlpArgs& a, void* images, cudaStream_t s)
 }
 
 }  // namespace rehyat
+
+// The feature-map backward's tensor-core passes share this unit too.
+#include "tc_phi_bwd.cuh"
