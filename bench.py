@@ -304,10 +304,17 @@ def measure_phi_backward(rh, p, q, k, v, Wq, bq, Wk, bk, flush, stream, calls=3)
     # plus the state pass it repeats (phi_k and phi_k^T v: 4*D*D').
     flops = B * H * N * D * p.Dp * 2.0 * (7 + 2)
     del y, nS, nL, ws, dy
-    return {"ms": ms, "calls": calls, "tflops": flops / (ms / 1e3) / 1e12,
-            "roofline": {"bound": "alu", "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
-                         "frac": flops / (ms / 1e3) / 1e12 / FP32_ALU_TFLOPS,
-                         "peak_source": "148 SMs x 128 fp32 FMA lanes x 2 x 1965 MHz"},
+    tflops = flops / (ms / 1e3) / 1e12
+    if D == 128 and p.Dp == 128:  # q and k passes on tcgen05 (bf16 operands)
+        peaks = load_peaks()
+        roof = {"bound": "tensor", "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": tflops / peaks["bf16_tflops"],
+                "peak_source": "measured bf16 burst (MEASURED_PEAKS.json)"}
+    else:
+        roof = {"bound": "alu", "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
+                "frac": tflops / FP32_ALU_TFLOPS,
+                "peak_source": "148 SMs x 128 fp32 FMA lanes x 2 x 1965 MHz"}
+    return {"ms": ms, "calls": calls, "tflops": tflops, "roofline": roof,
             "what": "rehyat_phi_bwd (dW_q, db_q, dW_k, db_k) on the bench workload, bf16 "
                     "q/k/v, fp32 y, dy, den; includes its state pass"}
 

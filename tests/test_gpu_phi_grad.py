@@ -4,9 +4,12 @@ against the fp64 gradient oracle on the same seeded inputs.
 Bar (per gradient tensor, error relative to its largest magnitude):
 * fp32 CUDA-core forward and state pass (force_simt): <= 1e-4 -- only fp32
   rounding separates the two;
-* default tensor-core forward and state pass, bf16 inputs: <= 3e-2 -- the
-  forward rounds P and phi_k to bf16 (relative 2^-9 per element), which
-  reaches y, the denominators and S_L that the gradient is built from.
+* default tensor-core path, bf16 inputs: <= 3e-2 -- the forward rounds P and
+  phi_k to bf16 (relative 2^-9 per element), which reaches y, the
+  denominators and S_L that the gradient is built from; with D = D' = 128
+  the backward's q and k passes run on tcgen05 too, with E = g / den, S_L,
+  Ghat, phi and du entering the products as bf16 (the same 2^-9 per element,
+  averaged over the sums over rows).
 """
 import numpy as np
 import pytest
@@ -119,3 +122,24 @@ def test_phi_grad_wan_320x480_causal_sampled_heads():
     heads = [0, 5, 11]
     got = _gpu_grads(p, dy, force_simt=True)
     _check(got, _ref(p, dy, heads), 1e-4, heads)
+
+
+def test_phi_grad_tensor_core_full_size_causal():
+    """Latent 21x20x30, 12 heads, D = D' = 128, causal, bf16: the tensor-core
+    forward and backward, three sampled heads against the oracle."""
+    p = config_problem("wan_320x480_causal")
+    dy = np.random.default_rng(12).standard_normal(np.shape(p.q)).astype(np.float32)
+    heads = [1, 6, 10]
+    got = _gpu_grads(p, dy, force_simt=False)
+    _check(got, _ref(p, dy, heads), 3e-2, heads)
+
+
+def test_phi_grad_tensor_core_bench_layer_sampled_heads():
+    """The bench layer (21x30x52, batch 2, 12 heads, bidirectional), bf16,
+    tensor-core path: two sampled heads (both batch elements) against the
+    oracle."""
+    p = config_problem("wan_480x832_bidir")
+    dy = np.random.default_rng(13).standard_normal(np.shape(p.q)).astype(np.float32)
+    heads = [3, 9]
+    got = _gpu_grads(p, dy, force_simt=False)
+    _check(got, _ref(p, dy, heads), 3e-2, heads)
