@@ -248,6 +248,52 @@ __global__ void phi_bwd_ghat_kernel(BwdParams P) {
   P.ghat[(static_cast<long long>(blockIdx.z) * P.T + s) * n + e] = acc;
 }
 
+// Pass 2 for up to kGhatRegChunks chunks: one thread per element e of one
+// (b*h, piece) forms every G_t[e] (the sum of its QS partials) once, then
+// writes Ghat_s[e] for every slice from those registers.
+// grid (ceil(n/256), BH*FP).
+constexpr int kGhatRegChunks = 32;
+
+__global__ void phi_bwd_ghat_reg_kernel(BwdParams P) {
+  const int D = P.D;
+  const long long n = static_cast<long long>(kPiece) * D + kPiece;
+  const long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (e >= n) return;
+  const long long psz = qpart_size(D);
+  const long long off = static_cast<long long>(D) * kPiece + kPiece + e;  // G, h block
+  float g[kGhatRegChunks];
+#pragma unroll
+  for (int t = 0; t < kGhatRegChunks; ++t) {
+    float acc = 0.f;
+    if (t < P.nchunks)
+      for (int qs = 0; qs < P.QS; ++qs)
+        acc += P.qpart[((static_cast<long long>(blockIdx.y) * P.nchunks + t) * P.QS + qs) * psz +
+                       off];
+    g[t] = acc;
+  }
+  for (int s = 0; s < P.T; ++s) {
+    float acc = 0.f;
+#pragma unroll
+    for (int t = 0; t < kGhatRegChunks; ++t) {
+      const int first = t * P.Tc, end = min(P.T, first + P.Tc);
+      const int w = max(first - P.To, 0);
+      const bool lin = P.causal ? s < w : (s < w || s >= end);
+      if (t < P.nchunks && lin) acc += g[t];
+    }
+    P.ghat[(static_cast<long long>(blockIdx.y) * P.T + s) * n + e] = acc;
+  }
+}
+
+// Ghat pass, either form.
+void launch_ghat(const BwdParams& bp, cudaStream_t s) {
+  const long long ng = static_cast<long long>(kPiece) * bp.D + kPiece;
+  const unsigned gx = static_cast<unsigned>((ng + 255) / 256);
+  if (bp.nchunks <= kGhatRegChunks)
+    phi_bwd_ghat_reg_kernel<<<dim3(gx, bp.BH * bp.FP), 256, 0, s>>>(bp);
+  else
+    phi_bwd_ghat_kernel<<<dim3(gx, bp.T, bp.BH * bp.FP), 256, 0, s>>>(bp);
+}
+
 // ---------------------------------------------------------------- pass 3
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1) phi_bwd_k_kernel(BwdParams P) {
@@ -376,9 +422,7 @@ cudaError_t launch_bwd_d(const BwdParams& bp, const PhiBwdArgs& a, cudaStream_t 
                            static_cast<int>(smk));
   if (e != cudaSuccess) return e;
   phi_bwd_q_kernel<D><<<dim3(bp.QS, bp.nchunks, bp.BH * bp.FP), kBwdThreads, smq, s>>>(bp);
-  const long long ng = static_cast<long long>(kPiece) * D + kPiece;
-  phi_bwd_ghat_kernel<<<dim3(static_cast<unsigned>((ng + 255) / 256), bp.T, bp.BH * bp.FP), 256,
-                        0, s>>>(bp);
+  launch_ghat(bp, s);
   phi_bwd_k_kernel<D><<<dim3(bp.KS, bp.T, bp.BH * bp.FP), kBwdThreads, smk, s>>>(bp);
   const long long nr = (static_cast<long long>(D) * bp.Dp + bp.Dp) * bp.heads;
   phi_bwd_reduce_kernel<<<dim3(static_cast<unsigned>((nr + 255) / 256), 2), 256, 0, s>>>(
@@ -429,9 +473,7 @@ cudaError_t launch_phi_bwd(const PhiBwdArgs& a, cudaStream_t s) {
     t.M = a.SL; t.vec = a.zL; t.part = bp.qpart; t.splits = bp.QS; t.q_side = 1;
     cudaError_t e = launch_phi_bwd_tc(t, s);
     if (e != cudaSuccess) return e;
-    const long long ng = static_cast<long long>(kPiece) * a.D + kPiece;
-    phi_bwd_ghat_kernel<<<dim3(static_cast<unsigned>((ng + 255) / 256), bp.T, bp.BH * bp.FP),
-                          256, 0, s>>>(bp);
+    launch_ghat(bp, s);
     t.x = a.k; t.v = a.v; t.w_img = a.wk_img; t.b = a.bk; t.M = bp.ghat; t.vec = nullptr;
     t.part = bp.kpart; t.splits = bp.KS; t.q_side = 0;
     e = launch_phi_bwd_tc(t, s);
