@@ -15,7 +15,9 @@
 // Passes (each CTA works on one feature piece of at most 128 features):
 //   1. q pass, per (b*h, piece, chunk, row range): u_q, dphi_q, du_q; partial
 //      dW_q, db_q, G_t, h_t of its rows;
-//   2. Ghat pass, per (b*h, piece, slice): Ghat_s, hhat_s from the partials;
+//   2. Ghat pass: G_t, h_t per chunk from its row-range partials, then per
+//      (b*h, piece, slice) Ghat_s, hhat_s as the sum over the chunks whose
+//      linear set holds the slice;
 //   3. k pass, per (b*h, piece, slice, row range): u_k, dphi_k, du_k; partial
 //      dW_k, db_k;
 //   4. reduction of the partials over the batch, chunks/slices and row
@@ -226,72 +228,48 @@ __global__ void __launch_bounds__(kBwdThreads, 1) phi_bwd_q_kernel(BwdParams P) 
 }
 
 // ---------------------------------------------------------------- pass 2
-// Ghat_s (and hhat_s) for slice s: the sum of G_t over chunks t whose linear
-// set holds s, each G_t the sum of its QS partials.  grid (ceil(n/256), T, BH*FP).
-__global__ void phi_bwd_ghat_kernel(BwdParams P) {
+// Pass 2 in two parallel steps.  (a) One thread per (element, chunk): G_t
+// (and h_t) as the sum of its QS partials, stored in place of partial 0.
+// grid (ceil(n/256), nchunks, BH*FP).
+__global__ void phi_bwd_gsum_kernel(BwdParams P) {
+  const int D = P.D;
+  const long long n = static_cast<long long>(kPiece) * D + kPiece;
+  const long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (e >= n) return;
+  const long long psz = qpart_size(D);
+  float* g = P.qpart + (static_cast<long long>(blockIdx.z) * P.nchunks + blockIdx.y) * P.QS * psz +
+             static_cast<long long>(D) * kPiece + kPiece + e;
+  float acc = 0.f;
+  for (int qs = 0; qs < P.QS; ++qs) acc += g[qs * psz];
+  g[0] = acc;
+}
+
+// (b) One thread per (element, slice): Ghat_s = the sum of G_t over the
+// chunks whose linear set holds s, in chunk order.  grid (ceil(n/256), T, BH*FP).
+__global__ void phi_bwd_gsel_kernel(BwdParams P) {
   const int D = P.D;
   const long long n = static_cast<long long>(kPiece) * D + kPiece;
   const long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (e >= n) return;
   const int s = blockIdx.y;
   const long long psz = qpart_size(D);
-  const long long off = static_cast<long long>(D) * kPiece + kPiece + e;  // G, h block
+  const float* g = P.qpart + static_cast<long long>(blockIdx.z) * P.nchunks * P.QS * psz +
+                   static_cast<long long>(D) * kPiece + kPiece + e;
   float acc = 0.f;
   for (int t = 0; t < P.nchunks; ++t) {
     const int first = t * P.Tc, end = min(P.T, first + P.Tc);
     const int w = max(first - P.To, 0);
-    const bool lin = P.causal ? s < w : (s < w || s >= end);
-    if (!lin) continue;
-    for (int qs = 0; qs < P.QS; ++qs)
-      acc += P.qpart[((static_cast<long long>(blockIdx.z) * P.nchunks + t) * P.QS + qs) * psz + off];
+    if (P.causal ? s < w : (s < w || s >= end)) acc += g[static_cast<long long>(t) * P.QS * psz];
   }
   P.ghat[(static_cast<long long>(blockIdx.z) * P.T + s) * n + e] = acc;
 }
 
-// Pass 2 for up to kGhatRegChunks chunks: one thread per element e of one
-// (b*h, piece) forms every G_t[e] (the sum of its QS partials) once, then
-// writes Ghat_s[e] for every slice from those registers.
-// grid (ceil(n/256), BH*FP).
-constexpr int kGhatRegChunks = 32;
-
-__global__ void phi_bwd_ghat_reg_kernel(BwdParams P) {
-  const int D = P.D;
-  const long long n = static_cast<long long>(kPiece) * D + kPiece;
-  const long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (e >= n) return;
-  const long long psz = qpart_size(D);
-  const long long off = static_cast<long long>(D) * kPiece + kPiece + e;  // G, h block
-  float g[kGhatRegChunks];
-#pragma unroll
-  for (int t = 0; t < kGhatRegChunks; ++t) {
-    float acc = 0.f;
-    if (t < P.nchunks)
-      for (int qs = 0; qs < P.QS; ++qs)
-        acc += P.qpart[((static_cast<long long>(blockIdx.y) * P.nchunks + t) * P.QS + qs) * psz +
-                       off];
-    g[t] = acc;
-  }
-  for (int s = 0; s < P.T; ++s) {
-    float acc = 0.f;
-#pragma unroll
-    for (int t = 0; t < kGhatRegChunks; ++t) {
-      const int first = t * P.Tc, end = min(P.T, first + P.Tc);
-      const int w = max(first - P.To, 0);
-      const bool lin = P.causal ? s < w : (s < w || s >= end);
-      if (t < P.nchunks && lin) acc += g[t];
-    }
-    P.ghat[(static_cast<long long>(blockIdx.y) * P.T + s) * n + e] = acc;
-  }
-}
-
-// Ghat pass, either form.
+// Ghat pass (both steps).
 void launch_ghat(const BwdParams& bp, cudaStream_t s) {
   const long long ng = static_cast<long long>(kPiece) * bp.D + kPiece;
   const unsigned gx = static_cast<unsigned>((ng + 255) / 256);
-  if (bp.nchunks <= kGhatRegChunks)
-    phi_bwd_ghat_reg_kernel<<<dim3(gx, bp.BH * bp.FP), 256, 0, s>>>(bp);
-  else
-    phi_bwd_ghat_kernel<<<dim3(gx, bp.T, bp.BH * bp.FP), 256, 0, s>>>(bp);
+  phi_bwd_gsum_kernel<<<dim3(gx, bp.nchunks, bp.BH * bp.FP), 256, 0, s>>>(bp);
+  phi_bwd_gsel_kernel<<<dim3(gx, bp.T, bp.BH * bp.FP), 256, 0, s>>>(bp);
 }
 
 // ---------------------------------------------------------------- pass 3

@@ -132,6 +132,11 @@ __global__ void __launch_bounds__(pb::kThreads, 1)
     // ================================================= TMA producer
     if (lane == 0) {
       bool ok = true;
+      // M (S_L of the chunk, or the Ghat block of the slice: contiguous) into
+      // L2 for the row warps converting it.
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(Msrc),
+                   "r"(static_cast<uint32_t>(kQ ? Dp * D * 4 : (128 * D + 128) * 4))
+                   : "memory");
       mbar_expect_tx(bar(pb::W_FULL), Dp * D * 2);
       bulk_load(base + kWOff, static_cast<const uint8_t*>(a.w_img) + static_cast<long long>(h) * Dp * D * 2,
                 Dp * D * 2, bar(pb::W_FULL));
@@ -142,6 +147,18 @@ __global__ void __launch_bounds__(pb::kThreads, 1)
         mbar_expect_tx(bar(pb::X_FULL), kQ ? 32768 : 65536);
         tma_load_3d(base + kXOff, &maps.x, bar(pb::X_FULL), 0, row, bh);
         tma_load_3d(base + kXOff + 16384, &maps.x, bar(pb::X_FULL), 64, row, bh);
+        if (kQ && tl + 1 < ntiles) {
+          // The next tile's g and y rows (contiguous, 512 bytes a row) into L2
+          // for the row warps that build E from them.
+          const long long nr0 = r0 + 128LL * (tl + 1);
+          const long long nrows = min(128LL, r1 - nr0);
+          const uint32_t bytes = static_cast<uint32_t>(nrows) * D * 4;
+          const long long gi = (static_cast<long long>(bh) * N + nr0) * D;
+          asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.dy + gi), "r"(bytes)
+                       : "memory");
+          asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.y + gi), "r"(bytes)
+                       : "memory");
+        }
         if (!kQ) {
           tma_load_3d(base + kEOff, &maps.v, bar(pb::X_FULL), 0, row, bh);
           tma_load_3d(base + kEOff + 16384, &maps.v, bar(pb::X_FULL), 64, row, bh);
@@ -208,6 +225,7 @@ __global__ void __launch_bounds__(pb::kThreads, 1)
     // operand [f][d] (thread r converts feature row r).
     bvec[r] = __ldg(a.b + static_cast<long long>(h) * Dp + r);
     bvec[128 + r] = __ldg(vsrc + r);
+#pragma unroll 4
     for (int d0 = 0; d0 < D; d0 += 8) {
       float m[8];
 #pragma unroll
@@ -230,6 +248,7 @@ __global__ void __launch_bounds__(pb::kThreads, 1)
         if (!ok) break;
         const long long gi = (static_cast<long long>(bh) * N + row) * D;
         const float inv = valid ? 1.f / __ldg(a.den + static_cast<long long>(bh) * N + row) : 0.f;
+#pragma unroll 2
         for (int d0 = 0; d0 < D; d0 += 8) {
           float4 g0 = make_float4(0.f, 0.f, 0.f, 0.f), g1 = g0, y0 = g0, y1 = g0;
           if (valid) {
