@@ -363,7 +363,7 @@ def hybrid_attn(q, k, v, Wq, bq, Wk, bk, *, T, Hs, Ws, Tc, To, causal, out_dtype
 
 
 def hybrid_attn_host(q, k, v, Wq, bq, Wk, bk, *, T, Hs, Ws, Tc, To, causal, out=None,
-                     heads_per_slab=2, workspace=None, stream=None):
+                     heads_per_slab=2, fp8_qk=False, workspace=None, stream=None):
     """hybrid_attn on CPU tensors q, k, v [B, h, N, D] (pin them for overlap):
     slabs of heads are uploaded, computed and downloaded concurrently by
     rehyat_hybrid_attn_fwd_host; the phi parameters are CUDA tensors.
@@ -373,7 +373,8 @@ def hybrid_attn_host(q, k, v, Wq, bq, Wk, bk, *, T, Hs, Ws, Tc, To, causal, out=
     B, H, N, D = q.shape
     Dp = 2 * Wq.shape[-1]
     p = make_params(batch=B, heads=H, T=T, Hs=Hs, Ws=Ws, D=D, Dp=Dp, Tc=Tc, To=To,
-                    causal=causal, in_dtype=_dtype_code(q.dtype), out_dtype=F32)
+                    causal=causal, in_dtype=_dtype_code(q.dtype), out_dtype=F32,
+                    flags=FLAG_FP8_QK if fp8_qk else 0)
     y = torch.empty(B, H, N, D, dtype=torch.float32, pin_memory=True) if out is None else out
     nbytes = rehyat_host_workspace_bytes(p, heads_per_slab)
     if nbytes == 0:

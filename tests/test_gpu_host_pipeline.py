@@ -81,3 +81,19 @@ def test_host_pipeline_refuses_short_workspace():
                                         h["v"].data_ptr(), phi, y.data_ptr(), 1, ws.data_ptr(),
                                         need - 256, None)
     assert st == 4  # REHYAT_ERR_WORKSPACE
+
+
+def test_host_pipeline_fp8_equals_device_fp8():
+    """REHYAT_FLAG_FP8_QK through the host-buffer forward: each slab's forward
+    makes its own E4M3 copies, bit-identical to the device fp8 forward."""
+    p = make_problem(batch=2, heads=3, T=5, Hs=7, Ws=9, D=128, Dp=128, Tc=2, To=1,
+                     causal=False, dtype="bf16", dist="scaled", seed=97)
+    dev = device_tensors(p)
+    kw = dict(T=p.T, Hs=p.Hs, Ws=p.Ws, Tc=p.Tc, To=p.To, causal=p.causal)
+    ref = rh.hybrid_attn(dev["q"], dev["k"], dev["v"], dev["Wq"], dev["bq"], dev["Wk"],
+                         dev["bk"], fp8_qk=True, **kw)
+    torch.cuda.synchronize()
+    host = {n: dev[n].cpu().pin_memory() for n in ("q", "k", "v")}
+    y = rh.hybrid_attn_host(host["q"], host["k"], host["v"], dev["Wq"], dev["bq"], dev["Wk"],
+                            dev["bk"], heads_per_slab=2, fp8_qk=True, **kw)
+    assert torch.equal(y, ref.cpu())
