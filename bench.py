@@ -833,6 +833,10 @@ def run_gpu(args, world, rank, local):
                 if peaks["source"] == "measured" else "fallback 1.59 PFLOP/s",
                 "work_per_launch": f"{w['attn_flops']:.4e} FLOP "
                                    f"(4*D per query-key pair in the window + phi_q + readout)"}
+    if peaks.get("bf16_tflops_sustained"):
+        # The same kernel against the seconds-long power-capped GEMM figure.
+        roofline["frac_of_sustained"] = achieved_tf / peaks["bf16_tflops_sustained"]
+        roofline["peak_sustained"] = peaks["bf16_tflops_sustained"]
     state_gbs = w["state_bytes"] / state_avg_s / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -846,6 +850,8 @@ def run_gpu(args, world, rank, local):
         "pct_bf16_peak": w["total_flops"] / (ms_per_step / 1e3) / 1e12 / peaks["bf16_tflops"],
         "stages_ms": {"state (per-slice + scan)": sum(state_ms) / len(state_ms),
                       "attention": sum(attn_ms) / len(attn_ms)},
+        "ms_per_step_median": sorted(step_ms)[len(step_ms) // 2],
+        "ms_per_step_min": min(step_ms),
         "state_stage_hbm": {"achieved": state_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                             "frac": state_gbs / peaks["hbm_gbs"],
                             "bytes_per_launch": w["state_bytes"]},
