@@ -311,10 +311,69 @@ def _stream_handle(stream=None) -> int:
     return s.cuda_stream
 
 
-def _phi_struct(Wq, bq, Wk, bk) -> RehyatPhi:
-    for t in (Wq, bq, Wk, bk):
-        if t.dtype != _torch().float32 or not t.is_cuda or not t.is_contiguous():
-            raise TypeError("phi parameters must be contiguous fp32 CUDA tensors")
+# The C ABI takes bare pointers and sizes: a tensor of the wrong shape,
+# strides or device would make the kernels read or write outside it.  The
+# torch layer therefore checks every tensor against the sizes it passes
+# before anything is launched.
+def _need(ok: bool, what: str, exc=ValueError):
+    if not ok:
+        raise exc(what)
+
+
+def _check_qkv(q, k, v, *, cuda=True):
+    """q, k, v: contiguous [B, h, N, D] tensors of one shape and dtype on one
+    device (a CUDA device for the device entry points, host memory for the
+    host-buffer forward)."""
+    _need(q.dim() == 4, "q must be a [B, h, N, D] tensor")
+    where = "CUDA tensors on one device" if cuda else "host (CPU) tensors"
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(tuple(t.shape) == tuple(q.shape), f"{name} must be shaped like q {tuple(q.shape)}")
+        _need(t.dtype == q.dtype, f"{name} must have q's dtype {q.dtype}", TypeError)
+        _need(t.is_contiguous(), f"{name} must be contiguous")
+        _need(t.is_cuda == cuda and t.device == q.device, f"q, k and v must be {where}")
+
+
+def _check_tokens(N, T, Hs, Ws):
+    _need(N == T * Hs * Ws, f"N = {N} tokens per head must equal T*Hs*Ws = {T * Hs * Ws}")
+
+
+def _check_out(t, shape, dtype, device, name="out"):
+    _need(tuple(t.shape) == tuple(shape), f"{name} must be shaped {tuple(shape)}")
+    _need(t.dtype == dtype, f"{name} must be {dtype}", TypeError)
+    _need(t.is_contiguous(), f"{name} must be contiguous")
+    _need(t.device == device, f"{name} must be on {device}")
+
+
+def _check_workspace(ws, device):
+    _need(ws.is_contiguous() and ws.device == device,
+          f"workspace must be a contiguous tensor on {device}")
+
+
+def _nbytes(t) -> int:
+    return t.numel() * t.element_size()
+
+
+def _check_params(named, sizes, device=None, what="phi parameters"):
+    """Each parameter tensor holds exactly its count of fp32 values, in a
+    contiguous CUDA tensor (on ``device`` when given)."""
+    torch = _torch()
+    for (name, t), n in zip(named, sizes):
+        _need(t.numel() == n, f"{name} must hold {n} values, not {t.numel()}")
+    for name, t in named:
+        _need(t.dtype == torch.float32 and t.is_cuda and t.is_contiguous(),
+              f"{what} must be contiguous fp32 CUDA tensors", TypeError)
+        _need(device is None or t.device == device, f"{name} must be on {device}")
+
+
+def _phi_struct(Wq, bq, Wk, bk, *, heads=None, D=None, Dp=None, device=None) -> RehyatPhi:
+    """phi_q, phi_k parameters: W [heads, 2, D, D'/2] and b [heads, 2, D'/2]
+    (heads x D x D' and heads x D' values) when the sizes are given."""
+    named = (("Wq", Wq), ("bq", bq), ("Wk", Wk), ("bk", bk))
+    if heads is None:
+        sizes = [t.numel() for _, t in named]
+    else:
+        sizes = [heads * D * Dp, heads * Dp, heads * D * Dp, heads * Dp]
+    _check_params(named, sizes, device)
     return RehyatPhi(Wq.data_ptr(), bq.data_ptr(), Wk.data_ptr(), bk.data_ptr())
 
 
@@ -337,26 +396,30 @@ def hybrid_attn(q, k, v, Wq, bq, Wk, bk, *, T, Hs, Ws, Tc, To, causal, out_dtype
     (REHYAT_FLAG_FP8_QK).  Returns y (and a dict of branch partials when
     ``debug``)."""
     torch = _torch()
+    _check_qkv(q, k, v)
     B, H, N, D = q.shape
-    if N != T * Hs * Ws:
-        raise ValueError("q.shape[2] must equal T*Hs*Ws")
+    _check_tokens(N, T, Hs, Ws)
     Dp = 2 * Wq.shape[-1]
+    phi = _phi_struct(Wq, bq, Wk, bk, heads=H, D=D, Dp=Dp, device=q.device)
     out_dtype = torch.float32 if out_dtype is None else out_dtype
     p = make_params(batch=B, heads=H, T=T, Hs=Hs, Ws=Ws, D=D, Dp=Dp, Tc=Tc, To=To,
                     causal=causal, in_dtype=_dtype_code(q.dtype),
                     out_dtype=_dtype_code(out_dtype), scale=scale,
                     flags=(FLAG_FORCE_SIMT if force_simt else 0) |
                     (FLAG_ONE_TILE if one_tile else 0) | (FLAG_FP8_QK if fp8_qk else 0))
+    if out is not None:
+        _check_out(out, (B, H, N, D), out_dtype, q.device)
     y = torch.empty(B, H, N, D, dtype=out_dtype, device=q.device) if out is None else out
     nbytes = rehyat_workspace_bytes(p)
     if nbytes == 0:
         raise RehyatError(1, "rehyat_workspace_bytes")
-    if workspace is None or workspace.numel() < nbytes:
+    if workspace is not None:
+        _check_workspace(workspace, q.device)
+    if workspace is None or _nbytes(workspace) < nbytes:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
     dbg_t, dbg_s = _debug_tensors((B, H, N, D), q.device) if debug else (None, None)
-    st = rehyat_hybrid_attn_fwd(p, q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                                _phi_struct(Wq, bq, Wk, bk), y.data_ptr(),
-                                workspace.data_ptr(), workspace.numel(), dbg_s,
+    st = rehyat_hybrid_attn_fwd(p, q.data_ptr(), k.data_ptr(), v.data_ptr(), phi, y.data_ptr(),
+                                workspace.data_ptr(), _nbytes(workspace), dbg_s,
                                 _stream_handle(stream))
     _check(st, "rehyat_hybrid_attn_fwd")
     return (y, dbg_t) if debug else y
@@ -370,21 +433,27 @@ def hybrid_attn_host(q, k, v, Wq, bq, Wk, bk, *, T, Hs, Ws, Tc, To, causal, out=
     Returns y (fp32, CPU; `out` if given), valid after `stream` syncs (this
     function synchronises it)."""
     torch = _torch()
+    _check_qkv(q, k, v, cuda=False)
     B, H, N, D = q.shape
+    _check_tokens(N, T, Hs, Ws)
     Dp = 2 * Wq.shape[-1]
+    phi = _phi_struct(Wq, bq, Wk, bk, heads=H, D=D, Dp=Dp)
     p = make_params(batch=B, heads=H, T=T, Hs=Hs, Ws=Ws, D=D, Dp=Dp, Tc=Tc, To=To,
                     causal=causal, in_dtype=_dtype_code(q.dtype), out_dtype=F32,
                     flags=FLAG_FP8_QK if fp8_qk else 0)
+    if out is not None:
+        _check_out(out, (B, H, N, D), torch.float32, q.device)
     y = torch.empty(B, H, N, D, dtype=torch.float32, pin_memory=True) if out is None else out
     nbytes = rehyat_host_workspace_bytes(p, heads_per_slab)
     if nbytes == 0:
         raise RehyatError(1, "rehyat_host_workspace_bytes")
-    if workspace is None or workspace.numel() < nbytes:
+    if workspace is not None:
+        _check_workspace(workspace, Wq.device)
+    if workspace is None or _nbytes(workspace) < nbytes:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=Wq.device)
-    st = rehyat_hybrid_attn_fwd_host(p, q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                                     _phi_struct(Wq, bq, Wk, bk), y.data_ptr(), heads_per_slab,
-                                     workspace.data_ptr(), workspace.numel(),
-                                     _stream_handle(stream))
+    st = rehyat_hybrid_attn_fwd_host(p, q.data_ptr(), k.data_ptr(), v.data_ptr(), phi,
+                                     y.data_ptr(), heads_per_slab, workspace.data_ptr(),
+                                     _nbytes(workspace), _stream_handle(stream))
     _check(st, "rehyat_hybrid_attn_fwd_host")
     (stream or torch.cuda.current_stream()).synchronize()
     return y
@@ -397,19 +466,25 @@ def feature_map_mlp(x, Wa, ba, Wb, bb, *, parts, T, Hs, Ws, stream=None, force_s
     Wb [h, Dh, D'], bb [h, D'] fp32.  Returns fp32 [B, h, N, D'].  bf16 x with
     D = 128 runs on the tensor cores (bf16 operands) unless force_simt."""
     torch = _torch()
+    _need(x.dim() == 4, "x must be a [B, h, N, D] tensor")
+    _need(x.is_contiguous() and x.is_cuda, "x must be a contiguous CUDA tensor")
     B, H, N, D = x.shape
+    _check_tokens(N, T, Hs, Ws)
     Dh, Dp = Wa.shape[-1], Wb.shape[-1]
-    for t in (Wa, ba, Wb, bb):
-        if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous():
-            raise TypeError("MLP parameters must be contiguous fp32 CUDA tensors")
+    _check_params((("Wa", Wa), ("ba", ba), ("Wb", Wb), ("bb", bb)),
+                  (H * D * Dh, H * Dh, H * Dh * Dp, H * Dp), x.device, "MLP parameters")
     p = make_params(batch=B, heads=H, T=T, Hs=Hs, Ws=Ws, D=D, Dp=Dp, Tc=1, To=0, causal=0,
                     in_dtype=_dtype_code(x.dtype), out_dtype=F32,
                     flags=FLAG_FORCE_SIMT if force_simt else 0)
+    if out is not None:
+        _check_out(out, (B, H, N, Dp), torch.float32, x.device)
     phi = out if out is not None else torch.empty(B, H, N, Dp, dtype=torch.float32,
                                                   device=x.device)
     mlp = RehyatPhiMlp(Wa.data_ptr(), ba.data_ptr(), Wb.data_ptr(), bb.data_ptr(), Dh, parts)
     nbytes = rehyat_feature_map_mlp_workspace_bytes(p, mlp, x.data_ptr(), phi.data_ptr())
-    if nbytes and (workspace is None or workspace.numel() < nbytes):
+    if nbytes and workspace is not None:
+        _check_workspace(workspace, x.device)
+    if nbytes and (workspace is None or _nbytes(workspace) < nbytes):
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=x.device)
     ws_ptr = workspace.data_ptr() if nbytes else None
     _check(rehyat_feature_map_mlp(p, x.data_ptr(), mlp, phi.data_ptr(), ws_ptr, nbytes,
@@ -424,26 +499,34 @@ def hybrid_attn_phi(q, k, v, phi_q, phi_k, *, T, Hs, Ws, Tc, To, causal, out_dty
     phi_k = phi_k(k), fp32 [B, h, N, D'] CUDA tensors.  Returns y (and the
     branch partials when ``debug``)."""
     torch = _torch()
+    _check_qkv(q, k, v)
     B, H, N, D = q.shape
+    _check_tokens(N, T, Hs, Ws)
     Dp = phi_q.shape[-1]
     for t in (phi_q, phi_k):
-        if t.dtype != torch.float32 or not t.is_contiguous() or t.shape[:3] != q.shape[:3]:
+        if (t.dtype != torch.float32 or not t.is_contiguous() or t.dim() != 4
+                or tuple(t.shape) != (B, H, N, Dp)):
             raise TypeError("phi_q, phi_k must be contiguous fp32 [B, h, N, D'] tensors")
+        _need(t.device == q.device, "phi_q, phi_k must be on q's device")
     out_dtype = torch.float32 if out_dtype is None else out_dtype
     p = make_params(batch=B, heads=H, T=T, Hs=Hs, Ws=Ws, D=D, Dp=Dp, Tc=Tc, To=To,
                     causal=causal, in_dtype=_dtype_code(q.dtype),
                     out_dtype=_dtype_code(out_dtype), scale=scale,
                     flags=FLAG_FORCE_SIMT if force_simt else 0)
+    if out is not None:
+        _check_out(out, (B, H, N, D), out_dtype, q.device)
     y = torch.empty(B, H, N, D, dtype=out_dtype, device=q.device) if out is None else out
     nbytes = rehyat_workspace_bytes(p)
     if nbytes == 0:
         raise RehyatError(1, "rehyat_workspace_bytes")
+    if workspace is not None:
+        _check_workspace(workspace, q.device)
     if workspace is None:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
     dbg_t, dbg_s = _debug_tensors((B, H, N, D), q.device) if debug else (None, None)
     st = rehyat_hybrid_attn_fwd_phi(p, q.data_ptr(), k.data_ptr(), v.data_ptr(),
                                     phi_q.data_ptr(), phi_k.data_ptr(), y.data_ptr(),
-                                    workspace.data_ptr(), workspace.numel(), dbg_s,
+                                    workspace.data_ptr(), _nbytes(workspace), dbg_s,
                                     _stream_handle(stream))
     _check(st, "rehyat_hybrid_attn_fwd_phi")
     return (y, dbg_t) if debug else y
@@ -456,25 +539,33 @@ def phi_grad(q, k, v, y, dy, den, Wq, bq, Wk, bk, *, T, Hs, Ws, Tc, To, causal, 
     query (``parts["nS"] + parts["nL"]`` of ``hybrid_attn(..., debug=True)``).
     Returns dict(dWq, dbq, dWk, dbk) shaped like the parameters."""
     torch = _torch()
+    _check_qkv(q, k, v)
     B, H, N, D = q.shape
+    _check_tokens(N, T, Hs, Ws)
     Dp = 2 * Wq.shape[-1]
     for t in (y, dy, den):
         if t.dtype != torch.float32 or not t.is_contiguous():
             raise TypeError("y, dy and den must be contiguous fp32 tensors")
+    _check_out(y, (B, H, N, D), torch.float32, q.device, "y")
+    _check_out(dy, (B, H, N, D), torch.float32, q.device, "dy")
+    _check_out(den, (B, H, N), torch.float32, q.device, "den")
+    phi = _phi_struct(Wq, bq, Wk, bk, heads=H, D=D, Dp=Dp, device=q.device)
     p = make_params(batch=B, heads=H, T=T, Hs=Hs, Ws=Ws, D=D, Dp=Dp, Tc=Tc, To=To,
                     causal=causal, in_dtype=_dtype_code(q.dtype), out_dtype=F32, scale=scale,
                     flags=FLAG_FORCE_SIMT if force_simt else 0)
     nbytes = rehyat_phi_bwd_workspace_bytes(p)
     if nbytes == 0:
         raise RehyatError(1, "rehyat_phi_bwd_workspace_bytes")
+    if workspace is not None:
+        _check_workspace(workspace, q.device)
     if workspace is None:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
-    g = {name: torch.empty_like(t) for name, t in
+    g = {name: torch.empty_like(t, memory_format=torch.contiguous_format) for name, t in
          (("dWq", Wq), ("dbq", bq), ("dWk", Wk), ("dbk", bk))}
     grad = RehyatPhiGrad(*(g[n].data_ptr() for n in ("dWq", "dbq", "dWk", "dbk")))
     st = rehyat_phi_bwd(p, q.data_ptr(), k.data_ptr(), v.data_ptr(), y.data_ptr(), dy.data_ptr(),
-                        den.data_ptr(), _phi_struct(Wq, bq, Wk, bk), grad, workspace.data_ptr(),
-                        workspace.numel(), _stream_handle(stream))
+                        den.data_ptr(), phi, grad, workspace.data_ptr(), _nbytes(workspace),
+                        _stream_handle(stream))
     _check(st, "rehyat_phi_bwd")
     return g
 
@@ -483,11 +574,14 @@ def softmax_attn(q, k, v, *, out_dtype=None, scale=0.0, force_simt=False, out=No
                  stream=None):
     """Plain softmax attention over all keys (the dense comparator)."""
     torch = _torch()
+    _check_qkv(q, k, v)
     B, H, N, D = q.shape
     out_dtype = torch.float32 if out_dtype is None else out_dtype
     p = make_params(batch=B, heads=H, T=1, Hs=1, Ws=N, D=D, Dp=32, Tc=1, To=0, causal=0,
                     in_dtype=_dtype_code(q.dtype), out_dtype=_dtype_code(out_dtype),
                     scale=scale, flags=FLAG_FORCE_SIMT if force_simt else 0)
+    if out is not None:
+        _check_out(out, (B, H, N, D), out_dtype, q.device)
     y = torch.empty(B, H, N, D, dtype=out_dtype, device=q.device) if out is None else out
     st = rehyat_softmax_attn_fwd(p, q.data_ptr(), k.data_ptr(), v.data_ptr(), y.data_ptr(),
                                  _stream_handle(stream))
@@ -512,8 +606,10 @@ class StreamingState:
                              To=To, causal=1, in_dtype=_dtype_code(in_dtype),
                              out_dtype=_dtype_code(self.out_dtype), scale=scale,
                              flags=FLAG_FORCE_SIMT if force_simt else 0)
+        self.shape = (batch, heads, D)
+        self.in_dtype = in_dtype
         self.phi_tensors = (Wq, bq, Wk, bk)
-        self.phi = _phi_struct(Wq, bq, Wk, bk)
+        self.phi = _phi_struct(Wq, bq, Wk, bk, heads=heads, D=D, Dp=Dp)
         nstate = rehyat_state_bytes(self.p)
         nws = rehyat_step_workspace_bytes(self.p)
         if nstate == 0 or nws == 0:
@@ -528,10 +624,17 @@ class StreamingState:
 
     def step(self, q, k, v, *, debug=False, out=None, stream=None):
         torch = _torch()
+        _check_qkv(q, k, v)
         B, H, rows, D = q.shape
+        _need((B, H, D) == self.shape, f"a chunk must be shaped [{self.shape[0]}, "
+              f"{self.shape[1]}, rows, {self.shape[2]}]")
+        _need(q.dtype == self.in_dtype, f"a chunk must be {self.in_dtype}", TypeError)
+        _need(q.device == self.state.device, f"a chunk must be on {self.state.device}")
         n = rows // self.HW
         if n * self.HW != rows:
             raise ValueError("a chunk must hold whole slices")
+        if out is not None:
+            _check_out(out, (B, H, rows, D), self.out_dtype, q.device)
         y = torch.empty(B, H, rows, D, dtype=self.out_dtype, device=q.device) if out is None else out
         dbg_t, dbg_s = _debug_tensors((B, H, rows, D), q.device) if debug else (None, None)
         st = rehyat_chunk_step(self.p, q.data_ptr(), k.data_ptr(), v.data_ptr(), n, self.phi,

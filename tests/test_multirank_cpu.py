@@ -37,7 +37,7 @@ def _worker(rank, world, port, times, out):
 def test_max_over_ranks_and_throughput_world_2():
     world = 2
     times = [12.5, 17.25]  # ms of device time per rank
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()  # no fork of a threaded process
     out = mgr.dict()
     mp.spawn(_worker, args=(world, _free_port(), times, out), nprocs=world, join=True)
     for rank in range(world):
