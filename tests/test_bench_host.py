@@ -1,0 +1,82 @@
+"""Host logic of bench.py's reference arm (the fp64 oracle timed on the host
+cores), on CPU: the JSON line it prints, its token accounting and its rank
+handling.  The workload is shrunk so that each test takes seconds."""
+import argparse
+import json
+
+import pytest
+
+import bench
+import rehyat_inputs
+from rehyat_inputs import make_problem
+
+TINY = dict(batch=1, heads=3, T=5, Hs=3, Ws=4, D=32, Dp=32, Tc=2, To=1, causal=False,
+            dtype="bf16")
+
+
+@pytest.fixture
+def small_workload(monkeypatch):
+    orig = rehyat_inputs.config_problem
+    monkeypatch.setattr(rehyat_inputs, "config_problem",
+                        lambda name, **kw: orig(name, **dict(kw, batch=1, heads=2, T=4, Hs=3,
+                                                             Ws=5, Tc=2, To=1)))
+
+
+def test_reference_line_keys_and_arithmetic(monkeypatch, capsys, small_workload):
+    seen = []
+
+    def fake_run(p, plan, start_head=0):
+        seen.append(start_head)
+        return dict(seconds=0.5, token_equiv=1000.0, sample="stub sample")
+
+    monkeypatch.setattr(bench, "plan_oracle_sample", lambda p, budget: dict(heads=1, chunks=1))
+    monkeypatch.setattr(bench, "run_oracle_sample", fake_run)
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    monkeypatch.delenv("RANK", raising=False)
+    assert bench.main(["--impl", "reference", "--steps", "4", "--warmup", "0"]) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert seen == list(range(7))          # 3 warm-up samples (the minimum), then 4 timed
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC
+    assert line["unit"] == "tokens/s" and line["higher_is_better"] is True
+    assert line["steps"] == 4 and line["warmup"] == 3 and line["n_gpus"] == 1
+    assert line["value"] == pytest.approx(2000.0)              # 4000 tokens in 2 s
+    assert line["ms_per_step"] == pytest.approx(500.0)
+    assert line["dtype"] == "f64" and line["data"] == "synthetic"
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1
+    assert "stub sample" in cb["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": "tokens/s",
+                           "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert line["config"]["workload"].startswith(bench.WORKLOAD)
+
+
+def test_reference_arm_other_ranks_do_no_work(monkeypatch, capsys):
+    def boom(*a, **k):
+        raise AssertionError("a non-zero rank ran the oracle")
+
+    monkeypatch.setattr(bench, "plan_oracle_sample", boom)
+    monkeypatch.setattr(bench, "run_oracle_sample", boom)
+    args = argparse.Namespace(steps=2, warmup=3, gpus=2)
+    assert bench.run_reference(args, 2, 1) == 0
+    assert capsys.readouterr().out == ""
+
+
+def test_oracle_sample_accounting_and_head_rotation():
+    p = make_problem(seed=5, **TINY)
+    BH = p.batch * p.heads
+    r = bench.run_oracle_sample(p, dict(heads=2, chunks=2), start_head=BH - 1)
+    rows = 2 * p.Tc * p.HW                 # chunks 0 and 1 hold T_c slices each
+    assert r["token_equiv"] == pytest.approx(rows * 2 / p.heads)
+    assert r["seconds"] > 0
+    assert r["sample"].startswith(f"2 of {BH} (batch, head) pairs x chunks 0..1 of 3")
+    # The ragged last chunk (one slice) counts its own rows.
+    r = bench.run_oracle_sample(p, dict(heads=1, chunks=3))
+    assert r["token_equiv"] == pytest.approx(p.T * p.HW / p.heads)
+
+
+def test_oracle_sample_plan_stays_in_budget():
+    p = make_problem(seed=6, **TINY)
+    tight = bench.plan_oracle_sample(p, 0.0)
+    assert tight["heads"] == 1 and tight["chunks"] >= 1
+    roomy = bench.plan_oracle_sample(p, 1e6)
+    assert roomy == dict(heads=p.batch * p.heads, chunks=3)
