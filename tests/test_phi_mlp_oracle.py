@@ -1,6 +1,7 @@
 """Pins of the general feature map and of the phi-given forward oracle
 (oracle/rehyat_phi_mlp.py), CPU only.
 
+* a hand-worked map (D = 2, D_h = 3, D' = 2) in terms of the normal CDF;
 * GELU against scipy.stats.norm.cdf (x * Phi(x)) and its odd part
   gelu(x) - gelu(-x) = x;
 * the P-part powers: part i of phi equals the i-th power of part i of the
@@ -23,6 +24,32 @@ def test_gelu_matches_normal_cdf_and_odd_part():
     assert np.allclose(gelu(x), x * norm.cdf(x), rtol=1e-13, atol=1e-15)
     assert np.allclose(gelu(x) - gelu(-x), x, rtol=1e-13, atol=1e-14)
     assert gelu(0.0) == 0.0
+
+
+def test_feature_map_mlp_hand_example():
+    """psi = GELU(x W_a + b_a) W_b + b_b worked by hand for D = 2, D_h = 3,
+    D' = 2 (non-square weights, non-zero biases), GELU(u) = u Phi(u):
+
+      row 1, x = (1, -2):    u = (1 + 0.5, 2, 2 - 1 - 1) = (1.5, 2, 0)
+        psi = (1.5 Phi(1.5) + 0.5 * 2 Phi(2) + 0.25,  -1.5 Phi(1.5) + 3 * 0 - 0.5)
+      row 2, x = (0.5, 0.25): u = (0.5 + 0.5, -0.25, 1 + 0.125 - 1) = (1, -0.25, 0.125)
+        psi = (Phi(1) + 0.5 * (-0.25) Phi(-0.25) + 0.25,
+               -Phi(1) + 3 * 0.125 Phi(0.125) - 0.5)
+
+    P = 2 keeps part 1 and squares part 2."""
+    x = np.array([[1.0, -2.0], [0.5, 0.25]])
+    Wa = np.array([[1.0, 0.0, 2.0], [0.0, -1.0, 0.5]])
+    ba = np.array([0.5, 0.0, -1.0])
+    Wb = np.array([[1.0, -1.0], [0.5, 0.0], [0.0, 3.0]])
+    bb = np.array([0.25, -0.5])
+    F = norm.cdf
+    psi = np.array([
+        [1.5 * F(1.5) + 0.5 * 2.0 * F(2.0) + 0.25, -1.5 * F(1.5) - 0.5],
+        [F(1.0) + 0.5 * (-0.25) * F(-0.25) + 0.25, -F(1.0) + 3.0 * 0.125 * F(0.125) - 0.5],
+    ])
+    np.testing.assert_allclose(feature_map_mlp(x, Wa, ba, Wb, bb, 1), psi, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(feature_map_mlp(x, Wa, ba, Wb, bb, 2),
+                               np.stack([psi[:, 0], psi[:, 1] ** 2], axis=1), rtol=0, atol=1e-14)
 
 
 @pytest.mark.parametrize("P", [1, 2, 4])
