@@ -25,8 +25,12 @@
  * Conventions shared by every entry point:
  *   - Ownership: the caller allocates and owns every buffer (inputs, outputs,
  *     phi parameters, workspace, streaming state).  The library never
- *     allocates, frees or synchronises; all work is enqueued on `stream`
- *     (a cudaStream_t passed as void*; NULL = the legacy default stream).
+ *     allocates device memory, frees or synchronises; all work is enqueued on
+ *     `stream` (a cudaStream_t passed as void*; NULL = the legacy default
+ *     stream).  Exceptions, stated at each: rehyat_hybrid_attn_fwd_host
+ *     creates two copy streams per device on first use (kept for the life of
+ *     the process) and a few events per call; rehyat_device_error_flags
+ *     synchronises the device.
  *   - All pointers are device pointers unless stated, 16-byte aligned.
  *   - Errors: arguments are checked before any launch; a bad argument
  *     returns a status and enqueues nothing.  A launch failure returns
@@ -257,7 +261,10 @@ REHYAT_API size_t rehyat_host_workspace_bytes(const rehyat_params* p, int heads_
  * valid on the host.  The copy streams are created on first use per device
  * and kept.  Results equal rehyat_hybrid_attn_fwd's bit for bit.  Errors as
  * for rehyat_hybrid_attn_fwd; REHYAT_ERR_WORKSPACE if ws_bytes <
- * rehyat_host_workspace_bytes; workspace 16-byte aligned. */
+ * rehyat_host_workspace_bytes; workspace 16-byte aligned.  A slab refused or
+ * failed after its upload was enqueued returns that status with `stream`
+ * still made to wait for every copy already enqueued, so synchronising
+ * `stream` before reusing the host buffers is enough on every path. */
 REHYAT_API rehyat_status rehyat_hybrid_attn_fwd_host(const rehyat_params* p, const void* q,
                                                      const void* k, const void* v,
                                                      const rehyat_phi* phi, void* y,

@@ -173,10 +173,15 @@ rehyat_status rehyat_hybrid_attn_fwd_host(const rehyat_params* p, const void* q,
                           cudaMemcpyDeviceToHost, down);
     if (e == cudaSuccess) e = cudaEventRecord(drained[slot], down);
   }
-  // The caller's stream ends after the last download.
-  if (e == cudaSuccess && st == REHYAT_OK) {
-    e = cudaEventRecord(start, down);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, start, 0);
+  // The caller's stream ends after the last upload and the last download,
+  // on an error too, so that synchronising it covers every copy this call
+  // enqueued (a refused or failed slab may leave an upload in flight).
+  if (made > 0) {
+    cudaError_t j = cudaEventRecord(start, up);
+    if (j == cudaSuccess) j = cudaStreamWaitEvent(s, start, 0);
+    if (j == cudaSuccess) j = cudaEventRecord(start, down);
+    if (j == cudaSuccess) j = cudaStreamWaitEvent(s, start, 0);
+    if (e == cudaSuccess) e = j;
   }
   // Events may be destroyed with work pending; their resources are released
   // once it completes.
