@@ -80,7 +80,8 @@ typedef enum { REHYAT_F32 = 0, REHYAT_BF16 = 1 } rehyat_dtype;
                                     tensor cores (kind::f8f6f4); P.V, the feature
                                     maps and the linear branch keep bf16.  Full
                                     forward only (rehyat_hybrid_attn_fwd, the
-                                    split stages, the host-buffer forward), bf16
+                                    split stages, the no-alloc and host-buffer
+                                    variants), bf16
                                     inputs, D = 128, Dp <= 128; every other entry
                                     point returns REHYAT_ERR_UNSUPPORTED with it.
                                     The workspace grows by the two E4M3 copies

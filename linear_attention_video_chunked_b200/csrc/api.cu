@@ -238,6 +238,7 @@ rehyat_status mlp_args(const rehyat_params* p, const void* x, const rehyat_phi_m
                        float* phi, PhiMlpArgs* a) {
   rehyat_status st = check_params(p);
   if (st != REHYAT_OK) return st;
+  if ((st = no_fp8(p)) != REHYAT_OK) return st;
   if (!x || !mlp || !phi || !mlp->Wa || !mlp->ba || !mlp->Wb || !mlp->bb)
     return REHYAT_ERR_INVALID_ARG;
   if (mlp->parts < 1 || p->Dp % mlp->parts != 0 || mlp->Dh < 1) return REHYAT_ERR_INVALID_ARG;

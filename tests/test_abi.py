@@ -132,3 +132,83 @@ def test_softmax_entry_checks():
     p = _params()
     assert rh.rehyat_softmax_attn_fwd(p, 0, 16, 16, 16, None) == 1
     assert rh.rehyat_softmax_attn_fwd(p, 24, 16, 16, 16, None) == 3
+
+
+def test_split_stage_argument_checks():
+    p = _params()
+    phi = rh.RehyatPhi(4096, 4096, 4096, 4096)
+    ws = rh.rehyat_workspace_bytes(p)
+    state, attn = rh.rehyat_fwd_state, rh.rehyat_fwd_attn
+    assert state(p, 0, 4096, phi, 4096, ws, None) == 1                  # null k
+    assert state(p, 4096, 4096, rh.RehyatPhi(4096, 4096, 0, 4096), 4096, ws, None) == 1
+    assert state(p, 4096, 4104, phi, 4096, ws, None) == 3               # misaligned v
+    assert state(p, 4096, 4096, phi, 4096, ws - 1, None) == 4
+    assert attn(p, 4096, 4096, 4096, phi, 0, 4096, ws, None, None) == 1  # null y
+    assert attn(p, 4096, 4096, 4096, phi, 4096, 4100, ws, None, None) == 3
+    assert attn(p, 4096, 4096, 4096, phi, 4096, 4096, ws - 1, None, None) == 4
+    assert attn(_params(batch=0), 4096, 4096, 4096, phi, 4096, 4096, ws, None, None) == 1
+
+
+def _mlp(parts=2, Dh=256, ptrs=(4096, 4096, 4096, 4096)):
+    return rh.RehyatPhiMlp(*ptrs, Dh, parts)
+
+
+def test_feature_map_argument_checks():
+    p = _params()
+    f = rh.rehyat_feature_map_mlp
+    assert f(p, 4096, _mlp(parts=0), 4096, None, 0, None) == 1
+    assert f(p, 4096, _mlp(parts=3), 4096, None, 0, None) == 1          # D' = 128 not in 3 parts
+    assert f(p, 4096, _mlp(Dh=0), 4096, None, 0, None) == 1
+    assert f(p, 4096, _mlp(Dh=640), 4096, None, 0, None) == 2           # D_h > 512
+    assert f(p, 0, _mlp(), 4096, None, 0, None) == 1                    # null x
+    assert f(p, 4096, _mlp(), 0, None, 0, None) == 1                    # null phi
+    assert f(p, 4096, _mlp(ptrs=(4096, 0, 4096, 4096)), 4096, None, 0, None) == 1  # null b_a
+    assert f(p, 4098, _mlp(), 4096, None, 0, None) == 3                 # x not 4-byte aligned
+    assert f(p, 4096, _mlp(ptrs=(4096, 4096, 4096, 4097)), 4096, None, 0, None) == 3
+    assert f(_params(T=0), 4096, _mlp(), 4096, None, 0, None) == 1
+    # The fp8 flag belongs to the softmax branch of the full forward only.
+    fp8 = _params(flags=rh.FLAG_FP8_QK)
+    assert f(fp8, 4096, _mlp(), 4096, None, 0, None) == 2
+    assert rh.rehyat_feature_map_mlp_workspace_bytes(fp8, _mlp(), 4096, 4096) == 0
+    assert rh.rehyat_feature_map_mlp_workspace_bytes(p, _mlp(parts=0), 4096, 4096) == 0
+
+
+def test_phi_given_forward_argument_checks():
+    p = _params()
+    ws = rh.rehyat_workspace_bytes(p)
+    f = rh.rehyat_hybrid_attn_fwd_phi
+    assert f(p, 4096, 4096, 4096, 0, 4096, 4096, 4096, ws, None, None) == 1     # null phi_q
+    assert f(p, 4096, 4096, 4096, 4096, 0, 4096, 4096, ws, None, None) == 1     # null phi_k
+    assert f(p, 4096, 4096, 4096, 4100, 4096, 4096, 4096, ws, None, None) == 3  # phi_q
+    assert f(p, 4096, 4096, 4096, 4096, 4096, 4096, 4096, ws - 1, None, None) == 4
+    dbg = rh.RehyatDebug(4096, 4098, 0, 0, 0)
+    assert f(p, 4096, 4096, 4096, 4096, 4096, 4096, 4096, ws, dbg, None) == 3
+    assert f(_params(flags=rh.FLAG_FP8_QK), 4096, 4096, 4096, 4096, 4096, 4096, 4096, ws,
+             None, None) == 2
+
+
+def test_phi_backward_argument_checks():
+    p = _params()
+    phi = rh.RehyatPhi(4096, 4096, 4096, 4096)
+    grad = rh.RehyatPhiGrad(4096, 4096, 4096, 4096)
+    ws = rh.rehyat_phi_bwd_workspace_bytes(p)
+    assert ws > rh.rehyat_workspace_bytes(p)      # the forward's state plus the partials
+    f = rh.rehyat_phi_bwd
+    args = [p, 4096, 4096, 4096, 4096, 4096, 4096, phi, grad, 4096, ws, None]
+
+    def call(**change):
+        a = list(args)
+        for i, val in change.items():
+            a[int(i[1:])] = val
+        return f(*a)
+
+    assert call(a6=0) == 1                                               # null den
+    assert call(a8=rh.RehyatPhiGrad(4096, 0, 4096, 4096)) == 1           # null db_q
+    assert call(a7=rh.RehyatPhi(0, 4096, 4096, 4096)) == 1               # null W_q
+    assert call(a5=4100) == 3                                            # dy not 16-byte aligned
+    assert call(a6=4098) == 3                                            # den not 4-byte aligned
+    assert call(a8=rh.RehyatPhiGrad(4096, 4096, 4097, 4096)) == 3
+    assert call(a10=ws - 1) == 4
+    assert call(a0=_params(flags=rh.FLAG_FP8_QK)) == 2
+    assert rh.rehyat_phi_bwd_workspace_bytes(_params(flags=rh.FLAG_FP8_QK)) == 0
+    assert rh.rehyat_phi_bwd_workspace_bytes(_params(heads=0)) == 0
