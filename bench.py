@@ -187,6 +187,29 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------- CPU oracle
+def host_info():
+    """CPU model and the BLAS library the oracle's numpy runs on (for the
+    CPU baseline's record); fields it cannot read are left out."""
+    info = {}
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    info["cpu"] = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        from threadpoolctl import threadpool_info
+        libs = [f"{i.get('internal_api', '?')} {i.get('version', '')}".strip()
+                for i in threadpool_info() if i.get("user_api") == "blas"]
+        if libs:
+            info["blas"] = ", ".join(sorted(set(libs)))
+    except Exception:
+        pass
+    return info
+
+
 def blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -671,7 +694,7 @@ def run_reference(args, world, rank):
                    "parallelism": "none (host cores)"},
         "tflops": w["total_flops"] / (p.batch * p.N) * value / 1e12,
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": f"per step: {samples[0]}"},
+                         "sample": f"per step: {samples[0]}", "host": host_info()},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -874,7 +897,7 @@ def run_gpu(args, world, rank, local):
         cv = r["token_equiv"] / r["seconds"]
         line["cpu_baseline"] = {"value": cv, "unit": "tokens/s", "cores": blas_threads(),
                                 "kind": "oracle", "sample": r["sample"],
-                                "seconds": r["seconds"]}
+                                "seconds": r["seconds"], "host": host_info()}
     print(json.dumps(line), flush=True)
     if dist:
         dist.destroy_process_group()

@@ -45,6 +45,7 @@ def test_reference_line_keys_and_arithmetic(monkeypatch, capsys, small_workload)
     cb = line["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1
     assert "stub sample" in cb["sample"]
+    assert isinstance(cb["host"], dict) and "cpu" in cb["host"]   # the CPU model is recorded
     assert line["e2e"] == {"value": line["value"], "unit": "tokens/s",
                            "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert line["config"]["workload"].startswith(bench.WORKLOAD)
