@@ -15,7 +15,9 @@ so that no input and no dirty line is left in L2), max over ranks.  ``--impl ref
 CPU oracle on a bounded sample instead (rank 0 only).
 
 Multi-GPU: every rank runs the same workload on its own GPU (replicas; the
-path has no exchange step), so ``value`` = all ranks' tokens / max time.
+path has no exchange step), so ``value`` = all ranks' tokens / max time.  The
+extra measurements beside the step (comparator, fp8, backward, general
+feature maps, streaming) run at N = 1 only.
 """
 from __future__ import annotations
 
@@ -816,7 +818,9 @@ def run_gpu(args, world, rank, local):
 
     extra = {}
     want = set(EXTRAS if args.extras is None else args.extras.split(","))
-    if args.no_extras:
+    if args.no_extras or world > 1:
+        # The extras describe one GPU; with replicas they would only hold every
+        # GPU of the job longer.
         want = set()
     if "full_softmax" in want:
         extra["full_softmax"] = measure_full_softmax(rh, q, k, v, y, flush, stream)
