@@ -333,6 +333,15 @@ def _check_qkv(q, k, v, *, cuda=True):
         _need(t.is_cuda == cuda and t.device == q.device, f"q, k and v must be {where}")
 
 
+def _check_current_device(device):
+    """The library launches on the current CUDA device: its tensors must live
+    there (a pointer into another GPU's memory would fault)."""
+    cur = _torch().cuda.current_device()
+    _need(device.type == "cuda" and device.index == cur,
+          f"tensors are on {device} but the current CUDA device is cuda:{cur}; "
+          "call torch.cuda.set_device first")
+
+
 def _check_tokens(N, T, Hs, Ws):
     _need(N == T * Hs * Ws, f"N = {N} tokens per head must equal T*Hs*Ws = {T * Hs * Ws}")
 
@@ -397,6 +406,7 @@ def hybrid_attn(q, k, v, Wq, bq, Wk, bk, *, T, Hs, Ws, Tc, To, causal, out_dtype
     ``debug``)."""
     torch = _torch()
     _check_qkv(q, k, v)
+    _check_current_device(q.device)
     B, H, N, D = q.shape
     _check_tokens(N, T, Hs, Ws)
     Dp = 2 * Wq.shape[-1]
@@ -438,6 +448,7 @@ def hybrid_attn_host(q, k, v, Wq, bq, Wk, bk, *, T, Hs, Ws, Tc, To, causal, out=
     _check_tokens(N, T, Hs, Ws)
     Dp = 2 * Wq.shape[-1]
     phi = _phi_struct(Wq, bq, Wk, bk, heads=H, D=D, Dp=Dp)
+    _check_current_device(Wq.device)
     p = make_params(batch=B, heads=H, T=T, Hs=Hs, Ws=Ws, D=D, Dp=Dp, Tc=Tc, To=To,
                     causal=causal, in_dtype=_dtype_code(q.dtype), out_dtype=F32,
                     flags=FLAG_FP8_QK if fp8_qk else 0)
@@ -468,6 +479,7 @@ def feature_map_mlp(x, Wa, ba, Wb, bb, *, parts, T, Hs, Ws, stream=None, force_s
     torch = _torch()
     _need(x.dim() == 4, "x must be a [B, h, N, D] tensor")
     _need(x.is_contiguous() and x.is_cuda, "x must be a contiguous CUDA tensor")
+    _check_current_device(x.device)
     B, H, N, D = x.shape
     _check_tokens(N, T, Hs, Ws)
     Dh, Dp = Wa.shape[-1], Wb.shape[-1]
@@ -500,6 +512,7 @@ def hybrid_attn_phi(q, k, v, phi_q, phi_k, *, T, Hs, Ws, Tc, To, causal, out_dty
     branch partials when ``debug``)."""
     torch = _torch()
     _check_qkv(q, k, v)
+    _check_current_device(q.device)
     B, H, N, D = q.shape
     _check_tokens(N, T, Hs, Ws)
     Dp = phi_q.shape[-1]
@@ -540,6 +553,7 @@ def phi_grad(q, k, v, y, dy, den, Wq, bq, Wk, bk, *, T, Hs, Ws, Tc, To, causal, 
     Returns dict(dWq, dbq, dWk, dbk) shaped like the parameters."""
     torch = _torch()
     _check_qkv(q, k, v)
+    _check_current_device(q.device)
     B, H, N, D = q.shape
     _check_tokens(N, T, Hs, Ws)
     Dp = 2 * Wq.shape[-1]
@@ -575,6 +589,7 @@ def softmax_attn(q, k, v, *, out_dtype=None, scale=0.0, force_simt=False, out=No
     """Plain softmax attention over all keys (the dense comparator)."""
     torch = _torch()
     _check_qkv(q, k, v)
+    _check_current_device(q.device)
     B, H, N, D = q.shape
     out_dtype = torch.float32 if out_dtype is None else out_dtype
     p = make_params(batch=B, heads=H, T=1, Hs=1, Ws=N, D=D, Dp=32, Tc=1, To=0, causal=0,
@@ -619,6 +634,7 @@ class StreamingState:
         self.reset()
 
     def reset(self, stream=None):
+        _check_current_device(self.state.device)
         _check(rehyat_state_init(self.p, self.state.data_ptr(), _stream_handle(stream)),
                "rehyat_state_init")
 
@@ -630,6 +646,7 @@ class StreamingState:
               f"{self.shape[1]}, rows, {self.shape[2]}]")
         _need(q.dtype == self.in_dtype, f"a chunk must be {self.in_dtype}", TypeError)
         _need(q.device == self.state.device, f"a chunk must be on {self.state.device}")
+        _check_current_device(q.device)
         n = rows // self.HW
         if n * self.HW != rows:
             raise ValueError("a chunk must hold whole slices")

@@ -75,7 +75,7 @@ def _shim():
         float32=torch.float32, bfloat16=torch.bfloat16, uint8=torch.uint8,
         contiguous_format=torch.contiguous_format, empty=empty,
         empty_like=lambda t, memory_format=None: FakeTensor(t.shape, t.dtype, t.device),
-        cuda=types.SimpleNamespace(current_stream=lambda: stream))
+        cuda=types.SimpleNamespace(current_stream=lambda: stream, current_device=lambda: 0))
 
 
 LAUNCHERS = ("rehyat_hybrid_attn_fwd", "rehyat_hybrid_attn_fwd_host", "rehyat_feature_map_mlp",
@@ -236,6 +236,28 @@ def test_hybrid_attn_refuses_before_launch(calls, what, change, exc):
 def test_hybrid_attn_refuses_bad_out(calls, out):
     with pytest.raises((ValueError, TypeError)):
         rh.hybrid_attn(*qkv(), *phi_params(), **GEOM, out=out)
+    assert calls == []
+
+
+def test_tensors_off_the_current_device_are_refused(calls):
+    """Everything on cuda:1 while cuda:0 is current: the library would launch
+    on cuda:0 with cuda:1's pointers."""
+    q, k, v = qkv(device="cuda:1")
+    W = phi_params(device="cuda:1")
+    with pytest.raises(ValueError, match="current CUDA device"):
+        rh.hybrid_attn(q, k, v, *W, **GEOM)
+    with pytest.raises(ValueError, match="current CUDA device"):
+        rh.softmax_attn(q, k, v)
+    mlp = [FakeTensor(s, F32, "cuda:1") for s in ((3, 128, 384), (3, 384), (3, 384, 128),
+                                                  (3, 128))]
+    with pytest.raises(ValueError, match="current CUDA device"):
+        rh.feature_map_mlp(q, *mlp, parts=2, T=5, Hs=7, Ws=9)
+    with pytest.raises(ValueError, match="current CUDA device"):
+        rh.hybrid_attn_host(*qkv(device="cpu"), *W, **GEOM)
+    with pytest.raises(ValueError, match="current CUDA device"):
+        rh.StreamingState(batch=1, heads=3, Hs=7, Ws=9, D=128, Dp=128, Tc=2, To=1,
+                          **dict(zip(("Wq", "bq", "Wk", "bk"), W)), in_dtype=BF,
+                          device="cuda:1")
     assert calls == []
 
 
