@@ -81,3 +81,38 @@ def test_oracle_sample_plan_stays_in_budget():
     assert tight["heads"] == 1 and tight["chunks"] >= 1
     roomy = bench.plan_oracle_sample(p, 1e6)
     assert roomy == dict(heads=p.batch * p.heads, chunks=3)
+
+
+# Independent counts of the method's work per configuration, from the planning
+# analysis (computed by a separate script, printed to a few digits):
+# (B, h, T, HW, D, D', T_c, T_o, causal) -> total FLOP, softmax FLOP, exps,
+# full-softmax FLOP.
+WORK = [
+    ((1, 2, 4, 16, 32, 32, 2, 1, False), "1.7e6", "0.66e6", "5.1e3", "1.0e6"),      # tiny fp32
+    ((1, 12, 21, 600, 128, 128, 3, 1, True), "199e9", "179e9", "0.35e9", "975e9"),  # 21x20x30
+    ((2, 12, 21, 1560, 128, 128, 3, 1, False), "2.525e12", "2.422e12", "4.73e9", "13.19e12"),
+    ((1, 12, 81, 1560, 128, 128, 3, 1, True), "5.0e12", "4.8e12", "9.4e9", "98e12"),  # stream
+]
+
+
+def _matches(value, printed):
+    """value agrees with a number printed as ``printed`` to within one unit
+    of its last printed digit."""
+    mant, exp = printed.lower().split("e")
+    decimals = len(mant.split(".")[1]) if "." in mant else 0
+    return abs(value - float(printed)) <= 10.0 ** (int(exp) - decimals)
+
+
+@pytest.mark.parametrize("cfg,total,soft,exps,full", WORK, ids=["tiny", "320x480", "480x832",
+                                                               "stream81"])
+def test_algorithmic_work_matches_independent_counts(cfg, total, soft, exps, full):
+    """The roofline numerator (bench.algorithmic_work) agrees with counts made
+    independently, to the digits those were printed with."""
+    B, h, T, HW, D, Dp, Tc, To, causal = cfg
+    w = bench.algorithmic_work(*cfg)
+    N = T * HW
+    phi_q_and_readout = (2.0 * N * D * Dp + 2.0 * N * Dp * D + 2.0 * N * Dp) * B * h
+    assert _matches(w["total_flops"], total), (w["total_flops"], total)
+    assert _matches(w["attn_flops"] - phi_q_and_readout, soft)
+    assert _matches(w["exps"], exps), (w["exps"], exps)
+    assert _matches(w["full_softmax_flops"], full)
