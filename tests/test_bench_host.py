@@ -116,3 +116,35 @@ def test_algorithmic_work_matches_independent_counts(cfg, total, soft, exps, ful
     assert _matches(w["attn_flops"] - phi_q_and_readout, soft)
     assert _matches(w["exps"], exps), (w["exps"], exps)
     assert _matches(w["full_softmax_flops"], full)
+
+
+def _smi_line(t, sm, reasons=("Not Active",) * 4, sm_max=1965):
+    stamp = __import__("datetime").datetime.fromtimestamp(t).strftime("%Y/%m/%d %H:%M:%S.%f")
+    return ", ".join([stamp[:-3], str(sm), str(sm_max), "812.40", "0x0000000000000000",
+                      *reasons])
+
+
+def test_clock_summary_keeps_the_timed_window_and_its_reasons():
+    """The clock record of the bench line: median SM clock, max clock and the
+    throttle reasons seen inside the timed window only."""
+    cs = bench.ClockSampler.__new__(bench.ClockSampler)   # no nvidia-smi process
+    t0 = 1_000_000.0
+    cs.lines = [
+        _smi_line(t0 - 5.0, 900, ("Active", "Not Active", "Not Active", "Not Active")),  # before
+        _smi_line(t0 + 0.1, 1950),
+        _smi_line(t0 + 0.2, 1965, ("Not Active", "Not Active", "Not Active", "Active")),
+        _smi_line(t0 + 0.3, 1800),
+        "garbage, line",
+        _smi_line(t0 + 9.0, 700, ("Not Active", "Active", "Not Active", "Not Active")),    # after
+    ]
+    s = cs.summary(t0, t0 + 0.5)
+    assert s == {"sm_mhz": 1950.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"],
+                 "samples": 3}
+    # A hardware slowdown inside the window is reported by name.
+    cs.lines.append(_smi_line(t0 + 0.4, 1200, ("Active", "Not Active", "Not Active",
+                                               "Not Active")))
+    assert cs.summary(t0, t0 + 0.5)["reasons"] == ["hw_slowdown", "sw_power_cap"]
+    # No sample inside the window: the last three samples stand in.
+    assert cs.summary(t0 + 100, t0 + 101)["samples"] == 3
+    cs.lines = []
+    assert cs.summary(t0, t0 + 1) is None
