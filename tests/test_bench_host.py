@@ -148,3 +148,16 @@ def test_clock_summary_keeps_the_timed_window_and_its_reasons():
     assert cs.summary(t0 + 100, t0 + 101)["samples"] == 3
     cs.lines = []
     assert cs.summary(t0, t0 + 1) is None
+
+
+def test_traffic_is_reported_only_for_the_captured_source():
+    """`roofline.traffic` comes from the committed ncu summary only while the
+    kernel source hashes to the value recorded with the capture."""
+    import os
+    d = json.load(open(os.path.join(bench.ROOT, "profiles", "traffic.json")))
+    for key in ("attn", "state"):
+        sha = d[key]["source_sha"]
+        assert bench.load_traffic(key, sha) == float(d[key]["dram_bytes_per_launch"])
+        assert bench.load_traffic(key, "0" * 16) is None
+    assert bench.load_traffic("no_such_kernel", d["attn"]["source_sha"]) is None
+    assert len(bench.kernel_source_sha(["bench.py"])) == 16
