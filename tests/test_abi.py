@@ -212,3 +212,50 @@ def test_phi_backward_argument_checks():
     assert call(a0=_params(flags=rh.FLAG_FP8_QK)) == 2
     assert rh.rehyat_phi_bwd_workspace_bytes(_params(flags=rh.FLAG_FP8_QK)) == 0
     assert rh.rehyat_phi_bwd_workspace_bytes(_params(heads=0)) == 0
+
+
+C_PROGRAM = r"""
+#include <stdio.h>
+#include "rehyat.h"
+int main(void) {
+  rehyat_params p = {2, 12, 21, 30, 52, 128, 128, 3, 1, 0, REHYAT_BF16, REHYAT_F32, 0.0f, 0};
+  rehyat_params bad = p;
+  rehyat_status st;
+  size_t ws = rehyat_workspace_bytes(&p);
+  int path = rehyat_attn_path(&p);
+  bad.T = 0;
+  st = rehyat_hybrid_attn_fwd(&bad, NULL, NULL, NULL, NULL, NULL, NULL, 0, NULL, NULL);
+  printf("%d %zu %d %d\n", rehyat_version(), ws, path, (int)st);
+  return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_the_library_links_from_c(tmp_path):
+    """include/rehyat.h compiles as strict C99 with no warnings, and a C
+    program linked against librehyat.so gets the same answers as the
+    binding (host-only calls; no GPU needed)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    root = os.path.dirname(HEADER)
+    pkg = os.path.dirname(rh.lib_path())
+    src = tmp_path / "abi.c"
+    src.write_text(C_PROGRAM)
+    exe = tmp_path / "abi"
+    res = subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                          "-I" + root, str(src), "-L" + pkg, "-lrehyat",
+                          "-Wl,-rpath," + pkg, "-o", str(exe)],
+                         capture_output=True, text=True, timeout=120)
+    assert res.returncode == 0, res.stderr
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, out.stderr
+    version, ws, path, st = (int(x) for x in out.stdout.split())
+    p = rh.make_params(batch=2, heads=12, T=21, Hs=30, Ws=52, D=128, Dp=128, Tc=3, To=1,
+                       causal=0)
+    assert version == rh.rehyat_version()
+    assert ws == rh.rehyat_workspace_bytes(p) > 0
+    assert path == rh.rehyat_attn_path(p) == 1
+    assert st == 1  # REHYAT_ERR_INVALID_ARG, before any launch
