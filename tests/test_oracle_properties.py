@@ -51,3 +51,33 @@ def test_rnn_equals_causal_forms_on_random_geometries(geom):
     y_fac, p_fac = orc.hybrid_factored(*args, T=T, HW=HW, Tc=Tc, To=To, causal=True)
     np.testing.assert_allclose(y_rnn, y_fac, rtol=1e-11, atol=1e-12)
     np.testing.assert_allclose(p_rnn["nL"], p_fac["nL"], rtol=1e-11, atol=1e-12)
+
+
+@settings(max_examples=15, deadline=None, derandomize=True)
+@given(GEOMETRY, st.booleans())
+def test_phi_gradients_match_central_differences_on_random_geometries(geom, causal):
+    """The feature-map gradient oracle against central differences of the
+    masked pairwise forward, on a few entries of each parameter tensor."""
+    from oracle.rehyat_phi_grad import phi_grads
+    T, HW, Tc, To, D, Dp, seed = geom
+    q, k, v, Wq, bq, Wk, bk = _case(T, HW, D, Dp, seed)
+    dy = np.random.default_rng(seed ^ 0x5A5A).standard_normal(q.shape)
+    kw = dict(T=T, HW=HW, Tc=Tc, To=To, causal=causal)
+    g = phi_grads(q, k, v, Wq, bq, Wk, bk, dy, **kw)
+    params = dict(Wq=Wq, bq=bq, Wk=Wk, bk=bk)
+
+    def loss(name, value):
+        a = dict(params, **{name: value})
+        y, _ = orc.hybrid_pairwise(q, k, v, a["Wq"], a["bq"], a["Wk"], a["bk"], **kw)
+        return float((dy * y).sum())
+
+    eps = 1e-6
+    rng = np.random.default_rng(seed)
+    for name, base in params.items():
+        for idx in rng.choice(base.size, size=min(3, base.size), replace=False):
+            plus, minus = base.copy(), base.copy()
+            plus.flat[idx] += eps
+            minus.flat[idx] -= eps
+            fd = (loss(name, plus) - loss(name, minus)) / (2 * eps)
+            an = g["d" + name].flat[idx]
+            assert abs(fd - an) <= 1e-5 * max(1.0, abs(an)), (name, idx, fd, an)
