@@ -169,9 +169,14 @@ REHYAT_API rehyat_status rehyat_fwd_attn(const rehyat_params* p, const void* q,
  *     and enqueue nothing (e.g. one 21x20x30 layer with 12 heads fits, the
  *     batch-2 21x30x52 layer does not).
  *   - Allocates nothing: no cudaMalloc/cudaFree and no allocating library
- *     call.  The first call on each device looks up the array's device
- *     address (cudaGetSymbolAddress, with that device current); make that
- *     first call before any stream capture.
+ *     call.  Every call made outside stream capture looks up the array's
+ *     device address (cudaGetSymbolAddress, with the device current), so
+ *     the address stays right after cudaDeviceReset or when another context
+ *     is made current.  A call on a capturing stream reuses the address of
+ *     the last uncaptured call on that device: make one uncaptured call on
+ *     each device (and again after a cudaDeviceReset) before capturing.  A
+ *     captured call with no earlier uncaptured one returns
+ *     REHYAT_ERR_INVALID_ARG and touches neither the capture nor the GPU.
  *   - The array is shared by every call on a device and keeps the last
  *     call's contents (each call overwrites all of it that it reads, so no
  *     clearing is needed).  Calls that overlap on the GPU (other streams,

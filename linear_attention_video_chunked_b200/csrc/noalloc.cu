@@ -26,24 +26,35 @@ constexpr size_t kScratchBytes = size_t(32) << 20;
 __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 128;
-void* g_scratch_addr[kMaxDevices] = {};  // device address per device ordinal
+void* g_scratch_addr[kMaxDevices] = {};  // last address looked up per device ordinal
 std::mutex g_scratch_mutex;
 
 // The array's name is a host-side stand-in in host code, not a device
-// address; the real address comes from cudaGetSymbolAddress, once per
-// device, with that device current.
-rehyat_status scratch_for_current_device(void** out) {
+// address; the real address comes from cudaGetSymbolAddress with the device
+// current.  It is looked up again on every call made outside stream capture
+// (cheap next to the forward), so a context created anew on the device
+// (after cudaDeviceReset, or another context made current) gets the array's
+// address in that context.  A call on a capturing stream cannot look it up
+// safely (the first lookup may load the module, which would break the
+// capture), so it uses the address of the last uncaptured call on the
+// device, and is refused when there was none.
+rehyat_status scratch_for_current_device(cudaStream_t stream, void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return REHYAT_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return REHYAT_ERR_UNSUPPORTED;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return REHYAT_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (g_scratch_addr[dev] == nullptr) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr)
-      return REHYAT_ERR_CUDA;
-    g_scratch_addr[dev] = ptr;
+  if (cap != cudaStreamCaptureStatusNone) {
+    if (g_scratch_addr[dev] == nullptr) return REHYAT_ERR_INVALID_ARG;
+    *out = g_scratch_addr[dev];
+    return REHYAT_OK;
   }
-  *out = g_scratch_addr[dev];
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr)
+    return REHYAT_ERR_CUDA;
+  g_scratch_addr[dev] = ptr;
+  *out = ptr;
   return REHYAT_OK;
 }
 
@@ -60,7 +71,8 @@ extern "C" rehyat_status rehyat_hybrid_attn_fwd_noalloc(const rehyat_params* p, 
     return rehyat_hybrid_attn_fwd(p, q, k, v, phi, y, nullptr, 0, dbg, stream);
   if (need > rehyat::kScratchBytes) return REHYAT_ERR_SCRATCH_LIMIT;
   void* scratch = nullptr;
-  const rehyat_status st = rehyat::scratch_for_current_device(&scratch);
+  const rehyat_status st =
+      rehyat::scratch_for_current_device(static_cast<cudaStream_t>(stream), &scratch);
   if (st != REHYAT_OK) return st;
   return rehyat_hybrid_attn_fwd(p, q, k, v, phi, y, scratch, rehyat::kScratchBytes, dbg, stream);
 }

@@ -15,10 +15,6 @@ __device__ unsigned int rehyat_tc_error = 0;
 namespace tc {
 
 constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at the boost clock
-#ifndef REHYAT_TEST_FIRST
-#define REHYAT_TEST_FIRST 1
-#endif
-constexpr bool kTestFirst = REHYAT_TEST_FIRST != 0;
 
 // ------------------------------------------------------------ PTX helpers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -89,7 +85,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
   // A phase that has already completed is seen by the non-blocking test;
   // otherwise try_wait suspends the thread until the phase completes (or a
   // time limit passes).
-  if (kTestFirst && mbar_test(bar, parity)) return true;
+  if (mbar_test(bar, parity)) return true;
 #pragma unroll 1
   for (int i = 0; i < 4; ++i)
     if (mbar_try(bar, parity)) return true;
@@ -254,33 +250,6 @@ __device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
   uint64_t d;
   asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
-}
-
-// 2^x for two fp32 values on the FMA pipe: n = round(x) via the 1.5*2^23
-// trick, f = x - n in [-1/2, 1/2], p(f) a cubic fitted for minimax relative
-// error (7.5e-5; coefficients from linear_attention_video_chunked_b200/
-// exp2_poly.py), 2^n applied by adding n << 23 to the bits of p(f).
-// x is clamped below at -125 (NaN propagates), so results stay normal.
-__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
-  constexpr float kC0 = 0.9999280571937561f, kC1 = 0.6932609677314758f;
-  constexpr float kC2 = 0.24261131882667542f, kC3 = 0.055171750485897064f;
-  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
-  float x0, x1;
-  f2_unpack(x, x0, x1);
-  asm("max.NaN.f32 %0, %0, 0fC2FA0000;" : "+f"(x0));  // -125
-  asm("max.NaN.f32 %0, %0, 0fC2FA0000;" : "+f"(x1));
-  const uint64_t xc = f2_pack(x0, x1);
-  const uint64_t magic = f2_pack(kMagic, kMagic);
-  const uint64_t t = f2_add(xc, magic);
-  const uint64_t f = f2_sub(xc, f2_sub(t, magic));
-  uint64_t p = f2_fma(f2_pack(kC3, kC3), f, f2_pack(kC2, kC2));
-  p = f2_fma(p, f, f2_pack(kC1, kC1));
-  p = f2_fma(p, f, f2_pack(kC0, kC0));
-  float t0, t1, p0, p1;
-  f2_unpack(t, t0, t1);
-  f2_unpack(p, p0, p1);
-  return f2_pack(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23)),
-                 __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
 }
 
 __device__ __forceinline__ void tmem_wait_ld() {

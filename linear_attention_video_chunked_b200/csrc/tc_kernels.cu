@@ -524,18 +524,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ===========================================================================
 namespace a2 {
 constexpr int kThreads = 320;
-// One fp32 pair in kPolyEvery takes the FMA-pipe exp2 (0 = all on MUFU).
-// Measured on the 21x30x52 workload (attention ms): all on MUFU 2.85,
-// one in 8 pairs 2.97, one in 4 3.01, one in 2 3.05 -- the softmax is
-// issue/latency bound here, not MUFU bound, so MUFU only by default.
-#ifndef REHYAT_POLY_EVERY
-#define REHYAT_POLY_EVERY 0
-#endif
-constexpr int kPolyEvery = REHYAT_POLY_EVERY;
-#ifndef REHYAT_TRUNC_P
-#define REHYAT_TRUNC_P 0
-#endif
-constexpr bool kTruncP = REHYAT_TRUNC_P != 0;
 constexpr uint32_t kQOff = 0;                      // Q_A, Q_B
 constexpr uint32_t kKOff = 65536;                  // K ring, 3 x 32 KB
 constexpr uint32_t kVOff = kKOff + 3 * 32768;      // V ring, 2 x 32 KB
@@ -576,8 +564,6 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
   using a2::kPhiOff1;
   using a2::kTmemSlot;
   using a2::kAbortSlot;
-  using a2::kPolyEvery;
-  using a2::kTruncP;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -889,9 +875,7 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
         alpha = ex2(m_used - m_max);
         m_used = m_max;
       }
-      // p = 2^(s * scale * log2(e) - m_used) on packed fp32 pairs; one pair
-      // in kPolyEvery goes through the FMA-pipe exp2 (exp2_poly2) instead of
-      // MUFU, which at D = 128 is as busy as the tensor core.
+      // p = 2^(s * scale * log2(e) - m_used) on packed fp32 pairs (MUFU ex2).
       const uint64_t scale2 = f2_pack(P.scale_log2, P.scale_log2);
       const uint64_t negm2 = f2_pack(-m_used, -m_used);
       uint64_t ls2[4] = {0, 0, 0, 0};
@@ -905,28 +889,13 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
           const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(x[2 * i]),
                                              __uint_as_float(x[2 * i + 1])),
                                      scale2, negm2);
-          uint64_t p2;
-          if (kPolyEvery > 0 && (i % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
-            p2 = exp2_poly2(x2);
-          } else {
-            float a0, a1;
-            f2_unpack(x2, a0, a1);
-            p2 = f2_pack(ex2(a0), ex2(a1));
-          }
+          float a0, a1;
+          f2_unpack(x2, a0, a1);
+          const uint64_t p2 = f2_pack(ex2(a0), ex2(a1));
           float p0, p1;
           f2_unpack(p2, p0, p1);
-          if (kTruncP) {
-            // bf16 by truncation (one byte permute on the ALU pipe instead of
-            // a conversion on the pipe that also runs ex2); the row sum takes
-            // the same truncated values, so P.V and l stay consistent.
-            const uint32_t u0 = __float_as_uint(p0), u1 = __float_as_uint(p1);
-            pk[i] = __byte_perm(u0, u1, 0x7632);
-            ls2[i & 3] = f2_add(ls2[i & 3], f2_pack(__uint_as_float(u0 & 0xFFFF0000u),
-                                                    __uint_as_float(u1 & 0xFFFF0000u)));
-          } else {
-            pk[i] = pack_bf16(p0, p1);
-            ls2[i & 3] = f2_add(ls2[i & 3], p2);
-          }
+          pk[i] = pack_bf16(p0, p1);
+          ls2[i & 3] = f2_add(ls2[i & 3], p2);
         }
         REHYAT_TMEM_ST16(lane_base + s_col + c * 16, pk);
       };
