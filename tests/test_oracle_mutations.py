@@ -21,6 +21,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 PINS = {
     "oracle.rehyat_oracle": "tests.test_oracle",
     "oracle.rehyat_phi_grad": "tests.test_phi_grad_oracle",
+    "oracle.rehyat_grad": "tests.test_grad_oracle",
     "oracle.rehyat_phi_mlp": "tests.test_phi_mlp_oracle",
     "oracle.rehyat_fp8": "tests.test_fp8_oracle",
 }
@@ -90,6 +91,34 @@ MUTANTS = [
      "lin = np.concatenate([before, after])"),
     ("oracle.rehyat_phi_grad", "db_k from the query side",
      "dbk[p] = duk.sum(axis=0)", "dbk[p] = duq.sum(axis=0)"),
+    # Full backward (gradients of q, k, v and the feature-map parameters).
+    ("oracle.rehyat_grad", "backward: gradient through the maximum c dropped",
+     "dS[np.arange(dS.shape[0]), jmax] -= Dc", "dS[np.arange(dS.shape[0]), jmax] -= 0.0"),
+    ("oracle.rehyat_grad", "backward: gradient through the maximum with the wrong sign",
+     "dS[np.arange(dS.shape[0]), jmax] -= Dc", "dS[np.arange(dS.shape[0]), jmax] += Dc"),
+    ("oracle.rehyat_grad", "backward: maximum's gradient without the n^S term",
+     "Dc = (gh * aS).sum(axis=1) - r * nS", "Dc = (gh * aS).sum(axis=1)"),
+    ("oracle.rehyat_grad", "backward: denominator term with the wrong sign",
+     "dE = gh @ v[win].T - r[:, None]", "dE = gh @ v[win].T + r[:, None]"),
+    ("oracle.rehyat_grad", "backward: dk without the logit scale",
+     "dk[win] += scale * (dS.T @ q[rows])", "dk[win] += dS.T @ q[rows]"),
+    ("oracle.rehyat_grad", "backward: dq from the values",
+     "dq[rows] += scale * (dS @ k[win])", "dq[rows] += scale * (dS @ v[win])"),
+    ("oracle.rehyat_grad", "backward: softmax dv from g, not g / den",
+     "dv[win] += E.T @ gh", "dv[win] += E.T @ g"),
+    ("oracle.rehyat_grad", "backward: linear-branch dv dropped",
+     "dv[lin] += fk[lin] @ G", "dv[lin] += 0.0 * fk[lin] @ G"),
+    ("oracle.rehyat_grad", "backward: dq through phi_q dropped",
+     'out["dq"] += duq @ Wq[p].T', 'out["dq"] += 0.0 * duq @ Wq[p].T'),
+    ("oracle.rehyat_grad", "backward: dk through phi_k with W_q",
+     'out["dk"] += duk @ Wk[p].T', 'out["dk"] += duk @ Wq[p].T'),
+    ("oracle.rehyat_grad", "backward: window one overlap slice short (dk, dv of the overlap)",
+     "win = slice(start * HW, end * HW)\n        lin = np.arange(0, start * HW) if causal else \\\n"
+     "            np.concatenate([np.arange(0, start * HW), np.arange(end * HW, N)])\n"
+     "        # Forward of this chunk.",
+     "win = slice(min(start + 1, first) * HW, end * HW)\n        lin = np.arange(0, start * HW) if causal else \\\n"
+     "            np.concatenate([np.arange(0, start * HW), np.arange(end * HW, N)])\n"
+     "        # Forward of this chunk."),
     # General feature map and the phi-given forward.
     ("oracle.rehyat_phi_mlp", "GELU: erf argument not divided by sqrt(2)",
      "erf(x / math.sqrt(2.0))", "erf(x)"),
