@@ -11,6 +11,9 @@ namespace rehyat {
 // Bit set per timed-out wait (see rehyat_device_error_flags).  Defined here:
 // include this header from exactly one translation unit (tc_kernels.cu).
 __device__ unsigned int rehyat_tc_error = 0;
+// Rows whose joint denominator fell below 2^-10 n^S in a forward with phi
+// given (rehyat_denominator_report).
+__device__ unsigned long long rehyat_tc_den_rows = 0;
 
 namespace tc {
 
@@ -216,6 +219,20 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
       "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),  \
       "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),        \
       "r"(r[15]))
+
+// One 32-bit column of this warp's 32 TMEM lanes (one value per thread).
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t tmem_ld1(uint32_t taddr) {
+  uint32_t v;
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];\n\t"
+               "tcgen05.wait::ld.sync.aligned;"
+               : "=r"(v)
+               : "r"(taddr)
+               : "memory");
+  return v;
+}
 
 // D += A.B with A read from TMEM (K-major, two bf16 per 32-bit column).
 __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,

@@ -540,7 +540,14 @@ constexpr uint32_t kK8Stage = 16384;
 constexpr uint32_t kQ8Off = kKOff + 3 * kK8Stage;
 enum { Q_FULL = 0, K_FULL = 1, K_EMPTY = 4, V_FULL = 7, V_EMPTY = 9, S_FULL = 11, P_FULL = 13,
        PV_DONE = 15, LAST_PV = 17, TAIL_FULL = 18, PHI_DONE = 19, PHI_READY = 20, READ_DONE = 22,
-       VEC_READY = 23, NBAR = 24 };
+       VEC_READY = 23, XCHG = 24, LX = 26, LX_DONE = 27, NBAR = 28 };
+// Row halves: each softmax thread owns 64 of a row's 128 key columns; the
+// two threads of a row (warps w and w + 4, same TMEM lane quarter) trade
+// their partial row maxima through TMEM column 63 (half 0) and 127 (half 1)
+// of the tile's S buffer, and their partial row sums, after the key loop,
+// through column 126 (a column no maximum passes through, so a slow partner
+// still reading its last maximum is never overwritten).
+constexpr uint32_t kXchgCol0 = 63, kXchgCol1 = 127, kLxCol = 126;
 constexpr uint32_t kTmemSlot = kBarOff + 8 * NBAR;
 constexpr uint32_t kAbortSlot = kTmemSlot + 4;
 // b_q of the head and z^L of the chunk (D' floats each), shared by both tiles.
@@ -630,9 +637,10 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
 
   if (tid == 0) {
     for (int i = 0; i < a2::NBAR; ++i) {
-      const bool by_warpgroup = i == a2::P_FULL || i == a2::P_FULL + 1 || i == a2::PHI_READY ||
-                                i == a2::PHI_READY + 1 || i == a2::VEC_READY;
-      mbar_init(bar(i), by_warpgroup ? kSoftmaxThreads : 1);
+      const bool by_warpgroup = i == a2::PHI_READY || i == a2::PHI_READY + 1 || i == a2::VEC_READY;
+      const bool by_all = i == a2::P_FULL || i == a2::P_FULL + 1 || i == a2::XCHG ||
+                          i == a2::XCHG + 1 || i == a2::LX || i == a2::LX_DONE;
+      mbar_init(bar(i), by_all ? 2 * kSoftmaxThreads : (by_warpgroup ? kSoftmaxThreads : 1));
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -768,8 +776,11 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
       if (linear && ok) {
         ok = mbar_wait(bar(a2::TAIL_FULL), 0, abort_flag, 9);
         if (ok) {
+          // The phi_q product overwrites S: the softmax warps have traded
+          // their row sums through it first.
+          if (!phi_given) ok = mbar_wait(bar(a2::LX_DONE), 0, abort_flag, 18);
           tc_fence_after();
-          if (!phi_given) {
+          if (ok && !phi_given) {
             const uint32_t id_phi = idesc(kBM, Dp, 1, false);
             for (int tile = 0; tile < ntiles; ++tile)
 #pragma unroll
@@ -798,94 +809,93 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp < 8 && (warp < 4 || has_b)) {
+  } else if (warp < 8) {
     // ================================================= softmax / epilogue
-    const int tile = warp >> 2;
-    const int r = tid & 127;                 // row within the tile == TMEM lane
+    // Key loop: all eight warps work on each query tile in turn (tile A,
+    // then tile B, per key step), two threads per row: warp w handles key
+    // columns [64 hf, 64 hf + 64) of rows 32 (w & 3) .. + 31, hf = w >> 2.
+    // Both threads of a row take the same reference point (the partial
+    // maxima are traded through TMEM), so their P values add up in one P.V.
+    // Tail: warps 0-3 finish tile A, warps 4-7 tile B (as one warpgroup each).
+    const int hf = warp >> 2;
+    const int r = tid & 127;                 // row within a tile == TMEM lane
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    const uint32_t s_col = tile * 256, o_col = s_col + 128;
-    const int nrows = nrows_t[tile];
-    float m_used = -INFINITY, m_max = -INFINITY, l = 0.f;
+    const int ntiles = has_b ? 2 : 1;
+    float m_used2[2] = {-INFINITY, -INFINITY}, m_max2[2] = {-INFINITY, -INFINITY};
+    float l2[2] = {0.f, 0.f};                // this thread's half of each row sum
     bool ok = true;
     auto wait_all = [&](uint32_t b, uint32_t parity, uint32_t code) {
       return __all_sync(0xffffffffu, mbar_wait(b, parity, abort_flag, code));
     };
     float* vec = reinterpret_cast<float*>(sbase + a2::kVecOff);  // [b_q (D') | z^L (D')]
-    if (linear && tile == 0) {
-      // Tile A's warpgroup stages b_q and z^L for the tail while it waits
-      // for the first scores (b_q of head h is h's D' consecutive values).
+    if (linear && hf == 0) {
+      // Warps 0-3 stage b_q and z^L for the tail while they wait for the
+      // first scores (b_q of head h is h's D' consecutive values).
       if (r < Dp) {
         vec[r] = phi_given ? 0.f : __ldg(P.bq + h * Dp + r);
         vec[Dp + r] = __ldg(P.zL + (static_cast<long long>(bh) * P.nchunks + t) * Dp + r);
       }
       mbar_arrive(bar(a2::VEC_READY));
     }
+    const uint64_t scale2 = f2_pack(P.scale_log2, P.scale_log2);
+    const uint32_t my_xcol = hf ? a2::kXchgCol1 : a2::kXchgCol0;
+    const uint32_t other_xcol = hf ? a2::kXchgCol0 : a2::kXchgCol1;
     for (int j = 0; j < nt && ok; ++j) {
-      // S_FULL(j) also covers this tile's P.V of step j-1 (issued earlier).
-      ok = wait_all(bar(a2::S_FULL + tile), j & 1, 11);
-      if (!ok) break;
-      tc_fence_after();
       const int nvalid = tile_src(j).nvalid;
       const bool ragged = nvalid < kBN;  // warp-uniform: keys past the end
-      // S is streamed from TMEM 32 columns at a time through two register
-      // buffers: the next load is in flight while the current chunk is used
-      // (S never sits whole in registers, which would spill).
-      uint32_t xa[32], xb[32];
-      auto mask = [&](uint32_t* x, int c) {
+      for (int tile = 0; tile < ntiles && ok; ++tile) {
+        const uint32_t s_col = tile * 256, o_col = s_col + 128;
+        // S_FULL(j) also covers this tile's P.V of step j-1 (issued earlier).
+        ok = wait_all(bar(a2::S_FULL + tile), j & 1, 11);
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t x[64];
+        REHYAT_TMEM_LD32(lane_base + s_col + 64 * hf, x);
+        REHYAT_TMEM_LD32(lane_base + s_col + 64 * hf + 32, (x + 32));
+        tmem_wait_ld();
         if (ragged) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (32 * c + i >= nvalid) x[i] = __float_as_uint(-INFINITY);
+          for (int i = 0; i < 64; ++i)
+            if (64 * hf + i >= nvalid) x[i] = __float_as_uint(-INFINITY);
         }
-      };
-      float mx[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
-      auto max_chunk = [&](const uint32_t* x) {
+        float mx[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i)
-          mx[i] = fmax3(mx[i], fmax3(__uint_as_float(x[i]), __uint_as_float(x[i + 8]),
-                                     __uint_as_float(x[i + 16])),
-                        __uint_as_float(x[i + 24]));
-      };
-      // Pass 1: row max.
-      REHYAT_TMEM_LD32(lane_base + s_col, xa);
-      REHYAT_TMEM_WAIT_LD32(xa);
-      REHYAT_TMEM_LD32(lane_base + s_col + 32, xb);
-      mask(xa, 0);
-      max_chunk(xa);
-      REHYAT_TMEM_WAIT_LD32(xb);
-      REHYAT_TMEM_LD32(lane_base + s_col + 64, xa);
-      mask(xb, 1);
-      max_chunk(xb);
-      REHYAT_TMEM_WAIT_LD32(xa);
-      REHYAT_TMEM_LD32(lane_base + s_col + 96, xb);
-      mask(xa, 2);
-      max_chunk(xa);
-      REHYAT_TMEM_WAIT_LD32(xb);
-      REHYAT_TMEM_LD32(lane_base + s_col, xa);  // pass 2, chunk 0
-      mask(xb, 3);
-      max_chunk(xb);
-      m_max = fmaxf(m_max, fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
-                                 fmaxf(mx[6], mx[7])) *
-                               P.scale_log2);
-      float alpha = 1.f;
-      const bool rescale = m_max > m_used + 8.f;
-      if (rescale) {
-        alpha = ex2(m_used - m_max);
-        m_used = m_max;
-      }
-      // p = 2^(s * scale * log2(e) - m_used) on packed fp32 pairs (MUFU ex2).
-      const uint64_t scale2 = f2_pack(P.scale_log2, P.scale_log2);
-      const uint64_t negm2 = f2_pack(-m_used, -m_used);
-      uint64_t ls2[4] = {0, 0, 0, 0};
-      // Pass 2: P (bf16 pairs) of chunk c is written over S columns already
-      // consumed, [16c, 16c + 16), while chunk c + 1 is being loaded.
-      auto exp_chunk = [&](uint32_t* x, int c) {
-        mask(x, c);
-        uint32_t pk[16];
+          mx[i] = fmax3(fmax3(__uint_as_float(x[i]), __uint_as_float(x[i + 8]),
+                              __uint_as_float(x[i + 16])),
+                        fmax3(__uint_as_float(x[i + 24]), __uint_as_float(x[i + 32]),
+                              __uint_as_float(x[i + 40])),
+                        fmaxf(__uint_as_float(x[i + 48]), __uint_as_float(x[i + 56])));
+        float pm = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
+                         fmaxf(mx[6], mx[7]));
+        // Trade the partial maxima: each thread writes its own into a column
+        // of its half of S (already in registers), reads its partner's.
+        tmem_st1(lane_base + s_col + my_xcol, __float_as_uint(pm));
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(a2::XCHG + tile));
+        ok = wait_all(bar(a2::XCHG + tile), j & 1, 16);
+        if (!ok) break;
+        tc_fence_after();
+        pm = fmaxf(pm, __uint_as_float(tmem_ld1(lane_base + s_col + other_xcol)));
+        float& m_max = m_max2[tile];
+        float& m_used = m_used2[tile];
+        m_max = fmaxf(m_max, pm * P.scale_log2);
+        float alpha = 1.f;
+        const bool rescale = m_max > m_used + 8.f;
+        if (rescale) {
+          alpha = ex2(m_used - m_max);  // 0 on the first tile
+          m_used = m_max;
+        }
+        // p = 2^(s * scale * log2(e) - m_used) on packed fp32 pairs (MUFU
+        // ex2); P (bf16 pairs) of this half goes to S columns
+        // [32 hf, 32 hf + 32): half 1 overwrites column 63 only after it
+        // has read it.
+        const uint64_t negm2 = f2_pack(-m_used, -m_used);
+        uint64_t ls2[4] = {0, 0, 0, 0};
+        uint32_t pk[32];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
+        for (int i = 0; i < 32; ++i) {
           const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(x[2 * i]),
                                              __uint_as_float(x[2 * i + 1])),
                                      scale2, negm2);
@@ -897,57 +907,70 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
           pk[i] = pack_bf16(p0, p1);
           ls2[i & 3] = f2_add(ls2[i & 3], p2);
         }
-        REHYAT_TMEM_ST16(lane_base + s_col + c * 16, pk);
-      };
-      REHYAT_TMEM_WAIT_LD32(xa);
-      REHYAT_TMEM_LD32(lane_base + s_col + 32, xb);
-      exp_chunk(xa, 0);
-      REHYAT_TMEM_WAIT_LD32(xb);
-      REHYAT_TMEM_LD32(lane_base + s_col + 64, xa);
-      exp_chunk(xb, 1);
-      REHYAT_TMEM_WAIT_LD32(xa);
-      REHYAT_TMEM_LD32(lane_base + s_col + 96, xb);
-      exp_chunk(xa, 2);
-      REHYAT_TMEM_WAIT_LD32(xb);
-      exp_chunk(xb, 3);
-      float ls[8];
-      f2_unpack(f2_add(ls2[0], ls2[1]), ls[0], ls[1]);
-      f2_unpack(f2_add(ls2[2], ls2[3]), ls[2], ls[3]);
-      ls[4] = ls[5] = ls[6] = ls[7] = 0.f;
-      // After the P stores (S is dead by now): bring the earlier a^S to the
-      // new reference point; this tile's P.V of step j-1 is complete (covered
-      // by S_FULL(j)).  Warp-collective; rows that did not move use alpha = 1.
-      if (j > 0 && __any_sync(0xffffffffu, rescale)) {
-        uint32_t o[32];
+        REHYAT_TMEM_ST32(lane_base + s_col + 32 * hf, pk);
+        float ls[4];
+        f2_unpack(f2_add(ls2[0], ls2[1]), ls[0], ls[1]);
+        f2_unpack(f2_add(ls2[2], ls2[3]), ls[2], ls[3]);
+        // This tile's P.V of step j-1 is complete (covered by S_FULL(j)):
+        // bring this half's columns of the earlier a^S to the new reference
+        // point.  Warp-collective; rows that did not move use alpha = 1.
+        if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+          uint32_t o[32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          REHYAT_TMEM_LD32(lane_base + o_col + c * 32, o);
-          tmem_wait_ld();
+          for (int c = 0; c < 2; ++c) {
+            REHYAT_TMEM_LD32(lane_base + o_col + 64 * hf + c * 32, o);
+            tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          REHYAT_TMEM_ST32(lane_base + o_col + c * 32, o);
-        }
-      }
-      tmem_wait_st();
-      l = l * alpha + (((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7])));
-      if (tile == 0 && nvalid < kBN) {
-        // Zero the V rows past the last valid key (shared by both tiles;
-        // tile B's P.V is issued after tile A's P_FULL).
-        ok = wait_all(bar(a2::V_FULL + (j & 1)), (j >> 1) & 1, 13);
-        if (!ok) break;
-        if (r >= nvalid) {
-          const uint32_t vrow = base + kVOff + (j & 1) * 32768 + r * 128;
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            st_shared_v4(vrow + c * 16, 0, 0, 0, 0);
-            st_shared_v4(vrow + 16384 + c * 16, 0, 0, 0, 0);
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            REHYAT_TMEM_ST32(lane_base + o_col + 64 * hf + c * 32, o);
           }
         }
-        fence_proxy_async();
+        tmem_wait_st();
+        l2[tile] = l2[tile] * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
+        if (tile == 0 && ragged) {
+          // Zero the V rows past the last valid key (shared by both tiles;
+          // tile B's P.V is issued after tile A's P_FULL): half hf clears
+          // box hf (64 columns) of row r.
+          ok = wait_all(bar(a2::V_FULL + (j & 1)), (j >> 1) & 1, 13);
+          if (!ok) break;
+          if (r >= nvalid) {
+            const uint32_t vrow = base + kVOff + (j & 1) * 32768 + hf * 16384 + r * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) st_shared_v4(vrow + c * 16, 0, 0, 0, 0);
+          }
+          fence_proxy_async();
+        }
+        tc_fence_before();
+        mbar_arrive(bar(a2::P_FULL + tile));
+      }
+    }
+    // Row sums: the tail of tile A runs on half 0, that of tile B on half 1;
+    // each needs the other half's part, passed through column 126 of the
+    // tile's S buffer (free now: P uses columns [0, 64)).  The MMA warp
+    // issues the phi_q product, which overwrites S, only after LX_DONE.
+    if (ok) {
+      const int give = 1 - hf;  // the tile whose tail the other half runs
+      if (give < ntiles) {
+        tmem_st1(lane_base + give * 256 + a2::kLxCol, __float_as_uint(l2[give]));
+        tmem_wait_st();
       }
       tc_fence_before();
-      mbar_arrive(bar(a2::P_FULL + tile));
+      mbar_arrive(bar(a2::LX));
+      ok = wait_all(bar(a2::LX), 0, 17);
     }
+    const int tile = hf;
+    if (ok && tile < ntiles) {
+      tc_fence_after();
+      l2[tile] += __uint_as_float(tmem_ld1(lane_base + tile * 256 + a2::kLxCol));
+    }
+    tc_fence_before();
+    mbar_arrive(bar(a2::LX_DONE));
+    if (tile >= ntiles) {
+      // Tile B is empty: warps 4-7 have no tail.
+    } else {
+    const uint32_t s_col = tile * 256, o_col = s_col + 128;
+    const int nrows = nrows_t[tile];
+    const float m_used = m_used2[tile], m_max = m_max2[tile], l = l2[tile];
     const float fscale = ex2(m_used - m_max);
     const long long grow = static_cast<long long>(bh) * P.rows_per_bh + row0 + tile * kBM + r;
     const bool dbg_split = P.dbg_aS != nullptr || P.dbg_aL != nullptr;
@@ -1027,6 +1050,9 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
       tc_fence_after();
       const float nS = l * fscale;
       const float den = nS + nL;
+      // A signed phi (given) can drive n^L towards -n^S: count the rows, the
+      // output stays as the formula gives it.
+      if (phi_given && r < nrows && !(den >= ldexpf(nS, -10))) atomicAdd(&rehyat_tc_den_rows, 1ull);
       // y = f * O / den: one IEEE division per row, then a product per value.
       const float ysc = __fdiv_rn(fscale, den);
       const bool dbg_num = P.dbg_aL != nullptr || (P.dbg_aS != nullptr && !linear);
@@ -1093,6 +1119,7 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
         reinterpret_cast<uint4*>(static_cast<float*>(P.y) + (grow0 + rr) * kD)[lane] =
             make_uint4(a0, a1, a2, a3);
       }
+    }
     }
   }
 
@@ -1770,6 +1797,25 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s) {
 
 // The general feature map's tensor-core kernel shares this unit's helpers.
 #include "tc_phi_mlp.cuh"
+
+namespace rehyat {
+cudaError_t read_den_rows_simt(unsigned long long* rows, int reset);
+}
+
+extern "C" rehyat_status rehyat_denominator_report(unsigned long long* rows, int reset) {
+  if (!rows) return REHYAT_ERR_INVALID_ARG;
+  unsigned long long tc = 0, simt = 0;
+  if (cudaMemcpyFromSymbol(&tc, rehyat::rehyat_tc_den_rows, sizeof(tc)) != cudaSuccess ||
+      rehyat::read_den_rows_simt(&simt, reset) != cudaSuccess)
+    return REHYAT_ERR_CUDA;
+  if (reset) {
+    const unsigned long long zero = 0;
+    if (cudaMemcpyToSymbol(rehyat::rehyat_tc_den_rows, &zero, sizeof(zero)) != cudaSuccess)
+      return REHYAT_ERR_CUDA;
+  }
+  *rows = tc + simt;
+  return REHYAT_OK;
+}
 
 extern "C" rehyat_status rehyat_device_error_flags(unsigned* flags, int reset) {
   if (!flags) return REHYAT_ERR_INVALID_ARG;
