@@ -341,6 +341,44 @@ REHYAT_API rehyat_status rehyat_phi_bwd(const rehyat_params* p, const void* q, c
                                         const rehyat_phi_grad* grad, void* workspace,
                                         size_t ws_bytes, void* stream);
 
+/* Workspace bytes rehyat_hybrid_attn_bwd needs (0 if p is invalid). */
+REHYAT_API size_t rehyat_hybrid_attn_bwd_workspace_bytes(const rehyat_params* p);
+
+/* Full backward of the forward of rehyat_hybrid_attn_fwd (either form):
+ * dL/dq, dL/dk, dL/dv and dL/dW_q, dL/db_q, dL/dW_k, dL/db_k of a scalar
+ * loss L, for the second training stage of the ReHyAt note (Method, Key
+ * design 5: the whole converted model is fine-tuned, so gradients pass
+ * through q, k and v).
+ * Inputs: the forward's q, k, v (in_dtype, [B][h][N][D]) and phi; its output
+ * y (fp32); dy = dL/dy (fp32, same shape); per query [B][h][N] fp32 the
+ * stabiliser c (the forward's row maximum of the scaled logits over the
+ * window, rehyat_debug.c) and den = n^S + n^L (rehyat_debug.nS + nL).
+ * Math (chain rule through Key designs 1-4; gh = dy/den, r = dy.y/den):
+ *   dS_ij = e_ij (gh_i.v_j - r_i) - [j = j*_i] Dc_i,  e_ij = exp(s_ij - c_i),
+ *   Dc_i = sum_j e_ij (gh_i.v_j - r_i)  (c_i is the window maximum and the
+ *   linear branch is not scaled by exp(-c_i), so the gradient also flows
+ *   through the maximum, to its key j*_i: the window key with the largest
+ *   logit as recomputed in fp32, the lowest index among equal ones),
+ *   dq_i = scale sum_j dS_ij k_j + du_q W_q^T,  dk_j = scale sum_i dS_ij q_i
+ *   + du_k W_k^T,  dv_j = sum_i e_ij gh_i + Ghat_s^T phi_k(k_j), where
+ *   du_q = 2u_q * (S_L gh - r z_L), du_k = 2u_k * (Ghat_s v_j + hhat_s), Ghat_s
+ *   the sum of the linear-set state gradients over the chunks whose linear
+ *   set holds slice s; the parameter gradients are those of rehyat_phi_bwd.
+ * Outputs (overwritten, not accumulated): dq, dk, dv fp32 [B][h][N][D];
+ * grad's four arrays as for rehyat_phi_bwd.  fp32 arithmetic on CUDA cores;
+ * no atomics, so repeated calls agree bit for bit.
+ * Pointers: q, k, v, y, dy, dq, dk, dv, workspace 16-byte aligned; c, den and
+ * the parameter gradients 4-byte aligned.  Errors as for
+ * rehyat_hybrid_attn_fwd; REHYAT_FLAG_FP8_QK is refused (UNSUPPORTED). */
+REHYAT_API rehyat_status rehyat_hybrid_attn_bwd(const rehyat_params* p, const void* q,
+                                                const void* k, const void* v,
+                                                const rehyat_phi* phi, const float* y,
+                                                const float* dy, const float* c,
+                                                const float* den, float* dq, float* dk,
+                                                float* dv, const rehyat_phi_grad* grad,
+                                                void* workspace, size_t ws_bytes,
+                                                void* stream);
+
 /* ---------------------------------------------------------------------- */
 /* Diagnostic: every wait inside the tensor-core kernels is bounded (~2 s);
  * a wait that runs out sets a bit in a device-side error word and the
@@ -349,6 +387,19 @@ REHYAT_API rehyat_status rehyat_phi_bwd(const rehyat_params* p, const void* q, c
  * clears it when reset != 0.  Unlike the other entry points it synchronises
  * the device (a blocking copy). */
 REHYAT_API rehyat_status rehyat_device_error_flags(unsigned* flags, int reset);
+
+/* Denominator report for the forward with phi given
+ * (rehyat_hybrid_attn_fwd_phi).  A general feature map with a degree-1 part
+ * (Key design 3 of the ReHyAt note) is signed, so n^L can be negative and
+ * the joint denominator n^S + n^L can approach zero or drop below it (n^S
+ * >= 1 always holds).  The forward keeps y = (a^S + a^L) / (n^S + n^L) as
+ * written, and counts the query rows where n^S + n^L < 2^-10 n^S (a
+ * non-positive or NaN denominator, or one cancelled to ~10 bits).  This
+ * reads the count for the current device into *rows (summed over every
+ * such forward since the last reset) and clears it when reset != 0.  The
+ * closed-form phi (a sum of squares) never adds to it.  Synchronises the
+ * device (blocking copies). */
+REHYAT_API rehyat_status rehyat_denominator_report(unsigned long long* rows, int reset);
 
 /* Which attention kernel these params select: 1 = the tensor-core kernel
  * (bf16 inputs, D = 128, Dp in {64, 128, 256}, no REHYAT_FLAG_FORCE_SIMT),

@@ -34,7 +34,8 @@ __all__ = [
     "rehyat_feature_map_mlp_workspace_bytes", "rehyat_host_workspace_bytes",
     "rehyat_hybrid_attn_fwd_host", "hybrid_attn_host",
     "make_params", "hybrid_attn", "hybrid_attn_phi", "feature_map_mlp", "softmax_attn",
-    "phi_grad", "StreamingState",
+    "phi_grad", "StreamingState", "rehyat_hybrid_attn_bwd_workspace_bytes",
+    "rehyat_hybrid_attn_bwd", "hybrid_attn_bwd", "rehyat_denominator_report",
 ]
 
 F32, BF16 = 0, 1
@@ -54,7 +55,8 @@ EXPORTED_SYMBOLS = (
     "rehyat_hybrid_attn_fwd_noalloc", "rehyat_phi_bwd_workspace_bytes", "rehyat_phi_bwd",
     "rehyat_hybrid_attn_fwd_phi", "rehyat_feature_map_mlp",
     "rehyat_feature_map_mlp_workspace_bytes", "rehyat_host_workspace_bytes",
-    "rehyat_hybrid_attn_fwd_host",
+    "rehyat_hybrid_attn_fwd_host", "rehyat_hybrid_attn_bwd_workspace_bytes",
+    "rehyat_hybrid_attn_bwd", "rehyat_denominator_report",
 )
 
 
@@ -139,6 +141,8 @@ def lib() -> ctypes.CDLL:
         L.rehyat_chunk_step.argtypes = [P(RehyatParams), vp, vp, vp, i, P(RehyatPhi), vp, vp, vp,
                                         sz, P(RehyatDebug), vp]
         L.rehyat_chunk_step.restype = i
+        L.rehyat_denominator_report.argtypes = [P(ctypes.c_ulonglong), i]
+        L.rehyat_denominator_report.restype = i
         L.rehyat_device_error_flags.argtypes = [P(ctypes.c_uint), i]
         L.rehyat_device_error_flags.restype = i
         L.rehyat_attn_path.argtypes = [P(RehyatParams)]
@@ -152,6 +156,11 @@ def lib() -> ctypes.CDLL:
         L.rehyat_phi_bwd.argtypes = [P(RehyatParams), vp, vp, vp, vp, vp, vp, P(RehyatPhi),
                                      P(RehyatPhiGrad), vp, sz, vp]
         L.rehyat_phi_bwd.restype = i
+        L.rehyat_hybrid_attn_bwd_workspace_bytes.argtypes = [P(RehyatParams)]
+        L.rehyat_hybrid_attn_bwd_workspace_bytes.restype = sz
+        L.rehyat_hybrid_attn_bwd.argtypes = [P(RehyatParams), vp, vp, vp, P(RehyatPhi), vp, vp,
+                                             vp, vp, vp, vp, vp, P(RehyatPhiGrad), vp, sz, vp]
+        L.rehyat_hybrid_attn_bwd.restype = i
         L.rehyat_hybrid_attn_fwd_phi.argtypes = [P(RehyatParams), vp, vp, vp, vp, vp, vp, vp, sz,
                                                  vp, vp]
         L.rehyat_hybrid_attn_fwd_phi.restype = i
@@ -201,6 +210,26 @@ def rehyat_hybrid_attn_fwd_noalloc(p, q, k, v, phi, y, dbg, stream) -> int:
 
 def rehyat_phi_bwd_workspace_bytes(p: RehyatParams) -> int:
     return lib().rehyat_phi_bwd_workspace_bytes(ctypes.byref(p))
+
+
+def rehyat_denominator_report(reset: bool = False) -> int:
+    """Rows with n^S + n^L < 2^-10 n^S in forwards with phi given, since the
+    last reset (blocking)."""
+    rows = ctypes.c_ulonglong(0)
+    _check(lib().rehyat_denominator_report(ctypes.byref(rows), 1 if reset else 0),
+           "rehyat_denominator_report")
+    return rows.value
+
+
+def rehyat_hybrid_attn_bwd_workspace_bytes(p: RehyatParams) -> int:
+    return lib().rehyat_hybrid_attn_bwd_workspace_bytes(ctypes.byref(p))
+
+
+def rehyat_hybrid_attn_bwd(p, q, k, v, phi, y, dy, c, den, dq, dk, dv, grad, workspace, ws_bytes,
+                           stream) -> int:
+    return lib().rehyat_hybrid_attn_bwd(ctypes.byref(p), q, k, v, ctypes.byref(phi), y, dy, c, den,
+                                        dq, dk, dv, ctypes.byref(grad), workspace, ws_bytes,
+                                        stream)
 
 
 def rehyat_phi_bwd(p, q, k, v, y, dy, den, phi, grad, workspace, ws_bytes, stream) -> int:
@@ -582,6 +611,51 @@ def phi_grad(q, k, v, y, dy, den, Wq, bq, Wk, bk, *, T, Hs, Ws, Tc, To, causal, 
                         _stream_handle(stream))
     _check(st, "rehyat_phi_bwd")
     return g
+
+
+def hybrid_attn_bwd(q, k, v, y, dy, c, den, Wq, bq, Wk, bk, *, T, Hs, Ws, Tc, To, causal,
+                    scale=0.0, force_simt=False, workspace=None, stream=None):
+    """Full backward: gradients of L with respect to q, k, v and the phi
+    parameters, given the forward's q, k, v, its fp32 output y, dy = dL/dy
+    (fp32), and per query the stabiliser c and den = n^S + n^L
+    (``parts["c"]`` and ``parts["nS"] + parts["nL"]`` of
+    ``hybrid_attn(..., debug=True)``).  Returns dict(dq, dk, dv (fp32, shaped
+    like q), dWq, dbq, dWk, dbk (shaped like the parameters))."""
+    torch = _torch()
+    _check_qkv(q, k, v)
+    _check_current_device(q.device)
+    B, H, N, D = q.shape
+    _check_tokens(N, T, Hs, Ws)
+    Dp = 2 * Wq.shape[-1]
+    for t in (y, dy, c, den):
+        if t.dtype != torch.float32 or not t.is_contiguous():
+            raise TypeError("y, dy, c and den must be contiguous fp32 tensors")
+    _check_out(y, (B, H, N, D), torch.float32, q.device, "y")
+    _check_out(dy, (B, H, N, D), torch.float32, q.device, "dy")
+    _check_out(c, (B, H, N), torch.float32, q.device, "c")
+    _check_out(den, (B, H, N), torch.float32, q.device, "den")
+    phi = _phi_struct(Wq, bq, Wk, bk, heads=H, D=D, Dp=Dp, device=q.device)
+    p = make_params(batch=B, heads=H, T=T, Hs=Hs, Ws=Ws, D=D, Dp=Dp, Tc=Tc, To=To,
+                    causal=causal, in_dtype=_dtype_code(q.dtype), out_dtype=F32, scale=scale,
+                    flags=FLAG_FORCE_SIMT if force_simt else 0)
+    nbytes = rehyat_hybrid_attn_bwd_workspace_bytes(p)
+    if nbytes == 0:
+        raise RehyatError(1, "rehyat_hybrid_attn_bwd_workspace_bytes")
+    if workspace is not None:
+        _check_workspace(workspace, q.device)
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    out = {name: torch.empty(B, H, N, D, dtype=torch.float32, device=q.device)
+           for name in ("dq", "dk", "dv")}
+    out.update({name: torch.empty_like(t, memory_format=torch.contiguous_format) for name, t in
+                (("dWq", Wq), ("dbq", bq), ("dWk", Wk), ("dbk", bk))})
+    grad = RehyatPhiGrad(*(out[n].data_ptr() for n in ("dWq", "dbq", "dWk", "dbk")))
+    st = rehyat_hybrid_attn_bwd(p, q.data_ptr(), k.data_ptr(), v.data_ptr(), phi, y.data_ptr(),
+                                dy.data_ptr(), c.data_ptr(), den.data_ptr(), out["dq"].data_ptr(),
+                                out["dk"].data_ptr(), out["dv"].data_ptr(), grad,
+                                workspace.data_ptr(), _nbytes(workspace), _stream_handle(stream))
+    _check(st, "rehyat_hybrid_attn_bwd")
+    return out
 
 
 def softmax_attn(q, k, v, *, out_dtype=None, scale=0.0, force_simt=False, out=None,

@@ -561,4 +561,61 @@ rehyat_status rehyat_phi_bwd(const rehyat_params* p, const void* q, const void* 
   return to_status(launch_phi_bwd(a, s));
 }
 
+size_t rehyat_hybrid_attn_bwd_workspace_bytes(const rehyat_params* p) {
+  const size_t phi_ws = rehyat_phi_bwd_workspace_bytes(p);
+  if (phi_ws == 0) return 0;
+  const size_t rows = static_cast<size_t>(p->batch) * p->heads * p->T * p->Hs * p->Ws;
+  return phi_ws + 3 * align_up(rows * sizeof(float));
+}
+
+rehyat_status rehyat_hybrid_attn_bwd(const rehyat_params* p, const void* q, const void* k,
+                                     const void* v, const rehyat_phi* phi, const float* y,
+                                     const float* dy, const float* c, const float* den,
+                                     float* dq, float* dk, float* dv,
+                                     const rehyat_phi_grad* grad, void* workspace,
+                                     size_t ws_bytes, void* stream) {
+  rehyat_status st = check_params(p);
+  if (st != REHYAT_OK) return st;
+  if ((st = no_fp8(p)) != REHYAT_OK) return st;
+  if (!q || !k || !v || !y || !dy || !c || !den || !dq || !dk || !dv || !grad || !workspace)
+    return REHYAT_ERR_INVALID_ARG;
+  if (!grad->dWq || !grad->dbq || !grad->dWk || !grad->dbk) return REHYAT_ERR_INVALID_ARG;
+  if ((st = check_phi(phi)) != REHYAT_OK) return st;
+  auto a4 = [](const void* x) { return (reinterpret_cast<uintptr_t>(x) & 3) == 0; };
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(y) || !aligned16(dy) ||
+      !aligned16(workspace) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !a4(c) ||
+      !a4(den) || !a4(grad->dWq) || !a4(grad->dbq) || !a4(grad->dWk) || !a4(grad->dbk))
+    return REHYAT_ERR_MISALIGNED;
+  if (ws_bytes < rehyat_hybrid_attn_bwd_workspace_bytes(p)) return REHYAT_ERR_WORKSPACE;
+  // Gradients of the feature-map parameters, and on the way the linear-set
+  // state per chunk (S_L, z_L) and the Ghat blocks the token gradients use.
+  if ((st = rehyat_phi_bwd(p, q, k, v, y, dy, den, phi, grad, workspace,
+                           rehyat_phi_bwd_workspace_bytes(p), stream)) != REHYAT_OK)
+    return st;
+  char* ws = static_cast<char*>(workspace);
+  const FwdWorkspace w = fwd_layout(p);
+  const int BH = p->batch * p->heads, HW = p->Hs * p->Ws;
+  int QS, KS;
+  phi_bwd_split(p->T, p->Tc, HW, &QS, &KS);
+  const float* partials = reinterpret_cast<const float*>(ws + w.total);
+  const size_t rows = static_cast<size_t>(BH) * p->T * HW;
+  char* scratch = ws + rehyat_phi_bwd_workspace_bytes(p);
+  AttnBwdParams a;
+  a.q = q; a.k = k; a.v = v; a.y = y; a.dy = dy; a.c = c; a.den = den;
+  a.Wq = phi->Wq; a.bq = phi->bq; a.Wk = phi->Wk; a.bk = phi->bk;
+  a.SL = reinterpret_cast<const float*>(ws + w.SL_off);
+  a.zL = reinterpret_cast<const float*>(ws + w.zL_off);
+  a.ghat = partials + phi_bwd_ghat_offset_floats(BH, nchunks_of(p), p->D, p->Dp, QS);
+  a.r = reinterpret_cast<float*>(scratch);
+  a.Dc = reinterpret_cast<float*>(scratch + align_up(rows * sizeof(float)));
+  a.jstar = reinterpret_cast<int*>(scratch + 2 * align_up(rows * sizeof(float)));
+  a.dq = dq; a.dk = dk; a.dv = dv;
+  a.BH = BH; a.heads = p->heads; a.T = p->T; a.HW = HW; a.D = p->D; a.Dp = p->Dp;
+  a.Tc = p->Tc; a.To = p->To; a.causal = p->causal; a.nchunks = nchunks_of(p);
+  a.in_bf16 = p->in_dtype == REHYAT_BF16;
+  a.FP = p->Dp > 128 ? p->Dp / 128 : 1;
+  a.scale = p->scale > 0.f ? p->scale : 1.0f / sqrtf(static_cast<float>(p->D));
+  return to_status(launch_attn_bwd_simt(a, static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -94,6 +94,30 @@ void phi_bwd_split(int T, int Tc, int HW, int* QS, int* KS);
 size_t phi_bwd_partial_floats(int BH, int T, int nchunks, int D, int Dp, int QS, int KS);
 cudaError_t launch_phi_bwd(const PhiBwdArgs& a, cudaStream_t s);
 
+// Offset (in floats) of the Ghat blocks inside the partials array of
+// launch_phi_bwd: per (b*h, feature piece of 128, slice) a [128][D] block
+// Ghat_s (feature-major) followed by hhat_s [128].
+size_t phi_bwd_ghat_offset_floats(int BH, int nchunks, int D, int Dp, int QS);
+
+// Full backward of the hybrid attention (attn_bwd.cu): dq, dk, dv given the
+// forward's inputs, y, dy = dL/dy, the stabiliser c and the joint
+// denominator den per query, the linear-set state per chunk (SL image
+// layout, zL) and the Ghat blocks of the feature-map backward.  r, Dc, jstar
+// are per-query scratch [BH][N] the dq kernel writes and the dk/dv kernel
+// reads.
+struct AttnBwdParams {
+  const void *q, *k, *v;
+  const float *y, *dy, *c, *den;
+  const float *Wq, *bq, *Wk, *bk;
+  const float *SL, *zL, *ghat;
+  float *r, *Dc;
+  int* jstar;
+  float *dq, *dk, *dv;
+  int BH, heads, T, HW, D, Dp, Tc, To, causal, nchunks, in_bf16, FP;
+  float scale;
+};
+cudaError_t launch_attn_bwd_simt(const AttnBwdParams& p, cudaStream_t s);
+
 // General feature map (phi_mlp.cu): phi = [psi_1^1 .. psi_P^P],
 // psi = GELU(x W_a + b_a) W_b + b_b per head; x [BH][N][D] (in dtype),
 // phi [BH][N][Dp] fp32.

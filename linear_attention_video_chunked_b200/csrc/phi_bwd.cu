@@ -427,6 +427,12 @@ size_t phi_bwd_partial_floats(int BH, int T, int nchunks, int D, int Dp, int QS,
               static_cast<size_t>(T) * KS * ksz);
 }
 
+size_t phi_bwd_ghat_offset_floats(int BH, int nchunks, int D, int Dp, int QS) {
+  const size_t FP = Dp > kPiece ? Dp / kPiece : 1;
+  return static_cast<size_t>(BH) * FP * nchunks * QS *
+         (2 * static_cast<size_t>(D) * kPiece + 2 * kPiece);
+}
+
 cudaError_t launch_phi_bwd(const PhiBwdArgs& a, cudaStream_t s) {
   BwdParams bp;
   bp.q = a.q; bp.k = a.k; bp.v = a.v;

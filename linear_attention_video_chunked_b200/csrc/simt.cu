@@ -16,6 +16,12 @@
 #include "layout.cuh"
 
 namespace rehyat {
+
+// Rows whose joint denominator n^S + n^L fell below 2^-10 n^S (non-positive,
+// NaN, or cancelled to ~10 bits) in a forward with phi given, since the last
+// reset (see rehyat_denominator_report).
+__device__ unsigned long long rehyat_simt_den_rows = 0;
+
 namespace {
 
 constexpr float kLn2 = 0.69314718055994530942f;
@@ -211,6 +217,10 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(AttnParams P) {
   if (r < nrows) {
     const long long row = qrow_base + r;
     const float den = l + nL;
+    // A signed phi (degree-1 parts) can drive n^L towards -n^S: count the
+    // rows, the output stays as the formula gives it.
+    if (P.phi_q && lane4 == 0 && !(den >= ldexpf(l, -10)))
+      atomicAdd(&rehyat_simt_den_rows, 1ull);
 #pragma unroll
     for (int c = 0; c < D / 4; ++c) {
       const int col = lane4 + 4 * c;
@@ -383,6 +393,48 @@ __global__ void scan_kernel(const float* __restrict__ P, const float* __restrict
           dst[static_cast<long long>(ts--) * stride] += suf;
       }
     }
+  }
+}
+
+// Chunk scan for T <= kScanRegs slices: each thread reads its element of
+// every per-slice state once into registers, then writes each chunk's
+// linear-set sum as a plain sum, in slice order, over the slices of that
+// chunk's linear set (slices < w_t, and in the bidirectional form also
+// slices >= end_t): no total-minus-window subtraction, and P is read once
+// instead of once per direction.
+constexpr int kScanRegs = 32;
+__global__ void scan_regs_kernel(const float* __restrict__ P, const float* __restrict__ z,
+                                 float* __restrict__ SL, float* __restrict__ zL, int T, int Tc,
+                                 int To, int nchunks, int Dp, int D, int causal) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const long long PD = static_cast<long long>(Dp) * D;
+  const long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int bh = blockIdx.y;
+  const float* src;
+  float* dst;
+  long long stride;
+  if (e < PD) {
+    src = P + bh * T * PD + e;
+    dst = SL + bh * nchunks * PD + e;
+    stride = PD;
+  } else if (e < PD + Dp) {
+    src = z + static_cast<long long>(bh) * T * Dp + (e - PD);
+    dst = zL + static_cast<long long>(bh) * nchunks * Dp + (e - PD);
+    stride = Dp;
+  } else {
+    return;
+  }
+  float v[kScanRegs];
+#pragma unroll
+  for (int i = 0; i < kScanRegs; ++i) v[i] = i < T ? src[static_cast<long long>(i) * stride] : 0.f;
+  for (int t = 0; t < nchunks; ++t) {
+    const int first = t * Tc, end = min(T, first + Tc), w = max(first - To, 0);
+    const int lim = causal ? T : end;  // slices >= lim join the linear set
+    float acc = 0.f;
+#pragma unroll
+    for (int i = 0; i < kScanRegs; ++i)
+      if (i < w || (i >= lim && i < T)) acc += v[i];
+    dst[static_cast<long long>(t) * stride] = acc;
   }
 }
 
@@ -564,6 +616,9 @@ cudaError_t launch_scan(const float* P, const float* z, float* SL, float* zL, in
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (T <= kScanRegs)
+    return cudaLaunchKernelEx(&cfg, scan_regs_kernel, P, z, SL, zL, T, Tc, To, nchunks, Dp, D,
+                              causal);
   return cudaLaunchKernelEx(&cfg, scan_kernel, P, z, SL, zL, T, Tc, To, nchunks, Dp, D, causal);
 }
 
@@ -599,6 +654,13 @@ cudaError_t launch_w_images(const float* Wq, void* out_q, const float* Wk, void*
   w_image_kernel<<<grid, 256, 0, s>>>(Wq, static_cast<__nv_bfloat16*>(out_q), Wk,
                                       static_cast<__nv_bfloat16*>(out_k), heads, D, Dp);
   return cudaGetLastError();
+}
+
+cudaError_t read_den_rows_simt(unsigned long long* rows, int reset) {
+  cudaError_t e = cudaMemcpyFromSymbol(rows, rehyat_simt_den_rows, sizeof(*rows));
+  if (e != cudaSuccess || !reset) return e;
+  const unsigned long long zero = 0;
+  return cudaMemcpyToSymbol(rehyat_simt_den_rows, &zero, sizeof(zero));
 }
 
 }  // namespace rehyat

@@ -80,7 +80,7 @@ def _shim():
 
 LAUNCHERS = ("rehyat_hybrid_attn_fwd", "rehyat_hybrid_attn_fwd_host", "rehyat_feature_map_mlp",
              "rehyat_hybrid_attn_fwd_phi", "rehyat_phi_bwd", "rehyat_softmax_attn_fwd",
-             "rehyat_state_init", "rehyat_chunk_step")
+             "rehyat_state_init", "rehyat_chunk_step", "rehyat_hybrid_attn_bwd")
 
 
 @pytest.fixture
@@ -169,6 +169,38 @@ def test_phi_given_feature_map_and_gradient_reach_the_abi(calls):
     assert [c[0] for c in calls] == ["rehyat_feature_map_mlp"] * 2 + [
         "rehyat_hybrid_attn_fwd_phi", "rehyat_phi_bwd"]
     assert tuple(pq.shape) == (2, 3, 315, 128) and set(g) == {"dWq", "dbq", "dWk", "dbk"}
+
+
+def test_full_backward_reaches_the_abi(calls):
+    q, k, v = qkv()
+    y, dy = FakeTensor(q.shape, F32), FakeTensor(q.shape, F32)
+    c, den = FakeTensor(q.shape[:3], F32), FakeTensor(q.shape[:3], F32)
+    g = rh.hybrid_attn_bwd(q, k, v, y, dy, c, den, *phi_params(), **GEOM)
+    (name, a), = calls
+    assert name == "rehyat_hybrid_attn_bwd"
+    assert a[1:4] == (q.data_ptr(), k.data_ptr(), v.data_ptr())
+    assert a[5:9] == (y.data_ptr(), dy.data_ptr(), c.data_ptr(), den.data_ptr())
+    assert a[9:12] == (g["dq"].data_ptr(), g["dk"].data_ptr(), g["dv"].data_ptr())
+    assert all(tuple(g[n].shape) == tuple(q.shape) and g[n].dtype == F32 for n in ("dq", "dk", "dv"))
+    assert a[14] >= rh.rehyat_hybrid_attn_bwd_workspace_bytes(a[0])
+
+
+@pytest.mark.parametrize("bad", ["c_shape", "den_dtype", "dy_shape", "y_bf16"])
+def test_full_backward_refuses_malformed_tensors(calls, bad):
+    q, k, v = qkv()
+    t = dict(y=FakeTensor(q.shape, F32), dy=FakeTensor(q.shape, F32),
+             c=FakeTensor(q.shape[:3], F32), den=FakeTensor(q.shape[:3], F32))
+    if bad == "c_shape":
+        t["c"] = FakeTensor((2, 3, 314), F32)
+    elif bad == "den_dtype":
+        t["den"] = FakeTensor(q.shape[:3], BF)
+    elif bad == "dy_shape":
+        t["dy"] = FakeTensor((2, 3, 315, 64), F32)
+    else:
+        t["y"] = FakeTensor(q.shape, BF)
+    with pytest.raises((ValueError, TypeError)):
+        rh.hybrid_attn_bwd(q, k, v, t["y"], t["dy"], t["c"], t["den"], *phi_params(), **GEOM)
+    assert calls == []
 
 
 def test_softmax_and_streaming_reach_the_abi(calls):

@@ -260,3 +260,37 @@ def test_feature_map_mlp_tensor_cores_gelu_identity_weights():
     bar = 2.0 ** -8 * np.abs(gl) + 1e-6 * np.maximum(1.0, np.abs(u))
     assert np.all(err <= bar), float((err - bar).max())
     assert (u < -3).any() and (u > 3).any()
+
+
+@pytest.mark.parametrize("force_simt", [False, True])
+def test_denominator_report_counts_cancelled_rows(force_simt):
+    """A signed phi_q that drives n^S + n^L below zero on chosen rows: the
+    forward keeps y as the formula gives it and the report counts exactly
+    those rows (tensor-core and CUDA-core kernels)."""
+    p = make_problem(batch=1, heads=2, T=4, Hs=8, Ws=8, D=128, Dp=64, Tc=1, To=0,
+                     causal=False, dtype="bf16", seed=31)
+    dev = device_tensors(p)
+    B, H, N = 1, 2, p.N
+    fk = torch.full((B, H, N, 64), 0.01, dtype=torch.float32, device="cuda")
+    fq = torch.full((B, H, N, 64), 0.01, dtype=torch.float32, device="cuda")
+    bad = torch.zeros(B, H, N, dtype=torch.bool, device="cuda")
+    bad[0, 0, 5:17] = True
+    bad[0, 1, 100:103] = True
+    # n^L = phi_q . z_L with z_L = 0.01 * 64 * (keys in the linear set) > 0:
+    # a large negative phi_q on the chosen rows makes n^S + n^L < 0.
+    fq[bad] = -1e3
+    rh.rehyat_denominator_report(reset=True)
+    y, parts = rh.hybrid_attn_phi(dev["q"], dev["k"], dev["v"], fq, fk, T=p.T, Hs=p.Hs, Ws=p.Ws,
+                                  Tc=p.Tc, To=p.To, causal=p.causal, debug=True,
+                                  force_simt=force_simt)
+    torch.cuda.synchronize()
+    den = parts["nS"] + parts["nL"]
+    assert bool((den[bad] < 0).all()) and bool((den[~bad] > 0).all())
+    assert rh.rehyat_denominator_report(reset=True) == int(bad.sum())
+    assert rh.rehyat_denominator_report() == 0
+    # The closed-form phi (squares) never adds to the count.
+    rh.hybrid_attn(dev["q"], dev["k"], dev["v"], dev["Wq"], dev["bq"], dev["Wk"], dev["bk"],
+                   T=p.T, Hs=p.Hs, Ws=p.Ws, Tc=p.Tc, To=p.To, causal=p.causal,
+                   force_simt=force_simt)
+    torch.cuda.synchronize()
+    assert rh.rehyat_denominator_report() == 0
