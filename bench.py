@@ -39,7 +39,7 @@ WORKLOAD = "wan_480x832_bidir"
 METRIC = "hybrid-attn fwd tokens/s & TFLOP/s (% BF16 tensor peak), 1 B200, 21x30x52 latent"
 L2_FLUSH_BYTES = 256 << 20
 KERNELS_PER_STEP = 4  # weight images, per-slice state, chunk scan, attention
-EXTRAS = ("full_softmax", "fp8_qk", "phi_backward", "general_phi", "streaming")
+EXTRAS = ("full_softmax", "fp8_qk", "phi_backward", "full_backward", "general_phi", "streaming")
 E2E_HEADS_PER_SLAB = 2
 
 
@@ -342,6 +342,71 @@ def measure_phi_backward(rh, p, q, k, v, Wq, bq, Wk, bk, flush, stream, calls=3)
     return {"ms": ms, "calls": calls, "tflops": tflops, "roofline": roof,
             "what": "rehyat_phi_bwd (dW_q, db_q, dW_k, db_k) on the bench workload, bf16 "
                     "q/k/v, fp32 y, dy, den; includes its state pass"}
+
+
+def measure_full_backward(rh, p, q, k, v, Wq, bq, Wk, bk, flush, stream, calls=3):
+    """rehyat_hybrid_attn_bwd on the bench workload: forward with c and the
+    denominators exported, an upstream gradient from a seeded torch generator,
+    then device time per full backward call (dq, dk, dv and the feature-map
+    gradients, its state pass included)."""
+    import torch
+    B, H, N, D = q.shape
+    dev = q.device
+    params = rh.make_params(batch=B, heads=H, T=p.T, Hs=p.Hs, Ws=p.Ws, D=D, Dp=p.Dp, Tc=p.Tc,
+                            To=p.To, causal=p.causal, in_dtype=rh.BF16, out_dtype=rh.F32)
+    sh = stream.cuda_stream
+    phi = rh.RehyatPhi(Wq.data_ptr(), bq.data_ptr(), Wk.data_ptr(), bk.data_ptr())
+    y = torch.empty(B, H, N, D, device=dev)
+    c = torch.empty(B, H, N, device=dev)
+    nS = torch.empty(B, H, N, device=dev)
+    nL = torch.empty(B, H, N, device=dev)
+    dbg = rh.RehyatDebug(None, nS.data_ptr(), c.data_ptr(), None, nL.data_ptr())
+    ws = torch.empty(max(rh.rehyat_workspace_bytes(params),
+                         rh.rehyat_hybrid_attn_bwd_workspace_bytes(params)),
+                     dtype=torch.uint8, device=dev)
+    if rh.rehyat_hybrid_attn_fwd(params, q.data_ptr(), k.data_ptr(), v.data_ptr(), phi,
+                                 y.data_ptr(), ws.data_ptr(), ws.numel(), dbg, sh):
+        raise RuntimeError("rehyat_hybrid_attn_fwd failed")
+    den = nS + nL
+    del nS, nL
+    g = torch.Generator(device=dev).manual_seed(6)
+    dy = torch.randn(B, H, N, D, generator=g, device=dev)
+    out = {n: torch.empty(B, H, N, D, device=dev) for n in ("dq", "dk", "dv")}
+    grads = {n: torch.empty_like(t) for n, t in (("dWq", Wq), ("dbq", bq), ("dWk", Wk), ("dbk", bk))}
+    gs = rh.RehyatPhiGrad(*(grads[n].data_ptr() for n in ("dWq", "dbq", "dWk", "dbk")))
+    call = lambda: rh.rehyat_hybrid_attn_bwd(
+        params, q.data_ptr(), k.data_ptr(), v.data_ptr(), phi, y.data_ptr(), dy.data_ptr(),
+        c.data_ptr(), den.data_ptr(), out["dq"].data_ptr(), out["dk"].data_ptr(),
+        out["dv"].data_ptr(), gs, ws.data_ptr(), ws.numel(), sh)
+    if call():
+        raise RuntimeError("rehyat_hybrid_attn_bwd failed")
+    times = []
+    for _ in range(calls):
+        flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        call()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    ms = sum(times) / len(times)
+    # Algorithmic FLOPs: the softmax branch's backward, 10 D per (query,
+    # window key) pair (S and dP recomputed, dV, dQ, dK), plus the feature-map
+    # part (the phi-gradient extra's count) and the linear branch's token
+    # gradients (dq, dk through phi: 2 D D' each; dv: 2 D D').
+    w = algorithmic_work(B, H, p.T, p.Hs * p.Ws, D, p.Dp, p.Tc, p.To, p.causal)
+    pairs = w["exps"]  # (query, window key) pairs over every (b, h)
+    flops = 10.0 * D * pairs + B * H * N * D * p.Dp * 2.0 * (7 + 2 + 3)
+    del y, c, den, ws, dy, out
+    tflops = flops / (ms / 1e3) / 1e12
+    peaks = load_peaks()
+    return {"ms": ms, "calls": calls, "tflops": tflops,
+            "roofline": {"bound": "tensor", "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": tflops / peaks["bf16_tflops"],
+                         "peak_source": "measured bf16 burst (MEASURED_PEAKS.json)",
+                         "work_per_call": f"{flops:.4e} FLOP"},
+            "what": "rehyat_hybrid_attn_bwd (dq, dk, dv, dW_q, db_q, dW_k, db_k) on the bench "
+                    "workload, bf16 q/k/v, fp32 y, dy, c, den; includes its state pass"}
 
 
 def measure_general_phi(rh, p, q, k, v, flush, stream, calls=3):
@@ -832,6 +897,10 @@ def run_gpu(args, world, rank, local):
     if "phi_backward" in want:
         extra["phi_backward"] = measure_phi_backward(rh, p, q, k, v, Wq, bq, Wk, bk, flush,
                                                      stream)
+        torch.cuda.empty_cache()
+    if "full_backward" in want:
+        extra["full_backward"] = measure_full_backward(rh, p, q, k, v, Wq, bq, Wk, bk, flush,
+                                                       stream)
         torch.cuda.empty_cache()
     if "general_phi" in want:
         extra["general_phi"] = measure_general_phi(rh, p, q, k, v, flush, stream)

@@ -365,8 +365,11 @@ REHYAT_API size_t rehyat_hybrid_attn_bwd_workspace_bytes(const rehyat_params* p)
  *   the sum of the linear-set state gradients over the chunks whose linear
  *   set holds slice s; the parameter gradients are those of rehyat_phi_bwd.
  * Outputs (overwritten, not accumulated): dq, dk, dv fp32 [B][h][N][D];
- * grad's four arrays as for rehyat_phi_bwd.  fp32 arithmetic on CUDA cores;
- * no atomics, so repeated calls agree bit for bit.
+ * grad's four arrays as for rehyat_phi_bwd.  bf16 inputs with D = 128 run
+ * the softmax branch on tensor cores (S, dP and the dq, dk, dv products in
+ * bf16 with fp32 accumulation: P, dS and dy/den are rounded to bf16); every
+ * other shape, fp32 inputs and REHYAT_FLAG_FORCE_SIMT run fp32 CUDA cores.
+ * No atomics, so repeated calls agree bit for bit.
  * Pointers: q, k, v, y, dy, dq, dk, dv, workspace 16-byte aligned; c, den and
  * the parameter gradients 4-byte aligned.  Errors as for
  * rehyat_hybrid_attn_fwd; REHYAT_FLAG_FP8_QK is refused (UNSUPPORTED). */

@@ -565,7 +565,9 @@ size_t rehyat_hybrid_attn_bwd_workspace_bytes(const rehyat_params* p) {
   const size_t phi_ws = rehyat_phi_bwd_workspace_bytes(p);
   if (phi_ws == 0) return 0;
   const size_t rows = static_cast<size_t>(p->batch) * p->heads * p->T * p->Hs * p->Ws;
-  return phi_ws + 3 * align_up(rows * sizeof(float));
+  // Shapes the tensor-core path takes (bf16, D = 128): a bf16 copy of dy / den.
+  const size_t gh = (p->in_dtype == REHYAT_BF16 && p->D == 128) ? align_up(rows * p->D * 2) : 0;
+  return phi_ws + 3 * align_up(rows * sizeof(float)) + gh;
 }
 
 rehyat_status rehyat_hybrid_attn_bwd(const rehyat_params* p, const void* q, const void* k,
@@ -615,7 +617,10 @@ rehyat_status rehyat_hybrid_attn_bwd(const rehyat_params* p, const void* q, cons
   a.in_bf16 = p->in_dtype == REHYAT_BF16;
   a.FP = p->Dp > 128 ? p->Dp / 128 : 1;
   a.scale = p->scale > 0.f ? p->scale : 1.0f / sqrtf(static_cast<float>(p->D));
-  return to_status(launch_attn_bwd_simt(a, static_cast<cudaStream_t>(stream)));
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!(p->flags & REHYAT_FLAG_FORCE_SIMT) && tc_attn_bwd_eligible(a.in_bf16, p->D))
+    return to_status(launch_attn_bwd_tc_path(a, scratch + 3 * align_up(rows * sizeof(float)), s));
+  return to_status(launch_attn_bwd_simt(a, s));
 }
 
 }  // extern "C"

@@ -34,6 +34,8 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <cuda_bf16.h>
+
 #include "internal.h"
 #include "layout.cuh"
 
@@ -376,6 +378,145 @@ __global__ void __launch_bounds__(kThr) bwd_dkv_kernel(AttnBwdParams P) {
   }
 }
 
+// ---------------------------------------------------------------- TC path
+// Per query row (D = 128): r = (dy . y) / den and gh = bf16(dy / den), the
+// A operand of the tensor-core products.  One warp per row, four columns
+// per lane.
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const float* __restrict__ y,
+                                                       const float* __restrict__ dy,
+                                                       const float* __restrict__ den,
+                                                       float* __restrict__ r,
+                                                       uint2* __restrict__ gh, long long rows) {
+  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const float4 g = reinterpret_cast<const float4*>(dy + row * 128)[lane];
+  const float4 yy = reinterpret_cast<const float4*>(y + row * 128)[lane];
+  float acc = g.x * yy.x + g.y * yy.y + g.z * yy.z + g.w * yy.w;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  const float dn = den[row];
+  if (lane == 0) r[row] = acc / dn;
+  const float e0 = g.x / dn, e1 = g.y / dn, e2 = g.z / dn, e3 = g.w / dn;
+  const __nv_bfloat162 lo = __floats2bfloat162_rn(e0, e1), hi = __floats2bfloat162_rn(e2, e3);
+  gh[row * 32 + lane] = make_uint2(*reinterpret_cast<const uint32_t*>(&lo),
+                                   *reinterpret_cast<const uint32_t*>(&hi));
+}
+
+// Linear branch of dq for 32 query rows of one chunk (added to dq):
+// du_q = 2 u_q * (S_L gh - r z_L), dq += sum_f du_q[f] W_q[d][f].
+template <int D>
+__global__ void __launch_bounds__(kThr) bwd_lin_q_kernel(AttnBwdParams P) {
+  extern __shared__ float sm[];
+  float* Qs = sm;                  // [32][D]
+  float* Gs = Qs + kT * D;         // [32][D] gh
+  float* Us = Gs + kT * D;         // [32][Dp] du_q
+  float* rowr = Us + kT * P.Dp;    // [32]
+  const int tid = threadIdx.x;
+  const int t = blockIdx.y, bh = blockIdx.z, h = bh % P.heads;
+  const int first = t * P.Tc, end = min(P.T, first + P.Tc);
+  const long long N = static_cast<long long>(P.T) * P.HW;
+  const long long q0 = static_cast<long long>(first) * P.HW + static_cast<long long>(blockIdx.x) * kT;
+  const long long qend = static_cast<long long>(end) * P.HW;
+  if (q0 >= qend) return;
+  const long long base = static_cast<long long>(bh) * N;
+  const int Dp = P.Dp;
+  for (int i = tid; i < kT * D; i += kThr) {
+    const int rr = i / D, d = i % D;
+    const long long g = q0 + rr;
+    const bool in = g < qend;
+    Qs[i] = in ? ldx(P.q, (base + g) * D + d, P.in_bf16) : 0.f;
+    Gs[i] = in ? P.dy[(base + g) * D + d] / P.den[base + g] : 0.f;
+  }
+  if (tid < kT) rowr[tid] = q0 + tid < qend ? P.r[base + q0 + tid] : 0.f;
+  __syncthreads();
+  const long long sl0 = (static_cast<long long>(bh) * P.nchunks + t) * Dp * D;
+  for (int i = tid; i < kT * Dp; i += kThr) {
+    const int rr = i / Dp, f = i % Dp;
+    float u = P.bq[b_idx(h, Dp, f)], dphi = 0.f;
+    for (int d = 0; d < D; ++d) {
+      u = fmaf(Qs[rr * D + d], P.Wq[w_idx(h, D, Dp, d, f)], u);
+      dphi = fmaf(P.SL[sl0 + sl_index(f, d, D, Dp)], Gs[rr * D + d], dphi);
+    }
+    dphi -= rowr[rr] * P.zL[(static_cast<long long>(bh) * P.nchunks + t) * Dp + f];
+    Us[i] = 2.f * u * dphi;
+  }
+  __syncthreads();
+  const int row = tid >> 3, sub = tid & 7;
+  const long long g = q0 + row;
+  if (g >= qend) return;
+#pragma unroll
+  for (int m = 0; m < D / 8; ++m) {
+    const int d = sub + 8 * m;
+    float lin = 0.f;
+    for (int f = 0; f < Dp; ++f) lin = fmaf(Us[row * Dp + f], P.Wq[w_idx(h, D, Dp, d, f)], lin);
+    P.dq[(base + g) * D + d] += lin;
+  }
+}
+
+// Linear branch of dk, dv for 32 key rows (added to dk, dv): u_k, phi_k,
+// du_k = 2 u_k * (Ghat_s v + hhat_s); dk += du_k W_k^T, dv += Ghat_s^T phi_k.
+template <int D>
+__global__ void __launch_bounds__(kThr) bwd_lin_kv_kernel(AttnBwdParams P) {
+  extern __shared__ float sm[];
+  float* Ks = sm;                  // [32][D]
+  float* Vs = Ks + kT * D;         // [32][D]
+  float* Us = Vs + kT * D;         // [32][Dp] du_k
+  float* Fs = Us + kT * P.Dp;      // [32][Dp] phi_k
+  const int tid = threadIdx.x;
+  const int bh = blockIdx.y, h = bh % P.heads;
+  const long long N = static_cast<long long>(P.T) * P.HW;
+  const long long j0 = static_cast<long long>(blockIdx.x) * kT;
+  if (j0 >= N) return;
+  const long long j1 = min(N, j0 + kT);
+  const long long base = static_cast<long long>(bh) * N;
+  const int Dp = P.Dp, pw = Dp < kGhatPiece ? Dp : kGhatPiece;
+  const long long gn = static_cast<long long>(kGhatPiece) * D + kGhatPiece;
+  for (int i = tid; i < kT * D; i += kThr) {
+    const int rr = i / D, d = i % D;
+    const long long g = j0 + rr;
+    Ks[i] = g < j1 ? ldx(P.k, (base + g) * D + d, P.in_bf16) : 0.f;
+    Vs[i] = g < j1 ? ldx(P.v, (base + g) * D + d, P.in_bf16) : 0.f;
+  }
+  __syncthreads();
+  for (int i = tid; i < kT * Dp; i += kThr) {
+    const int rr = i / Dp, f = i % Dp;
+    const long long g = j0 + rr;
+    float u = 0.f, dphi = 0.f;
+    if (g < j1) {
+      const int sl = static_cast<int>(g / P.HW);
+      const int pf = f / pw, fl = f - pf * pw;
+      const float* gb = P.ghat + ((static_cast<long long>(bh) * P.FP + pf) * P.T + sl) * gn;
+      u = P.bk[b_idx(h, Dp, f)];
+      dphi = gb[static_cast<long long>(kGhatPiece) * D + fl];
+      for (int d = 0; d < D; ++d) {
+        u = fmaf(Ks[rr * D + d], P.Wk[w_idx(h, D, Dp, d, f)], u);
+        dphi = fmaf(gb[static_cast<long long>(fl) * D + d], Vs[rr * D + d], dphi);
+      }
+    }
+    Us[i] = 2.f * u * dphi;
+    Fs[i] = u * u;
+  }
+  __syncthreads();
+  const int kr = tid >> 3, sub = tid & 7;
+  const long long key = j0 + kr;
+  if (key >= j1) return;
+  const int sl = static_cast<int>(key / P.HW);
+#pragma unroll
+  for (int m = 0; m < D / 8; ++m) {
+    const int d = sub + 8 * m;
+    float lk = 0.f, lv = 0.f;
+    for (int f = 0; f < Dp; ++f) {
+      const int pf = f / pw, fl = f - pf * pw;
+      const float* gb = P.ghat + ((static_cast<long long>(bh) * P.FP + pf) * P.T + sl) * gn;
+      lk = fmaf(Us[kr * Dp + f], P.Wk[w_idx(h, D, Dp, d, f)], lk);
+      lv = fmaf(gb[static_cast<long long>(fl) * D + d], Fs[kr * Dp + f], lv);
+    }
+    P.dk[(base + key) * D + d] += lk;
+    P.dv[(base + key) * D + d] += lv;
+  }
+}
+
 template <int D>
 cudaError_t launch_bwd_simt_d(const AttnBwdParams& p, cudaStream_t s) {
   const size_t smq = sizeof(float) * (2 * kT * D + 2 * kT * (D + 1) + kT * 33 +
@@ -401,6 +542,38 @@ cudaError_t launch_bwd_simt_d(const AttnBwdParams& p, cudaStream_t s) {
 }
 
 }  // namespace
+
+cudaError_t launch_attn_bwd_tc_path(const AttnBwdParams& p, void* gh_bf16, cudaStream_t s) {
+  const long long N = static_cast<long long>(p.T) * p.HW;
+  const long long rows = N * p.BH;
+  bwd_prep_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, s>>>(
+      p.y, p.dy, p.den, p.r, static_cast<uint2*>(gh_bf16), rows);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  AttnBwdTcArgs a;
+  a.q = p.q; a.k = p.k; a.v = p.v; a.gh = gh_bf16;
+  a.c = p.c; a.r = p.r; a.Dc = p.Dc; a.jstar = p.jstar;
+  a.dq = p.dq; a.dk = p.dk; a.dv = p.dv;
+  a.BH = p.BH; a.T = p.T; a.HW = p.HW; a.Tc = p.Tc; a.To = p.To; a.nchunks = p.nchunks;
+  a.scale = p.scale;
+  if ((e = launch_attn_bwd_dq_tc(a, s)) != cudaSuccess) return e;
+  if ((e = launch_attn_bwd_dkv_tc(a, s)) != cudaSuccess) return e;
+  // The linear branch's parts, added to dq, dk, dv.
+  constexpr int D = 128;
+  const size_t smq = sizeof(float) * (2 * kT * D + static_cast<size_t>(kT) * p.Dp + kT);
+  const size_t smk = sizeof(float) * (2 * kT * D + 2 * static_cast<size_t>(kT) * p.Dp);
+  if ((e = cudaFuncSetAttribute(bwd_lin_q_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(smq))) != cudaSuccess)
+    return e;
+  if ((e = cudaFuncSetAttribute(bwd_lin_kv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(smk))) != cudaSuccess)
+    return e;
+  const int chunk_rows = (p.Tc < p.T ? p.Tc : p.T) * p.HW;
+  bwd_lin_q_kernel<D><<<dim3((chunk_rows + kT - 1) / kT, p.nchunks, p.BH), kThr, smq, s>>>(p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  bwd_lin_kv_kernel<D><<<dim3(static_cast<unsigned>((N + kT - 1) / kT), p.BH), kThr, smk, s>>>(p);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_attn_bwd_simt(const AttnBwdParams& p, cudaStream_t s) {
   switch (p.D) {

@@ -117,6 +117,22 @@ struct AttnBwdParams {
   float scale;
 };
 cudaError_t launch_attn_bwd_simt(const AttnBwdParams& p, cudaStream_t s);
+// Tensor-core path (bf16, D = 128): prep (r, gh = bf16(dy / den) into
+// gh_bf16, [BH][N][128]), the dq and dk/dv kernels of tc_attn_bwd.cuh, then
+// the linear branch's parts added on CUDA cores.
+bool tc_attn_bwd_eligible(int in_bf16, int D);
+struct AttnBwdTcArgs {
+  const void *q, *k, *v, *gh;  // bf16 [BH][N][128]
+  const float *c, *r;          // per query [BH][N]: stabiliser, (g . y) / den
+  float* Dc;                   // per query: written by the dq kernel, read by dk/dv
+  int* jstar;                  // per query: arg-max key (absolute row), likewise
+  float *dq, *dk, *dv;         // fp32 [BH][N][128], overwritten
+  int BH, T, HW, Tc, To, nchunks;
+  float scale;
+};
+cudaError_t launch_attn_bwd_dq_tc(const AttnBwdTcArgs& a, cudaStream_t s);
+cudaError_t launch_attn_bwd_dkv_tc(const AttnBwdTcArgs& a, cudaStream_t s);
+cudaError_t launch_attn_bwd_tc_path(const AttnBwdParams& p, void* gh_bf16, cudaStream_t s);
 
 // General feature map (phi_mlp.cu): phi = [psi_1^1 .. psi_P^P],
 // psi = GELU(x W_a + b_a) W_b + b_b per head; x [BH][N][D] (in dtype),

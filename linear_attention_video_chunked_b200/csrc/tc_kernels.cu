@@ -540,7 +540,7 @@ constexpr uint32_t kK8Stage = 16384;
 constexpr uint32_t kQ8Off = kKOff + 3 * kK8Stage;
 enum { Q_FULL = 0, K_FULL = 1, K_EMPTY = 4, V_FULL = 7, V_EMPTY = 9, S_FULL = 11, P_FULL = 13,
        PV_DONE = 15, LAST_PV = 17, TAIL_FULL = 18, PHI_DONE = 19, PHI_READY = 20, READ_DONE = 22,
-       VEC_READY = 23, XCHG = 24, LX = 26, LX_DONE = 27, NBAR = 28 };
+       VEC_READY = 23, XCHG = 24, LX = 26, LX_DONE = 27, READ_A = 28, NBAR = 29 };
 // Row halves: each softmax thread owns 64 of a row's 128 key columns; the
 // two threads of a row (warps w and w + 4, same TMEM lane quarter) trade
 // their partial row maxima through TMEM column 63 (half 0) and 127 (half 1)
@@ -616,7 +616,9 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
   const int nt = nta + (nb + kBN - 1) / kBN;
   const bool linear = !P.full_softmax;
   const bool phi_given = P.phi_q != nullptr;  // phi_q(q) read from P.phi_q
-  const int Dp = P.Dp;  // <= 128 here: one feature piece
+  const int Dp = P.Dp;
+  const int npieces = Dp > 128 ? 2 : 1;       // feature pieces of the readout
+  const int pw = Dp / npieces;
 
   auto tile_src = [&](int j) {
     TileSrc s;
@@ -693,20 +695,25 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
         tma_load_3d(vdst + 16384, src.map_v, bar(a2::V_FULL + vs), 64, src.row, bh);
       }
       if (linear && ok) {
-        const uint32_t wbytes = static_cast<uint32_t>(Dp) * kD * 2;
-        const uint32_t slbytes = static_cast<uint32_t>(Dp) * kD * 4;
+        const uint32_t wbytes = static_cast<uint32_t>(pw) * kD * 2;
+        const uint32_t slbytes = static_cast<uint32_t>(pw) * kD * 4;
         // The tail operands go into the K ring as soon as the last three K
         // tiles have been consumed (their q.k^T MMAs completed), while the
-        // last softmax steps and P.V still run.
+        // last softmax steps and P.V still run; with two feature pieces the
+        // second piece follows once both readouts of the first are done.
         for (int tt = max(0, nt - 3); tt < nt && ok; ++tt)
           ok = mbar_wait(bar(a2::K_EMPTY + tt % 3), (tt / 3) & 1, abort_flag, 2);
-        if (ok) {
+        for (int pc = 0; pc < npieces && ok; ++pc) {
+          if (pc > 0) ok = mbar_wait(bar(a2::READ_DONE), (pc - 1) & 1, abort_flag, 2);
+          if (!ok) break;
           // With phi_q(q) given there is no W_q image to load.
           mbar_expect_tx(bar(a2::TAIL_FULL), (phi_given ? 0u : wbytes) + slbytes);
           if (!phi_given)
-            bulk_load(base + kWOff, wq_img + static_cast<long long>(h) * Dp * kD, wbytes,
-                      bar(a2::TAIL_FULL));
-          bulk_load(base + kSLOff, P.SL + (static_cast<long long>(bh) * P.nchunks + t) * Dp * kD,
+            bulk_load(base + kWOff, wq_img + (static_cast<long long>(h) * Dp + pc * pw) * kD,
+                      wbytes, bar(a2::TAIL_FULL));
+          bulk_load(base + kSLOff,
+                    P.SL + (static_cast<long long>(bh) * P.nchunks + t) * Dp * kD +
+                        static_cast<long long>(pc) * pw * kD,
                     slbytes, bar(a2::TAIL_FULL));
         }
       }
@@ -773,39 +780,43 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
         if (more) mma_commit(bar(a2::K_EMPTY + (j + 1) % 3));
         if (j == nt - 1) mma_commit(bar(a2::LAST_PV));
       }
-      if (linear && ok) {
-        ok = mbar_wait(bar(a2::TAIL_FULL), 0, abort_flag, 9);
-        if (ok) {
-          // The phi_q product overwrites S: the softmax warps have traded
-          // their row sums through it first.
-          if (!phi_given) ok = mbar_wait(bar(a2::LX_DONE), 0, abort_flag, 18);
-          tc_fence_after();
-          if (ok && !phi_given) {
-            const uint32_t id_phi = idesc(kBM, Dp, 1, false);
-            for (int tile = 0; tile < ntiles; ++tile)
+      // Linear readout, one feature piece of pw <= 128 at a time.
+      for (int pc = 0; linear && ok && pc < npieces; ++pc) {
+        ok = mbar_wait(bar(a2::TAIL_FULL), pc & 1, abort_flag, 9);
+        // The phi_q product overwrites S: the softmax warps have traded
+        // their row sums through it first.
+        if (ok && pc == 0 && !phi_given) ok = mbar_wait(bar(a2::LX_DONE), 0, abort_flag, 18);
+        if (!ok) break;
+        tc_fence_after();
+        if (!phi_given) {
+          const uint32_t id_phi = idesc(kBM, pw, 1, false);
+          for (int tile = 0; tile < ntiles; ++tile)
 #pragma unroll
-              for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t qoff = tile * 32768 + (kk >> 2) * 16384 + (kk & 3) * 32;
-                const uint32_t woff = (kk >> 2) * (Dp * 128) + (kk & 3) * 32;
-                mma_bf16(tmem + tile * 256, sdesc(base + kQOff + qoff, 16, 1024),
-                         sdesc(base + kWOff + woff, 16, 1024), id_phi, kk > 0);
-              }
-            mma_commit(bar(a2::PHI_DONE));
-          }
-          const uint32_t id_rd = idesc(kBM, kD, 2, false);
-          for (int tile = 0; tile < ntiles && ok; ++tile) {
-            ok = mbar_wait(bar(a2::PHI_READY + tile), 0, abort_flag, 10);
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t phi = base + (tile ? kPhiOff1 : kPhiOff0);
-            for (int kk = 0; kk < Dp / 8; ++kk) {
-              const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-              mma_tf32(tmem + tile * 256 + 128, sdesc(phi + off, 16, 1024),
-                       sdesc(base + kSLOff + off, 16, 1024), id_rd, 1u);
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t qoff = tile * 32768 + (kk >> 2) * 16384 + (kk & 3) * 32;
+              const uint32_t woff = (kk >> 2) * (pw * 128) + (kk & 3) * 32;
+              mma_bf16(tmem + tile * 256, sdesc(base + kQOff + qoff, 16, 1024),
+                       sdesc(base + kWOff + woff, 16, 1024), id_phi, kk > 0);
             }
-          }
-          if (ok) mma_commit(bar(a2::READ_DONE));
+          mma_commit(bar(a2::PHI_DONE));
         }
+        const uint32_t id_rd = idesc(kBM, kD, 2, false);
+        for (int tile = 0; tile < ntiles && ok; ++tile) {
+          ok = mbar_wait(bar(a2::PHI_READY + tile), pc & 1, abort_flag, 10);
+          if (!ok) break;
+          tc_fence_after();
+          // One piece: tile A's phi_q sits in the V ring, tile B's over Q.
+          // Two pieces: Q is read again for the second piece, so both tiles
+          // stage in the V ring, tile B after tile A's readout (READ_A).
+          const uint32_t phi = base + ((tile && npieces == 1) ? kPhiOff1 : kPhiOff0);
+          for (int kk = 0; kk < pw / 8; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            mma_tf32(tmem + tile * 256 + 128, sdesc(phi + off, 16, 1024),
+                     sdesc(base + kSLOff + off, 16, 1024), id_rd, 1u);
+          }
+          if (tile == 0 && npieces > 1) mma_commit(bar(a2::READ_A));
+        }
+        if (ok) mma_commit(bar(a2::READ_DONE));
       }
     }
     __syncwarp();
@@ -830,8 +841,9 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
     float* vec = reinterpret_cast<float*>(sbase + a2::kVecOff);  // [b_q (D') | z^L (D')]
     if (linear && hf == 0) {
       // Warps 0-3 stage b_q and z^L for the tail while they wait for the
-      // first scores (b_q of head h is h's D' consecutive values).
-      if (r < Dp) {
+      // first scores (b_q of head h is h's D' consecutive values; one
+      // feature piece only, D' <= 128).
+      if (r < Dp && npieces == 1) {
         vec[r] = phi_given ? 0.f : __ldg(P.bq + h * Dp + r);
         vec[Dp + r] = __ldg(P.zL + (static_cast<long long>(bh) * P.nchunks + t) * Dp + r);
       }
@@ -994,17 +1006,31 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
           }
         }
       }
-      // phi_q(q) is staged into the V ring (tile A) and over Q (tile B):
-      // with the closed form that waits for the phi MMAs (which read Q);
-      // with phi_q given, for the last P.V (every MMA of the loop is done).
-      if (ok) ok = wait_all(bar(a2::VEC_READY), 0, 14) &&
-                   wait_all(bar(phi_given ? a2::LAST_PV : a2::PHI_DONE), 0, 14);
-      if (ok) {
+      // phi_q(q) of each feature piece is staged as a tf32 operand.  One
+      // piece: tile A in the V ring, tile B over Q; the closed form waits for
+      // the phi MMAs (which read Q), phi_q given for the last P.V.  Two
+      // pieces: both tiles in the V ring (Q is read again for the second
+      // piece), tile B once tile A's readout of the piece has run (READ_A),
+      // tile A's second piece once the first piece's readouts have run; b_q
+      // and z^L come straight from global memory (the staged copy in shared
+      // memory holds one piece).
+      const float inv_f = 1.0f / fscale;
+      const uint32_t phi = base + ((tile && npieces == 1) ? kPhiOff1 : kPhiOff0);
+      for (int pc = 0; ok && pc < npieces; ++pc) {
+        if (npieces == 1) {
+          ok = wait_all(bar(a2::VEC_READY), 0, 14) &&
+               wait_all(bar(phi_given ? a2::LAST_PV : a2::PHI_DONE), 0, 14);
+        } else {
+          ok = wait_all(bar(phi_given ? a2::LAST_PV : a2::PHI_DONE), phi_given ? 0 : (pc & 1), 14);
+          if (ok && tile == 1) ok = wait_all(bar(a2::READ_A), pc & 1, 14);
+          if (ok && tile == 0 && pc > 0) ok = wait_all(bar(a2::READ_DONE), (pc - 1) & 1, 14);
+        }
+        if (!ok) break;
         tc_fence_after();
-        const float inv_f = 1.0f / fscale;
-        const uint32_t phi = base + (tile ? kPhiOff1 : kPhiOff0);
-        const float* given = phi_given && r < nrows ? P.phi_q + grow * Dp : nullptr;
-        for (int c = 0; c < Dp / 32; ++c) {
+        const int f0 = pc * pw;
+        const float* given = phi_given && r < nrows ? P.phi_q + grow * Dp + f0 : nullptr;
+        const float* zsrc = P.zL + (static_cast<long long>(bh) * P.nchunks + t) * Dp + f0;
+        for (int c = 0; c < pw / 32; ++c) {
           float ph[32];
           if (phi_given) {
 #pragma unroll
@@ -1022,13 +1048,15 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-              const float psi = __uint_as_float(v[i]) + vec[c * 32 + i];
+              const float b = npieces == 1 ? vec[c * 32 + i] : __ldg(P.bq + h * Dp + f0 + c * 32 + i);
+              const float psi = __uint_as_float(v[i]) + b;
               ph[i] = psi * psi;
             }
           }
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            nL = fmaf(ph[i], vec[Dp + c * 32 + i], nL);
+            const float z = npieces == 1 ? vec[Dp + c * 32 + i] : __ldg(zsrc + c * 32 + i);
+            nL = fmaf(ph[i], z, nL);
             ph[i] *= inv_f;
           }
           const uint32_t rowaddr = phi + c * 16384 + r * 128;
@@ -1041,8 +1069,8 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
         fence_proxy_async();
         tc_fence_before();
         mbar_arrive(bar(a2::PHI_READY + tile));
-        ok = wait_all(bar(a2::READ_DONE), 0, 15);
       }
+      if (ok) ok = wait_all(bar(a2::READ_DONE), (npieces - 1) & 1, 15);
     } else if (ok) {
       ok = wait_all(bar(a2::LAST_PV), 0, 15);
     }
@@ -1738,9 +1766,9 @@ bool tc_attn_supported(const AttnParams& p) {
   if (!p.in_bf16 || p.D != kD) return false;
   if (!p.full_softmax) {
     if (!tc_attn_eligible(p.in_bf16, p.D, p.Dp)) return false;
-    // phi_q given: the two-query-tile kernel (D' <= 128) reads it in its tail.
+    // phi_q given: the two-query-tile kernel reads it in its tail.
     if (p.phi_q != nullptr) {
-      if (p.Dp > 128 || p.one_tile) return false;
+      if (p.one_tile) return false;
     } else if (p.wq_img == nullptr) {
       return false;
     }
@@ -1766,7 +1794,7 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s) {
     }
   }
   const int qrows_max = p.seen ? p.nq_slices * p.HW : (p.Tc < p.T ? p.Tc : p.T) * p.HW;
-  const bool two_tiles = !p.one_tile && (p.full_softmax || p.Dp <= 128);
+  const bool two_tiles = !p.one_tile;
   cudaError_t e;
   if (p.q8 != nullptr) {  // fp8 softmax variant (full forward, two-tile kernel only)
     if (!two_tiles || p.seen || !make_map8(&maps.q8, p.q8, p.rows_per_bh, p.BH) ||
@@ -1795,8 +1823,10 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s) {
 
 }  // namespace rehyat
 
-// The general feature map's tensor-core kernel shares this unit's helpers.
+// The general feature map's and the backward's tensor-core kernels share
+// this unit's helpers.
 #include "tc_phi_mlp.cuh"
+#include "tc_attn_bwd.cuh"
 
 namespace rehyat {
 cudaError_t read_den_rows_simt(unsigned long long* rows, int reset);

@@ -231,6 +231,47 @@ int main(void) {
 """
 
 
+def test_full_backward_argument_checks():
+    p = _params()
+    phi = rh.RehyatPhi(4096, 4096, 4096, 4096)
+    grad = rh.RehyatPhiGrad(4096, 4096, 4096, 4096)
+    ws = rh.rehyat_hybrid_attn_bwd_workspace_bytes(p)
+    assert ws > rh.rehyat_phi_bwd_workspace_bytes(p)  # plus r, Dc, j* and bf16 dy / den
+    rows = 2 * 3 * 7 * 5 * 6
+    assert ws - rh.rehyat_phi_bwd_workspace_bytes(p) >= 3 * 4 * rows + 2 * 128 * rows
+    f = rh.rehyat_hybrid_attn_bwd
+    # p, q, k, v, phi, y, dy, c, den, dq, dk, dv, grad, workspace, ws_bytes, stream
+    args = [p, 4096, 4096, 4096, phi, 4096, 4096, 4096, 4096, 4096, 4096, 4096, grad, 4096, ws,
+            None]
+
+    def call(**change):
+        a = list(args)
+        for i, val in change.items():
+            a[int(i[1:])] = val
+        return f(*a)
+
+    assert call(a7=0) == 1                                               # null c
+    assert call(a8=0) == 1                                               # null den
+    assert call(a10=0) == 1                                              # null dk
+    assert call(a12=rh.RehyatPhiGrad(4096, 4096, 0, 4096)) == 1          # null dW_k
+    assert call(a4=rh.RehyatPhi(4096, 0, 4096, 4096)) == 1               # null b_q
+    assert call(a9=4104) == 3                                            # dq not 16-byte aligned
+    assert call(a7=4098) == 3                                            # c not 4-byte aligned
+    assert call(a14=ws - 1) == 4
+    assert call(a0=_params(flags=rh.FLAG_FP8_QK)) == 2
+    assert call(a0=_params(D=48)) == 2
+    assert rh.rehyat_hybrid_attn_bwd_workspace_bytes(_params(flags=rh.FLAG_FP8_QK)) == 0
+    assert rh.rehyat_hybrid_attn_bwd_workspace_bytes(_params(T=0)) == 0
+    # fp32 inputs or another D: no bf16 copy of dy / den.
+    p32 = _params(in_dtype=rh.F32)
+    assert (rh.rehyat_hybrid_attn_bwd_workspace_bytes(p32) - rh.rehyat_phi_bwd_workspace_bytes(p32)
+            < 3 * 4 * rows + 3 * 256 + 1)
+
+
+def test_denominator_report_needs_an_output():
+    assert rh.lib().rehyat_denominator_report(None, 0) == 1
+
+
 def test_header_is_plain_c_and_the_library_links_from_c(tmp_path):
     """include/rehyat.h compiles as strict C99 with no warnings, and a C
     program linked against librehyat.so gets the same answers as the

@@ -89,7 +89,7 @@ SHAPES = [
     # B, h, T, Hs, Ws, D, Dp, Tc, To, causal
     (1, 2, 5, 7, 9, 128, 128, 2, 1, False),    # ragged tiles
     (1, 2, 7, 10, 13, 128, 64, 3, 2, True),
-    (1, 2, 5, 9, 15, 128, 256, 2, 1, False),   # D' = 256: state halves, CUDA-core attention
+    (1, 2, 5, 9, 15, 128, 256, 2, 1, False),   # D' = 256: state halves, two readout pieces
 ]
 
 
