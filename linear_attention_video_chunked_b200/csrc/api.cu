@@ -523,10 +523,18 @@ size_t rehyat_phi_bwd_workspace_bytes(const rehyat_params* p) {
   return fwd_layout(p).total + align_up(parts * sizeof(float));
 }
 
-rehyat_status rehyat_phi_bwd(const rehyat_params* p, const void* q, const void* k, const void* v,
-                             const float* y, const float* dy, const float* den,
-                             const rehyat_phi* phi, const rehyat_phi_grad* grad,
-                             void* workspace, size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace rehyat {
+namespace {
+
+// The feature-map backward; with dq, dk, dv non-null and the tensor-core
+// passes in use, it also adds the linear branch's token gradients to them.
+rehyat_status phi_bwd_impl(const rehyat_params* p, const void* q, const void* k, const void* v,
+                           const float* y, const float* dy, const float* den,
+                           const rehyat_phi* phi, const rehyat_phi_grad* grad, void* workspace,
+                           size_t ws_bytes, void* stream, float* dq, float* dk, float* dv,
+                           bool* added) {
   rehyat_status st = check_params(p);
   if (st != REHYAT_OK) return st;
   if ((st = no_fp8(p)) != REHYAT_OK) return st;
@@ -558,7 +566,24 @@ rehyat_status rehyat_phi_bwd(const rehyat_params* p, const void* q, const void* 
   a.tc = tc_path(p) && tc_phi_bwd_eligible(a.in_bf16, p->D, p->Dp);
   a.wq_img = a.tc ? ws + w.wimg_off : nullptr;
   a.wk_img = a.tc ? ws + w.wkimg_off : nullptr;
+  a.dq = a.tc ? dq : nullptr;
+  a.dk = a.tc ? dk : nullptr;
+  a.dv = a.tc ? dv : nullptr;
+  if (added) *added = a.tc && dq != nullptr;
   return to_status(launch_phi_bwd(a, s));
+}
+
+}  // namespace
+}  // namespace rehyat
+
+extern "C" {
+
+rehyat_status rehyat_phi_bwd(const rehyat_params* p, const void* q, const void* k, const void* v,
+                             const float* y, const float* dy, const float* den,
+                             const rehyat_phi* phi, const rehyat_phi_grad* grad,
+                             void* workspace, size_t ws_bytes, void* stream) {
+  return rehyat::phi_bwd_impl(p, q, k, v, y, dy, den, phi, grad, workspace, ws_bytes, stream,
+                              nullptr, nullptr, nullptr, nullptr);
 }
 
 size_t rehyat_hybrid_attn_bwd_workspace_bytes(const rehyat_params* p) {
@@ -589,11 +614,6 @@ rehyat_status rehyat_hybrid_attn_bwd(const rehyat_params* p, const void* q, cons
       !a4(den) || !a4(grad->dWq) || !a4(grad->dbq) || !a4(grad->dWk) || !a4(grad->dbk))
     return REHYAT_ERR_MISALIGNED;
   if (ws_bytes < rehyat_hybrid_attn_bwd_workspace_bytes(p)) return REHYAT_ERR_WORKSPACE;
-  // Gradients of the feature-map parameters, and on the way the linear-set
-  // state per chunk (S_L, z_L) and the Ghat blocks the token gradients use.
-  if ((st = rehyat_phi_bwd(p, q, k, v, y, dy, den, phi, grad, workspace,
-                           rehyat_phi_bwd_workspace_bytes(p), stream)) != REHYAT_OK)
-    return st;
   char* ws = static_cast<char*>(workspace);
   const FwdWorkspace w = fwd_layout(p);
   const int BH = p->batch * p->heads, HW = p->Hs * p->Ws;
@@ -618,8 +638,24 @@ rehyat_status rehyat_hybrid_attn_bwd(const rehyat_params* p, const void* q, cons
   a.FP = p->Dp > 128 ? p->Dp / 128 : 1;
   a.scale = p->scale > 0.f ? p->scale : 1.0f / sqrtf(static_cast<float>(p->D));
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (!(p->flags & REHYAT_FLAG_FORCE_SIMT) && tc_attn_bwd_eligible(a.in_bf16, p->D))
-    return to_status(launch_attn_bwd_tc_path(a, scratch + 3 * align_up(rows * sizeof(float)), s));
+  const size_t phi_ws = rehyat_phi_bwd_workspace_bytes(p);
+  if (!(p->flags & REHYAT_FLAG_FORCE_SIMT) && tc_attn_bwd_eligible(a.in_bf16, p->D)) {
+    // Softmax branch on tensor cores (writes dq, dk, dv), then the
+    // feature-map backward, whose tensor-core passes add the linear branch's
+    // token gradients; otherwise those come from CUDA-core kernels after it.
+    cudaError_t e = launch_attn_bwd_tc_softmax(a, scratch + 3 * align_up(rows * sizeof(float)), s);
+    if (e != cudaSuccess) return to_status(e);
+    bool added = false;
+    if ((st = phi_bwd_impl(p, q, k, v, y, dy, den, phi, grad, workspace, phi_ws, stream, dq, dk,
+                           dv, &added)) != REHYAT_OK)
+      return st;
+    return added ? REHYAT_OK : to_status(launch_attn_bwd_lin_simt(a, s));
+  }
+  // CUDA cores: the feature-map backward first (S_L, z_L and the Ghat blocks
+  // the token gradients use), then dq and dk/dv with the linear parts fused.
+  if ((st = phi_bwd_impl(p, q, k, v, y, dy, den, phi, grad, workspace, phi_ws, stream, nullptr,
+                         nullptr, nullptr, nullptr)) != REHYAT_OK)
+    return st;
   return to_status(launch_attn_bwd_simt(a, s));
 }
 

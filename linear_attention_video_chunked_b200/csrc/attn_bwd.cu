@@ -543,7 +543,7 @@ cudaError_t launch_bwd_simt_d(const AttnBwdParams& p, cudaStream_t s) {
 
 }  // namespace
 
-cudaError_t launch_attn_bwd_tc_path(const AttnBwdParams& p, void* gh_bf16, cudaStream_t s) {
+cudaError_t launch_attn_bwd_tc_softmax(const AttnBwdParams& p, void* gh_bf16, cudaStream_t s) {
   const long long N = static_cast<long long>(p.T) * p.HW;
   const long long rows = N * p.BH;
   bwd_prep_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, s>>>(
@@ -557,9 +557,14 @@ cudaError_t launch_attn_bwd_tc_path(const AttnBwdParams& p, void* gh_bf16, cudaS
   a.BH = p.BH; a.T = p.T; a.HW = p.HW; a.Tc = p.Tc; a.To = p.To; a.nchunks = p.nchunks;
   a.scale = p.scale;
   if ((e = launch_attn_bwd_dq_tc(a, s)) != cudaSuccess) return e;
-  if ((e = launch_attn_bwd_dkv_tc(a, s)) != cudaSuccess) return e;
+  return launch_attn_bwd_dkv_tc(a, s);
+}
+
+cudaError_t launch_attn_bwd_lin_simt(const AttnBwdParams& p, cudaStream_t s) {
   // The linear branch's parts, added to dq, dk, dv.
   constexpr int D = 128;
+  cudaError_t e;
+  const long long N = static_cast<long long>(p.T) * p.HW;
   const size_t smq = sizeof(float) * (2 * kT * D + static_cast<size_t>(kT) * p.Dp + kT);
   const size_t smk = sizeof(float) * (2 * kT * D + 2 * static_cast<size_t>(kT) * p.Dp);
   if ((e = cudaFuncSetAttribute(bwd_lin_q_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,

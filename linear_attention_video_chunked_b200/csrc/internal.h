@@ -72,6 +72,9 @@ struct PhiBwdArgs {
   const void *wq_img, *wk_img;  // bf16 weight images (tensor-core passes) or nullptr
   float *partials;
   float *dWq, *dbq, *dWk, *dbk;
+  // Tensor-core passes only: the linear branch's token gradients are added
+  // into dq, dk, dv when non-null (the full backward).
+  float *dq, *dk, *dv;
   int batch, heads, T, HW, D, Dp, Tc, To, causal, nchunks, in_bf16;
   int tc;                       // run the q and k passes on tcgen05
 };
@@ -85,6 +88,10 @@ struct PhiBwdTcArgs {
   const float* M;             // q: S_L per chunk (image layout); k: Ghat blocks per slice
   const float* vec;           // q: z_L per chunk (k: hhat, inside the Ghat block)
   float* part;                // partial blocks of the pass
+  // Optional token gradients of the linear branch, added in place (fp32
+  // [BH][N][128]; null = not computed): q pass dx = dq (du_q W_q); k pass
+  // dx = dk (du_k W_k) and dv += Ghat_s^T phi_k(k).
+  float *dx, *dv;
   int BH, heads, T, HW, Tc, nchunks, splits, q_side;
 };
 bool tc_phi_bwd_eligible(int in_bf16, int D, int Dp);
@@ -118,8 +125,8 @@ struct AttnBwdParams {
 };
 cudaError_t launch_attn_bwd_simt(const AttnBwdParams& p, cudaStream_t s);
 // Tensor-core path (bf16, D = 128): prep (r, gh = bf16(dy / den) into
-// gh_bf16, [BH][N][128]), the dq and dk/dv kernels of tc_attn_bwd.cuh, then
-// the linear branch's parts added on CUDA cores.
+// gh_bf16, [BH][N][128]) and the dq and dk/dv kernels of tc_attn_bwd.cuh
+// (the softmax branch); the linear branch's parts are added afterwards.
 bool tc_attn_bwd_eligible(int in_bf16, int D);
 struct AttnBwdTcArgs {
   const void *q, *k, *v, *gh;  // bf16 [BH][N][128]
@@ -132,7 +139,10 @@ struct AttnBwdTcArgs {
 };
 cudaError_t launch_attn_bwd_dq_tc(const AttnBwdTcArgs& a, cudaStream_t s);
 cudaError_t launch_attn_bwd_dkv_tc(const AttnBwdTcArgs& a, cudaStream_t s);
-cudaError_t launch_attn_bwd_tc_path(const AttnBwdParams& p, void* gh_bf16, cudaStream_t s);
+cudaError_t launch_attn_bwd_tc_softmax(const AttnBwdParams& p, void* gh_bf16, cudaStream_t s);
+// The linear branch's token gradients on CUDA cores, added to dq, dk, dv
+// (D = 128; used when the feature-map passes do not run on tensor cores).
+cudaError_t launch_attn_bwd_lin_simt(const AttnBwdParams& p, cudaStream_t s);
 
 // General feature map (phi_mlp.cu): phi = [psi_1^1 .. psi_P^P],
 // psi = GELU(x W_a + b_a) W_b + b_b per head; x [BH][N][D] (in dtype),

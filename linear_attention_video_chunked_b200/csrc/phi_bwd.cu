@@ -455,11 +455,13 @@ cudaError_t launch_phi_bwd(const PhiBwdArgs& a, cudaStream_t s) {
     t.nchunks = bp.nchunks;
     t.x = a.q; t.dy = a.dy; t.y = a.y; t.den = a.den; t.w_img = a.wq_img; t.b = a.bq;
     t.M = a.SL; t.vec = a.zL; t.part = bp.qpart; t.splits = bp.QS; t.q_side = 1;
+    t.dx = a.dq; t.dv = nullptr;
     cudaError_t e = launch_phi_bwd_tc(t, s);
     if (e != cudaSuccess) return e;
     launch_ghat(bp, s);
     t.x = a.k; t.v = a.v; t.w_img = a.wk_img; t.b = a.bk; t.M = bp.ghat; t.vec = nullptr;
     t.part = bp.kpart; t.splits = bp.KS; t.q_side = 0;
+    t.dx = a.dk; t.dv = a.dv;
     e = launch_phi_bwd_tc(t, s);
     if (e != cudaSuccess) return e;
     const long long nr = (static_cast<long long>(a.D) * bp.Dp + bp.Dp) * bp.heads;

@@ -513,21 +513,23 @@ __global__ void __launch_bounds__(bk::kThreads, 1)
     constexpr float kLog2e = 1.4426950408889634f;
     const float sl2 = A.scale * kLog2e;
     const int key = j0 + kr;
-    float* vec = reinterpret_cast<float*>(sbase + kVecOff);  // [stage][m | r | Dc | j*][128]
-    // Per-query values of pair i into stage i & 1: thread t loads two of
-    // the 512 (query t & 127, arrays 2 (t >> 7) and 2 (t >> 7) + 1).
+    // Per-query values of pair i in stage i & 1, one 16-byte record per
+    // query (m = c log2(e), r, Dc, j*), so each column costs one broadcast
+    // 16-byte shared load.  Thread t fills two of the record's words
+    // (query t & 127, words 2 (t >> 7), 2 (t >> 7) + 1).
+    float4* vec = reinterpret_cast<float4*>(sbase + kVecOff);  // [stage][128]
     auto load_vec = [&](const QWalk& w, int i) {
       const int qi = tid & 127, which = tid >> 7;
       const int q = w.q0() + qi;
       const bool in = qi < w.qvalid();
-      float* v = vec + (i & 1) * 512;
+      float* v = reinterpret_cast<float*>(vec + (i & 1) * 128 + qi);
       const long long g = base_row + q;
       if (which == 0) {
-        v[qi] = in ? __ldg(A.c + g) * kLog2e : 0.f;
-        v[128 + qi] = in ? __ldg(A.r + g) : 0.f;
+        v[0] = in ? __ldg(A.c + g) * kLog2e : 0.f;
+        v[1] = in ? __ldg(A.r + g) : 0.f;
       } else {
-        v[256 + qi] = in ? __ldg(A.Dc + g) : 0.f;
-        v[384 + qi] = __int_as_float(in ? __ldg(A.jstar + g) : -1);
+        v[2] = in ? __ldg(A.Dc + g) : 0.f;
+        v[3] = __int_as_float(in ? __ldg(A.jstar + g) : -1);
       }
       mbar_arrive(bar(VEC_FULL + (i & 1)));
     };
@@ -541,7 +543,7 @@ __global__ void __launch_bounds__(bk::kThreads, 1)
       ok = wait_all(bar(ST_FULL), i & 1, 24) && wait_all(bar(VEC_FULL + (i & 1)), (i >> 1) & 1, 25);
       if (!ok) break;
       tc_fence_after();
-      const float* v = vec + (i & 1) * 512;
+      const float4* v = vec + (i & 1) * 128;
       uint32_t pp[32], pd[32];
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
@@ -553,15 +555,16 @@ __global__ void __launch_bounds__(bk::kThreads, 1)
         for (int i2 = 0; i2 < 32; i2 += 2) {
           const int qa = 64 * hf + 32 * c + i2;
           float p0 = 0.f, p1 = 0.f, d0 = 0.f, d1 = 0.f;
+          const float4 v0 = v[qa], v1 = v[qa + 1];
           if (key_in && qa < qv) {
-            p0 = ex2(fmaf(__uint_as_float(xs[i2]), sl2, -v[qa]));
-            d0 = p0 * (__uint_as_float(xd[i2]) - v[128 + qa]);
-            if (__float_as_int(v[384 + qa]) == key) d0 -= v[256 + qa];
+            p0 = ex2(fmaf(__uint_as_float(xs[i2]), sl2, -v0.x));
+            d0 = p0 * (__uint_as_float(xd[i2]) - v0.y);
+            if (__float_as_int(v0.w) == key) d0 -= v0.z;
           }
           if (key_in && qa + 1 < qv) {
-            p1 = ex2(fmaf(__uint_as_float(xs[i2 + 1]), sl2, -v[qa + 1]));
-            d1 = p1 * (__uint_as_float(xd[i2 + 1]) - v[128 + qa + 1]);
-            if (__float_as_int(v[384 + qa + 1]) == key) d1 -= v[256 + qa + 1];
+            p1 = ex2(fmaf(__uint_as_float(xs[i2 + 1]), sl2, -v1.x));
+            d1 = p1 * (__uint_as_float(xd[i2 + 1]) - v1.y);
+            if (__float_as_int(v1.w) == key) d1 -= v1.z;
           }
           pp[16 * c + i2 / 2] = pack_bf16(p0, p1);
           pd[16 * c + i2 / 2] = pack_bf16(d0, d1);

@@ -34,7 +34,7 @@ constexpr int kThreads = 192;
 constexpr uint32_t kWOff = 0, kMOff = 32768, kXOff = 65536, kEOff = 98304, kDUOff = 131072,
                    kPhiOff = 163840, kVecOff = 196608, kRedOff = 197632, kBarOff = 201728;
 enum { W_FULL = 0, M_READY = 1, X_FULL = 2, E_READY = 3, UT_FULL = 4, DU_READY = 5,
-       TILE_DONE = 6, NBAR = 7 };
+       TILE_DONE = 6, DX_FREE = 7, NBAR = 8 };
 constexpr uint32_t kSmemBytes = kBarOff + 128 + 1024;
 constexpr uint32_t kColU = 0, kColT = 128, kColW = 256, kColG = 384;
 
@@ -106,10 +106,12 @@ __global__ void __launch_bounds__(pb::kThreads, 1)
   // M (S_L of the chunk, or Ghat of the slice) and its vector (z_L or hhat).
   const float* Msrc = kQ ? a.M + set * Dp * D : a.M + set * (128LL * D + 128);
   const float* vsrc = kQ ? a.vec + set * Dp : Msrc + 128LL * D;
+  const bool with_dx = a.dx != nullptr;
 
   if (tid == 0) {
     for (int i = 0; i < pb::NBAR; ++i) {
-      const bool by_rows = i == pb::M_READY || i == pb::DU_READY || (kQ && i == pb::E_READY);
+      const bool by_rows = i == pb::M_READY || i == pb::DU_READY || (kQ && i == pb::E_READY) ||
+                           i == pb::DX_FREE;
       mbar_init(bar(i), by_rows ? 128 : 1);
     }
     *abort_flag = 0;
@@ -171,11 +173,15 @@ __global__ void __launch_bounds__(pb::kThreads, 1)
     if (lane == 0) {
       const uint32_t id_k = idesc(128, 128, 1, false);          // A, B K-major
       const uint32_t id_mn = idesc_ab(128, 128, 1, true, true);  // A, B MN-major
+      const uint32_t id_kmn = idesc(128, 128, 1, true);          // A K-major, B MN-major
       bool ok = mbar_wait(bar(pb::W_FULL), 0, abort_flag, 51) &&
                 mbar_wait(bar(pb::M_READY), 0, abort_flag, 52);
       for (int tl = 0; tl < ntiles && ok; ++tl) {
         ok = mbar_wait(bar(pb::X_FULL), tl & 1, abort_flag, 53);
         if (ok && kQ) ok = mbar_wait(bar(pb::E_READY), tl & 1, abort_flag, 54);
+        // U's columns hold the previous tile's token gradient until the row
+        // warps have read it.
+        if (ok && with_dx && tl > 0) ok = mbar_wait(bar(pb::DX_FREE), (tl - 1) & 1, abort_flag, 59);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
@@ -209,6 +215,26 @@ __global__ void __launch_bounds__(pb::kThreads, 1)
                      sdesc(base + kEOff + off, 16384, 1024), id_mn, (tl > 0 || kk > 0) ? 1u : 0u);
           }
         }
+        if (with_dx) {
+          // Token gradient through phi: dx = du W (A = du K-major, B = the W
+          // image [f][d] read MN-major), into U's columns.
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            mma_bf16(tmem + pb::kColU, sdesc(base + kDUOff + off, 16, 1024),
+                     sdesc(base + kWOff + kk * 2048, 16384, 1024), id_kmn, kk > 0);
+          }
+          if (!kQ && a.dv != nullptr) {
+            // dv += phi_k Ghat_s (B = the Ghat tile [f][d] read MN-major),
+            // into G's columns (unused by the k pass).
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+              mma_bf16(tmem + pb::kColG, sdesc(base + kPhiOff + off, 16, 1024),
+                       sdesc(base + kMOff + kk * 2048, 16384, 1024), id_kmn, kk > 0);
+            }
+          }
+        }
         mma_commit(bar(pb::TILE_DONE));
       }
     }
@@ -238,13 +264,59 @@ __global__ void __launch_bounds__(pb::kThreads, 1)
     mbar_arrive(bar(pb::M_READY));
     __syncwarp();
     float acc_db[4] = {0.f, 0.f, 0.f, 0.f}, acc_h[4] = {0.f, 0.f, 0.f, 0.f};
+    // Adds tile tl's token gradients (in U's and G's columns once TILE_DONE)
+    // to dx and dv, then frees the columns for the next tile's U.
+    auto flush_dx = [&](int tl) {
+      const long long row = r0 + 128LL * tl + r;
+      const long long gi = (static_cast<long long>(bh) * N + row) * D;
+      const bool with_dv = !kQ && a.dv != nullptr;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t rx[32], rv[32];
+        REHYAT_TMEM_LD32(lane_base + pb::kColU + c * 32, rx);
+        if (with_dv) REHYAT_TMEM_LD32(lane_base + pb::kColG + c * 32, rv);
+        tmem_wait_ld();
+        if (row < r1) {
+          float4* dx4 = reinterpret_cast<float4*>(a.dx + gi + c * 32);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            float4 o = dx4[i];
+            o.x += __uint_as_float(rx[4 * i]);
+            o.y += __uint_as_float(rx[4 * i + 1]);
+            o.z += __uint_as_float(rx[4 * i + 2]);
+            o.w += __uint_as_float(rx[4 * i + 3]);
+            dx4[i] = o;
+          }
+          if (with_dv) {
+            float4* dv4 = reinterpret_cast<float4*>(a.dv + gi + c * 32);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              float4 o = dv4[i];
+              o.x += __uint_as_float(rv[4 * i]);
+              o.y += __uint_as_float(rv[4 * i + 1]);
+              o.z += __uint_as_float(rv[4 * i + 2]);
+              o.w += __uint_as_float(rv[4 * i + 3]);
+              dv4[i] = o;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(pb::DX_FREE));
+    };
     for (int tl = 0; tl < ntiles && ok; ++tl) {
       const long long row = r0 + 128LL * tl + r;
       const bool valid = row < r1;
       float rdot = 0.f;  // (g . y) / den of this row (q pass)
+      if (with_dx && tl > 0) {
+        ok = wait_all(bar(pb::TILE_DONE), (tl - 1) & 1, 56);
+        if (!ok) break;
+        tc_fence_after();
+        flush_dx(tl - 1);
+      }
       if (kQ) {
         // E = g / den for the tile, once the previous tile's MMAs are done.
-        if (tl > 0) ok = wait_all(bar(pb::TILE_DONE), (tl - 1) & 1, 56);
+        if (tl > 0 && !with_dx) ok = wait_all(bar(pb::TILE_DONE), (tl - 1) & 1, 56);
         if (!ok) break;
         const long long gi = (static_cast<long long>(bh) * N + row) * D;
         const float inv = valid ? 1.f / __ldg(a.den + static_cast<long long>(bh) * N + row) : 0.f;
@@ -293,7 +365,7 @@ __global__ void __launch_bounds__(pb::kThreads, 1)
                        pack_bf16(du[8 * j], du[8 * j + 1]), pack_bf16(du[8 * j + 2], du[8 * j + 3]),
                        pack_bf16(du[8 * j + 4], du[8 * j + 5]),
                        pack_bf16(du[8 * j + 6], du[8 * j + 7]));
-          if (kQ)
+          if (kQ || (with_dx && a.dv != nullptr))
             st_shared_v4(base + kPhiOff + tile_off(r, c * 32 + 8 * j),
                          pack_bf16(ph[8 * j], ph[8 * j + 1]), pack_bf16(ph[8 * j + 2], ph[8 * j + 3]),
                          pack_bf16(ph[8 * j + 4], ph[8 * j + 5]),
@@ -314,6 +386,7 @@ __global__ void __launch_bounds__(pb::kThreads, 1)
     if (ok && ntiles > 0) ok = wait_all(bar(pb::TILE_DONE), (ntiles - 1) & 1, 58);
     if (ok && ntiles > 0) {
       tc_fence_after();
+      if (with_dx) flush_dx(ntiles - 1);
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         uint32_t rw[32];
