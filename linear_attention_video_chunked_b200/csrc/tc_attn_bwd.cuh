@@ -215,35 +215,47 @@ __global__ void __launch_bounds__(bq::kThreads, 1)
     for (int j = 0; j < nt && ok; ++j) {
       const int nvalid = min(128, na - j * 128);
       const uint32_t sb = lane_base + ((j & 1) ? kColS1 : kColS0);
-      ok = wait_all(bar(S_FULL + (j & 1)), (j >> 1) & 1, 25) && wait_all(bar(DP_FULL), j & 1, 26);
+      // Phase 1 (needs S only, so it overlaps dP's MMAs): P of this half's
+      // 64 key columns in fp32, and the arg-max.
+      ok = wait_all(bar(S_FULL + (j & 1)), (j >> 1) & 1, 25);
+      if (!ok) break;
+      tc_fence_after();
+      float pv[64];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t xs[32];
+        REHYAT_TMEM_LD32(sb + 64 * hf + 32 * c, xs);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int key = 64 * hf + 32 * c + i;
+          const float sv = __uint_as_float(xs[i]);
+          float p = 0.f;
+          if (key < nvalid) {
+            p = ex2(fmaf(sv, sl2, -m));
+            if (sv > best) {
+              best = sv;
+              barg = j * 128 + key;
+            }
+          }
+          pv[32 * c + i] = p;
+        }
+      }
+      // Phase 2: dS = P (dP - r) once dP is done; dS (bf16 pairs) goes over
+      // this half's own S columns.
+      ok = wait_all(bar(DP_FULL), j & 1, 26);
       if (!ok) break;
       tc_fence_after();
       uint32_t pk[32];
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        uint32_t xs[32], xd[32];
-        REHYAT_TMEM_LD32(sb + 64 * hf + 32 * c, xs);
+        uint32_t xd[32];
         REHYAT_TMEM_LD32(lane_base + kColDP + 64 * hf + 32 * c, xd);
         tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          const int key = 64 * hf + 32 * c + i;
-          float d0 = 0.f, d1 = 0.f;
-          const float s0 = __uint_as_float(xs[i]), s1 = __uint_as_float(xs[i + 1]);
-          if (key < nvalid) {
-            d0 = ex2(fmaf(s0, sl2, -m)) * (__uint_as_float(xd[i]) - rr);
-            if (s0 > best) {
-              best = s0;
-              barg = j * 128 + key;
-            }
-          }
-          if (key + 1 < nvalid) {
-            d1 = ex2(fmaf(s1, sl2, -m)) * (__uint_as_float(xd[i + 1]) - rr);
-            if (s1 > best) {
-              best = s1;
-              barg = j * 128 + key + 1;
-            }
-          }
+          const float d0 = pv[32 * c + i] * (__uint_as_float(xd[i]) - rr);
+          const float d1 = pv[32 * c + i + 1] * (__uint_as_float(xd[i + 1]) - rr);
           Dc += d0 + d1;
           pk[16 * c + i / 2] = pack_bf16(d0, d1);
         }
@@ -337,7 +349,7 @@ constexpr uint32_t kGOff = kQOff + 2 * 32768;                // GH ring (2 x 32 
 constexpr uint32_t kVecOff = kGOff + 2 * 32768;              // per-query m, r, Dc, j* (2 x 2 KB)
 constexpr uint32_t kBarOff = kVecOff + 2 * 2048;
 enum { KV_FULL = 0, QG_FULL = 1, QG_EMPTY = 3, VEC_FULL = 5, ST_FULL = 7, DS_FULL = 8,
-       KV_DONE = 9, NBAR = 10 };
+       KV_DONE = 9, DPT_FULL = 10, PT_FULL = 11, NBAR = 12 };
 constexpr uint32_t kTmemSlot = kBarOff + 8 * NBAR;
 constexpr uint32_t kAbortSlot = kTmemSlot + 4;
 constexpr uint32_t kSmemBytes = kBarOff + 256 + 1024;
@@ -393,6 +405,8 @@ __global__ void __launch_bounds__(bk::kThreads, 1)
   using bk::ST_FULL;
   using bk::DS_FULL;
   using bk::KV_DONE;
+  using bk::DPT_FULL;
+  using bk::PT_FULL;
   using bk::NBAR;
   using bk::QWalk;
   extern __shared__ uint8_t smem_raw[];
@@ -419,7 +433,8 @@ __global__ void __launch_bounds__(bk::kThreads, 1)
 
   if (tid == 0) {
     for (int i = 0; i < NBAR; ++i)
-      mbar_init(bar(i), (i == DS_FULL || i == VEC_FULL || i == VEC_FULL + 1) ? 256 : 1);
+      mbar_init(bar(i), (i == DS_FULL || i == PT_FULL || i == VEC_FULL || i == VEC_FULL + 1)
+                            ? 256 : 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -463,41 +478,57 @@ __global__ void __launch_bounds__(bk::kThreads, 1)
       const uint32_t id_kk = idesc(128, 128, 1, false);  // A, B K-major
       const uint32_t id_mn = idesc(128, 128, 1, true);   // B MN-major
       bool ok = mbar_wait(bar(KV_FULL), 0, abort_flag, 21);
-      for (int i = 0; i < niter && ok; ++i) {
-        const int st = i & 1;
-        const uint32_t qa = base + kQOff + st * 32768, ga = base + kGOff + st * 32768;
-        ok = mbar_wait(bar(QG_FULL + st), (i >> 1) & 1, abort_flag, 22);
-        if (!ok) break;
+      auto qa_of = [&](int i) { return base + kQOff + (i & 1) * 32768; };
+      auto ga_of = [&](int i) { return base + kGOff + (i & 1) * 32768; };
+      // S^T(i) = K Q(i)^T and dP^T(i) = V GH(i)^T, committed separately so
+      // the exponentials can start before dP^T is done.
+      auto issue_st = [&](int i) -> bool {
+        if (!mbar_wait(bar(QG_FULL + (i & 1)), (i >> 1) & 1, abort_flag, 22)) return false;
         tc_fence_after();
-        // S^T = K Q^T and dP^T = V GH^T (the previous pair's dV and dK,
-        // issued before, have read S^T and dP^T: in order).
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_bf16(tmem + kColS, sdesc(base + kKOff + off, 16, 1024), sdesc(qa + off, 16, 1024),
-                   id_kk, kk > 0);
-        }
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_bf16(tmem + kColDP, sdesc(base + kVOff + off, 16, 1024), sdesc(ga + off, 16, 1024),
+          mma_bf16(tmem + kColS, sdesc(base + kKOff + off, 16, 1024), sdesc(qa_of(i) + off, 16, 1024),
                    id_kk, kk > 0);
         }
         mma_commit(bar(ST_FULL));
-        ok = mbar_wait(bar(DS_FULL), i & 1, abort_flag, 23);
+        return true;
+      };
+      auto issue_dpt = [&](int i) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_bf16(tmem + kColDP, sdesc(base + kVOff + off, 16, 1024), sdesc(ga_of(i) + off, 16, 1024),
+                   id_kk, kk > 0);
+        }
+        mma_commit(bar(DPT_FULL));
+      };
+      if (ok && niter > 0) {
+        ok = issue_st(0);
+        if (ok) issue_dpt(0);
+      }
+      for (int i = 0; i < niter && ok; ++i) {
+        // P^T(i) is in S^T's columns: dV += P^T GH (query columns [0, 64)
+        // of the A operand in TMEM columns [0, 32), [64, 128) in [64, 96)),
+        // then S^T(i + 1) over them (in order).
+        ok = mbar_wait(bar(PT_FULL), i & 1, abort_flag, 23);
         if (!ok) break;
         tc_fence_after();
-        // dV += P^T GH and dK += dS^T Q, A from TMEM (query columns [0, 64)
-        // in columns [0, 32) of the buffer, [64, 128) in [64, 96)).
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_bf16_ts(tmem + kColDV, tmem + kColS + (kk >> 2) * 64 + (kk & 3) * 8,
-                      sdesc(ga + kk * 2048, 16384, 1024), id_mn, (i > 0 || kk > 0) ? 1u : 0u);
+                      sdesc(ga_of(i) + kk * 2048, 16384, 1024), id_mn, (i > 0 || kk > 0) ? 1u : 0u);
+        if (i + 1 < niter && !(ok = issue_st(i + 1))) break;
+        // dS^T(i) is in dP^T's columns: dK += dS^T Q, then dP^T(i + 1).
+        ok = mbar_wait(bar(DS_FULL), i & 1, abort_flag, 29);
+        if (!ok) break;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_bf16_ts(tmem + kColDK, tmem + kColDP + (kk >> 2) * 64 + (kk & 3) * 8,
-                      sdesc(qa + kk * 2048, 16384, 1024), id_mn, (i > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(bar(QG_EMPTY + st));
+                      sdesc(qa_of(i) + kk * 2048, 16384, 1024), id_mn, (i > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(bar(QG_EMPTY + (i & 1)));
+        if (i + 1 < niter) issue_dpt(i + 1);
       }
       if (ok) mma_commit(bar(KV_DONE));
     }
@@ -544,38 +575,35 @@ __global__ void __launch_bounds__(bk::kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const float4* v = vec + (i & 1) * 128;
-      uint32_t pp[32], pd[32];
+      // Phase 1: P^T = exp2(s scale log2(e) - m) of this half's 64 query
+      // columns, written over them as bf16 pairs; kept in fp32 for phase 2.
+      float pv[64];
+      {
+        uint32_t pp[32];
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t xs[32], xd[32];
-        REHYAT_TMEM_LD32(lane_base + kColS + 64 * hf + 32 * c, xs);
-        REHYAT_TMEM_LD32(lane_base + kColDP + 64 * hf + 32 * c, xd);
-        tmem_wait_ld();
+        for (int c = 0; c < 2; ++c) {
+          uint32_t xs[32];
+          REHYAT_TMEM_LD32(lane_base + kColS + 64 * hf + 32 * c, xs);
+          tmem_wait_ld();
 #pragma unroll
-        for (int i2 = 0; i2 < 32; i2 += 2) {
-          const int qa = 64 * hf + 32 * c + i2;
-          float p0 = 0.f, p1 = 0.f, d0 = 0.f, d1 = 0.f;
-          const float4 v0 = v[qa], v1 = v[qa + 1];
-          if (key_in && qa < qv) {
-            p0 = ex2(fmaf(__uint_as_float(xs[i2]), sl2, -v0.x));
-            d0 = p0 * (__uint_as_float(xd[i2]) - v0.y);
-            if (__float_as_int(v0.w) == key) d0 -= v0.z;
+          for (int i2 = 0; i2 < 32; ++i2) {
+            const int qa = 64 * hf + 32 * c + i2;
+            float p = 0.f;
+            if (key_in && qa < qv) p = ex2(fmaf(__uint_as_float(xs[i2]), sl2, -v[qa].x));
+            pv[32 * c + i2] = p;
           }
-          if (key_in && qa + 1 < qv) {
-            p1 = ex2(fmaf(__uint_as_float(xs[i2 + 1]), sl2, -v1.x));
-            d1 = p1 * (__uint_as_float(xd[i2 + 1]) - v1.y);
-            if (__float_as_int(v1.w) == key) d1 -= v1.z;
-          }
-          pp[16 * c + i2 / 2] = pack_bf16(p0, p1);
-          pd[16 * c + i2 / 2] = pack_bf16(d0, d1);
+#pragma unroll
+          for (int i2 = 0; i2 < 16; ++i2) pp[16 * c + i2] = pack_bf16(pv[32 * c + 2 * i2], pv[32 * c + 2 * i2 + 1]);
         }
+        REHYAT_TMEM_ST32(lane_base + kColS + 64 * hf, pp);
       }
-      REHYAT_TMEM_ST32(lane_base + kColS + 64 * hf, pp);
-      REHYAT_TMEM_ST32(lane_base + kColDP + 64 * hf, pd);
       tmem_wait_st();
+      // Q and GH rows past the chunk are zeroed before dV and dK read them
+      // (their P and dS are 0; this keeps 0 * garbage out), once dP^T,
+      // which reads GH, is done.
+      if (qv < 128) ok = wait_all(bar(DPT_FULL), i & 1, 30);
+      if (!ok) break;
       if (qv < 128 && kr >= qv) {
-        // Q and GH rows past the chunk are zeroed before dK and dV read them
-        // (their P and dS are 0; this keeps 0 * garbage out).
         const uint32_t qrow = base + kQOff + (i & 1) * 32768 + hf * 16384 + kr * 128;
         const uint32_t grow2 = base + kGOff + (i & 1) * 32768 + hf * 16384 + kr * 128;
 #pragma unroll
@@ -585,6 +613,33 @@ __global__ void __launch_bounds__(bk::kThreads, 1)
         }
       }
       if (qv < 128) fence_proxy_async();
+      tc_fence_before();
+      mbar_arrive(bar(PT_FULL));
+      // Phase 2: dS^T = P^T (dP^T - r) - [j = j*] Dc over dP^T's columns.
+      ok = wait_all(bar(DPT_FULL), i & 1, 30);
+      if (!ok) break;
+      tc_fence_after();
+      {
+        uint32_t pd[32];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t xd[32];
+          REHYAT_TMEM_LD32(lane_base + kColDP + 64 * hf + 32 * c, xd);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i2 = 0; i2 < 32; i2 += 2) {
+            const int qa = 64 * hf + 32 * c + i2;
+            const float4 v0 = v[qa], v1 = v[qa + 1];
+            float d0 = pv[32 * c + i2] * (__uint_as_float(xd[i2]) - v0.y);
+            float d1 = pv[32 * c + i2 + 1] * (__uint_as_float(xd[i2 + 1]) - v1.y);
+            if (__float_as_int(v0.w) == key && key_in && qa < qv) d0 -= v0.z;
+            if (__float_as_int(v1.w) == key && key_in && qa + 1 < qv) d1 -= v1.z;
+            pd[16 * c + i2 / 2] = pack_bf16(d0, d1);
+          }
+        }
+        REHYAT_TMEM_ST32(lane_base + kColDP + 64 * hf, pd);
+      }
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(DS_FULL));
       // The next pair's per-query values (stage (i + 1) & 1: every thread is
