@@ -396,44 +396,51 @@ __global__ void scan_kernel(const float* __restrict__ P, const float* __restrict
   }
 }
 
-// Chunk scan for T <= kScanRegs slices: each thread reads its element of
-// every per-slice state once into registers, then writes each chunk's
+// Chunk scan for T <= kScanRegs slices: each thread reads its four elements
+// of every per-slice state once into registers, then writes each chunk's
 // linear-set sum as a plain sum, in slice order, over the slices of that
 // chunk's linear set (slices < w_t, and in the bidirectional form also
 // slices >= end_t): no total-minus-window subtraction, and P is read once
-// instead of once per direction.
+// instead of once per direction.  Four elements per thread share the
+// per-slice set tests.
 constexpr int kScanRegs = 32;
-__global__ void scan_regs_kernel(const float* __restrict__ P, const float* __restrict__ z,
-                                 float* __restrict__ SL, float* __restrict__ zL, int T, int Tc,
+__global__ void scan_regs_kernel(const float4* __restrict__ P, const float4* __restrict__ z,
+                                 float4* __restrict__ SL, float4* __restrict__ zL, int T, int Tc,
                                  int To, int nchunks, int Dp, int D, int causal) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const long long PD = static_cast<long long>(Dp) * D;
+  const long long PD4 = static_cast<long long>(Dp) * D / 4;
   const long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int bh = blockIdx.y;
-  const float* src;
-  float* dst;
+  const float4* src;
+  float4* dst;
   long long stride;
-  if (e < PD) {
-    src = P + bh * T * PD + e;
-    dst = SL + bh * nchunks * PD + e;
-    stride = PD;
-  } else if (e < PD + Dp) {
-    src = z + static_cast<long long>(bh) * T * Dp + (e - PD);
-    dst = zL + static_cast<long long>(bh) * nchunks * Dp + (e - PD);
-    stride = Dp;
+  if (e < PD4) {
+    src = P + bh * T * PD4 + e;
+    dst = SL + bh * nchunks * PD4 + e;
+    stride = PD4;
+  } else if (e < PD4 + Dp / 4) {
+    src = z + static_cast<long long>(bh) * T * (Dp / 4) + (e - PD4);
+    dst = zL + static_cast<long long>(bh) * nchunks * (Dp / 4) + (e - PD4);
+    stride = Dp / 4;
   } else {
     return;
   }
-  float v[kScanRegs];
+  float4 v[kScanRegs];
 #pragma unroll
-  for (int i = 0; i < kScanRegs; ++i) v[i] = i < T ? src[static_cast<long long>(i) * stride] : 0.f;
+  for (int i = 0; i < kScanRegs; ++i)
+    v[i] = i < T ? src[static_cast<long long>(i) * stride] : make_float4(0.f, 0.f, 0.f, 0.f);
   for (int t = 0; t < nchunks; ++t) {
     const int first = t * Tc, end = min(T, first + Tc), w = max(first - To, 0);
     const int lim = causal ? T : end;  // slices >= lim join the linear set
-    float acc = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int i = 0; i < kScanRegs; ++i)
-      if (i < w || (i >= lim && i < T)) acc += v[i];
+      if (i < w || (i >= lim && i < T)) {
+        acc.x += v[i].x;
+        acc.y += v[i].y;
+        acc.z += v[i].z;
+        acc.w += v[i].w;
+      }
     dst[static_cast<long long>(t) * stride] = acc;
   }
 }
@@ -616,9 +623,14 @@ cudaError_t launch_scan(const float* P, const float* z, float* SL, float* zL, in
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (T <= kScanRegs)
-    return cudaLaunchKernelEx(&cfg, scan_regs_kernel, P, z, SL, zL, T, Tc, To, nchunks, Dp, D,
-                              causal);
+  if (T <= kScanRegs && Dp % 4 == 0) {
+    const long long n4 = static_cast<long long>(Dp) * D / 4 + Dp / 4;
+    cfg.gridDim = dim3(static_cast<unsigned>((n4 + 127) / 128), BH);
+    cfg.blockDim = dim3(128);
+    return cudaLaunchKernelEx(&cfg, scan_regs_kernel, reinterpret_cast<const float4*>(P),
+                              reinterpret_cast<const float4*>(z), reinterpret_cast<float4*>(SL),
+                              reinterpret_cast<float4*>(zL), T, Tc, To, nchunks, Dp, D, causal);
+  }
   return cudaLaunchKernelEx(&cfg, scan_kernel, P, z, SL, zL, T, Tc, To, nchunks, Dp, D, causal);
 }
 

@@ -148,12 +148,7 @@ __global__ void __launch_bounds__(bq::kThreads, 1)
         if (!mbar_wait(bar(K_FULL + j % 3), (j / 3) & 1, abort_flag, 22)) return false;
         tc_fence_after();
         const uint32_t kaddr = base + kKOff + (j % 3) * 32768;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_bf16(s_buf(j), sdesc(base + kQOff + off, 16, 1024), sdesc(kaddr + off, 16, 1024),
-                   id_kk, kk > 0);
-        }
+        mma8_ss_kmajor(s_buf(j), sdesc(base + kQOff, 16, 1024), sdesc(kaddr, 16, 1024), id_kk, 0u);
         mma_commit(bar(S_FULL + (j & 1)));
         return true;
       };
@@ -162,12 +157,8 @@ __global__ void __launch_bounds__(bq::kThreads, 1)
         if (!mbar_wait(bar(V_FULL + (j & 1)), (j >> 1) & 1, abort_flag, 23)) return false;
         tc_fence_after();
         const uint32_t vaddr = base + kVOff + (j & 1) * 32768;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_bf16(tmem + kColDP, sdesc(base + kGOff + off, 16, 1024), sdesc(vaddr + off, 16, 1024),
-                   id_kk, kk > 0);
-        }
+        mma8_ss_kmajor(tmem + kColDP, sdesc(base + kGOff, 16, 1024), sdesc(vaddr, 16, 1024), id_kk,
+                       0u);
         mma_commit(bar(DP_FULL));
         mma_commit(bar(V_EMPTY + (j & 1)));
         return true;
@@ -184,10 +175,8 @@ __global__ void __launch_bounds__(bq::kThreads, 1)
         // dQ += dS(j) K(j): dS of key columns [0, 64) sits in columns [0, 32)
         // of the buffer, of [64, 128) in columns [64, 96) (one run per half).
         const uint32_t kaddr = base + kKOff + (j % 3) * 32768;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts(tmem + kColDQ, s_buf(j) + (kk >> 2) * 64 + (kk & 3) * 8,
-                      sdesc(kaddr + kk * 2048, 16384, 1024), id_dq, (j > 0 || kk > 0) ? 1u : 0u);
+        mma8_ts_mn_split(tmem + kColDQ, s_buf(j), sdesc(kaddr, 16384, 1024), id_dq,
+                         j > 0 ? 1u : 0u);
         mma_commit(bar(K_EMPTY + j % 3));
         // S(j + 2) overwrites this buffer after dQ(j) has read it (in order).
         if (j + 2 < nt && !(ok = issue_s(j + 2))) break;
@@ -485,22 +474,14 @@ __global__ void __launch_bounds__(bk::kThreads, 1)
       auto issue_st = [&](int i) -> bool {
         if (!mbar_wait(bar(QG_FULL + (i & 1)), (i >> 1) & 1, abort_flag, 22)) return false;
         tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_bf16(tmem + kColS, sdesc(base + kKOff + off, 16, 1024), sdesc(qa_of(i) + off, 16, 1024),
-                   id_kk, kk > 0);
-        }
+        mma8_ss_kmajor(tmem + kColS, sdesc(base + kKOff, 16, 1024), sdesc(qa_of(i), 16, 1024),
+                       id_kk, 0u);
         mma_commit(bar(ST_FULL));
         return true;
       };
       auto issue_dpt = [&](int i) {
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_bf16(tmem + kColDP, sdesc(base + kVOff + off, 16, 1024), sdesc(ga_of(i) + off, 16, 1024),
-                   id_kk, kk > 0);
-        }
+        mma8_ss_kmajor(tmem + kColDP, sdesc(base + kVOff, 16, 1024), sdesc(ga_of(i), 16, 1024),
+                       id_kk, 0u);
         mma_commit(bar(DPT_FULL));
       };
       if (ok && niter > 0) {
@@ -514,19 +495,15 @@ __global__ void __launch_bounds__(bk::kThreads, 1)
         ok = mbar_wait(bar(PT_FULL), i & 1, abort_flag, 23);
         if (!ok) break;
         tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts(tmem + kColDV, tmem + kColS + (kk >> 2) * 64 + (kk & 3) * 8,
-                      sdesc(ga_of(i) + kk * 2048, 16384, 1024), id_mn, (i > 0 || kk > 0) ? 1u : 0u);
+        mma8_ts_mn_split(tmem + kColDV, tmem + kColS, sdesc(ga_of(i), 16384, 1024), id_mn,
+                         i > 0 ? 1u : 0u);
         if (i + 1 < niter && !(ok = issue_st(i + 1))) break;
         // dS^T(i) is in dP^T's columns: dK += dS^T Q, then dP^T(i + 1).
         ok = mbar_wait(bar(DS_FULL), i & 1, abort_flag, 29);
         if (!ok) break;
         tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts(tmem + kColDK, tmem + kColDP + (kk >> 2) * 64 + (kk & 3) * 8,
-                      sdesc(qa_of(i) + kk * 2048, 16384, 1024), id_mn, (i > 0 || kk > 0) ? 1u : 0u);
+        mma8_ts_mn_split(tmem + kColDK, tmem + kColDP, sdesc(qa_of(i), 16384, 1024), id_mn,
+                         i > 0 ? 1u : 0u);
         mma_commit(bar(QG_EMPTY + (i & 1)));
         if (i + 1 < niter) issue_dpt(i + 1);
       }

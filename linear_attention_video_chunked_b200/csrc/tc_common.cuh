@@ -234,6 +234,89 @@ __device__ __forceinline__ uint32_t tmem_ld1(uint32_t taddr) {
   return v;
 }
 
+// Eight bf16 MMAs (K = 8 x 16) of one 128 x 128 x 128 product in one asm
+// block: A and B both K-major in shared memory, 128-byte swizzle, as two
+// 64-column boxes 16 KB apart, so step kk's descriptors are the bases plus
+// ((kk / 4) * 16384 + (kk % 4) * 32) / 16.  acc0 = 0 starts a fresh
+// accumulation with the first step.  (Saves the per-step descriptor
+// arithmetic of the issuing thread.)
+__device__ __forceinline__ void mma8_ss_kmajor(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                               uint32_t id, uint32_t acc0) {
+  asm volatile(
+      "{\n\t.reg .pred p0, p1;\n\t.reg .b64 a1, b1;\n\t"
+      "setp.ne.b32 p0, %4, 0;\n\t"
+      "setp.eq.b32 p1, %4, %4;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p0;\n\t"
+      "add.s64 a1, %1, 2;\n\tadd.s64 b1, %2, 2;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, p1;\n\t"
+      "add.s64 a1, %1, 4;\n\tadd.s64 b1, %2, 4;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, p1;\n\t"
+      "add.s64 a1, %1, 6;\n\tadd.s64 b1, %2, 6;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, p1;\n\t"
+      "add.s64 a1, %1, 1024;\n\tadd.s64 b1, %2, 1024;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, p1;\n\t"
+      "add.s64 a1, %1, 1026;\n\tadd.s64 b1, %2, 1026;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, p1;\n\t"
+      "add.s64 a1, %1, 1028;\n\tadd.s64 b1, %2, 1028;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, p1;\n\t"
+      "add.s64 a1, %1, 1030;\n\tadd.s64 b1, %2, 1030;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, p1;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(id), "r"(acc0));
+}
+
+// Eight bf16 MMAs with A from TMEM (8 columns of bf16 pairs per step) and B
+// MN-major in shared memory (16 rows = 2048 bytes per step).
+__device__ __forceinline__ void mma8_ts_mn(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                           uint32_t id, uint32_t acc0) {
+  asm volatile(
+      "{\n\t.reg .pred p0, p1;\n\t.reg .b64 b1;\n\t.reg .b32 a1;\n\t"
+      "setp.ne.b32 p0, %4, 0;\n\t"
+      "setp.eq.b32 p1, %4, %4;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p0;\n\t"
+      "add.s32 a1, %1, 8;\n\tadd.s64 b1, %2, 128;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, p1;\n\t"
+      "add.s32 a1, %1, 16;\n\tadd.s64 b1, %2, 256;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, p1;\n\t"
+      "add.s32 a1, %1, 24;\n\tadd.s64 b1, %2, 384;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, p1;\n\t"
+      "add.s32 a1, %1, 32;\n\tadd.s64 b1, %2, 512;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, p1;\n\t"
+      "add.s32 a1, %1, 40;\n\tadd.s64 b1, %2, 640;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, p1;\n\t"
+      "add.s32 a1, %1, 48;\n\tadd.s64 b1, %2, 768;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, p1;\n\t"
+      "add.s32 a1, %1, 56;\n\tadd.s64 b1, %2, 896;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, p1;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(id), "r"(acc0));
+}
+
+// As mma8_ts_mn, with the A operand's K range in two runs of 32 TMEM columns
+// 64 apart (steps 0-3 at a + 8 kk, steps 4-7 at a + 64 + 8 (kk - 4)): the
+// layout the backward kernels leave their bf16 pairs in (one run per half).
+__device__ __forceinline__ void mma8_ts_mn_split(uint32_t d_tmem, uint32_t a_tmem,
+                                                 uint64_t bdesc, uint32_t id, uint32_t acc0) {
+  asm volatile(
+      "{\n\t.reg .pred p0, p1;\n\t.reg .b64 b1;\n\t.reg .b32 a1;\n\t"
+      "setp.ne.b32 p0, %4, 0;\n\t"
+      "setp.eq.b32 p1, %4, %4;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p0;\n\t"
+      "add.s32 a1, %1, 8;\n\tadd.s64 b1, %2, 128;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, p1;\n\t"
+      "add.s32 a1, %1, 16;\n\tadd.s64 b1, %2, 256;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, p1;\n\t"
+      "add.s32 a1, %1, 24;\n\tadd.s64 b1, %2, 384;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, p1;\n\t"
+      "add.s32 a1, %1, 64;\n\tadd.s64 b1, %2, 512;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, p1;\n\t"
+      "add.s32 a1, %1, 72;\n\tadd.s64 b1, %2, 640;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, p1;\n\t"
+      "add.s32 a1, %1, 80;\n\tadd.s64 b1, %2, 768;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, p1;\n\t"
+      "add.s32 a1, %1, 88;\n\tadd.s64 b1, %2, 896;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, p1;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(id), "r"(acc0));
+}
+
 // D += A.B with A read from TMEM (K-major, two bf16 per 32-bit column).
 __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
                                             uint32_t id, uint32_t accumulate) {

@@ -739,21 +739,15 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
         } else {
           const uint32_t kaddr = base + kKOff + (j % 3) * 32768;
           const uint32_t qaddr = base + kQOff + tile * 32768;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            mma_bf16(tmem + tile * 256, sdesc(qaddr + off, 16, 1024),
-                     sdesc(kaddr + off, 16, 1024), id_qk, kk > 0);
-          }
+          mma8_ss_kmajor(tmem + tile * 256, sdesc(qaddr, 16, 1024), sdesc(kaddr, 16, 1024), id_qk,
+                         0u);
         }
         mma_commit(bar(a2::S_FULL + tile));
       };
       auto issue_pv = [&](int tile, int j) {
         const uint32_t vaddr = base + kVOff + (j & 1) * 32768;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts(tmem + tile * 256 + 128, tmem + tile * 256 + kk * 8,
-                      sdesc(vaddr + kk * 2048, 16384, 1024), id_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        mma8_ts_mn(tmem + tile * 256 + 128, tmem + tile * 256, sdesc(vaddr, 16384, 1024), id_pv,
+                   j > 0 ? 1u : 0u);
         mma_commit(bar(a2::PV_DONE + tile));
       };
       if (ok) ok = mbar_wait(bar(a2::K_FULL), 0, abort_flag, 5);
