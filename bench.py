@@ -654,58 +654,78 @@ def run_sweep(args):
     flush = L2Flush(torch, dev)
     peaks = load_peaks()
     stream = torch.cuda.current_stream()
+    csrc = sorted(os.path.join("linear_attention_video_chunked_b200", "csrc", f)
+                  for f in os.listdir(os.path.join(ROOT, "linear_attention_video_chunked_b200",
+                                                   "csrc"))
+                  if f.endswith((".cu", ".cuh", ".h")))
+    print(json.dumps({"sweep": "21x30x52", "header": True,
+                      "source_sha": kernel_source_sha(csrc + ["include/rehyat.h"]),
+                      "peak_bf16_tflops": peaks["bf16_tflops"], "peak_source": peaks["source"],
+                      "peak_hbm_gbs": peaks["hbm_gbs"]}), flush=True)
+    points = [(Dp, causal, Tc, To, 0) for Dp in (64, 128, 256) for causal in (0, 1)
+              for Tc in (1, 2, 3, 5, 7) for To in (0, 1, 2)]
+    # The fp8 q.k^T variant at D' = 128, both forms.
+    points += [(128, causal, Tc, To, rh.FLAG_FP8_QK) for causal in (0, 1)
+               for Tc in (1, 2, 3, 5, 7) for To in (0, 1, 2)]
+    phis = {}
     for Dp in (64, 128, 256):
         Wq, Wk = (0.1 * torch.randn(H, 2, D, Dp // 2, generator=g, device=dev) for _ in range(2))
         bq, bk = (0.1 * torch.randn(H, 2, Dp // 2, generator=g, device=dev) for _ in range(2))
-        phi = rh.RehyatPhi(Wq.data_ptr(), bq.data_ptr(), Wk.data_ptr(), bk.data_ptr())
-        for causal in (0, 1):
-            for Tc in (1, 2, 3, 5, 7):
-                for To in (0, 1, 2):
-                    p = rh.make_params(batch=B, heads=H, T=T, Hs=Hs, Ws=Ws, D=D, Dp=Dp, Tc=Tc,
-                                       To=To, causal=causal, in_dtype=rh.BF16, out_dtype=rh.F32)
-                    nbytes = rh.rehyat_workspace_bytes(p)
-                    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        phis[Dp] = (rh.RehyatPhi(Wq.data_ptr(), bq.data_ptr(), Wk.data_ptr(), bk.data_ptr()),
+                    (Wq, bq, Wk, bk))
+    for Dp, causal, Tc, To, flags in points:
+        phi = phis[Dp][0]
+        p = rh.make_params(batch=B, heads=H, T=T, Hs=Hs, Ws=Ws, D=D, Dp=Dp, Tc=Tc,
+                           To=To, causal=causal, in_dtype=rh.BF16, out_dtype=rh.F32,
+                           flags=flags)
+        nbytes = rh.rehyat_workspace_bytes(p)
+        if nbytes == 0:
+            continue
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
 
-                    def call(evs=None):
-                        if evs:
-                            evs[0].record(stream)
-                        rh.rehyat_fwd_state(p, k.data_ptr(), v.data_ptr(), phi, ws.data_ptr(),
-                                            nbytes, stream.cuda_stream)
-                        if evs:
-                            evs[1].record(stream)
-                        st = rh.rehyat_fwd_attn(p, q.data_ptr(), k.data_ptr(), v.data_ptr(), phi,
-                                                y.data_ptr(), ws.data_ptr(), nbytes, None,
-                                                stream.cuda_stream)
-                        if st:
-                            raise rh.RehyatError(st, "rehyat_fwd_attn")
-                        if evs:
-                            evs[2].record(stream)
+        def call(evs=None):
+            if evs:
+                evs[0].record(stream)
+            rh.rehyat_fwd_state(p, k.data_ptr(), v.data_ptr(), phi, ws.data_ptr(),
+                                nbytes, stream.cuda_stream)
+            if evs:
+                evs[1].record(stream)
+            st = rh.rehyat_fwd_attn(p, q.data_ptr(), k.data_ptr(), v.data_ptr(), phi,
+                                    y.data_ptr(), ws.data_ptr(), nbytes, None,
+                                    stream.cuda_stream)
+            if st:
+                raise rh.RehyatError(st, "rehyat_fwd_attn")
+            if evs:
+                evs[2].record(stream)
 
-                    for _ in range(3):
-                        call()
-                    times = []
-                    for _ in range(max(3, args.steps // 6)):
-                        flush()
-                        evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-                        call(evs)
-                        torch.cuda.synchronize()
-                        times.append((evs[0].elapsed_time(evs[2]), evs[1].elapsed_time(evs[2])))
-                    step_ms = sum(t[0] for t in times) / len(times)
-                    attn_ms = sum(t[1] for t in times) / len(times)
-                    w = algorithmic_work(B, H, T, HW, D, Dp, Tc, To, causal)
-                    attn_tf = w["attn_flops"] / (attn_ms / 1e3) / 1e12
-                    print(json.dumps({
-                        "sweep": "21x30x52", "Tc": Tc, "To": To, "Dp": Dp,
-                        "form": "causal" if causal else "bidirectional",
-                        "attn_kernel": "tensor-core two-tile" if rh.rehyat_attn_path(p) == 1 and Dp <= 128
-                        else ("tensor-core one-tile" if rh.rehyat_attn_path(p) == 1 else "CUDA-core"),
-                        "ms_per_step": step_ms, "tokens_per_s": B * N / (step_ms / 1e3),
-                        "attn_ms": attn_ms, "attn_tflops": attn_tf,
-                        "attn_frac_bf16_peak": attn_tf / peaks["bf16_tflops"],
-                        "total_tflop": w["total_flops"] / 1e12,
-                        "full_softmax_over_hybrid_flops": w["full_softmax_flops"] / w["total_flops"],
-                    }), flush=True)
-                    del ws
+        for _ in range(3):
+            call()
+        times = []
+        for _ in range(max(3, args.steps // 6)):
+            flush()
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            call(evs)
+            torch.cuda.synchronize()
+            times.append((evs[0].elapsed_time(evs[2]), evs[1].elapsed_time(evs[2])))
+        step_ms = sum(t[0] for t in times) / len(times)
+        attn_ms = sum(t[1] for t in times) / len(times)
+        w = algorithmic_work(B, H, T, HW, D, Dp, Tc, To, causal)
+        attn_tf = w["attn_flops"] / (attn_ms / 1e3) / 1e12
+        state_gbs = w["state_bytes"] / ((step_ms - attn_ms) / 1e3) / 1e9
+        print(json.dumps({
+            "sweep": "21x30x52", "Tc": Tc, "To": To, "Dp": Dp,
+            "form": "causal" if causal else "bidirectional",
+            "qk": "fp8 e4m3" if flags else "bf16",
+            "attn_kernel": "tensor-core two-tile" if rh.rehyat_attn_path(p) == 1
+            else "CUDA-core",
+            "ms_per_step": step_ms, "tokens_per_s": B * N / (step_ms / 1e3),
+            "state_ms": step_ms - attn_ms, "state_frac_hbm": state_gbs / peaks["hbm_gbs"],
+            "attn_ms": attn_ms, "attn_tflops": attn_tf,
+            "attn_frac_bf16_peak": attn_tf / peaks["bf16_tflops"],
+            "total_tflop": w["total_flops"] / 1e12,
+            "full_softmax_over_hybrid_flops": w["full_softmax_flops"] / w["total_flops"],
+        }), flush=True)
+        del ws
     return 0
 
 
