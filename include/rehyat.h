@@ -201,16 +201,30 @@ REHYAT_API rehyat_status rehyat_softmax_attn_fwd(const rehyat_params* p, const v
 /* Bytes of the opaque streaming state: the running s [B][h][Dp][D] and
  * z [B][h][Dp] (fp32), a ring holding the keys and values of the last T_o
  * slices (in_dtype), and a device-side count of slices consumed (with a
- * completion count that is zero between steps).  Constant for any number of
- * steps; a copy taken between steps restores the stream exactly. */
+ * completion count and the split attention's arrival counters, all zero
+ * between steps).  Constant for any number of steps; a copy taken between
+ * steps restores the stream exactly.  After a step that set a bit in
+ * rehyat_device_error_flags the state must be re-initialised. */
 REHYAT_API size_t rehyat_state_bytes(const rehyat_params* p);
 
 /* Reset a state to the start of a video: s = 0, z = 0, empty ring. */
 REHYAT_API rehyat_status rehyat_state_init(const rehyat_params* p, void* state,
                                 void* stream);
 
-/* Workspace bytes rehyat_chunk_step needs. */
+/* Workspace bytes rehyat_chunk_step needs on the current device.  With the
+ * two-tile tensor-core attention the step may split each pair of query
+ * tiles' key window over several CTAs so that the chunk fills the device's
+ * SMs; the split is chosen from the shape and the device's SM count, and
+ * its partials (fp32 a^S, maximum and row sum per query row and piece) live
+ * here. */
 REHYAT_API size_t rehyat_step_workspace_bytes(const rehyat_params* p);
+
+/* Pieces the key window of each pair of query tiles is split into by
+ * rehyat_chunk_step for a chunk of `nslices` slices on the current device
+ * (1: no split; 0: p or nslices invalid).  A split runs the pieces as
+ * separate CTAs and merges their partial softmax sums exactly (the row
+ * maximum is the maximum of the pieces' maxima), in piece order. */
+REHYAT_API int rehyat_step_key_split(const rehyat_params* p, int nslices);
 
 /* One step of the chunk-wise RNN: consumes the next `nslices` latent slices
  * (1 <= nslices <= Tc; the last chunk of a video may be shorter) given as

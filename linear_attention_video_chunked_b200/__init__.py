@@ -36,6 +36,7 @@ __all__ = [
     "make_params", "hybrid_attn", "hybrid_attn_phi", "feature_map_mlp", "softmax_attn",
     "phi_grad", "StreamingState", "rehyat_hybrid_attn_bwd_workspace_bytes",
     "rehyat_hybrid_attn_bwd", "hybrid_attn_bwd", "rehyat_denominator_report",
+    "rehyat_step_key_split",
 ]
 
 F32, BF16 = 0, 1
@@ -56,7 +57,7 @@ EXPORTED_SYMBOLS = (
     "rehyat_hybrid_attn_fwd_phi", "rehyat_feature_map_mlp",
     "rehyat_feature_map_mlp_workspace_bytes", "rehyat_host_workspace_bytes",
     "rehyat_hybrid_attn_fwd_host", "rehyat_hybrid_attn_bwd_workspace_bytes",
-    "rehyat_hybrid_attn_bwd", "rehyat_denominator_report",
+    "rehyat_hybrid_attn_bwd", "rehyat_denominator_report", "rehyat_step_key_split",
 )
 
 
@@ -138,6 +139,8 @@ def lib() -> ctypes.CDLL:
         L.rehyat_state_init.restype = i
         L.rehyat_step_workspace_bytes.argtypes = [P(RehyatParams)]
         L.rehyat_step_workspace_bytes.restype = sz
+        L.rehyat_step_key_split.argtypes = [P(RehyatParams), ctypes.c_int]
+        L.rehyat_step_key_split.restype = ctypes.c_int
         L.rehyat_chunk_step.argtypes = [P(RehyatParams), vp, vp, vp, i, P(RehyatPhi), vp, vp, vp,
                                         sz, P(RehyatDebug), vp]
         L.rehyat_chunk_step.restype = i
@@ -278,6 +281,10 @@ def rehyat_state_init(p, state, stream) -> int:
 
 def rehyat_step_workspace_bytes(p: RehyatParams) -> int:
     return lib().rehyat_step_workspace_bytes(ctypes.byref(p))
+
+
+def rehyat_step_key_split(p: RehyatParams, nslices: int) -> int:
+    return lib().rehyat_step_key_split(ctypes.byref(p), int(nslices))
 
 
 def rehyat_chunk_step(p, q, k, v, nslices, phi, state, y, workspace, ws_bytes, dbg,

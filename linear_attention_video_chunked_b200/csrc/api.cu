@@ -97,8 +97,30 @@ cudaError_t run_partials(const rehyat_params* p, const PartialParams& pp, const 
 }
 
 struct StateLayout {
-  size_t s_off, z_off, rk_off, rv_off, total;
+  size_t s_off, z_off, cnt_off, rk_off, rv_off, total;
 };
+
+int device_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    return 148;
+  }
+  return n;
+}
+
+// Pieces of the key window per pair of query tiles in a streaming step of
+// nslices slices (the two-tile tensor-core kernel only; 1 = no split).
+StepSplit step_split(const rehyat_params* p, int nslices) {
+  if (!tc_path(p) || (p->flags & REHYAT_FLAG_ONE_TILE)) return StepSplit{1, 0};
+  return attn_step_split(p->batch * p->heads, p->Hs * p->Ws, nslices, p->To, device_sm_count());
+}
+
+size_t step_pairs(const rehyat_params* p) {
+  const size_t qrows = static_cast<size_t>(p->Tc) * p->Hs * p->Ws;
+  return (qrows + 255) / 256;
+}
 
 // Streaming state header (kAlign bytes, zeroed by rehyat_state_init): the
 // int64 count of slices consumed at offset 0, and at kStepDoneOffset the
@@ -111,7 +133,10 @@ StateLayout state_layout(const rehyat_params* p) {
   StateLayout s;
   s.s_off = kAlign;  // header: slice counter, step completion count
   s.z_off = align_up(s.s_off + BH * p->Dp * p->D * sizeof(float));
-  s.rk_off = align_up(s.z_off + BH * p->Dp * sizeof(float));
+  // Arrival counters of the split attention, one per (b, h, pair of query
+  // tiles); zeroed with the state and left zero by every step.
+  s.cnt_off = align_up(s.z_off + BH * p->Dp * sizeof(float));
+  s.rk_off = align_up(s.cnt_off + BH * step_pairs(p) * sizeof(unsigned));
   const size_t ring = BH * p->To * HW * p->D * elem_bytes(p->in_dtype);
   s.rv_off = align_up(s.rk_off + ring);
   s.total = align_up(s.rv_off + ring);
@@ -119,7 +144,7 @@ StateLayout state_layout(const rehyat_params* p) {
 }
 
 struct StepWorkspace {
-  size_t P_off, z_off, wimg_off, wkimg_off, total;
+  size_t P_off, z_off, wimg_off, wkimg_off, part_off, total;
   int nslots;
 };
 
@@ -131,7 +156,14 @@ StepWorkspace step_layout(const rehyat_params* p) {
   w.z_off = align_up(BH * w.nslots * static_cast<size_t>(p->Dp) * p->D * sizeof(float));
   w.wimg_off = align_up(w.z_off + BH * w.nslots * p->Dp * sizeof(float));
   w.wkimg_off = align_up(w.wimg_off + wimg_bytes(p));
-  w.total = align_up(w.wkimg_off + wimg_bytes(p));
+  w.part_off = align_up(w.wkimg_off + wimg_bytes(p));
+  size_t part = 0;  // split attention partials, for any chunk length <= T_c
+  for (int n = 1; n <= p->Tc; ++n) {
+    const size_t b = attn_split_part_bytes(static_cast<int>(BH), p->Hs * p->Ws, n,
+                                           step_split(p, n));
+    part = b > part ? b : part;
+  }
+  w.total = align_up(w.part_off + part);
   return w;
 }
 
@@ -379,6 +411,12 @@ size_t rehyat_step_workspace_bytes(const rehyat_params* p) {
   return step_layout(p).total;
 }
 
+int rehyat_step_key_split(const rehyat_params* p, int nslices) {
+  if (check_params(p) != REHYAT_OK || no_fp8(p) != REHYAT_OK || nslices < 1 || nslices > p->Tc)
+    return 0;
+  return step_split(p, nslices).ksplit;
+}
+
 rehyat_status rehyat_state_init(const rehyat_params* p, void* state, void* stream) {
   rehyat_status st = check_params(p);
   if (st != REHYAT_OK) return st;
@@ -433,6 +471,16 @@ rehyat_status rehyat_chunk_step(const rehyat_params* p, const void* q, const voi
   a.SL = s_state; a.zL = z_state;
   a.nchunks = 1;
   a.nq_slices = nslices;
+  const StepSplit sp = step_split(p, nslices);
+  a.ksplit = sp.ksplit;
+  a.kwhole = sp.whole;
+  if (a.ksplit > 1) {
+    // The partials of this call's split must fit the workspace's region.
+    const size_t need = attn_split_part_bytes(BH, HW, nslices, sp);
+    if (need == 0 || w.part_off + need > ws_bytes) return REHYAT_ERR_WORKSPACE;
+    a.part = reinterpret_cast<float*>(ws + w.part_off);
+    a.part_cnt = reinterpret_cast<unsigned*>(stb + L.cnt_off);
+  }
   cudaError_t e = cudaSuccess;
   if (tc_path(p) || tc_state_path(p)) {
     e = launch_w_images(phi->Wq, ws + w.wimg_off, phi->Wk, ws + w.wkimg_off, p->heads, p->D,

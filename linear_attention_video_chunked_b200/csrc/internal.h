@@ -37,7 +37,26 @@ struct AttnParams {
   int in_bf16, out_bf16, w_bf16, full_softmax;
   int one_tile;              // tensor-core path: force the one-query-tile kernel
   float scale_log2;          // logit scale * log2(e)
+  // Step mode, two-tile tensor-core kernel: with ksplit > 1 the pairs of
+  // query tiles past the first kwhole (in (b*h, pair) order; the pairs that
+  // hold only tile A always run whole) run as ksplit CTAs over consecutive
+  // pieces of the key window, which leave their partial a^S, maximum and row
+  // sum in part (attn_split_part_bytes) and count themselves in
+  // part_cnt[split pair] (zero between launches); the last piece to arrive
+  // merges all pieces in order and writes y.
+  int ksplit, kwhole;
+  float* part;
+  unsigned* part_cnt;
 };
+
+// Key-window split of a streaming step's attention (tc_kernels.cu) for a
+// chunk of nq_slices slices on a device with `sms` SMs: pieces per split
+// pair (1 = no split) and the number of two-tile pairs run whole.
+struct StepSplit {
+  int ksplit, whole;
+};
+StepSplit attn_step_split(int BH, int HW, int nq_slices, int To, int sms);
+size_t attn_split_part_bytes(int BH, int HW, int nq_slices, StepSplit sp);
 
 // Per-slice linear state: P_i = sum_{rows of slice i} phi_k(k) v^T ([Dp][D])
 // and z_i = sum phi_k(k) ([Dp]).

@@ -25,6 +25,12 @@
 // Every wait is bounded: a barrier that does not complete within ~2 s of
 // clock sets an error bit in rehyat_tc_error and the kernel unwinds.
 #include <atomic>
+#include <functional>
+#include <map>
+#include <mutex>
+#include <queue>
+#include <tuple>
+#include <vector>
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -550,6 +556,12 @@ enum { Q_FULL = 0, K_FULL = 1, K_EMPTY = 4, V_FULL = 7, V_EMPTY = 9, S_FULL = 11
 constexpr uint32_t kXchgCol0 = 63, kXchgCol1 = 127, kLxCol = 126;
 constexpr uint32_t kTmemSlot = kBarOff + 8 * NBAR;
 constexpr uint32_t kAbortSlot = kTmemSlot + 4;
+constexpr uint32_t kLastSlot = kAbortSlot + 4;     // split key window: this CTA merges
+constexpr uint32_t kSplitSlot = kLastSlot + 4;     // (split pair slot, piece, pieces) for the tail
+// Split key window (streaming step): per piece and tile, 33 float4 columns of
+// 128 rows -- a^S in 32 (relative to the piece's own row maximum), then
+// (maximum, row sum, 0, 0) -- so a warp's 32 rows are 512 contiguous bytes.
+constexpr int kPartVec = 33;
 // b_q of the head and z^L of the chunk (D' floats each), shared by both tiles.
 constexpr uint32_t kVecOff = kBarOff + 256;
 constexpr uint32_t kSmemBytes = kVecOff + 1024 + 1024;
@@ -584,12 +596,43 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int t = blockIdx.y;
-  const int bh = blockIdx.z;
+  const bool step_mode = P.seen != nullptr;
+  int t = blockIdx.y;
+  int bh = blockIdx.z;
+  int pair = blockIdx.x;      // pair of query tiles within the chunk
+  int split = 0, nsplit = 1;  // piece of the key window this CTA runs
+  int slot = 0;               // split pair index (partials, arrival counter)
+  if (step_mode && P.ksplit > 1) {
+    // Work list in dispatch order: the BH pairs that hold only tile A, then
+    // kwhole two-tile pairs run whole, then the remaining two-tile pairs as
+    // ksplit key pieces each.
+    const int qrows = P.nq_slices * P.HW;
+    const int npairs = (qrows + 2 * kBM - 1) / (2 * kBM);
+    const bool light = qrows - (npairs - 1) * 2 * kBM <= kBM;
+    const int nfull = npairs - (light ? 1 : 0);
+    const int nl = light ? P.BH : 0;
+    int L = blockIdx.x;
+    t = 0;
+    if (L < nl) {
+      bh = L;
+      pair = npairs - 1;
+    } else {
+      L -= nl;
+      int item = L;
+      if (L >= P.kwhole) {
+        L -= P.kwhole;
+        slot = L / P.ksplit;
+        split = L % P.ksplit;
+        nsplit = P.ksplit;
+        item = P.kwhole + slot;
+      }
+      bh = item / nfull;
+      pair = item % nfull;
+    }
+  }
   const int h = bh % P.heads;
 
   int q_first, q_end, na, nb, a_row0;
-  const bool step_mode = P.seen != nullptr;
   if (!step_mode) {
     const int first = t * P.Tc;
     const int end = min(P.T, first + P.Tc);
@@ -608,19 +651,25 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
     na = r_slices * P.HW;
     nb = q_end;
   }
-  const int row0 = q_first + blockIdx.x * 2 * kBM;
+  const int row0 = q_first + pair * 2 * kBM;
   if (row0 >= q_end) return;
   const int nrows_t[2] = {min(kBM, q_end - row0), max(0, min(kBM, q_end - row0 - kBM))};
   const bool has_b = nrows_t[1] > 0;
   const int nta = (na + kBN - 1) / kBN;
-  const int nt = nta + (nb + kBN - 1) / kBN;
+  const int nt_all = nta + (nb + kBN - 1) / kBN;
+  // Key tiles [j0, j0 + nt) of the window (all of it unless split; the host
+  // keeps ksplit <= the chunk's own key tiles, so every piece has one).
+  const int j0 = split * nt_all / nsplit;
+  const int nt = (split + 1) * nt_all / nsplit - j0;
+  const bool split_kv = nsplit > 1;
   const bool linear = !P.full_softmax;
   const bool phi_given = P.phi_q != nullptr;  // phi_q(q) read from P.phi_q
   const int Dp = P.Dp;
   const int npieces = Dp > 128 ? 2 : 1;       // feature pieces of the readout
   const int pw = Dp / npieces;
 
-  auto tile_src = [&](int j) {
+  auto tile_src = [&](int jl) {
+    const int j = j0 + jl;
     TileSrc s;
     if (j < nta) {
       s.map_k = step_mode ? &maps.rk : &maps.k;
@@ -645,6 +694,11 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
       mbar_init(bar(i), by_all ? 2 * kSoftmaxThreads : (by_warpgroup ? kSoftmaxThreads : 1));
     }
     *abort_flag = 0;
+    *reinterpret_cast<volatile uint32_t*>(sbase + a2::kLastSlot) = split_kv ? 0u : 1u;
+    volatile int* sp = reinterpret_cast<volatile int*>(sbase + a2::kSplitSlot);
+    sp[0] = slot;
+    sp[1] = split;
+    sp[2] = nsplit;
     fence_barrier_init();
   }
   if (warp == 9) {
@@ -657,6 +711,9 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sbase + kTmemSlot);
+  // Split key window: after LX_DONE this says whether this CTA merges the
+  // pieces and runs the tail (the last piece of the pair to finish).
+  auto merges = [&]() { return *reinterpret_cast<volatile uint32_t*>(sbase + a2::kLastSlot) != 0; };
 
   if (warp == 8) {
     // ================================================= TMA producer
@@ -694,6 +751,8 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
         tma_load_3d(vdst, src.map_v, bar(a2::V_FULL + vs), 0, src.row, bh);
         tma_load_3d(vdst + 16384, src.map_v, bar(a2::V_FULL + vs), 64, src.row, bh);
       }
+      // A split piece loads the tail operands only if it merges.
+      if (ok && split_kv) ok = mbar_wait(bar(a2::LX_DONE), 0, abort_flag, 20) && merges();
       if (linear && ok) {
         const uint32_t wbytes = static_cast<uint32_t>(pw) * kD * 2;
         const uint32_t slbytes = static_cast<uint32_t>(pw) * kD * 4;
@@ -774,6 +833,7 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
         if (more) mma_commit(bar(a2::K_EMPTY + (j + 1) % 3));
         if (j == nt - 1) mma_commit(bar(a2::LAST_PV));
       }
+      if (ok && split_kv) ok = mbar_wait(bar(a2::LX_DONE), 0, abort_flag, 20) && merges();
       // Linear readout, one feature piece of pw <= 128 at a time.
       for (int pc = 0; linear && ok && pc < npieces; ++pc) {
         ok = mbar_wait(bar(a2::TAIL_FULL), pc & 1, abort_flag, 9);
@@ -969,10 +1029,103 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
       tc_fence_after();
       l2[tile] += __uint_as_float(tmem_ld1(lane_base + tile * 256 + a2::kLxCol));
     }
+    bool run_tail = true;
+    if (split_kv) {
+      const volatile int* sp = reinterpret_cast<const volatile int*>(sbase + a2::kSplitSlot);
+      const int slot = sp[0], split = sp[1], nsplit = sp[2];
+      // Split key window (both tiles present): every piece leaves its a^S,
+      // row maximum and row sum in the partials; the last piece of the pair
+      // to arrive folds the others into its own TMEM accumulator and runs
+      // the tail.  Nothing waits on another CTA.
+      const int nrows = nrows_t[tile];
+      float4* part = reinterpret_cast<float4*>(P.part);
+      auto part_at = [&](int piece, int cc) {
+        return part + ((static_cast<long long>(slot * nsplit + piece) * 2 + tile) * a2::kPartVec +
+                       cc) * kBM + r;
+      };
+      ok = wait_all(bar(a2::LAST_PV), 0, 19);
+      if (ok) {
+        tc_fence_after();
+        const float fs = ex2(m_used2[tile] - m_max2[tile]);
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          REHYAT_TMEM_LD32(lane_base + tile * 256 + 128 + c * 32, o);
+          tmem_wait_ld();
+          if (r < nrows)
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              *part_at(split, c * 8 + i) =
+                  make_float4(__uint_as_float(o[4 * i]) * fs, __uint_as_float(o[4 * i + 1]) * fs,
+                              __uint_as_float(o[4 * i + 2]) * fs, __uint_as_float(o[4 * i + 3]) * fs);
+        }
+        if (r < nrows) *part_at(split, 32) = make_float4(m_max2[tile], l2[tile] * fs, 0.f, 0.f);
+      }
+      __threadfence();
+      asm volatile("bar.sync 3, %0;" ::"r"(2 * kSoftmaxThreads) : "memory");
+      volatile uint32_t* last_slot = reinterpret_cast<volatile uint32_t*>(sbase + a2::kLastSlot);
+      if (tid == 0) {
+        unsigned* cnt = P.part_cnt + slot;
+        const bool last = atomicAdd(cnt, 1u) == static_cast<unsigned>(nsplit - 1);
+        if (last) atomicExch(cnt, 0u);  // ready for the next launch
+        __threadfence();
+        *last_slot = last ? 1u : 0u;
+      }
+      asm volatile("bar.sync 3, %0;" ::"r"(2 * kSoftmaxThreads) : "memory");
+      run_tail = *last_slot != 0;
+      if (ok && run_tail) {  // warp-uniform: the TMEM stores are collective
+        // Every piece, this CTA's own included, is read back from the
+        // partials and summed in piece order, so y does not depend on which
+        // piece arrived last.
+        const bool valid = r < nrows;
+        float mp[4], w[4];
+        float mx = -INFINITY, l = 0.f;
+#pragma unroll
+        for (int pc = 0; pc < 4; ++pc) {
+          const float4 ml = valid && pc < nsplit ? __ldcg(part_at(pc, 32))
+                                                 : make_float4(-INFINITY, 0.f, 0.f, 0.f);
+          mp[pc] = ml.x;
+          w[pc] = ml.y;  // row sum for now
+          mx = fmaxf(mx, ml.x);
+        }
+        if (!valid) mx = 0.f;
+#pragma unroll
+        for (int pc = 0; pc < 4; ++pc) {
+          const float sum = w[pc];
+          w[pc] = valid && pc < nsplit ? ex2(mp[pc] - mx) : 0.f;
+          l = fmaf(sum, w[pc], l);
+        }
+        for (int c = 0; c < 4; ++c) {
+          float o[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = 0.f;
+#pragma unroll
+          for (int pc = 0; pc < 4; ++pc) {
+            if (!(valid && pc < nsplit)) continue;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float4 v4 = __ldcg(part_at(pc, c * 8 + i));
+              o[4 * i] = fmaf(v4.x, w[pc], o[4 * i]);
+              o[4 * i + 1] = fmaf(v4.y, w[pc], o[4 * i + 1]);
+              o[4 * i + 2] = fmaf(v4.z, w[pc], o[4 * i + 2]);
+              o[4 * i + 3] = fmaf(v4.w, w[pc], o[4 * i + 3]);
+            }
+          }
+          uint32_t ob[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ob[i] = __float_as_uint(o[i]);
+          REHYAT_TMEM_ST32(lane_base + tile * 256 + 128 + c * 32, ob);
+        }
+        tmem_wait_st();
+        m_used2[tile] = mx;
+        m_max2[tile] = mx;
+        l2[tile] = l;
+      }
+    }
     tc_fence_before();
     mbar_arrive(bar(a2::LX_DONE));
-    if (tile >= ntiles) {
-      // Tile B is empty: warps 4-7 have no tail.
+    if (tile >= ntiles || !run_tail) {
+      // Tile B is empty (warps 4-7 have no tail), or another piece of this
+      // pair merges and writes y.
     } else {
     const uint32_t s_col = tile * 256, o_col = s_col + 128;
     const int nrows = nrows_t[tile];
@@ -1770,6 +1923,92 @@ bool tc_attn_supported(const AttnParams& p) {
   return encode_fn() != nullptr;
 }
 
+namespace {
+struct StepSplitKey {
+  int BH, HW, nq, To, sms;
+  bool operator<(const StepSplitKey& o) const {
+    return std::tie(BH, HW, nq, To, sms) < std::tie(o.BH, o.HW, o.nq, o.To, o.sms);
+  }
+};
+std::mutex g_split_mu;
+std::map<StepSplitKey, StepSplit> g_split_cache;
+
+StepSplit choose_step_split(int BH, int HW, int nq_slices, int To, int sms) {
+  // Pieces run as CTAs, one per SM, in work-list order; a greedy list
+  // schedule of their estimated lengths on `sms` SMs gives the makespan.
+  // Units: one key step of a two-tile CTA (about 2.3 us on the 30x52
+  // layer).  A tile-A-only pair's step costs about 0.8 of that; a CTA's
+  // prologue 1.5 steps, its tail 4.5, a split piece's tail 6.5 on average
+  // (its partials, and for the last piece the merge).
+  StepSplit none{1, 0};
+  const int qrows = nq_slices * HW;
+  const int npairs = (qrows + 2 * kBM - 1) / (2 * kBM);
+  if (BH <= 0 || npairs <= 0 || sms <= 0) return none;
+  const bool light = qrows - (npairs - 1) * 2 * kBM <= kBM;
+  const int nfull = npairs - (light ? 1 : 0);
+  const int nl = light ? BH : 0;
+  const int full = BH * nfull;
+  const int ntb = (qrows + kBN - 1) / kBN;
+  const int nt = (To * HW + kBN - 1) / kBN + ntb;
+  if (full == 0 || nl + full > 3 * sms) return none;
+  std::vector<double> load(static_cast<size_t>(sms));
+  auto makespan = [&](int ks, int whole) {
+    std::priority_queue<double, std::vector<double>, std::greater<double>> q;
+    for (int i = 0; i < sms; ++i) q.push(0.0);
+    auto put = [&](double cost) {
+      const double t0 = q.top();
+      q.pop();
+      q.push(t0 + cost);
+    };
+    for (int i = 0; i < nl; ++i) put(1.5 + 0.8 * nt + 4.5);
+    for (int i = 0; i < whole; ++i) put(1.5 + nt + 4.5);
+    for (int i = whole; i < full; ++i)
+      for (int pc = 0; pc < ks; ++pc)
+        put(1.5 + static_cast<double>((pc + 1) * nt / ks - pc * nt / ks) + 6.5);
+    double mx = 0.0;
+    while (!q.empty()) {
+      mx = q.top() > mx ? q.top() : mx;
+      q.pop();
+    }
+    return mx;
+  };
+  const double base = makespan(1, full);
+  StepSplit best = none;
+  double best_t = base;
+  const int cand[] = {0, sms - nl, sms, 2 * sms - nl, 2 * sms};
+  for (int ks = 2; ks <= 4 && ks <= ntb; ++ks)
+    for (int w : cand) {
+      if (w < 0 || w >= full) continue;
+      const double tk = makespan(ks, w);
+      if (tk < best_t) {
+        best_t = tk;
+        best = StepSplit{ks, w};
+      }
+    }
+  return best_t < 0.97 * base ? best : none;
+}
+}  // namespace
+
+StepSplit attn_step_split(int BH, int HW, int nq_slices, int To, int sms) {
+  const StepSplitKey key{BH, HW, nq_slices, To, sms};
+  std::lock_guard<std::mutex> lock(g_split_mu);
+  auto it = g_split_cache.find(key);
+  if (it != g_split_cache.end()) return it->second;
+  const StepSplit r = choose_step_split(BH, HW, nq_slices, To, sms);
+  if (g_split_cache.size() < 4096) g_split_cache.emplace(key, r);
+  return r;
+}
+
+size_t attn_split_part_bytes(int BH, int HW, int nq_slices, StepSplit sp) {
+  if (sp.ksplit <= 1) return 0;
+  const int qrows = nq_slices * HW;
+  const int npairs = (qrows + 2 * kBM - 1) / (2 * kBM);
+  const bool light = qrows - (npairs - 1) * 2 * kBM <= kBM;
+  const long long full = static_cast<long long>(BH) * (npairs - (light ? 1 : 0));
+  if (sp.whole < 0 || sp.whole >= full) return 0;
+  return static_cast<size_t>(full - sp.whole) * sp.ksplit * 2 * a2::kPartVec * kBM * 16;
+}
+
 cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s) {
   TcMaps maps;
   memset(&maps, 0, sizeof(maps));
@@ -1803,6 +2042,16 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s) {
     e = ensure_smem(tc_attn2_kernel<false>, 1, a2::kSmemBytes);
     if (e != cudaSuccess) return e;
     dim3 grid((qrows_max + 2 * kBM - 1) / (2 * kBM), p.nchunks, p.BH);
+    if (p.seen && p.ksplit > 1) {
+      // Work list: the tile-A-only pairs, kwhole whole two-tile pairs, then
+      // ksplit pieces for each remaining two-tile pair.
+      const int npairs = static_cast<int>(grid.x);
+      const bool light = qrows_max - (npairs - 1) * 2 * kBM <= kBM;
+      const int full = p.BH * (npairs - (light ? 1 : 0));
+      if (!p.part || !p.part_cnt || p.nchunks != 1 || p.kwhole < 0 || p.kwhole >= full)
+        return cudaErrorInvalidValue;
+      grid = dim3((light ? p.BH : 0) + p.kwhole + (full - p.kwhole) * p.ksplit, 1, 1);
+    }
     tc_attn2_kernel<false><<<grid, a2::kThreads, a2::kSmemBytes, s>>>(
         maps, p, static_cast<const __nv_bfloat16*>(p.wq_img));
   } else {

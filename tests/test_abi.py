@@ -300,3 +300,25 @@ def test_header_is_plain_c_and_the_library_links_from_c(tmp_path):
     assert ws == rh.rehyat_workspace_bytes(p) > 0
     assert path == rh.rehyat_attn_path(p) == 1
     assert st == 1  # REHYAT_ERR_INVALID_ARG, before any launch
+
+
+def test_step_key_split_choice():
+    """The streaming step's key-window split: 0 for invalid arguments, 2
+    pieces for 12 heads of 30x52 with T_c = 3, T_o = 1 on a 148-SM B200 (228
+    CTAs would run in 1.54 waves; the pairs past the first wave split in two),
+    none where the chunk already makes several waves or the CUDA-core path
+    runs."""
+    kw = dict(batch=1, heads=12, T=3, Hs=30, Ws=52, D=128, Dp=128, Tc=3, To=1, causal=1,
+              in_dtype=rh.BF16, out_dtype=rh.F32)
+    p = rh.make_params(**kw)
+    assert rh.rehyat_step_key_split(p, 0) == 0
+    assert rh.rehyat_step_key_split(p, 4) == 0
+    assert rh.rehyat_step_key_split(p, 3) == 2
+    assert rh.rehyat_step_key_split(rh.make_params(**{**kw, "batch": 8}), 3) == 1
+    assert rh.rehyat_step_key_split(rh.make_params(**{**kw, "flags": rh.FLAG_FORCE_SIMT}), 3) == 1
+    assert rh.rehyat_step_key_split(rh.make_params(**{**kw, "in_dtype": rh.F32}), 3) == 1
+    # The workspace holds the partials of the split pairs: at most 12 x 19
+    # pairs x 4 pieces x 2 tiles x 128 rows x 33 float4.
+    ws = rh.rehyat_step_workspace_bytes(p)
+    ws_simt = rh.rehyat_step_workspace_bytes(rh.make_params(**{**kw, "flags": rh.FLAG_FORCE_SIMT}))
+    assert 0 < ws - ws_simt <= 12 * 19 * 4 * 2 * 128 * 33 * 16 + 256

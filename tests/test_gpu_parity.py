@@ -201,6 +201,28 @@ def test_streaming_wide_and_narrow_phi(Dp, Tc, To):
     assert_close_y(y_stream.double().cpu().numpy(), ref_y, "bf16")
 
 
+@pytest.mark.parametrize("Tc,To,T", [(3, 1, 10), (2, 2, 7), (4, 0, 9)])
+def test_streaming_split_key_window(Tc, To, T):
+    """Chunks of 16x20 slices on 2 heads: the step splits each pair of query
+    tiles' key window over several CTAs (the last chunk is one slice, split
+    or not by its own schedule, and at T_c = 2 every chunk ends in a pair with
+    tile A only, which runs whole).
+    Outputs against the RNN oracle and the full causal forward, and bit for
+    bit the same on a second run (the merge sums the pieces in order)."""
+    p = make_problem(batch=1, heads=2, T=T, Hs=16, Ws=20, D=128, Dp=128, Tc=Tc, To=To,
+                     causal=True, dtype="bf16", seed=71 + Tc + 5 * To)
+    dev = device_tensors(p)
+    y_stream, st = _stream_outputs(p, dev=dev)
+    assert rh.rehyat_step_key_split(st.p, Tc) > 1
+    ref_y, _ = orc.run_problem(p, form="rnn")
+    assert_close_y(y_stream.double().cpu().numpy(), ref_y, "bf16")
+    y_full = run_fwd(p)
+    mx, _ = err_stats(y_stream.double().cpu().numpy(), y_full)
+    assert mx <= 2e-2
+    y_again, _ = _stream_outputs(p, dev=dev)
+    assert torch.equal(y_again, y_stream)
+
+
 def test_stream_81_slices_constant_memory():
     """81 slices of 30x52, 27 steps: outputs of sampled heads match the oracle
     and free device memory does not move across steps."""
@@ -217,20 +239,27 @@ def test_stream_81_slices_constant_memory():
     torch.cuda.synchronize()
     free0 = torch.cuda.mem_get_info()[0]
     frees = []
+    # Head 3's pairs of query tiles run whole, head 10's as split key pieces
+    # (the step's work list puts the pairs past the first wave in pieces).
+    subset = [3, 10]
     for s in range(27):
         st.step(*chunks[s], out=out)
-        ys.append(out[0, 3].double().cpu().numpy())
+        ys.append(out[0, subset].double().cpu().numpy())
         frees.append(torch.cuda.mem_get_info()[0])
     assert all(f == free0 for f in frees)
-    subset = [3]
     ref_y, _ = orc.run_problem(p, heads_subset=subset)
-    assert_close_y(np.concatenate(ys), ref_y[0, 3], "bf16")
+    got = np.concatenate(ys, axis=1)
+    for i, h in enumerate(subset):
+        assert_close_y(got[i], ref_y[0, h], "bf16")
 
 
-def test_streaming_cuda_graph_replay_matches_eager():
+# 16x20 slices: the step splits the key window (the arrival counters live in
+# the state and return to zero every step).
+@pytest.mark.parametrize("Hs,Ws", [(6, 11), (16, 20)])
+def test_streaming_cuda_graph_replay_matches_eager(Hs, Ws):
     """One captured step replayed per chunk equals the eager steps bit for
     bit (the slice counter is read on the device)."""
-    p = make_problem(batch=1, heads=2, T=10, Hs=6, Ws=11, D=128, Dp=128, Tc=2, To=1,
+    p = make_problem(batch=1, heads=2, T=10, Hs=Hs, Ws=Ws, D=128, Dp=128, Tc=2, To=1,
                      causal=True, dtype="bf16", seed=43)
     y_eager, st = _stream_outputs(p)
     dev = device_tensors(p)
@@ -252,11 +281,12 @@ def test_streaming_cuda_graph_replay_matches_eager():
     assert torch.equal(torch.cat(outs, dim=2), y_eager)
 
 
-def test_streaming_sequence_graph_matches_eager():
+@pytest.mark.parametrize("Hs,Ws", [(6, 11), (16, 20)])
+def test_streaming_sequence_graph_matches_eager(Hs, Ws):
     """All steps of a stream captured as one CUDA graph (each step on its own
     chunk tensors) and replayed once give the eager outputs bit for bit, and
     a second replay after a reset gives them again."""
-    p = make_problem(batch=1, heads=2, T=10, Hs=6, Ws=11, D=128, Dp=128, Tc=2, To=1,
+    p = make_problem(batch=1, heads=2, T=10, Hs=Hs, Ws=Ws, D=128, Dp=128, Tc=2, To=1,
                      causal=True, dtype="bf16", seed=43)
     y_eager, st = _stream_outputs(p)
     dev = device_tensors(p)
@@ -273,11 +303,12 @@ def test_streaming_sequence_graph_matches_eager():
         assert torch.equal(out, y_eager[:, :, -rows:])
 
 
-def test_streaming_checkpoint_resume_bit_exact():
-    p = make_problem(batch=1, heads=2, T=9, Hs=6, Ws=11, D=128, Dp=128, Tc=2, To=1,
+@pytest.mark.parametrize("Hs,Ws", [(6, 11), (16, 20)])
+def test_streaming_checkpoint_resume_bit_exact(Hs, Ws):
+    p = make_problem(batch=1, heads=2, T=9, Hs=Hs, Ws=Ws, D=128, Dp=128, Tc=2, To=1,
                      causal=True, dtype="bf16", seed=41)
     dev = device_tensors(p)
-    mk = lambda: rh.StreamingState(batch=1, heads=2, Hs=6, Ws=11, D=128, Dp=128, Tc=2, To=1,
+    mk = lambda: rh.StreamingState(batch=1, heads=2, Hs=Hs, Ws=Ws, D=128, Dp=128, Tc=2, To=1,
                                    Wq=dev["Wq"], bq=dev["bq"], Wk=dev["Wk"], bk=dev["bk"],
                                    in_dtype=torch.bfloat16)
     HW = p.HW
