@@ -908,26 +908,32 @@ def run_gpu(args, world, rank, local):
         # GPU of the job longer.
         want = set()
     if "full_softmax" in want:
-        extra["full_softmax"] = measure_full_softmax(rh, q, k, v, y, flush, stream)
+        with torch.cuda.nvtx.range("full_softmax"):
+            extra["full_softmax"] = measure_full_softmax(rh, q, k, v, y, flush, stream)
     del y, ws
     torch.cuda.empty_cache()
     if "fp8_qk" in want:
-        extra["fp8_qk"] = measure_fp8_qk(rh, p, q, k, v, phi, flush, stream)
+        with torch.cuda.nvtx.range("fp8_qk"):
+            extra["fp8_qk"] = measure_fp8_qk(rh, p, q, k, v, phi, flush, stream)
         torch.cuda.empty_cache()
     if "phi_backward" in want:
-        extra["phi_backward"] = measure_phi_backward(rh, p, q, k, v, Wq, bq, Wk, bk, flush,
-                                                     stream)
+        with torch.cuda.nvtx.range("phi_backward"):
+            extra["phi_backward"] = measure_phi_backward(rh, p, q, k, v, Wq, bq, Wk, bk, flush,
+                                                         stream)
         torch.cuda.empty_cache()
     if "full_backward" in want:
-        extra["full_backward"] = measure_full_backward(rh, p, q, k, v, Wq, bq, Wk, bk, flush,
-                                                       stream)
+        with torch.cuda.nvtx.range("full_backward"):
+            extra["full_backward"] = measure_full_backward(rh, p, q, k, v, Wq, bq, Wk, bk,
+                                                           flush, stream)
         torch.cuda.empty_cache()
     if "general_phi" in want:
-        extra["general_phi"] = measure_general_phi(rh, p, q, k, v, flush, stream)
+        with torch.cuda.nvtx.range("general_phi"):
+            extra["general_phi"] = measure_general_phi(rh, p, q, k, v, flush, stream)
     del q, k, v
     torch.cuda.empty_cache()
     if "streaming" in want:
-        extra["streaming"] = measure_streaming(rh, dev, flush, stream)
+        with torch.cuda.nvtx.range("streaming"):
+            extra["streaming"] = measure_streaming(rh, dev, flush, stream)
 
     if rank != 0:
         if dist:
