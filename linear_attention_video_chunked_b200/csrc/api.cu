@@ -89,6 +89,32 @@ bool tc_state_path(const rehyat_params* p) {
          tc_state_eligible(p->in_dtype == REHYAT_BF16, p->D, p->Dp);
 }
 
+// Whether the feature-map backward's q and k passes run on tensor cores.
+bool phi_bwd_on_tc(const rehyat_params* p) {
+  return tc_path(p) && tc_phi_bwd_eligible(p->in_dtype == REHYAT_BF16, p->D, p->Dp);
+}
+
+// Feature-map backward workspace: the forward's layout, then the q and k
+// passes' partials ...
+size_t phi_bwd_base_bytes(const rehyat_params* p) {
+  if (check_params(p) != REHYAT_OK || no_fp8(p) != REHYAT_OK) return 0;
+  int QS, KS;
+  phi_bwd_split(p->T, p->Tc, p->Hs * p->Ws, &QS, &KS);
+  const size_t parts = phi_bwd_partial_floats(p->batch * p->heads, p->T, nchunks_of(p), p->D,
+                                              p->Dp, QS, KS);
+  return fwd_layout(p).total + align_up(parts * sizeof(float));
+}
+
+// ... and, for the tensor-core passes' shapes (bf16, D = D' = 128), r and
+// bf16 g / den per row for the q pass.
+size_t phi_bwd_prep_bytes(const rehyat_params* p) {
+  if ((p->flags & REHYAT_FLAG_FORCE_SIMT) || p->in_dtype != REHYAT_BF16 || p->D != 128 ||
+      p->Dp != 128)
+    return 0;
+  const size_t rows = static_cast<size_t>(p->batch) * p->heads * p->T * p->Hs * p->Ws;
+  return align_up(rows * sizeof(float)) + align_up(rows * p->D * 2);
+}
+
 // Per-slice states on the path these params select.
 cudaError_t run_partials(const rehyat_params* p, const PartialParams& pp, const void* wk_img,
                          cudaStream_t s) {
@@ -563,12 +589,8 @@ rehyat_status rehyat_feature_map_mlp(const rehyat_params* p, const void* x,
 }
 
 size_t rehyat_phi_bwd_workspace_bytes(const rehyat_params* p) {
-  if (check_params(p) != REHYAT_OK || no_fp8(p) != REHYAT_OK) return 0;
-  int QS, KS;
-  phi_bwd_split(p->T, p->Tc, p->Hs * p->Ws, &QS, &KS);
-  const size_t parts = phi_bwd_partial_floats(p->batch * p->heads, p->T, nchunks_of(p), p->D,
-                                              p->Dp, QS, KS);
-  return fwd_layout(p).total + align_up(parts * sizeof(float));
+  const size_t b = rehyat::phi_bwd_base_bytes(p);
+  return b == 0 ? 0 : b + rehyat::phi_bwd_prep_bytes(p);
 }
 
 }  // extern "C"
@@ -577,12 +599,16 @@ namespace rehyat {
 namespace {
 
 // The feature-map backward; with dq, dk, dv non-null and the tensor-core
-// passes in use, it also adds the linear branch's token gradients to them.
+// passes in use, it also writes the linear branch's token gradients to them.
+// The tensor-core q pass reads r and bf16 g / den per row: r_pre, gh_pre
+// when the caller has them (the full backward), else computed into the
+// workspace after the base region.
 rehyat_status phi_bwd_impl(const rehyat_params* p, const void* q, const void* k, const void* v,
                            const float* y, const float* dy, const float* den,
                            const rehyat_phi* phi, const rehyat_phi_grad* grad, void* workspace,
                            size_t ws_bytes, void* stream, float* dq, float* dk, float* dv,
-                           bool* added) {
+                           bool* added, const float* r_pre = nullptr,
+                           const void* gh_pre = nullptr) {
   rehyat_status st = check_params(p);
   if (st != REHYAT_OK) return st;
   if ((st = no_fp8(p)) != REHYAT_OK) return st;
@@ -594,7 +620,9 @@ rehyat_status phi_bwd_impl(const rehyat_params* p, const void* q, const void* k,
       (reinterpret_cast<uintptr_t>(grad->dWq) & 3) || (reinterpret_cast<uintptr_t>(grad->dbq) & 3) ||
       (reinterpret_cast<uintptr_t>(grad->dWk) & 3) || (reinterpret_cast<uintptr_t>(grad->dbk) & 3))
     return REHYAT_ERR_MISALIGNED;
-  if (ws_bytes < rehyat_phi_bwd_workspace_bytes(p)) return REHYAT_ERR_WORKSPACE;
+  const size_t base = phi_bwd_base_bytes(p);
+  const bool have_prep = r_pre != nullptr && gh_pre != nullptr;
+  if (ws_bytes < base + (have_prep ? 0 : phi_bwd_prep_bytes(p))) return REHYAT_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
   // The linear-set state of every chunk, as the forward computes it.
@@ -611,12 +639,23 @@ rehyat_status phi_bwd_impl(const rehyat_params* p, const void* q, const void* k,
   a.Dp = p->Dp; a.Tc = p->Tc; a.To = p->To; a.causal = p->causal; a.nchunks = nchunks_of(p);
   a.in_bf16 = p->in_dtype == REHYAT_BF16;
   // Tensor-core q and k passes where the weight images exist (bf16, D = D' = 128).
-  a.tc = tc_path(p) && tc_phi_bwd_eligible(a.in_bf16, p->D, p->Dp);
+  a.tc = phi_bwd_on_tc(p);
   a.wq_img = a.tc ? ws + w.wimg_off : nullptr;
   a.wk_img = a.tc ? ws + w.wkimg_off : nullptr;
   a.dq = a.tc ? dq : nullptr;
   a.dk = a.tc ? dk : nullptr;
   a.dv = a.tc ? dv : nullptr;
+  a.r = r_pre;
+  a.gh = gh_pre;
+  if (a.tc && !have_prep) {
+    const long long rows = static_cast<long long>(p->batch) * p->heads * p->T * p->Hs * p->Ws;
+    float* r = reinterpret_cast<float*>(ws + base);
+    void* gh = ws + base + align_up(static_cast<size_t>(rows) * sizeof(float));
+    const cudaError_t e = launch_bwd_prep(y, dy, den, r, gh, rows, s);
+    if (e != cudaSuccess) return to_status(e);
+    a.r = r;
+    a.gh = gh;
+  }
   if (added) *added = a.tc && dq != nullptr;
   return to_status(launch_phi_bwd(a, s));
 }
@@ -635,7 +674,7 @@ rehyat_status rehyat_phi_bwd(const rehyat_params* p, const void* q, const void* 
 }
 
 size_t rehyat_hybrid_attn_bwd_workspace_bytes(const rehyat_params* p) {
-  const size_t phi_ws = rehyat_phi_bwd_workspace_bytes(p);
+  const size_t phi_ws = rehyat::phi_bwd_base_bytes(p);
   if (phi_ws == 0) return 0;
   const size_t rows = static_cast<size_t>(p->batch) * p->heads * p->T * p->Hs * p->Ws;
   // Shapes the tensor-core path takes (bf16, D = 128): a bf16 copy of dy / den.
@@ -669,7 +708,7 @@ rehyat_status rehyat_hybrid_attn_bwd(const rehyat_params* p, const void* q, cons
   phi_bwd_split(p->T, p->Tc, HW, &QS, &KS);
   const float* partials = reinterpret_cast<const float*>(ws + w.total);
   const size_t rows = static_cast<size_t>(BH) * p->T * HW;
-  char* scratch = ws + rehyat_phi_bwd_workspace_bytes(p);
+  char* scratch = ws + phi_bwd_base_bytes(p);
   AttnBwdParams a;
   a.q = q; a.k = k; a.v = v; a.y = y; a.dy = dy; a.c = c; a.den = den;
   a.Wq = phi->Wq; a.bq = phi->bq; a.Wk = phi->Wk; a.bk = phi->bk;
@@ -686,18 +725,30 @@ rehyat_status rehyat_hybrid_attn_bwd(const rehyat_params* p, const void* q, cons
   a.FP = p->Dp > 128 ? p->Dp / 128 : 1;
   a.scale = p->scale > 0.f ? p->scale : 1.0f / sqrtf(static_cast<float>(p->D));
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const size_t phi_ws = rehyat_phi_bwd_workspace_bytes(p);
+  const size_t phi_ws = phi_bwd_base_bytes(p);
   if (!(p->flags & REHYAT_FLAG_FORCE_SIMT) && tc_attn_bwd_eligible(a.in_bf16, p->D)) {
-    // Softmax branch on tensor cores (writes dq, dk, dv), then the
-    // feature-map backward, whose tensor-core passes add the linear branch's
-    // token gradients; otherwise those come from CUDA-core kernels after it.
-    cudaError_t e = launch_attn_bwd_tc_softmax(a, scratch + 3 * align_up(rows * sizeof(float)), s);
+    // Softmax branch on tensor cores.  Where the feature-map passes run on
+    // tensor cores too they go first and write the linear branch's token
+    // gradients to dq, dk, dv (one plain store per element), and the softmax
+    // kernels add theirs in their epilogues; otherwise the softmax kernels
+    // write and CUDA-core kernels add the linear parts after the
+    // feature-map backward.  All read the same r and bf16 dy / den rows.
+    void* gh = scratch + 3 * align_up(rows * sizeof(float));
+    cudaError_t e = launch_bwd_prep(y, dy, den, a.r, gh, static_cast<long long>(rows), s);
     if (e != cudaSuccess) return to_status(e);
-    bool added = false;
-    if ((st = phi_bwd_impl(p, q, k, v, y, dy, den, phi, grad, workspace, phi_ws, stream, dq, dk,
-                           dv, &added)) != REHYAT_OK)
+    if (phi_bwd_on_tc(p)) {
+      bool added = false;
+      if ((st = phi_bwd_impl(p, q, k, v, y, dy, den, phi, grad, workspace, phi_ws, stream, dq,
+                             dk, dv, &added, a.r, gh)) != REHYAT_OK)
+        return st;
+      if (!added) return REHYAT_ERR_CUDA;
+      return to_status(launch_attn_bwd_tc_kernels(a, gh, true, s));
+    }
+    if ((e = launch_attn_bwd_tc_kernels(a, gh, false, s)) != cudaSuccess) return to_status(e);
+    if ((st = phi_bwd_impl(p, q, k, v, y, dy, den, phi, grad, workspace, phi_ws, stream, nullptr,
+                           nullptr, nullptr, nullptr, a.r, gh)) != REHYAT_OK)
       return st;
-    return added ? REHYAT_OK : to_status(launch_attn_bwd_lin_simt(a, s));
+    return to_status(launch_attn_bwd_lin_simt(a, s));
   }
   // CUDA cores: the feature-map backward first (S_L, z_L and the Ghat blocks
   // the token gradients use), then dq and dk/dv with the linear parts fused.

@@ -543,21 +543,33 @@ cudaError_t launch_bwd_simt_d(const AttnBwdParams& p, cudaStream_t s) {
 
 }  // namespace
 
-cudaError_t launch_attn_bwd_tc_softmax(const AttnBwdParams& p, void* gh_bf16, cudaStream_t s) {
-  const long long N = static_cast<long long>(p.T) * p.HW;
-  const long long rows = N * p.BH;
+cudaError_t launch_bwd_prep(const float* y, const float* dy, const float* den, float* r,
+                            void* gh_bf16, long long rows, cudaStream_t s) {
   bwd_prep_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, s>>>(
-      p.y, p.dy, p.den, p.r, static_cast<uint2*>(gh_bf16), rows);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+      y, dy, den, r, static_cast<uint2*>(gh_bf16), rows);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_bwd_tc_kernels(const AttnBwdParams& p, const void* gh_bf16,
+                                       bool accumulate, cudaStream_t s) {
   AttnBwdTcArgs a;
   a.q = p.q; a.k = p.k; a.v = p.v; a.gh = gh_bf16;
   a.c = p.c; a.r = p.r; a.Dc = p.Dc; a.jstar = p.jstar;
   a.dq = p.dq; a.dk = p.dk; a.dv = p.dv;
   a.BH = p.BH; a.T = p.T; a.HW = p.HW; a.Tc = p.Tc; a.To = p.To; a.nchunks = p.nchunks;
+  a.accumulate = accumulate ? 1 : 0;
   a.scale = p.scale;
-  if ((e = launch_attn_bwd_dq_tc(a, s)) != cudaSuccess) return e;
+  cudaError_t e = launch_attn_bwd_dq_tc(a, s);
+  if (e != cudaSuccess) return e;
   return launch_attn_bwd_dkv_tc(a, s);
+}
+
+cudaError_t launch_attn_bwd_tc_softmax(const AttnBwdParams& p, void* gh_bf16, bool accumulate,
+                                       cudaStream_t s) {
+  const long long rows = static_cast<long long>(p.T) * p.HW * p.BH;
+  const cudaError_t e = launch_bwd_prep(p.y, p.dy, p.den, p.r, gh_bf16, rows, s);
+  if (e != cudaSuccess) return e;
+  return launch_attn_bwd_tc_kernels(p, gh_bf16, accumulate, s);
 }
 
 cudaError_t launch_attn_bwd_lin_simt(const AttnBwdParams& p, cudaStream_t s) {

@@ -91,9 +91,14 @@ struct PhiBwdArgs {
   const void *wq_img, *wk_img;  // bf16 weight images (tensor-core passes) or nullptr
   float *partials;
   float *dWq, *dbq, *dWk, *dbk;
-  // Tensor-core passes only: the linear branch's token gradients are added
-  // into dq, dk, dv when non-null (the full backward).
+  // Tensor-core passes only: the linear branch's token gradients are
+  // written to dq, dk, dv when non-null (the full backward, which then adds
+  // the softmax branch's).
   float *dq, *dk, *dv;
+  // Tensor-core passes only: r = g . y / den per row and gh = bf16(g / den)
+  // [BH][N][D], as bwd_prep_kernel writes them.
+  const float* r;
+  const void* gh;
   int batch, heads, T, HW, D, Dp, Tc, To, causal, nchunks, in_bf16;
   int tc;                       // run the q and k passes on tcgen05
 };
@@ -101,15 +106,16 @@ struct PhiBwdArgs {
 // inputs, D = D' = 128), writing the CUDA-core passes' partial layout.
 struct PhiBwdTcArgs {
   const void *x, *v;          // q or k (the pass's rows), and v (k pass), bf16 [BH][N][128]
-  const float *dy, *y, *den;  // q pass: dL/dy, y, n^S + n^L
+  const void* gh;             // q pass: bf16 g / den [BH][N][128] (bwd_prep_kernel)
+  const float* r;             // q pass: g . y / den per row [BH][N] (bwd_prep_kernel)
   const void* w_img;          // bf16 image of W_q or W_k, [heads][Dp * D]
   const float* b;             // b_q or b_k [heads][Dp]
-  const float* M;             // q: S_L per chunk (image layout); k: Ghat blocks per slice
+  const float* M;             // q: S_L per chunk (image layout); k: Ghat^T blocks per slice
   const float* vec;           // q: z_L per chunk (k: hhat, inside the Ghat block)
-  float* part;                // partial blocks of the pass
-  // Optional token gradients of the linear branch, added in place (fp32
-  // [BH][N][128]; null = not computed): q pass dx = dq (du_q W_q); k pass
-  // dx = dk (du_k W_k) and dv += Ghat_s^T phi_k(k).
+  float* part;                // partial blocks of the pass (the q pass's G blocks as [d][f])
+  // Optional token gradients of the linear branch, written (fp32
+  // [BH][N][128]; null = not computed): q pass dx = dq = du_q W_q; k pass
+  // dx = dk = du_k W_k and dv = phi_k(k) Ghat_s.
   float *dx, *dv;
   int BH, heads, T, HW, Tc, nchunks, splits, q_side;
 };
@@ -152,13 +158,23 @@ struct AttnBwdTcArgs {
   const float *c, *r;          // per query [BH][N]: stabiliser, (g . y) / den
   float* Dc;                   // per query: written by the dq kernel, read by dk/dv
   int* jstar;                  // per query: arg-max key (absolute row), likewise
-  float *dq, *dk, *dv;         // fp32 [BH][N][128], overwritten
+  float *dq, *dk, *dv;         // fp32 [BH][N][128]: overwritten, or added to if accumulate
   int BH, T, HW, Tc, To, nchunks;
+  int accumulate;
   float scale;
 };
 cudaError_t launch_attn_bwd_dq_tc(const AttnBwdTcArgs& a, cudaStream_t s);
 cudaError_t launch_attn_bwd_dkv_tc(const AttnBwdTcArgs& a, cudaStream_t s);
-cudaError_t launch_attn_bwd_tc_softmax(const AttnBwdParams& p, void* gh_bf16, cudaStream_t s);
+// prep, then the dq and dk/dv kernels; with accumulate they add into dq,
+// dk, dv (which then hold the linear branch's parts already).
+cudaError_t launch_attn_bwd_tc_softmax(const AttnBwdParams& p, void* gh_bf16, bool accumulate,
+                                       cudaStream_t s);
+// The dq and dk/dv kernels alone, after launch_bwd_prep.
+cudaError_t launch_attn_bwd_tc_kernels(const AttnBwdParams& p, const void* gh_bf16,
+                                       bool accumulate, cudaStream_t s);
+// r = dy . y / den per row and gh = bf16(dy / den) for D = 128 rows.
+cudaError_t launch_bwd_prep(const float* y, const float* dy, const float* den, float* r,
+                            void* gh_bf16, long long rows, cudaStream_t s);
 // The linear branch's token gradients on CUDA cores, added to dq, dk, dv
 // (D = 128; used when the feature-map passes do not run on tensor cores).
 cudaError_t launch_attn_bwd_lin_simt(const AttnBwdParams& p, cudaStream_t s);

@@ -453,7 +453,7 @@ cudaError_t launch_phi_bwd(const PhiBwdArgs& a, cudaStream_t s) {
     PhiBwdTcArgs t = {};
     t.BH = bp.BH; t.heads = bp.heads; t.T = bp.T; t.HW = bp.HW; t.Tc = bp.Tc;
     t.nchunks = bp.nchunks;
-    t.x = a.q; t.dy = a.dy; t.y = a.y; t.den = a.den; t.w_img = a.wq_img; t.b = a.bq;
+    t.x = a.q; t.gh = a.gh; t.r = a.r; t.w_img = a.wq_img; t.b = a.bq;
     t.M = a.SL; t.vec = a.zL; t.part = bp.qpart; t.splits = bp.QS; t.q_side = 1;
     t.dx = a.dq; t.dv = nullptr;
     cudaError_t e = launch_phi_bwd_tc(t, s);

@@ -312,6 +312,13 @@ __global__ void __launch_bounds__(bq::kThreads, 1)
             v4.y = A.scale * (__uint_as_float(o[i + 1]) - Dc * k1v);
             v4.z = A.scale * (__uint_as_float(o[i + 2]) - Dc * k2v);
             v4.w = A.scale * (__uint_as_float(o[i + 3]) - Dc * k3v);
+            if (A.accumulate) {  // dq already holds the linear branch's part
+              const float4 p4 = *reinterpret_cast<const float4*>(dst + i);
+              v4.x += p4.x;
+              v4.y += p4.y;
+              v4.z += p4.z;
+              v4.w += p4.w;
+            }
             *reinterpret_cast<float4*>(dst + i) = v4;
           }
         }
@@ -641,12 +648,19 @@ __global__ void __launch_bounds__(bk::kThreads, 1)
           float* dk = A.dk + (base_row + key) * 128 + 64 * hf + 32 * c;
 #pragma unroll
           for (int i2 = 0; i2 < 32; i2 += 4) {
-            *reinterpret_cast<float4*>(dv + i2) =
-                make_float4(__uint_as_float(ov[i2]), __uint_as_float(ov[i2 + 1]),
-                            __uint_as_float(ov[i2 + 2]), __uint_as_float(ov[i2 + 3]));
-            *reinterpret_cast<float4*>(dk + i2) = make_float4(
+            float4 v4 = make_float4(__uint_as_float(ov[i2]), __uint_as_float(ov[i2 + 1]),
+                                    __uint_as_float(ov[i2 + 2]), __uint_as_float(ov[i2 + 3]));
+            float4 k4 = make_float4(
                 A.scale * __uint_as_float(ok2[i2]), A.scale * __uint_as_float(ok2[i2 + 1]),
                 A.scale * __uint_as_float(ok2[i2 + 2]), A.scale * __uint_as_float(ok2[i2 + 3]));
+            if (A.accumulate) {  // dk, dv already hold the linear branch's parts
+              const float4 pv = *reinterpret_cast<const float4*>(dv + i2);
+              const float4 pk = *reinterpret_cast<const float4*>(dk + i2);
+              v4.x += pv.x; v4.y += pv.y; v4.z += pv.z; v4.w += pv.w;
+              k4.x += pk.x; k4.y += pk.y; k4.z += pk.z; k4.w += pk.w;
+            }
+            *reinterpret_cast<float4*>(dv + i2) = v4;
+            *reinterpret_cast<float4*>(dk + i2) = k4;
           }
         }
       }
