@@ -264,10 +264,51 @@ __global__ void phi_bwd_gsel_kernel(BwdParams P) {
   P.ghat[(static_cast<long long>(blockIdx.z) * P.T + s) * n + e] = acc;
 }
 
-// Ghat pass (both steps).
+// Both steps in one launch when a (b, h) has at most kGhatChunks chunks: a
+// block takes 32 consecutive elements; its threads first form G_t of every
+// chunk for them (the sum of the QS partials, in order) in shared memory,
+// then Ghat_s of every slice (chunks in order).  The same sums in the same
+// order as (a) and (b), with each partial read once.
+constexpr int kGhatChunks = 64;
+__global__ void __launch_bounds__(256) phi_bwd_ghat_fused_kernel(BwdParams P) {
+  __shared__ float G[kGhatChunks][32];
+  const int D = P.D;
+  const long long n = static_cast<long long>(kPiece) * D + kPiece;
+  const long long e0 = static_cast<long long>(blockIdx.x) * 32;
+  const long long psz = qpart_size(D);
+  const float* g = P.qpart + static_cast<long long>(blockIdx.z) * P.nchunks * P.QS * psz +
+                   static_cast<long long>(D) * kPiece + kPiece + e0;
+  for (int idx = threadIdx.x; idx < P.nchunks * 32; idx += blockDim.x) {
+    const int t = idx >> 5, j = idx & 31;
+    float acc = 0.f;
+    if (e0 + j < n)
+      for (int qs = 0; qs < P.QS; ++qs) acc += g[(static_cast<long long>(t) * P.QS + qs) * psz + j];
+    G[t][j] = acc;
+  }
+  __syncthreads();
+  float* out = P.ghat + static_cast<long long>(blockIdx.z) * P.T * n + e0;
+  for (int idx = threadIdx.x; idx < P.T * 32; idx += blockDim.x) {
+    const int s = idx >> 5, j = idx & 31;
+    if (e0 + j >= n) continue;
+    float acc = 0.f;
+    for (int t = 0; t < P.nchunks; ++t) {
+      const int first = t * P.Tc, end = min(P.T, first + P.Tc);
+      const int w = max(first - P.To, 0);
+      if (P.causal ? s < w : (s < w || s >= end)) acc += G[t][j];
+    }
+    out[static_cast<long long>(s) * n + j] = acc;
+  }
+}
+
+// Ghat pass.
 void launch_ghat(const BwdParams& bp, cudaStream_t s) {
   const long long ng = static_cast<long long>(kPiece) * bp.D + kPiece;
   const unsigned gx = static_cast<unsigned>((ng + 255) / 256);
+  if (bp.nchunks <= kGhatChunks) {
+    const unsigned gb = static_cast<unsigned>((ng + 31) / 32);
+    phi_bwd_ghat_fused_kernel<<<dim3(gb, 1, bp.BH * bp.FP), 256, 0, s>>>(bp);
+    return;
+  }
   phi_bwd_gsum_kernel<<<dim3(gx, bp.nchunks, bp.BH * bp.FP), 256, 0, s>>>(bp);
   phi_bwd_gsel_kernel<<<dim3(gx, bp.T, bp.BH * bp.FP), 256, 0, s>>>(bp);
 }

@@ -56,7 +56,7 @@ constexpr uint32_t kRsOff = kVecOff + 1024;   // r of the tile's rows, two tiles
 constexpr uint32_t kRedOff = kRsOff + 1024;   // [2 halves][2][128] floats
 constexpr uint32_t kBarOff = kRedOff + 2048;
 enum { W_FULL = 0, M_READY = 1, X_FULL = 2, X_FREE = 4, UT_FULL = 6, DU_READY = 7,
-       TILE_DONE = 8, DX_FREE = 9, RS_READY = 10, NBAR = 11 };
+       TILE_DONE = 8, DX_FREE = 9, RS_READY = 10, M_LOAD = 11, NBAR = 12 };
 constexpr uint32_t kSmemBytes = kBarOff + 128 + 1024;
 constexpr uint32_t kColU = 0, kColT = 128, kColW = 256, kColG = 384;
 
@@ -143,9 +143,11 @@ __global__ void __launch_bounds__(pb::kThreads, 1)
     // ================================================= TMA producer
     if (lane == 0) {
       bool ok = true;
-      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(Msrc),
-                   "r"(static_cast<uint32_t>(kQ ? Dp * D * 4 : (128 * D + 128) * 4))
-                   : "memory");
+      // M in fp32 (64 KB, contiguous) into the second stage's space, where
+      // the converters turn it into the bf16 operand before that stage's
+      // first tile loads.
+      mbar_expect_tx(bar(pb::M_LOAD), Dp * D * 4);
+      bulk_load(base + pb::kStage1, Msrc, Dp * D * 4, bar(pb::M_LOAD));
       mbar_expect_tx(bar(pb::W_FULL), Dp * D * 2);
       bulk_load(base + pb::kWOff,
                 static_cast<const uint8_t*>(a.w_img) + static_cast<long long>(h) * Dp * D * 2,
@@ -153,6 +155,8 @@ __global__ void __launch_bounds__(pb::kThreads, 1)
       for (int tl = 0; tl < ntiles && ok; ++tl) {
         const int st = nstage == 2 ? (tl & 1) : 0;
         if (tl >= nstage) ok = mbar_wait(bar(pb::X_FREE + st), ((tl - nstage) / nstage) & 1, abort_flag, 50);
+        // The second stage's first tile waits for the fp32 M to be converted.
+        if (ok && nstage == 2 && tl == 1) ok = mbar_wait(bar(pb::M_READY), 0, abort_flag, 48);
         if (!ok) break;
         const int row = static_cast<int>(r0 + 128LL * tl);
         const uint32_t sb = stage_base(tl);
@@ -239,19 +243,21 @@ __global__ void __launch_bounds__(pb::kThreads, 1)
     };
     bool ok = true;
     // Once per CTA: b, the vector (z_L or hhat), and M as a bf16 [f][d]
-    // tile; thread (f, hf) converts dimensions [64 hf, 64 hf + 64) of
-    // feature f (both sources keep consecutive features contiguous for a
-    // fixed d, so a warp's loads are 128-byte segments).
+    // tile from its fp32 copy in shared memory; thread (f, hf) converts
+    // dimensions [64 hf, 64 hf + 64) of feature f (both sources keep
+    // consecutive features contiguous for a fixed d: no bank conflicts).
     if (hf == 0) {
       bvec[f] = __ldg(a.b + static_cast<long long>(h) * Dp + f);
       bvec[128 + f] = __ldg(vsrc + f);
     }
-#pragma unroll 4
-    for (int d0 = 64 * hf; d0 < 64 * hf + 64; d0 += 8) {
+    ok = wait_all(bar(pb::M_LOAD), 0, 47);
+    const float* Ms = reinterpret_cast<const float*>(sbase + pb::kStage1);
+#pragma unroll 2
+    for (int d0 = 64 * hf; d0 < 64 * hf + 64 && ok; d0 += 8) {
       float m[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i)
-        m[i] = kQ ? __ldg(Msrc + sl_index(f, d0 + i, D, Dp)) : __ldg(Msrc + (d0 + i) * 128 + f);
+        m[i] = kQ ? Ms[sl_index(f, d0 + i, D, Dp)] : Ms[(d0 + i) * 128 + f];
       st_shared_v4(base + pb::kMOff + tile_off(f, d0), pack_bf16(m[0], m[1]), pack_bf16(m[2], m[3]),
                    pack_bf16(m[4], m[5]), pack_bf16(m[6], m[7]));
     }
