@@ -728,6 +728,15 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
         tma_load_3d(base + a2::kQ8Off, &maps.q8, bar(a2::Q_FULL), 0, row0, bh);
         tma_load_3d(base + a2::kQ8Off + 16384, &maps.q8, bar(a2::Q_FULL), 0, row0 + kBM, bh);
       }
+      if (linear && phi_given) {
+        // The tail reads both tiles' rows of phi_q(q) (contiguous): into L2
+        // now, so those loads do not wait on DRAM at the end of the CTA.
+        const uint32_t bytes = static_cast<uint32_t>(nrows_t[0] + nrows_t[1]) * Dp * 4;
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(
+                         P.phi_q + (static_cast<long long>(bh) * P.rows_per_bh + row0) * Dp),
+                     "r"(bytes)
+                     : "memory");
+      }
       for (int j = 0; j < nt && ok; ++j) {
         const TileSrc src = tile_src(j);
         const int ks = j % 3;
@@ -1175,21 +1184,42 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         const int f0 = pc * pw;
-        const float* given = phi_given && r < nrows ? P.phi_q + grow * Dp + f0 : nullptr;
         const float* zsrc = P.zL + (static_cast<long long>(bh) * P.nchunks + t) * Dp + f0;
-        for (int c = 0; c < pw / 32; ++c) {
-          float ph[32];
-          if (phi_given) {
+        if (phi_given) {
+          // Each warp stages its 32 rows' phi_q(q) four rows per load
+          // instruction (eight lanes read a row's 32-feature chunk, 128
+          // contiguous bytes): row-per-thread fp32 loads would thrash the
+          // small L1 beside this kernel's shared memory.  The row's thread
+          // keeps its n^L (the eight lanes' parts summed, then passed on).
+          const int q4 = lane & 7, rsub = lane >> 3;
+          const long long gtile = static_cast<long long>(bh) * P.rows_per_bh + row0 + tile * kBM;
+          for (int c = 0; c < pw / 32; ++c) {
+            const int col = c * 32 + 4 * q4;
+            float z4[4];
 #pragma unroll
-            for (int i = 0; i < 32; i += 4) {
-              const float4 g4 = given ? __ldg(reinterpret_cast<const float4*>(given + c * 32 + i))
-                                      : make_float4(0.f, 0.f, 0.f, 0.f);
-              ph[i] = g4.x;
-              ph[i + 1] = g4.y;
-              ph[i + 2] = g4.z;
-              ph[i + 3] = g4.w;
+            for (int e = 0; e < 4; ++e)
+              z4[e] = npieces == 1 ? vec[Dp + col + e] : __ldg(zsrc + col + e);
+#pragma unroll 4
+            for (int it = 0; it < 8; ++it) {
+              const int rr = 32 * (warp & 3) + 4 * it + rsub;  // row within the tile
+              const float inv_r = __shfl_sync(0xffffffffu, inv_f, 4 * it + rsub);
+              float4 g4 = make_float4(0.f, 0.f, 0.f, 0.f);
+              if (rr < nrows)
+                g4 = __ldg(reinterpret_cast<const float4*>(P.phi_q + (gtile + rr) * Dp + f0 + col));
+              float part = g4.x * z4[0] + g4.y * z4[1] + g4.z * z4[2] + g4.w * z4[3];
+              part += __shfl_xor_sync(0xffffffffu, part, 4);
+              part += __shfl_xor_sync(0xffffffffu, part, 2);
+              part += __shfl_xor_sync(0xffffffffu, part, 1);
+              const float mine = __shfl_sync(0xffffffffu, part, 8 * (lane & 3));
+              if ((lane >> 2) == it) nL += mine;
+              st_shared_v4(phi + c * 16384 + rr * 128 + ((q4 ^ (rr & 7)) << 4),
+                           __float_as_uint(g4.x * inv_r), __float_as_uint(g4.y * inv_r),
+                           __float_as_uint(g4.z * inv_r), __float_as_uint(g4.w * inv_r));
             }
-          } else {
+          }
+        } else {
+          for (int c = 0; c < pw / 32; ++c) {
+            float ph[32];
             uint32_t v[32];
             REHYAT_TMEM_LD32(lane_base + s_col + c * 32, v);
             tmem_wait_ld();
@@ -1199,19 +1229,19 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
               const float psi = __uint_as_float(v[i]) + b;
               ph[i] = psi * psi;
             }
-          }
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float z = npieces == 1 ? vec[Dp + c * 32 + i] : __ldg(zsrc + c * 32 + i);
-            nL = fmaf(ph[i], z, nL);
-            ph[i] *= inv_f;
-          }
-          const uint32_t rowaddr = phi + c * 16384 + r * 128;
+            for (int i = 0; i < 32; ++i) {
+              const float z = npieces == 1 ? vec[Dp + c * 32 + i] : __ldg(zsrc + c * 32 + i);
+              nL = fmaf(ph[i], z, nL);
+              ph[i] *= inv_f;
+            }
+            const uint32_t rowaddr = phi + c * 16384 + r * 128;
 #pragma unroll
-          for (int ch = 0; ch < 8; ++ch)
-            st_shared_v4(rowaddr + ((ch ^ (r & 7)) << 4), __float_as_uint(ph[4 * ch]),
-                         __float_as_uint(ph[4 * ch + 1]), __float_as_uint(ph[4 * ch + 2]),
-                         __float_as_uint(ph[4 * ch + 3]));
+            for (int ch = 0; ch < 8; ++ch)
+              st_shared_v4(rowaddr + ((ch ^ (r & 7)) << 4), __float_as_uint(ph[4 * ch]),
+                           __float_as_uint(ph[4 * ch + 1]), __float_as_uint(ph[4 * ch + 2]),
+                           __float_as_uint(ph[4 * ch + 3]));
+          }
         }
         fence_proxy_async();
         tc_fence_before();
@@ -1338,6 +1368,7 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
 // the ring's k, v (streaming; equal to k, v otherwise).
 struct StMaps {
   CUtensorMap k, v, rk, rv;
+  CUtensorMap phik;  // phi_k(k) given: fp32 [BH][N][Dp], boxes of 32 features x 128 rows
 };
 
 namespace sp {
@@ -1356,6 +1387,11 @@ constexpr uint32_t kSmemBytes = kBarOff + 256 + 1024;
 // TMEM: psi^T fp32 [0,128) [128,256), phi^T bf16 pairs [256,320) [320,384)
 // (each alternating per token tile), P accumulator [384,512).
 constexpr uint32_t kColPsi = 0, kColPhi = 256, kColP = 384;
+// phi_k(k) given: the 16 KB box b (32 features x 128 tokens, fp32, token-major)
+// of stage s, in the K ring and the W_k area.
+__host__ __device__ constexpr uint32_t phi_box(int s, int b) {
+  return s == 0 ? kKOff + b * 16384 : (b < 2 ? kKOff + 65536 + b * 16384 : kWOff + (b - 2) * 16384);
+}
 
 // Walk over a CTA's run of items i = q * T + slice, q = bh * halves + half,
 // with a division only when one (bh, half) run of slices ends.
@@ -1461,7 +1497,8 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
   if (tid == 0) {
     for (int i = 0; i < NBAR; ++i) {
       const bool by_group = i == PSI_FREE || i == PSI_FREE + 1 || i == PHI_FULL ||
-                            i == PHI_FULL + 1 || i == P_FREE;
+                            i == PHI_FULL + 1 || i == P_FREE ||
+                            (phi_given && (i == K_EMPTY || i == K_EMPTY + 1));
       mbar_init(bar(i), by_group ? 128 : 1);
     }
     *abort_flag = 0;
@@ -1491,7 +1528,28 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
     // ================================================= TMA producers
     // warp 8 loads K tiles (and the W_k piece), warp 11 V tiles, so K runs
     // ahead on its own ring (psi^T) while V waits for phi^T V to free stages.
-    if (lane == 0 && !(warp == 8 && phi_given)) {  // no K or W_k with phi_k given
+    if (lane == 0 && warp == 8 && phi_given) {
+      // phi_k(k) given: its fp32 tiles (pw features x 128 tokens, boxes of
+      // 32 features) into two stages of the space K and W_k leave unused,
+      // so the converters read them from shared memory.
+      bool ok = true;
+      sp::ItemWalk w{T, halves, P.heads, pw, leave};
+      w.start(it0);
+      int gt = 0;
+      const uint32_t tile_bytes = static_cast<uint32_t>(pw) * 128 * 4;
+      for (int il = 0; il < nitems && ok; ++il, w.next()) {
+        if (!w.on()) continue;
+        for (int j = 0; j < nt && ok; ++j, ++gt) {
+          const int st = gt & 1;
+          if (gt >= 2) ok = mbar_wait(bar(K_EMPTY + st), ((gt - 2) >> 1) & 1, abort_flag, 39);
+          if (!ok) break;
+          mbar_expect_tx(bar(K_FULL + st), tile_bytes);
+          for (int bx = 0; bx < pw / 32; ++bx)
+            tma_load_3d(base + sp::phi_box(st, bx), &maps.phik, bar(K_FULL + st),
+                        w.half() * pw + 32 * bx, w.slice * HW + j * 128, w.bh());
+        }
+      }
+    } else if (lane == 0 && !(warp == 8 && phi_given)) {  // no K or W_k with phi_k given
       const bool kside = warp == 8;
       bool ok = true;
       int wloads = 0, wkey = -1;
@@ -1654,14 +1712,11 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
       }
       const uint64_t b2 = f2_pack(bias, bias);
       // phi_k(k) given: this thread's feature column of the item's rows.
-      const float* given = phi_given && f < pw
-                               ? P.phi_k + (static_cast<long long>(w.bh()) * P.rows_per_bh +
-                                            static_cast<long long>(w.slice) * HW) * Dp +
-                                     w.half() * pw + f
-                               : nullptr;
       for (int j = 0; j < nt && ok; ++j, ++gt) {
         const int b = gt & 1;
-        if (!phi_given) ok = wait_all(bar(PSI_FULL + b), (gt >> 1) & 1, 36);
+        // psi^T of the tile in TMEM buffer b, or (phi_k given) its phi_k
+        // tile in shared-memory stage b.
+        ok = wait_all(bar(phi_given ? K_FULL + b : PSI_FULL + b), (gt >> 1) & 1, 36);
         // phi^T buffer b is free once phi^T V of tile gt - 2 has read it.
         if (ok && gt >= 2) ok = wait_all(bar(PHI_FREE + b), ((gt - 2) >> 1) & 1, 38);
         if (!ok) break;
@@ -1675,12 +1730,14 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
         for (int c = 0; c < 4; ++c) {
           uint32_t ps[32], pk[16];
           if (phi_given) {
+            // Feature f of tokens 32c .. 32c + 31: a column of box f / 32
+            // (token-major rows of 32 floats; a warp reads whole rows).
+            const float* col = reinterpret_cast<const float*>(
+                                   sbase + sp::phi_box(b, f < pw ? f >> 5 : 0)) + (f & 31);
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
               const int t = c * 32 + i;
-              ps[i] = __float_as_uint(given && t < nvalid
-                                          ? __ldg(given + static_cast<long long>(j * 128 + t) * Dp)
-                                          : 0.f);
+              ps[i] = __float_as_uint(f < pw && t < nvalid ? col[t * 32] : 0.f);
             }
           } else {
             REHYAT_TMEM_LD32(cols + c * 32, ps);
@@ -1707,6 +1764,7 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
           }
           REHYAT_TMEM_ST16(pcols + c * 16, pk);
         }
+        if (phi_given) mbar_arrive(bar(K_EMPTY + b));  // the stage's reads are done
         tmem_wait_st();
         if (nvalid < 128) {
           // V rows past the slice are zeroed so that 0 * V stays 0 for any V.
@@ -1822,6 +1880,22 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // 3D 8-bit map over [planes][rows][128] with a 128 x 128 x 1 box (one 128-byte
 // row per token), 128B swizzle.
+// fp32 [planes][rows][cols] with boxes of 32 columns x 128 rows, unswizzled
+// (a box lands as 128 rows of 128 bytes).
+bool make_map_f32(CUtensorMap* m, const float* ptr, long long rows, int planes, int cols) {
+  auto fn = encode_fn();
+  if (!fn || rows <= 0 || cols % 32 != 0) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(planes)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols) * 4,
+                           static_cast<cuuint64_t>(rows) * cols * 4};
+  cuuint32_t box[3] = {32, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_map8(CUtensorMap* m, const void* ptr, long long rows, int planes) {
   auto fn = encode_fn();
   if (!fn || rows <= 0) return false;
@@ -1878,6 +1952,8 @@ cudaError_t launch_state_tc(const PartialParams& p, const void* wk_img, cudaStre
   const int ctas = (total + per_cta - 1) / per_cta;
   const __nv_bfloat16* wk = static_cast<const __nv_bfloat16*>(wk_img);
   if (p.phi_k != nullptr) {  // full forward with phi_k(k) given
+    if (!make_map_f32(&maps.phik, p.phi_k, p.rows_per_bh, p.BH, p.Dp))
+      return cudaErrorInvalidValue;
     const cudaError_t e = ensure_smem(tc_state_persistent_kernel<true>, 3, sp::kSmemBytes);
     if (e != cudaSuccess) return e;
     tc_state_persistent_kernel<true><<<ctas, sp::kThreads, sp::kSmemBytes, s>>>(maps, p, wk,
