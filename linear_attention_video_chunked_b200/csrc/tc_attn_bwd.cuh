@@ -528,23 +528,23 @@ __global__ void __launch_bounds__(bk::kThreads, 1)
     constexpr float kLog2e = 1.4426950408889634f;
     const float sl2 = A.scale * kLog2e;
     const int key = j0 + kr;
-    // Per-query values of pair i in stage i & 1, one 16-byte record per
-    // query (m = c log2(e), r, Dc, j*), so each column costs one broadcast
-    // 16-byte shared load.  Thread t fills two of the record's words
-    // (query t & 127, words 2 (t >> 7), 2 (t >> 7) + 1).
-    float4* vec = reinterpret_cast<float4*>(sbase + kVecOff);  // [stage][128]
+    // Per-query values of pair i in stage i & 1: four arrays of 128 (m =
+    // c log2(e), r, Dc, j*), so four consecutive columns cost one broadcast
+    // 16-byte shared load per array.  Thread t fills two of them for query
+    // t & 127 (m and r, or Dc and j*).
+    float* vec = reinterpret_cast<float*>(sbase + kVecOff);  // [stage][4][128]
     auto load_vec = [&](const QWalk& w, int i) {
       const int qi = tid & 127, which = tid >> 7;
       const int q = w.q0() + qi;
       const bool in = qi < w.qvalid();
-      float* v = reinterpret_cast<float*>(vec + (i & 1) * 128 + qi);
+      float* v = vec + (i & 1) * 512 + qi;
       const long long g = base_row + q;
       if (which == 0) {
         v[0] = in ? __ldg(A.c + g) * kLog2e : 0.f;
-        v[1] = in ? __ldg(A.r + g) : 0.f;
+        v[128] = in ? __ldg(A.r + g) : 0.f;
       } else {
-        v[2] = in ? __ldg(A.Dc + g) : 0.f;
-        v[3] = __int_as_float(in ? __ldg(A.jstar + g) : -1);
+        v[256] = in ? __ldg(A.Dc + g) : 0.f;
+        v[384] = __int_as_float(in ? __ldg(A.jstar + g) : -1);
       }
       mbar_arrive(bar(VEC_FULL + (i & 1)));
     };
@@ -558,7 +558,13 @@ __global__ void __launch_bounds__(bk::kThreads, 1)
       ok = wait_all(bar(ST_FULL), i & 1, 24) && wait_all(bar(VEC_FULL + (i & 1)), (i >> 1) & 1, 25);
       if (!ok) break;
       tc_fence_after();
-      const float4* v = vec + (i & 1) * 128;
+      const float4* vm = reinterpret_cast<const float4*>(vec + (i & 1) * 512);
+      const float4* vr = vm + 32;
+      const float4* vd = vm + 64;
+      const float4* vj = vm + 96;
+      // Every column of every row of the warp counts (the common case): no
+      // per-element masks.
+      const bool all_in = __all_sync(0xffffffffu, key_in) && qv == 128;
       // Phase 1: P^T = exp2(s scale log2(e) - m) of this half's 64 query
       // columns, written over them as bf16 pairs; kept in fp32 for phase 2.
       float pv[64];
@@ -570,11 +576,16 @@ __global__ void __launch_bounds__(bk::kThreads, 1)
           REHYAT_TMEM_LD32(lane_base + kColS + 64 * hf + 32 * c, xs);
           tmem_wait_ld();
 #pragma unroll
-          for (int i2 = 0; i2 < 32; ++i2) {
-            const int qa = 64 * hf + 32 * c + i2;
-            float p = 0.f;
-            if (key_in && qa < qv) p = ex2(fmaf(__uint_as_float(xs[i2]), sl2, -v[qa].x));
-            pv[32 * c + i2] = p;
+          for (int i4 = 0; i4 < 8; ++i4) {
+            const int qa = 64 * hf + 32 * c + 4 * i4;
+            const float4 m4 = vm[qa >> 2];
+            const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int i2 = 4 * i4 + e;
+              const float p = ex2(fmaf(__uint_as_float(xs[i2]), sl2, -mm[e]));
+              pv[32 * c + i2] = (all_in || (key_in && qa + e < qv)) ? p : 0.f;
+            }
           }
 #pragma unroll
           for (int i2 = 0; i2 < 16; ++i2) pp[16 * c + i2] = pack_bf16(pv[32 * c + 2 * i2], pv[32 * c + 2 * i2 + 1]);
@@ -611,14 +622,29 @@ __global__ void __launch_bounds__(bk::kThreads, 1)
           REHYAT_TMEM_LD32(lane_base + kColDP + 64 * hf + 32 * c, xd);
           tmem_wait_ld();
 #pragma unroll
-          for (int i2 = 0; i2 < 32; i2 += 2) {
-            const int qa = 64 * hf + 32 * c + i2;
-            const float4 v0 = v[qa], v1 = v[qa + 1];
-            float d0 = pv[32 * c + i2] * (__uint_as_float(xd[i2]) - v0.y);
-            float d1 = pv[32 * c + i2 + 1] * (__uint_as_float(xd[i2 + 1]) - v1.y);
-            if (__float_as_int(v0.w) == key && key_in && qa < qv) d0 -= v0.z;
-            if (__float_as_int(v1.w) == key && key_in && qa + 1 < qv) d1 -= v1.z;
-            pd[16 * c + i2 / 2] = pack_bf16(d0, d1);
+          for (int i4 = 0; i4 < 8; ++i4) {
+            const int qa = 64 * hf + 32 * c + 4 * i4;
+            const float4 r4 = vr[qa >> 2];
+            const int4 j4 = *reinterpret_cast<const int4*>(vj + (qa >> 2));
+            const float rr[4] = {r4.x, r4.y, r4.z, r4.w};
+            const int jj[4] = {j4.x, j4.y, j4.z, j4.w};
+            float d[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int i2 = 4 * i4 + e;
+              d[e] = pv[32 * c + i2] * (__uint_as_float(xd[i2]) - rr[e]);
+            }
+            // The maximum's term: this key is the arg-max of one of the
+            // four queries (rare; masked queries carry j* = -1).
+            if (jj[0] == key || jj[1] == key || jj[2] == key || jj[3] == key) {
+              const float4 dc4 = vd[qa >> 2];
+              const float dc[4] = {dc4.x, dc4.y, dc4.z, dc4.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                if (jj[e] == key && key_in && qa + e < qv) d[e] -= dc[e];
+            }
+            pd[16 * c + 2 * i4] = pack_bf16(d[0], d[1]);
+            pd[16 * c + 2 * i4 + 1] = pack_bf16(d[2], d[3]);
           }
         }
         REHYAT_TMEM_ST32(lane_base + kColDP + 64 * hf, pd);
