@@ -265,21 +265,21 @@ __global__ void phi_bwd_gsel_kernel(BwdParams P) {
 }
 
 // Both steps in one launch when a (b, h) has at most kGhatChunks chunks: a
-// block takes 32 consecutive elements; its threads first form G_t of every
-// chunk for them (the sum of the QS partials, in order) in shared memory,
-// then Ghat_s of every slice (chunks in order).  The same sums in the same
-// order as (a) and (b), with each partial read once.
-constexpr int kGhatChunks = 64;
+// block takes kGhatCols consecutive elements; its threads first form G_t of
+// every chunk for them (the sum of the QS partials, in order) in shared
+// memory, then Ghat_s of every slice (chunks in order).  The same sums in the
+// same order as (a) and (b), with each partial read once.
+constexpr int kGhatChunks = 48, kGhatCols = 128;
 __global__ void __launch_bounds__(256) phi_bwd_ghat_fused_kernel(BwdParams P) {
-  __shared__ float G[kGhatChunks][32];
+  __shared__ float G[kGhatChunks][kGhatCols];
   const int D = P.D;
   const long long n = static_cast<long long>(kPiece) * D + kPiece;
-  const long long e0 = static_cast<long long>(blockIdx.x) * 32;
+  const long long e0 = static_cast<long long>(blockIdx.x) * kGhatCols;
   const long long psz = qpart_size(D);
   const float* g = P.qpart + static_cast<long long>(blockIdx.z) * P.nchunks * P.QS * psz +
                    static_cast<long long>(D) * kPiece + kPiece + e0;
-  for (int idx = threadIdx.x; idx < P.nchunks * 32; idx += blockDim.x) {
-    const int t = idx >> 5, j = idx & 31;
+  for (int idx = threadIdx.x; idx < P.nchunks * kGhatCols; idx += blockDim.x) {
+    const int t = idx / kGhatCols, j = idx % kGhatCols;
     float acc = 0.f;
     if (e0 + j < n)
       for (int qs = 0; qs < P.QS; ++qs) acc += g[(static_cast<long long>(t) * P.QS + qs) * psz + j];
@@ -287,8 +287,8 @@ __global__ void __launch_bounds__(256) phi_bwd_ghat_fused_kernel(BwdParams P) {
   }
   __syncthreads();
   float* out = P.ghat + static_cast<long long>(blockIdx.z) * P.T * n + e0;
-  for (int idx = threadIdx.x; idx < P.T * 32; idx += blockDim.x) {
-    const int s = idx >> 5, j = idx & 31;
+  for (int idx = threadIdx.x; idx < P.T * kGhatCols; idx += blockDim.x) {
+    const int s = idx / kGhatCols, j = idx % kGhatCols;
     if (e0 + j >= n) continue;
     float acc = 0.f;
     for (int t = 0; t < P.nchunks; ++t) {
@@ -305,7 +305,7 @@ void launch_ghat(const BwdParams& bp, cudaStream_t s) {
   const long long ng = static_cast<long long>(kPiece) * bp.D + kPiece;
   const unsigned gx = static_cast<unsigned>((ng + 255) / 256);
   if (bp.nchunks <= kGhatChunks) {
-    const unsigned gb = static_cast<unsigned>((ng + 31) / 32);
+    const unsigned gb = static_cast<unsigned>((ng + kGhatCols - 1) / kGhatCols);
     phi_bwd_ghat_fused_kernel<<<dim3(gb, 1, bp.BH * bp.FP), 256, 0, s>>>(bp);
     return;
   }

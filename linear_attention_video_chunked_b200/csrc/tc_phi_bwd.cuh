@@ -212,6 +212,9 @@ __global__ void __launch_bounds__(pb::kThreads, 1)
         if (kQ)
           mma8_ts_mn_split(tmem + pb::kColG, tmem + pb::kColT, sdesc(sb + pb::kERel, 16384, 1024),
                            id_kmn, tl > 0 ? 1u : 0u);
+        // The stage's X and E are read by nothing after these: the TMA may
+        // refill it while the token-gradient products below run.
+        mma_commit(bar(pb::X_FREE + st));
         if (with_dx) {
           // dx^T = W^T du^T (A = W read MN-major, B = du^T [f][rows]) into
           // U^T's columns, after the products above have read them.
@@ -228,7 +231,6 @@ __global__ void __launch_bounds__(pb::kThreads, 1)
                        sdesc(base + pb::kPhiOff + kk * 2048, 16384, 1024), id_mn, kk > 0);
           }
         }
-        mma_commit(bar(pb::X_FREE + st));
         mma_commit(bar(pb::TILE_DONE));
       }
     }
