@@ -412,7 +412,8 @@ def measure_full_backward(rh, p, q, k, v, Wq, bq, Wk, bk, flush, stream, calls=3
 def measure_general_phi(rh, p, q, k, v, flush, stream, calls=3):
     """General feature maps on the bench workload: the per-head 2-layer MLP
     (hidden width 3D, P = 2 parts) for q and for k, then the forward with the
-    maps given (rehyat_hybrid_attn_fwd_phi).  Device time per call of each."""
+    maps given (rehyat_hybrid_attn_fwd_phi).  Device time per call of each,
+    with the maps in bf16 (REHYAT_FLAG_PHI_BF16) and in fp32."""
     import torch
     B, H, N, D = q.shape
     dev = q.device
@@ -422,26 +423,10 @@ def measure_general_phi(rh, p, q, k, v, flush, stream, calls=3):
     ba = 0.1 * torch.randn(H, Dh, generator=g, device=dev)
     Wb = 0.5 * torch.randn(H, Dh, Dp, generator=g, device=dev) / Dh ** 0.5
     bb = 0.05 * torch.randn(H, Dp, generator=g, device=dev)
-    params = rh.make_params(batch=B, heads=H, T=p.T, Hs=p.Hs, Ws=p.Ws, D=D, Dp=Dp, Tc=p.Tc,
-                            To=p.To, causal=p.causal, in_dtype=rh.BF16, out_dtype=rh.F32)
     sh = stream.cuda_stream
     mlp = rh.RehyatPhiMlp(Wa.data_ptr(), ba.data_ptr(), Wb.data_ptr(), bb.data_ptr(), Dh, 2)
-    pq = torch.empty(B, H, N, Dp, device=dev)
-    pk = torch.empty(B, H, N, Dp, device=dev)
     y = torch.empty(B, H, N, D, device=dev)
-    ws = torch.empty(rh.rehyat_workspace_bytes(params), dtype=torch.uint8, device=dev)
-    mlp_bytes = rh.rehyat_feature_map_mlp_workspace_bytes(params, mlp, q.data_ptr(), pq.data_ptr())
-    mws = torch.empty(max(mlp_bytes, 16), dtype=torch.uint8, device=dev)
-    tensor_cores = mlp_bytes > 0
-    feat = lambda: (rh.rehyat_feature_map_mlp(params, q.data_ptr(), mlp, pq.data_ptr(),
-                                              mws.data_ptr(), mlp_bytes, sh) or
-                    rh.rehyat_feature_map_mlp(params, k.data_ptr(), mlp, pk.data_ptr(),
-                                              mws.data_ptr(), mlp_bytes, sh))
-    fwd = lambda: rh.rehyat_hybrid_attn_fwd_phi(params, q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                                                pq.data_ptr(), pk.data_ptr(), y.data_ptr(),
-                                                ws.data_ptr(), ws.numel(), None, sh)
-    if feat() or fwd():
-        raise RuntimeError("general feature map path failed")
+    peaks = load_peaks()
 
     def timed(fn):
         times = []
@@ -455,26 +440,55 @@ def measure_general_phi(rh, p, q, k, v, flush, stream, calls=3):
             times.append(e0.elapsed_time(e1))
         return sum(times) / len(times)
 
-    feat_ms, fwd_ms = timed(feat), timed(fwd)
+    def run(phi_dtype):
+        flags = rh.FLAG_PHI_BF16 if phi_dtype == torch.bfloat16 else 0
+        params = rh.make_params(batch=B, heads=H, T=p.T, Hs=p.Hs, Ws=p.Ws, D=D, Dp=Dp, Tc=p.Tc,
+                                To=p.To, causal=p.causal, in_dtype=rh.BF16, out_dtype=rh.F32,
+                                flags=flags)
+        pq = torch.empty(B, H, N, Dp, device=dev, dtype=phi_dtype)
+        pk = torch.empty(B, H, N, Dp, device=dev, dtype=phi_dtype)
+        ws = torch.empty(rh.rehyat_workspace_bytes(params), dtype=torch.uint8, device=dev)
+        mlp_bytes = rh.rehyat_feature_map_mlp_workspace_bytes(params, mlp, q.data_ptr(),
+                                                              pq.data_ptr())
+        mws = torch.empty(max(mlp_bytes, 16), dtype=torch.uint8, device=dev)
+        feat = lambda: (rh.rehyat_feature_map_mlp(params, q.data_ptr(), mlp, pq.data_ptr(),
+                                                  mws.data_ptr(), mlp_bytes, sh) or
+                        rh.rehyat_feature_map_mlp(params, k.data_ptr(), mlp, pk.data_ptr(),
+                                                  mws.data_ptr(), mlp_bytes, sh))
+        fwd = lambda: rh.rehyat_hybrid_attn_fwd_phi(params, q.data_ptr(), k.data_ptr(),
+                                                    v.data_ptr(), pq.data_ptr(), pk.data_ptr(),
+                                                    y.data_ptr(), ws.data_ptr(), ws.numel(),
+                                                    None, sh)
+        if feat() or fwd():
+            raise RuntimeError("general feature map path failed")
+        feat_ms, fwd_ms = timed(feat), timed(fwd)
+        del pq, pk, ws, mws
+        return feat_ms, fwd_ms, mlp_bytes > 0
+
+    feat_ms, fwd_ms, tensor_cores = run(torch.bfloat16)
+    feat32_ms, fwd32_ms, _ = run(torch.float32)
     feat_flops = 2 * B * H * N * (2.0 * D * Dh + 2.0 * Dh * Dp)  # q and k
-    # Algorithmic bytes: x in (bf16) and phi out (fp32) for q and k; the
+    # Algorithmic bytes: x in (bf16) and phi out (bf16) for q and k; the
     # weights (2.4 MB of images) are negligible.
-    feat_bytes = 2 * B * H * N * (D * 2 + Dp * 4)
-    peaks = load_peaks()
+    feat_bytes = 2 * B * H * N * (D * 2 + Dp * 2)
     tflops = feat_flops / (feat_ms / 1e3) / 1e12
     gbs = feat_bytes / (feat_ms / 1e3) / 1e9
-    del pq, pk, y, ws, mws
+    del y
     out = {"feature_maps_ms": feat_ms,
            "feature_maps_path": "tensor cores (bf16 operands)" if tensor_cores
            else "fp32 CUDA cores",
+           "feature_maps_dtype": "bf16",
            "feature_maps_tflops": tflops,
            "feature_maps_gbs": gbs,
            "forward_phi_given_ms": fwd_ms,
            "forward_phi_given_tokens_per_s": B * N / (fwd_ms / 1e3),
+           "maps_plus_forward_ms": feat_ms + fwd_ms,
+           "fp32_maps": {"feature_maps_ms": feat32_ms, "forward_phi_given_ms": fwd32_ms,
+                         "maps_plus_forward_ms": feat32_ms + fwd32_ms},
            "what": "rehyat_feature_map_mlp for q and k (hidden 3D = 384, P = 2), then "
-                   "rehyat_hybrid_attn_fwd_phi (tensor-core path) on the bench workload"}
+                   "rehyat_hybrid_attn_fwd_phi (tensor-core path) on the bench workload; "
+                   "maps in bf16 (REHYAT_FLAG_PHI_BF16), and in fp32 under fp32_maps"}
     if tensor_cores:
-        # Both bounds are near: 3.09e11 FLOP and 1.21 GB per pair of maps.
         out["feature_maps_frac_bf16_peak"] = tflops / peaks["bf16_tflops"]
         out["feature_maps_frac_hbm"] = gbs / peaks["hbm_gbs"]
     else:

@@ -72,8 +72,8 @@ typedef enum { REHYAT_F32 = 0, REHYAT_BF16 = 1 } rehyat_dtype;
 #define REHYAT_FLAG_FORCE_SIMT 1 /* use the fp32 CUDA-core kernels even where a
                                     tensor-core kernel exists (testing aid) */
 #define REHYAT_FLAG_ONE_TILE 2   /* tensor-core attention: use the one-query-tile
-                                    kernel (the default for Dp = 256) instead of
-                                    the two-tile kernel (testing aid) */
+                                    kernel instead of the two-tile kernel (closed-
+                                    form phi only; testing aid) */
 #define REHYAT_FLAG_FP8_QK 4     /* fp8 softmax branch: the logits q.k^T are formed
                                     from q and k rounded to E4M3 (round to nearest
                                     even, saturating at +-448, unit scale) on the
@@ -87,6 +87,13 @@ typedef enum { REHYAT_F32 = 0, REHYAT_BF16 = 1 } rehyat_dtype;
                                     The workspace grows by the two E4M3 copies
                                     (2 * B * h * N * D bytes), which
                                     rehyat_fwd_attn writes. */
+#define REHYAT_FLAG_PHI_BF16 8   /* feature-map arrays in bf16 instead of fp32:
+                                    the output of rehyat_feature_map_mlp (phi
+                                    rounded to nearest even) and the phi_q,
+                                    phi_k inputs of rehyat_hybrid_attn_fwd_phi.
+                                    Halves the maps' memory traffic; the
+                                    tensor-core forward rounds phi_k to bf16
+                                    anyway.  Ignored by other entry points. */
 
 typedef struct {
   int batch, heads;   /* B >= 1, h >= 1 */
@@ -245,15 +252,16 @@ REHYAT_API rehyat_status rehyat_chunk_step(const rehyat_params* p, const void* q
  * raised to the i-th power, phi = [psi_1^1, ..., psi_P^P]).                */
 
 /* The same forward as rehyat_hybrid_attn_fwd with the feature maps given as
- * arrays: phi_q = phi_q(q), phi_k = phi_k(k), fp32 [B][h][N][Dp], 16-byte
- * aligned (any map, e.g. rehyat_feature_map_mlp's).  phi values may be
+ * arrays: phi_q = phi_q(q), phi_k = phi_k(k), [B][h][N][Dp] in fp32 (bf16
+ * with REHYAT_FLAG_PHI_BF16), 16-byte aligned (any map, e.g.
+ * rehyat_feature_map_mlp's).  phi values may be
  * negative (a degree-1 part), so n^L may be negative; y is the joint
  * normalisation as written, without clamping the denominator.  Workspace as
  * rehyat_workspace_bytes(p); other arguments and errors as for
  * rehyat_hybrid_attn_fwd. */
 REHYAT_API rehyat_status rehyat_hybrid_attn_fwd_phi(const rehyat_params* p, const void* q,
                                                     const void* k, const void* v,
-                                                    const float* phi_q, const float* phi_k,
+                                                    const void* phi_q, const void* phi_k,
                                                     void* y, void* workspace, size_t ws_bytes,
                                                     const rehyat_debug* dbg, void* stream);
 
@@ -307,9 +315,10 @@ typedef struct {
  * REHYAT_FLAG_FORCE_SIMT) keeps bf16 images of Wa and Wb there. */
 REHYAT_API size_t rehyat_feature_map_mlp_workspace_bytes(const rehyat_params* p,
                                                          const rehyat_phi_mlp* mlp,
-                                                         const void* x, const float* phi);
+                                                         const void* x, const void* phi);
 
-/* phi [B][h][N][Dp] (fp32) of x [B][h][N][D] (p->in_dtype), N = T*Hs*Ws,
+/* phi [B][h][N][Dp] (fp32, or bf16 with REHYAT_FLAG_PHI_BF16) of x
+ * [B][h][N][D] (p->in_dtype), N = T*Hs*Ws,
  * heads and shapes from p (Tc, To, causal unused).  Dh <= 512.  Pointers
  * 4-byte aligned; workspace (caller-owned, 16-byte aligned, may be NULL when
  * the size above is 0) of at least rehyat_feature_map_mlp_workspace_bytes
@@ -319,7 +328,7 @@ REHYAT_API size_t rehyat_feature_map_mlp_workspace_bytes(const rehyat_params* p,
  * throughout (erff).  REHYAT_ERR_INVALID_ARG for parts < 1 or Dp % parts != 0;
  * REHYAT_ERR_WORKSPACE if ws_bytes is too small. */
 REHYAT_API rehyat_status rehyat_feature_map_mlp(const rehyat_params* p, const void* x,
-                                                const rehyat_phi_mlp* mlp, float* phi,
+                                                const rehyat_phi_mlp* mlp, void* phi,
                                                 void* workspace, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------- */

@@ -24,7 +24,7 @@ from typing import Optional
 
 __all__ = [
     "RehyatParams", "RehyatPhi", "RehyatDebug", "RehyatError", "lib", "lib_path",
-    "EXPORTED_SYMBOLS", "F32", "BF16", "FLAG_FORCE_SIMT", "FLAG_FP8_QK",
+    "EXPORTED_SYMBOLS", "F32", "BF16", "FLAG_FORCE_SIMT", "FLAG_FP8_QK", "FLAG_PHI_BF16",
     "rehyat_workspace_bytes", "rehyat_hybrid_attn_fwd", "rehyat_fwd_state", "rehyat_fwd_attn",
     "rehyat_softmax_attn_fwd", "rehyat_state_bytes", "rehyat_state_init", "rehyat_step_workspace_bytes",
     "rehyat_chunk_step", "rehyat_device_error_flags", "rehyat_attn_path",
@@ -43,6 +43,7 @@ F32, BF16 = 0, 1
 FLAG_FORCE_SIMT = 1
 FLAG_ONE_TILE = 2
 FLAG_FP8_QK = 4
+FLAG_PHI_BF16 = 8
 
 STATUS = {0: "REHYAT_OK", 1: "REHYAT_ERR_INVALID_ARG", 2: "REHYAT_ERR_UNSUPPORTED",
           3: "REHYAT_ERR_MISALIGNED", 4: "REHYAT_ERR_WORKSPACE", 5: "REHYAT_ERR_CUDA",
@@ -507,11 +508,12 @@ def hybrid_attn_host(q, k, v, Wq, bq, Wk, bk, *, T, Hs, Ws, Tc, To, causal, out=
 
 
 def feature_map_mlp(x, Wa, ba, Wb, bb, *, parts, T, Hs, Ws, stream=None, force_simt=False,
-                    workspace=None, out=None):
+                    workspace=None, out=None, out_dtype=None):
     """phi = [psi_1^1, ..., psi_P^P], psi = GELU(x Wa + ba) Wb + bb per head,
     of a torch CUDA tensor x [B, h, N, D]; Wa [h, D, Dh], ba [h, Dh],
-    Wb [h, Dh, D'], bb [h, D'] fp32.  Returns fp32 [B, h, N, D'].  bf16 x with
-    D = 128 runs on the tensor cores (bf16 operands) unless force_simt."""
+    Wb [h, Dh, D'], bb [h, D'] fp32.  Returns [B, h, N, D'] in out_dtype
+    (fp32 by default, or bf16).  bf16 x with D = 128 runs on the tensor cores
+    (bf16 operands) unless force_simt."""
     torch = _torch()
     _need(x.dim() == 4, "x must be a [B, h, N, D] tensor")
     _need(x.is_contiguous() and x.is_cuda, "x must be a contiguous CUDA tensor")
@@ -521,12 +523,16 @@ def feature_map_mlp(x, Wa, ba, Wb, bb, *, parts, T, Hs, Ws, stream=None, force_s
     Dh, Dp = Wa.shape[-1], Wb.shape[-1]
     _check_params((("Wa", Wa), ("ba", ba), ("Wb", Wb), ("bb", bb)),
                   (H * D * Dh, H * Dh, H * Dh * Dp, H * Dp), x.device, "MLP parameters")
+    out_dtype = torch.float32 if out_dtype is None else out_dtype
+    _need(out_dtype in (torch.float32, torch.bfloat16), "out_dtype must be fp32 or bf16",
+          TypeError)
     p = make_params(batch=B, heads=H, T=T, Hs=Hs, Ws=Ws, D=D, Dp=Dp, Tc=1, To=0, causal=0,
                     in_dtype=_dtype_code(x.dtype), out_dtype=F32,
-                    flags=FLAG_FORCE_SIMT if force_simt else 0)
+                    flags=(FLAG_FORCE_SIMT if force_simt else 0) |
+                    (FLAG_PHI_BF16 if out_dtype == torch.bfloat16 else 0))
     if out is not None:
-        _check_out(out, (B, H, N, Dp), torch.float32, x.device)
-    phi = out if out is not None else torch.empty(B, H, N, Dp, dtype=torch.float32,
+        _check_out(out, (B, H, N, Dp), out_dtype, x.device)
+    phi = out if out is not None else torch.empty(B, H, N, Dp, dtype=out_dtype,
                                                   device=x.device)
     mlp = RehyatPhiMlp(Wa.data_ptr(), ba.data_ptr(), Wb.data_ptr(), bb.data_ptr(), Dh, parts)
     nbytes = rehyat_feature_map_mlp_workspace_bytes(p, mlp, x.data_ptr(), phi.data_ptr())
@@ -544,8 +550,8 @@ def hybrid_attn_phi(q, k, v, phi_q, phi_k, *, T, Hs, Ws, Tc, To, causal, out_dty
                     scale=0.0, debug=False, force_simt=False, workspace=None, out=None,
                     stream=None):
     """The hybrid forward with the feature maps given: phi_q = phi_q(q) and
-    phi_k = phi_k(k), fp32 [B, h, N, D'] CUDA tensors.  Returns y (and the
-    branch partials when ``debug``)."""
+    phi_k = phi_k(k), [B, h, N, D'] CUDA tensors, both fp32 or both bf16.
+    Returns y (and the branch partials when ``debug``)."""
     torch = _torch()
     _check_qkv(q, k, v)
     _check_current_device(q.device)
@@ -553,15 +559,17 @@ def hybrid_attn_phi(q, k, v, phi_q, phi_k, *, T, Hs, Ws, Tc, To, causal, out_dty
     _check_tokens(N, T, Hs, Ws)
     Dp = phi_q.shape[-1]
     for t in (phi_q, phi_k):
-        if (t.dtype != torch.float32 or not t.is_contiguous() or t.dim() != 4
-                or tuple(t.shape) != (B, H, N, Dp)):
-            raise TypeError("phi_q, phi_k must be contiguous fp32 [B, h, N, D'] tensors")
+        if (t.dtype not in (torch.float32, torch.bfloat16) or t.dtype != phi_q.dtype
+                or not t.is_contiguous() or t.dim() != 4 or tuple(t.shape) != (B, H, N, Dp)):
+            raise TypeError("phi_q, phi_k must be contiguous [B, h, N, D'] tensors, both fp32 "
+                            "or both bf16")
         _need(t.device == q.device, "phi_q, phi_k must be on q's device")
     out_dtype = torch.float32 if out_dtype is None else out_dtype
     p = make_params(batch=B, heads=H, T=T, Hs=Hs, Ws=Ws, D=D, Dp=Dp, Tc=Tc, To=To,
                     causal=causal, in_dtype=_dtype_code(q.dtype),
                     out_dtype=_dtype_code(out_dtype), scale=scale,
-                    flags=FLAG_FORCE_SIMT if force_simt else 0)
+                    flags=(FLAG_FORCE_SIMT if force_simt else 0) |
+                    (FLAG_PHI_BF16 if phi_q.dtype == torch.bfloat16 else 0))
     if out is not None:
         _check_out(out, (B, H, N, D), out_dtype, q.device)
     y = torch.empty(B, H, N, D, dtype=out_dtype, device=q.device) if out is None else out

@@ -257,10 +257,11 @@ cudaError_t run_attn(const rehyat_params* p, const AttnParams& a, cudaStream_t s
 // Per-slice states and the linear-set state per chunk into the workspace
 // laid out by fwd_layout (weight images, per-slice state kernel, chunk scan);
 // arguments already checked.
-// With phi_k given ([BH][N][Dp] fp32), phi is unused (may be null).
+// With phi_k given ([BH][N][Dp], fp32 or with REHYAT_FLAG_PHI_BF16 bf16),
+// phi is unused (may be null).
 rehyat_status state_pass(const rehyat_params* p, const void* k, const void* v,
                          const rehyat_phi* phi, char* ws, cudaStream_t s,
-                         const float* phi_k = nullptr) {
+                         const void* phi_k = nullptr) {
   const FwdWorkspace w = fwd_layout(p);
   float* P = reinterpret_cast<float*>(ws + w.P_off);
   float* z = reinterpret_cast<float*>(ws + w.z_off);
@@ -275,6 +276,7 @@ rehyat_status state_pass(const rehyat_params* p, const void* k, const void* v,
   pp.Wk = phi_k ? nullptr : phi->Wk;
   pp.bk = phi_k ? nullptr : phi->bk;
   pp.phi_k = phi_k;
+  pp.phi_bf16 = (p->flags & REHYAT_FLAG_PHI_BF16) ? 1 : 0;
   pp.P = P; pp.z = z;
   pp.BH = BH; pp.heads = p->heads; pp.HW = HW; pp.D = p->D; pp.Dp = p->Dp; pp.To = p->To;
   pp.nslots = p->T;
@@ -293,7 +295,7 @@ rehyat_status state_pass(const rehyat_params* p, const void* k, const void* v,
 
 // Checks and marshals the feature-map call; REHYAT_OK and *a filled, or the error.
 rehyat_status mlp_args(const rehyat_params* p, const void* x, const rehyat_phi_mlp* mlp,
-                       float* phi, PhiMlpArgs* a) {
+                       void* phi, PhiMlpArgs* a) {
   rehyat_status st = check_params(p);
   if (st != REHYAT_OK) return st;
   if ((st = no_fp8(p)) != REHYAT_OK) return st;
@@ -308,6 +310,7 @@ rehyat_status mlp_args(const rehyat_params* p, const void* x, const rehyat_phi_m
   a->N = static_cast<long long>(p->T) * p->Hs * p->Ws;
   a->BH = p->batch * p->heads; a->heads = p->heads; a->D = p->D; a->Dh = mlp->Dh;
   a->Dp = p->Dp; a->parts = mlp->parts; a->in_bf16 = p->in_dtype == REHYAT_BF16;
+  a->phi_bf16 = (p->flags & REHYAT_FLAG_PHI_BF16) ? 1 : 0;
   return REHYAT_OK;
 }
 
@@ -542,7 +545,7 @@ rehyat_status rehyat_chunk_step(const rehyat_params* p, const void* q, const voi
 }
 
 rehyat_status rehyat_hybrid_attn_fwd_phi(const rehyat_params* p, const void* q, const void* k,
-                                         const void* v, const float* phi_q, const float* phi_k,
+                                         const void* v, const void* phi_q, const void* phi_k,
                                          void* y, void* workspace, size_t ws_bytes,
                                          const rehyat_debug* dbg, void* stream) {
   rehyat_status st = check_params(p);
@@ -560,6 +563,7 @@ rehyat_status rehyat_hybrid_attn_fwd_phi(const rehyat_params* p, const void* q, 
   if ((st = state_pass(p, k, v, nullptr, ws, s, phi_k)) != REHYAT_OK) return st;
   AttnParams a = base_attn(p, q, k, v, nullptr, y, dbg);
   a.phi_q = phi_q;
+  a.phi_bf16 = (p->flags & REHYAT_FLAG_PHI_BF16) ? 1 : 0;
   a.rows_per_bh = static_cast<long long>(p->T) * p->Hs * p->Ws;
   a.SL = reinterpret_cast<const float*>(ws + w.SL_off);
   a.zL = reinterpret_cast<const float*>(ws + w.zL_off);
@@ -568,14 +572,14 @@ rehyat_status rehyat_hybrid_attn_fwd_phi(const rehyat_params* p, const void* q, 
 }
 
 size_t rehyat_feature_map_mlp_workspace_bytes(const rehyat_params* p, const rehyat_phi_mlp* mlp,
-                                              const void* x, const float* phi) {
+                                              const void* x, const void* phi) {
   PhiMlpArgs a;
-  if (mlp_args(p, x, mlp, const_cast<float*>(phi), &a) != REHYAT_OK || !mlp_tc(p, a)) return 0;
+  if (mlp_args(p, x, mlp, const_cast<void*>(phi), &a) != REHYAT_OK || !mlp_tc(p, a)) return 0;
   return align_up(phi_mlp_image_bytes(a.heads, a.Dh, a.Dp));
 }
 
 rehyat_status rehyat_feature_map_mlp(const rehyat_params* p, const void* x,
-                                     const rehyat_phi_mlp* mlp, float* phi, void* workspace,
+                                     const rehyat_phi_mlp* mlp, void* phi, void* workspace,
                                      size_t ws_bytes, void* stream) {
   PhiMlpArgs a;
   const rehyat_status st = mlp_args(p, x, mlp, phi, &a);

@@ -29,7 +29,8 @@ struct AttnParams {
   const float *SL, *zL;      // linear-set state per chunk
   const float *Wq, *bq;      // phi_q parameters, fp32 [h][2][D][Dp/2], [h][2][Dp/2]
   const void* wq_img;        // bf16 phi_q weight image per head (tensor-core path) or nullptr
-  const float* phi_q;        // phi_q(q) given as [BH][rows][Dp] fp32 (then Wq, bq unused) or nullptr
+  const void* phi_q;         // phi_q(q) given as [BH][rows][Dp] (then Wq, bq unused) or nullptr
+  int phi_bf16;              // the given phi_q is bf16 (else fp32)
   const void *q8, *k8;       // E4M3 copies of q, k for the softmax logits (fp8 variant) or nullptr
   void* y;
   float *dbg_aS, *dbg_nS, *dbg_c, *dbg_aL, *dbg_nL;
@@ -73,7 +74,8 @@ struct PartialParams {
   long long ring_rows_per_bh;
   const long long* seen;
   const float *Wk, *bk;
-  const float* phi_k;        // phi_k(k) given as [BH][rows][Dp] fp32 (then Wk, bk unused) or nullptr
+  const void* phi_k;         // phi_k(k) given as [BH][rows][Dp] (then Wk, bk unused) or nullptr
+  int phi_bf16;              // the given phi_k is bf16 (else fp32)
   float *P, *z;              // [BH][nslots][Dp][D], [BH][nslots][Dp]
   int BH, heads, HW, D, Dp, To, nslots, nq_slices;
   int in_bf16, w_bf16;
@@ -185,7 +187,8 @@ cudaError_t launch_attn_bwd_lin_simt(const AttnBwdParams& p, cudaStream_t s);
 struct PhiMlpArgs {
   const void* x;
   const float *Wa, *ba, *Wb, *bb;
-  float* phi;
+  void* phi;                 // fp32, or bf16 when phi_bf16
+  int phi_bf16;
   long long N;
   int BH, heads, D, Dh, Dp, parts, in_bf16;
 };

@@ -84,7 +84,11 @@ __global__ void __launch_bounds__(kMlpThreads) phi_mlp_kernel(PhiMlpArgs a) {
       if (r < nrows) {
         float v = acc[r];
         for (int i = 1; i < power; ++i) v *= acc[r];
-        a.phi[(rowbase + r0 + r) * a.Dp + f] = v;
+        const long long o = (rowbase + r0 + r) * a.Dp + f;
+        if (a.phi_bf16)
+          static_cast<__nv_bfloat16*>(a.phi)[o] = __float2bfloat16_rn(v);
+        else
+          static_cast<float*>(a.phi)[o] = v;
       }
     }
   }

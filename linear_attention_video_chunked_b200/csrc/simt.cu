@@ -24,6 +24,13 @@ __device__ unsigned long long rehyat_simt_den_rows = 0;
 
 namespace {
 
+// Element i of a given feature map: fp32, or bf16 when bf16 is set.
+__device__ __forceinline__ float ld_phi(const void* phi, int bf16, long long i) {
+  return bf16 ? __bfloat162float(__ldg(static_cast<const __nv_bfloat16*>(phi) + i))
+              : __ldg(static_cast<const float*>(phi) + i);
+}
+
+
 constexpr float kLn2 = 0.69314718055994530942f;
 
 __device__ __forceinline__ float load_in(const void* base, long long i, int bf16) {
@@ -193,7 +200,7 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(AttnParams P) {
     for (int f = lane4; f < Dp; f += 4) {
       float ph;
       if (P.phi_q) {  // phi_q(q) given
-        ph = r < nrows ? __ldg(P.phi_q + (qrow_base + r) * Dp + f) : 0.f;
+        ph = r < nrows ? ld_phi(P.phi_q, P.phi_bf16, (qrow_base + r) * Dp + f) : 0.f;
       } else {
         float psi = __ldg(P.bq + b_index(h, Dp, f));
         for (int d = 0; d < D; ++d)
@@ -301,7 +308,7 @@ __global__ void __launch_bounds__(256) partials_simt_kernel(PartialParams P) {
       float ph = 0.f;
       if (f < Dp && j0 + j < P.HW) {
         if (P.phi_k) {  // phi_k(k) given (full forward: rows as in k)
-          ph = __ldg(P.phi_k + (base + j0 + j) * Dp + f);
+          ph = ld_phi(P.phi_k, P.phi_bf16, (base + j0 + j) * Dp + f);
         } else {
           float psi = __ldg(P.bk + b_index(h, Dp, f));
           for (int d = 0; d < D; ++d)

@@ -731,9 +731,11 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
       if (linear && phi_given) {
         // The tail reads both tiles' rows of phi_q(q) (contiguous): into L2
         // now, so those loads do not wait on DRAM at the end of the CTA.
-        const uint32_t bytes = static_cast<uint32_t>(nrows_t[0] + nrows_t[1]) * Dp * 4;
+        const int eb = P.phi_bf16 ? 2 : 4;
+        const uint32_t bytes = static_cast<uint32_t>(nrows_t[0] + nrows_t[1]) * Dp * eb;
         asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(
-                         P.phi_q + (static_cast<long long>(bh) * P.rows_per_bh + row0) * Dp),
+                         static_cast<const uint8_t*>(P.phi_q) +
+                         (static_cast<long long>(bh) * P.rows_per_bh + row0) * Dp * eb),
                      "r"(bytes)
                      : "memory");
       }
@@ -1199,13 +1201,11 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 4; ++e)
               z4[e] = npieces == 1 ? vec[Dp + col + e] : __ldg(zsrc + col + e);
-#pragma unroll 4
-            for (int it = 0; it < 8; ++it) {
+            // One row group of four: its values (already loaded), n^L parts
+            // and the tf32 staging.
+            auto stage4 = [&](int it, float4 g4) {
               const int rr = 32 * (warp & 3) + 4 * it + rsub;  // row within the tile
               const float inv_r = __shfl_sync(0xffffffffu, inv_f, 4 * it + rsub);
-              float4 g4 = make_float4(0.f, 0.f, 0.f, 0.f);
-              if (rr < nrows)
-                g4 = __ldg(reinterpret_cast<const float4*>(P.phi_q + (gtile + rr) * Dp + f0 + col));
               float part = g4.x * z4[0] + g4.y * z4[1] + g4.z * z4[2] + g4.w * z4[3];
               part += __shfl_xor_sync(0xffffffffu, part, 4);
               part += __shfl_xor_sync(0xffffffffu, part, 2);
@@ -1215,6 +1215,33 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
               st_shared_v4(phi + c * 16384 + rr * 128 + ((q4 ^ (rr & 7)) << 4),
                            __float_as_uint(g4.x * inv_r), __float_as_uint(g4.y * inv_r),
                            __float_as_uint(g4.z * inv_r), __float_as_uint(g4.w * inv_r));
+            };
+            const int rbase = 32 * (warp & 3) + rsub;
+            if (P.phi_bf16) {
+              const __nv_bfloat16* src =
+                  static_cast<const __nv_bfloat16*>(P.phi_q) + (gtile + rbase) * Dp + f0 + col;
+              uint2 u[8];
+#pragma unroll
+              for (int it = 0; it < 8; ++it)
+                u[it] = rbase + 4 * it < nrows
+                            ? __ldg(reinterpret_cast<const uint2*>(src + 4LL * it * Dp))
+                            : make_uint2(0u, 0u);
+#pragma unroll
+              for (int it = 0; it < 8; ++it)
+                stage4(it, make_float4(__uint_as_float(u[it].x << 16),
+                                       __uint_as_float(u[it].x & 0xFFFF0000u),
+                                       __uint_as_float(u[it].y << 16),
+                                       __uint_as_float(u[it].y & 0xFFFF0000u)));
+            } else {
+              const float* src = static_cast<const float*>(P.phi_q) + (gtile + rbase) * Dp + f0 + col;
+              float4 g[8];
+#pragma unroll
+              for (int it = 0; it < 8; ++it)
+                g[it] = rbase + 4 * it < nrows
+                            ? __ldg(reinterpret_cast<const float4*>(src + 4LL * it * Dp))
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+              for (int it = 0; it < 8; ++it) stage4(it, g[it]);
             }
           }
         } else {
@@ -1387,10 +1414,15 @@ constexpr uint32_t kSmemBytes = kBarOff + 256 + 1024;
 // TMEM: psi^T fp32 [0,128) [128,256), phi^T bf16 pairs [256,320) [320,384)
 // (each alternating per token tile), P accumulator [384,512).
 constexpr uint32_t kColPsi = 0, kColPhi = 256, kColP = 384;
-// phi_k(k) given: the 16 KB box b (32 features x 128 tokens, fp32, token-major)
-// of stage s, in the K ring and the W_k area.
-__host__ __device__ constexpr uint32_t phi_box(int s, int b) {
-  return s == 0 ? kKOff + b * 16384 : (b < 2 ? kKOff + 65536 + b * 16384 : kWOff + (b - 2) * 16384);
+// phi_k(k) given: the 16 KB box b (128 tokens x 128 bytes of features,
+// token-major) of stage s.  fp32 tiles (four boxes for 128 features) use two
+// stages over the K ring and the W_k area; bf16 tiles (two boxes) three
+// stages in the K ring, like K tiles.
+constexpr int phi_stages(bool bf16) { return bf16 ? 3 : 2; }
+__host__ __device__ constexpr uint32_t phi_box(int s, int b, bool bf16) {
+  return bf16 ? kKOff + s * 32768 + b * 16384
+              : (s == 0 ? kKOff + b * 16384
+                        : (b < 2 ? kKOff + 65536 + b * 16384 : kWOff + (b - 2) * 16384));
 }
 
 // Walk over a CTA's run of items i = q * T + slice, q = bh * halves + half,
@@ -1425,9 +1457,9 @@ struct ItemWalk {
 }  // namespace sp
 
 // kPhiGiven: phi_k(k) is read from P.phi_k (full forward) instead of being
-// computed from K and W_k (a separate instantiation, so the default path
-// carries no branch for it).
-template <bool kPhiGiven>
+// computed from K and W_k, in fp32 or (kPhiBf16) bf16 (separate
+// instantiations, so no path carries branches for the others).
+template <bool kPhiGiven, bool kPhiBf16 = false>
 __global__ void __launch_bounds__(sp::kThreads, 1)
     tc_state_persistent_kernel(const __grid_constant__ StMaps maps, const PartialParams P,
                                const __nv_bfloat16* __restrict__ wk_img, int items_per_cta) {
@@ -1464,6 +1496,7 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
   // seen - min(seen, T_o) + i, in the ring if already seen, else in the chunk).
   const bool step = P.seen != nullptr;
   constexpr bool phi_given = kPhiGiven;
+  constexpr bool phi_bf16 = kPhiBf16;
   const int T = step ? P.nq_slices : P.nslots;
   const long long seen0 = step ? *P.seen : 0;
   const long long rseen = seen0 < P.To ? seen0 : P.To;
@@ -1498,7 +1531,7 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
     for (int i = 0; i < NBAR; ++i) {
       const bool by_group = i == PSI_FREE || i == PSI_FREE + 1 || i == PHI_FULL ||
                             i == PHI_FULL + 1 || i == P_FREE ||
-                            (phi_given && (i == K_EMPTY || i == K_EMPTY + 1));
+                            (phi_given && (i == K_EMPTY || i == K_EMPTY + 1 || i == K_EMPTY + 2));
       mbar_init(bar(i), by_group ? 128 : 1);
     }
     *abort_flag = 0;
@@ -1529,24 +1562,31 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
     // warp 8 loads K tiles (and the W_k piece), warp 11 V tiles, so K runs
     // ahead on its own ring (psi^T) while V waits for phi^T V to free stages.
     if (lane == 0 && warp == 8 && phi_given) {
-      // phi_k(k) given: its fp32 tiles (pw features x 128 tokens, boxes of
-      // 32 features) into two stages of the space K and W_k leave unused,
-      // so the converters read them from shared memory.
+      // phi_k(k) given: its tiles (pw features x 128 tokens, boxes of 128
+      // bytes of features: 32 fp32 or 64 bf16) into two stages of the space K
+      // and W_k leave unused, so the converters read them from shared memory.
       bool ok = true;
       sp::ItemWalk w{T, halves, P.heads, pw, leave};
       w.start(it0);
       int gt = 0;
-      const uint32_t tile_bytes = static_cast<uint32_t>(pw) * 128 * 4;
+      constexpr bool bf = phi_bf16;
+      constexpr int fpb = bf ? 64 : 32;  // features per box
+      constexpr int nst = sp::phi_stages(bf);
+      const uint32_t tile_bytes = static_cast<uint32_t>(pw) * 128 * (bf ? 2 : 4);
+      int st = 0, uses = 0;  // stage of tile gt, earlier uses of that stage
       for (int il = 0; il < nitems && ok; ++il, w.next()) {
         if (!w.on()) continue;
         for (int j = 0; j < nt && ok; ++j, ++gt) {
-          const int st = gt & 1;
-          if (gt >= 2) ok = mbar_wait(bar(K_EMPTY + st), ((gt - 2) >> 1) & 1, abort_flag, 39);
+          if (gt >= nst) ok = mbar_wait(bar(K_EMPTY + st), (uses - 1) & 1, abort_flag, 39);
           if (!ok) break;
           mbar_expect_tx(bar(K_FULL + st), tile_bytes);
-          for (int bx = 0; bx < pw / 32; ++bx)
-            tma_load_3d(base + sp::phi_box(st, bx), &maps.phik, bar(K_FULL + st),
-                        w.half() * pw + 32 * bx, w.slice * HW + j * 128, w.bh());
+          for (int bx = 0; bx < (pw + fpb - 1) / fpb; ++bx)
+            tma_load_3d(base + sp::phi_box(st, bx, bf), &maps.phik, bar(K_FULL + st),
+                        w.half() * pw + fpb * bx, w.slice * HW + j * 128, w.bh());
+          if (++st == nst) {
+            st = 0;
+            ++uses;
+          }
         }
       }
     } else if (lane == 0 && !(warp == 8 && phi_given)) {  // no K or W_k with phi_k given
@@ -1703,6 +1743,9 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
     sp::ItemWalk w{T, halves, P.heads, pw, leave};
     w.start(it0);
     int gt = 0, vst = 0, vuses = 0, wkey = -1;
+    // phi_k given: the shared-memory stage of the current tile, its uses.
+    constexpr int nfst = sp::phi_stages(phi_bf16);
+    int fst = 0, fuses = 0;
     for (int il = 0; il < nitems && ok; ++il, w.next()) {
       if (!w.on()) continue;
       // b_k of head h is h's D' consecutive features.
@@ -1716,7 +1759,8 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
         const int b = gt & 1;
         // psi^T of the tile in TMEM buffer b, or (phi_k given) its phi_k
         // tile in shared-memory stage b.
-        ok = wait_all(bar(phi_given ? K_FULL + b : PSI_FULL + b), (gt >> 1) & 1, 36);
+        ok = phi_given ? wait_all(bar(K_FULL + fst), fuses & 1, 36)
+                       : wait_all(bar(PSI_FULL + b), (gt >> 1) & 1, 36);
         // phi^T buffer b is free once phi^T V of tile gt - 2 has read it.
         if (ok && gt >= 2) ok = wait_all(bar(PHI_FREE + b), ((gt - 2) >> 1) & 1, 38);
         if (!ok) break;
@@ -1729,11 +1773,22 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t ps[32], pk[16];
-          if (phi_given) {
+          if (phi_given && phi_bf16) {
+            // Feature f of tokens 32c .. 32c + 31: a column of box f / 64
+            // (token-major rows of 64 bf16; a warp reads half a row).
+            const __nv_bfloat16* col = reinterpret_cast<const __nv_bfloat16*>(
+                                           sbase + sp::phi_box(fst, f < pw ? f >> 6 : 0, true)) +
+                                       (f & 63);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int t = c * 32 + i;
+              ps[i] = __float_as_uint(f < pw && t < nvalid ? __bfloat162float(col[t * 64]) : 0.f);
+            }
+          } else if (phi_given) {
             // Feature f of tokens 32c .. 32c + 31: a column of box f / 32
             // (token-major rows of 32 floats; a warp reads whole rows).
             const float* col = reinterpret_cast<const float*>(
-                                   sbase + sp::phi_box(b, f < pw ? f >> 5 : 0)) + (f & 31);
+                                   sbase + sp::phi_box(fst, f < pw ? f >> 5 : 0, false)) + (f & 31);
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
               const int t = c * 32 + i;
@@ -1764,7 +1819,13 @@ __global__ void __launch_bounds__(sp::kThreads, 1)
           }
           REHYAT_TMEM_ST16(pcols + c * 16, pk);
         }
-        if (phi_given) mbar_arrive(bar(K_EMPTY + b));  // the stage's reads are done
+        if (phi_given) {  // the stage's reads are done
+          mbar_arrive(bar(K_EMPTY + fst));
+          if (++fst == nfst) {
+            fst = 0;
+            ++fuses;
+          }
+        }
         tmem_wait_st();
         if (nvalid < 128) {
           // V rows past the slice are zeroed so that 0 * V stays 0 for any V.
@@ -1880,20 +1941,24 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // 3D 8-bit map over [planes][rows][128] with a 128 x 128 x 1 box (one 128-byte
 // row per token), 128B swizzle.
-// fp32 [planes][rows][cols] with boxes of 32 columns x 128 rows, unswizzled
-// (a box lands as 128 rows of 128 bytes).
-bool make_map_f32(CUtensorMap* m, const float* ptr, long long rows, int planes, int cols) {
+// A given feature map [planes][rows][cols], fp32 or bf16, with boxes of 128
+// bytes of columns (32 fp32 or 64 bf16) x 128 rows, unswizzled (a box lands
+// as 128 rows of 128 bytes).
+bool make_map_phi(CUtensorMap* m, const void* ptr, long long rows, int planes, int cols,
+                  bool bf16) {
   auto fn = encode_fn();
-  if (!fn || rows <= 0 || cols % 32 != 0) return false;
+  const int eb = bf16 ? 2 : 4;
+  if (!fn || rows <= 0 || (cols * eb) % 128 != 0) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows),
                         static_cast<cuuint64_t>(planes)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols) * 4,
-                           static_cast<cuuint64_t>(rows) * cols * 4};
-  cuuint32_t box[3] = {32, 128, 1};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols) * eb,
+                           static_cast<cuuint64_t>(rows) * cols * eb};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / eb), 128, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(ptr), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
+            const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 bool make_map8(CUtensorMap* m, const void* ptr, long long rows, int planes) {
@@ -1952,12 +2017,19 @@ cudaError_t launch_state_tc(const PartialParams& p, const void* wk_img, cudaStre
   const int ctas = (total + per_cta - 1) / per_cta;
   const __nv_bfloat16* wk = static_cast<const __nv_bfloat16*>(wk_img);
   if (p.phi_k != nullptr) {  // full forward with phi_k(k) given
-    if (!make_map_f32(&maps.phik, p.phi_k, p.rows_per_bh, p.BH, p.Dp))
+    if (!make_map_phi(&maps.phik, p.phi_k, p.rows_per_bh, p.BH, p.Dp, p.phi_bf16 != 0))
       return cudaErrorInvalidValue;
-    const cudaError_t e = ensure_smem(tc_state_persistent_kernel<true>, 3, sp::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    tc_state_persistent_kernel<true><<<ctas, sp::kThreads, sp::kSmemBytes, s>>>(maps, p, wk,
-                                                                                per_cta);
+    if (p.phi_bf16) {
+      const cudaError_t e = ensure_smem(tc_state_persistent_kernel<true, true>, 10, sp::kSmemBytes);
+      if (e != cudaSuccess) return e;
+      tc_state_persistent_kernel<true, true><<<ctas, sp::kThreads, sp::kSmemBytes, s>>>(
+          maps, p, wk, per_cta);
+    } else {
+      const cudaError_t e = ensure_smem(tc_state_persistent_kernel<true>, 3, sp::kSmemBytes);
+      if (e != cudaSuccess) return e;
+      tc_state_persistent_kernel<true><<<ctas, sp::kThreads, sp::kSmemBytes, s>>>(maps, p, wk,
+                                                                                  per_cta);
+    }
     return cudaGetLastError();
   }
   const cudaError_t e = ensure_smem(tc_state_persistent_kernel<false>, 0, sp::kSmemBytes);

@@ -56,9 +56,9 @@ struct Args {
   const __nv_bfloat16* img;  // [heads][w_bytes / 2] weight images
   const float* ba;           // [heads][Dh]
   const float* bb;           // [heads][Dp]
-  float* phi;                // [B*heads][N][Dp]
+  void* phi;                 // [B*heads][N][Dp], fp32 or (phi_bf16) bf16
   long long N;
-  int batch, heads, Dh, Dp, parts, ntile, tiles_per_cta;
+  int batch, heads, Dh, Dp, parts, ntile, tiles_per_cta, phi_bf16;
 };
 
 // Tile it of the walk: it = (h * batch + b) * ntile + tile.
@@ -139,8 +139,9 @@ __device__ __forceinline__ uint32_t gelu2_bf16(float u0, float u1) {
 // first row, `rows` of them valid).  kDp, kP > 0: the part width is a
 // compile-time constant and the power is applied with kP - 1 predicated
 // products; kP = 0: any P (a division per value).
-template <int kDp, int kP>
-__device__ __forceinline__ void store_rows(float* out, const float* bias, uint32_t tq, int rows,
+// out: fp32 [rows][Dp], or bf16 (round to nearest even) when kBf16.
+template <int kDp, int kP, bool kBf16>
+__device__ __forceinline__ void store_rows(void* out, const float* bias, uint32_t tq, int rows,
                                            int Dp, int parts) {
   const int dp = kDp > 0 ? kDp : Dp;
   const int width = kP > 0 ? dp / kP : Dp / parts;
@@ -177,12 +178,19 @@ __device__ __forceinline__ void store_rows(float* out, const float* bias, uint32
           }
           v[e] = y;
         }
-        if (ra < rows)
-          *reinterpret_cast<float2*>(out + static_cast<long long>(ra) * dp + c) =
-              make_float2(v[0], v[1]);
-        if (rb < rows)
-          *reinterpret_cast<float2*>(out + static_cast<long long>(rb) * dp + c) =
-              make_float2(v[2], v[3]);
+        if (kBf16) {
+          __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
+          if (ra < rows)
+            *reinterpret_cast<uint32_t*>(o + static_cast<long long>(ra) * dp + c) = pack_bf16(v[0], v[1]);
+          if (rb < rows)
+            *reinterpret_cast<uint32_t*>(o + static_cast<long long>(rb) * dp + c) = pack_bf16(v[2], v[3]);
+        } else {
+          float* o = static_cast<float*>(out);
+          if (ra < rows)
+            *reinterpret_cast<float2*>(o + static_cast<long long>(ra) * dp + c) = make_float2(v[0], v[1]);
+          if (rb < rows)
+            *reinterpret_cast<float2*>(o + static_cast<long long>(rb) * dp + c) = make_float2(v[2], v[3]);
+        }
       }
     }
   }
@@ -412,17 +420,26 @@ __global__ void __launch_bounds__(mlp::kThreads, 1)
       tc_fence_after();
       const long long row0 = static_cast<long long>(t.tile) * 128 + q * 32;
       const int rows = static_cast<int>(min(32LL, a.N - row0));
-      float* out = a.phi + (static_cast<long long>(t.b * a.heads + t.h) * a.N + row0) * Dp;
+      const long long o0 = (static_cast<long long>(t.b * a.heads + t.h) * a.N + row0) * Dp;
+      void* out = a.phi_bf16 ? static_cast<void*>(static_cast<__nv_bfloat16*>(a.phi) + o0)
+                             : static_cast<void*>(static_cast<float*>(a.phi) + o0);
       const float* bias = a.bb + static_cast<long long>(t.h) * Dp;
       const uint32_t tq = lane_base + kColPsi + pb * 128;
       const int P = a.parts;
-      if (Dp == 128 && P == 2) store_rows<128, 2>(out, bias, tq, rows, Dp, P);
-      else if (Dp == 128 && P == 1) store_rows<128, 1>(out, bias, tq, rows, Dp, P);
-      else if (Dp == 128 && P == 4) store_rows<128, 4>(out, bias, tq, rows, Dp, P);
-      else if (Dp == 64 && P == 2) store_rows<64, 2>(out, bias, tq, rows, Dp, P);
-      else if (Dp == 64 && P == 1) store_rows<64, 1>(out, bias, tq, rows, Dp, P);
-      else if (Dp == 64 && P == 4) store_rows<64, 4>(out, bias, tq, rows, Dp, P);
-      else store_rows<0, 0>(out, bias, tq, rows, Dp, P);
+      if (a.phi_bf16) {
+        if (Dp == 128 && P == 2) store_rows<128, 2, true>(out, bias, tq, rows, Dp, P);
+        else if (Dp == 128 && P == 1) store_rows<128, 1, true>(out, bias, tq, rows, Dp, P);
+        else if (Dp == 64 && P == 2) store_rows<64, 2, true>(out, bias, tq, rows, Dp, P);
+        else store_rows<0, 0, true>(out, bias, tq, rows, Dp, P);
+      } else {
+        if (Dp == 128 && P == 2) store_rows<128, 2, false>(out, bias, tq, rows, Dp, P);
+        else if (Dp == 128 && P == 1) store_rows<128, 1, false>(out, bias, tq, rows, Dp, P);
+        else if (Dp == 128 && P == 4) store_rows<128, 4, false>(out, bias, tq, rows, Dp, P);
+        else if (Dp == 64 && P == 2) store_rows<64, 2, false>(out, bias, tq, rows, Dp, P);
+        else if (Dp == 64 && P == 1) store_rows<64, 1, false>(out, bias, tq, rows, Dp, P);
+        else if (Dp == 64 && P == 4) store_rows<64, 4, false>(out, bias, tq, rows, Dp, P);
+        else store_rows<0, 0, false>(out, bias, tq, rows, Dp, P);
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(PSI_FREE + pb));
@@ -484,6 +501,7 @@ cudaError_t launch_phi_mlp_tc(const PhiMlpArgs& a, void* images, cudaStream_t s)
   m.ba = a.ba;
   m.bb = a.bb;
   m.phi = a.phi;
+  m.phi_bf16 = a.phi_bf16;
   m.N = a.N;
   m.batch = a.BH / a.heads;
   m.heads = a.heads;

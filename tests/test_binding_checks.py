@@ -340,7 +340,21 @@ def test_feature_map_and_phi_given_refusals(calls):
         rh.hybrid_attn_phi(q, k, v, FakeTensor((2, 3, 300, 128), F32), pq, **GEOM)
     with pytest.raises(ValueError):
         rh.hybrid_attn_phi(q, k, v, pq, FakeTensor((2, 3, 315, 128), F32, "cuda:1"), **GEOM)
+    with pytest.raises(TypeError):         # one map bf16, the other fp32
+        rh.hybrid_attn_phi(q, k, v, pq, FakeTensor((2, 3, 315, 128), BF), **GEOM)
+    with pytest.raises(TypeError):         # an fp16 map
+        rh.feature_map_mlp(q, *mlp, parts=2, T=5, Hs=7, Ws=9, out_dtype=torch.float16)
     assert calls == []
+
+
+def test_bf16_feature_maps_reach_the_abi_with_the_flag(calls):
+    q, k, v = qkv()
+    mlp = [FakeTensor(s, F32) for s in ((3, 128, 384), (3, 384), (3, 384, 128), (3, 128))]
+    pq = rh.feature_map_mlp(q, *mlp, parts=2, T=5, Hs=7, Ws=9, out_dtype=BF)
+    pk = rh.feature_map_mlp(k, *mlp, parts=2, T=5, Hs=7, Ws=9, out_dtype=BF)
+    rh.hybrid_attn_phi(q, k, v, pq, pk, **GEOM)
+    assert [c[0] for c in calls] == ["rehyat_feature_map_mlp"] * 2 + ["rehyat_hybrid_attn_fwd_phi"]
+    assert pq.dtype == BF and all(c[1][0].flags & rh.FLAG_PHI_BF16 for c in calls)
 
 
 def test_gradient_refusals(calls):

@@ -109,6 +109,44 @@ def test_phi_given_closed_form(shape, dtype):
     assert_close_partials(parts, ref_p, dtype)
 
 
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_phi_given_bf16_maps(shape, dtype):
+    """The maps given in bf16 (REHYAT_FLAG_PHI_BF16): equals the oracle's
+    phi-given forward on the same bf16-rounded maps."""
+    B, h, T, Hs, Ws, D, Dp, Tc, To, causal = shape
+    p = make_problem(batch=B, heads=h, T=T, Hs=Hs, Ws=Ws, D=D, Dp=Dp, Tc=Tc, To=To,
+                     causal=causal, dtype=dtype, dist="scaled", seed=450 + sum(shape[:9]))
+    fq, fk = _closed_form_phi(p)
+    fq16, fk16 = (_cuda32(f).to(torch.bfloat16) for f in (fq, fk))
+    rq, rk = (f.double().cpu().numpy() for f in (fq16, fk16))
+    ref_y, ref_p = hybrid_phi_given(p.q, p.k, p.v, rq, rk, T=p.T, HW=p.HW, Tc=p.Tc, To=p.To,
+                                    causal=p.causal)
+    dev = device_tensors(p)
+    y, parts = rh.hybrid_attn_phi(dev["q"], dev["k"], dev["v"], fq16, fk16, T=p.T, Hs=p.Hs,
+                                  Ws=p.Ws, Tc=p.Tc, To=p.To, causal=p.causal, debug=True,
+                                  force_simt=dtype == "f32")
+    torch.cuda.synchronize()
+    assert_close_y(y.double().cpu().numpy(), ref_y, dtype)
+    assert_close_partials({k: v.double().cpu().numpy() for k, v in parts.items()}, ref_p, dtype)
+
+
+@pytest.mark.parametrize("force_simt", [False, True])
+def test_feature_map_mlp_bf16_output_is_the_rounded_fp32_map(force_simt):
+    """REHYAT_FLAG_PHI_BF16 rounds the map the fp32 output holds (same
+    arithmetic, round to nearest even at the store): bit for bit."""
+    p = make_problem(batch=2, heads=2, T=3, Hs=7, Ws=9, D=128, Dp=128, Tc=1, To=0,
+                     causal=False, dtype="bf16", seed=77)
+    params = [_cuda32(a) for a in _mlp_params(2, 128, 256, 128, 78, scale=0.5)]
+    dev = device_tensors(p)
+    kw = dict(parts=2, T=p.T, Hs=p.Hs, Ws=p.Ws, force_simt=force_simt)
+    f32 = rh.feature_map_mlp(dev["q"], *params, **kw)
+    b16 = rh.feature_map_mlp(dev["q"], *params, out_dtype=torch.bfloat16, **kw)
+    torch.cuda.synchronize()
+    assert b16.dtype == torch.bfloat16
+    assert torch.equal(b16, f32.to(torch.bfloat16))
+
+
 @pytest.mark.parametrize("dtype,parts_n", [("bf16", 2), ("f32", 2), ("bf16", 4)])
 @pytest.mark.parametrize("causal", [False, True])
 def test_mlp_phi_end_to_end(dtype, parts_n, causal):
