@@ -309,25 +309,40 @@ def measure_phi_backward(rh, p, q, k, v, Wq, bq, Wk, bk, flush, stream, calls=3)
     dy = torch.randn(B, H, N, D, generator=g, device=dev)
     grads = {n: torch.empty_like(t) for n, t in (("dWq", Wq), ("dbq", bq), ("dWk", Wk), ("dbk", bk))}
     gs = rh.RehyatPhiGrad(*(grads[n].data_ptr() for n in ("dWq", "dbq", "dWk", "dbk")))
-    call = lambda: rh.rehyat_phi_bwd(params, q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                                     y.data_ptr(), dy.data_ptr(), den.data_ptr(), phi, gs,
-                                     ws.data_ptr(), ws.numel(), sh)
-    if call():
+    # The second form runs on the forward's workspace (REHYAT_FLAG_FWD_STATE):
+    # the backward reads the forward's linear-set state instead of repeating
+    # the state pass.  Every plain call rewrites that state with the same bits.
+    reuse = rh.make_params(batch=B, heads=H, T=p.T, Hs=p.Hs, Ws=p.Ws, D=D, Dp=p.Dp, Tc=p.Tc,
+                           To=p.To, causal=p.causal, in_dtype=rh.BF16, out_dtype=rh.F32,
+                           flags=rh.FLAG_FWD_STATE)
+    call = lambda prm: rh.rehyat_phi_bwd(prm, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                         y.data_ptr(), dy.data_ptr(), den.data_ptr(), phi, gs,
+                                         ws.data_ptr(), ws.numel(), sh)
+    if call(params):
         raise RuntimeError("rehyat_phi_bwd failed")
-    times = []
-    for _ in range(calls):
-        flush()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        call()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        times.append(e0.elapsed_time(e1))
-    ms = sum(times) / len(times)
+    ref = {n: t.clone() for n, t in grads.items()}
+    if call(reuse):
+        raise RuntimeError("rehyat_phi_bwd (forward's state) failed")
+    same = all(torch.equal(ref[n], grads[n]) for n in grads)
+
+    def timed(prm):
+        times = []
+        for _ in range(calls):
+            flush()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            call(prm)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1))
+        return sum(times) / len(times)
+    ms = timed(params)
+    ms_fs = timed(reuse)
     # Algorithmic FLOPs of the backward proper (per token and (b,h): u_q, dphi_q,
     # dW_q, G_t on the q side, u_k, dphi_k, dW_k on the k side, each 2*D*D'),
     # plus the state pass it repeats (phi_k and phi_k^T v: 4*D*D').
     flops = B * H * N * D * p.Dp * 2.0 * (7 + 2)
+    flops_fs = B * H * N * D * p.Dp * 2.0 * 7
     del y, nS, nL, ws, dy
     tflops = flops / (ms / 1e3) / 1e12
     if D == 128 and p.Dp == 128:  # q and k passes on tcgen05 (bf16 operands)
@@ -339,9 +354,13 @@ def measure_phi_backward(rh, p, q, k, v, Wq, bq, Wk, bk, flush, stream, calls=3)
         roof = {"bound": "alu", "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
                 "frac": tflops / FP32_ALU_TFLOPS,
                 "peak_source": "148 SMs x 128 fp32 FMA lanes x 2 x 1965 MHz"}
+    tf_fs = flops_fs / (ms_fs / 1e3) / 1e12
     return {"ms": ms, "calls": calls, "tflops": tflops, "roofline": roof,
+            "with_forward_state": {"ms": ms_fs, "tflops": tf_fs,
+                                   "frac": tf_fs / roof["peak"], "bitwise_equal": same},
             "what": "rehyat_phi_bwd (dW_q, db_q, dW_k, db_k) on the bench workload, bf16 "
-                    "q/k/v, fp32 y, dy, den; includes its state pass"}
+                    "q/k/v, fp32 y, dy, den; `ms` includes its state pass, "
+                    "`with_forward_state` reuses the forward's (REHYAT_FLAG_FWD_STATE)"}
 
 
 def measure_full_backward(rh, p, q, k, v, Wq, bq, Wk, bk, flush, stream, calls=3):
@@ -374,22 +393,29 @@ def measure_full_backward(rh, p, q, k, v, Wq, bq, Wk, bk, flush, stream, calls=3
     out = {n: torch.empty(B, H, N, D, device=dev) for n in ("dq", "dk", "dv")}
     grads = {n: torch.empty_like(t) for n, t in (("dWq", Wq), ("dbq", bq), ("dWk", Wk), ("dbk", bk))}
     gs = rh.RehyatPhiGrad(*(grads[n].data_ptr() for n in ("dWq", "dbq", "dWk", "dbk")))
-    call = lambda: rh.rehyat_hybrid_attn_bwd(
-        params, q.data_ptr(), k.data_ptr(), v.data_ptr(), phi, y.data_ptr(), dy.data_ptr(),
+    reuse = rh.make_params(batch=B, heads=H, T=p.T, Hs=p.Hs, Ws=p.Ws, D=D, Dp=p.Dp, Tc=p.Tc,
+                           To=p.To, causal=p.causal, in_dtype=rh.BF16, out_dtype=rh.F32,
+                           flags=rh.FLAG_FWD_STATE)
+    call = lambda prm: rh.rehyat_hybrid_attn_bwd(
+        prm, q.data_ptr(), k.data_ptr(), v.data_ptr(), phi, y.data_ptr(), dy.data_ptr(),
         c.data_ptr(), den.data_ptr(), out["dq"].data_ptr(), out["dk"].data_ptr(),
         out["dv"].data_ptr(), gs, ws.data_ptr(), ws.numel(), sh)
-    if call():
+    if call(params):
         raise RuntimeError("rehyat_hybrid_attn_bwd failed")
-    times = []
-    for _ in range(calls):
-        flush()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        call()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        times.append(e0.elapsed_time(e1))
-    ms = sum(times) / len(times)
+
+    def timed(prm):
+        times = []
+        for _ in range(calls):
+            flush()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            call(prm)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1))
+        return sum(times) / len(times)
+    ms = timed(params)
+    ms_fs = timed(reuse)
     # Algorithmic FLOPs: the softmax branch's backward, 10 D per (query,
     # window key) pair (S and dP recomputed, dV, dQ, dK), plus the feature-map
     # part (the phi-gradient extra's count) and the linear branch's token
@@ -405,8 +431,10 @@ def measure_full_backward(rh, p, q, k, v, Wq, bq, Wk, bk, flush, stream, calls=3
                          "frac": tflops / peaks["bf16_tflops"],
                          "peak_source": "measured bf16 burst (MEASURED_PEAKS.json)",
                          "work_per_call": f"{flops:.4e} FLOP"},
+            "with_forward_state": {"ms": ms_fs},
             "what": "rehyat_hybrid_attn_bwd (dq, dk, dv, dW_q, db_q, dW_k, db_k) on the bench "
-                    "workload, bf16 q/k/v, fp32 y, dy, c, den; includes its state pass"}
+                    "workload, bf16 q/k/v, fp32 y, dy, c, den; `ms` includes its state pass, "
+                    "`with_forward_state` reuses the forward's (REHYAT_FLAG_FWD_STATE)"}
 
 
 def measure_general_phi(rh, p, q, k, v, flush, stream, calls=3):

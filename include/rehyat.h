@@ -94,6 +94,23 @@ typedef enum { REHYAT_F32 = 0, REHYAT_BF16 = 1 } rehyat_dtype;
                                     Halves the maps' memory traffic; the
                                     tensor-core forward rounds phi_k to bf16
                                     anyway.  Ignored by other entry points. */
+#define REHYAT_FLAG_FWD_STATE 16 /* backward entry points (rehyat_phi_bwd,
+                                    rehyat_hybrid_attn_bwd): the workspace is
+                                    the one the forward ran on
+                                    (rehyat_hybrid_attn_fwd, or rehyat_fwd_state,
+                                    with the same k, v, phi and params apart
+                                    from this flag), unchanged since, so it
+                                    already holds the per-chunk linear-set
+                                    states S_L, z_L and the weight images; the
+                                    backward reads them instead of recomputing
+                                    them (the forward's state stage).  Size the
+                                    workspace with the backward's
+                                    *_workspace_bytes: the forward accepts the
+                                    larger buffer and uses its front part, which
+                                    the backward's layout shares.  A workspace
+                                    that does not hold that state gives wrong
+                                    gradients; nothing detects it.  Ignored by
+                                    other entry points. */
 
 typedef struct {
   int batch, heads;   /* B >= 1, h >= 1 */
@@ -357,7 +374,10 @@ REHYAT_API size_t rehyat_phi_bwd_workspace_bytes(const rehyat_params* p);
  * gradients are overwritten, not accumulated; fp32 arithmetic; the
  * reductions run in a fixed order, so repeated calls agree bit for bit.
  * Pointers: q, k, v, y, dy, workspace 16-byte aligned; den and the gradient
- * arrays 4-byte aligned.  Errors as for rehyat_hybrid_attn_fwd. */
+ * arrays 4-byte aligned.  Errors as for rehyat_hybrid_attn_fwd.
+ * The call first recomputes the forward's linear-set state into the
+ * workspace; with REHYAT_FLAG_FWD_STATE it takes that state from the
+ * forward's workspace instead (same results bit for bit). */
 REHYAT_API rehyat_status rehyat_phi_bwd(const rehyat_params* p, const void* q, const void* k,
                                         const void* v, const float* y, const float* dy,
                                         const float* den, const rehyat_phi* phi,
@@ -395,7 +415,8 @@ REHYAT_API size_t rehyat_hybrid_attn_bwd_workspace_bytes(const rehyat_params* p)
  * No atomics, so repeated calls agree bit for bit.
  * Pointers: q, k, v, y, dy, dq, dk, dv, workspace 16-byte aligned; c, den and
  * the parameter gradients 4-byte aligned.  Errors as for
- * rehyat_hybrid_attn_fwd; REHYAT_FLAG_FP8_QK is refused (UNSUPPORTED). */
+ * rehyat_hybrid_attn_fwd; REHYAT_FLAG_FP8_QK is refused (UNSUPPORTED).
+ * REHYAT_FLAG_FWD_STATE as for rehyat_phi_bwd. */
 REHYAT_API rehyat_status rehyat_hybrid_attn_bwd(const rehyat_params* p, const void* q,
                                                 const void* k, const void* v,
                                                 const rehyat_phi* phi, const float* y,

@@ -25,6 +25,7 @@ from typing import Optional
 __all__ = [
     "RehyatParams", "RehyatPhi", "RehyatDebug", "RehyatError", "lib", "lib_path",
     "EXPORTED_SYMBOLS", "F32", "BF16", "FLAG_FORCE_SIMT", "FLAG_FP8_QK", "FLAG_PHI_BF16",
+    "FLAG_FWD_STATE",
     "rehyat_workspace_bytes", "rehyat_hybrid_attn_fwd", "rehyat_fwd_state", "rehyat_fwd_attn",
     "rehyat_softmax_attn_fwd", "rehyat_state_bytes", "rehyat_state_init", "rehyat_step_workspace_bytes",
     "rehyat_chunk_step", "rehyat_device_error_flags", "rehyat_attn_path",
@@ -34,7 +35,7 @@ __all__ = [
     "rehyat_feature_map_mlp_workspace_bytes", "rehyat_host_workspace_bytes",
     "rehyat_hybrid_attn_fwd_host", "hybrid_attn_host",
     "make_params", "hybrid_attn", "hybrid_attn_phi", "feature_map_mlp", "softmax_attn",
-    "phi_grad", "StreamingState", "rehyat_hybrid_attn_bwd_workspace_bytes",
+    "phi_grad", "bwd_workspace", "StreamingState", "rehyat_hybrid_attn_bwd_workspace_bytes",
     "rehyat_hybrid_attn_bwd", "hybrid_attn_bwd", "rehyat_denominator_report",
     "rehyat_step_key_split",
 ]
@@ -44,6 +45,7 @@ FLAG_FORCE_SIMT = 1
 FLAG_ONE_TILE = 2
 FLAG_FP8_QK = 4
 FLAG_PHI_BF16 = 8
+FLAG_FWD_STATE = 16
 
 STATUS = {0: "REHYAT_OK", 1: "REHYAT_ERR_INVALID_ARG", 2: "REHYAT_ERR_UNSUPPORTED",
           3: "REHYAT_ERR_MISALIGNED", 4: "REHYAT_ERR_WORKSPACE", 5: "REHYAT_ERR_CUDA",
@@ -589,11 +591,33 @@ def hybrid_attn_phi(q, k, v, phi_q, phi_k, *, T, Hs, Ws, Tc, To, causal, out_dty
     return (y, dbg_t) if debug else y
 
 
+def bwd_workspace(q, Wq, *, T, Hs, Ws, Tc, To, causal, full=True, force_simt=False):
+    """A device workspace large enough for the forward and for the backward
+    (``hybrid_attn_bwd`` if ``full``, else ``phi_grad``) of q's shape: pass it
+    to ``hybrid_attn`` and then, with ``state_from_forward=True``, to the
+    backward, which reuses the forward's linear-set state."""
+    torch = _torch()
+    B, H, N, D = q.shape
+    _check_tokens(N, T, Hs, Ws)
+    p = make_params(batch=B, heads=H, T=T, Hs=Hs, Ws=Ws, D=D, Dp=2 * Wq.shape[-1], Tc=Tc,
+                    To=To, causal=causal, in_dtype=_dtype_code(q.dtype), out_dtype=F32,
+                    flags=FLAG_FORCE_SIMT if force_simt else 0)
+    nbytes = (rehyat_hybrid_attn_bwd_workspace_bytes(p) if full
+              else rehyat_phi_bwd_workspace_bytes(p))
+    if nbytes == 0:
+        raise RehyatError(1, "rehyat_*_bwd_workspace_bytes")
+    return torch.empty(max(nbytes, rehyat_workspace_bytes(p)), dtype=torch.uint8,
+                       device=q.device)
+
+
 def phi_grad(q, k, v, y, dy, den, Wq, bq, Wk, bk, *, T, Hs, Ws, Tc, To, causal, scale=0.0,
-             force_simt=False, workspace=None, stream=None):
+             force_simt=False, workspace=None, stream=None, state_from_forward=False):
     """Gradients of L with respect to the phi parameters, given the forward's
     q, k, v, its fp32 output y, dy = dL/dy (fp32) and den = n^S + n^L per
     query (``parts["nS"] + parts["nL"]`` of ``hybrid_attn(..., debug=True)``).
+    ``state_from_forward`` (REHYAT_FLAG_FWD_STATE): ``workspace`` is the
+    buffer the forward ran on (from ``bwd_workspace(..., full=False)``), so
+    its linear-set state is reused instead of recomputed.
     Returns dict(dWq, dbq, dWk, dbk) shaped like the parameters."""
     torch = _torch()
     _check_qkv(q, k, v)
@@ -608,9 +632,12 @@ def phi_grad(q, k, v, y, dy, den, Wq, bq, Wk, bk, *, T, Hs, Ws, Tc, To, causal, 
     _check_out(dy, (B, H, N, D), torch.float32, q.device, "dy")
     _check_out(den, (B, H, N), torch.float32, q.device, "den")
     phi = _phi_struct(Wq, bq, Wk, bk, heads=H, D=D, Dp=Dp, device=q.device)
+    _need(not state_from_forward or workspace is not None,
+          "state_from_forward needs the forward's workspace")
     p = make_params(batch=B, heads=H, T=T, Hs=Hs, Ws=Ws, D=D, Dp=Dp, Tc=Tc, To=To,
                     causal=causal, in_dtype=_dtype_code(q.dtype), out_dtype=F32, scale=scale,
-                    flags=FLAG_FORCE_SIMT if force_simt else 0)
+                    flags=(FLAG_FORCE_SIMT if force_simt else 0) |
+                    (FLAG_FWD_STATE if state_from_forward else 0))
     nbytes = rehyat_phi_bwd_workspace_bytes(p)
     if nbytes == 0:
         raise RehyatError(1, "rehyat_phi_bwd_workspace_bytes")
@@ -629,13 +656,16 @@ def phi_grad(q, k, v, y, dy, den, Wq, bq, Wk, bk, *, T, Hs, Ws, Tc, To, causal, 
 
 
 def hybrid_attn_bwd(q, k, v, y, dy, c, den, Wq, bq, Wk, bk, *, T, Hs, Ws, Tc, To, causal,
-                    scale=0.0, force_simt=False, workspace=None, stream=None):
+                    scale=0.0, force_simt=False, workspace=None, stream=None,
+                    state_from_forward=False):
     """Full backward: gradients of L with respect to q, k, v and the phi
     parameters, given the forward's q, k, v, its fp32 output y, dy = dL/dy
     (fp32), and per query the stabiliser c and den = n^S + n^L
     (``parts["c"]`` and ``parts["nS"] + parts["nL"]`` of
-    ``hybrid_attn(..., debug=True)``).  Returns dict(dq, dk, dv (fp32, shaped
-    like q), dWq, dbq, dWk, dbk (shaped like the parameters))."""
+    ``hybrid_attn(..., debug=True)``).  ``state_from_forward`` as for
+    ``phi_grad`` (the shared workspace from ``bwd_workspace(...)``).
+    Returns dict(dq, dk, dv (fp32, shaped like q), dWq, dbq, dWk, dbk (shaped
+    like the parameters))."""
     torch = _torch()
     _check_qkv(q, k, v)
     _check_current_device(q.device)
@@ -650,9 +680,12 @@ def hybrid_attn_bwd(q, k, v, y, dy, c, den, Wq, bq, Wk, bk, *, T, Hs, Ws, Tc, To
     _check_out(c, (B, H, N), torch.float32, q.device, "c")
     _check_out(den, (B, H, N), torch.float32, q.device, "den")
     phi = _phi_struct(Wq, bq, Wk, bk, heads=H, D=D, Dp=Dp, device=q.device)
+    _need(not state_from_forward or workspace is not None,
+          "state_from_forward needs the forward's workspace")
     p = make_params(batch=B, heads=H, T=T, Hs=Hs, Ws=Ws, D=D, Dp=Dp, Tc=Tc, To=To,
                     causal=causal, in_dtype=_dtype_code(q.dtype), out_dtype=F32, scale=scale,
-                    flags=FLAG_FORCE_SIMT if force_simt else 0)
+                    flags=(FLAG_FORCE_SIMT if force_simt else 0) |
+                    (FLAG_FWD_STATE if state_from_forward else 0))
     nbytes = rehyat_hybrid_attn_bwd_workspace_bytes(p)
     if nbytes == 0:
         raise RehyatError(1, "rehyat_hybrid_attn_bwd_workspace_bytes")

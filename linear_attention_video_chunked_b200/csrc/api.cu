@@ -629,8 +629,10 @@ rehyat_status phi_bwd_impl(const rehyat_params* p, const void* q, const void* k,
   if (ws_bytes < base + (have_prep ? 0 : phi_bwd_prep_bytes(p))) return REHYAT_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
-  // The linear-set state of every chunk, as the forward computes it.
-  if ((st = state_pass(p, k, v, phi, ws, s)) != REHYAT_OK) return st;
+  // The linear-set state of every chunk, as the forward computes it (or, with
+  // REHYAT_FLAG_FWD_STATE, as the forward left it in this workspace).
+  if (!(p->flags & REHYAT_FLAG_FWD_STATE) && (st = state_pass(p, k, v, phi, ws, s)) != REHYAT_OK)
+    return st;
   const FwdWorkspace w = fwd_layout(p);
   PhiBwdArgs a;
   a.q = q; a.k = k; a.v = v; a.y = y; a.dy = dy; a.den = den;

@@ -268,35 +268,54 @@ __global__ void phi_bwd_gsel_kernel(BwdParams P) {
 // block takes kGhatCols consecutive elements; its threads first form G_t of
 // every chunk for them (the sum of the QS partials, in order) in shared
 // memory, then Ghat_s of every slice (chunks in order).  The same sums in the
-// same order as (a) and (b), with each partial read once.
-constexpr int kGhatChunks = 48, kGhatCols = 128;
+// same order as (a) and (b), with each partial read once.  A thread owns four
+// consecutive elements (16-byte loads and stores; partial sizes, offsets and
+// the element count per (b, h) are multiples of four floats) and issues four
+// partials' loads before it adds them, in order.
+constexpr int kGhatChunks = 48, kGhatCols = 128, kGhatVec = kGhatCols / 4;
 __global__ void __launch_bounds__(256) phi_bwd_ghat_fused_kernel(BwdParams P) {
-  __shared__ float G[kGhatChunks][kGhatCols];
+  __shared__ float4 G[kGhatChunks][kGhatVec];
   const int D = P.D;
   const long long n = static_cast<long long>(kPiece) * D + kPiece;
   const long long e0 = static_cast<long long>(blockIdx.x) * kGhatCols;
   const long long psz = qpart_size(D);
   const float* g = P.qpart + static_cast<long long>(blockIdx.z) * P.nchunks * P.QS * psz +
                    static_cast<long long>(D) * kPiece + kPiece + e0;
-  for (int idx = threadIdx.x; idx < P.nchunks * kGhatCols; idx += blockDim.x) {
-    const int t = idx / kGhatCols, j = idx % kGhatCols;
-    float acc = 0.f;
-    if (e0 + j < n)
-      for (int qs = 0; qs < P.QS; ++qs) acc += g[(static_cast<long long>(t) * P.QS + qs) * psz + j];
-    G[t][j] = acc;
+  auto add4 = [](float4& a, const float4 b) {
+    a.x += b.x;
+    a.y += b.y;
+    a.z += b.z;
+    a.w += b.w;
+  };
+  for (int idx = threadIdx.x; idx < P.nchunks * kGhatVec; idx += blockDim.x) {
+    const int t = idx / kGhatVec, j4 = idx % kGhatVec;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (e0 + 4 * j4 < n) {
+      const float* src = g + static_cast<long long>(t) * P.QS * psz + 4 * j4;
+      for (int qs0 = 0; qs0 < P.QS; qs0 += 4) {
+        float4 x[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (qs0 + u < P.QS) x[u] = __ldg(reinterpret_cast<const float4*>(src + (qs0 + u) * psz));
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (qs0 + u < P.QS) add4(acc, x[u]);
+      }
+    }
+    G[t][j4] = acc;
   }
   __syncthreads();
   float* out = P.ghat + static_cast<long long>(blockIdx.z) * P.T * n + e0;
-  for (int idx = threadIdx.x; idx < P.T * kGhatCols; idx += blockDim.x) {
-    const int s = idx / kGhatCols, j = idx % kGhatCols;
-    if (e0 + j >= n) continue;
-    float acc = 0.f;
+  for (int idx = threadIdx.x; idx < P.T * kGhatVec; idx += blockDim.x) {
+    const int s = idx / kGhatVec, j4 = idx % kGhatVec;
+    if (e0 + 4 * j4 >= n) continue;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int t = 0; t < P.nchunks; ++t) {
       const int first = t * P.Tc, end = min(P.T, first + P.Tc);
       const int w = max(first - P.To, 0);
-      if (P.causal ? s < w : (s < w || s >= end)) acc += G[t][j];
+      if (P.causal ? s < w : (s < w || s >= end)) add4(acc, G[t][j4]);
     }
-    out[static_cast<long long>(s) * n + j] = acc;
+    *reinterpret_cast<float4*>(out + static_cast<long long>(s) * n + 4 * j4) = acc;
   }
 }
 
@@ -416,10 +435,20 @@ __global__ void phi_bwd_reduce_kernel(BwdParams P, float* dWq, float* dbq, float
   const float* base = qside ? P.qpart : P.kpart;
   const long long off = is_b ? static_cast<long long>(D) * kPiece + c
                              : static_cast<long long>(d) * kPiece + c;
+  // Eight partials' loads in flight before they are added, in order.
   float acc = 0.f;
   for (int b = 0; b < batch; ++b) {
     const long long z = static_cast<long long>(b * P.heads + h) * P.FP + pf;
-    for (int i = 0; i < nsets; ++i) acc += base[(z * nsets + i) * psz + off];
+    const float* src = base + z * nsets * psz + off;
+    int i = 0;
+    for (; i + 8 <= nsets; i += 8) {
+      float x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) x[u] = __ldg(src + (i + u) * psz);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) acc += x[u];
+    }
+    for (; i < nsets; ++i) acc += __ldg(src + i * psz);
   }
   if (is_b)
     (qside ? dbq : dbk)[b_at(h, Dp, f)] = acc;

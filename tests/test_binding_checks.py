@@ -203,6 +203,28 @@ def test_full_backward_refuses_malformed_tensors(calls, bad):
     assert calls == []
 
 
+def test_backward_with_the_forwards_state_shares_one_workspace(calls):
+    # forward, then both backward entry points on the same buffer, the
+    # backward calls with REHYAT_FLAG_FWD_STATE; the buffer holds both layouts.
+    q, k, v = qkv()
+    prm = phi_params()
+    ws = rh.bwd_workspace(q, prm[0], **GEOM)
+    y, parts = rh.hybrid_attn(q, k, v, *prm, **GEOM, debug=True, workspace=ws)
+    dy, den = FakeTensor(q.shape, F32), FakeTensor(q.shape[:3], F32)
+    rh.phi_grad(q, k, v, y, dy, den, *prm, **GEOM, workspace=ws, state_from_forward=True)
+    rh.hybrid_attn_bwd(q, k, v, y, dy, den, den, *prm, **GEOM, workspace=ws,
+                       state_from_forward=True)
+    (f, af), (g, ag), (b, ab) = calls
+    assert (f, g, b) == ("rehyat_hybrid_attn_fwd", "rehyat_phi_bwd", "rehyat_hybrid_attn_bwd")
+    assert af[6] == ag[9] == ab[13] == ws.data_ptr()
+    assert af[7] == ag[10] == ab[14] == ws.numel()
+    assert not af[0].flags & rh.FLAG_FWD_STATE
+    assert ag[0].flags & rh.FLAG_FWD_STATE and ab[0].flags & rh.FLAG_FWD_STATE
+    assert ws.numel() >= max(rh.rehyat_workspace_bytes(af[0]),
+                             rh.rehyat_hybrid_attn_bwd_workspace_bytes(ab[0]),
+                             rh.rehyat_phi_bwd_workspace_bytes(ag[0]))
+
+
 def test_softmax_and_streaming_reach_the_abi(calls):
     q, k, v = qkv(shape=(1, 2, 3 * 10 * 30, 128))
     rh.softmax_attn(q, k, v)
@@ -369,6 +391,12 @@ def test_gradient_refusals(calls):
     with pytest.raises(TypeError):
         rh.phi_grad(q, k, v, FakeTensor(q.shape, BF), FakeTensor(q.shape, F32), den,
                     *phi_params(), **GEOM)
+    with pytest.raises(ValueError):        # the forward's state lives in its workspace
+        rh.phi_grad(q, k, v, y, FakeTensor(q.shape, F32), den, *phi_params(), **GEOM,
+                    state_from_forward=True)
+    with pytest.raises(ValueError):
+        rh.hybrid_attn_bwd(q, k, v, y, FakeTensor(q.shape, F32), den, den, *phi_params(),
+                           **GEOM, state_from_forward=True)
     assert calls == []
 
 

@@ -175,3 +175,28 @@ def test_full_bwd_bench_layer_sampled_heads():
     dy = np.random.default_rng(22).standard_normal(np.shape(p.q)).astype(np.float32)
     heads = [2, 7]
     _check(_gpu(p, dy, force_simt=False), _ref(p, dy, heads), 3e-2, p, heads)
+
+
+@pytest.mark.parametrize("force_simt", [False, True], ids=["tc", "simt"])
+def test_full_bwd_with_the_forwards_state_is_bitwise_equal(force_simt):
+    """REHYAT_FLAG_FWD_STATE: the full backward on the forward's workspace
+    equals the one that recomputes the linear-set state, bit for bit."""
+    p = make_problem(batch=1, heads=2, T=7, Hs=10, Ws=13, D=128, Dp=128, Tc=3, To=2,
+                     causal=True, dtype="bf16", seed=23)
+    dy = np.random.default_rng(23).standard_normal(np.shape(p.q))
+    dev = device_tensors(p)
+    kw = dict(T=p.T, Hs=p.Hs, Ws=p.Ws, Tc=p.Tc, To=p.To, causal=p.causal)
+    prm = [dev[n] for n in ("Wq", "bq", "Wk", "bk")]
+    ws = rh.bwd_workspace(dev["q"], dev["Wq"], force_simt=force_simt, **kw)
+    y, parts = rh.hybrid_attn(dev["q"], dev["k"], dev["v"], *prm, debug=True,
+                              force_simt=force_simt, workspace=ws, **kw)
+    den = (parts["nS"] + parts["nL"]).contiguous()
+    dyt = torch.tensor(dy, dtype=torch.float32, device="cuda")
+    args = (dev["q"], dev["k"], dev["v"], y, dyt, parts["c"].contiguous(), den, *prm)
+    a = rh.hybrid_attn_bwd(*args, force_simt=force_simt, **kw)
+    b = rh.hybrid_attn_bwd(*args, force_simt=force_simt, workspace=ws, state_from_forward=True,
+                           **kw)
+    torch.cuda.synchronize()
+    for n in TOKEN + PARAM:
+        assert torch.equal(a[n], b[n]), n
+    assert rh.rehyat_device_error_flags() == 0

@@ -143,3 +143,32 @@ def test_phi_grad_tensor_core_bench_layer_sampled_heads():
     heads = [3, 9]
     got = _gpu_grads(p, dy, force_simt=False)
     _check(got, _ref(p, dy, heads), 3e-2, heads)
+
+
+@pytest.mark.parametrize("force_simt", [False, True], ids=["tc", "simt"])
+def test_phi_grad_with_the_forwards_state_is_bitwise_equal(force_simt):
+    """REHYAT_FLAG_FWD_STATE: the backward run on the forward's workspace reads
+    the forward's S_L, z_L and weight images and gives the same gradients bit
+    for bit as the call that recomputes them; on a zeroed workspace the same
+    call gives different gradients (so the state is read, not recomputed)."""
+    p = make_problem(batch=2, heads=2, T=5, Hs=7, Ws=9, D=128, Dp=128, Tc=2, To=1,
+                     causal=False, dtype="bf16", seed=12)
+    dy = np.random.default_rng(12).standard_normal(np.shape(p.q))
+    dev = device_tensors(p)
+    kw = dict(T=p.T, Hs=p.Hs, Ws=p.Ws, Tc=p.Tc, To=p.To, causal=p.causal)
+    prm = [dev[n] for n in ("Wq", "bq", "Wk", "bk")]
+    ws = rh.bwd_workspace(dev["q"], dev["Wq"], full=False, force_simt=force_simt, **kw)
+    y, parts = rh.hybrid_attn(dev["q"], dev["k"], dev["v"], *prm, debug=True,
+                              force_simt=force_simt, workspace=ws, **kw)
+    den = (parts["nS"] + parts["nL"]).contiguous()
+    dyt = torch.tensor(dy, dtype=torch.float32, device="cuda")
+    args = (dev["q"], dev["k"], dev["v"], y, dyt, den, *prm)
+    a = rh.phi_grad(*args, force_simt=force_simt, **kw)
+    b = rh.phi_grad(*args, force_simt=force_simt, workspace=ws, state_from_forward=True, **kw)
+    ws.zero_()
+    z = rh.phi_grad(*args, force_simt=force_simt, workspace=ws, state_from_forward=True, **kw)
+    torch.cuda.synchronize()
+    for n in NAMES:
+        assert torch.equal(a[n], b[n]), n
+    assert any(not torch.equal(a[n], z[n]) for n in NAMES)
+    assert rh.rehyat_device_error_flags() == 0
