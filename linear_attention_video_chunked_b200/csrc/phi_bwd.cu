@@ -413,14 +413,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1) phi_bwd_k_kernel(BwdParams P) 
 }
 
 // ---------------------------------------------------------------- pass 4
-// One thread per parameter element of one head: the sum over batch, chunks
-// (slices) and row ranges of the partials, in a fixed order.
-// grid (ceil(heads * (D*Dp + Dp) / 256), 2): y = 0 -> (W_q, b_q), 1 -> (W_k, b_k).
+// One thread per four consecutive parameter elements of one head (four
+// features of one W row, or of b, inside one feature piece: D' and the piece
+// width are multiples of four): the sum over batch, chunks (slices) and row
+// ranges of the partials, in a fixed order, read as 16-byte vectors with
+// eight partials' loads in flight before they are added.
+// grid (ceil(heads * (D*Dp + Dp) / 1024), 2): y = 0 -> (W_q, b_q), 1 -> (W_k, b_k).
 __global__ void phi_bwd_reduce_kernel(BwdParams P, float* dWq, float* dbq, float* dWk, float* dbk,
                                       int batch) {
   const int D = P.D, Dp = P.Dp, pw = Dp < kPiece ? Dp : kPiece;
   const long long per_head = static_cast<long long>(D) * Dp + Dp;
-  const long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long e = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
   if (e >= per_head * P.heads) return;
   const int h = static_cast<int>(e / per_head);
   const long long rem = e % per_head;
@@ -435,25 +438,34 @@ __global__ void phi_bwd_reduce_kernel(BwdParams P, float* dWq, float* dbq, float
   const float* base = qside ? P.qpart : P.kpart;
   const long long off = is_b ? static_cast<long long>(D) * kPiece + c
                              : static_cast<long long>(d) * kPiece + c;
-  // Eight partials' loads in flight before they are added, in order.
-  float acc = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  auto add4 = [&](const float4 x) {
+    acc.x += x.x;
+    acc.y += x.y;
+    acc.z += x.z;
+    acc.w += x.w;
+  };
   for (int b = 0; b < batch; ++b) {
     const long long z = static_cast<long long>(b * P.heads + h) * P.FP + pf;
     const float* src = base + z * nsets * psz + off;
     int i = 0;
     for (; i + 8 <= nsets; i += 8) {
-      float x[8];
+      float4 x[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) x[u] = __ldg(src + (i + u) * psz);
+      for (int u = 0; u < 8; ++u) x[u] = __ldg(reinterpret_cast<const float4*>(src + (i + u) * psz));
 #pragma unroll
-      for (int u = 0; u < 8; ++u) acc += x[u];
+      for (int u = 0; u < 8; ++u) add4(x[u]);
     }
-    for (; i < nsets; ++i) acc += __ldg(src + i * psz);
+    for (; i < nsets; ++i) add4(__ldg(reinterpret_cast<const float4*>(src + i * psz)));
   }
-  if (is_b)
-    (qside ? dbq : dbk)[b_at(h, Dp, f)] = acc;
-  else
-    (qside ? dWq : dWk)[w_at(h, D, Dp, d, f)] = acc;
+  const float v[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    if (is_b)
+      (qside ? dbq : dbk)[b_at(h, Dp, f + u)] = v[u];
+    else
+      (qside ? dWq : dWk)[w_at(h, D, Dp, d, f + u)] = v[u];
+  }
 }
 
 template <int D>
@@ -473,7 +485,7 @@ cudaError_t launch_bwd_d(const BwdParams& bp, const PhiBwdArgs& a, cudaStream_t 
   launch_ghat(bp, s);
   phi_bwd_k_kernel<D><<<dim3(bp.KS, bp.T, bp.BH * bp.FP), kBwdThreads, smk, s>>>(bp);
   const long long nr = (static_cast<long long>(D) * bp.Dp + bp.Dp) * bp.heads;
-  phi_bwd_reduce_kernel<<<dim3(static_cast<unsigned>((nr + 255) / 256), 2), 256, 0, s>>>(
+  phi_bwd_reduce_kernel<<<dim3(static_cast<unsigned>((nr / 4 + 255) / 256), 2), 256, 0, s>>>(
       bp, a.dWq, a.dbq, a.dWk, a.dbk, a.batch);
   return cudaGetLastError();
 }
@@ -535,7 +547,7 @@ cudaError_t launch_phi_bwd(const PhiBwdArgs& a, cudaStream_t s) {
     e = launch_phi_bwd_tc(t, s);
     if (e != cudaSuccess) return e;
     const long long nr = (static_cast<long long>(a.D) * bp.Dp + bp.Dp) * bp.heads;
-    phi_bwd_reduce_kernel<<<dim3(static_cast<unsigned>((nr + 255) / 256), 2), 256, 0, s>>>(
+    phi_bwd_reduce_kernel<<<dim3(static_cast<unsigned>((nr / 4 + 255) / 256), 2), 256, 0, s>>>(
         bp, a.dWq, a.dbq, a.dWk, a.dbk, a.batch);
     return cudaGetLastError();
   }
