@@ -847,7 +847,9 @@ def run_gpu(args, world, rank, local):
     dev = torch.device("cuda", local)
     rh.lib()
 
-    p = config_problem(WORKLOAD)
+    # --batch/--heads draw a smaller case of the same layer (profiler captures).
+    p = config_problem(WORKLOAD, **{k: v for k, v in (("batch", args.batch), ("heads", args.heads))
+                                    if v is not None})
     B, H, N, D = p.q.shape
     T, HW, Dp = p.T, p.HW, p.Dp
     bf = torch.bfloat16
@@ -1061,6 +1063,10 @@ def main(argv=None):
                          "general feature maps, streaming)")
     ap.add_argument("--extras", default=None,
                     help="comma-separated subset of " + ",".join(EXTRAS))
+    ap.add_argument("--batch", type=int, default=None,
+                    help="batch of a smaller case of the layer (default: the workload's 2)")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="heads of a smaller case of the layer (default: the workload's 12)")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     world, rank, local = dist_setup()
