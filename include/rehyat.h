@@ -297,9 +297,12 @@ REHYAT_API size_t rehyat_host_workspace_bytes(const rehyat_params* p, int heads_
 /* rehyat_hybrid_attn_fwd with q, k, v (p->in_dtype) and y (p->out_dtype) in
  * HOST memory, same [B][h][N][D] layouts; phi and workspace on the device.
  * Host buffers should be page-locked (cudaHostAlloc / cudaHostRegister):
- * pageable memory still works but its copies do not overlap.  Slab s
- * (batch s / G, heads (s mod G) * heads_per_slab ..., G groups of heads)
- * goes through device slot s mod 3: upload on an internal copy stream, the
+ * pageable memory still works but its copies do not overlap.  Slabs are
+ * runs of heads_per_slab consecutive heads of one batch element, in (batch,
+ * head) order, except that the first and the last slab of the call take
+ * ceil(heads_per_slab / 2) heads (their upload and download overlap no
+ * kernel, so shorter ones shorten the call).  Slab s goes through device
+ * slot s mod 3: upload on an internal copy stream, the
  * forward on `stream`, download on a second internal copy stream, ordered
  * by events.  The copies start after the work already on `stream`, and
  * `stream` waits for the last download: synchronising `stream` makes y

@@ -11,11 +11,15 @@
 // second copy stream, so the upload of slab s + 1, the forward of slab s and
 // the download of slab s - 1 proceed together (PCIe is full duplex).
 // Events order the three streams; each slot is reused only after the
-// forward has read its inputs and the download has read its output.
+// forward has read its inputs and the download has read its output.  The
+// first and the last slab of a call take half the heads (rounded up): the
+// first upload and the last download overlap nothing, so shorter ones start
+// the kernels earlier and end the call sooner.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
 #include <mutex>
+#include <vector>
 
 #include "internal.h"
 
@@ -63,6 +67,33 @@ rehyat_params slab_params(const rehyat_params* p, int heads) {
   s.batch = 1;
   s.heads = heads;
   return s;
+}
+
+// One slab: heads [h0, h0 + hn) of batch element b.
+struct Slab {
+  int b, h0, hn;
+};
+
+// The slabs of a call in order: per_slab heads each within a batch element,
+// except that the first slab of the call and the last one hold
+// ceil(per_slab / 2) heads.
+std::vector<Slab> slab_list(int batch, int heads, int per_slab) {
+  const int ramp = (per_slab + 1) / 2;
+  std::vector<Slab> out;
+  for (int b = 0; b < batch; ++b)
+    for (int h = 0; h < heads;) {
+      int hn = out.empty() ? ramp : per_slab;
+      hn = heads - h < hn ? heads - h : hn;
+      out.push_back(Slab{b, h, hn});
+      h += hn;
+    }
+  Slab& last = out.back();
+  if (last.hn > ramp) {
+    const Slab tail{last.b, last.h0 + last.hn - ramp, ramp};
+    last.hn -= ramp;
+    out.push_back(tail);
+  }
+  return out;
 }
 
 SlabLayout slab_layout(const rehyat_params* p, int heads_per_slab) {
@@ -125,8 +156,13 @@ rehyat_status rehyat_hybrid_attn_fwd_host(const rehyat_params* p, const void* q,
   const size_t phiW = static_cast<size_t>(p->D) * p->Dp;  // floats of W per head (both parts)
   char* ws = static_cast<char*>(workspace);
   char* fwd_ws = ws + kSlots * L.slot_bytes;
-  const int groups = (p->heads + L.per_slab - 1) / L.per_slab;
-  const int nslabs = p->batch * groups;
+  std::vector<Slab> slabs;
+  try {
+    slabs = slab_list(p->batch, p->heads, L.per_slab);
+  } catch (...) {  // host allocation failure
+    e = cudaErrorMemoryAllocation;
+  }
+  const int nslabs = static_cast<int>(slabs.size());
   rehyat_status st = REHYAT_OK;
 
   // The copy streams start after the work already on the caller's stream.
@@ -135,8 +171,7 @@ rehyat_status rehyat_hybrid_attn_fwd_host(const rehyat_params* p, const void* q,
   if (e == cudaSuccess) e = cudaStreamWaitEvent(down, start, 0);
   for (int sl = 0; sl < nslabs && e == cudaSuccess && st == REHYAT_OK; ++sl) {
     const int slot = sl % kSlots;
-    const int b = sl / groups, h0 = (sl % groups) * L.per_slab;
-    const int hn = p->heads - h0 < L.per_slab ? p->heads - h0 : L.per_slab;
+    const int b = slabs[sl].b, h0 = slabs[sl].h0, hn = slabs[sl].hn;
     const size_t head_index = static_cast<size_t>(b) * p->heads + h0;
     char* dq = ws + slot * L.slot_bytes;
     char* dk = dq + L.in_bytes;

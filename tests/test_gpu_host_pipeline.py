@@ -48,6 +48,21 @@ def test_host_pipeline_equals_device_forward(dtype, causal, per_slab):
     assert torch.equal(y, ref)
 
 
+@pytest.mark.parametrize("per_slab", [3, 4])
+def test_host_pipeline_uneven_slabs(per_slab):
+    # B = 2, h = 5: the call's first and last slabs take ceil(per_slab / 2)
+    # heads, the others per_slab or the rest of a batch element's heads.
+    p = make_problem(batch=2, heads=5, T=4, Hs=6, Ws=11, D=128, Dp=128, Tc=2, To=1,
+                     causal=False, dtype="bf16", dist="scaled", seed=95 + per_slab)
+    dev = device_tensors(p)
+    ref = _device_y(p, dev)
+    host = {n: dev[n].cpu().pin_memory() for n in ("q", "k", "v")}
+    y = rh.hybrid_attn_host(host["q"], host["k"], host["v"], dev["Wq"], dev["bq"], dev["Wk"],
+                            dev["bk"], T=p.T, Hs=p.Hs, Ws=p.Ws, Tc=p.Tc, To=p.To,
+                            causal=p.causal, heads_per_slab=per_slab)
+    assert torch.equal(y, ref)
+
+
 def test_host_pipeline_full_size_matches_device():
     """The bench layer (B = 2, h = 12, 21 x 30 x 52, bidirectional), two heads
     per slab, in the configuration the end-to-end measurement uses."""
