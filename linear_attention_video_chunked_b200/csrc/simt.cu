@@ -452,6 +452,67 @@ __global__ void scan_regs_kernel(const float4* __restrict__ P, const float4* __r
   }
 }
 
+// Chunk scan for at most kScanAcc chunks (any T): each thread keeps one
+// accumulator per chunk for its four elements and streams the per-slice
+// states in slice order, kScanBatch slices' loads in flight at a time, adding
+// each slice to the accumulators of the chunks whose linear set holds it.
+// The sums are the same as scan_regs_kernel's (each chunk's slices in slice
+// order, no subtraction), and P is read once, but a thread holds the
+// accumulators and one batch instead of every slice, so six blocks fit on an
+// SM and the whole grid of the bench layer is resident in one wave.
+constexpr int kScanAcc = 8, kScanBatch = 4;
+__global__ void __launch_bounds__(128, 6)
+    scan_stream_kernel(const float4* __restrict__ P, const float4* __restrict__ z,
+                       float4* __restrict__ SL, float4* __restrict__ zL, int T, int Tc, int To,
+                       int nchunks, int Dp, int D, int causal) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const long long PD4 = static_cast<long long>(Dp) * D / 4;
+  const long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int bh = blockIdx.y;
+  const float4* src;
+  float4* dst;
+  long long stride;
+  if (e < PD4) {
+    src = P + bh * T * PD4 + e;
+    dst = SL + bh * nchunks * PD4 + e;
+    stride = PD4;
+  } else if (e < PD4 + Dp / 4) {
+    src = z + static_cast<long long>(bh) * T * (Dp / 4) + (e - PD4);
+    dst = zL + static_cast<long long>(bh) * nchunks * (Dp / 4) + (e - PD4);
+    stride = Dp / 4;
+  } else {
+    return;
+  }
+  float4 acc[kScanAcc];
+#pragma unroll
+  for (int t = 0; t < kScanAcc; ++t) acc[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s0 = 0; s0 < T; s0 += kScanBatch) {
+    float4 v[kScanBatch];
+#pragma unroll
+    for (int u = 0; u < kScanBatch; ++u)
+      v[u] = s0 + u < T ? src[static_cast<long long>(s0 + u) * stride]
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < kScanBatch; ++u) {
+      const int sl = s0 + u;
+#pragma unroll
+      for (int t = 0; t < kScanAcc; ++t) {
+        const int first = t * Tc, end = min(T, first + Tc), w = max(first - To, 0);
+        const int lim = causal ? T : end;  // slices >= lim join the linear set
+        if (t < nchunks && sl < T && (sl < w || sl >= lim)) {
+          acc[t].x += v[u].x;
+          acc[t].y += v[u].y;
+          acc[t].z += v[u].z;
+          acc[t].w += v[u].w;
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < kScanAcc; ++t)
+    if (t < nchunks) dst[static_cast<long long>(t) * stride] = acc[t];
+}
+
 // ---------------------------------------------------------------------------
 // Streaming helpers.
 // ---------------------------------------------------------------------------
@@ -630,11 +691,12 @@ cudaError_t launch_scan(const float* P, const float* z, float* SL, float* zL, in
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (T <= kScanRegs && Dp % 4 == 0) {
+  if ((nchunks <= kScanAcc || T <= kScanRegs) && Dp % 4 == 0) {
     const long long n4 = static_cast<long long>(Dp) * D / 4 + Dp / 4;
     cfg.gridDim = dim3(static_cast<unsigned>((n4 + 127) / 128), BH);
     cfg.blockDim = dim3(128);
-    return cudaLaunchKernelEx(&cfg, scan_regs_kernel, reinterpret_cast<const float4*>(P),
+    return cudaLaunchKernelEx(&cfg, nchunks <= kScanAcc ? scan_stream_kernel : scan_regs_kernel,
+                              reinterpret_cast<const float4*>(P),
                               reinterpret_cast<const float4*>(z), reinterpret_cast<float4*>(SL),
                               reinterpret_cast<float4*>(zL), T, Tc, To, nchunks, Dp, D, causal);
   }
