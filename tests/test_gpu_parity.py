@@ -51,6 +51,7 @@ SMALL = [
     (1, 1, 9, 11, 12, 128, 128, 3, 1),   # HW=132, several chunks
     (1, 2, 5, 9, 15, 128, 256, 2, 1),    # D'=256 on the tensor-core state path
     (1, 1, 40, 3, 4, 128, 64, 3, 1),     # long sequence of short slices (T = 40)
+    (1, 1, 40, 3, 4, 128, 64, 5, 2),     # T = 40 in 8 chunks: the streaming chunk scan
 ]
 
 
