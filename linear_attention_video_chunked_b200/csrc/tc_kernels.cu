@@ -959,7 +959,11 @@ __global__ void __launch_bounds__(a2::kThreads, 1)
         float& m_used = m_used2[tile];
         m_max = fmaxf(m_max, pm * P.scale_log2);
         float alpha = 1.f;
-        const bool rescale = m_max > m_used + 8.f;
+        // The reference point moves only when the maximum passes it by more
+        // than 16 (log2 units): p <= 2^16 and a row's sum <= 2^16 per key stay
+        // far inside fp32 and bf16 range, and the final factor
+        // 2^(m_used - m_max) makes the result exact with respect to c.
+        const bool rescale = m_max > m_used + 16.f;
         if (rescale) {
           alpha = ex2(m_used - m_max);  // 0 on the first tile
           m_used = m_max;
